@@ -1,0 +1,200 @@
+/*
+ * sattn.h -- C ABI of libsattn.so: causal self-attention over a structured,
+ * data-dependent key set, for NVIDIA B200 (sm_100a).
+ *
+ * For query row i the key set is the union of
+ *   - the starting span  j < n_start                  ("LM-Infinite", NAACL
+ *     2024 summary, section 方法, equation A_i),
+ *   - the recent window  0 <= i-j <= window            (same equation),
+ *   - every earlier separator token, j < i            ("SepLLM", CSDN
+ *     article, section 五.2, mask M_ij),
+ *   - optionally, per query head, the topk middle tokens with the largest
+ *     attention logit                                  ("LM-Infinite",
+ *     section 方法, optional top-k paragraph),
+ * restricted to j <= i.  Masked keys get -inf before the softmax ("SepLLM",
+ * section 6.1 read together with 五.2).  The distance cap of LM-Infinite
+ * (section 方法, equations d_ij and d'_ij = min(d_ij, L)) applies to every
+ * logit: when L_pretrain > 0 and i-j > L_pretrain the logit is
+ * <R(L_pretrain) q_i, k_j> with k_j unrotated (the RoPE realisation in the
+ * same section); otherwise <R(i) q_i, R(j) k_j>.  Logits are scaled by
+ * 1/sqrt(d).  R(p) is rotate-half RoPE with inverse frequencies
+ * theta^(-2c/d); rope_theta = 0 disables rotation.  Query head h uses
+ * key/value head floor(h * Hkv / Hq).
+ *
+ * sattn_segment_fwd implements segmented execution ("Training-Inference
+ * Consistent Segmented Execution for Long-Context LLMs", sections 整体框架
+ * and 关键设计).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every function returns an int status (SATTN_OK or a negative code) and
+ *    never throws.  sattn_strerror() gives the text.
+ *  - Tensor arguments are DEVICE pointers owned by the caller.  The library
+ *    never allocates: all scratch lives in the caller's workspace `ws` of at
+ *    least the size returned by the matching *_workspace_size call.  `ws`
+ *    must be 256-byte aligned.
+ *  - Q/K/V/O are [B, H, T, d] with the head dimension contiguous and the
+ *    element strides given in sattn_params (batch, head, token).  For bf16
+ *    the token stride must make rows 16-byte aligned (stride * 2 % 16 == 0)
+ *    and base pointers 16-byte aligned (the tensor-memory-access engine
+ *    loads tiles straight from these tensors).
+ *  - Launches are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Argument errors are detected on
+ *    the host before any launch and leave every output untouched.
+ *  - Device-side failures (a bounded wait that timed out) are written to a
+ *    status word inside the workspace; sattn_stream_status() synchronises
+ *    the stream and reads it.  Each entry point clears the word first.
+ *  - Results are deterministic: no floating-point atomics; repeated calls on
+ *    the same inputs are bit-identical.
+ */
+#ifndef SATTN_H_
+#define SATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SATTN_OK 0
+#define SATTN_ERR_INVALID_ARG (-1)
+#define SATTN_ERR_UNSUPPORTED (-2)
+#define SATTN_ERR_CUDA (-3)
+#define SATTN_ERR_TIMEOUT (-4)
+
+#define SATTN_DTYPE_BF16 0
+#define SATTN_DTYPE_F32 1
+
+/* Problem description.  Field meanings follow the pages' problem statement. */
+typedef struct sattn_params {
+  int32_t B;          /* batch */
+  int32_t Hq;         /* query heads */
+  int32_t Hkv;        /* key/value heads; Hq % Hkv == 0 */
+  int32_t T;          /* sequence length, >= 1 */
+  int32_t d;          /* head dimension: 64 or 128 */
+  int32_t dtype;      /* SATTN_DTYPE_BF16 or SATTN_DTYPE_F32 (O has this type too) */
+  int64_t q_stride[3];  /* element strides of Q: batch, head, token */
+  int64_t k_stride[3];  /* of K */
+  int64_t v_stride[3];  /* of V */
+  int64_t o_stride[3];  /* of O */
+  int32_t n_start;    /* starting ("sink") span, >= 0           (LM-Infinite A_i; SepLLM a) */
+  int32_t window;     /* recent window w: keys with i-j <= w, >= 0 (LM-Infinite L; SepLLM n) */
+  int32_t L_pretrain; /* distance cap; 0 = no cap                 (LM-Infinite d'_ij) */
+  int32_t topk;       /* extra middle tokens per row and query head; 0 = none, <= 16 */
+  int32_t with_separators; /* nonzero: is_sep may be passed; the workspace then holds the
+                              separator compaction and gathered K/V (worst case: every token) */
+  double rope_theta;  /* rotary base; 0 = no rotation */
+} sattn_params;
+
+/* Text of a status code (static storage). */
+const char* sattn_strerror(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int sattn_version(void);
+
+/* Bytes of workspace needed by sattn_fwd, sattn_topk_select and
+ * sattn_build_blockmap for these parameters (the same buffer serves all
+ * three).  Returns SATTN_ERR_INVALID_ARG / SATTN_ERR_UNSUPPORTED for
+ * parameters the entry points would reject. */
+int sattn_workspace_size(const sattn_params* p, size_t* bytes);
+
+/* Bytes of workspace needed by sattn_segment_fwd; is_long is the same [Hq]
+ * HOST array the call will get (NULL: size for every head long). */
+int sattn_segment_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R,
+                                 int32_t retr_block, const uint8_t* is_long, size_t* bytes);
+
+/* Block map and separator compaction (the structural mask of the header
+ * comment, top-k excluded since it is per head), with 128x128 tiles.
+ *   is_sep          [B, T] uint8 flags (nonzero = separator), or NULL = none.
+ *   cls             [B, ceil(T/128), ceil(T/128)] uint8, out: 0 empty,
+ *                   1 partial, 2 full, over in-range (i, j) pairs; may be NULL.
+ *   sep_pos         [B, T] int32, out: positions j >= n_start of separators in
+ *                   ascending order, then -1.
+ *   sep_count       [B] int32, out: number of such separators.
+ *   qtile_sep_range [B, ceil(T/128), 2] int32, out: per query tile t, the
+ *                   number of separators with j < 128t - window (kept by every
+ *                   row of the tile) and with j < last_row(t) - window (kept by
+ *                   at least one row).
+ * All outputs are device pointers. */
+int sattn_build_blockmap(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
+                         int32_t* sep_count, int32_t* qtile_sep_range, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Top-k middle-token selection ("LM-Infinite", section 方法, optional top-k).
+ * For every (b, query head h, row i) the p->topk keys j with
+ * n_start <= j < i - window that are not separators, ranked by the unscaled
+ * logit z_ij (capped rule of the header comment), ties to the smaller j.
+ *   Q, K       inputs as in sattn_fwd (V is not needed).
+ *   is_sep     [B, T] uint8 or NULL.
+ *   idx        [B, Hq, T, topk] int32, out: selected j sorted by (z desc, j asc);
+ *              -1 when fewer than topk candidates exist.
+ *   logit      [B, Hq, T, topk] float, out: z_ij in fp32; -inf for padding.
+ * bf16 only.  Requires L_pretrain == 0 or L_pretrain == window. */
+int sattn_topk_select(const sattn_params* p, const void* Q, const void* K, const uint8_t* is_sep,
+                      int32_t* idx, float* logit, void* ws, size_t ws_bytes, void* stream);
+
+/* Forward attention over the structured key set.
+ *   Q [B,Hq,T,d], K,V [B,Hkv,T,d]   dtype p->dtype, strides in p.
+ *   is_sep      [B, T] uint8 or NULL (no separators).
+ *   topk_idx    [B, Hq, T, topk] int32 or NULL; topk_logit likewise (float).
+ *               When p->topk > 0 and topk_idx is NULL the selection of
+ *               sattn_topk_select runs inside this call.  When given, they
+ *               must be a selection in that format (middle, non-separator
+ *               keys; -1 padding); the logits are used as the keys' z.
+ *   O           [B, Hq, T, d], out, dtype p->dtype, strides p->o_stride.
+ *   lse         [B, Hq, T] float, out: natural-log logsumexp of the scaled
+ *               logits of each row.
+ * bf16 runs on the tensor cores; fp32 runs on the CUDA cores in fp32.
+ * With bf16 and L_pretrain > 0: window <= L_pretrain, and when separators
+ * or top-k are used, window == L_pretrain. */
+int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+              const int32_t* topk_idx, const float* topk_logit, void* O, float* lse, void* ws, size_t ws_bytes,
+              void* stream);
+
+/* Segmented execution of one layer ("Training-Inference Consistent Segmented
+ * Execution", sections 整体框架 and 关键设计).  The sequence is cut into T/S
+ * segments.  For a query in segment s:
+ *   local heads (is_long[h] == 0): the carried tail, keys [sS-M, sS), at
+ *     positions 0..P-1, then the segment's keys sS..i at P + (j - sS);
+ *   long heads (is_long[h] != 0): a prefix of R keys retrieved from the pool
+ *     [0, sS): the top R/retr_block blocks of retr_block keys scored by
+ *     max_{j in block} <q_{sS-1}, k_j> (unrotated; ties to the lower block),
+ *     in ascending block order at positions 0..P-1, then the segment.
+ *   Segment 0 has neither tail nor prefix.  No distance cap, no sinks.
+ *   is_long        [Hq] uint8 HOST array.
+ *   prefix_blocks  [B, Hq, T/S, R/retr_block] int32, out: the retrieved block
+ *                  indices, ascending; -1 for local heads, segment 0, or
+ *                  when the pool holds fewer blocks.
+ *   O, lse         as in sattn_fwd.
+ * bf16 only; S % 128 == 0, T % S == 0, 1 <= retr_block, R % retr_block == 0,
+ * R / retr_block <= 1024, Hq <= 256. */
+int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                      const uint8_t* is_long, const void* Q, const void* K, const void* V, void* O, float* lse,
+                      int32_t* prefix_blocks, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and reads the device status word of `ws` into
+ * *device_status (SATTN_OK or SATTN_ERR_TIMEOUT).  Returns SATTN_ERR_CUDA if
+ * the synchronisation itself failed (the CUDA error is then sticky). */
+int sattn_stream_status(void* stream, const void* ws, int32_t* device_status);
+
+/* Instrumentation (no counterpart on the pages).  While enabled, every kernel
+ * launch group of the library is bracketed by CUDA events recorded on the
+ * launch stream; the events cost a few hundred nanoseconds of device time
+ * each.  sattn_profile_collect synchronises those events and reports, per
+ * kernel group, the number of kernel launches and the summed device time
+ * (milliseconds) since the previous collect, then resets the record.
+ *   names     [max_groups][32] chars, out (NUL-terminated group names)
+ *   launches  [max_groups] int32, out: kernels launched by the group
+ *   total_ms  [max_groups] double, out
+ *   n_groups  out: number of groups written
+ * Host pointers.  Not thread-safe against concurrent entry-point calls. */
+int sattn_profile_enable(int on);
+int sattn_profile_collect(char* names, int32_t* launches, double* total_ms, int32_t max_groups,
+                          int32_t* n_groups);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SATTN_H_ */

@@ -1,0 +1,229 @@
+"""Structured-mask causal attention for B200 (sm_100a).
+
+Python binding of ``libsattn.so``.  Every computation runs in the library's
+CUDA kernels; this module only marshals arguments: it reads shapes and
+strides from torch tensors, allocates the caller-side workspace with torch,
+and passes raw device pointers and the current CUDA stream through the C ABI.
+
+Public calls (names follow the C ABI):
+    fwd(q, k, v, ...)            -> (O, lse)
+    topk_select(q, k, ...)       -> (idx, logit)
+    build_blockmap(is_sep, ...)  -> dict(cls, sep_pos, sep_count, qtile_sep_range)
+    segment_fwd(q, k, v, ...)    -> (O, lse, prefix_blocks)
+    stream_status(workspace)     -> device status code
+
+``fwd`` and ``segment_fwd`` also accept host (CPU) tensors: the inputs are
+then copied to the device, the call runs there, and the outputs are copied
+back -- the end-to-end path a host application uses.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
+
+__all__ = ["fwd", "topk_select", "build_blockmap", "segment_fwd", "stream_status", "workspace_size",
+           "segment_workspace_size", "params", "SattnError", "version", "TILE"]
+
+TILE = 128
+_ws_cache: dict = {}
+
+
+def version() -> int:
+    return _lib.load().sattn_version()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _strides(t: Optional[torch.Tensor]):
+    if t is None:
+        return (0, 0, 0)
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [B, H, T, d] tensor with a contiguous head dimension")
+    return (t.stride(0), t.stride(1), t.stride(2))
+
+
+def params(q, k, v=None, o=None, *, n_start=0, window=0, L_pretrain=0, topk=0, rope_theta=0.0,
+           with_separators=False) -> SattnParams:
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    p = SattnParams()
+    p.B, p.Hq, p.Hkv, p.T, p.d = B, Hq, Hkv, T, d
+    p.dtype = _dtype_code(q)
+    for name, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", o if o is not None else q)):
+        s = _strides(t)
+        arr = getattr(p, name)
+        arr[0], arr[1], arr[2] = s
+    p.n_start, p.window, p.L_pretrain, p.topk = int(n_start), int(window), int(L_pretrain), int(topk)
+    p.with_separators = 1 if with_separators else 0
+    p.rope_theta = float(rope_theta)
+    return p
+
+
+def workspace_size(p: SattnParams) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.load().sattn_workspace_size(ctypes.byref(p), ctypes.byref(n)), "sattn_workspace_size")
+    return int(n.value)
+
+
+def segment_workspace_size(p: SattnParams, S, M, R, retr_block, is_long) -> int:
+    n = ctypes.c_size_t(0)
+    il = None if is_long is None else (ctypes.c_uint8 * len(is_long))(*[int(x) for x in is_long])
+    _lib.check(_lib.load().sattn_segment_workspace_size(ctypes.byref(p), S, M, R, retr_block, il, ctypes.byref(n)),
+               "sattn_segment_workspace_size")
+    return int(n.value)
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small: need %d bytes" % nbytes)
+        return workspace
+    key = (str(device), nbytes)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        _ws_cache.clear()  # keep one buffer per process
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _to_dev(t, device):
+    if t is None:
+        return None
+    return t.to(device, non_blocking=True)
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, window: int = 0,
+        L_pretrain: int = 0, rope_theta: float = 0.0, topk: int = 0, is_sep: Optional[torch.Tensor] = None,
+        topk_idx: Optional[torch.Tensor] = None, topk_logit: Optional[torch.Tensor] = None,
+        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None):
+    """Structured-mask attention forward.  Returns (O [B,Hq,T,d], lse [B,Hq,T] fp32)."""
+    if not q.is_cuda:
+        return _host_call(fwd, (q, k, v), dict(n_start=n_start, window=window, L_pretrain=L_pretrain,
+                                               rope_theta=rope_theta, topk=topk, is_sep=is_sep,
+                                               topk_idx=topk_idx, topk_logit=topk_logit))
+    B, Hq, T, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    p = params(q, k, v, out, n_start=n_start, window=window, L_pretrain=L_pretrain, topk=topk,
+               rope_theta=rope_theta, with_separators=is_sep is not None)
+    nbytes = workspace_size(p)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = _lib.load().sattn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(topk_idx),
+                               _ptr(topk_logit), _ptr(out), _ptr(lse), _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_fwd")
+    return out, lse
+
+
+def topk_select(q: torch.Tensor, k: torch.Tensor, *, topk: int, n_start: int = 0, window: int = 0,
+                L_pretrain: int = 0, rope_theta: float = 0.0, is_sep: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None):
+    """Per-head top-k middle tokens.  Returns (idx [B,Hq,T,k] int32, logit [B,Hq,T,k] fp32)."""
+    B, Hq, T, d = q.shape
+    idx = torch.empty((B, Hq, T, topk), dtype=torch.int32, device=q.device)
+    logit = torch.empty((B, Hq, T, topk), dtype=torch.float32, device=q.device)
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    p = params(q, k, k, q, n_start=n_start, window=window, L_pretrain=L_pretrain, topk=topk,
+               rope_theta=rope_theta, with_separators=is_sep is not None)
+    nbytes = workspace_size(p)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = _lib.load().sattn_topk_select(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(is_sep), _ptr(idx), _ptr(logit),
+                                       _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_topk_select")
+    return idx, logit
+
+
+def build_blockmap(is_sep: Optional[torch.Tensor], *, B: int, T: int, n_start: int, window: int,
+                   device="cuda", with_classes: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Block map + separator compaction for [B, T] flags (None = no separators)."""
+    nqt = (T + TILE - 1) // TILE
+    dummy = torch.empty((B, 1, T, 64), dtype=torch.bfloat16, device=device)
+    p = params(dummy, dummy, dummy, dummy, n_start=n_start, window=window, with_separators=True)
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    cls = torch.empty((B, nqt, nqt), dtype=torch.uint8, device=device) if with_classes else None
+    sep_pos = torch.empty((B, T), dtype=torch.int32, device=device)
+    sep_count = torch.empty((B,), dtype=torch.int32, device=device)
+    ranges = torch.empty((B, nqt, 2), dtype=torch.int32, device=device)
+    nbytes = workspace_size(p)
+    ws = _workspace(nbytes, device, workspace)
+    rc = _lib.load().sattn_build_blockmap(ctypes.byref(p), _ptr(is_sep), _ptr(cls), _ptr(sep_pos), _ptr(sep_count),
+                                          _ptr(ranges), _ptr(ws), nbytes, _stream_ptr(sep_pos.device))
+    _lib.check(rc, "sattn_build_blockmap")
+    return {"cls": cls, "sep_pos": sep_pos, "sep_count": sep_count, "qtile_sep_range": ranges}
+
+
+def segment_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, S: int, M: int, R: int, retr_block: int,
+                is_long, rope_theta: float = 0.0, out: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Segmented execution of one layer.  Returns (O, lse, prefix_blocks [B,Hq,T/S,R/retr_block])."""
+    if not q.is_cuda:
+        return _host_call(segment_fwd, (q, k, v), dict(S=S, M=M, R=R, retr_block=retr_block, is_long=is_long,
+                                                       rope_theta=rope_theta))
+    B, Hq, T, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    nb = R // retr_block if retr_block > 0 else 0
+    prefix = torch.empty((B, Hq, T // S, max(nb, 1)), dtype=torch.int32, device=q.device)
+    il_list = [int(x) for x in (is_long.tolist() if hasattr(is_long, "tolist") else is_long)]
+    il = (ctypes.c_uint8 * Hq)(*il_list)
+    p = params(q, k, v, out, rope_theta=rope_theta)
+    nbytes = segment_workspace_size(p, S, M, R, retr_block, il_list)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = _lib.load().sattn_segment_fwd(ctypes.byref(p), S, M, R, retr_block, il, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                       _ptr(lse), _ptr(prefix), _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_segment_fwd")
+    return out, lse, prefix[..., :nb]
+
+
+def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> int:
+    """Synchronise the current stream and read the device status word of the
+    workspace (the cached one when None)."""
+    if workspace is None:
+        if not _ws_cache:
+            return 0
+        workspace = next(iter(_ws_cache.values()))
+    st = ctypes.c_int32(0)
+    _lib.check(_lib.load().sattn_stream_status(_stream_ptr(workspace.device), _ptr(workspace), ctypes.byref(st)),
+               "sattn_stream_status")
+    return int(st.value)
+
+
+def _host_call(fn, tensors, kw):
+    """Host tensors in, host tensors out: H2D copies, the device call, D2H copies."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dq, dk, dv = (_to_dev(t, dev) for t in tensors)
+    kw = dict(kw)
+    for name in ("is_sep", "topk_idx", "topk_logit"):
+        if kw.get(name) is not None:
+            kw[name] = _to_dev(kw[name], dev)
+    res = fn(dq, dk, dv, **kw)
+    outs = tuple(r.to("cpu", non_blocking=False) for r in res)
+    return outs

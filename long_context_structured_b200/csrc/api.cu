@@ -1,0 +1,816 @@
+// api.cu -- the C ABI of libsattn.so: argument validation, workspace layout,
+// tensor-map encoding and the launch sequence of each entry point.
+//
+// The library never allocates.  Each entry point carves its scratch out of
+// the caller's workspace with the layout computed by plan_fwd / plan_seg,
+// the same functions the *_workspace_size queries call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/sattn.h"
+#include "kernels.cuh"
+#include "status.cuh"
+
+using namespace sattn;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Region {
+  size_t off = 0, bytes = 0;
+};
+
+struct FwdPlan {
+  bool bf16 = true;
+  int nQT = 0, Tpad = 0, npos = 0, n_sink = 0, short_len = 0;
+  bool need_qc = false, capped_sep = false;
+  Region status, tab, qr, kr, qc, sink, kmax, prefix, sep_pos, sep_count, ranges, ks, vs, tk_idx, tk_z, fb,
+      short_idx, short_thr, n_cand;
+  size_t total = 0;
+};
+
+struct Alloc {
+  size_t cur = 0;
+  Region take(size_t bytes) {
+    Region r;
+    r.off = cur;
+    r.bytes = bytes;
+    cur = align256(cur + bytes);
+    return r;
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(const sattn_params* p) {
+  if (!p) return SATTN_ERR_INVALID_ARG;
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->T < 1) return SATTN_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv) return SATTN_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SATTN_ERR_UNSUPPORTED;
+  if (p->dtype != SATTN_DTYPE_BF16 && p->dtype != SATTN_DTYPE_F32) return SATTN_ERR_INVALID_ARG;
+  if (p->n_start < 0 || p->window < 0 || p->L_pretrain < 0 || p->topk < 0) return SATTN_ERR_INVALID_ARG;
+  if (p->topk > 16) return SATTN_ERR_UNSUPPORTED;
+  if (!(p->rope_theta >= 0.0) || !std::isfinite(p->rope_theta)) return SATTN_ERR_INVALID_ARG;
+  if ((int64_t)p->B * p->Hq * p->T > (int64_t)1 << 31) return SATTN_ERR_UNSUPPORTED;
+  const int64_t* st[4] = {p->q_stride, p->k_stride, p->v_stride, p->o_stride};
+  const int esz = p->dtype == SATTN_DTYPE_BF16 ? 2 : 4;
+  for (int x = 0; x < 4; ++x) {
+    for (int y = 0; y < 3; ++y)
+      if (st[x][y] < 0) return SATTN_ERR_INVALID_ARG;
+    if (st[x][2] < p->d && p->T > 1) return SATTN_ERR_INVALID_ARG;
+    if (p->dtype == SATTN_DTYPE_BF16 && ((st[x][0] * esz) % 16 || (st[x][1] * esz) % 16 || (st[x][2] * esz) % 16))
+      return SATTN_ERR_INVALID_ARG;
+  }
+  return SATTN_OK;
+}
+
+int check_fwd_rules(const sattn_params* p) {
+  int rc = check_common(p);
+  if (rc) return rc;
+  if (p->dtype == SATTN_DTYPE_BF16) {
+    if (p->n_start > 256) return SATTN_ERR_UNSUPPORTED;
+    if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
+    if (p->L_pretrain > 0 && (p->with_separators || p->topk > 0) && p->window != p->L_pretrain)
+      return SATTN_ERR_UNSUPPORTED;
+    if (p->Hq > 65535) return SATTN_ERR_UNSUPPORTED;
+  }
+  return SATTN_OK;
+}
+
+int plan_fwd(const sattn_params* p, FwdPlan* pl) {
+  int rc = check_fwd_rules(p);
+  if (rc) return rc;
+  FwdPlan P;
+  P.bf16 = p->dtype == SATTN_DTYPE_BF16;
+  P.nQT = (p->T + kTile - 1) / kTile;
+  P.Tpad = P.nQT * kTile;
+  P.npos = std::max(p->T, p->L_pretrain + 1);
+  P.n_sink = std::min(p->n_start, p->T);
+  P.short_len = p->topk <= 6 ? 8 : (p->topk <= 14 ? 16 : 32);
+  P.capped_sep = p->L_pretrain > 0;
+  P.need_qc = P.bf16 && p->L_pretrain > 0 && (p->with_separators || p->topk > 0);
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  P.prefix = A.take(B * (T + 1) * 4);
+  if (P.bf16) {
+    P.qr = A.take(B * Hq * T * d * 2);
+    P.kr = A.take(B * Hkv * T * d * 2);
+    if (P.need_qc) P.qc = A.take(B * Hq * T * d * 2);
+    if (P.n_sink > 0) P.sink = A.take(B * Hq * T * P.n_sink * 4);
+  }
+  if (p->with_separators) {
+    P.sep_pos = A.take(B * T * 4);
+    P.sep_count = A.take(B * 4);
+    P.ranges = A.take(B * P.nQT * 2 * 4);
+    if (P.bf16) {
+      P.ks = A.take(B * Hkv * P.Tpad * d * 2);
+      P.vs = A.take(B * Hkv * P.Tpad * d * 2);
+    }
+  }
+  if (p->topk > 0) {
+    P.tk_idx = A.take(B * Hq * T * p->topk * 4);
+    P.tk_z = A.take(B * Hq * T * p->topk * 4);
+    if (P.bf16) {
+      P.kmax = A.take(B * Hkv * 4);
+      P.fb = A.take(B * Hq * T * 4);
+      P.short_idx = A.take(B * Hq * T * P.short_len * 4);
+      P.short_thr = A.take(B * Hq * T * 4);
+      P.n_cand = A.take(B * Hq * T * 4);
+    }
+  }
+  P.total = A.cur;
+  *pl = P;
+  return SATTN_OK;
+}
+
+template <typename T>
+T* at(void* ws, const Region& r) {
+  return r.bytes ? reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + r.off) : nullptr;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// bf16 [n3][n2][rows][d] with element strides (s3, s2, srow); box 64 x 128,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t n2, int64_t n3, int64_t srow,
+              int64_t s2, int64_t s3) {
+  auto enc = encoder();
+  if (!enc) return false;
+  // strides of size-1 dimensions are never used; keep them legal
+  if (n2 == 1) s2 = srow * rows;
+  if (n3 == 1) s3 = s2 * n2;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)n2, (cuuint64_t)n3};
+  cuuint64_t strides[3] = {(cuuint64_t)srow * 2, (cuuint64_t)s2 * 2, (cuuint64_t)s3 * 2};
+  for (int x = 0; x < 3; ++x)
+    if (strides[x] == 0 || strides[x] % 16) return false;
+  cuuint32_t box[4] = {64, (cuuint32_t)kTile, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------
+// optional event instrumentation of launch groups
+// ---------------------------------------------------------------------------
+
+struct ProfRec {
+  const char* name;
+  int kernels;
+  cudaEvent_t a, b;
+};
+
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Records an event pair around one launch group when instrumentation is on.
+class ProfScope {
+ public:
+  ProfScope(const char* name, int kernels, cudaStream_t st) : st_(st) {
+    if (!g_prof_on) return;
+    rec_.name = name;
+    rec_.kernels = kernels;
+    rec_.a = prof_event();
+    rec_.b = prof_event();
+    active_ = rec_.a && rec_.b && cudaEventRecord(rec_.a, st_) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!active_) return;
+    if (cudaEventRecord(rec_.b, st_) == cudaSuccess) {
+      std::lock_guard<std::mutex> g(g_prof_mu);
+      g_prof_recs.push_back(rec_);
+    }
+  }
+
+ private:
+  cudaStream_t st_;
+  ProfRec rec_{};
+  bool active_ = false;
+};
+
+#define SATTN_TRY(expr)                   \
+  do {                                    \
+    int _rc = cuda_rc(expr);              \
+    if (_rc != SATTN_OK) return _rc;      \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// shared launch steps
+// ---------------------------------------------------------------------------
+
+int run_prep_bf16(const sattn_params* p, const FwdPlan& P, const void* Q, const void* K, void* ws, bool with_sinks,
+                  bool with_kmax, cudaStream_t st) {
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+  }
+  if (with_kmax && P.kmax.bytes) SATTN_TRY(cudaMemsetAsync(at<uint8_t>(ws, P.kmax), 0, P.kmax.bytes, st));
+  PrepArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.Q = Q;
+  a.K = K;
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.q_st = p->q_stride[2];
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.f32 = false;
+  a.tab = at<float2>(ws, P.tab);
+  a.L = p->L_pretrain;
+  a.Qr = at<__nv_bfloat16>(ws, P.qr);
+  a.Qc = at<__nv_bfloat16>(ws, P.qc);
+  a.Kr = at<__nv_bfloat16>(ws, P.kr);
+  a.sink_z = with_sinks ? at<float>(ws, P.sink) : nullptr;
+  a.n_sink = with_sinks ? P.n_sink : 0;
+  a.kmax = with_kmax ? at<uint32_t>(ws, P.kmax) : nullptr;
+  ProfScope ps("prep_rope", 1, st);
+  return cuda_rc(launch_prep(a, st));
+}
+
+int run_blockmap(const sattn_params* p, const FwdPlan& P, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
+                 int32_t* sep_count, int32_t* ranges, void* ws, cudaStream_t st) {
+  BlockmapArgs a{};
+  a.B = p->B;
+  a.T = p->T;
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.is_sep = is_sep;
+  a.prefix = at<int32_t>(ws, P.prefix);
+  a.sep_pos = sep_pos;
+  a.sep_count = sep_count;
+  a.ranges = ranges;
+  a.cls = cls;
+  ProfScope ps("blockmap", 2, st);
+  return cuda_rc(launch_blockmap(a, st));
+}
+
+TopkArgs topk_args(const sattn_params* p, const FwdPlan& P, const void* Q, const void* K, const uint8_t* is_sep,
+                   int32_t* idx, float* z, void* ws) {
+  TopkArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.nQT = P.nQT;
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.topk = p->topk;
+  a.L = p->L_pretrain;
+  a.is_sep = is_sep;
+  a.Q = Q;
+  a.K = K;
+  a.f32 = !P.bf16;
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.q_st = p->q_stride[2];
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.tab = at<float2>(ws, P.tab);
+  a.kmax = at<uint32_t>(ws, P.kmax);
+  a.idx = idx;
+  a.z = z;
+  a.fallback_rows = at<int32_t>(ws, P.fb);
+  a.status = at<int32_t>(ws, P.status);
+  a.short_len = P.short_len;
+  a.short_idx = at<int32_t>(ws, P.short_idx);
+  a.short_thr = at<float>(ws, P.short_thr);
+  a.n_cand = at<int32_t>(ws, P.n_cand);
+  return a;
+}
+
+// selection into (idx, z); prep must have run (bf16)
+int run_topk(const sattn_params* p, const FwdPlan& P, const void* Q, const void* K, const uint8_t* is_sep,
+             int32_t* idx, float* z, void* ws, cudaStream_t st) {
+  TopkArgs a = topk_args(p, P, Q, K, is_sep, idx, z, ws);
+  if (!P.bf16) {
+    if (P.tab.bytes) SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+    ProfScope ps("topk_exact", 1, st);
+    return cuda_rc(launch_topk_exact(a, true, st));
+  }
+  TopkMaps m;
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  if (p->L_pretrain > 0) {
+    if (!make_map(&m.qsel, at<void>(ws, P.qc), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+    if (!make_map(&m.ksel, K, p->d, p->T, Hkv, B, p->k_stride[2], p->k_stride[1], p->k_stride[0]))
+      return SATTN_ERR_CUDA;
+  } else {
+    if (!make_map(&m.qsel, at<void>(ws, P.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+    if (!make_map(&m.ksel, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
+  }
+  {
+    ProfScope ps("topk_score_rerank", 2, st);
+    SATTN_TRY(launch_topk_tc(a, m, st));
+  }
+  ProfScope ps("topk_exact", 1, st);
+  return cuda_rc(launch_topk_exact(a, false, st));
+}
+
+bool pointers_ok_bf16(const void* a, const void* b, const void* c) {
+  return aligned16(a) && aligned16(b) && aligned16(c);
+}
+
+}  // namespace
+
+// ===========================================================================
+// exported
+// ===========================================================================
+
+extern "C" {
+
+const char* sattn_strerror(int status) {
+  switch (status) {
+    case SATTN_OK: return "ok";
+    case SATTN_ERR_INVALID_ARG: return "invalid argument";
+    case SATTN_ERR_UNSUPPORTED: return "unsupported parameters";
+    case SATTN_ERR_CUDA: return "CUDA error";
+    case SATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int sattn_version(void) { return kVersion; }
+
+int sattn_workspace_size(const sattn_params* p, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  FwdPlan P;
+  int rc = plan_fwd(p, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_build_blockmap(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
+                         int32_t* sep_count, int32_t* qtile_sep_range, void* ws, size_t ws_bytes, void* stream) {
+  FwdPlan P;
+  int rc = plan_fwd(p, &P);
+  if (rc) return rc;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!sep_pos || !sep_count || !qtile_sep_range) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  return run_blockmap(p, P, is_sep, cls, sep_pos, sep_count, qtile_sep_range, ws, st);
+}
+
+int sattn_topk_select(const sattn_params* p, const void* Q, const void* K, const uint8_t* is_sep, int32_t* idx,
+                      float* logit, void* ws, size_t ws_bytes, void* stream) {
+  FwdPlan P;
+  int rc = plan_fwd(p, &P);
+  if (rc) return rc;
+  if (p->topk < 1 || !Q || !K || !idx || !logit) return SATTN_ERR_INVALID_ARG;
+  if (is_sep && !p->with_separators) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (P.bf16 && !pointers_ok_bf16(Q, K, K)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.bf16) {
+    rc = run_prep_bf16(p, P, Q, K, ws, false, true, st);
+    if (rc) return rc;
+  }
+  return run_topk(p, P, Q, K, is_sep, idx, logit, ws, st);
+}
+
+int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+              const int32_t* topk_idx, const float* topk_logit, void* O, float* lse, void* ws, size_t ws_bytes,
+              void* stream) {
+  FwdPlan P;
+  int rc = plan_fwd(p, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse) return SATTN_ERR_INVALID_ARG;
+  if (is_sep && !p->with_separators) return SATTN_ERR_INVALID_ARG;
+  if ((topk_idx == nullptr) != (topk_logit == nullptr)) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (P.bf16 && (!pointers_ok_bf16(Q, K, V) || !aligned16(O))) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+
+  int32_t* sep_pos = at<int32_t>(ws, P.sep_pos);
+  int32_t* sep_count = at<int32_t>(ws, P.sep_count);
+  int32_t* ranges = at<int32_t>(ws, P.ranges);
+  const int32_t* tki = topk_idx;
+  const float* tkz = topk_logit;
+
+  if (!P.bf16) {
+    // ---------------- fp32 path ----------------
+    if (P.tab.bytes) {
+      ProfScope ps("rope_table", 1, st);
+      SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+    }
+    if (is_sep) {
+      rc = run_blockmap(p, P, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
+      if (rc) return rc;
+    }
+    if (p->topk > 0 && !tki) {
+      TopkArgs ta = topk_args(p, P, Q, K, is_sep, at<int32_t>(ws, P.tk_idx), at<float>(ws, P.tk_z), ws);
+      {
+        ProfScope ps("topk_exact", 1, st);
+        SATTN_TRY(launch_topk_exact(ta, true, st));
+      }
+      tki = at<int32_t>(ws, P.tk_idx);
+      tkz = at<float>(ws, P.tk_z);
+    }
+    AttnF32Args a{};
+    a.B = p->B;
+    a.Hq = p->Hq;
+    a.Hkv = p->Hkv;
+    a.T = p->T;
+    a.d = p->d;
+    a.Q = static_cast<const float*>(Q);
+    a.K = static_cast<const float*>(K);
+    a.V = static_cast<const float*>(V);
+    a.q_sb = p->q_stride[0];
+    a.q_sh = p->q_stride[1];
+    a.q_st = p->q_stride[2];
+    a.k_sb = p->k_stride[0];
+    a.k_sh = p->k_stride[1];
+    a.k_st = p->k_stride[2];
+    a.v_sb = p->v_stride[0];
+    a.v_sh = p->v_stride[1];
+    a.v_st = p->v_stride[2];
+    a.tab = at<float2>(ws, P.tab);
+    a.L = p->L_pretrain;
+    a.n_start = p->n_start;
+    a.window = p->window;
+    a.sep_pos = is_sep ? sep_pos : nullptr;
+    a.sep_count = sep_count;
+    a.tk_idx = p->topk > 0 ? tki : nullptr;
+    a.tk_z = tkz;
+    a.topk = p->topk;
+    a.O = static_cast<float*>(O);
+    a.o_sb = p->o_stride[0];
+    a.o_sh = p->o_stride[1];
+    a.o_st = p->o_stride[2];
+    a.lse = lse;
+    ProfScope ps("attn_f32", 1, st);
+    return cuda_rc(launch_attn_f32(a, st));
+  }
+
+  // ---------------- bf16 tensor-core path ----------------
+  rc = run_prep_bf16(p, P, Q, K, ws, true, p->topk > 0 && !tki, st);
+  if (rc) return rc;
+  AttnMaps m;
+  if (!make_map(&m.q, at<void>(ws, P.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.k, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.v, V, p->d, p->T, Hkv, B, p->v_stride[2], p->v_stride[1], p->v_stride[0])) return SATTN_ERR_CUDA;
+  m.q2 = m.q;
+  m.kg = m.k;
+  m.vg = m.v;
+  bool q2 = false;
+  if (is_sep) {
+    rc = run_blockmap(p, P, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
+    if (rc) return rc;
+    GatherArgs ga{};
+    ga.B = p->B;
+    ga.Hkv = p->Hkv;
+    ga.T = p->T;
+    ga.Tpad = P.Tpad;
+    ga.d = p->d;
+    if (P.capped_sep) {
+      ga.Ksrc = static_cast<const __nv_bfloat16*>(K);
+      ga.k_sb = p->k_stride[0];
+      ga.k_sh = p->k_stride[1];
+      ga.k_st = p->k_stride[2];
+      q2 = true;
+      if (!make_map(&m.q2, at<void>(ws, P.qc), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+    } else {
+      ga.Ksrc = at<__nv_bfloat16>(ws, P.kr);
+      ga.k_sb = Hkv * T * d;
+      ga.k_sh = T * d;
+      ga.k_st = d;
+    }
+    ga.Vsrc = static_cast<const __nv_bfloat16*>(V);
+    ga.v_sb = p->v_stride[0];
+    ga.v_sh = p->v_stride[1];
+    ga.v_st = p->v_stride[2];
+    ga.sep_pos = sep_pos;
+    ga.sep_count = sep_count;
+    ga.Ks = at<__nv_bfloat16>(ws, P.ks);
+    ga.Vs = at<__nv_bfloat16>(ws, P.vs);
+    {
+      ProfScope ps("sep_gather", 1, st);
+      SATTN_TRY(launch_sep_gather(ga, st));
+    }
+    if (!make_map(&m.kg, ga.Ks, p->d, P.Tpad, Hkv, B, d, (int64_t)P.Tpad * d, Hkv * P.Tpad * d)) return SATTN_ERR_CUDA;
+    if (!make_map(&m.vg, ga.Vs, p->d, P.Tpad, Hkv, B, d, (int64_t)P.Tpad * d, Hkv * P.Tpad * d)) return SATTN_ERR_CUDA;
+  }
+  if (p->topk > 0 && !tki) {
+    rc = run_topk(p, P, Q, K, is_sep, at<int32_t>(ws, P.tk_idx), at<float>(ws, P.tk_z), ws, st);
+    if (rc) return rc;
+    tki = at<int32_t>(ws, P.tk_idx);
+    tkz = at<float>(ws, P.tk_z);
+  }
+  AttnArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.nQT = P.nQT;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.ns_band = p->n_start;
+  a.w_eff = p->window;
+  a.sink_z = at<float>(ws, P.sink);
+  a.n_sink = P.n_sink;
+  a.tk_idx = p->topk > 0 ? tki : nullptr;
+  a.tk_z = p->topk > 0 ? tkz : nullptr;
+  a.topk = p->topk > 0 ? p->topk : 0;
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.gather_mode = is_sep ? 1 : 0;
+  a.q2 = q2;
+  a.sep_pos = sep_pos;
+  a.ranges = ranges;
+  a.window = p->window;
+  for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.status = at<int32_t>(ws, P.status);
+  ProfScope ps("attn_tc", 1, st);
+  return cuda_rc(launch_attn_tc(a, m, st));
+}
+
+// ---------------------------------------------------------------------------
+// segmented execution
+// ---------------------------------------------------------------------------
+
+struct SegPlan {
+  int nQT, N, Rpad, n_long, npos;
+  Region status, tab, qr, kr, kpre, vpre, pcnt;
+  size_t total;
+};
+
+static int plan_seg(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t blk, const uint8_t* is_long,
+                    SegPlan* out) {
+  int rc = check_common(p);
+  if (rc) return rc;
+  if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
+  if (S < kTile || S % kTile || p->T % S || M < 0 || R < 0 || blk < 1 || R % blk) return SATTN_ERR_INVALID_ARG;
+  if (R / blk > 1024 || p->Hq > kMaxHeads) return SATTN_ERR_UNSUPPORTED;
+  if ((size_t)(p->T / blk + p->d) * 4 > 200 * 1024) return SATTN_ERR_UNSUPPORTED;
+  SegPlan P;
+  P.nQT = (p->T + kTile - 1) / kTile;
+  P.N = p->T / S;
+  P.Rpad = (R + kTile - 1) / kTile * kTile;
+  P.n_long = 0;
+  for (int h = 0; h < p->Hq; ++h) P.n_long += (is_long == nullptr || is_long[h]) ? 1 : 0;
+  P.npos = p->T;
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  P.qr = A.take(B * Hq * T * d * 2);
+  P.kr = A.take(B * Hkv * T * d * 2);
+  if (P.n_long > 0 && R > 0) {
+    P.kpre = A.take(B * P.n_long * P.N * P.Rpad * d * 2);
+    P.vpre = A.take(B * P.n_long * P.N * P.Rpad * d * 2);
+  }
+  P.pcnt = A.take(B * std::max(P.n_long, 1) * P.N * 4);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_segment_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                                 const uint8_t* is_long, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  SegPlan P;
+  int rc = plan_seg(p, S, M, R, retr_block, is_long, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                      const uint8_t* is_long, const void* Q, const void* K, const void* V, void* O, float* lse,
+                      int32_t* prefix_blocks, void* ws, size_t ws_bytes, void* stream) {
+  if (!is_long) return SATTN_ERR_INVALID_ARG;
+  SegPlan P;
+  int rc = plan_seg(p, S, M, R, retr_block, is_long, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse || !prefix_blocks) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+
+  // prep: rotate Q and K at their global positions (only distances matter)
+  FwdPlan F;
+  F.bf16 = true;
+  F.npos = P.npos;
+  F.tab = P.tab;
+  F.qr = P.qr;
+  F.kr = P.kr;
+  sattn_params pp = *p;
+  pp.L_pretrain = 0;
+  rc = run_prep_bf16(&pp, F, Q, K, ws, false, false, st);
+  if (rc) return rc;
+
+  const int nb = R / retr_block;
+  if (nb > 0) SATTN_TRY(cudaMemsetAsync(prefix_blocks, 0xFF, B * Hq * P.N * nb * 4, st));
+  SATTN_TRY(cudaMemsetAsync(at<uint8_t>(ws, P.pcnt), 0, P.pcnt.bytes, st));
+  AttnArgs a{};
+  for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
+  SegRetrArgs ra{};
+  {
+    int slot = 0;
+    for (int h = 0; h < p->Hq; ++h)
+      if (is_long[h]) {
+        a.long_slot[h] = (int16_t)slot;
+        ra.long_heads[slot] = (int16_t)h;
+        ++slot;
+      }
+  }
+  AttnMaps m;
+  if (!make_map(&m.q, at<void>(ws, P.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.k, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.v, V, p->d, p->T, Hkv, B, p->v_stride[2], p->v_stride[1], p->v_stride[0])) return SATTN_ERR_CUDA;
+  m.q2 = m.q;
+  m.kg = m.k;
+  m.vg = m.v;
+  if (P.n_long > 0 && R > 0 && P.N > 1) {
+    ra.B = p->B;
+    ra.Hq = p->Hq;
+    ra.Hkv = p->Hkv;
+    ra.T = p->T;
+    ra.d = p->d;
+    ra.S = S;
+    ra.N = P.N;
+    ra.R = R;
+    ra.blk = retr_block;
+    ra.n_long = P.n_long;
+    ra.Q = static_cast<const __nv_bfloat16*>(Q);
+    ra.K = static_cast<const __nv_bfloat16*>(K);
+    ra.V = static_cast<const __nv_bfloat16*>(V);
+    ra.q_sb = p->q_stride[0];
+    ra.q_sh = p->q_stride[1];
+    ra.q_st = p->q_stride[2];
+    ra.k_sb = p->k_stride[0];
+    ra.k_sh = p->k_stride[1];
+    ra.k_st = p->k_stride[2];
+    ra.v_sb = p->v_stride[0];
+    ra.v_sh = p->v_stride[1];
+    ra.v_st = p->v_stride[2];
+    ra.tab = at<float2>(ws, P.tab);
+    ra.prefix_blocks = prefix_blocks;
+    ra.prefix_cnt = at<int32_t>(ws, P.pcnt);
+    ra.Kpre = at<__nv_bfloat16>(ws, P.kpre);
+    ra.Vpre = at<__nv_bfloat16>(ws, P.vpre);
+    {
+      ProfScope ps("segment_retrieval", 2, st);
+      SATTN_TRY(launch_segment_retrieval(ra, st));
+    }
+    const int64_t planes = (int64_t)P.n_long * P.N;
+    if (!make_map(&m.kg, ra.Kpre, p->d, P.Rpad, planes, B, d, (int64_t)P.Rpad * d, planes * P.Rpad * d))
+      return SATTN_ERR_CUDA;
+    if (!make_map(&m.vg, ra.Vpre, p->d, P.Rpad, planes, B, d, (int64_t)P.Rpad * d, planes * P.Rpad * d))
+      return SATTN_ERR_CUDA;
+  }
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.nQT = P.nQT;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.ns_band = 0;
+  a.w_eff = 0x3fffffff;
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.gather_mode = 2;
+  a.q2 = false;
+  a.seg_S = S;
+  a.seg_M = M;
+  a.seg_N = P.N;
+  a.seg_R = R;
+  a.prefix_cnt = at<int32_t>(ws, P.pcnt);
+  a.n_long = std::max(P.n_long, 1);
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.status = at<int32_t>(ws, P.status);
+  ProfScope ps("attn_tc_segment", 1, st);
+  return cuda_rc(launch_attn_tc(a, m, st));
+}
+
+int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {
+  if (!ws || !device_status) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SATTN_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return SATTN_ERR_CUDA;
+  *device_status = v;
+  return SATTN_OK;
+}
+
+int sattn_profile_enable(int on) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = on != 0;
+  return SATTN_OK;
+}
+
+int sattn_profile_collect(char* names, int32_t* launches, double* total_ms, int32_t max_groups, int32_t* n_groups) {
+  if (!names || !launches || !total_ms || !n_groups || max_groups < 0) return SATTN_ERR_INVALID_ARG;
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    recs.swap(g_prof_recs);
+  }
+  std::map<std::string, std::pair<int64_t, double>> acc;
+  std::vector<std::string> order;
+  int rc = SATTN_OK;
+  for (const ProfRec& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) rc = SATTN_ERR_CUDA;
+    auto it = acc.find(r.name);
+    if (it == acc.end()) {
+      order.push_back(r.name);
+      acc[r.name] = {r.kernels, (double)ms};
+    } else {
+      it->second.first += r.kernels;
+      it->second.second += ms;
+    }
+  }
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    for (const ProfRec& r : recs) {
+      g_prof_pool.push_back(r.a);
+      g_prof_pool.push_back(r.b);
+    }
+  }
+  int n = 0;
+  for (const std::string& k : order) {
+    if (n >= max_groups) break;
+    std::strncpy(names + 32 * n, k.c_str(), 31);
+    names[32 * n + 31] = 0;
+    launches[n] = (int32_t)acc[k].first;
+    total_ms[n] = acc[k].second;
+    ++n;
+  }
+  *n_groups = n;
+  return rc;
+}
+
+}  // extern "C"

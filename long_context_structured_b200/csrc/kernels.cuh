@@ -1,0 +1,180 @@
+// kernels.cuh -- launch interfaces of the library's kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sattn {
+
+constexpr int kTile = 128;  // query-tile rows (BM) and key-tile columns (BN)
+constexpr int kMaxHeads = 256;
+
+// ---------------------------------------------------------------------------
+// K1: rotary table and the prep pass
+// ---------------------------------------------------------------------------
+// tab[p][c] = (cos, sin)(p * theta^(-2c/d)), computed in fp64, stored fp32.
+cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, cudaStream_t st);
+
+struct PrepArgs {
+  int B, Hq, Hkv, T, d;
+  const void* Q;  // bf16 or fp32 per `f32`
+  const void* K;
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st;
+  bool f32;
+  const float2* tab;  // nullptr: no rotation
+  int L;              // distance cap (0 = none)
+  __nv_bfloat16* Qr;  // [B,Hq,T,d] R(i) q_i            (may be null)
+  __nv_bfloat16* Qc;  // [B,Hq,T,d] R(L) q_i            (may be null)
+  __nv_bfloat16* Kr;  // [B,Hkv,T,d] R(j) k_j           (may be null)
+  float* sink_z;      // [B,Hq,T,n_sink] side logits    (may be null)
+  int n_sink;
+  uint32_t* kmax;     // [B*Hkv] max_j ||k_j|| as float bits (may be null)
+};
+cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K2: block map
+// ---------------------------------------------------------------------------
+struct BlockmapArgs {
+  int B, T, n_start, window;
+  const uint8_t* is_sep;  // may be null
+  int32_t* prefix;        // [B, T+1] workspace: separators (j >= n_start) before x
+  int32_t* sep_pos;       // [B, T]
+  int32_t* sep_count;     // [B]
+  int32_t* ranges;        // [B, nQT, 2]
+  uint8_t* cls;           // [B, nQT, nKT] or null
+};
+cudaError_t launch_blockmap(const BlockmapArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K3: separator K/V gather into dense per-(b, kv-head) arrays
+// ---------------------------------------------------------------------------
+struct GatherArgs {
+  int B, Hkv, T, Tpad, d;
+  const __nv_bfloat16* Ksrc;
+  int64_t k_sb, k_sh, k_st;
+  const __nv_bfloat16* Vsrc;
+  int64_t v_sb, v_sh, v_st;
+  const int32_t* sep_pos;    // [B, T]
+  const int32_t* sep_count;  // [B]
+  __nv_bfloat16* Ks;         // [B, Hkv, Tpad, d]
+  __nv_bfloat16* Vs;
+};
+cudaError_t launch_sep_gather(const GatherArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K5: tcgen05 attention
+// ---------------------------------------------------------------------------
+struct AttnArgs {
+  int B, Hq, Hkv, T, d, nQT;
+  float scale_log2;  // log2(e) / sqrt(d)
+  // band tiles over the main K/V
+  int ns_band;       // keys j < ns_band never go through the band (sinks use the side path)
+  int w_eff;         // band keeps j >= i - w_eff
+  // side keys (fp32 logits)
+  const float* sink_z;  // [B, Hq, T, n_sink]
+  int n_sink;
+  const int32_t* tk_idx;  // [B, Hq, T, topk]
+  const float* tk_z;
+  int topk;
+  const __nv_bfloat16* V;  // raw V for side keys
+  int64_t v_sb, v_sh, v_st;
+  // gathered tiles: 0 none, 1 separators, 2 segmented prefix
+  int gather_mode;
+  bool q2;                     // gathered tiles use the second query tile (Qc)
+  const int32_t* sep_pos;      // [B, T]
+  const int32_t* ranges;       // [B, nQT, 2]
+  int window;                  // w for the separator rule (sep kept iff pos < i - w)
+  // segmented execution
+  int seg_S, seg_M, seg_N, seg_R;
+  int16_t long_slot[kMaxHeads]; // head -> index among long heads, -1 for local
+  const int32_t* prefix_cnt;   // [B, Hl, N] number of prefix keys
+  int n_long;
+  // outputs
+  __nv_bfloat16* O;
+  int64_t o_sb, o_sh, o_st;
+  float* lse;
+  int32_t* status;
+};
+struct AttnMaps {
+  CUtensorMap q, q2, k, v, kg, vg;
+};
+cudaError_t launch_attn_tc(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K6: fp32 attention on CUDA cores
+// ---------------------------------------------------------------------------
+struct AttnF32Args {
+  int B, Hq, Hkv, T, d;
+  const float* Q;
+  const float* K;
+  const float* V;
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st;
+  const float2* tab;  // null: no rotation
+  int L, n_start, window;
+  const int32_t* sep_pos;    // [B, T] or null
+  const int32_t* sep_count;  // [B]
+  const int32_t* tk_idx;     // [B, Hq, T, topk] or null
+  const float* tk_z;
+  int topk;
+  float* O;
+  int64_t o_sb, o_sh, o_st;
+  float* lse;
+};
+cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K4: top-k middle-token selection
+// ---------------------------------------------------------------------------
+struct TopkArgs {
+  int B, Hq, Hkv, T, d, nQT;
+  int n_start, window, topk, L;
+  const uint8_t* is_sep;       // [B, T] or null
+  // raw inputs for the exact fp32 re-rank
+  const void* Q;
+  const void* K;
+  bool f32;
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st;
+  const float2* tab;           // null: no rotation
+  const uint32_t* kmax;        // [B*Hkv] max key norm (float bits)
+  int32_t* idx;                // [B, Hq, T, topk]
+  float* z;
+  int32_t* fallback_rows;      // [B*Hq*T] rows whose bf16 shortlist was not certified
+  int32_t* status;             // status[2] counts fallback rows
+  // shortlist from the tensor-core scoring pass
+  int short_len;               // shortlist length: 8, 16 or 32 (>= topk + 2)
+  int32_t* short_idx;          // [B*Hq*T, short_len]
+  float* short_thr;            // [B*Hq*T] coarse score of the last shortlisted key
+  int32_t* n_cand;             // [B*Hq*T] number of candidates of the row
+};
+constexpr int kShortlistMax = 32;
+struct TopkMaps {
+  CUtensorMap qsel, ksel;      // bf16 scoring operands: (Qc, K) capped, (Qr, Kr) otherwise
+};
+// scoring + shortlist (tensor cores), then exact re-rank and certification
+cudaError_t launch_topk_tc(const TopkArgs& a, const TopkMaps& m, cudaStream_t st);
+// exact fp32 scan for the rows listed in fallback_rows (count in status[2]),
+// or for every row when all_rows is set
+cudaError_t launch_topk_exact(const TopkArgs& a, bool all_rows, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// K7: segmented execution -- retrieval and prefix assembly
+// ---------------------------------------------------------------------------
+struct SegRetrArgs {
+  int B, Hq, Hkv, T, d, S, N, R, blk, n_long;
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st;
+  int16_t long_heads[kMaxHeads]; // head id of each long slot
+  const float2* tab;
+  int32_t* prefix_blocks;      // [B, Hq, N, R/blk] (all heads; -1 filled)
+  int32_t* prefix_cnt;         // [B, n_long, N]
+  __nv_bfloat16* Kpre;         // [B, n_long, N, R, d] rotated at virtual positions
+  __nv_bfloat16* Vpre;
+};
+cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st);
+
+}  // namespace sattn

@@ -1,0 +1,303 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Bars: block maps, separator lists, top-k selections and retrieved prefix
+blocks bit-exact (top-k / retrieval rows exempt only where the oracle's k-th
+and (k+1)-th logits are within 1e-4 relative); O and LSE within max-abs 2e-2
+and mean-abs 2e-3 for bf16 inputs, 1e-4 for the fp32 path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import long_context_structured_b200 as sa
+from long_context_structured_b200 import synth
+from _util import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, compare, gather_rows, to_dev, topk_agreement)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def _status_ok():
+    assert sa.stream_status() == 0, "device status word reports a failure"
+
+
+def _run_fwd(wl, inp, **kw):
+    q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
+    sep = to_dev(inp["is_sep"])
+    O, lse = sa.fwd(q, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                    rope_theta=wl.rope_theta, topk=wl.topk, is_sep=sep, **kw)
+    torch.cuda.synchronize()
+    _status_ok()
+    return O, lse
+
+
+def _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=None):
+    p = oracle_mod.params_of(wl)
+    Oref, lref, *_ = oracle_mod.fwd_rows(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows, forced_topk=forced)
+    Og = gather_rows(O, rows)
+    lg = gather_rows(lse, rows)
+    if wl.dtype == "f32":
+        compare("O", Og, Oref, F32_MAX_ABS)
+        compare("LSE", lg, lref, F32_MAX_ABS)
+    else:
+        compare("O", Og, Oref, BF16_MAX_ABS, BF16_MEAN_ABS)
+        compare("LSE", lg, lref, BF16_MAX_ABS, BF16_MEAN_ABS)
+
+
+# ---------------------------------------------------------------------------
+# block map (integer, bit-exact)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,T,ns,w,rate", [(1, 1024, 4, 128, 0.08), (3, 1000, 4, 37, 0.2), (2, 300, 0, 0, 0.5),
+                                           (1, 129, 7, 300, 1.0), (4, 8192, 4, 256, 0.10), (2, 777, 2, 5, 0.0)])
+def test_blockmap_bitexact(oracle_mod, B, T, ns, w, rate):
+    rng = np.random.default_rng(B * 1000 + T)
+    flags = (rng.random((B, T)) < rate).astype(np.uint8)
+    out = sa.build_blockmap(to_dev(flags), B=B, T=T, n_start=ns, window=w)
+    torch.cuda.synchronize()
+    cls, pos, cnt, rng_ = oracle_mod.blockmap(B, T, ns, w, 128, 128, flags)
+    assert np.array_equal(out["sep_count"].cpu().numpy(), cnt)
+    assert np.array_equal(out["sep_pos"].cpu().numpy(), pos)
+    assert np.array_equal(out["qtile_sep_range"].cpu().numpy(), rng_)
+    assert np.array_equal(out["cls"].cpu().numpy(), cls)
+
+
+def test_blockmap_c3_token_flags(oracle_mod):
+    wl = synth.WORKLOADS["c3_sepllm_gqa_8k"]
+    flags = synth.separator_flags(wl, 0)
+    out = sa.build_blockmap(to_dev(flags), B=wl.B, T=wl.T, n_start=wl.n_start, window=wl.window)
+    cls, pos, cnt, rng_ = oracle_mod.blockmap(wl.B, wl.T, wl.n_start, wl.window, 128, 128, flags)
+    assert np.array_equal(out["sep_count"].cpu().numpy(), cnt)
+    assert np.array_equal(out["sep_pos"].cpu().numpy(), pos)
+    assert np.array_equal(out["qtile_sep_range"].cpu().numpy(), rng_)
+    assert np.array_equal(out["cls"].cpu().numpy(), cls)
+
+
+# ---------------------------------------------------------------------------
+# fp32 path
+# ---------------------------------------------------------------------------
+
+def test_c1_f32_full(oracle_mod):
+    wl = synth.WORKLOADS["c1_f32_sep"]
+    inp = synth.make_inputs(wl, seed=0)
+    O, lse = _run_fwd(wl, inp)
+    rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows)
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(B=1, Hq=2, Hkv=1, T=300, d=64, n_start=2, window=20, L_pretrain=40, rope_theta=1e4, topk=3, sep_rate=0.1),
+    dict(B=2, Hq=2, Hkv=2, T=200, d=128, n_start=0, window=199, rope_theta=5e5),
+])
+def test_f32_features(oracle_mod, cfg):
+    wl = synth.Workload(name="f32", dtype="f32", **cfg)
+    inp = synth.make_inputs(wl, seed=5)
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, oracle_mod.all_rows(wl.B, wl.Hq, wl.T))
+
+
+# ---------------------------------------------------------------------------
+# bf16 tensor-core path, small shapes, every row
+# ---------------------------------------------------------------------------
+
+SMALL = [
+    ("dense_one_tile", dict(B=1, Hq=1, Hkv=1, T=128, d=128, n_start=0, window=127)),
+    ("causal_ragged_rope", dict(B=1, Hq=2, Hkv=2, T=300, d=128, n_start=0, window=1000, rope_theta=1e4)),
+    ("lambda_capped_gqa", dict(B=1, Hq=2, Hkv=1, T=1000, d=128, n_start=4, window=100, L_pretrain=100,
+                               rope_theta=1e4, sink_scale=8.0)),
+    ("sep_d64", dict(B=2, Hq=4, Hkv=2, T=700, d=64, n_start=1, window=37, rope_theta=1e4, sep_rate=0.1)),
+    ("sep_capped_q2", dict(B=1, Hq=2, Hkv=2, T=513, d=128, n_start=4, window=64, L_pretrain=64, rope_theta=1e4,
+                           sep_rate=0.3)),
+    ("window0_sep", dict(B=1, Hq=2, Hkv=2, T=400, d=128, n_start=0, window=0, sep_rate=0.5)),
+    ("all_separators", dict(B=1, Hq=1, Hkv=1, T=200, d=128, n_start=4, window=3, sep_rate=1.0)),
+    ("tiny_T", dict(B=1, Hq=1, Hkv=1, T=5, d=128, n_start=4, window=2, rope_theta=1e4)),
+    ("all_sinks", dict(B=1, Hq=1, Hkv=1, T=3, d=128, n_start=8, window=1)),
+    ("window_uncapped_long", dict(B=1, Hq=1, Hkv=1, T=900, d=128, n_start=4, window=200, L_pretrain=300,
+                                  rope_theta=1e4)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", SMALL, ids=[s[0] for s in SMALL])
+def test_bf16_small(oracle_mod, name, cfg):
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    inp = synth.make_inputs(wl, seed=7)
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, oracle_mod.all_rows(wl.B, wl.Hq, wl.T))
+
+
+def test_bf16_topk_small(oracle_mod):
+    wl = synth.Workload(name="topk_small", B=1, Hq=2, Hkv=2, T=2048, d=128, dtype="bf16", n_start=4, window=256,
+                        L_pretrain=256, rope_theta=1e4, topk=5, plant=2)
+    inp = synth.make_inputs(wl, seed=11)
+    q, k = to_dev(inp["q"]), to_dev(inp["k"])
+    idx, z = sa.topk_select(q, k, topk=wl.topk, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                            rope_theta=wl.rope_theta)
+    torch.cuda.synchronize()
+    _status_ok()
+    rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + 1))
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], None, rows)
+    gi = idx.cpu().numpy().reshape(-1, wl.topk)
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
+    assert not bad, "rows %s differ without a near tie" % bad[:10]
+    # logits of agreeing rows match the oracle's in fp32
+    gz = z.cpu().numpy().reshape(-1, wl.topk).astype(np.float64)
+    same = np.all(gi == ref_idx[:, : wl.topk], axis=1)
+    fin = np.isfinite(ref_z[same, : wl.topk])
+    assert np.allclose(gz[same][fin], ref_z[same, : wl.topk][fin], rtol=1e-5, atol=1e-4)
+    # attention with the selection inside the call
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi)
+
+
+# ---------------------------------------------------------------------------
+# properties on the GPU
+# ---------------------------------------------------------------------------
+
+def test_full_causal_matches_sdpa():
+    torch.manual_seed(0)
+    B, H, T, d = 1, 4, 1000, 128
+    q = torch.randn(B, H, T, d, device="cuda").bfloat16()
+    k = torch.randn(B, H, T, d, device="cuda").bfloat16()
+    v = torch.randn(B, H, T, d, device="cuda").bfloat16()
+    O, lse = sa.fwd(q, k, v, n_start=0, window=T)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(), is_causal=True)
+    compare("O vs SDPA", O.double().cpu().numpy(), ref.cpu().numpy(), BF16_MAX_ABS, BF16_MEAN_ABS)
+
+
+def test_invariant_outside_kept_set():
+    wl = synth.Workload(name="inv", B=1, Hq=1, Hkv=1, T=1500, d=128, dtype="bf16", n_start=4, window=100,
+                        L_pretrain=100, rope_theta=1e4, sep_rate=0.05)
+    inp = synth.make_inputs(wl, seed=3)
+    O0, l0 = _run_fwd(wl, inp)
+    i = 1400
+    flags = inp["is_sep"][0]
+    keep = np.zeros(wl.T, bool)
+    keep[: wl.n_start] = True
+    keep[i - wl.window: i + 1] = True
+    keep[np.flatnonzero(flags[: i])] = True
+    inp2 = dict(inp)
+    v2 = inp["v"].copy()
+    k2 = inp["k"].copy()
+    out_idx = np.flatnonzero(~keep[: i])
+    v2[0, 0, out_idx] ^= np.uint16(0x0123)
+    k2[0, 0, out_idx] ^= np.uint16(0x0101)
+    inp2["v"], inp2["k"] = v2, k2
+    O1, l1 = _run_fwd(wl, inp2)
+    assert torch.equal(O0[0, 0, i], O1[0, 0, i]) and torch.equal(l0[0, 0, i], l1[0, 0, i])
+
+
+def test_deterministic():
+    wl = synth.Workload(name="det", B=1, Hq=2, Hkv=2, T=2000, d=128, dtype="bf16", n_start=4, window=500,
+                        L_pretrain=500, rope_theta=1e4, topk=3)
+    inp = synth.make_inputs(wl, seed=4)
+    a = _run_fwd(wl, inp)
+    b = _run_fwd(wl, inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_host_tensors_end_to_end():
+    wl = synth.Workload(name="e2e", B=1, Hq=2, Hkv=2, T=600, d=128, dtype="bf16", n_start=4, window=128,
+                        L_pretrain=128, rope_theta=1e4)
+    inp = synth.make_inputs(wl, seed=9)
+    Od, ld = _run_fwd(wl, inp)
+    qh, kh, vh = (to_dev(inp[x], device="cpu") for x in ("q", "k", "v"))
+    Oh, lh = sa.fwd(qh, kh, vh, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                    rope_theta=wl.rope_theta)
+    assert Oh.device.type == "cpu"
+    assert torch.equal(Oh, Od.cpu()) and torch.equal(lh, ld.cpu())
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads on sampled rows
+# ---------------------------------------------------------------------------
+
+def test_c2_full_size_sampled(oracle_mod):
+    wl = synth.WORKLOADS["c2_lminf_16k"]
+    inp = synth.make_inputs(wl, seed=0)
+    O, lse = _run_fwd(wl, inp)
+    rows = synth.sample_rows(wl, 48, seed=1)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows)
+
+
+def test_c3_full_size_sampled(oracle_mod):
+    wl = synth.WORKLOADS["c3_sepllm_gqa_8k"]
+    inp = synth.make_inputs(wl, seed=0)
+    O, lse = _run_fwd(wl, inp)
+    rows = synth.sample_rows(wl, 12, seed=2)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows)
+
+
+def test_c4_topk_full_size_sampled(oracle_mod):
+    wl = synth.WORKLOADS["c4_lminf_topk_32k"]
+    inp = synth.make_inputs(wl, seed=0)
+    q, k = to_dev(inp["q"]), to_dev(inp["k"])
+    idx, z = sa.topk_select(q, k, topk=wl.topk, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                            rope_theta=wl.rope_theta)
+    torch.cuda.synchronize()
+    _status_ok()
+    planted_rows = [(b, h, s + x) for (b, h, j, s) in inp["meta"]["planted"][::16] for x in (0, 31)]
+    rows = synth.sample_rows(wl, 6, seed=3, extra=planted_rows)
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + 1))
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], None, rows)
+    gi = gather_rows(idx, rows).astype(np.int64)
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
+    assert not bad, "rows %s differ without a near tie" % [tuple(rows[r]) for r in bad[:10]]
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi.astype(np.int32))
+
+
+def test_c5_segmented_full_size(oracle_mod):
+    wl = synth.WORKLOADS["c5_segmented_32k"]
+    inp = synth.make_inputs(wl, seed=0)
+    q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
+    O, lse, pb = sa.segment_fwd(q, k, v, S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
+                                is_long=inp["is_long"], rope_theta=wl.rope_theta)
+    torch.cuda.synchronize()
+    _status_ok()
+    p = oracle_mod.params_of(wl)
+    ref_pb, kth = oracle_mod.segment_blocks(p, wl.seg_S, wl.seg_R, wl.retr_block, inp["is_long"], inp["q"], inp["k"])
+    got_pb = pb.cpu().numpy()
+    diff = np.argwhere(np.any(got_pb != ref_pb, axis=-1))
+    for (b, h, s) in diff:
+        a, c = kth[b, h, s]
+        assert abs(a - c) <= 1e-4 * max(abs(a), abs(c)), "prefix blocks differ at (%d,%d,%d) without a tie" % (b, h, s)
+    assert len(diff) <= 2
+    rows = synth.sample_rows(wl, 24, seed=4)
+    Oref, lref, _ = oracle_mod.segment_rows(p, wl.seg_S, wl.seg_M, wl.seg_R, wl.retr_block, inp["is_long"],
+                                            inp["q"], inp["k"], inp["v"], rows)
+    compare("O", gather_rows(O, rows), Oref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare("LSE", gather_rows(lse, rows), lref, BF16_MAX_ABS, BF16_MEAN_ABS)
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(T=1024, S=256, M=64, R=128, blk=64, long=(0, 1)),
+    dict(T=768, S=256, M=300, R=256, blk=32, long=(1, 1)),
+    dict(T=512, S=128, M=0, R=0, blk=16, long=(0, 1)),
+])
+def test_segmented_small_all_rows(oracle_mod, cfg):
+    wl = synth.Workload(name="seg", B=1, Hq=2, Hkv=2, T=cfg["T"], d=128, dtype="bf16", rope_theta=1e4,
+                        seg_S=cfg["S"], seg_M=cfg["M"], seg_R=cfg["R"], retr_block=cfg["blk"],
+                        long_heads=tuple(h for h in range(2) if cfg["long"][h]))
+    inp = synth.make_inputs(wl, seed=12)
+    q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
+    O, lse, pb = sa.segment_fwd(q, k, v, S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
+                                is_long=inp["is_long"], rope_theta=wl.rope_theta)
+    torch.cuda.synchronize()
+    _status_ok()
+    p = oracle_mod.params_of(wl)
+    if wl.seg_R > 0:
+        ref_pb, _ = oracle_mod.segment_blocks(p, wl.seg_S, wl.seg_R, wl.retr_block, inp["is_long"], inp["q"], inp["k"])
+        assert np.array_equal(pb.cpu().numpy(), ref_pb)
+    rows = oracle_mod.all_rows(1, 2, wl.T)
+    Oref, lref, _ = oracle_mod.segment_rows(p, wl.seg_S, wl.seg_M, wl.seg_R, wl.retr_block, inp["is_long"],
+                                            inp["q"], inp["k"], inp["v"], rows)
+    compare("O", gather_rows(O, rows), Oref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare("LSE", gather_rows(lse, rows), lref, BF16_MAX_ABS, BF16_MEAN_ABS)
