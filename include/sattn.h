@@ -178,6 +178,25 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
  * the synchronisation itself failed (the CUDA error is then sticky). */
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status);
 
+/* Block map without a workspace (no counterpart on the pages: it exists for
+ * callers that may not allocate device memory or hand over a workspace, e.g.
+ * an extension running inside a host framework that owns all device memory,
+ * or a latency-critical loop where an allocation -- which can synchronise
+ * the device -- is not allowed).  Same arguments and outputs as
+ * sattn_build_blockmap minus ws/ws_bytes; the scratch (separator prefix
+ * counts) lives in a fixed 4 MiB device array that every GPU loading the
+ * library keeps until exit.
+ *  - B * (T + 1) <= 1048576, else SATTN_ERR_UNSUPPORTED (nothing launched).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
+ *  - All calls share the array, which keeps the last call's contents (no part
+ *    of it needs to start at zero).  Calls that overlap on the GPU -- other
+ *    streams, other host threads -- race on it: serialise them. */
+int sattn_build_blockmap_noalloc(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
+                                 int32_t* sep_count, int32_t* qtile_sep_range, void* stream);
+
 /* Instrumentation (no counterpart on the pages).  While enabled, every kernel
  * launch group of the library is bracketed by CUDA events recorded on the
  * launch stream; the events cost a few hundred nanoseconds of device time

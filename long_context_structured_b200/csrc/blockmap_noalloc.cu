@@ -1,0 +1,80 @@
+// blockmap_noalloc.cu -- sattn_build_blockmap_noalloc: the block map and
+// separator compaction with its scratch in a fixed device array, for callers
+// that cannot give the library a workspace.
+//
+// Who needs this: code that runs where it may not allocate device memory or
+// own a workspace buffer -- for example a plugin or callback inside a host
+// framework that manages every byte of device memory itself and forbids its
+// extensions from allocating, or a latency-critical loop in which an
+// allocation (which can implicitly synchronise the device) is not allowed.
+// Such a caller still provides the inputs and outputs; the only scratch the
+// block map needs (per-sequence separator prefix counts) lives in the static
+// array below.
+//
+// Cost and limits:
+//   - every GPU that loads libsattn.so holds kNoallocScratchInts int32
+//     (4 MiB) for this array until the process exits;
+//   - B * (T + 1) must not exceed kNoallocScratchInts;
+//   - all calls share the one array: calls whose executions overlap on the
+//     GPU (different streams, or several host threads) race on it and give
+//     undefined results; serialise them;
+//   - the array keeps the previous call's contents; nothing in it has to
+//     start at zero, because the scan kernel rewrites every entry
+//     [b*(T+1), b*(T+1)+T] before the class kernel reads it.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/sattn.h"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr size_t kNoallocScratchInts = size_t(1) << 20;  // 4 MiB of int32
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_blockmap_scratch[kNoallocScratchInts];
+
+std::mutex g_setup_mu;
+int32_t* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The first call
+// on each device resolves it with cudaGetSymbolAddress; the name of a
+// __device__ array is only a host-side stand-in, never a device pointer.
+int scratch_for_current_device(int32_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> g(g_setup_mu);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_blockmap_scratch) != cudaSuccess || !ptr) return SATTN_ERR_CUDA;
+    g_scratch_addr[dev] = static_cast<int32_t*>(ptr);
+  }
+  *out = g_scratch_addr[dev];
+  return SATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int sattn_build_blockmap_noalloc(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls,
+                                            int32_t* sep_pos, int32_t* sep_count, int32_t* qtile_sep_range,
+                                            void* stream) {
+  if (!p || !sep_pos || !sep_count || !qtile_sep_range) return SATTN_ERR_INVALID_ARG;
+  if (p->B < 1 || p->T < 1 || p->n_start < 0 || p->window < 0) return SATTN_ERR_INVALID_ARG;
+  if ((size_t)p->B * ((size_t)p->T + 1) > kNoallocScratchInts) return SATTN_ERR_UNSUPPORTED;
+  int32_t* scratch = nullptr;
+  int rc = scratch_for_current_device(&scratch);
+  if (rc != SATTN_OK) return rc;
+  sattn::BlockmapArgs a{};
+  a.B = p->B;
+  a.T = p->T;
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.is_sep = is_sep;
+  a.prefix = scratch;
+  a.sep_pos = sep_pos;
+  a.sep_count = sep_count;
+  a.ranges = qtile_sep_range;
+  a.cls = cls;
+  return sattn::launch_blockmap(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
