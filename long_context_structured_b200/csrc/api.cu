@@ -584,7 +584,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.lse = lse;
   a.status = at<int32_t>(ws, P.status);
   ProfScope ps("attn_tc", 1, st);
-  return cuda_rc(launch_attn_tc(a, m, st));
+  return cuda_rc(q2 ? launch_attn_tc(a, m, st) : launch_attn_tc2(a, m, st));
 }
 
 // ---------------------------------------------------------------------------
@@ -752,7 +752,7 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
   a.lse = lse;
   a.status = at<int32_t>(ws, P.status);
   ProfScope ps("attn_tc_segment", 1, st);
-  return cuda_rc(launch_attn_tc(a, m, st));
+  return cuda_rc((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc(a, m, st));
 }
 
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {

@@ -205,7 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO = tmem + 256;
   volatile int* abort_flag = sm.abort_flag;
 
@@ -240,9 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           c2 = g;
         }
         mbar_expect_tx(sm.k_full + st, kTileBytes);
-        for (int c = 0; c < kChunks; ++c) tma_load_4d(sm.k[st] + c * kChunkBytes, mk, sm.k_full + st, c * 64, row, c2, b);
+        for (int c = 0; c < kChunks; ++c) tma_load_4d((sm.k[0] + st * kTileBytes) + c * kChunkBytes, mk, sm.k_full + st, c * 64, row, c2, b);
         mbar_expect_tx(sm.v_full + st, kTileBytes);
-        for (int c = 0; c < kChunks; ++c) tma_load_4d(sm.v[st] + c * kChunkBytes, mv, sm.v_full + st, c * 64, row, c2, b);
+        for (int c = 0; c < kChunks; ++c) tma_load_4d((sm.v[0] + st * kTileBytes) + c * kChunkBytes, mv, sm.v_full + st, c * 64, row, c2, b);
         ++issued;
       }
       if (!ok) {
@@ -266,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(sm.p_full, jt & 1, abort_flag, a.status, kSitePFull)) return false;
         if (!mbar_wait(sm.v_full + st, (jt / kNS) & 1, abort_flag, a.status, kSiteVFull)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.v[st]);
+        const uint32_t v_addr = smem_u32((sm.v[0] + st * kTileBytes));
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
@@ -285,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_addr = (it < tp.n_gather && a.q2) ? q2_addr : q_addr;
-        const uint32_t k_addr = smem_u32(sm.k[st]);
+        const uint32_t k_addr = smem_u32((sm.k[0] + st * kTileBytes));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
           const uint64_t ad = smem_desc_sw128(a_addr + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_addr + off, 16, 1024);
-          tc_mma_ss(tS[sb], ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          tc_mma_ss((tmem + sb * 128u), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(sm.s_full + sb);
         if (it >= 1) ok = issue_pv(it - 1);
@@ -319,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tcgen05.ld is warp-collective: all lanes take part even after a failure
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS[sb] + lane_off + c * 32, sv + c * 32);
+      for (int c = 0; c < 4; ++c) tmem_ld32((tmem + sb * 128u) + lane_off + c * 32, sv + c * 32);
       tc_wait_ld();
       tc_fence_before();
       if (ok) mbar_arrive(sm.s_free + sb);
@@ -352,16 +351,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           c_hi = i - j0;
         }
       }
-      float mx = -CUDART_INF_F;
+      // row max with 8 independent partial maxima (short dependency chains)
       if (c_lo > 0 || c_hi < kTile - 1) {
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) {
+        for (int c = 0; c < kTile; ++c)
           if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;
-          mx = fmaxf(mx, sv[c]);
-        }
-      } else {
+      }
+      float mx;
+      {
+        float pm[8];
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, sv[c]);
+        for (int x = 0; x < 8; ++x) pm[x] = sv[x];
+#pragma unroll
+        for (int c = 8; c < kTile; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
+        mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       }
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_used, m_tile);
@@ -374,18 +377,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum *= alpha;
         m_used = m_new;
       }
-      float rs = 0.f;
-      if (m_used == -CUDART_INF_F) {
+      // P = 2^(s*log2e/sqrt(d) - m), packed to bf16 pairs at once; 8 partial sums
+      uint32_t pk[kTile / 2];
+      {
+        float ps[8];
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) sv[c] = 0.f;
-      } else {
+        for (int x = 0; x < 8; ++x) ps[x] = 0.f;
+        const float neg_m = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
+        const bool none = (m_used == -CUDART_INF_F);
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          sv[c] = ex2_approx(fmaf(sv[c], sl2, -m_used));
-          rs += sv[c];
+        for (int c = 0; c < kTile; c += 2) {
+          float p0 = ex2_approx(fmaf(sv[c], sl2, neg_m));
+          float p1 = ex2_approx(fmaf(sv[c + 1], sl2, neg_m));
+          if (none) p0 = p1 = 0.f;
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
         }
+        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
-      l_sum += rs;
 
       // PV of the previous tile must be done: P buffer free and O stable
       if (it > 0) {
@@ -409,11 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int gq = 0; gq < 16; ++gq) {
         const int kc = gq >> 3, gg = gq & 7;
-        uint4 val;
-        val.x = pack_bf16x2(sv[gq * 8 + 0], sv[gq * 8 + 1]);
-        val.y = pack_bf16x2(sv[gq * 8 + 2], sv[gq * 8 + 3]);
-        val.z = pack_bf16x2(sv[gq * 8 + 4], sv[gq * 8 + 5]);
-        val.w = pack_bf16x2(sv[gq * 8 + 6], sv[gq * 8 + 7]);
+        const uint4 val = make_uint4(pk[gq * 4 + 0], pk[gq * 4 + 1], pk[gq * 4 + 2], pk[gq * 4 + 3]);
         *reinterpret_cast<uint4*>(sm.p + kc * kChunkBytes + sw128_offset(r, gg)) = val;
       }
       fence_proxy_async_smem();

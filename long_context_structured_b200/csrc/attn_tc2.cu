@@ -1,0 +1,575 @@
+// attn_tc2.cu -- K5, two query tiles per CTA: the production attention
+// kernel for every case except capped separator tiles (those need a second
+// query operand per tile and run on attn_tc.cu).
+//
+// Same mathematics as attn_tc.cu (see its header): band tiles, gathered
+// separator / prefix tiles, fp32 side keys merged in the epilogue.  What
+// changes is the schedule:
+//   - one CTA = two 128-row query tiles (Q0 rows i0..i0+127, Q1 the next 128)
+//     of one (batch, head); every K/V tile either of them needs is loaded
+//     once and used by both;
+//   - two softmax warpgroups (one per query tile) ping-pong against the
+//     tensor core; the single-thread MMA issuer interleaves
+//         PV0(prev), S0(p), PV1(prev), S1(p)
+//     so that while one warpgroup turns S into P the tensor core works on the
+//     other tile;
+//   - P (bf16) is written back into TMEM over its own S columns and the PV
+//     product reads it from there (A operand in tensor memory), so P never
+//     touches shared memory;
+//   - TMEM: S0 | S1 | O0 | O1 (4 x 128 fp32 columns);
+//   - K ring of 3 stages, V ring of 2 stages.
+// Ordering facts used: tcgen05.commit arrives only after every earlier MMA
+// of the issuing thread completed, so "S_i(p) done" implies "PV_i(prev)
+// done" (O_i stable for rescaling, P_i columns free).  Before S_i(p)
+// overwrites the columns that PV_i(prev) reads, the issuer waits for that PV.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace sattn {
+
+namespace {
+
+constexpr int kThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
+constexpr int kKS = 3;         // K stages
+constexpr int kVS = 2;         // V stages
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+
+__device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
+  uint32_t a = smem_u32(bar);
+  uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 100000000ull) return false;
+  }
+  return true;
+}
+
+// A[tmem] operand form: D[tmem] (+)= A[tmem] * B[smem]^T
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
+// then band key tiles [u_lo, u_lo + n_band).
+struct Plan {
+  int g_count, g_full, n_gather, band_lo, u_lo, n_band, rows;  // rows: valid rows of the tile (0 = none)
+};
+
+__device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t) {
+  Plan p;
+  p.g_count = 0;
+  p.g_full = 0;
+  p.band_lo = 0;
+  const int i0 = t * kTile;
+  p.rows = (i0 < a.T) ? min(kTile, a.T - i0) : 0;
+  if (p.rows == 0) {
+    p.n_gather = p.n_band = p.u_lo = 0;
+    return p;
+  }
+  if (a.gather_mode == 1) {
+    p.g_full = a.ranges[(b * a.nQT + t) * 2 + 0];
+    p.g_count = a.ranges[(b * a.nQT + t) * 2 + 1];
+  } else if (a.gather_mode == 2) {
+    const int s = i0 / a.seg_S;
+    const int seg0 = s * a.seg_S;
+    const int slot = a.long_slot[h];
+    if (slot >= 0) {
+      p.band_lo = seg0;
+      if (s > 0) p.g_count = p.g_full = a.prefix_cnt[(b * a.n_long + slot) * a.seg_N + s];
+    } else {
+      p.band_lo = s > 0 ? max(0, seg0 - a.seg_M) : 0;
+    }
+  }
+  p.n_gather = (p.g_count + kTile - 1) / kTile;
+  const int i_last = i0 + p.rows - 1;
+  const int j_lo = max(max(p.band_lo, 0), max(i0 - a.w_eff, a.ns_band));
+  if (j_lo > i_last) {
+    p.u_lo = 0;
+    p.n_band = 0;
+  } else {
+    p.u_lo = j_lo / kTile;
+    p.n_band = i_last / kTile - p.u_lo + 1;
+  }
+  return p;
+}
+
+// Union order: gathered positions [0, NG), then band tiles u in [U0, U1].
+struct Union {
+  int NG, U0, n;
+};
+
+__device__ __forceinline__ bool needs(const Plan& p, const Union& un, int pos) {
+  if (p.rows == 0) return false;
+  if (pos < un.NG) return pos < p.n_gather;
+  const int u = un.U0 + (pos - un.NG);
+  return u >= p.u_lo && u < p.u_lo + p.n_band;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
+                    const __grid_constant__ CUtensorMap tmVg, const AttnArgs a, int nQB) {
+  constexpr uint32_t kTileBytes = D * kTile * 2;
+  constexpr int kChunks = D / 64;
+  constexpr uint32_t kChunkBytes = kTile * 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;                                 // Q0 | Q1
+  uint8_t* sK = base + 2 * kTileBytes;                // kKS stages
+  uint8_t* sV = sK + kKS * kTileBytes;                // kVS stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVS * kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kKS;
+  uint64_t* v_full = k_empty + kKS;
+  uint64_t* v_empty = v_full + kVS;
+  uint64_t* s_full = v_empty + kVS;   // [2]
+  uint64_t* p_full = s_full + 2;      // [2]
+  uint64_t* o_done = p_full + 2;      // [2]
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_i = reinterpret_cast<int*>(tmem_slot + 1);
+  int* early = abort_i + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qb = blockIdx.x % nQB;
+  const int bh = blockIdx.x / nQB;
+  const int h = bh % a.Hq;
+  const int b = bh / a.Hq;
+  const int g = h / (a.Hq / a.Hkv);
+  const Plan pl0 = make_plan(a, b, h, 2 * qb);
+  const Plan pl1 = make_plan(a, b, h, 2 * qb + 1);
+  Union un;
+  un.NG = max(pl0.n_gather, pl1.n_gather);
+  {
+    int u0 = 1 << 30, u1 = -1;
+    if (pl0.n_band > 0) {
+      u0 = min(u0, pl0.u_lo);
+      u1 = max(u1, pl0.u_lo + pl0.n_band - 1);
+    }
+    if (pl1.n_band > 0) {
+      u0 = min(u0, pl1.u_lo);
+      u1 = max(u1, pl1.u_lo + pl1.n_band - 1);
+    }
+    un.U0 = (u1 >= 0) ? u0 : 0;
+    un.n = un.NG + ((u1 >= 0) ? (u1 - u0 + 1) : 0);
+  }
+  const int g_plane = (a.gather_mode == 2 && a.long_slot[h] >= 0)
+                          ? a.long_slot[h] * a.seg_N + (2 * qb * kTile) / a.seg_S
+                          : g;
+
+  if (threadIdx.x == 0) {
+    *early = status_failed(a.status) ? 1 : 0;
+    *abort_i = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kKS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, 128);
+      mbar_init(o_done + x, 1);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (*early) return;
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_flag = abort_i;
+
+  if (warp == 8) {
+    // ===================== TMA producer =====================
+    if (lane == 0 && un.n > 0) {
+      const int i0 = 2 * qb * kTile;
+      mbar_expect_tx(q_full, 2 * kTileBytes);
+      for (int x = 0; x < 2; ++x)
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_4d(sQ + x * kTileBytes + c * kChunkBytes, &tmQ, q_full, c * 64, i0 + x * kTile, h, b);
+      int issued = 0;
+      bool ok = true;
+      for (int p = 0; p < un.n && ok; ++p) {
+        const bool gat = p < un.NG;
+        const int row = gat ? p * kTile : (un.U0 + p - un.NG) * kTile;
+        const int c2 = gat ? g_plane : g;
+        const CUtensorMap* mk = gat ? &tmKg : &tmK;
+        const CUtensorMap* mv = gat ? &tmVg : &tmV;
+        const int ks = p % kKS, vs = p % kVS;
+        if (p >= kKS) ok = mbar_wait(k_empty + ks, ((p / kKS) - 1) & 1, abort_flag, a.status, 31);
+        if (!ok) break;
+        mbar_expect_tx(k_full + ks, kTileBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_4d(sK + ks * kTileBytes + c * kChunkBytes, mk, k_full + ks, c * 64, row, c2, b);
+        if (p >= kVS) ok = mbar_wait(v_empty + vs, ((p / kVS) - 1) & 1, abort_flag, a.status, 32);
+        if (!ok) break;
+        mbar_expect_tx(v_full + vs, kTileBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_4d(sV + vs * kTileBytes + c * kChunkBytes, mv, v_full + vs, c * 64, row, c2, b);
+        ++issued;
+      }
+      if (!ok) {
+        mbar_wait_raw(q_full, 0);
+        for (int p = max(0, issued - kVS); p < issued; ++p) {
+          mbar_wait_raw(k_full + p % kKS, (p / kKS) & 1);
+          mbar_wait_raw(v_full + p % kVS, (p / kVS) & 1);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ===================== MMA issuer =====================
+    if (lane == 0 && un.n > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.status, 33);
+      int n_pv[2] = {0, 0};    // PV issued per tile
+      int prev[2] = {-1, -1};  // union position whose PV is still pending, per tile
+      int v_users[kVS];        // PVs still to come for the position held by each V stage
+      for (int y = 0; y < kVS; ++y) v_users[y] = 0;
+      auto issue_pv = [&](int x) -> bool {
+        const int pp = prev[x];
+        const int vs = pp % kVS;
+        if (!mbar_wait(p_full + x, n_pv[x] & 1, abort_flag, a.status, 34 + x)) return false;
+        if (!mbar_wait(v_full + vs, (pp / kVS) & 1, abort_flag, a.status, 36)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV + vs * kTileBytes);
+        const uint32_t p_tmem = tmem + x * 128;
+        const uint32_t o_tmem = tmem + 256 + x * 128;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
+          tc_mma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_o, (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(o_done + x);
+        // the V stage is free once every tile that uses this position ran its PV
+        if (--v_users[vs] == 0) tc_commit(v_empty + vs);
+        ++n_pv[x];
+        prev[x] = -1;
+        return true;
+      };
+      for (int p = 0; p < un.n && ok; ++p) {
+        const int ks = p % kKS;
+        const bool need[2] = {needs(pl0, un, p), needs(pl1, un, p)};
+        const int users = (need[0] ? 1 : 0) + (need[1] ? 1 : 0);
+        bool k_ready = false;
+        for (int x = 0; x < 2 && ok; ++x) {
+          // the tile's pending PV goes first (ping-pong: PV0, S0, PV1, S1)
+          const bool had_pv = prev[x] >= 0;
+          if (had_pv) ok = issue_pv(x);
+          if (!ok || !need[x]) continue;
+          if (had_pv) {
+            // P_x (read by that PV) lives in the columns S_x is about to overwrite
+            ok = mbar_wait(o_done + x, (n_pv[x] - 1) & 1, abort_flag, a.status, 38 + x);
+            if (!ok) break;
+          }
+          if (!k_ready) {
+            ok = mbar_wait(k_full + ks, (p / kKS) & 1, abort_flag, a.status, 40);
+            if (!ok) break;
+            k_ready = true;
+            v_users[p % kVS] = users;
+          }
+          tc_fence_after();
+          const uint32_t a_base = q_addr + x * kTileBytes;
+          const uint32_t k_addr = smem_u32(sK + ks * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+            tc_mma_ss(tmem + x * 128, smem_desc_sw128(a_base + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                      idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full + x);
+          prev[x] = p;
+          const bool later_user = (x == 0) && need[1];
+          if (!later_user) tc_commit(k_empty + ks);
+        }
+        if (ok && users == 0) {
+          // no tile reads this position (cannot happen for contiguous plans); release it
+          ok = mbar_wait(k_full + ks, (p / kKS) & 1, abort_flag, a.status, 40);
+          if (!ok) break;
+          tc_commit(k_empty + ks);
+          ok = mbar_wait(v_full + p % kVS, (p / kVS) & 1, abort_flag, a.status, 36);
+          if (ok) tc_commit(v_empty + p % kVS);
+        }
+      }
+      for (int x = 0; x < 2 && ok; ++x)
+        if (prev[x] >= 0) ok = issue_pv(x);
+      tc_commit(drain);
+      mbar_wait_raw(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ===================== softmax + epilogue (warpgroups 0 and 1) =====================
+    const int x = warp >> 2;  // query tile of this warpgroup
+    const Plan& pl = x == 0 ? pl0 : pl1;
+    const int r = threadIdx.x & 127;
+    const int i0 = (2 * qb + x) * kTile;
+    const int i = i0 + r;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + x * 128;
+    const uint32_t tO = tmem + 256 + x * 128;
+    const float sl2 = a.scale_log2;
+    float m_used = -CUDART_INF_F;
+    float l_sum = 0.f;
+    bool ok = true;
+    int k = 0;  // tiles processed by this warpgroup
+    for (int p = 0; p < un.n; ++p) {
+      if (!needs(pl, un, p)) continue;
+      ok = ok && mbar_wait(s_full + x, k & 1, abort_flag, a.status, 41 + x);
+      tc_fence_after();
+      int c_lo = 0, c_hi = kTile - 1;
+      if (p < un.NG) {
+        const int r0 = p * kTile;
+        if (r0 + kTile > pl.g_full) {
+          int lim = min(kTile, pl.g_count - r0);
+          if (a.gather_mode == 1) {
+            const int* pos = a.sep_pos + (size_t)b * a.T + r0;
+            const int thr = i - a.window;
+            int lo = 0, hi = max(lim, 0);
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (__ldg(pos + mid) < thr) lo = mid + 1; else hi = mid;
+            }
+            lim = lo;
+          }
+          c_hi = lim - 1;
+        }
+      } else {
+        const int j0 = (un.U0 + p - un.NG) * kTile;
+        const int lo_fix = max(pl.band_lo, a.ns_band);
+        const bool full = (j0 + kTile - 1 <= i0) && (j0 >= max(lo_fix, i0 + kTile - 1 - a.w_eff));
+        if (!full) {
+          c_lo = max(lo_fix, i - a.w_eff) - j0;
+          c_hi = i - j0;
+        }
+      }
+      const bool partial = (c_lo > 0 || c_hi < kTile - 1);
+      // pass 1: row max over the two 64-column halves of S (8 partial maxima)
+      float pm[8];
+#pragma unroll
+      for (int y = 0; y < 8; ++y) pm[y] = -CUDART_INF_F;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        float sv[64];
+        tmem_ld32(tS + lane_off + hf * 64, sv);
+        tmem_ld32(tS + lane_off + hf * 64 + 32, sv + 32);
+        tc_wait_ld();
+        if (partial) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int cc = hf * 64 + c;
+            if (cc < c_lo || cc > c_hi) sv[c] = -CUDART_INF_F;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
+      }
+      const float mx =
+          fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float m_new = fmaxf(m_used, mx * sl2);
+      float alpha = 1.f;
+      bool rescale_o = false;
+      if (m_new > m_used + kRescaleThreshold) {
+        alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_new);
+        rescale_o = (k > 0) && (m_used != -CUDART_INF_F);
+        l_sum *= alpha;
+        m_used = m_new;
+      }
+      // O_x is stable here: S_x(p) completing implies the tile's previous PV completed
+      if (__any_sync(0xffffffffu, rescale_o)) {
+        const float f = rescale_o ? alpha : 1.f;
+        float ov[32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          tmem_ld32(tO + lane_off + c * 32, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int y = 0; y < 32; ++y) ov[y] *= f;
+          tmem_st32(tO + lane_off + c * 32, ov);
+        }
+      }
+      // pass 2: P = 2^(s*log2e/sqrt(d) - m) per half, packed to bf16 and stored
+      // into TMEM over the S columns already consumed (P half h -> columns
+      // [32h, 32h+32), i.e. over S columns this half has read)
+      {
+        float ps[8];
+#pragma unroll
+        for (int y = 0; y < 8; ++y) ps[y] = 0.f;
+        // a row with no key so far has m_used = -inf and every entry masked:
+        // with a zero offset each exp2(-inf) is exactly 0
+        const float neg_m = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          float sv[64];
+          tmem_ld32(tS + lane_off + hf * 64, sv);
+          tmem_ld32(tS + lane_off + hf * 64 + 32, sv + 32);
+          tc_wait_ld();
+          if (partial) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const int cc = hf * 64 + c;
+              if (cc < c_lo || cc > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0
+            }
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2_approx(fmaf(sv[c], sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(sv[c + 1], sl2, neg_m));
+            ps[(c >> 1) & 7] += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32u(tS + lane_off + hf * 32, pk);
+        }
+        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      }
+      tc_wait_st();
+      tc_fence_before();
+      if (ok) mbar_arrive(p_full + x);
+      ++k;
+    }
+
+    // ---- epilogue ----
+    if (k > 0) {
+      ok = ok && mbar_wait(o_done + x, (k - 1) & 1, abort_flag, a.status, 43 + x);
+      tc_fence_after();
+    }
+    const bool row_ok = (i < a.T);
+    const int ir = row_ok ? i : a.T - 1;
+    const size_t row_id = ((size_t)b * a.Hq + h) * a.T + ir;
+    const int n_sink = min(a.n_sink, ir + 1);
+    const float* sz = a.sink_z ? a.sink_z + row_id * a.n_sink : nullptr;
+    const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
+    const float* tkz = a.tk_z ? a.tk_z + row_id * a.topk : nullptr;
+    float m_fin = m_used;
+    for (int j = 0; j < n_sink; ++j) m_fin = fmaxf(m_fin, sz[j] * sl2);
+    for (int y = 0; y < a.topk; ++y)
+      if (tki[y] >= 0 && tki[y] < a.T) m_fin = fmaxf(m_fin, tkz[y] * sl2);
+    const float alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_fin);
+    float l_fin = l_sum * alpha;
+    for (int j = 0; j < n_sink; ++j) l_fin += ex2_approx(sz[j] * sl2 - m_fin);
+    for (int y = 0; y < a.topk; ++y)
+      if (tki[y] >= 0 && tki[y] < a.T) l_fin += ex2_approx(tkz[y] * sl2 - m_fin);
+    const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;
+    const __nv_bfloat16* vbase = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
+    __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)ir * a.o_st;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float ov[32];
+      if (k > 0) {
+        tmem_ld32(tO + lane_off + c * 32, ov);
+        tc_wait_ld();
+#pragma unroll
+        for (int y = 0; y < 32; ++y) ov[y] *= alpha;
+      } else {
+#pragma unroll
+        for (int y = 0; y < 32; ++y) ov[y] = 0.f;
+      }
+      for (int j = 0; j < n_sink; ++j) {
+        const float pkv = ex2_approx(sz[j] * sl2 - m_fin);
+        const __nv_bfloat16* vr = vbase + (size_t)j * a.v_st + c * 32;
+#pragma unroll
+        for (int y = 0; y < 32; y += 2) {
+          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr + y));
+          ov[y] = fmaf(pkv, vv.x, ov[y]);
+          ov[y + 1] = fmaf(pkv, vv.y, ov[y + 1]);
+        }
+      }
+      for (int t2 = 0; t2 < a.topk; ++t2) {
+        const int j = tki[t2];
+        if (j < 0 || j >= a.T) continue;
+        const float pkv = ex2_approx(tkz[t2] * sl2 - m_fin);
+        const __nv_bfloat16* vr = vbase + (size_t)j * a.v_st + c * 32;
+#pragma unroll
+        for (int y = 0; y < 32; y += 2) {
+          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr + y));
+          ov[y] = fmaf(pkv, vv.x, ov[y]);
+          ov[y + 1] = fmaf(pkv, vv.y, ov[y + 1]);
+        }
+      }
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 val;
+          val.x = pack_bf16x2(ov[q4 * 8 + 0] * inv_l, ov[q4 * 8 + 1] * inv_l);
+          val.y = pack_bf16x2(ov[q4 * 8 + 2] * inv_l, ov[q4 * 8 + 3] * inv_l);
+          val.z = pack_bf16x2(ov[q4 * 8 + 4] * inv_l, ov[q4 * 8 + 5] * inv_l);
+          val.w = pack_bf16x2(ov[q4 * 8 + 6] * inv_l, ov[q4 * 8 + 7] * inv_l);
+          dst[q4] = val;
+        }
+      }
+    }
+    if (row_ok) a.lse[row_id] = (l_fin > 0.f) ? (m_fin + __log2f(l_fin)) * 0.69314718055994531f : -CUDART_INF_F;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
+  const size_t tile = (size_t)D * kTile * 2;
+  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (2 + kKS + kVS) + 256);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  const int nQB = (a.nQT + 1) / 2;
+  const unsigned grid = (unsigned)a.B * a.Hq * nQB;
+  attn_tc2_kernel<D><<<grid, kThreads, bytes, st>>>(m.q, m.k, m.v, m.kg, m.vg, a, nQB);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Two-tile kernel; the caller routes capped separator tiles (q2) and
+// segment lengths that are not multiples of 256 to launch_attn_tc.
+cudaError_t launch_attn_tc2(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
+  if (a.B * a.Hq * a.nQT == 0) return cudaSuccess;
+  if (a.q2) return cudaErrorInvalidValue;
+  if (a.d == 128) return launch_d<128>(a, m, st);
+  if (a.d == 64) return launch_d<64>(a, m, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sattn

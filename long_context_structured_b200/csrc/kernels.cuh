@@ -101,7 +101,11 @@ struct AttnArgs {
 struct AttnMaps {
   CUtensorMap q, q2, k, v, kg, vg;
 };
+// one 128-row query tile per CTA (every case, incl. capped separator tiles)
 cudaError_t launch_attn_tc(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
+// two query tiles per CTA; not for q2 (capped separator tiles) and, in
+// segmented mode, only when the segment length is a multiple of 256
+cudaError_t launch_attn_tc2(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
 // K6: fp32 attention on CUDA cores
