@@ -33,11 +33,22 @@ namespace sattn {
 
 namespace {
 
-constexpr int kThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
+constexpr int kThreads = 384;  // 2 softmax warpgroups + 1 warpgroup holding the producer and MMA warps
+// register split (per thread): the producer/MMA warpgroup gives registers to
+// the softmax warpgroups; 2*128*kRegSoftmax + 128*kRegCtrl <= 384*168
+constexpr int kRegSoftmax = 216;
+constexpr int kRegCtrl = 72;
+static_assert(2 * 128 * kRegSoftmax + 128 * kRegCtrl <= kThreads * 168, "register split exceeds the launch budget");
 constexpr int kKS = 3;         // K stages
 constexpr int kVS = 2;         // V stages
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+// tcgen05.mma operations issued by one thread execute in issue order, so the
+// S_x product issued after PV_x cannot overwrite P_x before PV_x has read
+// it.  Setting this to 1 adds an explicit wait for PV_x before issuing S_x.
+#ifndef SATTN_WAR_WAIT
+#define SATTN_WAR_WAIT 0
+#endif
 
 __device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
   uint32_t a = smem_u32(bar);
@@ -70,6 +81,15 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
@@ -215,8 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = abort_i;
-
-  if (warp == 8) {
+  if (warp >= 8) {
+    regs_dec<kRegCtrl>();
+    if (warp == 8) {
     // ===================== TMA producer =====================
     if (lane == 0 && un.n > 0) {
       const int i0 = 2 * qb * kTile;
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
+    } else if (warp == 9) {
     // ===================== MMA issuer =====================
     if (lane == 0 && un.n > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
@@ -295,11 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool had_pv = prev[x] >= 0;
           if (had_pv) ok = issue_pv(x);
           if (!ok || !need[x]) continue;
+#if SATTN_WAR_WAIT
           if (had_pv) {
             // P_x (read by that PV) lives in the columns S_x is about to overwrite
             ok = mbar_wait(o_done + x, (n_pv[x] - 1) & 1, abort_flag, a.status, 38 + x);
             if (!ok) break;
           }
+#endif
           if (!k_ready) {
             ok = mbar_wait(k_full + ks, (p / kKS) & 1, abort_flag, a.status, 40);
             if (!ok) break;
@@ -335,7 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_raw(drain, 0);
     }
     __syncwarp();
+    }
   } else {
+    regs_inc<kRegSoftmax>();
     // ===================== softmax + epilogue (warpgroups 0 and 1) =====================
     const int x = warp >> 2;  // query tile of this warpgroup
     const Plan& pl = x == 0 ? pl0 : pl1;
@@ -381,28 +406,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const bool partial = (c_lo > 0 || c_hi < kTile - 1);
-      // pass 1: row max over the two 64-column halves of S (8 partial maxima)
-      float pm[8];
+      float sv[128];
 #pragma unroll
-      for (int y = 0; y < 8; ++y) pm[y] = -CUDART_INF_F;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        float sv[64];
-        tmem_ld32(tS + lane_off + hf * 64, sv);
-        tmem_ld32(tS + lane_off + hf * 64 + 32, sv + 32);
-        tc_wait_ld();
-        if (partial) {
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + c * 32, sv + c * 32);
+      tc_wait_ld();
+      if (partial) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int cc = hf * 64 + c;
-            if (cc < c_lo || cc > c_hi) sv[c] = -CUDART_INF_F;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
+        for (int c = 0; c < kTile; ++c)
+          if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
-      const float mx =
-          fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      float mx;
+      {
+        float pm[8];
+#pragma unroll
+        for (int y = 0; y < 8; ++y) pm[y] = sv[y];
+#pragma unroll
+        for (int c = 8; c < kTile; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
+        mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      }
       const float m_new = fmaxf(m_used, mx * sl2);
       float alpha = 1.f;
       bool rescale_o = false;
@@ -415,9 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_x is stable here: S_x(p) completing implies the tile's previous PV completed
       if (__any_sync(0xffffffffu, rescale_o)) {
         const float f = rescale_o ? alpha : 1.f;
-        float ov[32];
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
           tmem_ld32(tO + lane_off + c * 32, ov);
           tc_wait_ld();
 #pragma unroll
@@ -425,34 +446,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + lane_off + c * 32, ov);
         }
       }
-      // pass 2: P = 2^(s*log2e/sqrt(d) - m) per half, packed to bf16 and stored
-      // into TMEM over the S columns already consumed (P half h -> columns
-      // [32h, 32h+32), i.e. over S columns this half has read)
+      // P = 2^(s*log2e/sqrt(d) - m) packed to bf16; half h (S columns 64h..64h+63)
+      // goes to TMEM columns 32h..32h+31 over S values already in registers.
+      // A row with no key so far has m_used = -inf and every entry masked:
+      // with a zero offset each exp2(-inf) is exactly 0.
       {
         float ps[8];
 #pragma unroll
         for (int y = 0; y < 8; ++y) ps[y] = 0.f;
-        // a row with no key so far has m_used = -inf and every entry masked:
-        // with a zero offset each exp2(-inf) is exactly 0
         const float neg_m = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          float sv[64];
-          tmem_ld32(tS + lane_off + hf * 64, sv);
-          tmem_ld32(tS + lane_off + hf * 64 + 32, sv + 32);
-          tc_wait_ld();
-          if (partial) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const int cc = hf * 64 + c;
-              if (cc < c_lo || cc > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0
-            }
-          }
+        for (int hf = 0; hf < 2; ++hf) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2_approx(fmaf(sv[c], sl2, neg_m));
-            const float p1 = ex2_approx(fmaf(sv[c + 1], sl2, neg_m));
+            const float p0 = ex2_approx(fmaf(sv[hf * 64 + c], sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(sv[hf * 64 + c + 1], sl2, neg_m));
             ps[(c >> 1) & 7] += p0 + p1;
             pk[c >> 1] = pack_bf16x2(p0, p1);
           }

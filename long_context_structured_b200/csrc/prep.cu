@@ -11,10 +11,12 @@
 // logits do not inherit bf16 operand rounding; and per (batch, kv head) the
 // largest key norm, used by the top-k selector to bound bf16 scoring error.
 //
-// Layout of the work: one block = 32 consecutive rows of one head (8 warps,
-// 4 rows each); lane l owns the pairs c = l*PP .. l*PP+PP-1 (PP = d/64), so a
-// row's loads and stores are 128-byte coalesced per half.  Sink keys are
-// staged once per block in shared memory (raw and rotated, fp32).
+// Work layout (HBM-bound): a thread owns 8 consecutive rotary pairs of one
+// row -- one 16-byte load from each half of the row, four 16-byte table
+// loads, two 16-byte stores -- so d/16 threads cover a row (8 for d = 128)
+// and a 256-thread block covers 256/(d/16) rows per step.  A block walks
+// kRowsPerBlock rows of one head; the sink keys of that head are staged
+// once per block in shared memory (raw and rotated, fp32).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -24,9 +26,10 @@ namespace sattn {
 
 namespace {
 
-constexpr int kRowsPerBlock = 32;
 constexpr int kPrepThreads = 256;
+constexpr int kRowsPerBlock = 256;
 constexpr int kMaxSmemSinks = 16;
+constexpr int kPairsPerThread = 8;
 
 __global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double theta) {
   __shared__ double inv_freq[128];
@@ -42,117 +45,107 @@ __global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double
   }
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// PP consecutive bf16 of a row starting at element c -> floats
-template <int PP>
-__device__ __forceinline__ void load_pp(const __nv_bfloat16* p, float* out) {
-  if constexpr (PP == 2) {
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-    out[0] = v.x;
-    out[1] = v.y;
-  } else {
-    out[0] = __bfloat162float(*p);
+  for (int e = 0; e < 4; ++e) {
+    const float2 v = __bfloat1622float2(h[e]);
+    f[2 * e] = v.x;
+    f[2 * e + 1] = v.y;
   }
 }
 
-template <int PP>
-__device__ __forceinline__ void store_pp(__nv_bfloat16* p, const float* v) {
-  if constexpr (PP == 2) {
-    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
-  } else {
-    *p = __float2bfloat16_rn(v[0]);
-  }
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+  return u;
 }
 
-template <int PP>
-__device__ __forceinline__ void load_tab(const float2* tab, int64_t pos, int half, int c, float* cs, float* sn) {
+// cos/sin of 8 consecutive pairs c0..c0+7 at position pos (identity without a table)
+__device__ __forceinline__ void load_tab8(const float2* tab, int64_t pos, int half, int c0, float* cs, float* sn) {
   if (!tab) {
 #pragma unroll
-    for (int e = 0; e < PP; ++e) {
+    for (int e = 0; e < 8; ++e) {
       cs[e] = 1.f;
       sn[e] = 0.f;
     }
     return;
   }
-  const float2* t = tab + pos * half + c;
-  if constexpr (PP == 2) {
-    const float4 v = *reinterpret_cast<const float4*>(t);
-    cs[0] = v.x;
-    sn[0] = v.y;
-    cs[1] = v.z;
-    sn[1] = v.w;
-  } else {
-    const float2 v = *t;
-    cs[0] = v.x;
-    sn[0] = v.y;
+  const float4* t = reinterpret_cast<const float4*>(tab + pos * half + c0);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float4 v = t[e];
+    cs[2 * e] = v.x;
+    sn[2 * e] = v.y;
+    cs[2 * e + 1] = v.z;
+    sn[2 * e + 1] = v.w;
   }
 }
 
-// grid (ceil(T/32), H, B) for the query part (blockIdx.z < B) followed by
-// the key part (blockIdx.z >= B, head = blockIdx.y < Hkv)
-template <int PP>
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a) {
+// grid (ceil(T / kRowsPerBlock), H, 2B): blockIdx.z < B -> query rows of head
+// blockIdx.y; blockIdx.z >= B -> key rows of kv head blockIdx.y (< Hkv)
+__global__ void __launch_bounds__(kPrepThreads, 4) prep_kernel(PrepArgs a) {
   __shared__ float s_sink_raw[kMaxSmemSinks][128];
   __shared__ float s_sink_rot[kMaxSmemSinks][128];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ float s_lc[64], s_ls[64];  // cos/sin of the rotation to the cap L
   const int half = a.d / 2;
-  const int c0 = lane * PP;
+  const int tpr = half / kPairsPerThread;  // threads per row: 8 (d=128) or 4 (d=64)
+  const int rows_per_step = kPrepThreads / tpr;
+  const int sub = threadIdx.x % tpr;       // which 8-pair chunk of the row
+  const int c0 = sub * kPairsPerThread;
   const bool key_part = blockIdx.z >= (unsigned)a.B;
   const int b = key_part ? blockIdx.z - a.B : blockIdx.z;
   const int h = blockIdx.y;
   const int row0 = blockIdx.x * kRowsPerBlock;
   const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.Q);
   const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(a.K);
+  // lanes of this thread's row group (8 or 4 consecutive lanes)
+  const unsigned grp_mask = (tpr == 8) ? (0xffu << (threadIdx.x & 24)) : (0xfu << (threadIdx.x & 28));
 
   if (key_part) {
     if (h >= a.Hkv) return;
-    constexpr int kRowsPerWarp = kRowsPerBlock / (kPrepThreads / 32);
-    float k0[kRowsPerWarp][PP], k1[kRowsPerWarp][PP], cs[kRowsPerWarp][PP], sn[kRowsPerWarp][PP];
-#pragma unroll
-    for (int x = 0; x < kRowsPerWarp; ++x) {
-      const int j = min(row0 + warp + x * (kPrepThreads / 32), a.T - 1);
-      const __nv_bfloat16* kp = K + b * a.k_sb + h * a.k_sh + (int64_t)j * a.k_st;
-      load_pp<PP>(kp + c0, k0[x]);
-      load_pp<PP>(kp + c0 + half, k1[x]);
-      load_tab<PP>(a.tab, j, half, c0, cs[x], sn[x]);
-    }
-#pragma unroll
-    for (int x = 0; x < kRowsPerWarp; ++x) {
-      const int j = row0 + warp + x * (kPrepThreads / 32);
+    for (int rr = threadIdx.x / tpr; rr < kRowsPerBlock; rr += rows_per_step) {
+      const int j = row0 + rr;
       if (j >= a.T) break;
+      const __nv_bfloat16* kp = K + b * a.k_sb + h * a.k_sh + (int64_t)j * a.k_st;
+      float k0[8], k1[8], cs[8], sn[8];
+      unpack8(*reinterpret_cast<const uint4*>(kp + c0), k0);
+      unpack8(*reinterpret_cast<const uint4*>(kp + c0 + half), k1);
       float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < PP; ++e) ss = fmaf(k0[x][e], k0[x][e], fmaf(k1[x][e], k1[x][e], ss));
+      for (int e = 0; e < 8; ++e) ss = fmaf(k0[e], k0[e], fmaf(k1[e], k1[e], ss));
       if (a.Kr) {
-        float r0[PP], r1[PP];
+        load_tab8(a.tab, j, half, c0, cs, sn);
+        float r0[8], r1[8];
 #pragma unroll
-        for (int e = 0; e < PP; ++e) {
-          r0[e] = k0[x][e] * cs[x][e] - k1[x][e] * sn[x][e];
-          r1[e] = k1[x][e] * cs[x][e] + k0[x][e] * sn[x][e];
+        for (int e = 0; e < 8; ++e) {
+          r0[e] = k0[e] * cs[e] - k1[e] * sn[e];
+          r1[e] = k1[e] * cs[e] + k0[e] * sn[e];
         }
         __nv_bfloat16* kr = a.Kr + (((int64_t)b * a.Hkv + h) * a.T + j) * a.d;
-        store_pp<PP>(kr + c0, r0);
-        store_pp<PP>(kr + c0 + half, r1);
+        *reinterpret_cast<uint4*>(kr + c0) = pack8(r0);
+        *reinterpret_cast<uint4*>(kr + c0 + half) = pack8(r1);
       }
       if (a.kmax) {
-        ss = warp_sum(ss);
-        if (lane == 0) atomicMax(a.kmax + (size_t)b * a.Hkv + h, __float_as_uint(sqrtf(ss)));
+        for (int o = tpr / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(grp_mask, ss, o);
+        if (sub == 0) atomicMax(a.kmax + (size_t)b * a.Hkv + h, __float_as_uint(sqrtf(ss)));
       }
     }
     return;
   }
 
-  // ---- query part ----
+  // ---- query rows ----
   const int g = h / (a.Hq / a.Hkv);
   const int n_sink = a.sink_z ? a.n_sink : 0;
   const bool sinks_in_smem = n_sink > 0 && n_sink <= kMaxSmemSinks;
+  for (int c = threadIdx.x; c < half; c += kPrepThreads) {
+    const float2 t = (a.L > 0 && a.tab) ? a.tab[(int64_t)a.L * half + c] : make_float2(1.f, 0.f);
+    s_lc[c] = t.x;
+    s_ls[c] = t.y;
+  }
   if (sinks_in_smem) {
-    // raw and rotated sink keys of this (b, kv head), fp32
     for (int x = threadIdx.x; x < n_sink * half; x += kPrepThreads) {
       const int j = x / half, c = x % half;
       const __nv_bfloat16* kp = K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
@@ -163,81 +156,67 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a) {
       s_sink_rot[j][c] = k0 * t.x - k1 * t.y;
       s_sink_rot[j][c + half] = k1 * t.x + k0 * t.y;
     }
-    __syncthreads();
   }
-  const bool need_qc = a.Qc != nullptr || n_sink > 0;
-  float lc[PP], ls[PP];
-  if (need_qc) load_tab<PP>(a.L > 0 ? a.tab : nullptr, a.L, half, c0, lc, ls);
-  constexpr int kRowsPerWarp = kRowsPerBlock / (kPrepThreads / 32);
-  float xa[kRowsPerWarp][PP], xb[kRowsPerWarp][PP], ca[kRowsPerWarp][PP], sa[kRowsPerWarp][PP];
-#pragma unroll
-  for (int x = 0; x < kRowsPerWarp; ++x) {
-    const int i = min(row0 + warp + x * (kPrepThreads / 32), a.T - 1);
-    const __nv_bfloat16* qp = Q + b * a.q_sb + h * a.q_sh + (int64_t)i * a.q_st;
-    load_pp<PP>(qp + c0, xa[x]);
-    load_pp<PP>(qp + c0 + half, xb[x]);
-    load_tab<PP>(a.tab, i, half, c0, ca[x], sa[x]);
-  }
-#pragma unroll
-  for (int x = 0; x < kRowsPerWarp; ++x) {
-    const int i = row0 + warp + x * (kPrepThreads / 32);
+  __syncthreads();
+  for (int rr = threadIdx.x / tpr; rr < kRowsPerBlock; rr += rows_per_step) {
+    const int i = row0 + rr;
     if (i >= a.T) break;
-    float r0[PP], r1[PP], q0[PP], q1[PP];
+    const __nv_bfloat16* qp = Q + b * a.q_sb + h * a.q_sh + (int64_t)i * a.q_st;
+    float x0[8], x1[8], cs[8], sn[8], r0[8], r1[8], q0[8], q1[8];
+    unpack8(*reinterpret_cast<const uint4*>(qp + c0), x0);
+    unpack8(*reinterpret_cast<const uint4*>(qp + c0 + half), x1);
+    load_tab8(a.tab, i, half, c0, cs, sn);
 #pragma unroll
-    for (int e = 0; e < PP; ++e) {
-      r0[e] = xa[x][e] * ca[x][e] - xb[x][e] * sa[x][e];
-      r1[e] = xb[x][e] * ca[x][e] + xa[x][e] * sa[x][e];
-      q0[e] = xa[x][e] * lc[e] - xb[x][e] * ls[e];
-      q1[e] = xb[x][e] * lc[e] + xa[x][e] * ls[e];
+    for (int e = 0; e < 8; ++e) {
+      r0[e] = x0[e] * cs[e] - x1[e] * sn[e];
+      r1[e] = x1[e] * cs[e] + x0[e] * sn[e];
+      q0[e] = x0[e] * s_lc[c0 + e] - x1[e] * s_ls[c0 + e];
+      q1[e] = x1[e] * s_lc[c0 + e] + x0[e] * s_ls[c0 + e];
     }
     const int64_t orow = (((int64_t)b * a.Hq + h) * a.T + i) * a.d;
     if (a.Qr) {
-      store_pp<PP>(a.Qr + orow + c0, r0);
-      store_pp<PP>(a.Qr + orow + c0 + half, r1);
+      *reinterpret_cast<uint4*>(a.Qr + orow + c0) = pack8(r0);
+      *reinterpret_cast<uint4*>(a.Qr + orow + c0 + half) = pack8(r1);
     }
     if (a.Qc) {
-      store_pp<PP>(a.Qc + orow + c0, q0);
-      store_pp<PP>(a.Qc + orow + c0 + half, q1);
+      *reinterpret_cast<uint4*>(a.Qc + orow + c0) = pack8(q0);
+      *reinterpret_cast<uint4*>(a.Qc + orow + c0 + half) = pack8(q1);
     }
     if (n_sink > 0) {
       const int64_t zrow = (((int64_t)b * a.Hq + h) * a.T + i) * n_sink;
-      for (int j0 = 0; j0 < n_sink; j0 += 32) {
-        float mine = -CUDART_INF_F;
-        const int jn = min(32, n_sink - j0);
-        for (int jj = 0; jj < jn; ++jj) {
-          const int j = j0 + jj;
-          float z = -CUDART_INF_F;
-          if (j <= i) {
-            const bool capped = a.L > 0 && (i - j) > a.L;
-            float acc = 0.f;
-            if (sinks_in_smem) {
-              const float* kv = capped ? s_sink_raw[j] : s_sink_rot[j];
+      for (int j = 0; j < n_sink; ++j) {
+        // every thread of a row group takes the same branch (same i and j)
+        float z = -CUDART_INF_F;
+        if (j <= i) {
+          const bool capped = a.L > 0 && (i - j) > a.L;
+          float acc = 0.f;
+          if (sinks_in_smem) {
+            const float* kv = capped ? s_sink_raw[j] : s_sink_rot[j];
 #pragma unroll
-              for (int e = 0; e < PP; ++e) {
-                acc = fmaf(capped ? q0[e] : r0[e], kv[c0 + e], acc);
-                acc = fmaf(capped ? q1[e] : r1[e], kv[c0 + e + half], acc);
-              }
-            } else {
-              const __nv_bfloat16* kp = K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
-              float k0[PP], k1[PP], kc[PP], ks[PP];
-              load_pp<PP>(kp + c0, k0);
-              load_pp<PP>(kp + c0 + half, k1);
-              load_tab<PP>(a.tab, j, half, c0, kc, ks);
+            for (int e = 0; e < 8; ++e) {
+              acc = fmaf(capped ? q0[e] : r0[e], kv[c0 + e], acc);
+              acc = fmaf(capped ? q1[e] : r1[e], kv[c0 + e + half], acc);
+            }
+          } else {
+            const __nv_bfloat16* kp = K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
+            float k0[8], k1[8], kc[8], ks[8];
+            unpack8(*reinterpret_cast<const uint4*>(kp + c0), k0);
+            unpack8(*reinterpret_cast<const uint4*>(kp + c0 + half), k1);
+            load_tab8(a.tab, j, half, c0, kc, ks);
 #pragma unroll
-              for (int e = 0; e < PP; ++e) {
-                if (capped) {
-                  acc = fmaf(q0[e], k0[e], fmaf(q1[e], k1[e], acc));
-                } else {
-                  acc = fmaf(r0[e], k0[e] * kc[e] - k1[e] * ks[e], acc);
-                  acc = fmaf(r1[e], k1[e] * kc[e] + k0[e] * ks[e], acc);
-                }
+            for (int e = 0; e < 8; ++e) {
+              if (capped) {
+                acc = fmaf(q0[e], k0[e], fmaf(q1[e], k1[e], acc));
+              } else {
+                acc = fmaf(r0[e], k0[e] * kc[e] - k1[e] * ks[e], acc);
+                acc = fmaf(r1[e], k1[e] * kc[e] + k0[e] * ks[e], acc);
               }
             }
-            z = warp_sum(acc);
           }
-          if (lane == jj) mine = z;
+          for (int o = tpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(grp_mask, acc, o);
+          z = acc;
         }
-        if (lane < jn) a.sink_z[zrow + j0 + lane] = mine;
+        if (sub == (j % tpr)) a.sink_z[zrow + j] = z;
       }
     }
   }
@@ -257,14 +236,10 @@ cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, cudaSt
 
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st) {
   if (a.f32) return cudaErrorInvalidValue;  // the fp32 path rotates inside its own kernel
+  if (a.d != 64 && a.d != 128) return cudaErrorInvalidValue;
   if (a.B == 0 || a.T == 0) return cudaSuccess;
   dim3 grid((a.T + kRowsPerBlock - 1) / kRowsPerBlock, std::max(a.Hq, a.Hkv), 2 * a.B);
-  if (a.d == 128)
-    prep_kernel<2><<<grid, kPrepThreads, 0, st>>>(a);
-  else if (a.d == 64)
-    prep_kernel<1><<<grid, kPrepThreads, 0, st>>>(a);
-  else
-    return cudaErrorInvalidValue;
+  prep_kernel<<<grid, kPrepThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
