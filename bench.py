@@ -1,13 +1,17 @@
 """Benchmark of the structured-mask attention hot path on B200.
 
-One step = one ``sattn_fwd`` call (rotary prep pass, block/band planning and
-the tcgen05 attention kernel) over the Llama-2-7B-shaped LM-Infinite layer:
-B=1, 32 heads, T=16384, d=128, bf16, n_start=4, L_pretrain=w=4096, capped
-RoPE theta=1e4, sink keys scaled x8.  Metric: effective TFLOP/s counted over
-unmasked (q, k) pairs at 4*d FLOPs each (whole job, all ranks), with tokens/s
-alongside.
+One step = one call of the whole hot path over one batch of synthetic input
+(rotary prep, block map / separator gather / top-k selection where the
+workload has them, and the tcgen05 attention kernel).  The default workload is
+the Llama-2-7B-shaped LM-Infinite layer: B=1, 32 heads, T=16384, d=128, bf16,
+n_start=4, L_pretrain=w=4096, capped RoPE theta=1e4, sink keys scaled x8.
+``--workload`` selects one of the other workloads (SepLLM GQA layer, top-k
+middle tokens, segmented execution) to measure their kernels the same way.
+Metric: effective TFLOP/s counted over unmasked (q, k) pairs at 4*d FLOPs
+each (whole job, all ranks), with tokens/s alongside.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c2|c3|c4|c5]
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own
 independent problem (heads/batches are independent), so per-GPU work is
@@ -36,24 +40,66 @@ sys.path.insert(0, ROOT)
 
 from long_context_structured_b200 import synth  # noqa: E402
 
-WORKLOAD = "c2_lminf_16k"
+WORKLOAD_ALIASES = {"c2": "c2_lminf_16k", "c3": "c3_sepllm_gqa_8k", "c4": "c4_lminf_topk_32k",
+                    "c5": "c5_segmented_32k"}
+DEFAULT_WORKLOAD = "c2"
 METRIC = "effective TFLOP/s over unmasked pairs (fraction of bf16 TC peak), tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per launch of the attention kernel on this
-# workload, from the ncu capture summarised in profiles/; None when the
-# kernel changed since the counters were taken.
-ATTN_TRAFFIC_BYTES = None  # the kernel changed since the last DRAM capture
+# DRAM bytes (read + write) per launch of the attention kernel on the default
+# workload, from the ncu capture summarised in profiles/; None when the kernel
+# changed since the counters were taken.
+ATTN_TRAFFIC_BYTES = None
 
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
-def unmasked_pairs_per_head(wl) -> int:
-    """Closed-form count of kept (q, k) pairs of one head for a workload with
-    no separators and no top-k: row i keeps min(i+1, n_start+w+1) keys."""
+# ---------------------------------------------------------------------------
+# algorithmic work per workload (closed-form counts of kept (q, k) pairs)
+# ---------------------------------------------------------------------------
+
+def lambda_pairs_per_row(wl) -> np.ndarray:
+    """Kept keys of each row from the starting span and the window: row i
+    keeps min(i+1, n_start+w+1) keys."""
     i = np.arange(wl.T, dtype=np.int64)
-    return int(np.minimum(i + 1, wl.n_start + wl.window + 1).sum())
+    return np.minimum(i + 1, wl.n_start + wl.window + 1)
+
+
+def middle_candidates_per_row(wl) -> np.ndarray:
+    """Middle keys n_start <= j < i - w of each row (no separators)."""
+    i = np.arange(wl.T, dtype=np.int64)
+    return np.maximum(0, i - wl.window - wl.n_start)
+
+
+def unmasked_pairs(wl, is_sep=None) -> int:
+    """Kept (q, k) pairs summed over batch and heads for one workload."""
+    if wl.segmented:
+        S, N = wl.seg_S, wl.T // wl.seg_S
+        t = np.arange(S, dtype=np.int64) + 1
+        per_local = N * int(t.sum()) + (N - 1) * S * wl.seg_M
+        per_long = N * int(t.sum()) + (N - 1) * S * wl.seg_R
+        n_long = len(wl.long_heads)
+        return wl.B * ((wl.Hq - n_long) * per_local + n_long * per_long)
+    base = lambda_pairs_per_row(wl)
+    per_head = np.full(wl.B, int(base.sum()), dtype=np.int64)
+    if is_sep is not None:
+        i = np.arange(wl.T, dtype=np.int64)
+        for b in range(wl.B):
+            f = is_sep[b].astype(np.int64).copy()
+            f[: wl.n_start] = 0
+            pre = np.concatenate([[0], np.cumsum(f)])  # pre[x] = separators n_start <= j < x
+            per_head[b] += int(pre[np.clip(i - wl.window, 0, wl.T)].sum())
+    if wl.topk > 0:
+        per_head += int(np.minimum(wl.topk, middle_candidates_per_row(wl)).sum())
+    return int(per_head.sum()) * wl.Hq
+
+
+def scored_candidates(wl) -> int:
+    """Middle (q, k) pairs the top-k selector scores (2*d FLOPs each)."""
+    if wl.topk <= 0:
+        return 0
+    return int(middle_candidates_per_row(wl).sum()) * wl.B * wl.Hq
 
 
 def load_peaks():
@@ -65,16 +111,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def describe(wl) -> str:
+    if wl.segmented:
+        return ("%s: segmented execution, one layer, B=%d H=%d (%d long) T=%d d=%d bf16, S=%d, tail M=%d, "
+                "prefix R=%d (top-%d blocks of %d), RoPE theta=%g" % (
+                    wl.name, wl.B, wl.Hq, len(wl.long_heads), wl.T, wl.d, wl.seg_S, wl.seg_M, wl.seg_R,
+                    wl.seg_R // wl.retr_block, wl.retr_block, wl.rope_theta))
+    if wl.sep_rate > 0:
+        return ("%s: SepLLM layer, B=%d Hq=%d Hkv=%d T=%d d=%d bf16, separator ids %d of %d at rate %.2f, "
+                "n_start=%d, w=%d, RoPE theta=%g" % (wl.name, wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.sep_ids,
+                                                     wl.sep_vocab, wl.sep_rate, wl.n_start, wl.window,
+                                                     wl.rope_theta))
+    s = ("%s: LM-Infinite Lambda-mask layer, B=%d H=%d T=%d d=%d bf16, n_start=%d, L_pretrain=w=%d, "
+         "capped RoPE theta=%g" % (wl.name, wl.B, wl.Hq, wl.T, wl.d, wl.n_start, wl.window, wl.rope_theta))
+    if wl.sink_scale != 1.0:
+        s += ", keys 0-3 x%g" % wl.sink_scale
+    if wl.topk > 0:
+        s += ", top-%d middle keys per head (%d planted clusters)" % (wl.topk, wl.plant)
+    return s
+
+
 def config_dict(wl, pairs_per_rank):
-    return {
-        "workload": "%s: LM-Infinite Lambda-mask layer, B=%d H=%d T=%d d=%d bf16, n_start=%d, L_pretrain=w=%d, "
-                    "capped RoPE theta=%g, keys 0-3 x8" % (wl.name, wl.B, wl.Hq, wl.T, wl.d, wl.n_start, wl.window,
-                                                          wl.rope_theta),
-        "B": wl.B, "H": wl.Hq, "T": wl.T, "d": wl.d, "n_start": wl.n_start, "window": wl.window,
-        "L_pretrain": wl.L_pretrain, "rope_theta": wl.rope_theta,
-        "unmasked_pairs_per_rank": pairs_per_rank,
-        "l2": "no flush: each step reads Q,K,V (384 MB) and its 256 MB rotated copies, > 126 MB L2",
-    }
+    c = {"workload": describe(wl), "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d}
+    if wl.segmented:
+        c.update({"S": wl.seg_S, "M": wl.seg_M, "R": wl.seg_R, "retr_block": wl.retr_block,
+                  "long_heads": len(wl.long_heads), "rope_theta": wl.rope_theta})
+    else:
+        c.update({"n_start": wl.n_start, "window": wl.window, "L_pretrain": wl.L_pretrain,
+                  "rope_theta": wl.rope_theta, "topk": wl.topk})
+    c["unmasked_pairs_per_rank"] = pairs_per_rank
+    in_bytes = (wl.B * wl.Hq + 2 * wl.B * wl.Hkv) * wl.T * wl.d * 2
+    c["l2"] = ("no flush: each step reads Q,K,V (%d MB) and writes their rotated copies, > 126 MB L2"
+               % (in_bytes >> 20))
+    return c
 
 
 # ---------------------------------------------------------------------------
@@ -144,6 +213,100 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# one workload: inputs, the step, the end-to-end call, algorithmic work
+# ---------------------------------------------------------------------------
+
+class Job:
+    """Inputs of one workload on one rank (pinned host copies and device
+    copies) and the hot-path call over them."""
+
+    def __init__(self, wl, seed, dev):
+        import torch
+
+        import long_context_structured_b200 as sa
+        self.sa, self.torch, self.wl, self.dev = sa, torch, wl, dev
+        inp = synth.make_inputs(wl, seed=seed)
+        self.inp = inp
+        to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        self.host = {x: to_t(inp[x]).pin_memory() for x in ("q", "k", "v")}
+        if inp["is_sep"] is not None:
+            self.host["is_sep"] = torch.from_numpy(inp["is_sep"]).pin_memory()
+        self.devt = {x: t.to(dev) for x, t in self.host.items()}
+        q = self.devt["q"]
+        self.O = torch.empty_like(q)
+        self.lse = torch.empty((wl.B, wl.Hq, wl.T), dtype=torch.float32, device=dev)
+        if wl.segmented:
+            self.kw = dict(S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
+                           is_long=[int(x) for x in inp["is_long"]], rope_theta=wl.rope_theta)
+        else:
+            self.kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                           rope_theta=wl.rope_theta, topk=wl.topk)
+        self.pairs = unmasked_pairs(wl, inp["is_sep"])
+        self.flops = 4.0 * wl.d * self.pairs
+        self.n_sep = 0 if inp["is_sep"] is None else int(inp["is_sep"][:, wl.n_start:].sum())
+
+    def step(self):
+        d = self.devt
+        if self.wl.segmented:
+            self.sa.segment_fwd(d["q"], d["k"], d["v"], out=self.O, lse=self.lse, **self.kw)
+        else:
+            self.sa.fwd(d["q"], d["k"], d["v"], is_sep=d.get("is_sep"), out=self.O, lse=self.lse, **self.kw)
+
+    def host_step(self):
+        """The public call on pinned host tensors: H2D, the hot path, D2H."""
+        h = self.host
+        if self.wl.segmented:
+            return self.sa.segment_fwd(h["q"], h["k"], h["v"], **self.kw)
+        return self.sa.fwd(h["q"], h["k"], h["v"], is_sep=h.get("is_sep"), **self.kw)
+
+    def h2d_bytes(self):
+        return int(sum(t.nbytes for t in self.host.values()))
+
+    # algorithmic work of each launch group the library times ---------------
+    def group_work(self):
+        """{group: (bound, work per launch, unit)} for the groups whose
+        algorithmic work has a closed form: FLOPs for the tensor-core kernels,
+        bytes read + written of the named arrays for the HBM-bound ones."""
+        wl = self.wl
+        e = 2  # bf16 bytes
+        rows_q = wl.B * wl.Hq * wl.T * wl.d * e
+        rows_k = wl.B * wl.Hkv * wl.T * wl.d * e
+        out = {}
+        attn = "attn_tc_segment" if wl.segmented else "attn_tc"
+        out[attn] = ("tensor", self.flops, "FLOP")
+        prep = 2 * rows_q + 2 * rows_k  # Q, K read; Qr, Kr written
+        if not wl.segmented:
+            if wl.L_pretrain > 0 and (wl.topk > 0 or wl.sep_rate > 0):
+                prep += rows_q  # Qc written
+            prep += wl.B * wl.Hq * wl.T * min(wl.n_start, wl.T) * 4  # sink logits written
+        out["prep_rope"] = ("hbm", prep, "B")
+        if self.n_sep:
+            out["sep_gather"] = ("hbm", self.n_sep * wl.Hkv * 4 * wl.d * e, "B")
+        if wl.topk > 0:
+            out["topk_score_rerank"] = ("tensor", 2.0 * wl.d * scored_candidates(wl), "FLOP")
+        return out
+
+
+def roofline_of(group, work, avg_ms, peaks, peak_src):
+    bound, amount, unit = work
+    if bound == "tensor":
+        peak = float(peaks["bf16_tflops"])
+        ach = amount / (avg_ms * 1e-3) / 1e12
+        r = {"kernel": group, "bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+             "frac": round(ach / peak, 4), "peak_source": "%s bf16_tflops (burst)" % peak_src,
+             "frac_of_sustained": round(ach / float(peaks.get("bf16_tflops_sustained", peak)), 4),
+             "algorithmic_flops_per_launch": amount}
+    else:
+        peak = float(peaks["hbm_gbs"])
+        ach = amount / (avg_ms * 1e-3) / 1e9
+        r = {"kernel": group, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+             "frac": round(ach / peak, 4), "peak_source": "%s hbm_gbs" % peak_src,
+             "algorithmic_bytes_per_launch": amount}
+    r["avg_launch_ms"] = round(avg_ms, 4)
+    return r
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -159,6 +322,17 @@ def profile_collect(lib):
         nm = names.raw[32 * x: 32 * x + 32].split(b"\0")[0].decode()
         out[nm] = (int(launches[x]), float(total[x]))
     return out
+
+
+def kernel_name(wl, group):
+    """The kernel behind a launch group on this workload (for the JSON line)."""
+    if group == "attn_tc":
+        capped_sep = wl.L_pretrain > 0 and wl.sep_rate > 0
+        return "attn_tc3_kernel<%d>" % wl.d if capped_sep else "attn_tc2_kernel<%d>" % wl.d
+    if group == "attn_tc_segment":
+        return "attn_tc2_kernel<%d>" % wl.d if wl.seg_S % 256 == 0 else "attn_tc3_kernel<%d>" % wl.d
+    return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel",
+            "sep_gather": "sep_gather_kernel"}.get(group, group)
 
 
 def run_ours(args):
@@ -179,23 +353,15 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[WORKLOAD_ALIASES.get(args.workload, args.workload)]
     if args.heads:
-        wl = wl.scaled(Hq=args.heads, Hkv=args.heads)
-    pairs_head = unmasked_pairs_per_head(wl)
-    pairs = pairs_head * wl.B * wl.Hq
-    flops_step = 4.0 * wl.d * pairs  # per rank
-    inp = synth.make_inputs(wl, seed=rank)
-    to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-    qh, kh, vh = (to_t(inp[x]).pin_memory() for x in ("q", "k", "v"))
-    q, k, v = qh.to(dev), kh.to(dev), vh.to(dev)
-    kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta)
-    O = torch.empty_like(q)
-    lse = torch.empty((wl.B, wl.Hq, wl.T), dtype=torch.float32, device=dev)
+        wl = wl.scaled(Hq=args.heads, Hkv=max(1, args.heads * wl.Hkv // wl.Hq),
+                       long_heads=tuple(h for h in wl.long_heads if h < args.heads))
+    job = Job(wl, seed=rank, dev=dev)
     lib = _lib.load()
 
     for _ in range(args.warmup):
-        sa.fwd(q, k, v, out=O, lse=lse, **kw)
+        job.step()
     torch.cuda.synchronize()
     if sa.stream_status() != 0:
         raise RuntimeError("device status word reports a failure after warm-up")
@@ -215,7 +381,7 @@ def run_ours(args):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        sa.fwd(q, k, v, out=O, lse=lse, **kw)
+        job.step()
     e1.record()
     torch.cuda.synchronize()
     if world > 1:
@@ -230,72 +396,80 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = job.flops * world / (ms_step * 1e-3) / 1e12
     tokens_s = wl.B * wl.T * world / (ms_step * 1e-3)
 
-    attn_launches, attn_ms = prof.get("attn_tc", (0, 0.0))
-    attn_avg_ms = attn_ms / max(attn_launches, 1)
-    at = torch.tensor([attn_avg_ms], dtype=torch.float64, device=dev)
+    # per-group device time per step (every group runs once per step; a group
+    # may hold more than one kernel), max over ranks (same group order on
+    # every rank)
+    groups = sorted(prof)
+    avg = torch.tensor([prof[g][1] / args.steps for g in groups] or [0.0], dtype=torch.float64, device=dev)
     if world > 1:
-        dist.all_reduce(at, op=dist.ReduceOp.MAX)
-    attn_avg_ms = float(at.item())
+        dist.all_reduce(avg, op=dist.ReduceOp.MAX)
+    avg_ms = {g: float(avg[x].item()) for x, g in enumerate(groups)}
     peaks, peak_src = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    achieved = flops_step / (attn_avg_ms * 1e-3) / 1e12 if attn_avg_ms > 0 else None
+    work = job.group_work()
+    kernels = {}
+    for g in groups:
+        n, ms = prof[g]
+        kernels[g] = {"kernel": kernel_name(wl, g), "launches": n, "ms_per_step": round(avg_ms[g], 5),
+                      "share": round(ms / max(sum(v[1] for v in prof.values()), 1e-12), 4)}
+        if g in work and avg_ms[g] > 0:
+            r = roofline_of(g, work[g], avg_ms[g], peaks, peak_src)
+            kernels[g].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+    # the roofline line is the dominant kernel's (largest share of device time)
+    dom = max((g for g in groups if g in work), key=lambda g: prof[g][1], default=None)
+    roof = None
+    if dom is not None:
+        roof = roofline_of(dom, work[dom], avg_ms[dom], peaks, peak_src)
+        roof["kernel"] = kernel_name(wl, dom)
+        roof["traffic"] = ATTN_TRAFFIC_BYTES if (dom == "attn_tc" and args.workload == DEFAULT_WORKLOAD
+                                                 and not args.heads) else None
     gpu_launches = sum(n for n, _ in prof.values())
 
     # end to end through the public call with host buffers (H2D + D2H inside)
-    e2e = None
-    if rank == 0 or world > 1:
-        n_e2e = max(3, min(10, args.steps))
-        sa.fwd(qh, kh, vh, **kw)  # warm the host path
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record()
-        for _ in range(n_e2e):
-            Oh, lh = sa.fwd(qh, kh, vh, **kw)
-        s1.record()
-        torch.cuda.synchronize()
-        te = torch.tensor([s0.elapsed_time(s1) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        ms_e2e = float(te.item())
-        e2e = {"value": round(flops_step * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-               "ms_per_step": round(ms_e2e, 3), "steps": n_e2e,
-               "h2d_bytes_per_step": int(qh.nbytes + kh.nbytes + vh.nbytes),
-               "d2h_bytes_per_step": int(Oh.nbytes + lh.nbytes),
-               "path": "long_context_structured_b200.fwd on pinned host tensors"}
+    n_e2e = max(3, min(10, args.steps))
+    outs = job.host_step()  # warm the host path
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(n_e2e):
+        outs = job.host_step()
+    s1.record()
+    torch.cuda.synchronize()
+    te = torch.tensor([s0.elapsed_time(s1) / n_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    ms_e2e = float(te.item())
+    e2e = {"value": round(job.flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "ms_per_step": round(ms_e2e, 3), "steps": n_e2e, "h2d_bytes_per_step": job.h2d_bytes(),
+           "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
+           "path": "long_context_structured_b200.%s on pinned host tensors (outputs into pinned host memory)"
+                   % ("segment_fwd" if wl.segmented else "fwd")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, inp, args.cpu_rows)
+        cpu = cpu_baseline(wl, job.inp, args.cpu_rows)
 
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
+    peak = float(peaks["bf16_tflops"])
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); keys 0-3 x8)",
-        "config": config_dict(wl, pairs),
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
+        "config": config_dict(wl, job.pairs),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_bf16_peak": round(value / world / peak, 4),
-        "roofline": {
-            "kernel": "attn_tc2_kernel<128>", "bound": "tensor",
-            "achieved": None if achieved is None else round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": None if achieved is None else round(achieved / peak, 4),
-            "traffic": ATTN_TRAFFIC_BYTES,
-            "peak_source": "%s bf16_tflops (burst)" % peak_src,
-            "frac_of_sustained": None if achieved is None else round(achieved / float(peaks.get(
-                "bf16_tflops_sustained", peak)), 4),
-            "avg_launch_ms": round(attn_avg_ms, 4), "algorithmic_flops_per_launch": flops_step,
-        },
-        "kernels": {k: {"launches": n, "avg_ms": round(ms / max(n, 1), 5)} for k, (n, ms) in prof.items()},
+        "roofline": roof,
+        "kernels": kernels,
         "gpu_launches": gpu_launches,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -310,28 +484,51 @@ def run_ours(args):
 # ---------------------------------------------------------------------------
 
 def _oracle_sample(wl, n_rows, seed):
-    """Rows spread over all heads and positions, seeded."""
+    """Rows (b, h, i) spread over all batches, heads and positions, seeded."""
     rng = np.random.default_rng(seed)
+    bs = rng.integers(0, wl.B, n_rows)
     heads = rng.integers(0, wl.Hq, n_rows)
     pos = rng.integers(0, wl.T, n_rows)
-    return np.stack([np.zeros(n_rows, np.int64), heads, pos], axis=1)
+    return np.stack([bs, heads, pos], axis=1).astype(np.int64)
 
 
-def _pairs_of_rows(wl, rows):
-    i = rows[:, 2]
-    return int(np.minimum(i + 1, wl.n_start + wl.window + 1).sum())
+def _pairs_of_rows(wl, rows, is_sep):
+    """Kept (q, k) pairs of the sampled rows (same counting as unmasked_pairs)."""
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    if wl.segmented:
+        s, t = i // wl.seg_S, i % wl.seg_S
+        is_long = np.isin(h, np.array(wl.long_heads, dtype=np.int64))
+        extra = np.where(s > 0, np.where(is_long, wl.seg_R, wl.seg_M), 0)
+        return int((t + 1 + extra).sum())
+    n = np.minimum(i + 1, wl.n_start + wl.window + 1)
+    if is_sep is not None:
+        f = is_sep.astype(np.int64).copy()
+        f[:, : wl.n_start] = 0
+        pre = np.concatenate([np.zeros((wl.B, 1), np.int64), np.cumsum(f, axis=1)], axis=1)
+        n = n + pre[b, np.clip(i - wl.window, 0, wl.T)]
+    if wl.topk > 0:
+        n = n + np.minimum(wl.topk, np.maximum(0, i - wl.window - wl.n_start))
+    return int(n.sum())
+
+
+def _oracle_rows(O, wl, inp, rows, nthreads):
+    p = O.params_of(wl)
+    if wl.segmented:
+        O.segment_rows(p, wl.seg_S, wl.seg_M, wl.seg_R, wl.retr_block, inp["is_long"], inp["q"], inp["k"],
+                       inp["v"], rows, nthreads=nthreads)
+    else:
+        O.fwd_rows(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows, nthreads=nthreads)
 
 
 def cpu_baseline(wl, inp, n_rows):
     from oracle import oracle as O
     O.build()
-    p = O.params_of(wl)
     rows = _oracle_sample(wl, n_rows, 1234)
     nthreads = O.nthreads_default()
     t0 = time.perf_counter()
-    O.fwd_rows(p, inp["q"], inp["k"], inp["v"], None, rows, nthreads=nthreads)
+    _oracle_rows(O, wl, inp, rows, nthreads)
     dt = time.perf_counter() - t0
-    flops = 4.0 * wl.d * _pairs_of_rows(wl, rows)
+    flops = 4.0 * wl.d * _pairs_of_rows(wl, rows, inp["is_sep"])
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
             "sample": "%d seeded rows (b, h, i) of the same workload, all heads, fp64, %.1f s" % (n_rows, dt),
             "seconds": round(dt, 2)}
@@ -343,9 +540,8 @@ def run_reference(args):
         return
     from oracle import oracle as O
     O.build()
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[WORKLOAD_ALIASES.get(args.workload, args.workload)]
     inp = synth.make_inputs(wl, seed=0)
-    p = O.params_of(wl)
     nthreads = O.nthreads_default()
     rows_per_step = args.ref_rows
 
@@ -353,8 +549,8 @@ def run_reference(args):
         # one head per step, rows spread over positions
         rows = _oracle_sample(wl, rows_per_step, 100 + s)
         rows[:, 1] = s % wl.Hq
-        O.fwd_rows(p, inp["q"], inp["k"], inp["v"], None, rows, nthreads=nthreads)
-        return _pairs_of_rows(wl, rows)
+        _oracle_rows(O, wl, inp, rows, nthreads)
+        return _pairs_of_rows(wl, rows, inp["is_sep"])
 
     for s in range(args.warmup):
         step(s)
@@ -368,8 +564,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded N(0,1); keys 0-3 x8)",
-        "config": config_dict(wl, unmasked_pairs_per_head(wl) * wl.B * wl.Hq),
+        "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
+        "config": config_dict(wl, unmasked_pairs(wl, inp["is_sep"])),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                          "sample": "each step: %d seeded rows of one head (heads cycle), fp64 C oracle"
                                    % rows_per_step},
@@ -384,6 +580,8 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -391,6 +589,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    args.workload = {v: k for k, v in WORKLOAD_ALIASES.items()}.get(args.workload, args.workload)
     if args.impl == "reference":
         run_reference(args)
     else:

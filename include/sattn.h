@@ -168,7 +168,8 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
  *                  when the pool holds fewer blocks.
  *   O, lse         as in sattn_fwd.
  * bf16 only; S % 128 == 0, T % S == 0, 1 <= retr_block, R % retr_block == 0,
- * R / retr_block <= 1024, Hq <= 256. */
+ * R / retr_block <= 1024, Hq <= 256, and at most 16384 blocks in the largest
+ * pool ((T - S) / retr_block), else SATTN_ERR_UNSUPPORTED. */
 int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
                       const uint8_t* is_long, const void* Q, const void* K, const void* V, void* O, float* lse,
                       int32_t* prefix_blocks, void* ws, size_t ws_bytes, void* stream);

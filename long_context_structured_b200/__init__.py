@@ -225,5 +225,10 @@ def _host_call(fn, tensors, kw):
         if kw.get(name) is not None:
             kw[name] = _to_dev(kw[name], dev)
     res = fn(dq, dk, dv, **kw)
-    outs = tuple(r.to("cpu", non_blocking=False) for r in res)
+    # results land in pinned host buffers (asynchronous copies on the current
+    # stream), then the stream is synchronised once
+    outs = tuple(torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res)
+    for o, r in zip(outs, res):
+        o.copy_(r, non_blocking=True)
+    torch.cuda.current_stream(dev).synchronize()
     return outs

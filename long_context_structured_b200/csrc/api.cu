@@ -98,7 +98,10 @@ int plan_fwd(const sattn_params* p, FwdPlan* pl) {
   P.Tpad = P.nQT * kTile;
   P.npos = std::max(p->T, p->L_pretrain + 1);
   P.n_sink = std::min(p->n_start, p->T);
-  P.short_len = p->topk <= 6 ? 8 : (p->topk <= 14 ? 16 : 32);
+  // shortlist of the scoring pass: wide enough that the gap between the k-th
+  // logit and the last shortlisted score almost always exceeds the bf16
+  // error bound, so that rows rarely need the exact fp32 rescan
+  P.short_len = p->topk <= 8 ? 16 : 32;
   P.capped_sep = p->L_pretrain > 0;
   P.need_qc = P.bf16 && p->L_pretrain > 0 && (p->with_separators || p->topk > 0);
   const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
@@ -584,7 +587,9 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.lse = lse;
   a.status = at<int32_t>(ws, P.status);
   ProfScope ps("attn_tc", 1, st);
-  return cuda_rc(q2 ? launch_attn_tc(a, m, st) : launch_attn_tc2(a, m, st));
+  // capped separator tiles need the second (capped) query tile: one query
+  // tile per CTA; otherwise two query tiles per CTA
+  return cuda_rc(q2 ? launch_attn_tc3(a, m, st) : launch_attn_tc2(a, m, st));
 }
 
 // ---------------------------------------------------------------------------
@@ -593,7 +598,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
 
 struct SegPlan {
   int nQT, N, Rpad, n_long, npos;
-  Region status, tab, qr, kr, kpre, vpre, pcnt;
+  Region status, tab, qr, kr, kpre, vpre, pcnt, score;
   size_t total;
 };
 
@@ -604,7 +609,7 @@ static int plan_seg(const sattn_params* p, int32_t S, int32_t M, int32_t R, int3
   if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
   if (S < kTile || S % kTile || p->T % S || M < 0 || R < 0 || blk < 1 || R % blk) return SATTN_ERR_INVALID_ARG;
   if (R / blk > 1024 || p->Hq > kMaxHeads) return SATTN_ERR_UNSUPPORTED;
-  if ((size_t)(p->T / blk + p->d) * 4 > 200 * 1024) return SATTN_ERR_UNSUPPORTED;
+  if (!segment_retrieval_supported(p->T, S, blk)) return SATTN_ERR_UNSUPPORTED;
   SegPlan P;
   P.nQT = (p->T + kTile - 1) / kTile;
   P.N = p->T / S;
@@ -623,6 +628,7 @@ static int plan_seg(const sattn_params* p, int32_t S, int32_t M, int32_t R, int3
     P.vpre = A.take(B * P.n_long * P.N * P.Rpad * d * 2);
   }
   P.pcnt = A.take(B * std::max(P.n_long, 1) * P.N * 4);
+  if (P.n_long > 0 && R > 0) P.score = A.take(segment_score_bytes(p->B, P.n_long, P.N, p->T, blk));
   P.total = A.cur;
   *out = P;
   return SATTN_OK;
@@ -714,8 +720,9 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
     ra.prefix_cnt = at<int32_t>(ws, P.pcnt);
     ra.Kpre = at<__nv_bfloat16>(ws, P.kpre);
     ra.Vpre = at<__nv_bfloat16>(ws, P.vpre);
+    ra.score = at<float>(ws, P.score);
     {
-      ProfScope ps("segment_retrieval", 2, st);
+      ProfScope ps("segment_retrieval", 3, st);
       SATTN_TRY(launch_segment_retrieval(ra, st));
     }
     const int64_t planes = (int64_t)P.n_long * P.N;
@@ -752,7 +759,7 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
   a.lse = lse;
   a.status = at<int32_t>(ws, P.status);
   ProfScope ps("attn_tc_segment", 1, st);
-  return cuda_rc((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc(a, m, st));
+  return cuda_rc((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc3(a, m, st));
 }
 
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {

@@ -1,10 +1,20 @@
 // attn_tc2.cu -- K5, two query tiles per CTA: the production attention
 // kernel for every case except capped separator tiles (those need a second
-// query operand per tile and run on attn_tc.cu).
+// query operand per tile and run on attn_tc3.cu, one query tile per CTA).
 //
-// Same mathematics as attn_tc.cu (see its header): band tiles, gathered
-// separator / prefix tiles, fp32 side keys merged in the epilogue.  What
-// changes is the schedule:
+// What it computes (per query row i of head h):
+//   O_i = sum_{j in A_i} softmax_j(s_ij) v_j,  LSE_i = ln sum_{j in A_i} exp(s_ij),
+//   s_ij = z_ij / sqrt(d), with A_i split into disjoint parts:
+//     band      keys j in [lo(i), i], lo(i) = max(i - w, n_start) ("LM-Infinite",
+//               section 方法: the recent window; sinks are excluded here),
+//     gathered  separator keys j < i - w from the compacted separator list
+//               ("SepLLM", section 五.2), or the retrieved prefix of a long
+//               head in segmented execution ("Training-Inference Consistent
+//               Segmented Execution", section 整体框架),
+//     side      sink keys j < n_start and top-k keys, whose fp32 logits were
+//               computed elsewhere (prep pass / selector); merged in the
+//               epilogue.
+// Schedule:
 //   - one CTA = two 128-row query tiles (Q0 rows i0..i0+127, Q1 the next 128)
 //     of one (batch, head); every K/V tile either of them needs is loaded
 //     once and used by both;
@@ -12,16 +22,21 @@
 //     tensor core; the single-thread MMA issuer interleaves
 //         PV0(prev), S0(p), PV1(prev), S1(p)
 //     so that while one warpgroup turns S into P the tensor core works on the
-//     other tile;
+//     other tile (two independent issuers let the warpgroups fall into
+//     lockstep and measured slower);
 //   - P (bf16) is written back into TMEM over its own S columns and the PV
 //     product reads it from there (A operand in tensor memory), so P never
 //     touches shared memory;
 //   - TMEM: S0 | S1 | O0 | O1 (4 x 128 fp32 columns);
-//   - K ring of 3 stages, V ring of 2 stages.
+//   - K ring of 2 stages, V ring of 3 stages, each fed by its own producer
+//     warp;
+//   - the row maximum is taken only on a row's first tile (and on the rare
+//     tile whose sum shows that the running reference fell too far behind),
+//     not on every tile: see kSumAccept below.
 // Ordering facts used: tcgen05.commit arrives only after every earlier MMA
 // of the issuing thread completed, so "S_i(p) done" implies "PV_i(prev)
-// done" (O_i stable for rescaling, P_i columns free).  Before S_i(p)
-// overwrites the columns that PV_i(prev) reads, the issuer waits for that PV.
+// done" (O_i stable for rescaling); and one thread's MMAs execute in issue
+// order, so S_i(p) cannot overwrite P_i before PV_i(prev) has read it.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -36,20 +51,22 @@ namespace {
 constexpr int kThreads = 384;  // 2 softmax warpgroups + 1 warpgroup holding the producer and MMA warps
 // register split (per thread): the producer/MMA warpgroup gives registers to
 // the softmax warpgroups; 2*128*kRegSoftmax + 128*kRegCtrl <= 384*168
-constexpr int kRegSoftmax = 216;
-constexpr int kRegCtrl = 72;
+constexpr int kRegSoftmax = 208;
+constexpr int kRegCtrl = 88;
 static_assert(2 * 128 * kRegSoftmax + 128 * kRegCtrl <= kThreads * 168, "register split exceeds the launch budget");
-constexpr int kKS = 3;         // K stages
-constexpr int kVS = 2;         // V stages
+constexpr int kKS = 2;         // K stages (K is consumed early: both S products of a position)
+constexpr int kVS = 3;         // V stages (V is consumed one position later, by the PV products)
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
-// tcgen05.mma operations issued by one thread execute in issue order, so the
-// S_x product issued after PV_x cannot overwrite P_x before PV_x has read
-// it.  Setting this to 1 adds an explicit wait for PV_x before issuing S_x.
-#ifndef SATTN_WAR_WAIT
-#define SATTN_WAR_WAIT 0
-#endif
-
+// A tile's P is computed against the row's running reference m (log2
+// units) without first taking the tile's row maximum.  That is exact
+// arithmetic for softmax as long as nothing overflows: P = 2^(s - m) is
+// stored in bf16 and summed in fp32, both of which keep their relative
+// precision at any magnitude.  A row whose tile sum exceeds 2^kSumAccept
+// (this includes +inf) redoes the tile against its true maximum; a row whose
+// accepted sum exceeds 2^kSumRebase moves m up by a power of two before its
+// next tile, so the rescale of O and l is exact.
+constexpr float kSumAccept = 0x1p32f;
+constexpr float kSumRebase = 0x1p8f;
 __device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
   uint32_t a = smem_u32(bar);
   uint64_t t0 = globaltimer_ns();
@@ -59,14 +76,36 @@ __device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// A[tmem] operand form: D[tmem] (+)= A[tmem] * B[smem]^T
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// MMA and commit issued by one elected lane of a warp that runs the issue
+// loop in lockstep: the loop's values stay warp-uniform (so they live in
+// uniform registers), and a single lane issues each instruction.
+// D[tmem] (+)= A[smem] * B[smem]^T
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
@@ -82,6 +121,66 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+
+// paired fp32 arithmetic (one instruction for two lanes of work)
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+
+
+// P = 2^(s*sl2 + neg_m) for this thread's row of a 128-key tile, packed to
+// bf16 and stored to TMEM over the first 64 S columns (keys 64h..64h+63 go
+// to columns 32h..32h+31); returns the fp32 sum of the row's P.
+// Masked entries hold -inf and give exactly 0.
+__device__ __forceinline__ float emit_p(const float (&sv)[128], float sl2, float neg_m, uint32_t taddr) {
+  float ps[8];
+#pragma unroll
+  for (int y = 0; y < 8; ++y) ps[y] = 0.f;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+      float a0, a1;
+      fma2(a0, a1, sv[hf * 64 + c], sv[hf * 64 + c + 1], sl2, sl2, neg_m, neg_m);
+      const float p0 = ex2_approx(a0);
+      const float p1 = ex2_approx(a1);
+      add2(ps[(c >> 1) & 3], ps[4 + ((c >> 1) & 3)], p0, p1);
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32u(taddr + hf * 32, pk);
+  }
+  return ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+}
+
+// O row *= f (warp-collective: every lane takes part, f = 1 leaves a row as is)
+template <int D>
+__device__ __forceinline__ void scale_o(uint32_t taddr, float f) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float ov[32];
+    tmem_ld32(taddr + c * 32, ov);
+    tc_wait_ld();
+#pragma unroll
+    for (int y = 0; y < 32; ++y) ov[y] *= f;
+    tmem_st32(taddr + c * 32, ov);
+  }
+}
+
+// 2^-e for an integer e in [0, 126]
+__device__ __forceinline__ float exp2_neg_int(int e) { return __int_as_float((127 - e) << 23); }
 
 template <int N>
 __device__ __forceinline__ void regs_dec() {
@@ -237,50 +336,62 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = abort_i;
   if (warp >= 8) {
     regs_dec<kRegCtrl>();
-    if (warp == 8) {
-    // ===================== TMA producer =====================
+    if (warp == 8 || warp == 10) {
+    // ===================== TMA producers: warp 8 Q and K, warp 10 V =====================
+    // two independent streams, so a V stage still in use never delays the next K load
+    const bool kstream = (warp == 8);
     if (lane == 0 && un.n > 0) {
-      const int i0 = 2 * qb * kTile;
-      mbar_expect_tx(q_full, 2 * kTileBytes);
-      for (int x = 0; x < 2; ++x)
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sQ + x * kTileBytes + c * kChunkBytes, &tmQ, q_full, c * 64, i0 + x * kTile, h, b);
+      if (kstream) {
+        const int i0 = 2 * qb * kTile;
+        mbar_expect_tx(q_full, 2 * kTileBytes);
+        for (int x = 0; x < 2; ++x)
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_4d(sQ + x * kTileBytes + c * kChunkBytes, &tmQ, q_full, c * 64, i0 + x * kTile, h, b);
+      }
+      const int NS = kstream ? kKS : kVS;
+      uint8_t* ring = kstream ? sK : sV;
+      uint64_t* full = kstream ? k_full : v_full;
+      uint64_t* empty = kstream ? k_empty : v_empty;
       int issued = 0;
       bool ok = true;
       for (int p = 0; p < un.n && ok; ++p) {
         const bool gat = p < un.NG;
         const int row = gat ? p * kTile : (un.U0 + p - un.NG) * kTile;
         const int c2 = gat ? g_plane : g;
-        const CUtensorMap* mk = gat ? &tmKg : &tmK;
-        const CUtensorMap* mv = gat ? &tmVg : &tmV;
-        const int ks = p % kKS, vs = p % kVS;
-        if (p >= kKS) ok = mbar_wait(k_empty + ks, ((p / kKS) - 1) & 1, abort_flag, a.status, 31);
+        const CUtensorMap* mp = kstream ? (gat ? &tmKg : &tmK) : (gat ? &tmVg : &tmV);
+        const int st = p % NS;
+        if (p >= NS) ok = mbar_wait(empty + st, ((p / NS) - 1) & 1, abort_flag, a.status, kstream ? 31 : 32);
         if (!ok) break;
-        mbar_expect_tx(k_full + ks, kTileBytes);
+        mbar_expect_tx(full + st, kTileBytes);
         for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sK + ks * kTileBytes + c * kChunkBytes, mk, k_full + ks, c * 64, row, c2, b);
-        if (p >= kVS) ok = mbar_wait(v_empty + vs, ((p / kVS) - 1) & 1, abort_flag, a.status, 32);
-        if (!ok) break;
-        mbar_expect_tx(v_full + vs, kTileBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sV + vs * kTileBytes + c * kChunkBytes, mv, v_full + vs, c * 64, row, c2, b);
+          tma_load_4d(ring + st * kTileBytes + c * kChunkBytes, mp, full + st, c * 64, row, c2, b);
         ++issued;
       }
       if (!ok) {
-        mbar_wait_raw(q_full, 0);
-        for (int p = max(0, issued - kVS); p < issued; ++p) {
-          mbar_wait_raw(k_full + p % kKS, (p / kKS) & 1);
-          mbar_wait_raw(v_full + p % kVS, (p / kVS) & 1);
-        }
+        if (kstream) mbar_wait_raw(q_full, 0);
+        for (int p = max(0, issued - NS); p < issued; ++p) mbar_wait_raw(full + p % NS, (p / NS) & 1);
       }
     }
     } else if (warp == 9) {
     // ===================== MMA issuer =====================
-    if (lane == 0 && un.n > 0) {
+    // The whole warp runs this loop (an elected lane issues each MMA and
+    // commit); both tiles' products go out in the order
+    //   PV0(prev), S0(p), PV1(prev), S1(p)
+    // which keeps the two softmax warpgroups half a position apart.
+    if (un.n > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.status, 33);
+      // descriptors of stage / tile bases; the start-address field is addr >> 4
+      // in the low 14 bits, so adding (offset >> 4) moves a descriptor within
+      // shared memory (below 256 KB, the field cannot carry out)
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(sV), kChunkBytes, 1024);
+      auto wait_all = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        const bool r = mbar_wait(bar, parity, abort_flag, a.status, site);
+        return __all_sync(0xffffffffu, r);
+      };
+      bool ok = wait_all(q_full, 0, 33);
       int n_pv[2] = {0, 0};    // PV issued per tile
       int prev[2] = {-1, -1};  // union position whose PV is still pending, per tile
       int v_users[kVS];        // PVs still to come for the position held by each V stage
@@ -288,20 +399,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int x) -> bool {
         const int pp = prev[x];
         const int vs = pp % kVS;
-        if (!mbar_wait(p_full + x, n_pv[x] & 1, abort_flag, a.status, 34 + x)) return false;
-        if (!mbar_wait(v_full + vs, (pp / kVS) & 1, abort_flag, a.status, 36)) return false;
+        if (!wait_all(p_full + x, n_pv[x] & 1, 34 + x)) return false;
+        if (!wait_all(v_full + vs, (pp / kVS) & 1, 36)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + vs * kTileBytes);
-        const uint32_t p_tmem = tmem + x * 128;
-        const uint32_t o_tmem = tmem + 256 + x * 128;
+        const uint64_t bv = dv + (uint64_t)((vs * kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
-          tc_mma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_o, (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(o_done + x);
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts_elect(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
+                       (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
+        commit_elect(o_done + x);
         // the V stage is free once every tile that uses this position ran its PV
-        if (--v_users[vs] == 0) tc_commit(v_empty + vs);
+        if (--v_users[vs] == 0) commit_elect(v_empty + vs);
         ++n_pv[x];
         prev[x] = -1;
         return true;
@@ -312,49 +420,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int users = (need[0] ? 1 : 0) + (need[1] ? 1 : 0);
         bool k_ready = false;
         for (int x = 0; x < 2 && ok; ++x) {
-          // the tile's pending PV goes first (ping-pong: PV0, S0, PV1, S1)
-          const bool had_pv = prev[x] >= 0;
-          if (had_pv) ok = issue_pv(x);
+          if (prev[x] >= 0) ok = issue_pv(x);
           if (!ok || !need[x]) continue;
-#if SATTN_WAR_WAIT
-          if (had_pv) {
-            // P_x (read by that PV) lives in the columns S_x is about to overwrite
-            ok = mbar_wait(o_done + x, (n_pv[x] - 1) & 1, abort_flag, a.status, 38 + x);
-            if (!ok) break;
-          }
-#endif
           if (!k_ready) {
-            ok = mbar_wait(k_full + ks, (p / kKS) & 1, abort_flag, a.status, 40);
+            ok = wait_all(k_full + ks, (p / kKS) & 1, 40);
             if (!ok) break;
             k_ready = true;
             v_users[p % kVS] = users;
           }
           tc_fence_after();
-          const uint32_t a_base = q_addr + x * kTileBytes;
-          const uint32_t k_addr = smem_u32(sK + ks * kTileBytes);
+          const uint64_t ba = dq + (uint64_t)((x * kTileBytes) >> 4);
+          const uint64_t bk = dk + (uint64_t)((ks * kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            tc_mma_ss(tmem + x * 128, smem_desc_sw128(a_base + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                      idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+            mma_ss_elect(tmem + x * 128, ba + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          tc_commit(s_full + x);
+          commit_elect(s_full + x);
           prev[x] = p;
-          const bool later_user = (x == 0) && need[1];
-          if (!later_user) tc_commit(k_empty + ks);
+          if (!((x == 0) && need[1])) commit_elect(k_empty + ks);
         }
         if (ok && users == 0) {
           // no tile reads this position (cannot happen for contiguous plans); release it
-          ok = mbar_wait(k_full + ks, (p / kKS) & 1, abort_flag, a.status, 40);
+          ok = wait_all(k_full + ks, (p / kKS) & 1, 40);
           if (!ok) break;
-          tc_commit(k_empty + ks);
-          ok = mbar_wait(v_full + p % kVS, (p / kVS) & 1, abort_flag, a.status, 36);
-          if (ok) tc_commit(v_empty + p % kVS);
+          commit_elect(k_empty + ks);
+          ok = wait_all(v_full + p % kVS, (p / kVS) & 1, 36);
+          if (ok) commit_elect(v_empty + p % kVS);
         }
       }
+      // pending PVs of the last positions
       for (int x = 0; x < 2 && ok; ++x)
         if (prev[x] >= 0) ok = issue_pv(x);
-      tc_commit(drain);
+      commit_elect(drain);
       mbar_wait_raw(drain, 0);
     }
     __syncwarp();
@@ -371,8 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + x * 128;
     const uint32_t tO = tmem + 256 + x * 128;
     const float sl2 = a.scale_log2;
-    float m_used = -CUDART_INF_F;
+    float m_used = -CUDART_INF_F;  // running reference (log2 units) P is taken against
     float l_sum = 0.f;
+    int rebase = 0;                // pending: m_used += rebase, O and l_sum *= 2^-rebase
     bool ok = true;
     int k = 0;  // tiles processed by this warpgroup
     for (int p = 0; p < un.n; ++p) {
@@ -399,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int j0 = (un.U0 + p - un.NG) * kTile;
         const int lo_fix = max(pl.band_lo, a.ns_band);
-        const bool full = (j0 + kTile - 1 <= i0) && (j0 >= max(lo_fix, i0 + kTile - 1 - a.w_eff));
+        const bool full = (j0 + kTile - 1 <= i0) && (j0 >= max(lo_fix, i0 + kTile - 1 - a.w_eff)) &&
+                          (i0 + kTile <= a.T);
         if (!full) {
           c_lo = max(lo_fix, i - a.w_eff) - j0;
           c_hi = i - j0;
@@ -415,60 +515,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTile; ++c)
           if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
-      float mx;
-      {
-        float pm[8];
-#pragma unroll
-        for (int y = 0; y < 8; ++y) pm[y] = sv[y];
-#pragma unroll
-        for (int c = 8; c < kTile; ++c) pm[c & 7] = fmaxf(pm[c & 7], sv[c]);
-        mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // O_x is stable from here on: S_x(p) completing implies the tile's
+      // previous PV completed.  First the rebase the previous tile asked for.
+      if (__any_sync(0xffffffffu, rebase != 0)) scale_o<D>(tO + lane_off, exp2_neg_int(rebase));
+      if (rebase != 0) {
+        m_used += (float)rebase;
+        l_sum *= exp2_neg_int(rebase);
+        rebase = 0;
       }
-      const float m_new = fmaxf(m_used, mx * sl2);
-      float alpha = 1.f;
-      bool rescale_o = false;
-      if (m_new > m_used + kRescaleThreshold) {
-        alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_new);
-        rescale_o = (k > 0) && (m_used != -CUDART_INF_F);
-        l_sum *= alpha;
-        m_used = m_new;
-      }
-      // O_x is stable here: S_x(p) completing implies the tile's previous PV completed
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        const float f = rescale_o ? alpha : 1.f;
+      bool exact = __any_sync(0xffffffffu, m_used == -CUDART_INF_F);
+      float l_tile;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tmem_ld32(tO + lane_off + c * 32, ov);
-          tc_wait_ld();
+      for (;;) {
+        if (exact) {
+          // 16 independent 2-input chains of 8 steps
+          float pm[16];
 #pragma unroll
-          for (int y = 0; y < 32; ++y) ov[y] *= f;
-          tmem_st32(tO + lane_off + c * 32, ov);
-        }
-      }
-      // P = 2^(s*log2e/sqrt(d) - m) packed to bf16; half h (S columns 64h..64h+63)
-      // goes to TMEM columns 32h..32h+31 over S values already in registers.
-      // A row with no key so far has m_used = -inf and every entry masked:
-      // with a zero offset each exp2(-inf) is exactly 0.
-      {
-        float ps[8];
+          for (int y = 0; y < 16; ++y) pm[y] = sv[y];
 #pragma unroll
-        for (int y = 0; y < 8; ++y) ps[y] = 0.f;
-        const float neg_m = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
+          for (int c = 16; c < kTile; ++c) pm[c & 15] = fmaxf(pm[c & 15], sv[c]);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t pk[32];
+          for (int w = 8; w > 0; w >>= 1)
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2_approx(fmaf(sv[hf * 64 + c], sl2, neg_m));
-            const float p1 = ex2_approx(fmaf(sv[hf * 64 + c + 1], sl2, neg_m));
-            ps[(c >> 1) & 7] += p0 + p1;
-            pk[c >> 1] = pack_bf16x2(p0, p1);
+            for (int y = 0; y < w; ++y) pm[y] = fmaxf(pm[y], pm[y + w]);
+          const float m_new = fmaxf(m_used, pm[0] * sl2);
+          float alpha = 1.f;
+          bool rescale_o = false;
+          if (m_new > m_used) {
+            alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_new);
+            rescale_o = (k > 0) && (m_used != -CUDART_INF_F);
+            l_sum *= alpha;
+            m_used = m_new;
           }
-          tmem_st32u(tS + lane_off + hf * 32, pk);
+          if (__any_sync(0xffffffffu, rescale_o)) scale_o<D>(tO + lane_off, rescale_o ? alpha : 1.f);
         }
-        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        // a row with no key so far has m_used = -inf and every entry masked:
+        // with a zero offset each exp2(-inf) is exactly 0
+        l_tile = emit_p(sv, sl2, (m_used == -CUDART_INF_F) ? 0.f : -m_used, tS + lane_off);
+        if (exact || !__any_sync(0xffffffffu, !(l_tile <= kSumAccept))) break;
+        exact = true;  // some row overflowed its bound: redo against the true maxima
       }
+      l_sum += l_tile;
+      if (l_tile > kSumRebase) rebase = ((__float_as_int(l_tile) >> 23) & 0xff) - 126;  // 2^rebase > l_tile
       tc_wait_st();
       tc_fence_before();
       if (ok) mbar_arrive(p_full + x);
@@ -479,6 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (k > 0) {
       ok = ok && mbar_wait(o_done + x, (k - 1) & 1, abort_flag, a.status, 43 + x);
       tc_fence_after();
+    }
+    float o_rebase = 1.f;
+    if (rebase != 0) {
+      m_used += (float)rebase;
+      l_sum *= exp2_neg_int(rebase);
+      o_rebase = exp2_neg_int(rebase);
     }
     const bool row_ok = (i < a.T);
     const int ir = row_ok ? i : a.T - 1;
@@ -506,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tO + lane_off + c * 32, ov);
         tc_wait_ld();
 #pragma unroll
-        for (int y = 0; y < 32; ++y) ov[y] *= alpha;
+        for (int y = 0; y < 32; ++y) ov[y] *= alpha * o_rebase;
       } else {
 #pragma unroll
         for (int y = 0; y < 32; ++y) ov[y] = 0.f;
@@ -572,7 +666,7 @@ cudaError_t launch_d(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
 }  // namespace
 
 // Two-tile kernel; the caller routes capped separator tiles (q2) and
-// segment lengths that are not multiples of 256 to launch_attn_tc.
+// segment lengths that are not multiples of 256 to launch_attn_tc3.
 cudaError_t launch_attn_tc2(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
   if (a.B * a.Hq * a.nQT == 0) return cudaSuccess;
   if (a.q2) return cudaErrorInvalidValue;

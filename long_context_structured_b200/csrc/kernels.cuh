@@ -101,11 +101,11 @@ struct AttnArgs {
 struct AttnMaps {
   CUtensorMap q, q2, k, v, kg, vg;
 };
-// one 128-row query tile per CTA (every case, incl. capped separator tiles)
-cudaError_t launch_attn_tc(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
 // two query tiles per CTA; not for q2 (capped separator tiles) and, in
 // segmented mode, only when the segment length is a multiple of 256
 cudaError_t launch_attn_tc2(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
+// one query tile per CTA with the score tile double-buffered in TMEM; every case
+cudaError_t launch_attn_tc3(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
 // K6: fp32 attention on CUDA cores
@@ -178,7 +178,14 @@ struct SegRetrArgs {
   int32_t* prefix_cnt;         // [B, n_long, N]
   __nv_bfloat16* Kpre;         // [B, n_long, N, R, d] rotated at virtual positions
   __nv_bfloat16* Vpre;
+  float* score;                // [B, n_long, N, T / blk] block scores (workspace)
 };
+// largest shared-memory sort buffer of the block selection (bytes)
+constexpr size_t kSegSelectSmemMax = 128 * 1024;
+// bytes of the block-score workspace
+size_t segment_score_bytes(int B, int n_long, int N, int T, int blk);
+// whether the block selection's sort fits in shared memory
+bool segment_retrieval_supported(int T, int S, int blk);
 cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st);
 
 }  // namespace sattn

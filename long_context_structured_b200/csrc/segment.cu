@@ -17,115 +17,194 @@
 // queries and keys keep their global positions and each prefix key p is
 // rotated to the virtual position sS - P + p, which puts it at distance
 // P + t - p from the query at sS + t, exactly as positions p and P + t do.
+//
+// Three kernels:
+//  1. block_score_kernel: every key of the largest pool is read once and
+//     dotted with up to 16 segment-end queries at a time (fp32, queries held
+//     in registers, a key spread over d/8 lanes with 16-byte loads); the
+//     per-key dots go through shared memory into per-block maxima;
+//  2. block_select_kernel: per (segment, long head) a bitonic sort of the
+//     pool's block scores by (score desc, block asc), the first R/blk kept
+//     and put in ascending block order;
+//  3. prefix_assemble_kernel: gathers the chosen K rows (rotated to their
+//     virtual positions) and V rows into the dense prefix planes the
+//     attention kernel loads by TMA.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "kernels.cuh"
+#include "simt.cuh"
 
 namespace sattn {
 
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kChunkKeys = 128;  // keys scored per pass of a CTA
+constexpr int kQG = 16;          // segment-end queries per pass
 
-// grid (N - 1, n_long, B): segment s = blockIdx.x + 1
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 v = __bfloat1622float2(h[e]);
+    f[2 * e] = v.x;
+    f[2 * e + 1] = v.y;
+  }
+}
+
+// grid (ceil(nblk_pool / nblk_cta), n_long, B).  CTA x scores blocks
+// [x * nblk_cta, ...) of the pool of its long head for every segment s >= 1:
+// score[b, slot, s, u] = max over the block's keys of <q_{sS-1}, k_j>.
+// Entries whose block lies beyond segment s's pool are written too and
+// never read.
+template <int D>
+__global__ void __launch_bounds__(kThreads) block_score_kernel(SegRetrArgs a, int nblk_pool, int nblk_cta) {
+  constexpr int LPK = D / 8;     // lanes per key, 8 elements each
+  constexpr int KPW = 32 / LPK;  // keys per warp per step
+  __shared__ float sdot[kChunkKeys][kQG + 1];
+  __shared__ float smax[kChunkKeys][kQG];  // per block of this CTA (nblk_cta <= kChunkKeys)
+  const int slot = blockIdx.y, b = blockIdx.z;
+  const int h = a.long_heads[slot];
+  const int g = h / (a.Hq / a.Hkv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPK;
+  const int u0 = blockIdx.x * nblk_cta;
+  const int u1 = min(u0 + nblk_cta, nblk_pool);
+  const int k_begin = u0 * a.blk, k_end = u1 * a.blk;
+  const __nv_bfloat16* kb = a.K + b * a.k_sb + g * a.k_sh;
+  const __nv_bfloat16* qb = a.Q + b * a.q_sb + h * a.q_sh;
+  for (int s0 = 1; s0 < a.N; s0 += kQG) {
+    // this lane's 8 elements of the (up to) 16 segment-end queries
+    float qr[kQG][8];
+#pragma unroll
+    for (int q = 0; q < kQG; ++q) {
+      const int s = s0 + q;
+      if (s < a.N) {
+        unpack8(*reinterpret_cast<const uint4*>(qb + (int64_t)(s * a.S - 1) * a.q_st + sub * 8), qr[q]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qr[q][e] = 0.f;
+      }
+    }
+    for (int x = threadIdx.x; x < (u1 - u0) * kQG; x += kThreads) smax[x / kQG][x % kQG] = -CUDART_INF_F;
+    for (int c0 = k_begin; c0 < k_end; c0 += kChunkKeys) {
+      for (int kk = warp * KPW + lane / LPK; kk < kChunkKeys; kk += (kThreads / 32) * KPW) {
+        const int j = c0 + kk;
+        float kv[8];
+        if (j < k_end) {
+          unpack8(*reinterpret_cast<const uint4*>(kb + (int64_t)j * a.k_st + sub * 8), kv);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
+        }
+        float dot[kQG];
+#pragma unroll
+        for (int q = 0; q < kQG; ++q) {
+          float A0 = 0.f, A1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) fma2(A0, A1, qr[q][e], qr[q][e + 1], kv[e], kv[e + 1], A0, A1);
+          dot[q] = A0 + A1;
+        }
+        // the whole warp takes part (keys past the end carry zeros)
+        group_reduce_transposed<kQG, LPK>(dot, 0xffffffffu, lane);
+        constexpr int per = kQG >= LPK ? kQG / LPK : 1;
+        constexpr int dup = kQG >= LPK ? 1 : LPK / kQG;
+        if (j < k_end && sub % dup == 0) {
+#pragma unroll
+          for (int q = 0; q < per; ++q) sdot[kk][(sub / dup) * per + q] = dot[q];
+        }
+      }
+      __syncthreads();
+      // block maxima of this chunk: a warp per (block, query)
+      const int c1 = min(c0 + kChunkKeys, k_end);
+      for (int pr = warp; pr < (u1 - u0) * kQG; pr += kThreads / 32) {
+        const int bl = pr / kQG, q = pr % kQG;
+        const int lo = max((u0 + bl) * a.blk, c0), hi = min((u0 + bl + 1) * a.blk, c1);
+        float m = -CUDART_INF_F;
+        for (int j = lo + lane; j < hi; j += 32) m = fmaxf(m, sdot[j - c0][q]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) smax[bl][q] = fmaxf(smax[bl][q], m);
+      }
+      __syncthreads();
+    }
+    const int nblk_all = a.T / a.blk;
+    for (int x = threadIdx.x; x < (u1 - u0) * kQG; x += kThreads) {
+      const int bl = x / kQG, q = x % kQG;
+      const int s = s0 + q;
+      if (s < a.N) a.score[(((size_t)b * a.n_long + slot) * a.N + s) * nblk_all + u0 + bl] = smax[bl][q];
+    }
+    __syncthreads();
+  }
+}
+
+// total order key for a descending sort: larger score first, then the lower block
+__device__ __forceinline__ unsigned long long order_key(float z, int u) {
+  const uint32_t bits = __float_as_uint(z);
+  const uint32_t ord = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);  // monotone in z
+  return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)u);
+}
+
+// grid (N - 1, n_long, B): segment s = blockIdx.x + 1.  Dynamic shared
+// memory: next_pow2(blocks of the largest pool) 64-bit keys.
 __global__ void __launch_bounds__(kThreads) block_select_kernel(SegRetrArgs a) {
-  extern __shared__ float sm[];
+  extern __shared__ unsigned long long keys[];
+  __shared__ int chosen[1024];
   const int s = blockIdx.x + 1;
   const int slot = blockIdx.y;
   const int b = blockIdx.z;
   const int h = a.long_heads[slot];
-  const int g = h / (a.Hq / a.Hkv);
   const int nb = a.R / a.blk;
   const int nblocks = s * a.S / a.blk;
-  float* q = sm;                         // [d]
-  float* score = sm + a.d;               // [nblocks]
-  __shared__ float red_z[kThreads / 32];
-  __shared__ int red_u[kThreads / 32];
-  __shared__ int chosen[1024];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const __nv_bfloat16* qp = a.Q + b * a.q_sb + h * a.q_sh + (int64_t)(s * a.S - 1) * a.q_st;
-  for (int c = threadIdx.x; c < a.d; c += blockDim.x) q[c] = __bfloat162float(qp[c]);
-  __syncthreads();
-  const __nv_bfloat16* kb = a.K + b * a.k_sb + g * a.k_sh;
-  for (int u = warp; u < nblocks; u += kThreads / 32) {
-    float best = -CUDART_INF_F;
-    for (int x = lane; x < a.blk; x += 32) {
-      const __nv_bfloat16* kp = kb + (int64_t)(u * a.blk + x) * a.k_st;
-      float acc = 0.f;
-      for (int c = 0; c < a.d; c += 2) {
-        const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kp + c));
-        acc = fmaf(q[c], kv.x, fmaf(q[c + 1], kv.y, acc));
-      }
-      best = fmaxf(best, acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-    if (lane == 0) score[u] = best;
-  }
-  __syncthreads();
   const int nsel = min(nb, nblocks);
-  for (int r = 0; r < nsel; ++r) {
-    float bz = -CUDART_INF_F;
-    int bu = -1;
-    for (int u = threadIdx.x; u < nblocks; u += blockDim.x) {
-      const float z = score[u];
-      if (z == -CUDART_INF_F) continue;  // taken (scores of real blocks are finite)
-      if (bu < 0 || z > bz) {
-        bz = z;
-        bu = u;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-      const int ou = __shfl_xor_sync(0xffffffffu, bu, o);
-      if (ou >= 0 && (bu < 0 || oz > bz || (oz == bz && ou < bu))) {
-        bz = oz;
-        bu = ou;
-      }
-    }
-    if (lane == 0) {
-      red_z[warp] = bz;
-      red_u[warp] = bu;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float wz = red_z[0];
-      int wu = red_u[0];
-      for (int w = 1; w < kThreads / 32; ++w) {
-        const float oz = red_z[w];
-        const int ou = red_u[w];
-        if (ou >= 0 && (wu < 0 || oz > wz || (oz == wz && ou < wu))) {
-          wz = oz;
-          wu = ou;
+  int P2 = 1;
+  while (P2 < nblocks) P2 <<= 1;
+  const int nblk_all = a.T / a.blk;
+  const float* score = a.score + (((size_t)b * a.n_long + slot) * a.N + s) * nblk_all;
+  for (int u = threadIdx.x; u < P2; u += kThreads) keys[u] = (u < nblocks) ? order_key(score[u], u) : 0ull;
+  __syncthreads();
+  // bitonic sort, descending
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int x = threadIdx.x; x < P2; x += kThreads) {
+        const int y = x ^ jj;
+        if (y > x) {
+          const unsigned long long p = keys[x], q = keys[y];
+          const bool first_half = (x & k) == 0;
+          if (first_half ? (p < q) : (p > q)) {
+            keys[x] = q;
+            keys[y] = p;
+          }
         }
       }
-      chosen[r] = wu;
-      score[wu] = -CUDART_INF_F;
+      __syncthreads();
     }
-    __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    // ascending block order
-    for (int x = 1; x < nsel; ++x) {
-      const int v = chosen[x];
-      int y = x - 1;
-      while (y >= 0 && chosen[y] > v) {
-        chosen[y + 1] = chosen[y];
-        --y;
-      }
-      chosen[y + 1] = v;
+  // the first nsel blocks, in ascending block order (rank by count)
+  for (int x = threadIdx.x; x < nsel; x += kThreads) {
+    const int u = (int)(0xFFFFFFFFu - (uint32_t)(keys[x] & 0xFFFFFFFFull));
+    int rank = 0;
+    for (int y = 0; y < nsel; ++y) {
+      const int v = (int)(0xFFFFFFFFu - (uint32_t)(keys[y] & 0xFFFFFFFFull));
+      rank += (v < u) ? 1 : 0;
     }
-    a.prefix_cnt[((size_t)b * a.n_long + slot) * a.N + s] = nsel * a.blk;
+    chosen[rank] = u;
   }
   __syncthreads();
+  if (threadIdx.x == 0) a.prefix_cnt[((size_t)b * a.n_long + slot) * a.N + s] = nsel * a.blk;
   int32_t* out = a.prefix_blocks + (((size_t)b * a.Hq + h) * a.N + s) * nb;
-  for (int x = threadIdx.x; x < nb; x += blockDim.x) out[x] = x < nsel ? chosen[x] : -1;
+  for (int x = threadIdx.x; x < nb; x += kThreads) out[x] = x < nsel ? chosen[x] : -1;
 }
 
-// grid (Rpad / 8, (N - 1) * n_long, B); one warp per prefix row
+// grid (Rpad / 8, (N - 1) * n_long, B); one warp per prefix row.  Lanes
+// [0, d/8) rotate 4 pairs of K each (8-byte loads from both halves, the
+// virtual position's cos/sin as two float4), lanes [16, 16 + d/8) copy 16
+// bytes of V each.
+template <int D>
 __global__ void prefix_assemble_kernel(SegRetrArgs a, int Rpad) {
+  constexpr int half = D / 2;
+  constexpr int kLanes = D / 8;  // K lanes (4 pairs each) = V lanes (16 bytes each)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x * 8 + warp;
   const int s = blockIdx.y % (a.N - 1) + 1;
@@ -135,46 +214,107 @@ __global__ void prefix_assemble_kernel(SegRetrArgs a, int Rpad) {
   const int h = a.long_heads[slot];
   const int g = h / (a.Hq / a.Hkv);
   const int cnt = a.prefix_cnt[((size_t)b * a.n_long + slot) * a.N + s];
-  const size_t orow = ((((size_t)b * a.n_long + slot) * a.N + s) * Rpad + p) * a.d;
-  const int half = a.d / 2;
-  const int nb = a.R / a.blk;
+  const size_t orow = ((((size_t)b * a.n_long + slot) * a.N + s) * Rpad + p) * D;
   if (p >= cnt) {
-    for (int c = lane; c < a.d; c += 32) {
-      a.Kpre[orow + c] = __float2bfloat16_rn(0.f);
-      a.Vpre[orow + c] = __float2bfloat16_rn(0.f);
+    if (lane < kLanes) {
+      reinterpret_cast<uint4*>(a.Kpre + orow)[lane] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(a.Vpre + orow)[lane] = make_uint4(0, 0, 0, 0);
     }
     return;
   }
+  const int nb = a.R / a.blk;
   const int blk_id = a.prefix_blocks[(((size_t)b * a.Hq + h) * a.N + s) * nb + p / a.blk];
   const int j = blk_id * a.blk + p % a.blk;
   const int vpos = s * a.S - cnt + p;
-  const __nv_bfloat16* kp = a.K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
-  const __nv_bfloat16* vp = a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st;
-  for (int c = lane; c < half; c += 32) {
-    const float k0 = __bfloat162float(kp[c]), k1 = __bfloat162float(kp[c + half]);
-    const float2 cs = a.tab ? a.tab[(int64_t)vpos * half + c] : make_float2(1.f, 0.f);
-    a.Kpre[orow + c] = __float2bfloat16_rn(k0 * cs.x - k1 * cs.y);
-    a.Kpre[orow + c + half] = __float2bfloat16_rn(k1 * cs.x + k0 * cs.y);
+  if (lane < kLanes) {
+    const int c = lane * 4;
+    const __nv_bfloat16* kp = a.K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
+    const uint2 lo = *reinterpret_cast<const uint2*>(kp + c);
+    const uint2 hi = *reinterpret_cast<const uint2*>(kp + c + half);
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+    float k0[4], k1[4], cs[4], sn[4];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 x = __bfloat1622float2(l2[e]), y = __bfloat1622float2(h2[e]);
+      k0[2 * e] = x.x;
+      k0[2 * e + 1] = x.y;
+      k1[2 * e] = y.x;
+      k1[2 * e + 1] = y.y;
+    }
+    if (a.tab) {
+      const float4* t = reinterpret_cast<const float4*>(a.tab + (int64_t)vpos * half + c);
+      const float4 t0 = t[0], t1 = t[1];
+      cs[0] = t0.x; sn[0] = t0.y; cs[1] = t0.z; sn[1] = t0.w;
+      cs[2] = t1.x; sn[2] = t1.y; cs[3] = t1.z; sn[3] = t1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cs[e] = 1.f;
+        sn[e] = 0.f;
+      }
+    }
+    uint2 olo, ohi;
+    __nv_bfloat162* o_l = reinterpret_cast<__nv_bfloat162*>(&olo);
+    __nv_bfloat162* o_h = reinterpret_cast<__nv_bfloat162*>(&ohi);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      o_l[e] = __floats2bfloat162_rn(k0[2 * e] * cs[2 * e] - k1[2 * e] * sn[2 * e],
+                                     k0[2 * e + 1] * cs[2 * e + 1] - k1[2 * e + 1] * sn[2 * e + 1]);
+      o_h[e] = __floats2bfloat162_rn(k1[2 * e] * cs[2 * e] + k0[2 * e] * sn[2 * e],
+                                     k1[2 * e + 1] * cs[2 * e + 1] + k0[2 * e + 1] * sn[2 * e + 1]);
+    }
+    *reinterpret_cast<uint2*>(a.Kpre + orow + c) = olo;
+    *reinterpret_cast<uint2*>(a.Kpre + orow + c + half) = ohi;
+  } else if (lane >= 16 && lane < 16 + kLanes) {
+    const __nv_bfloat16* vp = a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st;
+    reinterpret_cast<uint4*>(a.Vpre + orow)[lane - 16] = reinterpret_cast<const uint4*>(vp)[lane - 16];
   }
-  for (int c = lane; c < a.d; c += 32) a.Vpre[orow + c] = vp[c];
+}
+
+template <int D>
+cudaError_t launch_d(const SegRetrArgs& a, cudaStream_t st) {
+  const int nblk_pool = (a.N - 1) * a.S / a.blk;  // blocks of the largest pool
+  if (nblk_pool > 0) {
+    const int nblk_cta = std::max(1, kChunkKeys / a.blk);
+    dim3 g1((nblk_pool + nblk_cta - 1) / nblk_cta, a.n_long, a.B);
+    block_score_kernel<D><<<g1, kThreads, 0, st>>>(a, nblk_pool, nblk_cta);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  int P2 = 1;
+  while (P2 < nblk_pool) P2 <<= 1;
+  const size_t smem = (size_t)P2 * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 g2(a.N - 1, a.n_long, a.B);
+  block_select_kernel<<<g2, kThreads, smem, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int Rpad = (a.R + kTile - 1) / kTile * kTile;
+  dim3 g3(Rpad / 8, (a.N - 1) * a.n_long, a.B);
+  prefix_assemble_kernel<D><<<g3, 256, 0, st>>>(a, Rpad);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t segment_score_bytes(int B, int n_long, int N, int T, int blk) {
+  return (size_t)B * n_long * N * (size_t)(T / blk) * sizeof(float);
+}
+
+bool segment_retrieval_supported(int T, int S, int blk) {
+  const int nblk_pool = (T / S - 1) * S / blk;
+  int P2 = 1;
+  while (P2 < nblk_pool) P2 <<= 1;
+  return (size_t)P2 * sizeof(unsigned long long) <= kSegSelectSmemMax;
+}
+
 cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st) {
   if (a.N <= 1 || a.n_long == 0 || a.R == 0 || a.B == 0) return cudaSuccess;
-  const int nblocks_max = (a.N - 1) * a.S / a.blk;
-  const size_t smem = (size_t)(a.d + nblocks_max) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 g1(a.N - 1, a.n_long, a.B);
-  block_select_kernel<<<g1, kThreads, smem, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int Rpad = (a.R + kTile - 1) / kTile * kTile;
-  dim3 g2(Rpad / 8, (a.N - 1) * a.n_long, a.B);
-  prefix_assemble_kernel<<<g2, 256, 0, st>>>(a, Rpad);
-  return cudaGetLastError();
+  if (a.d == 128) return launch_d<128>(a, st);
+  if (a.d == 64) return launch_d<64>(a, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sattn

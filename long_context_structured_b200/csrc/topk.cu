@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kStages = 4;
+constexpr int kScratchStride = 33;  // floats per scan thread's scratch row (odd: no bank conflicts)
 
 template <typename Tin>
 __device__ __forceinline__ float ld_in(const Tin* p);
@@ -184,9 +185,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
+    // scan warps: thread r owns query row i0 + r (TMEM lane r)
     const int r = threadIdx.x;
     const int i = i0 + r;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // candidates of this row: n_start <= j <= i - w - 1; of the warp's rows,
+    // the smallest upper bound decides which tiles need no per-column mask
+    const int j_hi = i - a.window - 1;
+    float* my_scratch = reinterpret_cast<float*>(base + kTileBytes * (1 + kStages) + 1024) + r * kScratchStride;
+    const int warp_j_hi = i0 + warp * 32 - a.window - 1;
     float vals[KC];
     int idxs[KC];
 #pragma unroll
@@ -201,39 +208,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = it % kStages;
       ok = ok && mbar_wait(s_full + st, (it / kStages) & 1, abort_flag, a.status, 25);
       tc_fence_after();
-      const int j0 = (u_lo + it) * kTile;
-      const int c_lo = max(0, a.n_start - j0);
-      const int c_hi = min(kTile - 1, i - a.window - 1 - j0);
-#pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tmem_ld32(tmem + st * 128 + lane_off + c4 * 32, v);
-        tc_wait_ld();
-        uint32_t sepm = 0;
-        if (flags) {
-          const int jj = j0 + c4 * 32 + lane;
-          sepm = __ballot_sync(0xffffffffu, jj < a.T && flags[jj] != 0);
-        }
-        const int lo = max(c_lo - c4 * 32, 0);
-        const int hi = min(c_hi - c4 * 32, 31);
-        uint32_t vm = 0;
-        if (lo <= hi) vm = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
-        vm &= ~sepm;
-        ncand += __popc(vm);
-        float mx = -CUDART_INF_F;
+      float v[128];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          v[x] = ((vm >> x) & 1u) ? v[x] : -CUDART_INF_F;
-          mx = fmaxf(mx, v[x]);
-        }
-        if (mx > vals[KC - 1]) {
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (v[x] > vals[KC - 1]) list_insert<KC>(v[x], j0 + c4 * 32 + x, vals, idxs);
-        }
-      }
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + st * 128 + lane_off + c4 * 32, v + c4 * 32);
+      tc_wait_ld();
+      // the scores are in registers: hand the TMEM buffer back to the MMA warp
       tc_fence_before();
       if (ok) mbar_arrive(s_free + st);
+      const int j0 = (u_lo + it) * kTile;
+      const bool interior = (j0 >= a.n_start) && (j0 + kTile - 1 <= warp_j_hi);
+      if (!interior || flags) {
+        const int c_lo = max(0, a.n_start - j0);
+        const int c_hi = min(kTile - 1, j_hi - j0);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t sepm = 0;
+          if (flags) {
+            const int jj = j0 + c4 * 32 + lane;
+            sepm = __ballot_sync(0xffffffffu, jj < a.T && flags[jj] != 0);
+          }
+          const int lo = max(c_lo - c4 * 32, 0);
+          const int hi = min(c_hi - c4 * 32, 31);
+          uint32_t vm = 0;
+          if (lo <= hi) vm = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
+          vm &= ~sepm;
+          ncand += __popc(vm);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[c4 * 32 + x] = ((vm >> x) & 1u) ? v[c4 * 32 + x] : -CUDART_INF_F;
+        }
+      } else {
+        ncand += kTile;
+      }
+      // per 32-column chunk maxima (independent chains), then the insertion
+      // path only for chunks that beat the row's current threshold
+      float cm[4];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float pm[8];
+#pragma unroll
+        for (int y = 0; y < 8; ++y) pm[y] = v[c4 * 32 + y];
+#pragma unroll
+        for (int x = 8; x < 32; ++x) pm[x & 7] = fmaxf(pm[x & 7], v[c4 * 32 + x]);
+        cm[c4] = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      }
+      // a chunk that beats the threshold goes through this thread's shared
+      // scratch row, so one copy of the insertion code serves every column
+      // (an unrolled insertion per column would not fit the instruction cache)
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        if (cm[c4] > vals[KC - 1]) {
+          uint32_t msk = 0;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            my_scratch[x] = v[c4 * 32 + x];
+            msk |= (v[c4 * 32 + x] > vals[KC - 1]) ? (1u << x) : 0u;
+          }
+          while (msk) {
+            const int x = __ffs(msk) - 1;
+            msk &= msk - 1;
+            const float z = my_scratch[x];
+            if (z > vals[KC - 1]) list_insert<KC>(z, j0 + c4 * 32 + x, vals, idxs);
+          }
+        }
+      }
     }
     if (i < a.T) {
       const size_t row = ((size_t)b * a.Hq + h) * a.T + i;
@@ -501,7 +538,7 @@ template <int D, int KC>
 cudaError_t launch_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
   const size_t tile = (size_t)D * kTile * 2;
   // at least 116 KB: one CTA per SM, so the 512-column TMEM allocation never waits
-  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (1 + kStages) + 256);
+  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (1 + kStages) + 1024 + 128 * kScratchStride * 4);
   cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   topk_score_kernel<D, KC><<<(unsigned)(a.B * a.Hq * a.nQT), kThreads, bytes, st>>>(m.qsel, m.ksel, a);
