@@ -216,19 +216,87 @@ def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> in
     return int(st.value)
 
 
-def _host_call(fn, tensors, kw):
-    """Host tensors in, host tensors out: H2D copies, the device call, D2H copies."""
+_copy_streams: dict = {}
+
+
+def _copy_stream_pair(dev):
+    """(host-to-device stream, device-to-host stream) of a device."""
+    st = _copy_streams.get(dev)
+    if st is None:
+        st = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        _copy_streams[dev] = st
+    return st
+
+
+def _host_chunks(B: int, Hq: int, Hkv: int, n: int):
+    """Independent pieces of a problem: ("b", b0, b1) batch ranges when B > 1,
+    else ("h", kv0, kv1) ranges of kv heads (whole GQA groups)."""
+    if B > 1:
+        n = min(n, B)
+        return [("b", B * c // n, B * (c + 1) // n) for c in range(n)]
+    n = min(n, Hkv)
+    return [("h", Hkv * c // n, Hkv * (c + 1) // n) for c in range(n)]
+
+
+def _host_call(fn, tensors, kw, n_chunks: int = 4):
+    """Host tensors in, host tensors out: the end-to-end path.
+
+    Batches (or, for one sequence, groups of kv heads) are independent, so the
+    problem is cut into a few pieces: one copy stream moves piece c+1 to the
+    device while the compute stream runs piece c, and a second copy stream
+    brings each piece's results back as soon as they are ready (the two
+    directions overlap).  Outputs land in pinned host memory; the result
+    equals the one-piece call bit for bit."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    dq, dk, dv = (_to_dev(t, dev) for t in tensors)
+    q, k, v = tensors
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    rep = Hq // Hkv
+    compute = torch.cuda.current_stream(dev)
+    copy, back = _copy_stream_pair(dev)
+    copy.wait_stream(compute)  # device buffers below are allocated on the compute stream
+    dq, dk, dv = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (q, k, v))
     kw = dict(kw)
-    for name in ("is_sep", "topk_idx", "topk_logit"):
-        if kw.get(name) is not None:
-            kw[name] = _to_dev(kw[name], dev)
-    res = fn(dq, dk, dv, **kw)
-    # results land in pinned host buffers (asynchronous copies on the current
-    # stream), then the stream is synchronised once
-    outs = tuple(torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res)
-    for o, r in zip(outs, res):
-        o.copy_(r, non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
-    return outs
+    side = {name: kw.pop(name) for name in ("is_sep", "topk_idx", "topk_logit") if kw.get(name) is not None}
+    dside = {name: torch.empty(t.shape, dtype=t.dtype, device=dev) for name, t in side.items()}
+    outs_host = None
+    res_keep = []
+    for kind, x0, x1 in _host_chunks(B, Hq, Hkv, n_chunks):
+        if kind == "b":
+            sl_q = sl_kv = sl_side = (slice(x0, x1),)
+        else:
+            sl_q = (slice(None), slice(x0 * rep, x1 * rep))
+            sl_kv = (slice(None), slice(x0, x1))
+            sl_side = (slice(None),)
+        with torch.cuda.stream(copy):
+            for src, dst, sl in ((q, dq, sl_q), (k, dk, sl_kv), (v, dv, sl_kv)):
+                dst[sl].copy_(src[sl], non_blocking=True)
+            for name, t in side.items():
+                if name == "is_sep":
+                    if kind == "b" or x0 == 0:  # flags are per sequence, shared by head pieces
+                        dside[name][sl_side].copy_(t[sl_side], non_blocking=True)
+                else:
+                    dside[name][sl_q].copy_(t[sl_q], non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(copy)
+        compute.wait_event(ready)
+        ckw = dict(kw)
+        for name, t in dside.items():
+            ckw[name] = t[sl_side] if name == "is_sep" else t[sl_q]
+        if "is_long" in ckw and kind == "h":
+            ckw["is_long"] = list(ckw["is_long"])[x0 * rep:x1 * rep]
+        res = fn(dq[sl_q], dk[sl_kv], dv[sl_kv], **ckw)
+        done = torch.cuda.Event()
+        done.record(compute)
+        if outs_host is None:
+            shapes = [((B,) + tuple(r.shape[1:])) if kind == "b" else ((B, Hq) + tuple(r.shape[2:])) for r in res]
+            outs_host = tuple(torch.empty(sh, dtype=r.dtype, pin_memory=True) for sh, r in zip(shapes, res))
+        back.wait_event(done)
+        with torch.cuda.stream(back):
+            for oh, r in zip(outs_host, res):
+                oh[sl_q].copy_(r, non_blocking=True)
+        res_keep.append(res)  # device results stay alive until the copies finish
+    back.synchronize()
+    copy.synchronize()
+    compute.synchronize()
+    return outs_host

@@ -577,6 +577,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.gather_mode = is_sep ? 1 : 0;
   a.q2 = q2;
   a.sep_pos = sep_pos;
+  a.sep_prefix = at<int32_t>(ws, P.prefix);
   a.ranges = ranges;
   a.window = p->window;
   for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;

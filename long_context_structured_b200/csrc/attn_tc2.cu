@@ -182,14 +182,6 @@ __device__ __forceinline__ void scale_o(uint32_t taddr, float f) {
 // 2^-e for an integer e in [0, 126]
 __device__ __forceinline__ float exp2_neg_int(int e) { return __int_as_float((127 - e) << 23); }
 
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
 
 // Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
 // then band key tiles [u_lo, u_lo + n_band).
@@ -484,14 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r0 + kTile > pl.g_full) {
           int lim = min(kTile, pl.g_count - r0);
           if (a.gather_mode == 1) {
-            const int* pos = a.sep_pos + (size_t)b * a.T + r0;
+            // separators kept by row i: pos < i - w; their count is a prefix count
             const int thr = i - a.window;
-            int lo = 0, hi = max(lim, 0);
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              if (__ldg(pos + mid) < thr) lo = mid + 1; else hi = mid;
-            }
-            lim = lo;
+            const int cnt = thr > 0 ? __ldg(a.sep_prefix + (size_t)b * (a.T + 1) + min(thr, a.T)) : 0;
+            lim = max(0, min(lim, cnt - r0));
           }
           c_hi = lim - 1;
         }

@@ -461,14 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r0 + kTile > pl.g_full) {
           int lim = min(kTile, pl.g_count - r0);
           if (a.gather_mode == 1) {
-            const int* pos = a.sep_pos + (size_t)b * a.T + r0;
+            // separators kept by row i: pos < i - w; their count is a prefix count
             const int thr = i - a.window;
-            int lo = 0, hi = max(lim, 0);
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              if (__ldg(pos + mid) < thr) lo = mid + 1; else hi = mid;
-            }
-            lim = lo;
+            const int cnt = thr > 0 ? __ldg(a.sep_prefix + (size_t)b * (a.T + 1) + min(thr, a.T)) : 0;
+            lim = max(0, min(lim, cnt - r0));
           }
           c_hi = lim - 1;
         }

@@ -85,6 +85,7 @@ struct AttnArgs {
   int gather_mode;
   bool q2;                     // gathered tiles use the second query tile (Qc)
   const int32_t* sep_pos;      // [B, T]
+  const int32_t* sep_prefix;   // [B, T+1]: separators n_start <= j < x
   const int32_t* ranges;       // [B, nQT, 2]
   int window;                  // w for the separator rule (sep kept iff pos < i - w)
   // segmented execution

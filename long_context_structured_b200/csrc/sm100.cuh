@@ -32,6 +32,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Register split between warpgroups: every warp of a warpgroup executes the
+// same call; the block's launch allocation (threads x registers at launch)
+// must cover the sum of the warpgroups' new limits.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

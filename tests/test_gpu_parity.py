@@ -203,16 +203,32 @@ def test_deterministic():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_host_tensors_end_to_end():
-    wl = synth.Workload(name="e2e", B=1, Hq=2, Hkv=2, T=600, d=128, dtype="bf16", n_start=4, window=128,
-                        L_pretrain=128, rope_theta=1e4)
+@pytest.mark.parametrize("B,Hq,Hkv,sep", [(1, 8, 8, 0.0), (1, 8, 2, 0.1), (3, 4, 2, 0.1)])
+def test_host_tensors_end_to_end(B, Hq, Hkv, sep):
+    """The host-tensor path (pieces copied, computed and copied back on two
+    streams) gives the device path's result bit for bit."""
+    wl = synth.Workload(name="e2e", B=B, Hq=Hq, Hkv=Hkv, T=600, d=128, dtype="bf16", n_start=4, window=128,
+                        L_pretrain=0 if sep else 128, rope_theta=1e4, sep_rate=sep)
     inp = synth.make_inputs(wl, seed=9)
     Od, ld = _run_fwd(wl, inp)
     qh, kh, vh = (to_dev(inp[x], device="cpu") for x in ("q", "k", "v"))
+    sep_h = None if inp["is_sep"] is None else torch.from_numpy(inp["is_sep"])
     Oh, lh = sa.fwd(qh, kh, vh, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
-                    rope_theta=wl.rope_theta)
-    assert Oh.device.type == "cpu"
+                    rope_theta=wl.rope_theta, is_sep=sep_h)
+    assert Oh.device.type == "cpu" and Oh.is_pinned()
     assert torch.equal(Oh, Od.cpu()) and torch.equal(lh, ld.cpu())
+
+
+def test_host_tensors_segmented():
+    wl = synth.Workload(name="e2e_seg", B=1, Hq=4, Hkv=4, T=1024, d=128, dtype="bf16", rope_theta=1e4,
+                        seg_S=256, seg_M=64, seg_R=128, retr_block=32, long_heads=(1, 3))
+    inp = synth.make_inputs(wl, seed=4)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    kw = dict(S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block, is_long=list(inp["is_long"]),
+              rope_theta=wl.rope_theta)
+    Od, ld, pd = sa.segment_fwd(q, k, v, **kw)
+    Oh, lh, ph = sa.segment_fwd(q.cpu(), k.cpu(), v.cpu(), **kw)
+    assert torch.equal(Oh, Od.cpu()) and torch.equal(lh, ld.cpu()) and torch.equal(ph, pd.cpu())
 
 
 # ---------------------------------------------------------------------------
