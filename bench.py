@@ -46,9 +46,10 @@ DEFAULT_WORKLOAD = "c2"
 METRIC = "effective TFLOP/s over unmasked pairs (fraction of bf16 TC peak), tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per launch of the attention kernel on the default
-# workload, from the ncu capture summarised in profiles/; None when the kernel
-# changed since the counters were taken.
-ATTN_TRAFFIC_BYTES = None
+# workload: dram__bytes_read.sum + dram__bytes_write.sum of an ncu capture of
+# the 8-head cut (117.6 MB), times 4 for 32 heads (bytes scale with heads);
+# None when the kernel changed since the counters were taken.
+ATTN_TRAFFIC_BYTES = 470.3e6
 
 
 def log(*a):
