@@ -66,6 +66,8 @@ constexpr uint32_t kTmemCols = 512;
 // accepted sum exceeds 2^kSumRebase moves m up by a power of two before its
 // next tile, so the rescale of O and l is exact.
 constexpr float kSumAccept = 0x1p32f;
+constexpr int kMaxSideTopk = 16;  // top-k side keys per row (the library's limit on k)
+constexpr int kSinkSmem = 16;     // sink V rows staged in shared memory up to this many
 constexpr float kSumRebase = 0x1p8f;
 __device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
   uint32_t a = smem_u32(bar);
@@ -569,18 +571,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* sz = a.sink_z ? a.sink_z + row_id * a.n_sink : nullptr;
     const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
     const float* tkz = a.tk_z ? a.tk_z + row_id * a.topk : nullptr;
+    // side keys: the starting span (sinks) and the row's top-k keys, fp32
     float m_fin = m_used;
     for (int j = 0; j < n_sink; ++j) m_fin = fmaxf(m_fin, sz[j] * sl2);
-    for (int y = 0; y < a.topk; ++y)
-      if (tki[y] >= 0 && tki[y] < a.T) m_fin = fmaxf(m_fin, tkz[y] * sl2);
+    float pt[kMaxSideTopk];  // top-k weights, 0 for absent keys
+    int jt[kMaxSideTopk];
+#pragma unroll
+    for (int y = 0; y < kMaxSideTopk; ++y) {
+      jt[y] = (y < a.topk) ? tki[y] : -1;
+      if (jt[y] >= a.T) jt[y] = -1;
+      if (jt[y] >= 0) m_fin = fmaxf(m_fin, tkz[y] * sl2);
+    }
     const float alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_fin);
     float l_fin = l_sum * alpha;
     for (int j = 0; j < n_sink; ++j) l_fin += ex2_approx(sz[j] * sl2 - m_fin);
-    for (int y = 0; y < a.topk; ++y)
-      if (tki[y] >= 0 && tki[y] < a.T) l_fin += ex2_approx(tkz[y] * sl2 - m_fin);
+#pragma unroll
+    for (int y = 0; y < kMaxSideTopk; ++y) {
+      pt[y] = (jt[y] >= 0) ? ex2_approx(tkz[y] * sl2 - m_fin) : 0.f;
+      l_fin += pt[y];
+    }
     const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;
     const __nv_bfloat16* vbase = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
     __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)ir * a.o_st;
+    // The sinks' V rows are the same for every row of the tile: stage them in
+    // this warpgroup's Q tile (free once its last MMA completed).
+    const bool sinks_smem = a.n_sink > 0 && a.n_sink <= kSinkSmem;
+    const __nv_bfloat16* vsink = reinterpret_cast<const __nv_bfloat16*>(sQ + x * kTileBytes);
+    if (sinks_smem) {
+      if (k == 0 && un.n > 0) ok = ok && mbar_wait(q_full, 0, abort_flag, a.status, 47);  // its load may be in flight
+      uint4* dst = reinterpret_cast<uint4*>(sQ + x * kTileBytes);
+      for (int e = r; e < a.n_sink * (D / 8); e += 128)
+        dst[e] = *reinterpret_cast<const uint4*>(vbase + (size_t)(e / (D / 8)) * a.v_st + (e % (D / 8)) * 8);
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + x) : "memory");  // this warpgroup only
+    }
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       float ov[32];
@@ -595,24 +618,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < n_sink; ++j) {
         const float pkv = ex2_approx(sz[j] * sl2 - m_fin);
-        const __nv_bfloat16* vr = vbase + (size_t)j * a.v_st + c * 32;
+        const __nv_bfloat16* vr = sinks_smem ? vsink + j * D + c * 32 : vbase + (size_t)j * a.v_st + c * 32;
 #pragma unroll
-        for (int y = 0; y < 32; y += 2) {
-          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr + y));
-          ov[y] = fmaf(pkv, vv.x, ov[y]);
-          ov[y + 1] = fmaf(pkv, vv.y, ov[y + 1]);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 u = reinterpret_cast<const uint4*>(vr)[q4];
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 vv = __bfloat1622float2(hv[e]);
+            ov[q4 * 8 + 2 * e] = fmaf(pkv, vv.x, ov[q4 * 8 + 2 * e]);
+            ov[q4 * 8 + 2 * e + 1] = fmaf(pkv, vv.y, ov[q4 * 8 + 2 * e + 1]);
+          }
         }
       }
-      for (int t2 = 0; t2 < a.topk; ++t2) {
-        const int j = tki[t2];
-        if (j < 0 || j >= a.T) continue;
-        const float pkv = ex2_approx(tkz[t2] * sl2 - m_fin);
-        const __nv_bfloat16* vr = vbase + (size_t)j * a.v_st + c * 32;
+      // top-k rows: the 64-byte pieces of up to 4 rows are loaded before any is used
+      for (int t0 = 0; t0 < a.topk; t0 += 4) {
+        uint4 vv4[4][4];
 #pragma unroll
-        for (int y = 0; y < 32; y += 2) {
-          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr + y));
-          ov[y] = fmaf(pkv, vv.x, ov[y]);
-          ov[y + 1] = fmaf(pkv, vv.y, ov[y + 1]);
+        for (int u = 0; u < 4; ++u) {
+          int jj = -1;
+#pragma unroll
+          for (int y = 0; y < kMaxSideTopk; ++y)
+            if (y == t0 + u) jj = jt[y];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            vv4[u][q4] = (jj >= 0) ? reinterpret_cast<const uint4*>(vbase + (size_t)jj * a.v_st + c * 32)[q4]
+                                   : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float pkv = 0.f;
+#pragma unroll
+          for (int y = 0; y < kMaxSideTopk; ++y)
+            if (y == t0 + u) pkv = pt[y];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&vv4[u][q4]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 vv = __bfloat1622float2(hv[e]);
+              ov[q4 * 8 + 2 * e] = fmaf(pkv, vv.x, ov[q4 * 8 + 2 * e]);
+              ov[q4 * 8 + 2 * e + 1] = fmaf(pkv, vv.y, ov[q4 * 8 + 2 * e + 1]);
+            }
+          }
         }
       }
       if (row_ok) {

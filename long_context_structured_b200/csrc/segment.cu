@@ -89,15 +89,23 @@ __global__ void __launch_bounds__(kThreads) block_score_kernel(SegRetrArgs a, in
     }
     for (int x = threadIdx.x; x < (u1 - u0) * kQG; x += kThreads) smax[x / kQG][x % kQG] = -CUDART_INF_F;
     for (int c0 = k_begin; c0 < k_end; c0 += kChunkKeys) {
-      for (int kk = warp * KPW + lane / LPK; kk < kChunkKeys; kk += (kThreads / 32) * KPW) {
+      // every key load of this warp's share of the chunk is issued before the
+      // first dot product (kSteps 16-byte loads in flight per lane)
+      constexpr int kStep = (kThreads / 32) * KPW;  // keys per step of the whole CTA
+      constexpr int kSteps = kChunkKeys / kStep;
+      uint4 raw[kSteps];
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        const int j = c0 + u * kStep + warp * KPW + lane / LPK;
+        raw[u] = (j < k_end) ? *reinterpret_cast<const uint4*>(kb + (int64_t)j * a.k_st + sub * 8)
+                             : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        const int kk = u * kStep + warp * KPW + lane / LPK;
         const int j = c0 + kk;
         float kv[8];
-        if (j < k_end) {
-          unpack8(*reinterpret_cast<const uint4*>(kb + (int64_t)j * a.k_st + sub * 8), kv);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
-        }
+        unpack8(raw[u], kv);  // keys past the end carry zeros
         float dot[kQG];
 #pragma unroll
         for (int q = 0; q < kQG; ++q) {
@@ -106,7 +114,7 @@ __global__ void __launch_bounds__(kThreads) block_score_kernel(SegRetrArgs a, in
           for (int e = 0; e < 8; e += 2) fma2(A0, A1, qr[q][e], qr[q][e + 1], kv[e], kv[e + 1], A0, A1);
           dot[q] = A0 + A1;
         }
-        // the whole warp takes part (keys past the end carry zeros)
+        // the whole warp takes part
         group_reduce_transposed<kQG, LPK>(dot, 0xffffffffu, lane);
         constexpr int per = kQG >= LPK ? kQG / LPK : 1;
         constexpr int dup = kQG >= LPK ? 1 : LPK / kQG;
