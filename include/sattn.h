@@ -198,6 +198,18 @@ int sattn_stream_status(void* stream, const void* ws, int32_t* device_status);
 int sattn_build_blockmap_noalloc(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
                                  int32_t* sep_count, int32_t* qtile_sep_range, void* stream);
 
+/* Failure-path self-test (no counterpart on the pages).  Launches, on
+ * `stream`, one small kernel that waits -- through the same bounded mbarrier
+ * wait every kernel of the library uses -- on a barrier nothing arrives at.
+ * After limit_ns nanoseconds (1 <= limit_ns <= 2e9) the wait gives up: the
+ * kernel writes SATTN_ERR_TIMEOUT to the status word of `ws` (status[0]) and
+ * the waiting site (99) to status[1], and returns normally, so the CUDA
+ * context stays usable.  Read the result with sattn_stream_status.  The
+ * status word is cleared first.  ws: device workspace of at least 256 bytes,
+ * 256-byte aligned.  Returns SATTN_ERR_INVALID_ARG (nothing launched) for a
+ * bad workspace or limit, SATTN_ERR_CUDA if the launch failed. */
+int sattn_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
+
 /* Instrumentation (no counterpart on the pages).  While enabled, every kernel
  * launch group of the library is bracketed by CUDA events recorded on the
  * launch stream; the events cost a few hundred nanoseconds of device time

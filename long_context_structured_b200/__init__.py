@@ -27,7 +27,7 @@ from . import _lib
 from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
 
 __all__ = ["fwd", "topk_select", "build_blockmap", "segment_fwd", "stream_status", "workspace_size",
-           "segment_workspace_size", "params", "SattnError", "version", "TILE"]
+           "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout"]
 
 TILE = 128
 _ws_cache: dict = {}
@@ -226,6 +226,20 @@ def _copy_stream_pair(dev):
         st = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
         _copy_streams[dev] = st
     return st
+
+
+def selftest_wait_timeout(limit_ms: float = 20.0, device="cuda") -> tuple:
+    """Run the library's bounded-wait failure path: a kernel waits on a
+    barrier nothing arrives at and gives up after ``limit_ms``.  Returns
+    (status, site) read back from a fresh workspace's status word; the
+    expected result is (SATTN_ERR_TIMEOUT, 99) with the CUDA context intact."""
+    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    st = _stream_ptr(ws.device)
+    _lib.check(_lib.load().sattn_selftest_wait_timeout(_ptr(ws), 256, int(limit_ms * 1e6), st),
+               "sattn_selftest_wait_timeout")
+    status = stream_status(ws)
+    site = int(ws[4:8].view(torch.int32).item())
+    return status, site
 
 
 def _host_chunks(B: int, Hq: int, Hkv: int, n: int):

@@ -24,7 +24,7 @@ DTYPE_F32 = 1
 EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd", "sattn_stream_status",
-    "sattn_build_blockmap_noalloc", "sattn_profile_enable", "sattn_profile_collect",
+    "sattn_build_blockmap_noalloc", "sattn_selftest_wait_timeout", "sattn_profile_enable", "sattn_profile_collect",
 )
 
 
@@ -81,6 +81,8 @@ def load():
         L.sattn_stream_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.sattn_build_blockmap_noalloc.restype = ctypes.c_int
         L.sattn_build_blockmap_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
+        L.sattn_selftest_wait_timeout.restype = ctypes.c_int
+        L.sattn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
         L.sattn_profile_enable.restype = ctypes.c_int
         L.sattn_profile_enable.argtypes = [ctypes.c_int]
         L.sattn_profile_collect.restype = ctypes.c_int

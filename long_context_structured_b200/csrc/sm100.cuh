@@ -91,8 +91,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait on phase `parity`.  Gives up after the deadline, or as soon as
 // the CTA-wide abort flag is raised, records the failure in the device status
 // word and returns false.  Callers then skip the rest of their work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status, int where) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                int32_t* status, int where, uint64_t limit_ns) {
   uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   uint64_t t0 = globaltimer_ns();
@@ -100,13 +100,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         report_timeout(status, where);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status, int where) {
+  return mbar_wait_limit(bar, parity, abort_flag, status, where, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------
