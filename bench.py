@@ -40,6 +40,8 @@ sys.path.insert(0, ROOT)
 
 from long_context_structured_b200 import synth  # noqa: E402
 
+# decoding steps (one new token per sequence) over the caches of these workloads
+DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
 WORKLOAD_ALIASES = {"c2": "c2_lminf_16k", "c3": "c3_sepllm_gqa_8k", "c4": "c4_lminf_topk_32k",
                     "c5": "c5_segmented_32k"}
 DEFAULT_WORKLOAD = "c2"
@@ -132,8 +134,9 @@ def describe(wl) -> str:
     return s
 
 
-def config_dict(wl, pairs_per_rank):
-    c = {"workload": describe(wl), "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d}
+def config_dict(wl, pairs_per_rank, decode=False, n_copies=0):
+    c = {"workload": ("decoding step (one new token per sequence at position T-1) over the cache of " if decode
+                      else "") + describe(wl), "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d}
     if wl.segmented:
         c.update({"S": wl.seg_S, "M": wl.seg_M, "R": wl.seg_R, "retr_block": wl.retr_block,
                   "long_heads": len(wl.long_heads), "rope_theta": wl.rope_theta})
@@ -142,8 +145,12 @@ def config_dict(wl, pairs_per_rank):
                   "rope_theta": wl.rope_theta, "topk": wl.topk})
     c["unmasked_pairs_per_rank"] = pairs_per_rank
     in_bytes = (wl.B * wl.Hq + 2 * wl.B * wl.Hkv) * wl.T * wl.d * 2
-    c["l2"] = ("no flush: each step reads Q,K,V (%d MB) and writes their rotated copies, > 126 MB L2"
-               % (in_bytes >> 20))
+    if decode:
+        c["l2"] = ("no flush: steps cycle through %d copies of the K/V cache, so successive steps read "
+                   "more than the 126 MB L2 holds" % n_copies)
+    else:
+        c["l2"] = ("no flush: each step reads Q,K,V (%d MB) and writes their rotated copies, > 126 MB L2"
+                   % (in_bytes >> 20))
     return c
 
 
@@ -288,6 +295,80 @@ class Job:
         return out
 
 
+def decode_keys(wl, is_sep) -> np.ndarray:
+    """Kept keys of the last position i = T-1 per sequence (sinks, window,
+    earlier separators)."""
+    i = wl.T - 1
+    n = min(wl.n_start, wl.T) + max(0, i - max(min(wl.n_start, wl.T), i - wl.window) + 1)
+    out = np.full(wl.B, n, dtype=np.int64)
+    if is_sep is not None:
+        for b in range(wl.B):
+            f = is_sep[b].astype(np.int64).copy()
+            f[: wl.n_start] = 0
+            out[b] += int(f[: max(0, i - wl.window)].sum())
+    return out
+
+
+class DecodeJob:
+    """One decoding step per sequence over a workload's cache: the query of
+    position T-1 against the structured key set of that position.  Several
+    copies of the cache are cycled through so that successive steps read
+    more than the L2 cache holds."""
+
+    L2_BYTES = 126 * 2 ** 20
+
+    def __init__(self, wl, seed, dev):
+        import torch
+
+        import long_context_structured_b200 as sa
+        self.sa, self.torch, self.wl, self.dev = sa, torch, wl, dev
+        inp = synth.make_inputs(wl, seed=seed)
+        self.inp = inp
+        to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        q = to_t(inp["q"])[:, :, wl.T - 1:wl.T, :].contiguous()
+        self.host = {"q": q.pin_memory()}
+        keys = decode_keys(wl, inp["is_sep"])
+        self.kv_bytes = int(keys.sum()) * wl.Hkv * 2 * wl.d * 2  # kept K and V rows read per step
+        self.n_copies = int(min(8, max(1, -(-2 * self.L2_BYTES // max(self.kv_bytes, 1)))))
+        k, v = to_t(inp["k"]).to(dev), to_t(inp["v"]).to(dev)
+        self.caches = [(k, v)] + [(k.clone(), v.clone()) for _ in range(self.n_copies - 1)]
+        self.sep = None if inp["is_sep"] is None else torch.from_numpy(inp["is_sep"]).to(dev)
+        self.qd = self.host["q"].to(dev)
+        self.O = torch.empty_like(self.qd)
+        self.lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
+        self.kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta)
+        self.pairs = int(keys.sum()) * wl.Hq
+        self.flops = 4.0 * wl.d * self.pairs
+        self.n_step = 0
+
+    def step(self):
+        k, v = self.caches[self.n_step % self.n_copies]
+        self.n_step += 1
+        self.sa.decode_fwd(self.qd, k, v, is_sep=self.sep, out=self.O, lse=self.lse, **self.kw)
+
+    def host_step(self):
+        """The query from pinned host memory, the step on the device-resident
+        cache, O and LSE back to pinned host memory."""
+        torch = self.torch
+        qd = self.host["q"].to(self.dev, non_blocking=True)
+        k, v = self.caches[0]
+        O, lse = self.sa.decode_fwd(qd, k, v, is_sep=self.sep, **self.kw)
+        oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        oh.copy_(O, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream(self.dev).synchronize()
+        return oh, lh
+
+    def h2d_bytes(self):
+        return int(self.host["q"].nbytes)
+
+    def group_work(self):
+        wl = self.wl
+        q_o = 2 * wl.B * wl.Hq * wl.d * 2
+        return {"decode": ("hbm", self.kv_bytes + q_o, "B")}
+
+
 def roofline_of(group, work, avg_ms, peaks, peak_src):
     bound, amount, unit = work
     if bound == "tensor":
@@ -333,6 +414,7 @@ def kernel_name(wl, group):
     if group == "attn_tc_segment":
         return "attn_tc2_kernel<%d>" % wl.d if wl.seg_S % 256 == 0 else "attn_tc3_kernel<%d>" % wl.d
     return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel",
+            "decode": "decode_partial_kernel + decode_combine_kernel",
             "sep_gather": "sep_gather_kernel"}.get(group, group)
 
 
@@ -354,11 +436,12 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wl = synth.WORKLOADS[WORKLOAD_ALIASES.get(args.workload, args.workload)]
+    decode = args.workload in DECODE_ALIASES
+    wl = synth.WORKLOADS[(DECODE_ALIASES if decode else WORKLOAD_ALIASES).get(args.workload, args.workload)]
     if args.heads:
         wl = wl.scaled(Hq=args.heads, Hkv=max(1, args.heads * wl.Hkv // wl.Hq),
                        long_heads=tuple(h for h in wl.long_heads if h < args.heads))
-    job = Job(wl, seed=rank, dev=dev)
+    job = (DecodeJob if decode else Job)(wl, seed=rank, dev=dev)
     lib = _lib.load()
 
     for _ in range(args.warmup):
@@ -398,7 +481,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
     value = job.flops * world / (ms_step * 1e-3) / 1e12
-    tokens_s = wl.B * wl.T * world / (ms_step * 1e-3)
+    tokens_s = wl.B * (1 if decode else wl.T) * world / (ms_step * 1e-3)
 
     # per-group device time per step (every group runs once per step; a group
     # may hold more than one kernel), max over ranks (same group order on
@@ -448,12 +531,14 @@ def run_ours(args):
     e2e = {"value": round(job.flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
            "ms_per_step": round(ms_e2e, 3), "steps": n_e2e, "h2d_bytes_per_step": job.h2d_bytes(),
            "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
-           "path": "long_context_structured_b200.%s on pinned host tensors (outputs into pinned host memory)"
-                   % ("segment_fwd" if wl.segmented else "fwd")}
+           "path": ("long_context_structured_b200.decode_fwd: query from pinned host memory, device-resident cache, "
+                    "outputs into pinned host memory") if decode else
+                   ("long_context_structured_b200.%s on pinned host tensors (outputs into pinned host memory)"
+                    % ("segment_fwd" if wl.segmented else "fwd"))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, job.inp, args.cpu_rows)
+        cpu = cpu_baseline(wl, job.inp, args.cpu_rows, decode=decode)
 
     if world > 1:
         dist.barrier()
@@ -466,7 +551,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
-        "config": config_dict(wl, job.pairs),
+        "config": config_dict(wl, job.pairs, decode=decode, n_copies=getattr(job, "n_copies", 0)),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_bf16_peak": round(value / world / peak, 4),
         "roofline": roof,
@@ -521,17 +606,22 @@ def _oracle_rows(O, wl, inp, rows, nthreads):
         O.fwd_rows(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows, nthreads=nthreads)
 
 
-def cpu_baseline(wl, inp, n_rows):
+def cpu_baseline(wl, inp, n_rows, decode=False):
     from oracle import oracle as O
     O.build()
-    rows = _oracle_sample(wl, n_rows, 1234)
+    if decode:  # the decoded rows (b, h, T-1), repeated to a bounded sample
+        base = np.array([(b, h, wl.T - 1) for b in range(wl.B) for h in range(wl.Hq)], dtype=np.int64)
+        rows = np.tile(base, (max(1, n_rows // (16 * len(base))), 1))
+    else:
+        rows = _oracle_sample(wl, n_rows, 1234)
     nthreads = O.nthreads_default()
     t0 = time.perf_counter()
     _oracle_rows(O, wl, inp, rows, nthreads)
     dt = time.perf_counter() - t0
     flops = 4.0 * wl.d * _pairs_of_rows(wl, rows, inp["is_sep"])
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
-            "sample": "%d seeded rows (b, h, i) of the same workload, all heads, fp64, %.1f s" % (n_rows, dt),
+            "sample": "%d %s rows (b, h, i) of the same workload, all heads, fp64, %.1f s" % (
+                len(rows), "decoded" if decode else "seeded", dt),
             "seconds": round(dt, 2)}
 
 
@@ -541,15 +631,18 @@ def run_reference(args):
         return
     from oracle import oracle as O
     O.build()
-    wl = synth.WORKLOADS[WORKLOAD_ALIASES.get(args.workload, args.workload)]
+    decode = args.workload in DECODE_ALIASES
+    wl = synth.WORKLOADS[(DECODE_ALIASES if decode else WORKLOAD_ALIASES).get(args.workload, args.workload)]
     inp = synth.make_inputs(wl, seed=0)
     nthreads = O.nthreads_default()
     rows_per_step = args.ref_rows
 
     def step(s):
-        # one head per step, rows spread over positions
-        rows = _oracle_sample(wl, rows_per_step, 100 + s)
-        rows[:, 1] = s % wl.Hq
+        if decode:  # the decoded row of every sequence, one head per step
+            rows = np.array([(b, s % wl.Hq, wl.T - 1) for b in range(wl.B)], dtype=np.int64)
+        else:  # one head per step, rows spread over positions
+            rows = _oracle_sample(wl, rows_per_step, 100 + s)
+            rows[:, 1] = s % wl.Hq
         _oracle_rows(O, wl, inp, rows, nthreads)
         return _pairs_of_rows(wl, rows, inp["is_sep"])
 
@@ -566,7 +659,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
-        "config": config_dict(wl, unmasked_pairs(wl, inp["is_sep"])),
+        "config": config_dict(wl, int(decode_keys(wl, inp["is_sep"]).sum()) * wl.Hq if decode
+                              else unmasked_pairs(wl, inp["is_sep"]), decode=decode),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                          "sample": "each step: %d seeded rows of one head (heads cycle), fp64 C oracle"
                                    % rows_per_step},
@@ -582,7 +676,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()))
+                    choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -174,6 +174,30 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
                       const uint8_t* is_long, const void* Q, const void* K, const void* V, void* O, float* lse,
                       int32_t* prefix_blocks, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace needed by sattn_decode_fwd for *p (p->T = cache length). */
+int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
+
+/* One decoding step: the query of the newest token, at position i = T-1,
+ * attends over the structured key set of that position among the cache's
+ * T entries (its own key and value are the last entry).  The key set and the
+ * logits are those of sattn_fwd's row i: starting span j < n_start and
+ * window i-w <= j <= i ("LM-Infinite", section 方法), earlier separators
+ * n_start <= j < i-w ("SepLLM", section 五.2), the capped logit
+ * <R(L) q, k_j> for i-j > L_pretrain and <R(i) q, R(j) k_j> otherwise.
+ *   p        shape and mask parameters; T is the cache length, topk must be
+ *            0, Hq/Hkv one of 1, 2, 4, 8, bf16 only.
+ *   Q        [B, Hq, 1, d] bf16 device, strides q_stride[0..1].
+ *   K, V     [B, Hkv, T, d] bf16 device cache (keys unrotated), strides as
+ *            in sattn_fwd.
+ *   is_sep   [B, T] uint8 device flags or NULL (needs p->with_separators).
+ *   O        [B, Hq, 1, d] bf16 device, out, strides o_stride[0..1].
+ *   lse      [B, Hq] fp32 device, out (natural log).
+ * Reads each kept key and value row once (split over chunks of 128 kept keys,
+ * the query heads of a kv-head group together, then a merge of the chunks).
+ * Asynchronous on `stream`; validation as sattn_fwd. */
+int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                     void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and reads the device status word of `ws` into
  * *device_status (SATTN_OK or SATTN_ERR_TIMEOUT).  Returns SATTN_ERR_CUDA if
  * the synchronisation itself failed (the CUDA error is then sticky). */

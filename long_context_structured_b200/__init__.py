@@ -27,7 +27,8 @@ from . import _lib
 from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
 
 __all__ = ["fwd", "topk_select", "build_blockmap", "segment_fwd", "stream_status", "workspace_size",
-           "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout"]
+           "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout",
+           "decode_fwd"]
 
 TILE = 128
 _ws_cache: dict = {}
@@ -201,6 +202,36 @@ def segment_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, S: int, M:
                                        _ptr(lse), _ptr(prefix), _ptr(ws), nbytes, _stream_ptr(q.device))
     _lib.check(rc, "sattn_segment_fwd")
     return out, lse, prefix[..., :nb]
+
+
+def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, window: int = 0,
+               L_pretrain: int = 0, rope_theta: float = 0.0, is_sep: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None):
+    """One decoding step: q [B, Hq, 1, d] is the query of the cache's last
+    position (k, v [B, Hkv, T, d]).  Returns (O [B, Hq, 1, d], lse [B, Hq])."""
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode_fwd takes one query per (batch, head): q is [B, Hq, 1, d]")
+    T = k.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, 1, d), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    p = params(q, k, v, out, n_start=n_start, window=window, L_pretrain=L_pretrain, rope_theta=rope_theta,
+               with_separators=is_sep is not None)
+    p.T = T
+    n = ctypes.c_size_t(0)
+    L = _lib.load()
+    _lib.check(L.sattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)), "sattn_decode_workspace_size")
+    nbytes = int(n.value)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = L.sattn_decode_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(out), _ptr(lse),
+                            _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_decode_fwd")
+    return out, lse
 
 
 def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> int:

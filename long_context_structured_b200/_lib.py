@@ -23,7 +23,8 @@ DTYPE_F32 = 1
 # every function the header declares, in header order
 EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
-    "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd", "sattn_stream_status",
+    "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
+    "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_stream_status",
     "sattn_build_blockmap_noalloc", "sattn_selftest_wait_timeout", "sattn_profile_enable", "sattn_profile_collect",
 )
 
@@ -77,6 +78,10 @@ def load():
         L.sattn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sattn_segment_fwd.restype = ctypes.c_int
         L.sattn_segment_fwd.argtypes = [P, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sattn_decode_workspace_size.restype = ctypes.c_int
+        L.sattn_decode_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.sattn_decode_fwd.restype = ctypes.c_int
+        L.sattn_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sattn_stream_status.restype = ctypes.c_int
         L.sattn_stream_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.sattn_build_blockmap_noalloc.restype = ctypes.c_int

@@ -763,6 +763,109 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
   return cuda_rc((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc3(a, m, st));
 }
 
+// ---------------------------------------------------------------------------
+// decoding step
+// ---------------------------------------------------------------------------
+
+struct DecPlan {
+  int nQT, npos, n_chunks;
+  Region status, tab, prefix, sep_pos, sep_count, ranges, part;
+  size_t total;
+};
+
+static int plan_decode(const sattn_params* p, DecPlan* out) {
+  int rc = check_common(p);
+  if (rc) return rc;
+  if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
+  if (p->topk != 0) return SATTN_ERR_UNSUPPORTED;
+  const int rep = p->Hq / p->Hkv;
+  if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return SATTN_ERR_UNSUPPORTED;
+  if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
+  DecPlan P;
+  P.nQT = (p->T + kTile - 1) / kTile;
+  P.npos = std::max(p->T, p->L_pretrain + 1);
+  P.n_chunks = decode_chunks(p->T);
+  const size_t B = p->B, Hq = p->Hq, T = p->T, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  if (p->with_separators) {
+    P.prefix = A.take(B * (T + 1) * 4);
+    P.sep_pos = A.take(B * T * 4);
+    P.sep_count = A.take(B * 4);
+    P.ranges = A.take(B * P.nQT * 2 * 4);
+  }
+  P.part = A.take(B * Hq * (size_t)P.n_chunks * (d + 2) * 4);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  DecPlan P;
+  int rc = plan_decode(p, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                     void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  DecPlan P;
+  int rc = plan_decode(p, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse) return SATTN_ERR_INVALID_ARG;
+  if (is_sep && !p->with_separators) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+  }
+  if (is_sep) {
+    FwdPlan F;
+    F.prefix = P.prefix;
+    rc = run_blockmap(p, F, is_sep, nullptr, at<int32_t>(ws, P.sep_pos), at<int32_t>(ws, P.sep_count),
+                      at<int32_t>(ws, P.ranges), ws, st);
+    if (rc) return rc;
+  }
+  DecodeArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.L = p->L_pretrain;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  a.sep_prefix = is_sep ? at<int32_t>(ws, P.prefix) : nullptr;
+  a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
+  a.part = at<float>(ws, P.part);
+  a.n_chunks = P.n_chunks;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.lse = lse;
+  ProfScope ps("decode", 2, st);
+  return cuda_rc(launch_decode(a, st));
+}
+
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {
   if (!ws || !device_status) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

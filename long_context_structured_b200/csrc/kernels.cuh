@@ -189,4 +189,30 @@ size_t segment_score_bytes(int B, int n_long, int N, int T, int blk);
 bool segment_retrieval_supported(int T, int S, int blk);
 cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st);
 
+// ---------------------------------------------------------------------------
+// decoding step: one query per (batch, head) at position T - 1
+// ---------------------------------------------------------------------------
+struct DecodeArgs {
+  int B, Hq, Hkv, T, d;
+  int n_start, window, L;
+  float scale_log2;
+  const __nv_bfloat16* Q;  // [B, Hq, 1, d]
+  int64_t q_sb, q_sh;
+  const __nv_bfloat16* K;  // [B, Hkv, T, d] cache, unrotated
+  int64_t k_sb, k_sh, k_st;
+  const __nv_bfloat16* V;
+  int64_t v_sb, v_sh, v_st;
+  const float2* tab;            // rotary table or null
+  const int32_t* sep_prefix;    // [B, T+1] or null (no separators)
+  const int32_t* sep_pos;       // [B, T]
+  float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
+  int n_chunks;
+  __nv_bfloat16* O;             // [B, Hq, 1, d]
+  int64_t o_sb, o_sh;
+  float* lse;                   // [B, Hq]
+};
+// chunks of kept keys a decoding step of cache length T may need
+int decode_chunks(int T);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
 }  // namespace sattn

@@ -69,3 +69,15 @@ def test_full_workload_counts():
 def test_workload_aliases_resolve():
     for short, full in bench.WORKLOAD_ALIASES.items():
         assert full in synth.WORKLOADS, short
+
+
+def test_decode_key_counts_match_oracle(oracle_mod):
+    """Kept keys of the decoded position per sequence equal the oracle's mask
+    counts of row T-1."""
+    O = oracle_mod
+    for wl in SMALL[:3]:
+        inp = synth.make_inputs(wl, seed=4)
+        rows = np.array([(b, 0, wl.T - 1) for b in range(wl.B)], dtype=np.int64)
+        *_, cnt = O.fwd_rows(O.params_of(wl.scaled(topk=0)), inp["q"], inp["k"], inp["v"], inp["is_sep"], rows,
+                             nthreads=2)
+        assert list(bench.decode_keys(wl, inp["is_sep"])) == list(cnt)

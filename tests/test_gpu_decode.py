@@ -1,0 +1,103 @@
+"""GPU parity of the decoding step against the fp64 oracle.
+
+A decoding step is row i = T-1 of the structured attention: the oracle's
+row (b, h, T-1), computed from the materialised 0/1 mask, is the reference.
+Bars as for the bf16 prefill: max-abs 2e-2, mean-abs 2e-3 on O and LSE.
+"""
+import numpy as np
+import pytest
+import torch
+
+import long_context_structured_b200 as sa
+from long_context_structured_b200 import _lib, synth
+from _util import BF16_MAX_ABS, BF16_MEAN_ABS, compare, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def _decode_and_check(oracle_mod, wl, seed):
+    inp = synth.make_inputs(wl, seed=seed)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    qd = q[:, :, wl.T - 1:wl.T, :].contiguous()
+    O, lse = sa.decode_fwd(qd, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                           rope_theta=wl.rope_theta, is_sep=sep)
+    torch.cuda.synchronize()
+    assert sa.stream_status() == 0
+    rows = np.array([(b, h, wl.T - 1) for b in range(wl.B) for h in range(wl.Hq)], dtype=np.int64)
+    Oref, lref, *_ = oracle_mod.fwd_rows(oracle_mod.params_of(wl), inp["q"], inp["k"], inp["v"], inp["is_sep"],
+                                         rows)
+    got = O[:, :, 0, :].reshape(-1, wl.d).float().cpu().numpy().astype(np.float64)
+    gl = lse.reshape(-1).float().cpu().numpy().astype(np.float64)
+    compare("O", got, Oref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare("LSE", gl, lref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    return O, lse
+
+
+CASES = [
+    ("lambda_capped_sinks", dict(B=2, Hq=4, Hkv=4, T=1000, d=128, n_start=4, window=100, L_pretrain=100,
+                                 rope_theta=1e4, sink_scale=8.0)),
+    ("sep_gqa4_d64", dict(B=3, Hq=8, Hkv=2, T=777, d=64, n_start=4, window=37, rope_theta=5e5, sep_rate=0.1)),
+    ("sep_capped_gqa8", dict(B=1, Hq=8, Hkv=1, T=600, d=128, n_start=2, window=50, L_pretrain=50,
+                             rope_theta=1e4, sep_rate=0.3)),
+    ("full_causal_no_rope", dict(B=1, Hq=2, Hkv=2, T=300, d=128, n_start=0, window=1000)),
+    ("all_sinks", dict(B=1, Hq=2, Hkv=1, T=3, d=128, n_start=8, window=1, rope_theta=1e4)),
+    ("window0_all_seps", dict(B=1, Hq=2, Hkv=2, T=257, d=128, n_start=1, window=0, sep_rate=1.0)),
+    ("one_token", dict(B=2, Hq=2, Hkv=2, T=1, d=64, n_start=0, window=4, rope_theta=1e4)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", CASES, ids=[c[0] for c in CASES])
+def test_decode_matches_oracle(oracle_mod, name, cfg):
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    _decode_and_check(oracle_mod, wl, seed=13)
+
+
+def test_decode_full_size_lambda(oracle_mod):
+    """The 16K-token LM-Infinite layer's last position (32 heads)."""
+    _decode_and_check(oracle_mod, synth.WORKLOADS["c2_lminf_16k"], seed=0)
+
+
+def test_decode_full_size_sepllm_gqa(oracle_mod):
+    """The SepLLM GQA layer's last positions (4 sequences, 32 query heads)."""
+    _decode_and_check(oracle_mod, synth.WORKLOADS["c3_sepllm_gqa_8k"], seed=0)
+
+
+def test_decode_deterministic_and_invariant_outside_kept_set():
+    wl = synth.Workload(name="inv", B=1, Hq=4, Hkv=2, T=900, d=128, dtype="bf16", n_start=4, window=64,
+                        L_pretrain=64, rope_theta=1e4, sep_rate=0.1)
+    inp = synth.make_inputs(wl, seed=3)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta, is_sep=sep)
+    qd = q[:, :, -1:, :].contiguous()
+    O1, l1 = sa.decode_fwd(qd, k, v, **kw)
+    O2, l2 = sa.decode_fwd(qd, k, v, **kw)
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    # change K and V at positions the last row does not keep
+    i = wl.T - 1
+    flags = inp["is_sep"][0]
+    kept = np.zeros(wl.T, dtype=bool)
+    kept[: wl.n_start] = True
+    kept[max(0, i - wl.window):] = True
+    kept |= (flags != 0) & (np.arange(wl.T) < i - wl.window) & (np.arange(wl.T) >= wl.n_start)
+    drop = torch.from_numpy(np.nonzero(~kept)[0]).cuda()
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, drop] = 3.0
+    v2[:, :, drop] = -7.0
+    O3, l3 = sa.decode_fwd(qd, k2, v2, **kw)
+    assert torch.equal(O1, O3) and torch.equal(l1, l3)
+
+
+def test_decode_rejects_unsupported():
+    q = torch.zeros((1, 3, 1, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 10, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.SattnError):
+        sa.decode_fwd(q, k, k)  # Hq / Hkv = 3
