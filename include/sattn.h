@@ -85,6 +85,8 @@ typedef struct sattn_params {
   int32_t with_separators; /* nonzero: is_sep may be passed; the workspace then holds the
                               separator compaction and gathered K/V (worst case: every token) */
   double rope_theta;  /* rotary base; 0 = no rotation */
+  double rope_pos_scale; /* position interpolation: rotary positions are multiplied by this
+                            before rotation (distances too); 0 or 1 = none; (0, 1] */
 } sattn_params;
 
 /* Text of a status code (static storage). */

@@ -63,6 +63,7 @@ int check_common(const sattn_params* p) {
   if (p->n_start < 0 || p->window < 0 || p->L_pretrain < 0 || p->topk < 0) return SATTN_ERR_INVALID_ARG;
   if (p->topk > 16) return SATTN_ERR_UNSUPPORTED;
   if (!(p->rope_theta >= 0.0) || !std::isfinite(p->rope_theta)) return SATTN_ERR_INVALID_ARG;
+  if (!(p->rope_pos_scale >= 0.0) || p->rope_pos_scale > 1.0) return SATTN_ERR_INVALID_ARG;
   if ((int64_t)p->B * p->Hq * p->T > (int64_t)1 << 31) return SATTN_ERR_UNSUPPORTED;
   const int64_t* st[4] = {p->q_stride, p->k_stride, p->v_stride, p->o_stride};
   const int esz = p->dtype == SATTN_DTYPE_BF16 ? 2 : 4;
@@ -186,6 +187,9 @@ bool make_map(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t n2,
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA; }
 
+// rotary position scale (position interpolation); 0 means none
+double pos_scale(const sattn_params* p) { return p->rope_pos_scale > 0.0 ? p->rope_pos_scale : 1.0; }
+
 // ---------------------------------------------------------------------------
 // optional event instrumentation of launch groups
 // ---------------------------------------------------------------------------
@@ -251,7 +255,7 @@ int run_prep_bf16(const sattn_params* p, const FwdPlan& P, const void* Q, const 
                   bool with_kmax, cudaStream_t st) {
   if (P.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
-    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
   }
   if (with_kmax && P.kmax.bytes) SATTN_TRY(cudaMemsetAsync(at<uint8_t>(ws, P.kmax), 0, P.kmax.bytes, st));
   PrepArgs a{};
@@ -339,7 +343,7 @@ int run_topk(const sattn_params* p, const FwdPlan& P, const void* Q, const void*
              int32_t* idx, float* z, void* ws, cudaStream_t st) {
   TopkArgs a = topk_args(p, P, Q, K, is_sep, idx, z, ws);
   if (!P.bf16) {
-    if (P.tab.bytes) SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+    if (P.tab.bytes) SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
     ProfScope ps("topk_exact", 1, st);
     return cuda_rc(launch_topk_exact(a, true, st));
   }
@@ -450,7 +454,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
     // ---------------- fp32 path ----------------
     if (P.tab.bytes) {
       ProfScope ps("rope_table", 1, st);
-      SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+      SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
     }
     if (is_sep) {
       rc = run_blockmap(p, P, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
@@ -823,7 +827,7 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
   if (P.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
-    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, st));
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
   }
   if (is_sep) {
     FwdPlan F;

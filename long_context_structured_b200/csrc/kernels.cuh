@@ -14,8 +14,9 @@ constexpr int kMaxHeads = 256;
 // ---------------------------------------------------------------------------
 // K1: rotary table and the prep pass
 // ---------------------------------------------------------------------------
-// tab[p][c] = (cos, sin)(p * theta^(-2c/d)), computed in fp64, stored fp32.
-cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, cudaStream_t st);
+// tab[p][c] = (cos, sin)(p * scale * theta^(-2c/d)), computed in fp64, stored
+// fp32; scale < 1 is position interpolation.
+cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, double scale, cudaStream_t st);
 
 struct PrepArgs {
   int B, Hq, Hkv, T, d;

@@ -1,7 +1,7 @@
 // prep.cu -- K1: rotary table and the elementwise prep pass.
 //
 // Rotary convention: rotate-half; pair (c, c + d/2) turns by the angle
-// p * theta^(-2c/d).  The capped logit ("LM-Infinite", section 方法, RoPE
+// p * s * theta^(-2c/d), s the position-interpolation scale (1 = none).  The capped logit ("LM-Infinite", section 方法, RoPE
 // realisation of d'_ij = min(d_ij, L)) needs, besides R(i) q_i and R(j) k_j,
 // the query rotated to the cap, R(L) q_i, paired with the unrotated key.
 //
@@ -37,7 +37,7 @@ constexpr int kU = 2;  // rows per thread whose loads are in flight together
 constexpr int kMaxSmemSinks = 16;
 constexpr int kPairsPerThread = 8;
 
-__global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double theta) {
+__global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double theta, double scale) {
   __shared__ double inv_freq[128];
   for (int c = threadIdx.x; c < half; c += blockDim.x) inv_freq[c] = pow(theta, -2.0 * (double)c / (double)d);
   __syncthreads();
@@ -46,7 +46,7 @@ __global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double
     const int p = (int)(x / half);
     const int c = (int)(x % half);
     double s, co;
-    sincos((double)p * inv_freq[c], &s, &co);
+    sincos((double)p * scale * inv_freq[c], &s, &co);
     tab[x] = make_float2((float)co, (float)s);
   }
 }
@@ -308,13 +308,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
 
 }  // namespace
 
-cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, cudaStream_t st) {
+cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, double scale, cudaStream_t st) {
   const int half = d / 2;
   const int64_t n = (int64_t)npos * half;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
-  rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(tab, npos, half, d, theta);
+  rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(tab, npos, half, d, theta, scale);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ class Workload:
     window: int = 0
     L_pretrain: int = 0        # 0 disables the distance cap
     rope_theta: float = 0.0    # 0 disables RoPE
+    rope_pos_scale: float = 1.0  # position interpolation: rotary positions multiplied by this
     topk: int = 0
     sep_rate: float = 0.0      # Bernoulli flag rate (c1-style) ...
     sep_vocab: int = 0         # ... or token-id derived flags (c3-style) when > 0

@@ -43,7 +43,11 @@
  *       out, the k largest unscaled logits; ties go to the smaller j;
  *       fewer than k candidates -> all of them, padded with -1 / -inf;
  *   R7  rotary convention: rotate-half, inv_freq_c = theta^(-2c/d), angle
- *       pos*inv_freq_c; theta == 0 means no rotation; positions 0..T-1;
+ *       pos*s*inv_freq_c; theta == 0 means no rotation; positions 0..T-1;
+ *       s is the position-interpolation scale (the talk page, section on
+ *       position interpolation: every position is squeezed by one constant
+ *       factor so that extended positions stay in the pretraining range);
+ *       s = 1 unless given; distances, the cap L included, scale alike;
  *   R8  GQA: query head h uses key/value head floor(h*Hkv/Hq);
  *   R9  segmented: local heads see tail+segment, long heads prefix+segment;
  *   R10 retrieval: block score = max over a block of the unrotated
@@ -69,7 +73,13 @@ typedef struct oracle_params {
   int32_t dtype; /* 0: inputs are bf16 bit patterns (uint16); 1: float32 */
   int32_t n_start, window, L_pretrain, topk;
   double rope_theta;
+  double rope_pos_scale; /* position interpolation scale s (R7); 0 means 1 */
 } oracle_params;
+
+/* rotary position of token position `pos` (R7) */
+static double rot_pos(const oracle_params* p, double pos) {
+  return pos * (p->rope_pos_scale > 0.0 ? p->rope_pos_scale : 1.0);
+}
 
 /* ------------------------------------------------------------------ */
 /* exact input decoding                                                */
@@ -211,8 +221,8 @@ static int attn_row(const head_ctx* hc, const double* qraw, int i, const int32_t
   int T = p->T, d = p->d, L = p->L_pretrain;
   double* q_i = work;
   double* q_L = work + d;
-  oracle_rope(qraw, d, (double)i, p->rope_theta, q_i);
-  oracle_rope(qraw, d, (double)(L > 0 ? L : 0), p->rope_theta, q_L);
+  oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
+  oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
 
   int64_t cnt = oracle_mask_row(T, i, p->n_start, p->window, hc->sep, m);
 
@@ -327,7 +337,7 @@ static int load_head(const oracle_params* p, const void* K, const void* V, int b
       Kraw[(size_t)j * d + c] = load_elem(K, p->dtype, base + (int64_t)j * d + c);
       Vd[(size_t)j * d + c] = load_elem(V, p->dtype, base + (int64_t)j * d + c);
     }
-    oracle_rope(Kraw + (size_t)j * d, d, (double)j, p->rope_theta, Krot + (size_t)j * d);
+    oracle_rope(Kraw + (size_t)j * d, d, rot_pos(p, (double)j), p->rope_theta, Krot + (size_t)j * d);
   }
   return OR_OK;
 }
@@ -629,12 +639,12 @@ static void seg_one(void* a, int64_t t) {
   int P = 0;
   int n = segment_key_list(J->Q, p, J->Kraw, J->S, J->M, J->R, J->blk, J->is_long, b, h, i, kj, kp, &P,
                            blocks, qlast);
-  oracle_rope(q, d, (double)(P + tt), p->rope_theta, qrot);
+  oracle_rope(q, d, rot_pos(p, (double)(P + tt)), p->rope_theta, qrot);
   double inv_sqrt_d = 1.0 / sqrt((double)d);
   double* sbuf = (double*)malloc(sizeof(double) * (size_t)(n + 1));
   double mx = -INFINITY;
   for (int x = 0; x < n; ++x) {
-    oracle_rope(J->Kraw + (size_t)kj[x] * d, d, (double)kp[x], p->rope_theta, krot);
+    oracle_rope(J->Kraw + (size_t)kj[x] * d, d, rot_pos(p, (double)kp[x]), p->rope_theta, krot);
     sbuf[x] = dot(qrot, krot, d) * inv_sqrt_d;
     if (sbuf[x] > mx) mx = sbuf[x];
   }

@@ -32,7 +32,7 @@ def _run_fwd(wl, inp, **kw):
     q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
     sep = to_dev(inp["is_sep"])
     O, lse = sa.fwd(q, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
-                    rope_theta=wl.rope_theta, topk=wl.topk, is_sep=sep, **kw)
+                    rope_theta=wl.rope_theta, topk=wl.topk, is_sep=sep, rope_pos_scale=wl.rope_pos_scale, **kw)
     torch.cuda.synchronize()
     _status_ok()
     return O, lse
@@ -121,6 +121,10 @@ SMALL = [
     ("all_sinks", dict(B=1, Hq=1, Hkv=1, T=3, d=128, n_start=8, window=1)),
     ("window_uncapped_long", dict(B=1, Hq=1, Hkv=1, T=900, d=128, n_start=4, window=200, L_pretrain=300,
                                   rope_theta=1e4)),
+    ("pos_interp_capped_sinks", dict(B=1, Hq=2, Hkv=2, T=1000, d=128, n_start=4, window=100, L_pretrain=100,
+                                     rope_theta=1e4, sink_scale=8.0, rope_pos_scale=0.25)),
+    ("pos_interp_sep_gqa", dict(B=2, Hq=4, Hkv=2, T=700, d=64, n_start=2, window=40, rope_theta=5e5,
+                                sep_rate=0.15, rope_pos_scale=0.5)),
 ]
 
 
@@ -275,7 +279,8 @@ def test_c5_segmented_full_size(oracle_mod):
     inp = synth.make_inputs(wl, seed=0)
     q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
     O, lse, pb = sa.segment_fwd(q, k, v, S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
-                                is_long=inp["is_long"], rope_theta=wl.rope_theta)
+                                is_long=inp["is_long"], rope_theta=wl.rope_theta,
+                                rope_pos_scale=wl.rope_pos_scale)
     torch.cuda.synchronize()
     _status_ok()
     p = oracle_mod.params_of(wl)
@@ -297,15 +302,18 @@ def test_c5_segmented_full_size(oracle_mod):
     dict(T=1024, S=256, M=64, R=128, blk=64, long=(0, 1)),
     dict(T=768, S=256, M=300, R=256, blk=32, long=(1, 1)),
     dict(T=512, S=128, M=0, R=0, blk=16, long=(0, 1)),
+    dict(T=1024, S=256, M=64, R=128, blk=64, long=(1, 0), pos_scale=0.25),
 ])
 def test_segmented_small_all_rows(oracle_mod, cfg):
     wl = synth.Workload(name="seg", B=1, Hq=2, Hkv=2, T=cfg["T"], d=128, dtype="bf16", rope_theta=1e4,
                         seg_S=cfg["S"], seg_M=cfg["M"], seg_R=cfg["R"], retr_block=cfg["blk"],
-                        long_heads=tuple(h for h in range(2) if cfg["long"][h]))
+                        long_heads=tuple(h for h in range(2) if cfg["long"][h]),
+                        rope_pos_scale=cfg.get("pos_scale", 1.0))
     inp = synth.make_inputs(wl, seed=12)
     q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
     O, lse, pb = sa.segment_fwd(q, k, v, S=wl.seg_S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
-                                is_long=inp["is_long"], rope_theta=wl.rope_theta)
+                                is_long=inp["is_long"], rope_theta=wl.rope_theta,
+                                rope_pos_scale=wl.rope_pos_scale)
     torch.cuda.synchronize()
     _status_ok()
     p = oracle_mod.params_of(wl)

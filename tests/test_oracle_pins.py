@@ -552,3 +552,52 @@ def test_segment_retrieval_ties_go_to_lower_block(oracle_mod):
     got, _ = oracle_mod.segment_blocks(p, S, R, blk, np.array([1], np.uint8), q, k)
     assert list(got[0, 0, 1]) == [0, 1]
     assert list(got[0, 0, 2]) == [0, 1]
+
+
+# ----------------------------------------------------------------------------
+# position interpolation (rotary positions squeezed by one constant factor)
+# ----------------------------------------------------------------------------
+
+def test_position_interpolation_equals_spread_sequence(oracle_mod):
+    """Position interpolation with scale 1/4 on a sequence whose real tokens
+    sit at positions 4j equals plain RoPE attention on the dense sequence:
+    a row 4i that keeps exactly the keys 4j (j <= i) -- SepLLM mask with
+    window 0 and separators at 4j -- sees rotary positions i and j.  Both
+    sides come from the oracle with different masks and scales, so a scale
+    applied to only one operand, twice, or to the frequency instead of the
+    position fails."""
+    B, H, T, d, s = 1, 2, 24, 16, 4
+    theta = 1e4
+    q, k, v = _rand_inputs(B, H, H, T, d, 21)
+    # dense sequence: plain causal attention with rotation
+    pd = oracle_mod.params(B, H, H, T, d, "bf16", 0, T, 0, 0, theta)
+    Od, ld, *_ = oracle_mod.fwd_rows(pd, q, k, v, None, oracle_mod.all_rows(B, H, T))
+    # spread sequence: token j at position s*j, filler elsewhere
+    g = np.random.default_rng(5)
+    Ts = s * T
+    qs = g.integers(0, 2 ** 16, (B, H, Ts, d)).astype(np.uint16) & np.uint16(0x3fff)  # finite bf16 fillers
+    ks = g.integers(0, 2 ** 16, (B, H, Ts, d)).astype(np.uint16) & np.uint16(0x3fff)
+    vs = g.integers(0, 2 ** 16, (B, H, Ts, d)).astype(np.uint16) & np.uint16(0x3fff)
+    qs[:, :, ::s], ks[:, :, ::s], vs[:, :, ::s] = q, k, v
+    sep = np.zeros((B, Ts), dtype=np.uint8)
+    sep[:, ::s] = 1
+    ps = oracle_mod.params(B, H, H, Ts, d, "bf16", 0, 0, 0, 0, theta, 1.0 / s)
+    rows = np.array([(0, h, s * i) for h in range(H) for i in range(T)], dtype=np.int64)
+    Os, ls, *_ = oracle_mod.fwd_rows(ps, qs, ks, vs, sep, rows)
+    dense_rows = np.array([(0, h, i) for h in range(H) for i in range(T)], dtype=np.int64)
+    Od2, ld2, *_ = oracle_mod.fwd_rows(pd, q, k, v, None, dense_rows)
+    assert np.abs(Os - Od2).max() < 1e-12
+    assert np.abs(ls - ld2).max() < 1e-12
+    # and the interpolated rotation is not the plain one
+    p1 = oracle_mod.params(B, H, H, Ts, d, "bf16", 0, 0, 0, 0, theta)
+    O1, *_ = oracle_mod.fwd_rows(p1, qs, ks, vs, sep, rows)
+    assert np.abs(O1 - Od2).max() > 1e-3
+
+
+def test_position_scale_one_is_identity(oracle_mod):
+    B, H, T, d = 1, 2, 50, 16
+    q, k, v = _rand_inputs(B, H, H, T, d, 22)
+    rows = oracle_mod.all_rows(B, H, T)
+    a = oracle_mod.fwd_rows(oracle_mod.params(B, H, H, T, d, "bf16", 4, 9, 9, 0, 1e4), q, k, v, None, rows)
+    b = oracle_mod.fwd_rows(oracle_mod.params(B, H, H, T, d, "bf16", 4, 9, 9, 0, 1e4, 1.0), q, k, v, None, rows)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
