@@ -87,6 +87,13 @@ typedef struct sattn_params {
   double rope_theta;  /* rotary base; 0 = no rotation */
   double rope_pos_scale; /* position interpolation: rotary positions are multiplied by this
                             before rotation (distances too); 0 or 1 = none; (0, 1] */
+  int32_t alibi;      /* nonzero: ALiBi bias instead of rotation (rope_theta must be 0):
+                         s_ij = q.k/sqrt(d) - m_h * min(i-j, L_pretrain) (no clip when
+                         L_pretrain == 0), head slopes m_h = 2^(-8 (h+1) / Hq)
+                         ("LM-Infinite", section 方法: the bias clipped at the same cap).
+                         SATTN_ERR_UNSUPPORTED: with top-k unless L_pretrain > 0 and
+                         window >= L_pretrain; with separators on the bf16 path unless
+                         L_pretrain > 0; in sattn_segment_fwd */
 } sattn_params;
 
 /* Text of a status code (static storage). */

@@ -63,7 +63,7 @@ def _strides(t: Optional[torch.Tensor]):
 
 
 def params(q, k, v=None, o=None, *, n_start=0, window=0, L_pretrain=0, topk=0, rope_theta=0.0,
-           with_separators=False, rope_pos_scale=1.0) -> SattnParams:
+           with_separators=False, rope_pos_scale=1.0, alibi=False) -> SattnParams:
     B, Hq, T, d = q.shape
     Hkv = k.shape[1]
     p = SattnParams()
@@ -77,6 +77,7 @@ def params(q, k, v=None, o=None, *, n_start=0, window=0, L_pretrain=0, topk=0, r
     p.with_separators = 1 if with_separators else 0
     p.rope_theta = float(rope_theta)
     p.rope_pos_scale = float(rope_pos_scale)
+    p.alibi = 1 if alibi else 0
     return p
 
 
@@ -118,14 +119,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, 
         L_pretrain: int = 0, rope_theta: float = 0.0, topk: int = 0, is_sep: Optional[torch.Tensor] = None,
         topk_idx: Optional[torch.Tensor] = None, topk_logit: Optional[torch.Tensor] = None,
         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-        workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0):
+        workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
     """Structured-mask attention forward.  Returns (O [B,Hq,T,d], lse [B,Hq,T] fp32).
-    rope_pos_scale < 1 is position interpolation (rotary positions scaled)."""
+    rope_pos_scale < 1 is position interpolation (rotary positions scaled);
+    alibi adds the (clipped) ALiBi bias instead of rotating (rope_theta = 0)."""
     if not q.is_cuda:
         return _host_call(fwd, (q, k, v), dict(n_start=n_start, window=window, L_pretrain=L_pretrain,
                                                rope_theta=rope_theta, topk=topk, is_sep=is_sep,
                                                topk_idx=topk_idx, topk_logit=topk_logit,
-                                               rope_pos_scale=rope_pos_scale))
+                                               rope_pos_scale=rope_pos_scale, alibi=alibi))
     B, Hq, T, d = q.shape
     if out is None:
         out = torch.empty((B, Hq, T, d), dtype=q.dtype, device=q.device)
@@ -134,7 +136,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, 
     if is_sep is not None:
         is_sep = is_sep.to(torch.uint8).contiguous()
     p = params(q, k, v, out, n_start=n_start, window=window, L_pretrain=L_pretrain, topk=topk,
-               rope_theta=rope_theta, with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale)
+               rope_theta=rope_theta, with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale,
+               alibi=alibi)
     nbytes = workspace_size(p)
     ws = _workspace(nbytes, q.device, workspace)
     rc = _lib.load().sattn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(topk_idx),
@@ -145,7 +148,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, 
 
 def topk_select(q: torch.Tensor, k: torch.Tensor, *, topk: int, n_start: int = 0, window: int = 0,
                 L_pretrain: int = 0, rope_theta: float = 0.0, is_sep: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0):
+                workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
     """Per-head top-k middle tokens.  Returns (idx [B,Hq,T,k] int32, logit [B,Hq,T,k] fp32)."""
     B, Hq, T, d = q.shape
     idx = torch.empty((B, Hq, T, topk), dtype=torch.int32, device=q.device)
@@ -153,7 +156,8 @@ def topk_select(q: torch.Tensor, k: torch.Tensor, *, topk: int, n_start: int = 0
     if is_sep is not None:
         is_sep = is_sep.to(torch.uint8).contiguous()
     p = params(q, k, k, q, n_start=n_start, window=window, L_pretrain=L_pretrain, topk=topk,
-               rope_theta=rope_theta, with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale)
+               rope_theta=rope_theta, with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale,
+               alibi=alibi)
     nbytes = workspace_size(p)
     ws = _workspace(nbytes, q.device, workspace)
     rc = _lib.load().sattn_topk_select(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(is_sep), _ptr(idx), _ptr(logit),
@@ -211,7 +215,7 @@ def segment_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, S: int, M:
 def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, window: int = 0,
                L_pretrain: int = 0, rope_theta: float = 0.0, is_sep: Optional[torch.Tensor] = None,
                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-               workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0):
+               workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
     """One decoding step: q [B, Hq, 1, d] is the query of the cache's last
     position (k, v [B, Hkv, T, d]).  Returns (O [B, Hq, 1, d], lse [B, Hq])."""
     B, Hq, one, d = q.shape
@@ -225,7 +229,7 @@ def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: in
     if is_sep is not None:
         is_sep = is_sep.to(torch.uint8).contiguous()
     p = params(q, k, v, out, n_start=n_start, window=window, L_pretrain=L_pretrain, rope_theta=rope_theta,
-               with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale)
+               with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale, alibi=alibi)
     p.T = T
     n = ctypes.c_size_t(0)
     L = _lib.load()

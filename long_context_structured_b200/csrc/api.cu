@@ -64,6 +64,7 @@ int check_common(const sattn_params* p) {
   if (p->topk > 16) return SATTN_ERR_UNSUPPORTED;
   if (!(p->rope_theta >= 0.0) || !std::isfinite(p->rope_theta)) return SATTN_ERR_INVALID_ARG;
   if (!(p->rope_pos_scale >= 0.0) || p->rope_pos_scale > 1.0) return SATTN_ERR_INVALID_ARG;
+  if (p->alibi && p->rope_theta != 0.0) return SATTN_ERR_INVALID_ARG;  // ALiBi replaces the rotation
   if ((int64_t)p->B * p->Hq * p->T > (int64_t)1 << 31) return SATTN_ERR_UNSUPPORTED;
   const int64_t* st[4] = {p->q_stride, p->k_stride, p->v_stride, p->o_stride};
   const int esz = p->dtype == SATTN_DTYPE_BF16 ? 2 : 4;
@@ -80,6 +81,13 @@ int check_common(const sattn_params* p) {
 int check_fwd_rules(const sattn_params* p) {
   int rc = check_common(p);
   if (rc) return rc;
+  // an unclipped ALiBi bias would change the top-k ranking and make the bias
+  // of a gathered separator depend on its position: not supported
+  if (p->alibi && p->L_pretrain == 0 && (p->topk > 0 || (p->with_separators && p->dtype == SATTN_DTYPE_BF16)))
+    return SATTN_ERR_UNSUPPORTED;
+  // top-k ranks by q.k; with ALiBi that is the logit's order only when every
+  // candidate (i - j > window) is past the cap
+  if (p->alibi && p->topk > 0 && p->window < p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
   if (p->dtype == SATTN_DTYPE_BF16) {
     if (p->n_start > 256) return SATTN_ERR_UNSUPPORTED;
     if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
@@ -280,6 +288,7 @@ int run_prep_bf16(const sattn_params* p, const FwdPlan& P, const void* Q, const 
   a.Kr = at<__nv_bfloat16>(ws, P.kr);
   a.sink_z = with_sinks ? at<float>(ws, P.sink) : nullptr;
   a.n_sink = with_sinks ? P.n_sink : 0;
+  a.alibi = p->alibi ? 1 : 0;
   a.kmax = with_kmax ? at<uint32_t>(ws, P.kmax) : nullptr;
   ProfScope ps("prep_rope", 1, st);
   return cuda_rc(launch_prep(a, st));
@@ -489,6 +498,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
     a.v_st = p->v_stride[2];
     a.tab = at<float2>(ws, P.tab);
     a.L = p->L_pretrain;
+    a.alibi = p->alibi ? 1 : 0;
     a.n_start = p->n_start;
     a.window = p->window;
     a.sep_pos = is_sep ? sep_pos : nullptr;
@@ -567,6 +577,8 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.d = p->d;
   a.nQT = P.nQT;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.alibi = p->alibi ? 1 : 0;
+  a.alibi_cap = p->L_pretrain;
   a.ns_band = p->n_start;
   a.w_eff = p->window;
   a.sink_z = at<float>(ws, P.sink);
@@ -612,6 +624,7 @@ static int plan_seg(const sattn_params* p, int32_t S, int32_t M, int32_t R, int3
   int rc = check_common(p);
   if (rc) return rc;
   if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
+  if (p->alibi) return SATTN_ERR_UNSUPPORTED;
   if (S < kTile || S % kTile || p->T % S || M < 0 || R < 0 || blk < 1 || R % blk) return SATTN_ERR_INVALID_ARG;
   if (R / blk > 1024 || p->Hq > kMaxHeads) return SATTN_ERR_UNSUPPORTED;
   if (!segment_retrieval_supported(p->T, S, blk)) return SATTN_ERR_UNSUPPORTED;
@@ -845,6 +858,7 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   a.n_start = p->n_start;
   a.window = p->window;
   a.L = p->L_pretrain;
+  a.alibi = p->alibi ? 1 : 0;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.q_sb = p->q_stride[0];

@@ -73,8 +73,11 @@ __global__ void attn_f32_kernel(AttnF32Args a) {
     }
     return warp_sum(acc);
   };
+  // ALiBi: -m_h * min(i - j, L) (no clip when L = 0), m_h = 2^(-8 (h+1) / Hq)
+  const float slope = a.alibi ? exp2f(-8.f * (float)(h + 1) / (float)a.Hq) : 0.f;
   auto add = [&](int j, float z) {
-    const float s = z * scale;
+    const int dist = (a.L > 0) ? min(i - j, a.L) : (i - j);
+    const float s = z * scale - slope * (float)dist;
     const float mn = fmaxf(m, s);
     const float al = expf(m - mn);  // m = -inf -> 0
     const float p = expf(s - mn);

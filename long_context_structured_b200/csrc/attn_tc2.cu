@@ -505,6 +505,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTile; ++c)
           if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
+      if (a.alibi) {
+        // ALiBi bias in units of q.k: band keys -m (i - j) (inside the window,
+        // below the cap); gathered separators lie beyond w = L: -m L
+        const float sq = alibi_slope_qk(h, a.Hq, a.d);
+        if (p < un.NG) {
+          const float cb = sq * (float)a.alibi_cap;
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) sv[c] -= cb;
+        } else {
+          const float base = -sq * (float)(i - (un.U0 + p - un.NG) * kTile);
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) sv[c] += fmaf((float)c, sq, base);
+        }
+      }
       // O_x is stable from here on: S_x(p) completing implies the tile's
       // previous PV completed.  First the rebase the previous tile asked for.
       if (__any_sync(0xffffffffu, rebase != 0)) scale_o<D>(tO + lane_off, exp2_neg_int(rebase));
@@ -572,6 +586,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
     const float* tkz = a.tk_z ? a.tk_z + row_id * a.topk : nullptr;
     // side keys: the starting span (sinks) and the row's top-k keys, fp32
+    // top-k keys are middle keys beyond the cap: ALiBi gives them -m L (sink
+    // logits carry their bias from the prep pass)
+    const float tkb = a.alibi ? alibi_slope_qk(h, a.Hq, a.d) * (float)a.alibi_cap : 0.f;
     float m_fin = m_used;
     for (int j = 0; j < n_sink; ++j) m_fin = fmaxf(m_fin, sz[j] * sl2);
     float pt[kMaxSideTopk];  // top-k weights, 0 for absent keys
@@ -580,14 +597,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int y = 0; y < kMaxSideTopk; ++y) {
       jt[y] = (y < a.topk) ? tki[y] : -1;
       if (jt[y] >= a.T) jt[y] = -1;
-      if (jt[y] >= 0) m_fin = fmaxf(m_fin, tkz[y] * sl2);
+      if (jt[y] >= 0) m_fin = fmaxf(m_fin, (tkz[y] - tkb) * sl2);
     }
     const float alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_fin);
     float l_fin = l_sum * alpha;
     for (int j = 0; j < n_sink; ++j) l_fin += ex2_approx(sz[j] * sl2 - m_fin);
 #pragma unroll
     for (int y = 0; y < kMaxSideTopk; ++y) {
-      pt[y] = (jt[y] >= 0) ? ex2_approx(tkz[y] * sl2 - m_fin) : 0.f;
+      pt[y] = (jt[y] >= 0) ? ex2_approx((tkz[y] - tkb) * sl2 - m_fin) : 0.f;
       l_fin += pt[y];
     }
     const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;

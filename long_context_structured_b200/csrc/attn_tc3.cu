@@ -491,6 +491,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
+      if (a.alibi) {
+        // ALiBi bias in units of q.k: band keys -m (i - j) (inside the window,
+        // below the cap); gathered separators lie beyond w = L: -m L
+        const float sq = alibi_slope_qk(h, a.Hq, a.d);
+        if (j < pl.n_gather) {
+          const float cb = sq * (float)a.alibi_cap;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] -= cb;
+        } else {
+          const float base = -sq * (float)(i - (pl.u_lo + j - pl.n_gather) * kTile - 64 * hc);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] += fmaf((float)c, sq, base);
+        }
+      }
       if (__any_sync(0xffffffffu, rebase != 0)) {
         o_stable(j);
         scale_o<D>(tO, exp2_neg_int(rebase));
@@ -551,15 +565,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* sz = a.sink_z ? a.sink_z + row_id * a.n_sink : nullptr;
     const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
     const float* tkz = a.tk_z ? a.tk_z + row_id * a.topk : nullptr;
+    // top-k keys are middle keys beyond the cap: ALiBi gives them -m L (sink
+    // logits carry their bias from the prep pass)
+    const float tkb = a.alibi ? alibi_slope_qk(h, a.Hq, a.d) * (float)a.alibi_cap : 0.f;
     float m_fin = m_used;
     for (int jj = 0; jj < n_sink; ++jj) m_fin = fmaxf(m_fin, sz[jj] * sl2);
     for (int y = 0; y < a.topk; ++y)
-      if (tki[y] >= 0 && tki[y] < a.T) m_fin = fmaxf(m_fin, tkz[y] * sl2);
+      if (tki[y] >= 0 && tki[y] < a.T) m_fin = fmaxf(m_fin, (tkz[y] - tkb) * sl2);
     const float alpha = (m_used == -CUDART_INF_F) ? 0.f : ex2_approx(m_used - m_fin);
     float l_fin = l_sum * alpha;
     for (int jj = 0; jj < n_sink; ++jj) l_fin += ex2_approx(sz[jj] * sl2 - m_fin);
     for (int y = 0; y < a.topk; ++y)
-      if (tki[y] >= 0 && tki[y] < a.T) l_fin += ex2_approx(tkz[y] * sl2 - m_fin);
+      if (tki[y] >= 0 && tki[y] < a.T) l_fin += ex2_approx((tkz[y] - tkb) * sl2 - m_fin);
     const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;
     const int col0 = hc * (D / 2);
     const __nv_bfloat16* vbase = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh + col0;
@@ -589,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t2 = 0; t2 < a.topk; ++t2) {
         const int jk = tki[t2];
         if (jk < 0 || jk >= a.T) continue;
-        const float pkv = ex2_approx(tkz[t2] * sl2 - m_fin);
+        const float pkv = ex2_approx((tkz[t2] - tkb) * sl2 - m_fin);
         const __nv_bfloat16* vr = vbase + (size_t)jk * a.v_st + c;
 #pragma unroll
         for (int y = 0; y < 32; y += 2) {

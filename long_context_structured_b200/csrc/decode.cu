@@ -148,6 +148,10 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         z[r] = acc * sl2;
+        if (a.alibi) {  // -m_h * min(i - j, L), in log2 units of the scaled logit
+          const int dist = (a.L > 0) ? min(i - jj[u], a.L) : (i - jj[u]);
+          z[r] -= exp2f(-8.f * (float)(g * REP + r + 1) / (float)a.Hq) * 1.4426950408889634f * (float)dist;
+        }
       }
 #pragma unroll
       for (int r = 0; r < REP; ++r) {

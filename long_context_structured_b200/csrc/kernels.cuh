@@ -31,6 +31,7 @@ struct PrepArgs {
   __nv_bfloat16* Kr;  // [B,Hkv,T,d] R(j) k_j           (may be null)
   float* sink_z;      // [B,Hq,T,n_sink] side logits    (may be null)
   int n_sink;
+  int alibi;          // nonzero: sink logits carry the clipped ALiBi bias (in q.k units)
   uint32_t* kmax;     // [B*Hkv] max_j ||k_j|| as float bits (may be null)
 };
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
@@ -94,12 +95,19 @@ struct AttnArgs {
   int16_t long_slot[kMaxHeads]; // head -> index among long heads, -1 for local
   const int32_t* prefix_cnt;   // [B, Hl, N] number of prefix keys
   int n_long;
+  // ALiBi: s_ij gets -m_h * min(i - j, L) (L = 0: no clip), m_h = 2^(-8 (h+1) / Hq)
+  int alibi, alibi_cap;
   // outputs
   __nv_bfloat16* O;
   int64_t o_sb, o_sh, o_st;
   float* lse;
   int32_t* status;
 };
+// ALiBi slope of query head h, times sqrt(d): the bias per unit distance in
+// units of the unscaled logit q.k
+__device__ __forceinline__ float alibi_slope_qk(int h, int Hq, int d) {
+  return exp2f(-8.f * (float)(h + 1) / (float)Hq) * sqrtf((float)d);
+}
 struct AttnMaps {
   CUtensorMap q, q2, k, v, kg, vg;
 };
@@ -125,6 +133,7 @@ struct AttnF32Args {
   const int32_t* tk_idx;     // [B, Hq, T, topk] or null
   const float* tk_z;
   int topk;
+  int alibi;                 // ALiBi bias clipped at L (no rotation)
   float* O;
   int64_t o_sb, o_sh, o_st;
   float* lse;
@@ -207,6 +216,7 @@ struct DecodeArgs {
   const int32_t* sep_prefix;    // [B, T+1] or null (no separators)
   const int32_t* sep_pos;       // [B, T]
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
+  int alibi;                    // ALiBi bias clipped at L (no rotation)
   int n_chunks;
   __nv_bfloat16* O;             // [B, Hq, 1, d]
   int64_t o_sb, o_sh;

@@ -93,6 +93,13 @@ __device__ __forceinline__ void rotate8(const float* x0, const float* x1, const 
   }
 }
 
+// ALiBi bias of pair (i, j) in units of the unscaled logit q.k (0 without ALiBi)
+__device__ __forceinline__ float alibi_bias_qk(const PrepArgs& a, int h, int i, int j) {
+  if (!a.alibi) return 0.f;
+  const int dist = (a.L > 0) ? min(i - j, a.L) : (i - j);
+  return alibi_slope_qk(h, a.Hq, a.d) * (float)dist;
+}
+
 // Shared-memory slot of element c (< d/2) of a staged sink-key half: the 8
 // elements c0..c0+7 of thread `sub` = c / 8 sit as two float4 at
 // q * 4 * TPR + sub * 4 (q = 0, 1), so the TPR threads of a row read 64
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
 #pragma unroll
           for (int q = 0; q < per; ++q) {
             const int j = (sub / dup) * per + q;
-            if (j < n_sink) a.sink_z[zrow + j] = (j <= i) ? z[q] : -CUDART_INF_F;
+            if (j < n_sink) a.sink_z[zrow + j] = (j <= i) ? z[q] - alibi_bias_qk(a, h, i, j) : -CUDART_INF_F;
           }
         }
       } else if (NSP < 0) {
@@ -294,7 +301,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
             for (int o = tpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(grp_mask, acc, o);
             z = acc;
           }
-          if (sub == (j % tpr)) a.sink_z[zrow + j] = z;
+          if (sub == (j % tpr)) a.sink_z[zrow + j] = (j <= i) ? z - alibi_bias_qk(a, h, i, j) : z;
         }
       }
     }

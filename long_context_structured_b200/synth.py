@@ -39,6 +39,7 @@ class Workload:
     L_pretrain: int = 0        # 0 disables the distance cap
     rope_theta: float = 0.0    # 0 disables RoPE
     rope_pos_scale: float = 1.0  # position interpolation: rotary positions multiplied by this
+    alibi: bool = False        # clipped ALiBi bias in place of the rotation (rope_theta 0)
     topk: int = 0
     sep_rate: float = 0.0      # Bernoulli flag rate (c1-style) ...
     sep_vocab: int = 0         # ... or token-id derived flags (c3-style) when > 0

@@ -41,6 +41,7 @@ class OracleParams(ctypes.Structure):
         ("n_start", ctypes.c_int32), ("window", ctypes.c_int32),
         ("L_pretrain", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("rope_theta", ctypes.c_double), ("rope_pos_scale", ctypes.c_double),
+        ("alibi", ctypes.c_int32),
     ]
 
 
@@ -105,14 +106,14 @@ def nthreads_default() -> int:
 
 
 def params(B, Hq, Hkv, T, d, dtype="bf16", n_start=0, window=0, L_pretrain=0, topk=0,
-           rope_theta=0.0, rope_pos_scale=1.0) -> OracleParams:
+           rope_theta=0.0, rope_pos_scale=1.0, alibi=False) -> OracleParams:
     return OracleParams(B, Hq, Hkv, T, d, 0 if dtype == "bf16" else 1, n_start, window,
-                        L_pretrain, topk, float(rope_theta), float(rope_pos_scale))
+                        L_pretrain, topk, float(rope_theta), float(rope_pos_scale), int(bool(alibi)))
 
 
 def params_of(wl) -> OracleParams:
     return params(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.dtype, wl.n_start, wl.window,
-                  wl.L_pretrain, wl.topk, wl.rope_theta, wl.rope_pos_scale)
+                  wl.L_pretrain, wl.topk, wl.rope_theta, wl.rope_pos_scale, wl.alibi)
 
 
 def _inputs(p: OracleParams, q, k, v):

@@ -53,6 +53,13 @@
  *   R10 retrieval: block score = max over a block of the unrotated
  *       <q_{sS-1}, k_j>, top R/blk blocks (ties to the lower block), prefix
  *       in ascending block order; segment 0 has no tail and no prefix.
+ *   R11 ALiBi ([LMI] 方法: for a model with ALiBi the distance bias is
+ *       clipped at the same cap): the scaled logit gets -m_h * d'_ij with
+ *       d'_ij = min(i-j, L) (i-j when L = 0); the pages name no slopes, so
+ *       head h of H takes ALiBi's own geometric set m_h = 2^(-8(h+1)/H);
+ *       distances are token distances (the rotary scale s does not apply);
+ *       top-k ranks by z - sqrt(d) m_h d'_ij, the unscaled form of the
+ *       biased logit, and reports z.
  *
  * Parity pins: every function here is checked by the CPU tests against
  * closed forms, hand-written golden masks, library routines on degenerate
@@ -74,11 +81,24 @@ typedef struct oracle_params {
   int32_t n_start, window, L_pretrain, topk;
   double rope_theta;
   double rope_pos_scale; /* position interpolation scale s (R7); 0 means 1 */
+  int32_t alibi;         /* 1: clipped ALiBi bias (R11) instead of a rotation */
 } oracle_params;
 
 /* rotary position of token position `pos` (R7) */
 static double rot_pos(const oracle_params* p, double pos) {
   return pos * (p->rope_pos_scale > 0.0 ? p->rope_pos_scale : 1.0);
+}
+
+/* ALiBi slope of query head h (R11) */
+static double alibi_slope(const oracle_params* p, int h) {
+  return pow(2.0, -8.0 * (double)(h + 1) / (double)p->Hq);
+}
+
+/* clipped ALiBi distance d'_ij (R11) */
+static double alibi_dist(int i, int j, int L) {
+  int dist = i - j;
+  if (L > 0 && dist > L) dist = L;
+  return (double)dist;
 }
 
 /* ------------------------------------------------------------------ */
@@ -188,15 +208,16 @@ double oracle_logit(const double* q, const double* k, int d, int i, int j, int L
 /* ------------------------------------------------------------------ */
 
 typedef struct {
-  double z;
+  double z;    /* unscaled logit */
+  double rank; /* ranking key: z, less the unscaled ALiBi bias (R11) */
   int32_t j;
 } cand_t;
 
 static int cand_cmp(const void* a, const void* b) {
   const cand_t* x = (const cand_t*)a;
   const cand_t* y = (const cand_t*)b;
-  if (x->z > y->z) return -1;
-  if (x->z < y->z) return 1;
+  if (x->rank > y->rank) return -1;
+  if (x->rank < y->rank) return 1;
   return (x->j < y->j) ? -1 : (x->j > y->j);
 }
 
@@ -214,7 +235,7 @@ typedef struct {
 
 /* Computes O_i and LSE_i for one row.  If forced != NULL the top-k set is
  * taken from it (k entries, -1 = none) instead of being selected. */
-static int attn_row(const head_ctx* hc, const double* qraw, int i, const int32_t* forced,
+static int attn_row(const head_ctx* hc, const double* qraw, int h, int i, const int32_t* forced,
                     double* o_out, double* lse_out, int32_t* tk_idx, double* tk_z, int64_t* count,
                     uint8_t* m, double* zbuf, cand_t* cands, double* work) {
   const oracle_params* p = hc->p;
@@ -223,6 +244,7 @@ static int attn_row(const head_ctx* hc, const double* qraw, int i, const int32_t
   double* q_L = work + d;
   oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
   oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
+  double slope = p->alibi ? alibi_slope(p, h) : 0.0;
 
   int64_t cnt = oracle_mask_row(T, i, p->n_start, p->window, hc->sep, m);
 
@@ -240,6 +262,8 @@ static int attn_row(const head_ctx* hc, const double* qraw, int i, const int32_t
       for (int j = 0; j <= i; ++j) {
         if (m[j]) continue;
         cands[n].z = capped_logit(i, j, L, d, q_i, q_L, hc->Krot + (size_t)j * d, hc->Kraw + (size_t)j * d);
+        cands[n].rank = cands[n].z;
+        if (p->alibi) cands[n].rank -= sqrt((double)d) * slope * alibi_dist(i, j, L);
         cands[n].j = j;
         ++n;
       }
@@ -266,6 +290,7 @@ static int attn_row(const head_ctx* hc, const double* qraw, int i, const int32_t
   for (int j = 0; j < T; ++j) {
     if (!m[j]) continue;
     double s = capped_logit(i, j, L, d, q_i, q_L, hc->Krot + (size_t)j * d, hc->Kraw + (size_t)j * d) * inv_sqrt_d;
+    if (p->alibi) s -= slope * alibi_dist(i, j, L);
     zbuf[j] = s;
     if (s > mx) mx = s;
   }
@@ -372,7 +397,7 @@ static void fwd_one(void* a, int64_t t) {
   double* qraw = work + 2 * d;
   int64_t qb = (((int64_t)b * p->Hq + h) * T + i) * d;
   for (int c = 0; c < d; ++c) qraw[c] = load_elem(J->Q, p->dtype, qb + c);
-  attn_row(&J->hc, qraw, i, J->forced ? J->forced + r * k : NULL, J->O + r * d, J->lse + r,
+  attn_row(&J->hc, qraw, h, i, J->forced ? J->forced + r * k : NULL, J->O + r * d, J->lse + r,
            (J->tk_idx && k) ? J->tk_idx + r * k : NULL, (J->tk_z && k) ? J->tk_z + r * k : NULL,
            J->counts ? J->counts + r : NULL, m, zbuf, cands, work);
   free(m);

@@ -28,7 +28,7 @@ def _decode_and_check(oracle_mod, wl, seed):
     sep = to_dev(inp["is_sep"])
     qd = q[:, :, wl.T - 1:wl.T, :].contiguous()
     O, lse = sa.decode_fwd(qd, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
-                           rope_theta=wl.rope_theta, is_sep=sep, rope_pos_scale=wl.rope_pos_scale)
+                           rope_theta=wl.rope_theta, is_sep=sep, rope_pos_scale=wl.rope_pos_scale, alibi=wl.alibi)
     torch.cuda.synchronize()
     assert sa.stream_status() == 0
     rows = np.array([(b, h, wl.T - 1) for b in range(wl.B) for h in range(wl.Hq)], dtype=np.int64)
@@ -53,6 +53,10 @@ CASES = [
     ("one_token", dict(B=2, Hq=2, Hkv=2, T=1, d=64, n_start=0, window=4, rope_theta=1e4)),
     ("pos_interp", dict(B=1, Hq=4, Hkv=1, T=900, d=128, n_start=4, window=64, L_pretrain=64, rope_theta=1e4,
                         sep_rate=0.1, rope_pos_scale=0.25)),
+    ("alibi_capped_sep_gqa4", dict(B=2, Hq=8, Hkv=2, T=900, d=128, n_start=4, window=64, L_pretrain=64,
+                                   sep_rate=0.1, alibi=True)),
+    ("alibi_unclipped_sep_d64", dict(B=1, Hq=4, Hkv=4, T=500, d=64, n_start=2, window=40, sep_rate=0.2,
+                                     alibi=True)),
 ]
 
 

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import long_context_structured_b200 as sa
-from long_context_structured_b200 import synth
+from long_context_structured_b200 import _lib, synth
 from _util import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, compare, gather_rows, to_dev, topk_agreement)
 
 pytestmark = pytest.mark.gpu
@@ -32,7 +32,8 @@ def _run_fwd(wl, inp, **kw):
     q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
     sep = to_dev(inp["is_sep"])
     O, lse = sa.fwd(q, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
-                    rope_theta=wl.rope_theta, topk=wl.topk, is_sep=sep, rope_pos_scale=wl.rope_pos_scale, **kw)
+                    rope_theta=wl.rope_theta, topk=wl.topk, is_sep=sep, rope_pos_scale=wl.rope_pos_scale,
+                    alibi=wl.alibi, **kw)
     torch.cuda.synchronize()
     _status_ok()
     return O, lse
@@ -95,6 +96,10 @@ def test_c1_f32_full(oracle_mod):
 @pytest.mark.parametrize("cfg", [
     dict(B=1, Hq=2, Hkv=1, T=300, d=64, n_start=2, window=20, L_pretrain=40, rope_theta=1e4, topk=3, sep_rate=0.1),
     dict(B=2, Hq=2, Hkv=2, T=200, d=128, n_start=0, window=199, rope_theta=5e5),
+    # clipped ALiBi: separators at their own (unclipped) distance; top-k past the cap; window below the cap
+    dict(B=1, Hq=4, Hkv=2, T=300, d=64, n_start=3, window=20, sep_rate=0.15, alibi=True),
+    dict(B=1, Hq=4, Hkv=1, T=250, d=128, n_start=2, window=30, L_pretrain=30, topk=3, sep_rate=0.1, alibi=True),
+    dict(B=1, Hq=2, Hkv=2, T=260, d=64, n_start=4, window=20, L_pretrain=60, sep_rate=0.1, alibi=True),
 ])
 def test_f32_features(oracle_mod, cfg):
     wl = synth.Workload(name="f32", dtype="f32", **cfg)
@@ -125,6 +130,16 @@ SMALL = [
                                      rope_theta=1e4, sink_scale=8.0, rope_pos_scale=0.25)),
     ("pos_interp_sep_gqa", dict(B=2, Hq=4, Hkv=2, T=700, d=64, n_start=2, window=40, rope_theta=5e5,
                                 sep_rate=0.15, rope_pos_scale=0.5)),
+    # clipped ALiBi (LM-Infinite, section 方法): band keys -m (i - j), keys past the cap -m L
+    ("alibi_causal_h8", dict(B=1, Hq=8, Hkv=2, T=700, d=128, n_start=0, window=1000, alibi=True)),
+    ("alibi_lambda_capped", dict(B=1, Hq=4, Hkv=1, T=1000, d=128, n_start=4, window=100, L_pretrain=100,
+                                 sink_scale=8.0, alibi=True)),
+    ("alibi_sep_capped_d64", dict(B=2, Hq=4, Hkv=2, T=600, d=64, n_start=4, window=64, L_pretrain=64,
+                                  sep_rate=0.2, alibi=True)),
+    ("alibi_window_below_cap", dict(B=1, Hq=2, Hkv=2, T=800, d=128, n_start=4, window=50, L_pretrain=200,
+                                    sink_scale=8.0, alibi=True)),
+    ("alibi_sep_capped_even", dict(B=1, Hq=2, Hkv=1, T=1024, d=128, n_start=4, window=128, L_pretrain=128,
+                                   sep_rate=0.1, alibi=True)),
 ]
 
 
@@ -159,6 +174,37 @@ def test_bf16_topk_small(oracle_mod):
     # attention with the selection inside the call
     O, lse = _run_fwd(wl, inp)
     _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi)
+
+
+def test_bf16_topk_alibi(oracle_mod):
+    """Top-k with the clipped ALiBi bias: every candidate is past the cap
+    (L = w), so the ranking is by q.k and the gathered keys carry -m L."""
+    wl = synth.Workload(name="topk_alibi", B=1, Hq=4, Hkv=2, T=1536, d=128, dtype="bf16", n_start=4, window=128,
+                        L_pretrain=128, topk=4, plant=2, alibi=True)
+    inp = synth.make_inputs(wl, seed=12)
+    q, k = to_dev(inp["q"]), to_dev(inp["k"])
+    idx, _ = sa.topk_select(q, k, topk=wl.topk, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                            alibi=True)
+    torch.cuda.synchronize()
+    _status_ok()
+    rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(oracle_mod.params_of(wl.scaled(topk=wl.topk + 1)), inp["q"],
+                                                  inp["k"], inp["v"], None, rows)
+    gi = idx.cpu().numpy().reshape(-1, wl.topk)
+    _, _, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
+    assert not bad, "rows %s differ without a near tie" % bad[:10]
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi)
+
+
+def test_alibi_rejects_unsupported():
+    q = torch.zeros((1, 2, 256, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.SattnError):
+        sa.fwd(q, q, q, window=8, rope_theta=1e4, alibi=True)  # ALiBi replaces the rotation
+    with pytest.raises(_lib.SattnError):
+        sa.fwd(q, q, q, window=8, topk=2, alibi=True)          # uncapped bias would reorder top-k
+    with pytest.raises(_lib.SattnError):
+        sa.fwd(q, q, q, window=8, L_pretrain=16, topk=2, alibi=True)
 
 
 # ---------------------------------------------------------------------------

@@ -601,3 +601,119 @@ def test_position_scale_one_is_identity(oracle_mod):
     a = oracle_mod.fwd_rows(oracle_mod.params(B, H, H, T, d, "bf16", 4, 9, 9, 0, 1e4), q, k, v, None, rows)
     b = oracle_mod.fwd_rows(oracle_mod.params(B, H, H, T, d, "bf16", 4, 9, 9, 0, 1e4, 1.0), q, k, v, None, rows)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ----------------------------------------------------------------------------
+# clipped ALiBi (LM-Infinite, section 方法: the distance bias clipped at L)
+# ----------------------------------------------------------------------------
+
+# ALiBi's published slope sets: 8 heads take 1/2, 1/4, ..., 1/256 and 4 heads
+# 1/4, 1/16, 1/64, 1/256 (each the geometric sequence from 2^(-8/H))
+ALIBI_SLOPES = {8: [2.0 ** -x for x in range(1, 9)], 4: [2.0 ** -x for x in (2, 4, 6, 8)]}
+
+
+def _sdpa_bias(q64, k64, v64, bias):
+    """torch SDPA in fp64 with an additive float mask bias [H, T, T] (-inf =
+    masked); returns O and the natural-log LSE of the biased scaled logits."""
+    rep = q64.shape[1] // k64.shape[1]
+    k = np.repeat(k64, rep, axis=1)
+    v = np.repeat(v64, rep, axis=1)
+    bt = torch.from_numpy(bias)[None]
+    O = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q64), torch.from_numpy(k),
+                                                         torch.from_numpy(v), attn_mask=bt).numpy()
+    s = np.einsum("bhid,bhjd->bhij", q64, k) / math.sqrt(q64.shape[-1]) + bias[None]
+    mx = s.max(-1, keepdims=True)
+    lse = (mx + np.log(np.exp(s - mx).sum(-1, keepdims=True)))[..., 0]
+    return O, lse
+
+
+def _alibi_bias(H, T, mask, L):
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    dist = (i - j).astype(np.float64)
+    if L > 0:
+        dist = np.minimum(dist, L)
+    m = np.array(ALIBI_SLOPES[H])[:, None, None]
+    return np.where(mask[None], -m * dist[None], -np.inf)
+
+
+def test_alibi_unclipped_causal_equals_sdpa_with_bias(oracle_mod):
+    """L = 0: plain ALiBi over full causal attention, 8 heads with the
+    published slopes."""
+    B, H, T, d = 1, 8, 40, 16
+    q, k, v = _rand_inputs(B, H, 2, T, d, 31)
+    p = oracle_mod.params(B, H, 2, T, d, "bf16", 0, T, 0, 0, 0.0, alibi=True)
+    O, lse, *_ = oracle_mod.fwd_rows(p, q, k, v, None, oracle_mod.all_rows(B, H, T))
+    ref, lref = _sdpa_bias(_f64(q), _f64(k), _f64(v), _alibi_bias(H, T, _tri(T), 0))
+    assert np.abs(O.reshape(ref.shape) - ref).max() < 1e-12
+    assert np.abs(lse.reshape(lref.shape) - lref).max() < 1e-12
+
+
+def test_alibi_clipped_lambda_equals_sdpa_with_bias(oracle_mod):
+    """Lambda mask (sinks + window w = L) with the bias clipped at L: the
+    starting-span keys beyond the window get -m L, window keys -m (i - j)."""
+    B, H, T, d = 2, 4, 48, 16
+    ns, L = 3, 6
+    q, k, v = _rand_inputs(B, H, H, T, d, 32, "f32")
+    p = oracle_mod.params(B, H, H, T, d, "f32", ns, L, L, 0, 0.0, alibi=True)
+    O, lse, *_ = oracle_mod.fwd_rows(p, q, k, v, None, oracle_mod.all_rows(B, H, T))
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    lam = (j <= i) & ((j < ns) | (i - j <= L))
+    ref, lref = _sdpa_bias(_f64(q), _f64(k), _f64(v), _alibi_bias(H, T, lam, L))
+    assert np.abs(O.reshape(ref.shape) - ref).max() < 1e-12
+    assert np.abs(lse.reshape(lref.shape) - lref).max() < 1e-12
+    # the clip matters: the unclipped bias gives another answer
+    ref2, _ = _sdpa_bias(_f64(q), _f64(k), _f64(v), _alibi_bias(H, T, lam, 0))
+    assert np.abs(O.reshape(ref.shape) - ref2).max() > 1e-3
+
+
+def test_alibi_clipped_separators_equals_sdpa_with_bias(oracle_mod):
+    """SepLLM mask with the clipped bias: every separator beyond the window
+    sits at the cap."""
+    B, H, T, d = 1, 4, 45, 8
+    ns, w = 2, 5
+    q, k, v = _rand_inputs(B, H, 1, T, d, 33)
+    rng = np.random.default_rng(34)
+    sep = (rng.random((B, T)) < 0.25).astype(np.uint8)
+    p = oracle_mod.params(B, H, 1, T, d, "bf16", ns, w, w, 0, 0.0, alibi=True)
+    O, lse, *_ = oracle_mod.fwd_rows(p, q, k, v, sep, oracle_mod.all_rows(B, H, T))
+    mask = np.stack([oracle_mod.mask_row(T, i, ns, w, sep[0])[0] for i in range(T)]).astype(bool)
+    ref, lref = _sdpa_bias(_f64(q), _f64(k), _f64(v), _alibi_bias(H, T, mask, w))
+    assert np.abs(O.reshape(ref.shape) - ref).max() < 1e-12
+    assert np.abs(lse.reshape(lref.shape) - lref).max() < 1e-12
+
+
+def test_alibi_topk_ranks_by_biased_logit(oracle_mod):
+    """Brute force: with the cap above the window the bias varies among the
+    candidates and decides the ranking (key z - sqrt(d) m min(i-j, L));
+    reported values stay the unbiased z.  With L = w every candidate is past
+    the cap and the set equals the one without the bias."""
+    T, d, H = 40, 8, 4
+    q, k, v = _rand_inputs(1, H, H, T, d, 35, "f32")
+    ns, w, L, kk = 2, 3, 12, 4
+    p = oracle_mod.params(1, H, H, T, d, "f32", ns, w, L, kk, 0.0, alibi=True)
+    _, _, tki, tkz, _ = oracle_mod.fwd_rows(p, q, k, v, None, oracle_mod.all_rows(1, H, T))
+    tki = tki.reshape(H, T, kk)
+    tkz = tkz.reshape(H, T, kk)
+    qd, kd = _f64(q)[0], _f64(k)[0]
+    differs = 0
+    for h in range(H):
+        m = ALIBI_SLOPES[H][h]
+        for i in range(T):
+            cands = []
+            for j in range(ns, max(ns, i - w)):
+                z = float(qd[h, i] @ kd[h, j])
+                cands.append((z - math.sqrt(d) * m * min(i - j, L), z, j))
+            best = sorted(cands, key=lambda t: (-t[0], t[2]))[:kk]
+            plain = sorted(cands, key=lambda t: (-t[1], t[2]))[:kk]
+            assert list(tki[h, i]) == [j for *_, j in best] + [-1] * (kk - len(best)), (h, i)
+            for r, (_, z, _) in enumerate(best):
+                assert abs(tkz[h, i, r] - z) < 1e-12
+            differs += int([t[2] for t in best] != [t[2] for t in plain])
+    assert differs > 0
+    p2 = oracle_mod.params(1, H, H, T, d, "f32", ns, w, w, kk, 0.0, alibi=True)
+    p3 = oracle_mod.params(1, H, H, T, d, "f32", ns, w, w, kk, 0.0)
+    a = oracle_mod.fwd_rows(p2, q, k, v, None, oracle_mod.all_rows(1, H, T))
+    b = oracle_mod.fwd_rows(p3, q, k, v, None, oracle_mod.all_rows(1, H, T))
+    assert np.array_equal(a[2], b[2])
