@@ -257,7 +257,7 @@ struct Cfg {
   static constexpr size_t kSmem = 1024 + (size_t)kTileBytes * (kQTiles + kKS + kVS) + 256;
 };
 
-template <int D, bool Q2>
+template <int D, bool Q2, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
-      if (a.alibi) {
+      if constexpr (kAlibi) {
         // ALiBi bias in units of q.k: band keys -m (i - j) (inside the window,
         // below the cap); gathered separators lie beyond w = L: -m L
         const float sq = alibi_slope_qk(h, a.Hq, a.d);
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* tkz = a.tk_z ? a.tk_z + row_id * a.topk : nullptr;
     // top-k keys are middle keys beyond the cap: ALiBi gives them -m L (sink
     // logits carry their bias from the prep pass)
-    const float tkb = a.alibi ? alibi_slope_qk(h, a.Hq, a.d) * (float)a.alibi_cap : 0.f;
+    const float tkb = kAlibi ? alibi_slope_qk(h, a.Hq, a.d) * (float)a.alibi_cap : 0.f;
     float m_fin = m_used;
     for (int jj = 0; jj < n_sink; ++jj) m_fin = fmaxf(m_fin, sz[jj] * sl2);
     for (int y = 0; y < a.topk; ++y)
@@ -640,22 +640,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool Q2>
+// ALiBi is a template parameter, so the kernels without it carry no code for it
+template <int D, bool Q2, bool kAlibi>
 cudaError_t launch_d(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
   const size_t bytes = Cfg<D, Q2>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc3_kernel<D, Q2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_tc3_kernel<D, Q2, kAlibi>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)a.B * a.Hq * a.nQT;
-  attn_tc3_kernel<D, Q2><<<grid, kThreads, bytes, st>>>(m.q, m.q2, m.k, m.v, m.kg, m.vg, a);
+  attn_tc3_kernel<D, Q2, kAlibi><<<grid, kThreads, bytes, st>>>(m.q, m.q2, m.k, m.v, m.kg, m.vg, a);
   return cudaGetLastError();
+}
+
+template <int D, bool Q2>
+cudaError_t launch_q(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
+  return a.alibi ? launch_d<D, Q2, true>(a, m, st) : launch_d<D, Q2, false>(a, m, st);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_tc3(const AttnArgs& a, const AttnMaps& m, cudaStream_t st) {
   if (a.B * a.Hq * a.nQT == 0) return cudaSuccess;
-  if (a.d == 128) return a.q2 ? launch_d<128, true>(a, m, st) : launch_d<128, false>(a, m, st);
-  if (a.d == 64) return a.q2 ? launch_d<64, true>(a, m, st) : launch_d<64, false>(a, m, st);
+  if (a.d == 128) return a.q2 ? launch_q<128, true>(a, m, st) : launch_q<128, false>(a, m, st);
+  if (a.d == 64) return a.q2 ? launch_q<64, true>(a, m, st) : launch_q<64, false>(a, m, st);
   return cudaErrorInvalidValue;
 }
 
