@@ -76,6 +76,8 @@ def lib():
             L.oracle_fwd_rows.restype = ctypes.c_int
             L.oracle_fwd_rows.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 4 + [
                 ctypes.c_int64] + [ctypes.c_void_p] * 7 + [ctypes.c_int]
+            L.oracle_bwd.restype = ctypes.c_int
+            L.oracle_bwd.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
             L.oracle_blockmap.restype = ctypes.c_int
             L.oracle_blockmap.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 5
             L.oracle_segment_rows.restype = ctypes.c_int
@@ -168,6 +170,24 @@ def fwd_rows(p: OracleParams, q, k, v, is_sep, rows, forced_topk=None, nthreads=
     if rc != 0:
         raise RuntimeError("oracle_fwd_rows failed: %d" % rc)
     return O, lse, tki[:, : p.topk], tkz[:, : p.topk], cnt
+
+
+def bwd(p: OracleParams, q, k, v, is_sep, dO, forced_topk=None, nthreads=None):
+    """Gradients of sum(dO * O): (dQ [B,Hq,T,d], dK [B,Hkv,T,d], dV [B,Hkv,T,d]) in float64.
+    dO has the inputs' encoding; forced_topk [B,Hq,T,k] fixes the top-k sets."""
+    q, k, v = _inputs(p, q, k, v)
+    g = _c(dO, np.uint16 if p.dtype == 0 else np.float32)
+    assert g.size == q.size
+    s = _c(is_sep, np.uint8)
+    f = _c(forced_topk, np.int32)
+    dQ = np.zeros((p.B, p.Hq, p.T, p.d), dtype=np.float64)
+    dK = np.zeros((p.B, p.Hkv, p.T, p.d), dtype=np.float64)
+    dV = np.zeros((p.B, p.Hkv, p.T, p.d), dtype=np.float64)
+    rc = lib().oracle_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(s), _ptr(f), _ptr(g), _ptr(dQ),
+                          _ptr(dK), _ptr(dV), nthreads or nthreads_default())
+    if rc != 0:
+        raise RuntimeError("oracle_bwd failed: %d" % rc)
+    return dQ, dK, dV
 
 
 def all_rows(B, H, T) -> np.ndarray:

@@ -60,6 +60,12 @@
  *       distances are token distances (the rotary scale s does not apply);
  *       top-k ranks by z - sqrt(d) m_h d'_ij, the unscaled form of the
  *       biased logit, and reports z.
+ *   R12 backward ([SEP] 6.2: training runs the forward and the backward
+ *       pass through the masked product): the gradients of sum(dO . O)
+ *       in exact arithmetic; the
+ *       top-k selection and the mask are constants (no gradient flows
+ *       through a choice); a capped pair contributes to k_j directly and to
+ *       q_i through R(L)^T, an uncapped one through R(j)^T and R(i)^T.
  *
  * Parity pins: every function here is checked by the CPU tests against
  * closed forms, hand-written golden masks, library routines on degenerate
@@ -233,17 +239,13 @@ typedef struct {
   const uint8_t* sep; /* [T] or NULL */
 } head_ctx;
 
-/* Computes O_i and LSE_i for one row.  If forced != NULL the top-k set is
- * taken from it (k entries, -1 = none) instead of being selected. */
-static int attn_row(const head_ctx* hc, const double* qraw, int h, int i, const int32_t* forced,
-                    double* o_out, double* lse_out, int32_t* tk_idx, double* tk_z, int64_t* count,
-                    uint8_t* m, double* zbuf, cand_t* cands, double* work) {
+/* The key set of row i: the structural mask, then the top-k middle keys
+ * (taken from `forced` -- k entries, -1 = none -- or selected here).
+ * q_i = R(i)q and q_L = R(L)q must be set.  Returns the number of keys. */
+static int64_t row_key_set(const head_ctx* hc, const double* q_i, const double* q_L, int h, int i,
+                           const int32_t* forced, int32_t* tk_idx, double* tk_z, uint8_t* m, cand_t* cands) {
   const oracle_params* p = hc->p;
   int T = p->T, d = p->d, L = p->L_pretrain;
-  double* q_i = work;
-  double* q_L = work + d;
-  oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
-  oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
   double slope = p->alibi ? alibi_slope(p, h) : 0.0;
 
   int64_t cnt = oracle_mask_row(T, i, p->n_start, p->window, hc->sep, m);
@@ -281,16 +283,41 @@ static int attn_row(const head_ctx* hc, const double* qraw, int h, int i, const 
       }
     }
   }
+  return cnt;
+}
+
+/* Scaled logit s_ij of a kept key: the capped rotary logit over sqrt(d),
+ * less the clipped ALiBi bias (R5, R11). */
+static double row_logit(const head_ctx* hc, const double* q_i, const double* q_L, double slope, int i, int j) {
+  const oracle_params* p = hc->p;
+  int d = p->d, L = p->L_pretrain;
+  double s = capped_logit(i, j, L, d, q_i, q_L, hc->Krot + (size_t)j * d, hc->Kraw + (size_t)j * d) *
+             (1.0 / sqrt((double)d));
+  if (p->alibi) s -= slope * alibi_dist(i, j, L);
+  return s;
+}
+
+/* Computes O_i and LSE_i for one row.  If forced != NULL the top-k set is
+ * taken from it (k entries, -1 = none) instead of being selected. */
+static int attn_row(const head_ctx* hc, const double* qraw, int h, int i, const int32_t* forced,
+                    double* o_out, double* lse_out, int32_t* tk_idx, double* tk_z, int64_t* count,
+                    uint8_t* m, double* zbuf, cand_t* cands, double* work) {
+  const oracle_params* p = hc->p;
+  int T = p->T, d = p->d, L = p->L_pretrain;
+  double* q_i = work;
+  double* q_L = work + d;
+  oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
+  oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
+  double slope = p->alibi ? alibi_slope(p, h) : 0.0;
+  int64_t cnt = row_key_set(hc, q_i, q_L, h, i, forced, tk_idx, tk_z, m, cands);
   if (count) *count = cnt;
 
   /* logits of kept keys, scaled by 1/sqrt(d); masked keys are -inf and
    * contribute exactly zero, so they are skipped */
-  double inv_sqrt_d = 1.0 / sqrt((double)d);
   double mx = -INFINITY;
   for (int j = 0; j < T; ++j) {
     if (!m[j]) continue;
-    double s = capped_logit(i, j, L, d, q_i, q_L, hc->Krot + (size_t)j * d, hc->Kraw + (size_t)j * d) * inv_sqrt_d;
-    if (p->alibi) s -= slope * alibi_dist(i, j, L);
+    double s = row_logit(hc, q_i, q_L, slope, i, j);
     zbuf[j] = s;
     if (s > mx) mx = s;
   }
@@ -453,6 +480,152 @@ int oracle_fwd_rows(const oracle_params* p, const void* Q, const void* K, const 
   free(Krot);
   free(Vd);
   free(sel);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* backward: gradients of L = sum dO . O (R12)                          */
+/* ------------------------------------------------------------------ */
+
+/* One (batch, kv head): every row of every query head of the group.  The
+ * key-side sums run over all rows, so a job owns its kv head's dK / dV. */
+typedef struct {
+  const oracle_params* p;
+  const void *Q, *K, *V, *dO;
+  const uint8_t* is_sep;
+  const int32_t* forced; /* [B, Hq, T, k] or NULL */
+  double *dQ, *dK, *dV;
+} bwd_job;
+
+static void bwd_one(void* arg, int64_t t) {
+  bwd_job* J = (bwd_job*)arg;
+  const oracle_params* p = J->p;
+  int T = p->T, d = p->d, L = p->L_pretrain, k = p->topk;
+  int b = (int)(t / p->Hkv), g = (int)(t % p->Hkv);
+  double* Kraw = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Krot = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Vd = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* gKrot = (double*)calloc((size_t)T * d, sizeof(double)); /* d L / d (R(j) k_j), uncapped pairs */
+  double* gKraw = (double*)calloc((size_t)T * d, sizeof(double)); /* d L / d k_j, capped pairs */
+  double* gV = (double*)calloc((size_t)T * d, sizeof(double));
+  uint8_t* m = (uint8_t*)malloc((size_t)T);
+  double* P = (double*)malloc(sizeof(double) * (size_t)T);
+  double* dP = (double*)malloc(sizeof(double) * (size_t)T);
+  cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T + 1));
+  double* work = (double*)malloc(sizeof(double) * 8 * (size_t)d);
+  double *qraw = work, *q_i = work + d, *q_L = work + 2 * d, *doi = work + 3 * d;
+  double *gqr = work + 4 * d, *gqc = work + 5 * d, *tmp = work + 6 * d;
+  head_ctx hc;
+  hc.p = p;
+  hc.Kraw = Kraw;
+  hc.Krot = Krot;
+  hc.Vd = Vd;
+  hc.sep = J->is_sep ? J->is_sep + (size_t)b * T : NULL;
+  load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
+  int rep = p->Hq / p->Hkv;
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  for (int h = g * rep; h < (g + 1) * rep; ++h) {
+    double slope = p->alibi ? alibi_slope(p, h) : 0.0;
+    for (int i = 0; i < T; ++i) {
+      int64_t qb = (((int64_t)b * p->Hq + h) * T + i) * d;
+      for (int c = 0; c < d; ++c) {
+        qraw[c] = load_elem(J->Q, p->dtype, qb + c);
+        doi[c] = load_elem(J->dO, p->dtype, qb + c);
+      }
+      oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
+      oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
+      const int32_t* fr = J->forced ? J->forced + ((((int64_t)b * p->Hq + h) * T) + i) * k : NULL;
+      int64_t cnt = row_key_set(&hc, q_i, q_L, h, i, fr, NULL, NULL, m, cands);
+      for (int c = 0; c < d; ++c) gqr[c] = gqc[c] = 0.0;
+      if (cnt > 0) {
+        /* forward quantities of the row: P_ij = exp(s_ij - LSE_i) */
+        double mx = -INFINITY;
+        for (int j = 0; j < T; ++j)
+          if (m[j]) {
+            P[j] = row_logit(&hc, q_i, q_L, slope, i, j);
+            if (P[j] > mx) mx = P[j];
+          }
+        double sum = 0.0;
+        for (int j = 0; j < T; ++j)
+          if (m[j]) sum += exp(P[j] - mx);
+        double lse = mx + log(sum);
+        /* dP_ij = dO_i . v_j and D_i = sum_j P_ij dP_ij (= dO_i . O_i) */
+        double D = 0.0;
+        for (int j = 0; j < T; ++j)
+          if (m[j]) {
+            P[j] = exp(P[j] - lse);
+            dP[j] = dot(doi, Vd + (size_t)j * d, d);
+            D += P[j] * dP[j];
+          }
+        for (int j = 0; j < T; ++j) {
+          if (!m[j]) continue;
+          /* dL/dz_ij: softmax Jacobian, then the 1/sqrt(d) scale */
+          double dz = P[j] * (dP[j] - D) * inv_sqrt_d;
+          double* gv = gV + (size_t)j * d;
+          for (int c = 0; c < d; ++c) gv[c] += P[j] * doi[c];
+          if (L > 0 && i - j > L) {
+            /* z = <R(L) q_i, k_j> */
+            for (int c = 0; c < d; ++c) {
+              gqc[c] += dz * Kraw[(size_t)j * d + c];
+              gKraw[(size_t)j * d + c] += dz * q_L[c];
+            }
+          } else {
+            /* z = <R(i) q_i, R(j) k_j> */
+            for (int c = 0; c < d; ++c) {
+              gqr[c] += dz * Krot[(size_t)j * d + c];
+              gKrot[(size_t)j * d + c] += dz * q_i[c];
+            }
+          }
+        }
+      }
+      /* back through the rotations: R(p)^T = R(-p) */
+      double* dq = J->dQ + qb;
+      oracle_rope(gqr, d, -rot_pos(p, (double)i), p->rope_theta, tmp);
+      for (int c = 0; c < d; ++c) dq[c] = tmp[c];
+      oracle_rope(gqc, d, -rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, tmp);
+      for (int c = 0; c < d; ++c) dq[c] += tmp[c];
+    }
+  }
+  int64_t kb = ((int64_t)b * p->Hkv + g) * (int64_t)T * d;
+  for (int j = 0; j < T; ++j) {
+    oracle_rope(gKrot + (size_t)j * d, d, -rot_pos(p, (double)j), p->rope_theta, tmp);
+    for (int c = 0; c < d; ++c) {
+      J->dK[kb + (int64_t)j * d + c] = tmp[c] + gKraw[(size_t)j * d + c];
+      J->dV[kb + (int64_t)j * d + c] = gV[(size_t)j * d + c];
+    }
+  }
+  free(Kraw);
+  free(Krot);
+  free(Vd);
+  free(gKrot);
+  free(gKraw);
+  free(gV);
+  free(m);
+  free(P);
+  free(dP);
+  free(cands);
+  free(work);
+}
+
+/* dQ [B, Hq, T, d], dK / dV [B, Hkv, T, d] in double: the gradients of
+ * sum(dO * O) with O the forward of the same parameters.  dO has the input
+ * encoding (p->dtype).  forced [B, Hq, T, k]: the top-k sets (NULL: selected
+ * here); the selection itself is a constant of the backward pass. */
+int oracle_bwd(const oracle_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+               const int32_t* forced, const void* dO, double* dQ, double* dK, double* dV, int nthreads) {
+  if (!p || p->d <= 0 || (p->d & 1) || p->T <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv) return OR_ERR_ARG;
+  bwd_job J;
+  J.p = p;
+  J.Q = Q;
+  J.K = K;
+  J.V = V;
+  J.dO = dO;
+  J.is_sep = is_sep;
+  J.forced = forced;
+  J.dQ = dQ;
+  J.dK = dK;
+  J.dV = dV;
+  run_parallel(bwd_one, &J, (int64_t)p->B * p->Hkv, nthreads);
   return OR_OK;
 }
 
