@@ -207,6 +207,34 @@ int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
 int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
                      void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace needed by sattn_bwd for *p. */
+int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes);
+
+/* Backward pass of sattn_fwd ("SepLLM", section 6.2: training runs the
+ * forward and the backward pass through the masked product): the gradients
+ * of sum(dO * O) with respect to Q, K and V for the same parameters, key
+ * sets and logits as the forward.  With P_ij = exp(s_ij - LSE_i) and
+ * dz_ij = P_ij (dO_i.v_j - dO_i.O_i) / sqrt(d):
+ *   dV_j = sum_i P_ij dO_i;
+ *   an uncapped pair (z = <R(i)q_i, R(j)k_j>) adds R(i)^T dz R(j)k_j to dq_i
+ *   and R(j)^T dz R(i)q_i to dk_j; a capped pair (L_pretrain > 0, i-j > L;
+ *   z = <R(L)q_i, k_j>, "LM-Infinite", section 方法) adds R(L)^T dz k_j to
+ *   dq_i and dz R(L)q_i to dk_j.
+ *   p          as for sattn_fwd (same validation).
+ *   Q, K, V    the forward's inputs, strides q/k/v_stride.
+ *   is_sep     [B, T] uint8 device flags or NULL, as for the forward.
+ *   topk_idx   [B, Hq, T, topk] int32 device: the forward's top-k selection
+ *              (required when topk > 0; the selection is a constant here).
+ *   O, lse     the forward's outputs (O strides o_stride; lse [B, Hq, T]).
+ *   dO         gradient of the loss w.r.t. O, strides o_stride.
+ *   dQ, dK, dV out, shaped and strided like Q, K, V (dtype of the inputs).
+ * fp32 only in this version (bf16: SATTN_ERR_UNSUPPORTED).  Deterministic:
+ * one kernel writes dq per query row, another dk and dv per key, no
+ * atomics.  Asynchronous on `stream`. */
+int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+              const int32_t* topk_idx, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
+              void* dV, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and reads the device status word of `ws` into
  * *device_status (SATTN_OK or SATTN_ERR_TIMEOUT).  Returns SATTN_ERR_CUDA if
  * the synchronisation itself failed (the CUDA error is then sticky). */

@@ -242,6 +242,36 @@ def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: in
     return out, lse
 
 
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+        do: torch.Tensor, *, n_start: int = 0, window: int = 0, L_pretrain: int = 0, rope_theta: float = 0.0,
+        topk: int = 0, is_sep: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
+    """Backward pass of ``fwd``: gradients of sum(do * o) for the forward's
+    inputs and outputs.  ``topk_idx`` is the forward's selection (needed when
+    topk > 0).  Returns (dq, dk, dv), shaped and strided like q, k, v."""
+    if do.stride() != o.stride() or do.dtype != o.dtype or do.shape != o.shape:
+        raise ValueError("do must match o in shape, dtype and strides")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for g, x in ((dq, q), (dk, k), (dv, v)):
+        if g.stride() != x.stride():
+            raise ValueError("gradient buffers must share the strides of their inputs")
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    if topk_idx is not None:
+        topk_idx = topk_idx.to(torch.int32).contiguous()
+    p = params(q, k, v, o, n_start=n_start, window=window, L_pretrain=L_pretrain, topk=topk, rope_theta=rope_theta,
+               with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale, alibi=alibi)
+    n = ctypes.c_size_t(0)
+    L = _lib.load()
+    _lib.check(L.sattn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)), "sattn_bwd_workspace_size")
+    nbytes = int(n.value)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = L.sattn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(topk_idx), _ptr(o), _ptr(lse),
+                     _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_bwd")
+    return dq, dk, dv
+
+
 def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> int:
     """Synchronise the current stream and read the device status word of the
     workspace (the cached one when None)."""

@@ -24,7 +24,8 @@ DTYPE_F32 = 1
 EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
-    "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_stream_status",
+    "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_bwd_workspace_size", "sattn_bwd",
+    "sattn_stream_status",
     "sattn_build_blockmap_noalloc", "sattn_selftest_wait_timeout", "sattn_profile_enable", "sattn_profile_collect",
 )
 
@@ -83,6 +84,10 @@ def load():
         L.sattn_decode_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_decode_fwd.restype = ctypes.c_int
         L.sattn_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sattn_bwd_workspace_size.restype = ctypes.c_int
+        L.sattn_bwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.sattn_bwd.restype = ctypes.c_int
+        L.sattn_bwd.argtypes = [P] + [vp] * 12 + [sz, vp]
         L.sattn_stream_status.restype = ctypes.c_int
         L.sattn_stream_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.sattn_build_blockmap_noalloc.restype = ctypes.c_int

@@ -884,6 +884,124 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   return cuda_rc(launch_decode(a, st));
 }
 
+// ---------------------------------------------------------------------------
+// backward pass
+// ---------------------------------------------------------------------------
+
+struct BwdPlan {
+  bool bf16 = true;
+  int nQT = 0, npos = 0;
+  Region status, tab, prefix, sep_pos, sep_count, ranges, dsum;
+  size_t total = 0;
+};
+
+static int plan_bwd(const sattn_params* p, BwdPlan* out) {
+  int rc = check_fwd_rules(p);
+  if (rc) return rc;
+  BwdPlan P;
+  P.bf16 = p->dtype == SATTN_DTYPE_BF16;
+  if (P.bf16) return SATTN_ERR_UNSUPPORTED;
+  P.nQT = (p->T + kTile - 1) / kTile;
+  P.npos = std::max(p->T, p->L_pretrain + 1);
+  const size_t B = p->B, Hq = p->Hq, T = p->T, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  if (p->with_separators) {
+    P.prefix = A.take(B * (T + 1) * 4);
+    P.sep_pos = A.take(B * T * 4);
+    P.sep_count = A.take(B * 4);
+    P.ranges = A.take(B * P.nQT * 2 * 4);
+  }
+  P.dsum = A.take(B * Hq * T * 4);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  BwdPlan P;
+  int rc = plan_bwd(p, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+              const int32_t* topk_idx, const void* O, const float* lse, const void* dO, void* dQ, void* dK, void* dV,
+              void* ws, size_t ws_bytes, void* stream) {
+  BwdPlan P;
+  int rc = plan_bwd(p, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV) return SATTN_ERR_INVALID_ARG;
+  if (is_sep && !p->with_separators) return SATTN_ERR_INVALID_ARG;
+  if (p->topk > 0 && !topk_idx) return SATTN_ERR_INVALID_ARG;  // the forward's selection is an input
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+  }
+  if (is_sep) {
+    FwdPlan F;
+    F.prefix = P.prefix;
+    rc = run_blockmap(p, F, is_sep, nullptr, at<int32_t>(ws, P.sep_pos), at<int32_t>(ws, P.sep_count),
+                      at<int32_t>(ws, P.ranges), ws, st);
+    if (rc) return rc;
+  }
+  BwdF32Args a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.Q = static_cast<const float*>(Q);
+  a.K = static_cast<const float*>(K);
+  a.V = static_cast<const float*>(V);
+  a.O = static_cast<const float*>(O);
+  a.dO = static_cast<const float*>(dO);
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.q_st = p->q_stride[2];
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  a.L = p->L_pretrain;
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.is_sep = is_sep;
+  a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
+  a.sep_count = is_sep ? at<int32_t>(ws, P.sep_count) : nullptr;
+  a.tk_idx = p->topk > 0 ? topk_idx : nullptr;
+  a.topk = p->topk;
+  a.alibi = p->alibi ? 1 : 0;
+  a.Dsum = at<float>(ws, P.dsum);
+  a.dQ = static_cast<float*>(dQ);
+  a.dK = static_cast<float*>(dK);
+  a.dV = static_cast<float*>(dV);
+  a.dq_sb = p->q_stride[0];
+  a.dq_sh = p->q_stride[1];
+  a.dq_st = p->q_stride[2];
+  a.dk_sb = p->k_stride[0];
+  a.dk_sh = p->k_stride[1];
+  a.dk_st = p->k_stride[2];
+  a.dv_sb = p->v_stride[0];
+  a.dv_sh = p->v_stride[1];
+  a.dv_st = p->v_stride[2];
+  ProfScope ps("bwd_f32", 2, st);
+  return cuda_rc(launch_bwd_f32(a, st));
+}
+
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {
   if (!ws || !device_status) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

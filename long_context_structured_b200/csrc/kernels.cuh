@@ -141,6 +141,34 @@ struct AttnF32Args {
 cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
+// backward pass, fp32 on CUDA cores
+// ---------------------------------------------------------------------------
+struct BwdF32Args {
+  int B, Hq, Hkv, T, d;
+  const float* Q;
+  const float* K;
+  const float* V;
+  const float* O;
+  const float* dO;           // strides of O
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st, o_sb, o_sh, o_st;
+  const float* lse;          // [B, Hq, T] natural log, from the forward
+  const float2* tab;         // null: no rotation
+  int L, n_start, window;
+  const uint8_t* is_sep;     // [B, T] or null
+  const int32_t* sep_pos;    // [B, T] or null
+  const int32_t* sep_count;  // [B]
+  const int32_t* tk_idx;     // [B, Hq, T, topk] or null: the forward's selection
+  int topk;
+  int alibi;
+  float* Dsum;               // [B, Hq, T] workspace: dO_i . O_i
+  float* dQ;
+  float* dK;
+  float* dV;
+  int64_t dq_sb, dq_sh, dq_st, dk_sb, dk_sh, dk_st, dv_sb, dv_sh, dv_st;
+};
+cudaError_t launch_bwd_f32(const BwdF32Args& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
 // K4: top-k middle-token selection
 // ---------------------------------------------------------------------------
 struct TopkArgs {

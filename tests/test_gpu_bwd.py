@@ -1,0 +1,105 @@
+"""GPU parity of the backward pass against the oracle's fp64 gradients.
+
+The forward runs on the GPU first (its O and LSE are inputs of the backward,
+as in training); the top-k sets are the GPU selection, handed to the oracle
+as forced sets.  Gradients are compared element by element with a bar
+relative to the gradient's largest magnitude (sums over many rows make dK and
+dV grow with the number of rows that keep a key): fp32 1e-4.
+"""
+import numpy as np
+import pytest
+import torch
+
+import long_context_structured_b200 as sa
+from long_context_structured_b200 import _lib, synth
+from _util import to_dev
+
+pytestmark = pytest.mark.gpu
+
+F32_GRAD_REL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def compare_grad(name, got, ref, rel, mean_rel=None):
+    scale = max(1.0, float(np.abs(ref).max()))
+    err = np.abs(got - ref)
+    mx, mn = float(err.max()) / scale, float(err.mean()) / scale
+    msg = "%s: max-abs/scale %.3e (bar %.1e), mean-abs/scale %.3e, scale %.3g" % (name, mx, rel, mn, scale)
+    print(msg)
+    assert np.isfinite(got).all() and mx <= rel and (mean_rel is None or mn <= mean_rel), msg
+
+
+def _kw(wl):
+    return dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta,
+                rope_pos_scale=wl.rope_pos_scale, alibi=wl.alibi)
+
+
+def _run(oracle_mod, wl, seed, rel, mean_rel=None):
+    inp = synth.make_inputs(wl, seed=seed)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    g = np.random.default_rng(seed + 100)
+    if wl.dtype == "f32":
+        dO_h = g.standard_normal(inp["q"].shape).astype(np.float32)
+    else:
+        dO_h = (g.standard_normal(inp["q"].shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    dO = to_dev(dO_h)
+    idx = None
+    if wl.topk > 0:
+        idx, z = sa.topk_select(q, k, topk=wl.topk, is_sep=sep, **_kw(wl))
+        O, lse = sa.fwd(q, k, v, topk=wl.topk, is_sep=sep, topk_idx=idx, topk_logit=z, **_kw(wl))
+    else:
+        O, lse = sa.fwd(q, k, v, is_sep=sep, **_kw(wl))
+    dq, dk, dv = sa.bwd(q, k, v, O, lse, dO, topk=wl.topk, is_sep=sep, topk_idx=idx, **_kw(wl))
+    torch.cuda.synchronize()
+    assert sa.stream_status() == 0
+    forced = None if idx is None else idx.cpu().numpy()
+    ref = oracle_mod.bwd(oracle_mod.params_of(wl), inp["q"], inp["k"], inp["v"], inp["is_sep"], dO_h,
+                         forced_topk=forced)
+    for name, t, r in (("dQ", dq, ref[0]), ("dK", dk, ref[1]), ("dV", dv, ref[2])):
+        compare_grad(name, t.float().cpu().numpy().astype(np.float64), r, rel, mean_rel)
+    return (dq, dk, dv), (q, k, v, O, lse, dO, sep, idx)
+
+
+F32_CASES = [
+    ("lambda_capped_gqa", dict(B=1, Hq=4, Hkv=2, T=300, d=128, n_start=4, window=40, L_pretrain=40,
+                               rope_theta=1e4, sink_scale=8.0)),
+    ("sep_topk_cap_above_window_pi", dict(B=2, Hq=2, Hkv=1, T=257, d=64, n_start=2, window=20, L_pretrain=40,
+                                          rope_theta=1e4, topk=3, sep_rate=0.1, rope_pos_scale=0.5)),
+    ("alibi_sep", dict(B=1, Hq=4, Hkv=4, T=200, d=128, n_start=3, window=30, L_pretrain=30, sep_rate=0.15,
+                       alibi=True)),
+    ("causal_no_rope", dict(B=1, Hq=2, Hkv=2, T=150, d=64, n_start=0, window=1000)),
+    ("tiny", dict(B=1, Hq=1, Hkv=1, T=3, d=64, n_start=4, window=1, rope_theta=1e4)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", F32_CASES, ids=[c[0] for c in F32_CASES])
+def test_bwd_f32(oracle_mod, name, cfg):
+    wl = synth.Workload(name=name, dtype="f32", **cfg)
+    _run(oracle_mod, wl, 21, F32_GRAD_REL)
+
+
+def test_bwd_f32_sepllm_config(oracle_mod):
+    """The fp32 SepLLM-mask layer (T=1024, d=64, separators at rate 0.08)."""
+    _run(oracle_mod, synth.WORKLOADS["c1_f32_sep"], 0, F32_GRAD_REL)
+
+
+def test_bwd_f32_deterministic(oracle_mod):
+    wl = synth.Workload(name="det", B=1, Hq=2, Hkv=1, T=300, d=128, dtype="f32", n_start=4, window=30,
+                        L_pretrain=30, rope_theta=1e4, sep_rate=0.1)
+    grads, (q, k, v, O, lse, dO, sep, idx) = _run(oracle_mod, wl, 5, F32_GRAD_REL)
+    again = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, **_kw(wl))
+    assert all(torch.equal(a, b) for a, b in zip(grads, again))
+
+
+def test_bwd_rejects_missing_topk_selection():
+    q = torch.zeros((1, 1, 64, 64), dtype=torch.float32, device="cuda")
+    lse = torch.zeros((1, 1, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(_lib.SattnError):
+        sa.bwd(q, q, q, q, lse, q, window=4, L_pretrain=4, topk=2)
