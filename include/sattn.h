@@ -228,9 +228,12 @@ int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes);
  *   O, lse     the forward's outputs (O strides o_stride; lse [B, Hq, T]).
  *   dO         gradient of the loss w.r.t. O, strides o_stride.
  *   dQ, dK, dV out, shaped and strided like Q, K, V (dtype of the inputs).
- * fp32 only in this version (bf16: SATTN_ERR_UNSUPPORTED).  Deterministic:
- * one kernel writes dq per query row, another dk and dv per key, no
- * atomics.  Asynchronous on `stream`. */
+ * fp32: CUDA cores, one kernel writes dq per query row, another dk and dv
+ * per key.  bf16: tensor cores (a dq kernel per 128-row query tile, a dk/dv
+ * kernel per 128-key tile of positions or of compacted separators, both
+ * recomputing P from lse), the sink keys on CUDA cores, fp32 partial sums
+ * combined in a fixed order; bf16 with topk > 0: SATTN_ERR_UNSUPPORTED.
+ * Deterministic (no atomics).  Asynchronous on `stream`. */
 int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
               const int32_t* topk_idx, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
               void* dV, void* ws, size_t ws_bytes, void* stream);

@@ -889,9 +889,9 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
 // ---------------------------------------------------------------------------
 
 struct BwdPlan {
-  bool bf16 = true;
-  int nQT = 0, npos = 0;
-  Region status, tab, prefix, sep_pos, sep_count, ranges, dsum;
+  FwdPlan F;  // regions shared with the forward's steps (status, table, prep products, block map, gather)
+  int nRB = 0;
+  Region dsum, nlse2, sink_ds, sink_p, sink_part, dq_side, dk_band, dv_band, dk_sep, dv_sep;
   size_t total = 0;
 };
 
@@ -899,24 +899,197 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
   int rc = check_fwd_rules(p);
   if (rc) return rc;
   BwdPlan P;
-  P.bf16 = p->dtype == SATTN_DTYPE_BF16;
-  if (P.bf16) return SATTN_ERR_UNSUPPORTED;
-  P.nQT = (p->T + kTile - 1) / kTile;
-  P.npos = std::max(p->T, p->L_pretrain + 1);
-  const size_t B = p->B, Hq = p->Hq, T = p->T, d = p->d;
+  FwdPlan& F = P.F;
+  F.bf16 = p->dtype == SATTN_DTYPE_BF16;
+  if (F.bf16 && p->topk > 0) return SATTN_ERR_UNSUPPORTED;  // top-k backward: fp32 path only
+  F.nQT = (p->T + kTile - 1) / kTile;
+  F.Tpad = F.nQT * kTile;
+  F.npos = std::max(p->T, p->L_pretrain + 1);
+  F.n_sink = std::min(p->n_start, p->T);
+  F.capped_sep = p->L_pretrain > 0 && p->with_separators;
+  F.need_qc = F.bf16 && F.capped_sep;
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d, Tpad = F.Tpad;
   Alloc A;
-  P.status = A.take(kStatusBytes);
-  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  F.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) F.tab = A.take((size_t)F.npos * (d / 2) * sizeof(float2));
   if (p->with_separators) {
-    P.prefix = A.take(B * (T + 1) * 4);
-    P.sep_pos = A.take(B * T * 4);
-    P.sep_count = A.take(B * 4);
-    P.ranges = A.take(B * P.nQT * 2 * 4);
+    F.prefix = A.take(B * (T + 1) * 4);
+    F.sep_pos = A.take(B * T * 4);
+    F.sep_count = A.take(B * 4);
+    F.ranges = A.take(B * F.nQT * 2 * 4);
   }
-  P.dsum = A.take(B * Hq * T * 4);
+  if (!F.bf16) {
+    P.dsum = A.take(B * Hq * T * 4);
+  } else {
+    F.qr = A.take(B * Hq * T * d * 2);
+    F.kr = A.take(B * Hkv * T * d * 2);
+    if (F.need_qc) F.qc = A.take(B * Hq * T * d * 2);
+    if (p->with_separators) {
+      F.ks = A.take(B * Hkv * Tpad * d * 2);
+      F.vs = A.take(B * Hkv * Tpad * d * 2);
+      P.dk_sep = A.take(B * Hkv * Tpad * d * 4);
+      P.dv_sep = A.take(B * Hkv * Tpad * d * 4);
+    }
+    P.dsum = A.take(B * Hq * Tpad * 4);
+    P.nlse2 = A.take(B * Hq * Tpad * 4);
+    if (F.n_sink > 0) {
+      F.sink = A.take(B * Hq * T * F.n_sink * 4);
+      P.sink_ds = A.take(B * Hq * T * F.n_sink * 4);
+      P.sink_p = A.take(B * Hq * T * F.n_sink * 4);
+      P.nRB = (int)((T + bwd_sink_row_block() - 1) / bwd_sink_row_block());
+      P.sink_part = A.take(B * Hkv * F.n_sink * (size_t)P.nRB * 2 * d * 4);
+    }
+    if (F.n_sink > 0 || F.capped_sep) P.dq_side = A.take(B * Hq * T * d * 4);
+    P.dk_band = A.take(B * Hkv * T * d * 4);
+    P.dv_band = A.take(B * Hkv * T * d * 4);
+  }
   P.total = A.cur;
   *out = P;
   return SATTN_OK;
+}
+
+static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, const void* K, const void* V,
+                        const uint8_t* is_sep, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
+                        void* dV, void* ws, cudaStream_t st) {
+  const FwdPlan& F = P.F;
+  const int64_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  int rc = run_prep_bf16(p, F, Q, K, ws, F.n_sink > 0, false, st);
+  if (rc) return rc;
+  BwdMaps m;
+  if (!make_map(&m.q, at<void>(ws, F.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.k, at<void>(ws, F.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.v, V, p->d, p->T, Hkv, B, p->v_stride[2], p->v_stride[1], p->v_stride[0])) return SATTN_ERR_CUDA;
+  if (!make_map(&m.dO, dO, p->d, p->T, Hq, B, p->o_stride[2], p->o_stride[1], p->o_stride[0])) return SATTN_ERR_CUDA;
+  m.qc = m.q;
+  m.kg = m.k;
+  m.vg = m.v;
+  int32_t* sep_pos = at<int32_t>(ws, F.sep_pos);
+  int32_t* sep_count = at<int32_t>(ws, F.sep_count);
+  int32_t* ranges = at<int32_t>(ws, F.ranges);
+  if (is_sep) {
+    rc = run_blockmap(p, F, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
+    if (rc) return rc;
+    GatherArgs ga{};
+    ga.B = p->B;
+    ga.Hkv = p->Hkv;
+    ga.T = p->T;
+    ga.Tpad = F.Tpad;
+    ga.d = p->d;
+    if (F.capped_sep) {
+      ga.Ksrc = static_cast<const __nv_bfloat16*>(K);
+      ga.k_sb = p->k_stride[0];
+      ga.k_sh = p->k_stride[1];
+      ga.k_st = p->k_stride[2];
+      if (!make_map(&m.qc, at<void>(ws, F.qc), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+    } else {
+      ga.Ksrc = at<__nv_bfloat16>(ws, F.kr);
+      ga.k_sb = Hkv * T * d;
+      ga.k_sh = T * d;
+      ga.k_st = d;
+    }
+    ga.Vsrc = static_cast<const __nv_bfloat16*>(V);
+    ga.v_sb = p->v_stride[0];
+    ga.v_sh = p->v_stride[1];
+    ga.v_st = p->v_stride[2];
+    ga.sep_pos = sep_pos;
+    ga.sep_count = sep_count;
+    ga.Ks = at<__nv_bfloat16>(ws, F.ks);
+    ga.Vs = at<__nv_bfloat16>(ws, F.vs);
+    {
+      ProfScope ps("sep_gather", 1, st);
+      SATTN_TRY(launch_sep_gather(ga, st));
+    }
+    if (!make_map(&m.kg, ga.Ks, p->d, F.Tpad, Hkv, B, d, (int64_t)F.Tpad * d, Hkv * F.Tpad * d)) return SATTN_ERR_CUDA;
+    if (!make_map(&m.vg, ga.Vs, p->d, F.Tpad, Hkv, B, d, (int64_t)F.Tpad * d, Hkv * F.Tpad * d)) return SATTN_ERR_CUDA;
+  }
+  BwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.nQT = F.nQT;
+  a.Tpad = F.Tpad;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.n_start = p->n_start;
+  a.window = p->window;
+  a.L = p->L_pretrain;
+  a.alibi = p->alibi ? 1 : 0;
+  a.alibi_cap = p->L_pretrain;
+  a.tab = F.tab.bytes ? at<float2>(ws, F.tab) : nullptr;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.O = static_cast<const __nv_bfloat16*>(O);
+  a.dO = static_cast<const __nv_bfloat16*>(dO);
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.q_st = p->q_stride[2];
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.Qr = at<__nv_bfloat16>(ws, F.qr);
+  a.Qc = F.qc.bytes ? at<__nv_bfloat16>(ws, F.qc) : nullptr;
+  a.sink_z = F.n_sink > 0 ? at<float>(ws, F.sink) : nullptr;
+  a.n_sink = F.n_sink;
+  a.gather = is_sep ? 1 : 0;
+  a.capped_sep = (is_sep && F.capped_sep) ? 1 : 0;
+  a.sep_pos = is_sep ? sep_pos : nullptr;
+  a.sep_count = is_sep ? sep_count : nullptr;
+  a.sep_prefix = is_sep ? at<int32_t>(ws, F.prefix) : nullptr;
+  a.ranges = is_sep ? ranges : nullptr;
+  a.Dsum = at<float>(ws, P.dsum);
+  a.nlse2 = at<float>(ws, P.nlse2);
+  a.sink_ds = F.n_sink > 0 ? at<float>(ws, P.sink_ds) : nullptr;
+  a.sink_p = F.n_sink > 0 ? at<float>(ws, P.sink_p) : nullptr;
+  a.sink_part = F.n_sink > 0 ? at<float>(ws, P.sink_part) : nullptr;
+  a.nRB = P.nRB;
+  a.dq_side = P.dq_side.bytes ? at<float>(ws, P.dq_side) : nullptr;
+  a.dk_band = at<float>(ws, P.dk_band);
+  a.dv_band = at<float>(ws, P.dv_band);
+  a.dk_sep = is_sep ? at<float>(ws, P.dk_sep) : nullptr;
+  a.dv_sep = is_sep ? at<float>(ws, P.dv_sep) : nullptr;
+  a.dQ = static_cast<__nv_bfloat16*>(dQ);
+  a.dK = static_cast<__nv_bfloat16*>(dK);
+  a.dV = static_cast<__nv_bfloat16*>(dV);
+  a.status = at<int32_t>(ws, F.status);
+  {
+    ProfScope ps("bwd_rowstats", 1, st);
+    SATTN_TRY(launch_bwd_rowstats(a, st));
+  }
+  if (F.n_sink > 0) {
+    ProfScope ps("bwd_sink_rows", 1, st);
+    SATTN_TRY(launch_bwd_sink_rows(a, st));
+  }
+  a.side_valid = F.n_sink > 0;
+  if (a.capped_sep) {
+    a.dq_mode = 1;
+    ProfScope ps("bwd_dq", 1, st);
+    SATTN_TRY(launch_bwd_dq(a, m, st));
+    a.side_valid = true;
+  }
+  a.dq_mode = 0;
+  {
+    ProfScope ps("bwd_dq", 1, st);
+    SATTN_TRY(launch_bwd_dq(a, m, st));
+  }
+  {
+    ProfScope ps("bwd_dkv", 1, st);
+    SATTN_TRY(launch_bwd_dkv(a, m, st));
+  }
+  if (F.n_sink > 0) {
+    ProfScope ps("bwd_sink_keys", 1, st);
+    SATTN_TRY(launch_bwd_sink_keys(a, st));
+  }
+  ProfScope ps("bwd_combine", 1, st);
+  return cuda_rc(launch_bwd_combine(a, st));
 }
 
 int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes) {
@@ -938,17 +1111,19 @@ int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V
   if (is_sep && !p->with_separators) return SATTN_ERR_INVALID_ARG;
   if (p->topk > 0 && !topk_idx) return SATTN_ERR_INVALID_ARG;  // the forward's selection is an input
   if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  const FwdPlan& F = P.F;
+  if (F.bf16 && (!pointers_ok_bf16(Q, K, V) || !pointers_ok_bf16(O, dO, dQ) || !aligned16(dK) || !aligned16(dV)))
+    return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
-  if (P.tab.bytes) {
+  if (F.bf16) return run_bwd_bf16(p, P, Q, K, V, is_sep, O, lse, dO, dQ, dK, dV, ws, st);
+  if (F.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
-    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+    SATTN_TRY(launch_rope_table(at<float2>(ws, F.tab), F.npos, p->d, p->rope_theta, pos_scale(p), st));
   }
   if (is_sep) {
-    FwdPlan F;
-    F.prefix = P.prefix;
-    rc = run_blockmap(p, F, is_sep, nullptr, at<int32_t>(ws, P.sep_pos), at<int32_t>(ws, P.sep_count),
-                      at<int32_t>(ws, P.ranges), ws, st);
+    rc = run_blockmap(p, F, is_sep, nullptr, at<int32_t>(ws, F.sep_pos), at<int32_t>(ws, F.sep_count),
+                      at<int32_t>(ws, F.ranges), ws, st);
     if (rc) return rc;
   }
   BwdF32Args a{};
@@ -975,13 +1150,13 @@ int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.o_sh = p->o_stride[1];
   a.o_st = p->o_stride[2];
   a.lse = lse;
-  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  a.tab = F.tab.bytes ? at<float2>(ws, F.tab) : nullptr;
   a.L = p->L_pretrain;
   a.n_start = p->n_start;
   a.window = p->window;
   a.is_sep = is_sep;
-  a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
-  a.sep_count = is_sep ? at<int32_t>(ws, P.sep_count) : nullptr;
+  a.sep_pos = is_sep ? at<int32_t>(ws, F.sep_pos) : nullptr;
+  a.sep_count = is_sep ? at<int32_t>(ws, F.sep_count) : nullptr;
   a.tk_idx = p->topk > 0 ? topk_idx : nullptr;
   a.topk = p->topk;
   a.alibi = p->alibi ? 1 : 0;

@@ -169,6 +169,68 @@ struct BwdF32Args {
 cudaError_t launch_bwd_f32(const BwdF32Args& a, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
+// backward pass, bf16 on tensor cores (sinks on CUDA cores)
+// ---------------------------------------------------------------------------
+struct BwdArgs {
+  int B, Hq, Hkv, T, d, nQT, Tpad;
+  float scale_log2;             // log2(e) / sqrt(d)
+  int n_start, window, L;       // L: distance cap (0 = none)
+  int alibi, alibi_cap;
+  const float2* tab;            // rotary table (null: no rotation)
+  // the forward's inputs and outputs (raw layouts, explicit strides)
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const __nv_bfloat16* O;
+  const __nv_bfloat16* dO;      // strides of O
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st, o_sb, o_sh, o_st;
+  const float* lse;             // [B, Hq, T] natural log
+  // products of the prep pass
+  const __nv_bfloat16* Qr;      // [B, Hq, T, d] R(i) q_i
+  const __nv_bfloat16* Qc;      // [B, Hq, T, d] R(L) q_i (capped separators)
+  const float* sink_z;          // [B, Hq, T, n_sink] fp32 sink logits (capped rule, ALiBi bias included)
+  int n_sink;
+  // separators (compacted by the block map)
+  int gather;                   // 1: separators present
+  int capped_sep;               // gathered tiles take Qc and raw keys
+  const int32_t* sep_pos;       // [B, T]
+  const int32_t* sep_count;     // [B]
+  const int32_t* sep_prefix;    // [B, T+1]
+  const int32_t* ranges;        // [B, nQT, 2]
+  // row statistics, padded to Tpad rows (pad: D = 0, -lse2 = -inf)
+  float* Dsum;                  // [B, Hq, Tpad] dO_i . O_i
+  float* nlse2;                 // [B, Hq, Tpad] -LSE_i * log2(e)
+  // sinks
+  float* sink_ds;               // [B, Hq, T, n_sink] dS of the sink pairs (unscaled)
+  float* sink_p;                // [B, Hq, T, n_sink] P of the sink pairs
+  float* sink_part;             // [B, Hkv, n_sink, nRB, 2, d] partial key-side sums per row block
+  int nRB;                      // row blocks of the sink reduction
+  // fp32 scratch
+  float* dq_side;               // [B, Hq, T, d] dq from sinks and capped separators (raw frame)
+  float* dk_band;               // [B, Hkv, T, d] band-tile dk (raw frame)
+  float* dv_band;
+  float* dk_sep;                // [B, Hkv, Tpad, d] separator dk, compacted order (raw frame)
+  float* dv_sep;
+  // outputs (strides of Q, K, V)
+  __nv_bfloat16* dQ;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  int32_t* status;
+  int dq_mode;                  // dq kernel: 0 band (+ uncapped separators), 1 capped separators only
+  bool side_valid;              // dq_side holds data (else it is not read)
+};
+struct BwdMaps {
+  CUtensorMap q, qc, dO, k, v, kg, vg;
+};
+cudaError_t launch_bwd_rowstats(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_sink_rows(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_sink_keys(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_dq(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
+cudaError_t launch_bwd_dkv(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
+cudaError_t launch_bwd_combine(const BwdArgs& a, cudaStream_t st);
+int bwd_sink_row_block();  // rows per partial sum of the sink-key reduction
+
+// ---------------------------------------------------------------------------
 // K4: top-k middle-token selection
 // ---------------------------------------------------------------------------
 struct TopkArgs {

@@ -98,6 +98,39 @@ def test_bwd_f32_deterministic(oracle_mod):
     assert all(torch.equal(a, b) for a, b in zip(grads, again))
 
 
+BF16_GRAD_REL, BF16_GRAD_MEAN_REL = 2e-2, 2e-3
+
+BF16_CASES = [
+    ("causal_no_rope", dict(B=1, Hq=2, Hkv=2, T=300, d=128, n_start=0, window=1000)),
+    ("lambda_capped_sinks_gqa", dict(B=1, Hq=4, Hkv=2, T=700, d=128, n_start=4, window=100, L_pretrain=100,
+                                     rope_theta=1e4, sink_scale=8.0)),
+    ("sep_uncapped_d64", dict(B=2, Hq=4, Hkv=2, T=600, d=64, n_start=1, window=37, rope_theta=1e4, sep_rate=0.1)),
+    ("sep_capped", dict(B=1, Hq=2, Hkv=2, T=513, d=128, n_start=4, window=64, L_pretrain=64, rope_theta=1e4,
+                        sep_rate=0.3)),
+    ("alibi_sep_capped", dict(B=1, Hq=4, Hkv=1, T=400, d=128, n_start=4, window=64, L_pretrain=64, sep_rate=0.2,
+                              alibi=True)),
+    ("pos_interp_gqa", dict(B=1, Hq=2, Hkv=1, T=500, d=128, n_start=4, window=64, L_pretrain=64, rope_theta=1e4,
+                            rope_pos_scale=0.5)),
+    ("window0_all_seps", dict(B=1, Hq=2, Hkv=2, T=257, d=128, n_start=1, window=0, sep_rate=1.0)),
+    ("tiny", dict(B=1, Hq=1, Hkv=1, T=5, d=128, n_start=4, window=2, rope_theta=1e4)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", BF16_CASES, ids=[c[0] for c in BF16_CASES])
+def test_bwd_bf16(oracle_mod, name, cfg):
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    _run(oracle_mod, wl, 31, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
+
+
+def test_bwd_bf16_deterministic(oracle_mod):
+    wl = synth.Workload(name="det16", B=1, Hq=4, Hkv=2, T=600, d=128, dtype="bf16", n_start=4, window=64,
+                        L_pretrain=64, rope_theta=1e4, sep_rate=0.1)
+    grads, (q, k, v, O, lse, dO, sep, idx) = _run(oracle_mod, wl, 8, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
+    again = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, **_kw(wl))
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(grads, again))
+
+
 def test_bwd_rejects_missing_topk_selection():
     q = torch.zeros((1, 1, 64, 64), dtype=torch.float32, device="cuda")
     lse = torch.zeros((1, 1, 64), dtype=torch.float32, device="cuda")
