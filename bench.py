@@ -42,6 +42,8 @@ from long_context_structured_b200 import synth  # noqa: E402
 
 # decoding steps (one new token per sequence) over the caches of these workloads
 DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
+BWD_ALIASES = {"c2b": "c2_lminf_16k", "c3b": "c3_sepllm_gqa_8k"}
+BWD_FLOPS_PER_PAIR_D = 10  # backward: S recomputed, dP, dV, dK, dQ -- five products of 2d FLOPs per pair
 WORKLOAD_ALIASES = {"c2": "c2_lminf_16k", "c3": "c3_sepllm_gqa_8k", "c4": "c4_lminf_topk_32k",
                     "c5": "c5_segmented_32k"}
 DEFAULT_WORKLOAD = "c2"
@@ -134,9 +136,11 @@ def describe(wl) -> str:
     return s
 
 
-def config_dict(wl, pairs_per_rank, decode=False, n_copies=0):
-    c = {"workload": ("decoding step (one new token per sequence at position T-1) over the cache of " if decode
-                      else "") + describe(wl), "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d}
+def config_dict(wl, pairs_per_rank, decode=False, n_copies=0, backward=False):
+    prefix = ("decoding step (one new token per sequence at position T-1) over the cache of " if decode else
+              "backward pass (dQ, dK, dV of sum(dO*O); %d FLOPs per kept pair per d) of " % BWD_FLOPS_PER_PAIR_D
+              if backward else "")
+    c = {"workload": prefix + describe(wl), "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d}
     if wl.segmented:
         c.update({"S": wl.seg_S, "M": wl.seg_M, "R": wl.seg_R, "retr_block": wl.retr_block,
                   "long_heads": len(wl.long_heads), "rope_theta": wl.rope_theta})
@@ -369,6 +373,92 @@ class DecodeJob:
         return {"decode": ("hbm", self.kv_bytes + q_o, "B")}
 
 
+def sink_pairs(wl) -> int:
+    """(q, k) pairs with k in the starting span j < n_start (fp32 side keys)."""
+    i = np.arange(wl.T, dtype=np.int64)
+    return int(np.minimum(min(wl.n_start, wl.T), i + 1).sum()) * wl.B * wl.Hq
+
+
+class BwdJob:
+    """One backward step of a workload: the forward's O and LSE and a seeded
+    dO are resident; each step computes dQ, dK, dV through sattn_bwd."""
+
+    def __init__(self, wl, seed, dev):
+        import torch
+
+        import long_context_structured_b200 as sa
+        self.sa, self.torch, self.wl, self.dev = sa, torch, wl, dev
+        inp = synth.make_inputs(wl, seed=seed)
+        self.inp = inp
+        f32 = wl.dtype == "f32"
+        to_t = (lambda a: torch.from_numpy(a)) if f32 else \
+            (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16))
+        self.host = {x: to_t(inp[x]).pin_memory() for x in ("q", "k", "v")}
+        g = np.random.default_rng(seed + 7)
+        do = g.standard_normal(inp["q"].shape).astype(np.float32)
+        self.host["do"] = (torch.from_numpy(do) if f32 else torch.from_numpy(do).to(torch.bfloat16)).pin_memory()
+        if inp["is_sep"] is not None:
+            self.host["is_sep"] = torch.from_numpy(inp["is_sep"]).pin_memory()
+        self.devt = {x: t.to(dev) for x, t in self.host.items()}
+        d = self.devt
+        self.kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta)
+        self.O, self.lse = sa.fwd(d["q"], d["k"], d["v"], is_sep=d.get("is_sep"), **self.kw)
+        torch.cuda.synchronize()
+        self.host["o"] = self.O.cpu().pin_memory()
+        self.host["lse"] = self.lse.cpu().pin_memory()
+        self.grads = (torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"]))
+        self.pairs = unmasked_pairs(wl, inp["is_sep"])
+        self.tc_pairs = self.pairs - sink_pairs(wl)
+        self.flops = float(BWD_FLOPS_PER_PAIR_D) * wl.d * self.pairs
+        self.n_sep = 0 if inp["is_sep"] is None else int(inp["is_sep"][:, wl.n_start:].sum())
+
+    def step(self):
+        d = self.devt
+        self.sa.bwd(d["q"], d["k"], d["v"], self.O, self.lse, d["do"], is_sep=d.get("is_sep"), grads=self.grads,
+                    **self.kw)
+
+    def host_step(self):
+        """Inputs from pinned host memory, the backward call, the gradients
+        back into pinned host memory."""
+        torch = self.torch
+        h = self.host
+        dv = {x: t.to(self.dev, non_blocking=True) for x, t in h.items()}
+        grads = self.sa.bwd(dv["q"], dv["k"], dv["v"], dv["o"], dv["lse"], dv["do"], is_sep=dv.get("is_sep"),
+                            **self.kw)
+        outs = []
+        for t in grads:
+            o = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            o.copy_(t, non_blocking=True)
+            outs.append(o)
+        torch.cuda.current_stream(self.dev).synchronize()
+        return outs
+
+    def h2d_bytes(self):
+        return int(sum(t.nbytes for t in self.host.values()))
+
+    def group_work(self):
+        wl = self.wl
+        if wl.dtype == "f32":
+            return {"bwd_f32": ("tensor", self.flops, "FLOP")}
+        e = 2
+        rows_q = wl.B * wl.Hq * wl.T * wl.d * e
+        rows_k = wl.B * wl.Hkv * wl.T * wl.d * e
+        out = {"bwd_dq": ("tensor", 6.0 * wl.d * self.tc_pairs, "FLOP"),      # S, dP, dQ
+               "bwd_dkv": ("tensor", 8.0 * wl.d * self.tc_pairs, "FLOP"),     # S^T, dP^T, dV, dK
+               # O, dO read; D and -LSE written; with sinks also dq_side (fp32) and per-pair P, dS
+               "bwd_rows": ("hbm", 2 * rows_q + 8 * wl.B * wl.Hq * wl.T + (
+                   2 * rows_q + 8 * min(wl.n_start, wl.T) * wl.B * wl.Hq * wl.T if wl.n_start else 0), "B"),
+               # fp32 band dk/dv read, bf16 dk/dv written (separator and sink parts are small)
+               "bwd_combine": ("hbm", 2 * rows_k * 2 + 2 * rows_k, "B")}
+        if wl.n_start:  # Q and dO read, P and dS of the sink pairs read
+            out["bwd_sink_keys"] = ("hbm", 2 * rows_q + 8 * min(wl.n_start, wl.T) * wl.B * wl.Hq * wl.T, "B")
+        prep = 2 * rows_q + 2 * rows_k + wl.B * wl.Hq * wl.T * min(wl.n_start, wl.T) * 4
+        if wl.L_pretrain > 0 and wl.sep_rate > 0:
+            prep += rows_q
+        out["prep_rope"] = ("hbm", prep, "B")
+        return out
+
+
 def roofline_of(group, work, avg_ms, peaks, peak_src):
     bound, amount, unit = work
     if bound == "tensor":
@@ -415,7 +505,10 @@ def kernel_name(wl, group):
         return "attn_tc2_kernel<%d>" % wl.d if wl.seg_S % 256 == 0 else "attn_tc3_kernel<%d>" % wl.d
     return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel",
             "decode": "decode_partial_kernel + decode_combine_kernel",
-            "sep_gather": "sep_gather_kernel"}.get(group, group)
+            "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % wl.d,
+            "bwd_dkv": "bwd_dkv_kernel<%d>" % wl.d, "bwd_f32": "bwd_f32_dq_kernel + bwd_f32_dkv_kernel",
+            "bwd_rows": "bwd_rows_kernel", "bwd_combine": "bwd_combine_kernel",
+            "bwd_sink_keys": "bwd_sink_keys_kernel"}.get(group, group)
 
 
 def run_ours(args):
@@ -437,11 +530,13 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     decode = args.workload in DECODE_ALIASES
-    wl = synth.WORKLOADS[(DECODE_ALIASES if decode else WORKLOAD_ALIASES).get(args.workload, args.workload)]
+    backward = args.workload in BWD_ALIASES
+    aliases = DECODE_ALIASES if decode else (BWD_ALIASES if backward else WORKLOAD_ALIASES)
+    wl = synth.WORKLOADS[aliases.get(args.workload, args.workload)]
     if args.heads:
         wl = wl.scaled(Hq=args.heads, Hkv=max(1, args.heads * wl.Hkv // wl.Hq),
                        long_heads=tuple(h for h in wl.long_heads if h < args.heads))
-    job = (DecodeJob if decode else Job)(wl, seed=rank, dev=dev)
+    job = (DecodeJob if decode else (BwdJob if backward else Job))(wl, seed=rank, dev=dev)
     lib = _lib.load()
 
     for _ in range(args.warmup):
@@ -533,12 +628,14 @@ def run_ours(args):
            "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
            "path": ("long_context_structured_b200.decode_fwd: query from pinned host memory, device-resident cache, "
                     "outputs into pinned host memory") if decode else
+                   ("long_context_structured_b200.bwd: Q, K, V, O, LSE, dO from pinned host memory, dQ, dK, dV "
+                    "into pinned host memory") if backward else
                    ("long_context_structured_b200.%s on pinned host tensors (outputs into pinned host memory)"
                     % ("segment_fwd" if wl.segmented else "fwd"))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, job.inp, args.cpu_rows, decode=decode)
+        cpu = cpu_baseline_bwd(wl) if backward else cpu_baseline(wl, job.inp, args.cpu_rows, decode=decode)
 
     if world > 1:
         dist.barrier()
@@ -549,9 +646,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16",
+        "vs_baseline": None, "dtype": "f32" if wl.dtype == "f32" else "bf16",
         "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
-        "config": config_dict(wl, job.pairs, decode=decode, n_copies=getattr(job, "n_copies", 0)),
+        "config": config_dict(wl, job.pairs, decode=decode, n_copies=getattr(job, "n_copies", 0), backward=backward),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_bf16_peak": round(value / world / peak, 4),
         "roofline": roof,
@@ -625,6 +722,32 @@ def cpu_baseline(wl, inp, n_rows, decode=False):
             "seconds": round(dt, 2)}
 
 
+def bwd_sample(wl):
+    """A bounded sample of a backward workload for the CPU oracle: the same
+    mask parameters on one kv-head group of one sequence, T cut to 4096."""
+    return wl.scaled(B=1, Hq=wl.Hq // wl.Hkv, Hkv=1, T=min(wl.T, 4096))
+
+
+def cpu_baseline_bwd(wl):
+    from oracle import oracle as O
+    O.build()
+    sw = bwd_sample(wl)
+    inp = synth.make_inputs(sw, seed=0)
+    g = np.random.default_rng(3)
+    do = g.standard_normal(inp["q"].shape).astype(np.float32)
+    if sw.dtype == "bf16":
+        do = (do.view(np.uint32) >> 16).astype(np.uint16)
+    nthreads = O.nthreads_default()
+    t0 = time.perf_counter()
+    O.bwd(O.params_of(sw), inp["q"], inp["k"], inp["v"], inp["is_sep"], do, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    flops = float(BWD_FLOPS_PER_PAIR_D) * sw.d * unmasked_pairs(sw, inp["is_sep"])
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": "backward of one kv-head group (%d query heads), B=1, T=%d, same mask parameters, fp64, "
+                      "%.1f s (the oracle's backward runs one thread per kv head)" % (sw.Hq, sw.T, dt),
+            "seconds": round(dt, 2)}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -632,6 +755,20 @@ def run_reference(args):
     from oracle import oracle as O
     O.build()
     decode = args.workload in DECODE_ALIASES
+    if args.workload in BWD_ALIASES:
+        wl = synth.WORKLOADS[BWD_ALIASES[args.workload]]
+        t0 = time.perf_counter()
+        for _ in range(args.warmup + args.steps):
+            cpu = cpu_baseline_bwd(wl)
+        line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "TFLOP/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round((time.perf_counter() - t0) * 1e3 / (args.warmup + args.steps), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1))", "config": config_dict(bwd_sample(wl), 0, backward=True),
+                "cpu_baseline": cpu,
+                "e2e": {"value": cpu["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     wl = synth.WORKLOADS[(DECODE_ALIASES if decode else WORKLOAD_ALIASES).get(args.workload, args.workload)]
     inp = synth.make_inputs(wl, seed=0)
     nthreads = O.nthreads_default()
@@ -676,7 +813,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES))
+                    choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
+                    + sorted(BWD_ALIASES))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -245,13 +245,15 @@ def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: in
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
         do: torch.Tensor, *, n_start: int = 0, window: int = 0, L_pretrain: int = 0, rope_theta: float = 0.0,
         topk: int = 0, is_sep: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
-        workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
+        workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False,
+        grads: Optional[tuple] = None):
     """Backward pass of ``fwd``: gradients of sum(do * o) for the forward's
     inputs and outputs.  ``topk_idx`` is the forward's selection (needed when
-    topk > 0).  Returns (dq, dk, dv), shaped and strided like q, k, v."""
+    topk > 0).  Returns (dq, dk, dv), shaped and strided like q, k, v (written
+    into ``grads`` when given)."""
     if do.stride() != o.stride() or do.dtype != o.dtype or do.shape != o.shape:
         raise ValueError("do must match o in shape, dtype and strides")
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     for g, x in ((dq, q), (dk, k), (dv, v)):
         if g.stride() != x.stride():
             raise ValueError("gradient buffers must share the strides of their inputs")

@@ -1061,12 +1061,8 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   a.dV = static_cast<__nv_bfloat16*>(dV);
   a.status = at<int32_t>(ws, F.status);
   {
-    ProfScope ps("bwd_rowstats", 1, st);
-    SATTN_TRY(launch_bwd_rowstats(a, st));
-  }
-  if (F.n_sink > 0) {
-    ProfScope ps("bwd_sink_rows", 1, st);
-    SATTN_TRY(launch_bwd_sink_rows(a, st));
+    ProfScope ps("bwd_rows", 1, st);
+    SATTN_TRY(launch_bwd_rows(a, st));
   }
   a.side_valid = F.n_sink > 0;
   if (a.capped_sep) {

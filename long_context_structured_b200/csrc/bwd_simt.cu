@@ -2,13 +2,13 @@
 // section 6.2: training runs the forward and the backward pass through the
 // masked product).
 //
-//   bwd_rowstats_kernel    D_i = dO_i . O_i and -LSE_i log2(e) per row,
-//                          padded to whole 128-row tiles;
-//   bwd_sink_rows_kernel   the starting-span keys j < n_start ("LM-Infinite",
-//                          section 方法) are fp32 side keys in the forward, and
-//                          here too: per row, P and dS of its sink pairs and
-//                          their dq (capped pairs through R(L)^T, others
-//                          through R(i)^T of R(j) k_j);
+//   bwd_rows_kernel        per row: D_i = dO_i . O_i and -LSE_i log2(e)
+//                          (padded to whole 128-row tiles) and, since the
+//                          starting-span keys j < n_start ("LM-Infinite",
+//                          section 方法) are fp32 side keys in the forward and
+//                          here too, P and dS of the row's sink pairs and their
+//                          dq (capped pairs through R(L)^T, others through
+//                          R(i)^T of R(j) k_j);
 //   bwd_sink_keys_kernel   dk and dv of the sink keys: fixed-order sums over
 //                          row blocks (no atomics);
 //   bwd_combine_kernel     dk_j, dv_j = band-tile part + separator part (its
@@ -44,146 +44,254 @@ __device__ __forceinline__ void rot_t(float y0, float y1, float2 cs, float& x0, 
 }
 __device__ __forceinline__ float bf(const __nv_bfloat16* p, int64_t idx) { return __bfloat162float(p[idx]); }
 
-// one warp per padded row
-__global__ void bwd_rowstats_kernel(BwdArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nrows = (int64_t)a.B * a.Hq * a.Tpad;
-  if (wid >= nrows) return;
-  const int i = (int)(wid % a.Tpad);
-  const int64_t bh = wid / a.Tpad;
-  const int h = (int)(bh % a.Hq), b = (int)(bh / a.Hq);
-  float dd = 0.f, nl = -CUDART_INF_F;
-  if (i < a.T) {
-    const __nv_bfloat16* o = a.O + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st;
-    const __nv_bfloat16* g = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st;
-    for (int c = lane; c < a.d; c += 32) dd = fmaf(bf(o, c), bf(g, c), dd);
-    dd = warp_sum(dd);
-    nl = -a.lse[bh * a.T + i] * kLog2e;
-  }
-  if (lane == 0) {
-    a.Dsum[wid] = dd;
-    a.nlse2[wid] = nl;
+// Per-row pass: D_i = dO_i . O_i, -LSE_i log2(e) (padded rows: 0, -inf) and,
+// for the sink keys, P_ij, dS_ij and their dq (fp32, raw frame, scaled).
+// 8 lanes per row, lane l owning the rotary pairs [8l/2 .. ) -- E = D/16
+// pairs per lane: elements c0 + e and c0 + e + D/2 for c0 = l * E, e < E.
+// A block is 32 rows of one (b, h); the group's sink K (rotated and raw)
+// and V rows are staged in shared memory as fp32.
+constexpr int kSinkStage = 16;  // sink rows staged in shared memory at a time
+
+// 8 consecutive bf16 (16 bytes, E = 8) or 4 (8 bytes, E = 4) as floats
+template <int E>
+__device__ __forceinline__ void load_row_part(const __nv_bfloat16* p, float* out) {
+  if constexpr (E == 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const float2 f = __bfloat1622float2(h[y]);
+      out[2 * y] = f.x;
+      out[2 * y + 1] = f.y;
+    }
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int y = 0; y < 2; ++y) {
+      const float2 f = __bfloat1622float2(h[y]);
+      out[2 * y] = f.x;
+      out[2 * y + 1] = f.y;
+    }
   }
 }
 
-// one warp per row; PP rotary pairs per lane (d = 64 PP)
-template <int PP>
-__global__ void bwd_sink_rows_kernel(BwdArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nrows = (int64_t)a.B * a.Hq * a.T;
-  if (wid >= nrows) return;
-  const int half = a.d / 2;
-  const int i = (int)(wid % a.T);
-  const int64_t bh = wid / a.T;
+template <int D>
+__global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
+  constexpr int E = D / 16;  // pairs per lane
+  constexpr int H = D / 2;
+  __shared__ float s_sink[kSinkStage][3][D];  // R(j) k_j, k_j, v_j of a stage of sinks
+  const int blocks_per_head = a.Tpad / 32;
+  const int64_t bh = blockIdx.x / blocks_per_head;
+  const int i = (int)(blockIdx.x % blocks_per_head) * 32 + (threadIdx.x >> 3);
+  const int l = threadIdx.x & 7;
   const int h = (int)(bh % a.Hq), b = (int)(bh / a.Hq);
   const int g = h / (a.Hq / a.Hkv);
+  const int ns_all = a.n_sink;
+  const bool row_ok = i < a.T;
   const int64_t prow = bh * a.Tpad + i;
-  const float D = a.Dsum[prow], nl2 = a.nlse2[prow];
-  const __nv_bfloat16* gp = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st;
-  float g0[PP], g1[PP], ar0[PP], ar1[PP], ac0[PP], ac1[PP];
+  const int c0 = l * E;
+  float g0[E], g1[E];
+  float dd = 0.f, nl2 = -CUDART_INF_F;
+  if (row_ok) {
+    const int64_t ooff = b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st;
+    float o0[E], o1[E];
+    load_row_part<E>(a.dO + ooff + c0, g0);
+    load_row_part<E>(a.dO + ooff + c0 + H, g1);
+    load_row_part<E>(a.O + ooff + c0, o0);
+    load_row_part<E>(a.O + ooff + c0 + H, o1);
 #pragma unroll
-  for (int e = 0; e < PP; ++e) {
-    const int c = lane * PP + e;
-    g0[e] = bf(gp, c);
-    g1[e] = bf(gp, c + half);
-    ar0[e] = ar1[e] = ac0[e] = ac1[e] = 0.f;
+    for (int e = 0; e < E; ++e) dd = fmaf(g0[e], o0[e], fmaf(g1[e], o1[e], dd));
+    nl2 = -a.lse[bh * a.T + i] * kLog2e;
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) g0[e] = g1[e] = 0.f;
   }
-  const int ns = min(a.n_sink, i + 1);
-  for (int j = 0; j < ns; ++j) {
-    const __nv_bfloat16* vp = a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st;
-    const __nv_bfloat16* kp = a.K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
-    float dp = 0.f;
+  dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+  dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+  dd += __shfl_xor_sync(0xffffffffu, dd, 4);
+  if (l == 0) {
+    a.Dsum[prow] = dd;
+    a.nlse2[prow] = nl2;
+  }
+  if (ns_all == 0) return;  // uniform over the block
+  const int ns = row_ok ? min(ns_all, i + 1) : 0;
+  float ar0[E], ar1[E], ac0[E], ac1[E];
 #pragma unroll
-    for (int e = 0; e < PP; ++e) {
-      const int c = lane * PP + e;
-      dp = fmaf(g0[e], bf(vp, c), fmaf(g1[e], bf(vp, c + half), dp));
+  for (int e = 0; e < E; ++e) ar0[e] = ar1[e] = ac0[e] = ac1[e] = 0.f;
+  const int64_t wid = bh * a.T + i;
+  for (int js = 0; js < ns_all; js += kSinkStage) {
+    const int nst = min(kSinkStage, ns_all - js);
+    __syncthreads();  // the previous stage is consumed
+    for (int x = threadIdx.x; x < nst * H; x += blockDim.x) {
+      const int jj = x / H, p = x % H, j = js + jj;
+      const __nv_bfloat16* kp = a.K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
+      const __nv_bfloat16* vp = a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st;
+      const float k0 = bf(kp, p), k1 = bf(kp, p + H);
+      float r0, r1;
+      rot(k0, k1, tab_at(a.tab, j, H, p), r0, r1);
+      s_sink[jj][0][p] = r0;
+      s_sink[jj][0][p + H] = r1;
+      s_sink[jj][1][p] = k0;
+      s_sink[jj][1][p + H] = k1;
+      s_sink[jj][2][p] = bf(vp, p);
+      s_sink[jj][2][p + H] = bf(vp, p + H);
     }
-    dp = warp_sum(dp);
-    const float p = exp2f(fmaf(a.sink_z[wid * a.n_sink + j], a.scale_log2, nl2));
-    const float ds = p * (dp - D);
-    if (lane == 0) {
-      a.sink_ds[wid * a.n_sink + j] = ds;
-      a.sink_p[wid * a.n_sink + j] = p;
-    }
-    const bool capped = a.L > 0 && (i - j) > a.L;
+    __syncthreads();
+    // every lane of a row takes the same branches (same i, same j)
+    for (int jj = 0; jj < nst && js + jj < ns; ++jj) {
+      const int j = js + jj;
+      float dp = 0.f;
 #pragma unroll
-    for (int e = 0; e < PP; ++e) {
-      const int c = lane * PP + e;
-      const float x0 = bf(kp, c), x1 = bf(kp, c + half);
-      if (capped) {
-        ac0[e] = fmaf(ds, x0, ac0[e]);
-        ac1[e] = fmaf(ds, x1, ac1[e]);
-      } else {
-        float y0, y1;
-        rot(x0, x1, tab_at(a.tab, j, half, c), y0, y1);
-        ar0[e] = fmaf(ds, y0, ar0[e]);
-        ar1[e] = fmaf(ds, y1, ar1[e]);
+      for (int e = 0; e < E; ++e) dp = fmaf(g0[e], s_sink[jj][2][c0 + e], fmaf(g1[e], s_sink[jj][2][c0 + e + H], dp));
+      dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 1);
+      dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 2);
+      dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 4);
+      const float p = exp2f(fmaf(a.sink_z[wid * ns_all + j], a.scale_log2, nl2));
+      const float ds = p * (dp - dd);
+      if (l == 0) {
+        a.sink_ds[wid * ns_all + j] = ds;
+        a.sink_p[wid * ns_all + j] = p;
+      }
+      const bool capped = a.L > 0 && (i - j) > a.L;
+      const float* kr = s_sink[jj][capped ? 1 : 0];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if (capped) {
+          ac0[e] = fmaf(ds, kr[c0 + e], ac0[e]);
+          ac1[e] = fmaf(ds, kr[c0 + e + H], ac1[e]);
+        } else {
+          ar0[e] = fmaf(ds, kr[c0 + e], ar0[e]);
+          ar1[e] = fmaf(ds, kr[c0 + e + H], ar1[e]);
+        }
       }
     }
   }
-  const float scale = rsqrtf((float)a.d);
-  float* out = a.dq_side + wid * a.d;
+  if (!row_ok) return;
+  const float scale = rsqrtf((float)D);
+  float* out = a.dq_side + wid * D;
+  float y0[E], y1[E];
 #pragma unroll
-  for (int e = 0; e < PP; ++e) {
-    const int c = lane * PP + e;
-    float x0, x1, y0, y1;
-    rot_t(ar0[e], ar1[e], tab_at(a.tab, i, half, c), x0, x1);
-    rot_t(ac0[e], ac1[e], a.L > 0 ? tab_at(a.tab, a.L, half, c) : make_float2(1.f, 0.f), y0, y1);
-    out[c] = (x0 + y0) * scale;
-    out[c + half] = (x1 + y1) * scale;
+  for (int e = 0; e < E; ++e) {
+    float x0, x1, z0, z1;
+    rot_t(ar0[e], ar1[e], tab_at(a.tab, i, H, c0 + e), x0, x1);
+    rot_t(ac0[e], ac1[e], a.L > 0 ? tab_at(a.tab, a.L, H, c0 + e) : make_float2(1.f, 0.f), z0, z1);
+    y0[e] = (x0 + z0) * scale;
+    y1[e] = (x1 + z1) * scale;
+  }
+#pragma unroll
+  for (int e = 0; e < E; e += 4) {
+    *reinterpret_cast<float4*>(out + c0 + e) = make_float4(y0[e], y0[e + 1], y0[e + 2], y0[e + 3]);
+    *reinterpret_cast<float4*>(out + c0 + e + H) = make_float4(y1[e], y1[e + 1], y1[e + 2], y1[e + 3]);
   }
 }
 
-// One CTA per (b, g, sink j, row block), d/2 threads, thread p owning pair
-// (p, p + d/2): sums over the block's rows i >= j of every query head of
-// the group of dS_ij R(i) q_i (uncapped pairs) and dS_ij R(L) q_i (capped),
-// and of P_ij dO_i.  Writes the raw-frame dk part (R(j)^T applied to the
-// uncapped sum; unscaled) and the dv part.
-__global__ void bwd_sink_keys_kernel(BwdArgs a) {
-  const int p = threadIdx.x;
-  const int half = a.d / 2;
+// Sink-key partial sums of one row block: CTA per (b, g, row block, group of
+// kSinkGroup sinks), 256 threads = 8 warps taking the block's rows of every
+// query head of the group in turn; lane l owns pairs 2l, 2l + 1 (elements
+// 2l, 2l+1, 2l+D/2, 2l+1+D/2; D = 128) or pair l (D = 64).  Per sink: sums
+// of dS_ij R(i) q_i (uncapped), dS_ij R(L) q_i (capped), P_ij dO_i; the 8
+// warps' sums are added in a fixed order through shared memory.  Writes the
+// raw-frame dk part (R(j)^T of the uncapped sum plus the capped sum,
+// unscaled) and the dv part of each sink.
+constexpr int kSinkGroup = 4;
+template <int D>
+__global__ void __launch_bounds__(256) bwd_sink_keys_kernel(BwdArgs a) {
+  constexpr int PL = D / 64;  // pairs per lane
+  constexpr int H = D / 2;
+  __shared__ float red[8][kSinkGroup][3][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_grp = (a.n_sink + kSinkGroup - 1) / kSinkGroup;
   int64_t x = blockIdx.x;
+  const int sg = (int)(x % n_grp);
+  x /= n_grp;
   const int rb = (int)(x % a.nRB);
   x /= a.nRB;
-  const int j = (int)(x % a.n_sink);
-  x /= a.n_sink;
   const int g = (int)(x % a.Hkv), b = (int)(x / a.Hkv);
   const int rep = a.Hq / a.Hkv;
-  float ur0 = 0.f, ur1 = 0.f, uc0 = 0.f, uc1 = 0.f, v0 = 0.f, v1 = 0.f;
-  const int i_lo = max(j, rb * kSinkRowBlock), i_hi = min(a.T, (rb + 1) * kSinkRowBlock);
-  const float2 cl = a.L > 0 ? tab_at(a.tab, a.L, half, p) : make_float2(1.f, 0.f);
+  const int j0 = sg * kSinkGroup;
+  const int nj = min(kSinkGroup, a.n_sink - j0);
+  float ar[kSinkGroup][2 * PL], ac[kSinkGroup][2 * PL], av[kSinkGroup][2 * PL];
+#pragma unroll
+  for (int q = 0; q < kSinkGroup; ++q)
+#pragma unroll
+    for (int e = 0; e < 2 * PL; ++e) ar[q][e] = ac[q][e] = av[q][e] = 0.f;
+  const int i_lo = max(j0, rb * kSinkRowBlock), i_hi = min(a.T, (rb + 1) * kSinkRowBlock);
+  float2 cl[PL];
+#pragma unroll
+  for (int e = 0; e < PL; ++e) cl[e] = a.L > 0 ? tab_at(a.tab, a.L, H, PL * lane + e) : make_float2(1.f, 0.f);
   for (int h = g * rep; h < (g + 1) * rep; ++h) {
     const int64_t bh = (int64_t)b * a.Hq + h;
-    for (int i = i_lo; i < i_hi; ++i) {
+    for (int i = i_lo + warp; i < i_hi; i += 8) {
       const int64_t wid = bh * a.T + i;
-      const float ds = a.sink_ds[wid * a.n_sink + j];
-      const float pj = a.sink_p[wid * a.n_sink + j];
-      const __nv_bfloat16* qp = a.Q + b * a.q_sb + h * a.q_sh + (int64_t)i * a.q_st;
-      const __nv_bfloat16* gp = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st;
-      const float q0 = bf(qp, p), q1 = bf(qp, p + half);
-      const bool capped = a.L > 0 && (i - j) > a.L;
-      float y0, y1;
-      rot(q0, q1, capped ? cl : tab_at(a.tab, i, half, p), y0, y1);
-      if (capped) {
-        uc0 = fmaf(ds, y0, uc0);
-        uc1 = fmaf(ds, y1, uc1);
-      } else {
-        ur0 = fmaf(ds, y0, ur0);
-        ur1 = fmaf(ds, y1, ur1);
+      const __nv_bfloat16* qp = a.Q + b * a.q_sb + h * a.q_sh + (int64_t)i * a.q_st + PL * lane;
+      const __nv_bfloat16* gp = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st + PL * lane;
+      float q0[PL], q1[PL], d0[PL], d1[PL], qi0[PL], qi1[PL], ql0[PL], ql1[PL];
+#pragma unroll
+      for (int e = 0; e < PL; ++e) {
+        q0[e] = bf(qp, e);
+        q1[e] = bf(qp, e + H);
+        d0[e] = bf(gp, e);
+        d1[e] = bf(gp, e + H);
+        rot(q0[e], q1[e], tab_at(a.tab, i, H, PL * lane + e), qi0[e], qi1[e]);
+        rot(q0[e], q1[e], cl[e], ql0[e], ql1[e]);
       }
-      v0 = fmaf(pj, bf(gp, p), v0);
-      v1 = fmaf(pj, bf(gp, p + half), v1);
+#pragma unroll
+      for (int q = 0; q < kSinkGroup; ++q) {
+        if (q >= nj) break;
+        const int j = j0 + q;
+        if (i < j) continue;
+        const float ds = a.sink_ds[wid * a.n_sink + j];
+        const float pj = a.sink_p[wid * a.n_sink + j];
+        const bool capped = a.L > 0 && (i - j) > a.L;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) {
+          if (capped) {
+            ac[q][e] = fmaf(ds, ql0[e], ac[q][e]);
+            ac[q][PL + e] = fmaf(ds, ql1[e], ac[q][PL + e]);
+          } else {
+            ar[q][e] = fmaf(ds, qi0[e], ar[q][e]);
+            ar[q][PL + e] = fmaf(ds, qi1[e], ar[q][PL + e]);
+          }
+          av[q][e] = fmaf(pj, d0[e], av[q][e]);
+          av[q][PL + e] = fmaf(pj, d1[e], av[q][PL + e]);
+        }
+      }
     }
   }
-  float x0, x1;
-  rot_t(ur0, ur1, tab_at(a.tab, j, half, p), x0, x1);
-  float* part = a.sink_part + (size_t)blockIdx.x * 2 * a.d;
-  part[p] = x0 + uc0;
-  part[p + half] = x1 + uc1;
-  part[a.d + p] = v0;
-  part[a.d + p + half] = v1;
+  // fixed-order reduction over the 8 warps
+#pragma unroll
+  for (int q = 0; q < kSinkGroup; ++q)
+#pragma unroll
+    for (int e = 0; e < PL; ++e) {
+      const int c = PL * lane + e;
+      red[warp][q][0][c] = ar[q][e];
+      red[warp][q][0][c + H] = ar[q][PL + e];
+      red[warp][q][1][c] = ac[q][e];
+      red[warp][q][1][c + H] = ac[q][PL + e];
+      red[warp][q][2][c] = av[q][e];
+      red[warp][q][2][c + H] = av[q][PL + e];
+    }
+  __syncthreads();
+  for (int t = threadIdx.x; t < nj * H; t += blockDim.x) {
+    const int q = t / H, p = t % H, j = j0 + q;
+    float r0 = 0.f, r1 = 0.f, c0 = 0.f, c1 = 0.f, v0 = 0.f, v1 = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      r0 += red[w][q][0][p];
+      r1 += red[w][q][0][p + H];
+      c0 += red[w][q][1][p];
+      c1 += red[w][q][1][p + H];
+      v0 += red[w][q][2][p];
+      v1 += red[w][q][2][p + H];
+    }
+    float x0, x1;
+    rot_t(r0, r1, tab_at(a.tab, j, H, p), x0, x1);
+    float* part = a.sink_part + ((((int64_t)b * a.Hkv + g) * a.n_sink + j) * a.nRB + rb) * 2 * D;
+    part[p] = x0 + c0;
+    part[p + H] = x1 + c1;
+    part[D + p] = v0;
+    part[D + p + H] = v1;
+  }
 }
 
 // one thread per 8 consecutive elements of one key row
@@ -248,30 +356,29 @@ __global__ void bwd_combine_kernel(BwdArgs a) {
 
 int bwd_sink_row_block() { return kSinkRowBlock; }
 
-cudaError_t launch_bwd_rowstats(const BwdArgs& a, cudaStream_t st) {
-  const int64_t rows = (int64_t)a.B * a.Hq * a.Tpad;
-  if (rows == 0) return cudaSuccess;
-  bwd_rowstats_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_sink_rows(const BwdArgs& a, cudaStream_t st) {
-  const int64_t rows = (int64_t)a.B * a.Hq * a.T;
-  if (rows == 0 || a.n_sink == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)((rows * 32 + 127) / 128);
-  if (a.d == 128)
-    bwd_sink_rows_kernel<2><<<blocks, 128, 0, st>>>(a);
-  else if (a.d == 64)
-    bwd_sink_rows_kernel<1><<<blocks, 128, 0, st>>>(a);
-  else
+cudaError_t launch_bwd_rows(const BwdArgs& a, cudaStream_t st) {
+  const int64_t blocks = (int64_t)a.B * a.Hq * (a.Tpad / 32);
+  if (blocks == 0) return cudaSuccess;
+  if (a.d == 128) {
+    bwd_rows_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
+  } else if (a.d == 64) {
+    bwd_rows_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
+  } else {
     return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_sink_keys(const BwdArgs& a, cudaStream_t st) {
-  const int64_t blocks = (int64_t)a.B * a.Hkv * a.n_sink * a.nRB;
-  if (blocks == 0) return cudaSuccess;
-  bwd_sink_keys_kernel<<<(unsigned)blocks, a.d / 2, 0, st>>>(a);
+  const int n_grp = (a.n_sink + kSinkGroup - 1) / kSinkGroup;
+  const int64_t blocks = (int64_t)a.B * a.Hkv * a.nRB * n_grp;
+  if (blocks == 0 || a.n_sink == 0) return cudaSuccess;
+  if (a.d == 128)
+    bwd_sink_keys_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
+  else if (a.d == 64)
+    bwd_sink_keys_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

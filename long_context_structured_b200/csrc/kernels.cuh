@@ -222,8 +222,7 @@ struct BwdArgs {
 struct BwdMaps {
   CUtensorMap q, qc, dO, k, v, kg, vg;
 };
-cudaError_t launch_bwd_rowstats(const BwdArgs& a, cudaStream_t st);
-cudaError_t launch_bwd_sink_rows(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_rows(const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_sink_keys(const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_dq(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
 cudaError_t launch_bwd_dkv(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
