@@ -76,6 +76,11 @@ def lib():
             L.oracle_fwd_rows.restype = ctypes.c_int
             L.oracle_fwd_rows.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 4 + [
                 ctypes.c_int64] + [ctypes.c_void_p] * 7 + [ctypes.c_int]
+            L.oracle_tree_index.restype = ctypes.c_int
+            L.oracle_tree_index.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p]
+            L.oracle_tree_cross.restype = ctypes.c_int
+            L.oracle_tree_cross.argtypes = [P(OracleParams)] + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 5 + [
+                ctypes.c_int]
             L.oracle_bwd.restype = ctypes.c_int
             L.oracle_bwd.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
             L.oracle_blockmap.restype = ctypes.c_int
@@ -188,6 +193,28 @@ def bwd(p: OracleParams, q, k, v, is_sep, dO, forced_topk=None, nthreads=None):
     if rc != 0:
         raise RuntimeError("oracle_bwd failed: %d" % rc)
     return dQ, dK, dV
+
+
+def tree_index(chunk_len, depth, alpha_leaf) -> np.ndarray:
+    """Kept offsets of one context chunk of the tree cross-attention."""
+    n = lib().oracle_tree_index(chunk_len, depth, alpha_leaf, None)
+    if n < 1:
+        raise RuntimeError("oracle_tree_index failed: %d" % n)
+    out = np.zeros(n, dtype=np.int32)
+    lib().oracle_tree_index(chunk_len, depth, alpha_leaf, _ptr(out))
+    return out
+
+
+def tree_cross(p: OracleParams, n_chunks, chunk_len, depth, alpha_leaf, q, k, v, nthreads=None):
+    """Tree cross-attention: (O [B,Hq,T,d], lse [B,Hq,T]) in float64."""
+    q, k, v = _inputs(p, q, k, v)
+    O = np.zeros((p.B, p.Hq, p.T, p.d), dtype=np.float64)
+    lse = np.zeros((p.B, p.Hq, p.T), dtype=np.float64)
+    rc = lib().oracle_tree_cross(ctypes.byref(p), n_chunks, chunk_len, depth, alpha_leaf, _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(O), _ptr(lse), nthreads or nthreads_default())
+    if rc != 0:
+        raise RuntimeError("oracle_tree_cross failed: %d" % rc)
+    return O, lse
 
 
 def all_rows(B, H, T) -> np.ndarray:

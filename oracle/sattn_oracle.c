@@ -22,6 +22,10 @@
  *   [SEP] "SepLLM" (CSDN article), sections 五.2 and 6.1: mask
  *         M_ij = 1 iff j in {initial a, separator before i, neighbouring n};
  *         masked positions are set to -inf before the softmax.
+ *   [SHL] "SharedLLM" (papernotes summary), sections 关键设计 2 (context
+ *         tree: halving splits, level rates alpha_w = 2 alpha_{w+1},
+ *         equally spaced downsampling) and 4 (tree cross-attention with
+ *         chunk-level rotary positions: queries n, chunk c's keys c).
  *   [SEG] "Training-Inference Consistent Segmented Execution for
  *         Long-Context LLMs", section "整体框架" and "关键设计": local heads
  *         attend a carried tail of the last M keys plus the segment
@@ -60,6 +64,17 @@
  *       distances are token distances (the rotary scale s does not apply);
  *       top-k ranks by z - sqrt(d) m_h d'_ij, the unscaled form of the
  *       biased logit, and reports z.
+ *   R13 tree cross-attention ([SHL] "SharedLLM", sections 关键设计 2 and 4):
+ *       each of the n context chunks (length l) is a binary tree; the
+ *       language-modelling policy always expands the right child, so at
+ *       levels w = 1..D the left child is kept and, at w = D, the right
+ *       child too (depth D = 0 keeps the root); the split of a node of
+ *       length m is b = floor(m/2) (the noise is 0 at test time); level w
+ *       keeps a node of length m at rate alpha_w = alpha_D * 2^(D - w):
+ *       m' = max(1, floor(m / alpha_w)) rows at offsets floor(k m / m'),
+ *       k < m'; the kept rows of a chunk keep their text order; chunk c's
+ *       keys take rotary position c and every query position n; the
+ *       attention is a plain softmax over all kept rows of all chunks;
  *   R12 backward ([SEP] 6.2: training runs the forward and the backward
  *       pass through the masked product): the gradients of sum(dO . O)
  *       in exact arithmetic; the
@@ -626,6 +641,120 @@ int oracle_bwd(const oracle_params* p, const void* Q, const void* K, const void*
   J.dK = dK;
   J.dV = dV;
   run_parallel(bwd_one, &J, (int64_t)p->B * p->Hkv, nthreads);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* SharedLLM tree cross-attention (R13)                                */
+/* ------------------------------------------------------------------ */
+
+/* Kept offsets of one chunk of length l, in text order; returns how many
+ * (out may be NULL to count only). */
+int oracle_tree_index(int l, int depth, int alpha_leaf, int32_t* out) {
+  if (l < 1 || depth < 0 || alpha_leaf < 1 || depth > 30) return OR_ERR_ARG;
+  int n = 0;
+  int start = 0, len = l;
+  for (int w = (depth == 0 ? 0 : 1); w <= depth; ++w) {
+    /* the nodes kept at level w: [start, start + m) pieces */
+    int piece_start[2], piece_len[2], pieces = 0;
+    if (depth == 0) {
+      piece_start[0] = 0;
+      piece_len[0] = l;
+      pieces = 1;
+    } else {
+      int b = len / 2;
+      piece_start[pieces] = start;
+      piece_len[pieces] = b;
+      ++pieces;
+      if (w == depth) {
+        piece_start[pieces] = start + b;
+        piece_len[pieces] = len - b;
+        ++pieces;
+      }
+      start += b;
+      len -= b;
+    }
+    double alpha = (double)alpha_leaf * pow(2.0, (double)(depth - w));
+    for (int x = 0; x < pieces; ++x) {
+      int m = piece_len[x];
+      if (m <= 0) continue;
+      int kept = (int)floor((double)m / alpha);
+      if (kept < 1) kept = 1;
+      for (int k = 0; k < kept; ++k) {
+        if (out) out[n] = piece_start[x] + (int)(((int64_t)k * m) / kept);
+        ++n;
+      }
+    }
+  }
+  return n;
+}
+
+typedef struct {
+  const oracle_params* p;
+  const void *Q, *K, *V;
+  int n_chunks, chunk_len, n_kept;
+  const int32_t* idx;
+  double *O, *lse;
+} tree_job;
+
+static void tree_one(void* arg, int64_t r) {
+  tree_job* J = (tree_job*)arg;
+  const oracle_params* p = J->p;
+  int d = p->d, T = p->T, b = (int)(r / ((int64_t)p->Hq * T)), h = (int)((r / T) % p->Hq), i = (int)(r % T);
+  int g = (int)(((int64_t)h * p->Hkv) / p->Hq);
+  int S = J->n_chunks * J->n_kept, Tc = J->n_chunks * J->chunk_len;
+  double* q = (double*)malloc(sizeof(double) * 4 * (size_t)d);
+  double *qr = q + d, *k = q + 2 * d, *kr = q + 3 * d;
+  double* z = (double*)malloc(sizeof(double) * (size_t)S);
+  for (int c = 0; c < d; ++c) q[c] = load_elem(J->Q, p->dtype, (((int64_t)b * p->Hq + h) * T + i) * d + c);
+  oracle_rope(q, d, rot_pos(p, (double)J->n_chunks), p->rope_theta, qr);
+  double mx = -INFINITY;
+  for (int s = 0; s < S; ++s) {
+    int c = s / J->n_kept, j = c * J->chunk_len + J->idx[s % J->n_kept];
+    int64_t kb = (((int64_t)b * p->Hkv + g) * Tc + j) * d;
+    for (int x = 0; x < d; ++x) k[x] = load_elem(J->K, p->dtype, kb + x);
+    oracle_rope(k, d, rot_pos(p, (double)c), p->rope_theta, kr);
+    z[s] = dot(qr, kr, d) * (1.0 / sqrt((double)d));
+    if (z[s] > mx) mx = z[s];
+  }
+  double sum = 0.0;
+  for (int s = 0; s < S; ++s) sum += exp(z[s] - mx);
+  double l = mx + log(sum);
+  double* o = J->O + r * d;
+  for (int x = 0; x < d; ++x) o[x] = 0.0;
+  for (int s = 0; s < S; ++s) {
+    int c = s / J->n_kept, j = c * J->chunk_len + J->idx[s % J->n_kept];
+    int64_t vb = (((int64_t)b * p->Hkv + g) * Tc + j) * d;
+    double w = exp(z[s] - l);
+    for (int x = 0; x < d; ++x) o[x] += w * load_elem(J->V, p->dtype, vb + x);
+  }
+  J->lse[r] = l;
+  free(q);
+  free(z);
+}
+
+/* O [B, Hq, T, d], lse [B, Hq, T] of the tree cross-attention: queries Q
+ * [B, Hq, T, d] (p->T rows), context K, V [B, Hkv, n_chunks * chunk_len, d]. */
+int oracle_tree_cross(const oracle_params* p, int n_chunks, int chunk_len, int depth, int alpha_leaf, const void* Q,
+                      const void* K, const void* V, double* O, double* lse, int nthreads) {
+  if (!p || n_chunks < 1 || p->d <= 0 || (p->d & 1) || p->Hq % p->Hkv) return OR_ERR_ARG;
+  int n_kept = oracle_tree_index(chunk_len, depth, alpha_leaf, NULL);
+  if (n_kept < 1) return OR_ERR_ARG;
+  int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)n_kept);
+  oracle_tree_index(chunk_len, depth, alpha_leaf, idx);
+  tree_job J;
+  J.p = p;
+  J.Q = Q;
+  J.K = K;
+  J.V = V;
+  J.n_chunks = n_chunks;
+  J.chunk_len = chunk_len;
+  J.n_kept = n_kept;
+  J.idx = idx;
+  J.O = O;
+  J.lse = lse;
+  run_parallel(tree_one, &J, (int64_t)p->B * p->Hq * p->T, nthreads);
+  free(idx);
   return OR_OK;
 }
 

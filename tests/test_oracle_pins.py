@@ -717,3 +717,83 @@ def test_alibi_topk_ranks_by_biased_logit(oracle_mod):
     a = oracle_mod.fwd_rows(p2, q, k, v, None, oracle_mod.all_rows(1, H, T))
     b = oracle_mod.fwd_rows(p3, q, k, v, None, oracle_mod.all_rows(1, H, T))
     assert np.array_equal(a[2], b[2])
+
+
+# ----------------------------------------------------------------------------
+# SharedLLM tree cross-attention (sections 关键设计 2 and 4)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("m,depth,alpha", [(6, 1, 1), (6, 2, 1), (6, 3, 2), (8, 4, 1), (8, 2, 4)])
+def test_tree_index_closed_form(oracle_mod, m, depth, alpha):
+    """Chunk length l = 2^m: the kept left node of level w spans
+    [l - l/2^(w-1), l - l/2^w) at rate alpha 2^(D-w), the kept right node of
+    level D the last l/2^D positions at rate alpha; every node keeps
+    l / (alpha 2^D) rows, equally spaced from its start."""
+    l = 2 ** m
+    per = l // (alpha * 2 ** depth)
+    exp = []
+    for w in range(1, depth + 1):
+        start = l - l // 2 ** (w - 1)
+        exp += [start + k * alpha * 2 ** (depth - w) for k in range(per)]
+    exp += [l - l // 2 ** depth + k * alpha for k in range(per)]
+    assert list(oracle_mod.tree_index(l, depth, alpha)) == exp
+
+
+@pytest.mark.parametrize("l", [1, 2, 3, 7, 100, 1000, 1023])
+def test_tree_index_properties(oracle_mod, l):
+    """Any length: offsets strictly increasing inside [0, l); depth 0 at rate
+    1 keeps everything; the kept count is the sum of max(1, floor(m/alpha))
+    over the kept nodes of the halving splits."""
+    for depth in range(0, 5):
+        for alpha in (1, 2, 3):
+            idx = oracle_mod.tree_index(l, depth, alpha)
+            assert np.all(np.diff(idx) > 0) and idx[0] >= 0 and idx[-1] < l
+            # node lengths of the halving splits, independently of the oracle
+            nodes, length = [], l
+            if depth == 0:
+                nodes = [(l, 0)]
+            for w in range(1, depth + 1):
+                b = length // 2
+                nodes.append((b, w))
+                if w == depth:
+                    nodes.append((length - b, w))
+                length -= b
+            want = sum(max(1, m // (alpha * 2 ** (depth - w))) for m, w in nodes if m > 0)
+            assert len(idx) == want
+    assert list(oracle_mod.tree_index(l, 0, 1)) == list(range(l))
+
+
+def _rot_np(O, x, pos, theta):
+    return O.rope(np.ascontiguousarray(x, dtype=np.float64), pos, theta)
+
+
+@pytest.mark.parametrize("theta,depth,alpha", [(0.0, 0, 1), (1e4, 2, 1), (1e4, 3, 2), (5e5, 1, 4)])
+def test_tree_cross_equals_sdpa_on_kept_rows(oracle_mod, theta, depth, alpha):
+    """Unmasked SDPA over the kept rows of every chunk, the query rotated to
+    position n and chunk c's keys to position c (depth 0, rate 1, no
+    rotation: plain dense attention over the whole context)."""
+    O = oracle_mod
+    B, Hq, Hkv, T, d = 1, 4, 2, 7, 16
+    n, l = 5, 24
+    q, _, _ = _rand_inputs(B, Hq, Hkv, T, d, 40)
+    _, k, v = _rand_inputs(B, Hq, Hkv, n * l, d, 41)
+    p = O.params(B, Hq, Hkv, T, d, "bf16", rope_theta=theta)
+    got, lse = O.tree_cross(p, n, l, depth, alpha, q, k, v)
+    idx = O.tree_index(l, depth, alpha)
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    rows = [c * l + j for c in range(n) for j in idx]
+    kk = k64[:, :, rows].copy()
+    for x, r in enumerate(rows):
+        for g in range(Hkv):
+            kk[0, g, x] = _rot_np(O, kk[0, g, x], r // l, theta)
+    qq = q64.copy()
+    for h in range(Hq):
+        for i in range(T):
+            qq[0, h, i] = _rot_np(O, qq[0, h, i], n, theta)
+    ref = _sdpa(qq, kk, v64[:, :, rows], np.ones((T, len(rows)), dtype=bool))
+    assert np.abs(got - ref).max() < 1e-12
+    if depth == 0 and alpha == 1 and theta == 0.0:
+        full = _sdpa(q64, k64, v64, np.ones((T, n * l), dtype=bool))
+        assert np.abs(got - full).max() < 1e-12
+    lref = _lse_ref(qq, kk, np.ones((T, len(rows)), dtype=bool))
+    assert np.abs(lse - lref).max() < 1e-12
