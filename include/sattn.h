@@ -238,6 +238,36 @@ int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V
               const int32_t* topk_idx, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
               void* dV, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace needed by sattn_tree_cross_fwd. */
+int sattn_tree_cross_workspace_size(const sattn_params* p, int32_t n_chunks, int32_t chunk_len, int32_t depth,
+                                    int32_t alpha_leaf, size_t* bytes);
+
+/* SharedLLM's position-aware tree cross-attention ("SharedLLM", sections
+ * 关键设计 2 and 4) with the language-modelling policy (the right child of a
+ * context-tree node is always the one expanded):
+ *   - the context is n_chunks chunks of chunk_len tokens; in each chunk,
+ *     levels w = 1..depth keep the left child of the node being expanded and
+ *     level `depth` also its right child (depth 0 keeps the whole chunk);
+ *     a node of length m splits at floor(m/2);
+ *   - a kept node of length m at level w keeps max(1, floor(m / a_w)) rows
+ *     at offsets floor(k m / m'), a_w = alpha_leaf * 2^(depth - w);
+ *   - the kept rows of chunk c take rotary position c, every query
+ *     position n_chunks; O = softmax(Q K'^T / sqrt(d)) V' over all kept
+ *     rows of all chunks (no mask).
+ *   p          B, Hq, Hkv, d, rope_theta, rope_pos_scale; T = query rows;
+ *              bf16 only; topk, L_pretrain, alibi, with_separators must be 0.
+ *   Q          [B, Hq, T, d] bf16 device, strides q_stride.
+ *   K, V       [B, Hkv, n_chunks * chunk_len, d] bf16 device (the context's
+ *              keys, unrotated, and values), strides k_stride / v_stride.
+ *   O, lse     [B, Hq, T, d] bf16 (strides o_stride), [B, Hq, T] fp32, out.
+ *   kept_index [n_kept] int32 device, out, or NULL: the kept offsets within
+ *              a chunk, in order (n_kept from the workspace query's rules).
+ * Limits: 1 <= alpha_leaf <= 1024, 0 <= depth <= 20, else
+ * SATTN_ERR_INVALID_ARG.  Asynchronous on `stream`. */
+int sattn_tree_cross_fwd(const sattn_params* p, int32_t n_chunks, int32_t chunk_len, int32_t depth,
+                         int32_t alpha_leaf, const void* Q, const void* K, const void* V, void* O, float* lse,
+                         int32_t* kept_index, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and reads the device status word of `ws` into
  * *device_status (SATTN_OK or SATTN_ERR_TIMEOUT).  Returns SATTN_ERR_CUDA if
  * the synchronisation itself failed (the CUDA error is then sticky). */

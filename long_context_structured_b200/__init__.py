@@ -274,6 +274,36 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     return dq, dk, dv
 
 
+def tree_cross_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_chunks: int, chunk_len: int, depth: int,
+                   alpha_leaf: int = 1, rope_theta: float = 0.0, rope_pos_scale: float = 1.0,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, with_index: bool = False):
+    """SharedLLM tree cross-attention: queries q [B, Hq, T, d] over the
+    compressed context k, v [B, Hkv, n_chunks * chunk_len, d].  Returns
+    (O, lse) or, with ``with_index``, (O, lse, kept offsets within a chunk)."""
+    B, Hq, T, d = q.shape
+    if k.shape[2] != n_chunks * chunk_len or v.shape[2] != k.shape[2]:
+        raise ValueError("k, v must hold n_chunks * chunk_len context rows")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    p = params(q, k, v, out, rope_theta=rope_theta, rope_pos_scale=rope_pos_scale)
+    n = ctypes.c_size_t(0)
+    L = _lib.load()
+    _lib.check(L.sattn_tree_cross_workspace_size(ctypes.byref(p), n_chunks, chunk_len, depth, alpha_leaf,
+                                                 ctypes.byref(n)), "sattn_tree_cross_workspace_size")
+    nbytes = int(n.value)
+    ws = _workspace(nbytes, q.device, workspace)
+    idx = torch.full((chunk_len,), -1, dtype=torch.int32, device=q.device) if with_index else None
+    rc = L.sattn_tree_cross_fwd(ctypes.byref(p), n_chunks, chunk_len, depth, alpha_leaf, _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(out), _ptr(lse), _ptr(idx), _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_tree_cross_fwd")
+    if with_index:
+        return out, lse, idx
+    return out, lse
+
+
 def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> int:
     """Synchronise the current stream and read the device status word of the
     workspace (the cached one when None)."""

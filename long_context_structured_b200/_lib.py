@@ -25,6 +25,7 @@ EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
     "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_bwd_workspace_size", "sattn_bwd",
+    "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd",
     "sattn_stream_status",
     "sattn_build_blockmap_noalloc", "sattn_selftest_wait_timeout", "sattn_profile_enable", "sattn_profile_collect",
 )
@@ -88,6 +89,10 @@ def load():
         L.sattn_bwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_bwd.restype = ctypes.c_int
         L.sattn_bwd.argtypes = [P] + [vp] * 12 + [sz, vp]
+        L.sattn_tree_cross_workspace_size.restype = ctypes.c_int
+        L.sattn_tree_cross_workspace_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
+        L.sattn_tree_cross_fwd.restype = ctypes.c_int
+        L.sattn_tree_cross_fwd.argtypes = [P, i32, i32, i32, i32] + [vp] * 7 + [sz, vp]
         L.sattn_stream_status.restype = ctypes.c_int
         L.sattn_stream_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.sattn_build_blockmap_noalloc.restype = ctypes.c_int

@@ -781,6 +781,44 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
 }
 
 // ---------------------------------------------------------------------------
+// SharedLLM tree cross-attention
+// ---------------------------------------------------------------------------
+
+struct TreePlan {
+  int n_kept = 0, S = 0, Spad = 0, nQT = 0, npos = 0;
+  Region status, tab, qr, kt, vt;
+  size_t total = 0;
+};
+
+static int plan_tree(const sattn_params* p, int32_t n_chunks, int32_t chunk_len, int32_t depth, int32_t alpha_leaf,
+                     TreePlan* out) {
+  int rc = check_common(p);
+  if (rc) return rc;
+  if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
+  if (p->topk != 0 || p->L_pretrain != 0 || p->alibi || p->with_separators) return SATTN_ERR_INVALID_ARG;
+  if (n_chunks < 1 || chunk_len < 1) return SATTN_ERR_INVALID_ARG;
+  TreePlan P;
+  P.n_kept = tree_kept_count(chunk_len, depth, alpha_leaf);
+  if (P.n_kept < 1) return SATTN_ERR_INVALID_ARG;
+  if ((int64_t)n_chunks * chunk_len > ((int64_t)1 << 30) || (int64_t)n_chunks * P.n_kept > ((int64_t)1 << 28))
+    return SATTN_ERR_UNSUPPORTED;
+  P.S = n_chunks * P.n_kept;
+  P.Spad = (P.S + kTile - 1) / kTile * kTile;
+  P.nQT = (p->T + kTile - 1) / kTile;
+  P.npos = n_chunks + 1;
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  P.qr = A.take(B * Hq * T * d * 2);
+  P.kt = A.take(B * Hkv * (size_t)P.Spad * d * 2);
+  P.vt = A.take(B * Hkv * (size_t)P.Spad * d * 2);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+// ---------------------------------------------------------------------------
 // decoding step
 // ---------------------------------------------------------------------------
 
@@ -1171,6 +1209,99 @@ int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.dv_st = p->v_stride[2];
   ProfScope ps("bwd_f32", 2, st);
   return cuda_rc(launch_bwd_f32(a, st));
+}
+
+int sattn_tree_cross_workspace_size(const sattn_params* p, int32_t n_chunks, int32_t chunk_len, int32_t depth,
+                                    int32_t alpha_leaf, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  TreePlan P;
+  int rc = plan_tree(p, n_chunks, chunk_len, depth, alpha_leaf, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_tree_cross_fwd(const sattn_params* p, int32_t n_chunks, int32_t chunk_len, int32_t depth,
+                         int32_t alpha_leaf, const void* Q, const void* K, const void* V, void* O, float* lse,
+                         int32_t* kept_index, void* ws, size_t ws_bytes, void* stream) {
+  TreePlan P;
+  int rc = plan_tree(p, n_chunks, chunk_len, depth, alpha_leaf, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+  }
+  TreeArgs t{};
+  t.B = p->B;
+  t.Hq = p->Hq;
+  t.Hkv = p->Hkv;
+  t.Tq = p->T;
+  t.d = p->d;
+  t.n_chunks = n_chunks;
+  t.chunk_len = chunk_len;
+  t.depth = depth;
+  t.alpha_leaf = alpha_leaf;
+  t.n_kept = P.n_kept;
+  t.Spad = P.Spad;
+  t.tab = at<float2>(ws, P.tab);
+  t.Q = static_cast<const __nv_bfloat16*>(Q);
+  t.q_sb = p->q_stride[0];
+  t.q_sh = p->q_stride[1];
+  t.q_st = p->q_stride[2];
+  t.K = static_cast<const __nv_bfloat16*>(K);
+  t.V = static_cast<const __nv_bfloat16*>(V);
+  t.k_sb = p->k_stride[0];
+  t.k_sh = p->k_stride[1];
+  t.k_st = p->k_stride[2];
+  t.v_sb = p->v_stride[0];
+  t.v_sh = p->v_stride[1];
+  t.v_st = p->v_stride[2];
+  t.Qr = at<__nv_bfloat16>(ws, P.qr);
+  t.Kt = at<__nv_bfloat16>(ws, P.kt);
+  t.Vt = at<__nv_bfloat16>(ws, P.vt);
+  t.kept_index = kept_index;
+  {
+    ProfScope ps("tree_prep", 1, st);
+    SATTN_TRY(launch_tree_prep(t, st));
+  }
+  const int64_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  AttnMaps m;
+  if (!make_map(&m.q, t.Qr, p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.kg, t.Kt, p->d, P.Spad, Hkv, B, d, (int64_t)P.Spad * d, Hkv * P.Spad * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.vg, t.Vt, p->d, P.Spad, Hkv, B, d, (int64_t)P.Spad * d, Hkv * P.Spad * d)) return SATTN_ERR_CUDA;
+  m.q2 = m.q;
+  m.k = m.kg;
+  m.v = m.vg;
+  AttnArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.nQT = P.nQT;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.ns_band = 0;
+  a.w_eff = 0;
+  a.V = t.Vt;
+  a.v_sb = Hkv * P.Spad * d;
+  a.v_sh = (int64_t)P.Spad * d;
+  a.v_st = d;
+  a.gather_mode = 3;
+  a.cross_len = P.S;
+  a.q2 = false;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.status = at<int32_t>(ws, P.status);
+  ProfScope ps("attn_tc_cross", 1, st);
+  return cuda_rc(launch_attn_tc2(a, m, st));
 }
 
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {

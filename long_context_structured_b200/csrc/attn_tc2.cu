@@ -205,6 +205,9 @@ __device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t
   if (a.gather_mode == 1) {
     p.g_full = a.ranges[(b * a.nQT + t) * 2 + 0];
     p.g_count = a.ranges[(b * a.nQT + t) * 2 + 1];
+  } else if (a.gather_mode == 3) {
+    // cross-attention over a compressed context: every row keeps all of it
+    p.g_count = p.g_full = a.cross_len;
   } else if (a.gather_mode == 2) {
     const int s = i0 / a.seg_S;
     const int seg0 = s * a.seg_S;
@@ -219,7 +222,7 @@ __device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t
   p.n_gather = (p.g_count + kTile - 1) / kTile;
   const int i_last = i0 + p.rows - 1;
   const int j_lo = max(max(p.band_lo, 0), max(i0 - a.w_eff, a.ns_band));
-  if (j_lo > i_last) {
+  if (j_lo > i_last || a.gather_mode == 3) {
     p.u_lo = 0;
     p.n_band = 0;
   } else {

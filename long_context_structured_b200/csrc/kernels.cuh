@@ -83,8 +83,10 @@ struct AttnArgs {
   int topk;
   const __nv_bfloat16* V;  // raw V for side keys
   int64_t v_sb, v_sh, v_st;
-  // gathered tiles: 0 none, 1 separators, 2 segmented prefix
+  // gathered tiles: 0 none, 1 separators, 2 segmented prefix, 3 cross-attention
+  // over a compressed context (every row keeps all cross_len gathered rows)
   int gather_mode;
+  int cross_len;
   bool q2;                     // gathered tiles use the second query tile (Qc)
   const int32_t* sep_pos;      // [B, T]
   const int32_t* sep_prefix;   // [B, T+1]: separators n_start <= j < x
@@ -139,6 +141,26 @@ struct AttnF32Args {
   float* lse;
 };
 cudaError_t launch_attn_f32(const AttnF32Args& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// SharedLLM tree cross-attention: compressed context and rotated queries
+// ---------------------------------------------------------------------------
+struct TreeArgs {
+  int B, Hq, Hkv, Tq, d;            // Tq query rows per (b, h)
+  int n_chunks, chunk_len, depth, alpha_leaf, n_kept, Spad;
+  const float2* tab;                // rotary table (null: no rotation), positions 0..n_chunks
+  const __nv_bfloat16* Q;           // [B, Hq, Tq, d] strided
+  int64_t q_sb, q_sh, q_st;
+  const __nv_bfloat16* K;           // [B, Hkv, n_chunks * chunk_len, d] strided
+  const __nv_bfloat16* V;
+  int64_t k_sb, k_sh, k_st, v_sb, v_sh, v_st;
+  __nv_bfloat16* Qr;                // [B, Hq, Tq, d]: R(n) q
+  __nv_bfloat16* Kt;                // [B, Hkv, Spad, d]: kept keys of chunk c, R(c) k
+  __nv_bfloat16* Vt;
+  int32_t* kept_index;              // [n_kept] or null: kept offsets within a chunk
+};
+cudaError_t launch_tree_prep(const TreeArgs& a, cudaStream_t st);
+int tree_kept_count(int chunk_len, int depth, int alpha_leaf);  // host; < 0 on bad arguments
 
 // ---------------------------------------------------------------------------
 // backward pass, fp32 on CUDA cores
