@@ -43,6 +43,11 @@ from long_context_structured_b200 import synth  # noqa: E402
 # decoding steps (one new token per sequence) over the caches of these workloads
 DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
 BWD_ALIASES = {"c2b": "c2_lminf_16k", "c3b": "c3_sepllm_gqa_8k"}
+TREE_ALIASES = {"c6t": "tree_cross_128k"}
+# SharedLLM tree cross-attention: a 128K-token context in 64 chunks of 2048,
+# depth 3, leaf rate 2 (global compression 4), 4096 decoder queries
+TREE_WORKLOADS = {"tree_cross_128k": dict(B=1, Hq=32, Hkv=32, Tq=4096, d=128, n_chunks=64, chunk_len=2048,
+                                          depth=3, alpha_leaf=2, rope_theta=1e4)}
 BWD_FLOPS_PER_PAIR_D = 10  # backward: S recomputed, dP, dV, dK, dQ -- five products of 2d FLOPs per pair
 WORKLOAD_ALIASES = {"c2": "c2_lminf_16k", "c3": "c3_sepllm_gqa_8k", "c4": "c4_lminf_topk_32k",
                     "c5": "c5_segmented_32k"}
@@ -459,6 +464,81 @@ class BwdJob:
         return out
 
 
+class TreeJob:
+    """SharedLLM tree cross-attention over a compressed long context: the
+    decoder queries against the kept rows of every context chunk."""
+
+    def __init__(self, cfg, seed, dev):
+        import torch
+
+        import long_context_structured_b200 as sa
+        self.sa, self.torch, self.cfg, self.dev = sa, torch, cfg, dev
+        c = cfg
+        g = torch.Generator().manual_seed(seed)
+        Tc = c["n_chunks"] * c["chunk_len"]
+        self.host = {"q": torch.randn(c["B"], c["Hq"], c["Tq"], c["d"], generator=g).bfloat16().pin_memory(),
+                     "k": torch.randn(c["B"], c["Hkv"], Tc, c["d"], generator=g).bfloat16().pin_memory(),
+                     "v": torch.randn(c["B"], c["Hkv"], Tc, c["d"], generator=g).bfloat16().pin_memory()}
+        self.devt = {x: t.to(dev) for x, t in self.host.items()}
+        self.kw = dict(n_chunks=c["n_chunks"], chunk_len=c["chunk_len"], depth=c["depth"],
+                       alpha_leaf=c["alpha_leaf"], rope_theta=c["rope_theta"])
+        self.O = torch.empty_like(self.devt["q"])
+        self.lse = torch.empty(c["B"], c["Hq"], c["Tq"], dtype=torch.float32, device=dev)
+        # the kept rows per chunk, as the library reports them
+        _, _, idx = sa.tree_cross_fwd(self.devt["q"], self.devt["k"], self.devt["v"], with_index=True, **self.kw)
+        self.n_kept = int((idx >= 0).sum().item())
+        self.S = c["n_chunks"] * self.n_kept
+        self.pairs = c["B"] * c["Hq"] * c["Tq"] * self.S
+        self.flops = 4.0 * c["d"] * self.pairs
+
+    def step(self):
+        d = self.devt
+        self.sa.tree_cross_fwd(d["q"], d["k"], d["v"], out=self.O, lse=self.lse, **self.kw)
+
+    def host_step(self):
+        h = self.host
+        dv = {x: t.to(self.dev, non_blocking=True) for x, t in h.items()}
+        O, lse = self.sa.tree_cross_fwd(dv["q"], dv["k"], dv["v"], **self.kw)
+        oh = self.torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        lh = self.torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        oh.copy_(O, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+        self.torch.cuda.current_stream(self.dev).synchronize()
+        return oh, lh
+
+    def h2d_bytes(self):
+        return int(sum(t.nbytes for t in self.host.values()))
+
+    def group_work(self):
+        c = self.cfg
+        rows_q = c["B"] * c["Hq"] * c["Tq"] * c["d"] * 2
+        kept = c["B"] * c["Hkv"] * self.S * c["d"] * 2
+        return {"attn_tc_cross": ("tensor", self.flops, "FLOP"),
+                "tree_prep": ("hbm", 2 * rows_q + 4 * kept, "B")}
+
+
+def cpu_baseline_tree(cfg, n_rows=256):
+    from oracle import oracle as O
+    O.build()
+    import torch
+    c = cfg
+    g = torch.Generator().manual_seed(0)
+    bits = lambda t: t.bfloat16().view(torch.int16).numpy().view(np.uint16)
+    Tc = c["n_chunks"] * c["chunk_len"]
+    q = bits(torch.randn(1, 1, n_rows, c["d"], generator=g))
+    k = bits(torch.randn(1, 1, Tc, c["d"], generator=g))
+    v = bits(torch.randn(1, 1, Tc, c["d"], generator=g))
+    p = O.params(1, 1, 1, n_rows, c["d"], "bf16", rope_theta=c["rope_theta"])
+    nthreads = O.nthreads_default()
+    t0 = time.perf_counter()
+    O.tree_cross(p, c["n_chunks"], c["chunk_len"], c["depth"], c["alpha_leaf"], q, k, v, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    S = c["n_chunks"] * len(O.tree_index(c["chunk_len"], c["depth"], c["alpha_leaf"]))
+    return {"value": round(4.0 * c["d"] * n_rows * S / dt / 1e12, 6), "unit": "TFLOP/s", "cores": nthreads,
+            "kind": "oracle", "sample": "%d query rows of one head against all %d kept context rows, fp64, %.1f s"
+            % (n_rows, S, dt), "seconds": round(dt, 2)}
+
+
 def roofline_of(group, work, avg_ms, peaks, peak_src):
     bound, amount, unit = work
     if bound == "tensor":
@@ -503,10 +583,13 @@ def kernel_name(wl, group):
         return "attn_tc3_kernel<%d>" % wl.d if capped_sep else "attn_tc2_kernel<%d>" % wl.d
     if group == "attn_tc_segment":
         return "attn_tc2_kernel<%d>" % wl.d if wl.seg_S % 256 == 0 else "attn_tc3_kernel<%d>" % wl.d
-    return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel",
+    if group == "attn_tc_cross":
+        return "attn_tc2_kernel<%d>" % TREE_WORKLOADS["tree_cross_128k"]["d"]
+    d = wl.d if wl is not None else 128
+    return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel", "tree_prep": "tree_prep_kernel",
             "decode": "decode_partial_kernel + decode_combine_kernel",
-            "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % wl.d,
-            "bwd_dkv": "bwd_dkv_kernel<%d>" % wl.d, "bwd_f32": "bwd_f32_dq_kernel + bwd_f32_dkv_kernel",
+            "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % d,
+            "bwd_dkv": "bwd_dkv_kernel<%d>" % d, "bwd_f32": "bwd_f32_dq_kernel + bwd_f32_dkv_kernel",
             "bwd_rows": "bwd_rows_kernel", "bwd_combine": "bwd_combine_kernel",
             "bwd_sink_keys": "bwd_sink_keys_kernel"}.get(group, group)
 
@@ -531,6 +614,9 @@ def run_ours(args):
 
     decode = args.workload in DECODE_ALIASES
     backward = args.workload in BWD_ALIASES
+    tree = args.workload in TREE_ALIASES
+    if tree:
+        return run_tree(args, world, rank, dev)
     aliases = DECODE_ALIASES if decode else (BWD_ALIASES if backward else WORKLOAD_ALIASES)
     wl = synth.WORKLOADS[aliases.get(args.workload, args.workload)]
     if args.heads:
@@ -662,6 +748,106 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def run_tree(args, world, rank, dev):
+    """The tree cross-attention workload: same timing, clocks and JSON line
+    as the other workloads."""
+    import torch
+    import torch.distributed as dist
+
+    import long_context_structured_b200 as sa
+    from long_context_structured_b200 import _lib
+    cfg = dict(TREE_WORKLOADS[TREE_ALIASES[args.workload]])
+    if args.heads:
+        cfg["Hq"] = cfg["Hkv"] = args.heads
+    job = TreeJob(cfg, seed=rank, dev=dev)
+    lib = _lib.load()
+    for _ in range(args.warmup):
+        job.step()
+    torch.cuda.synchronize()
+    if sa.stream_status() != 0:
+        raise RuntimeError("device status word reports a failure after warm-up")
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    profile_collect(lib)
+    lib.sattn_profile_enable(1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        job.step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    lib.sattn_profile_enable(0)
+    clk = clocks.stop()
+    prof = profile_collect(lib)
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    value = job.flops * world / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    work = job.group_work()
+    kernels, roof = {}, None
+    for g in sorted(prof):
+        n, ms = prof[g]
+        avg = ms / args.steps
+        kernels[g] = {"kernel": kernel_name(None, g), "launches": n, "ms_per_step": round(avg, 5),
+                      "share": round(ms / max(sum(v[1] for v in prof.values()), 1e-12), 4)}
+        if g in work and avg > 0:
+            r = roofline_of(g, work[g], avg, peaks, peak_src)
+            kernels[g].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+    dom = max((g for g in prof if g in work), key=lambda g: prof[g][1], default=None)
+    if dom is not None:
+        roof = roofline_of(dom, work[dom], prof[dom][1] / args.steps, peaks, peak_src)
+        roof["kernel"] = kernel_name(None, dom)
+        roof["traffic"] = None
+    n_e2e = max(3, min(10, args.steps))
+    outs = job.host_step()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(n_e2e):
+        outs = job.host_step()
+    s1.record()
+    torch.cuda.synchronize()
+    ms_e2e = s0.elapsed_time(s1) / n_e2e
+    cpu = cpu_baseline_tree(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    c = cfg
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": "SharedLLM tree cross-attention (language-modelling policy): %d decoder queries over "
+                               "a %d-token context in %d chunks of %d, depth %d, leaf rate %d (%d kept rows)"
+                               % (c["Tq"], c["n_chunks"] * c["chunk_len"], c["n_chunks"], c["chunk_len"], c["depth"],
+                                  c["alpha_leaf"], job.S),
+                   "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "d": c["d"], "rope_theta": c["rope_theta"],
+                   "pairs_per_rank": job.pairs,
+                   "l2": "no flush: each step reads the %d MB context K/V and writes the kept rows, > 126 MB L2"
+                         % (job.h2d_bytes() >> 20)},
+        "tokens_per_s": round(c["B"] * c["Tq"] * world / (ms_step * 1e-3), 1),
+        "frac_of_bf16_peak": round(value / world / float(peaks["bf16_tflops"]), 4),
+        "roofline": roof, "kernels": kernels, "gpu_launches": sum(n for n, _ in prof.values()),
+        "e2e": {"value": round(job.flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 3), "steps": n_e2e, "h2d_bytes_per_step": job.h2d_bytes(),
+                "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
+                "path": "long_context_structured_b200.tree_cross_fwd on inputs from pinned host memory"},
+        "cpu_baseline": cpu, "clocks": clk, "device_status": sa.stream_status(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
@@ -755,6 +941,20 @@ def run_reference(args):
     from oracle import oracle as O
     O.build()
     decode = args.workload in DECODE_ALIASES
+    if args.workload in TREE_ALIASES:
+        cfg = TREE_WORKLOADS[TREE_ALIASES[args.workload]]
+        t0 = time.perf_counter()
+        for _ in range(args.warmup + args.steps):
+            cpu = cpu_baseline_tree(cfg, n_rows=8)
+        line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "TFLOP/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round((time.perf_counter() - t0) * 1e3 / (args.warmup + args.steps), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1))", "config": {"workload": "tree_cross_128k (oracle sample)"},
+                "cpu_baseline": cpu,
+                "e2e": {"value": cpu["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     if args.workload in BWD_ALIASES:
         wl = synth.WORKLOADS[BWD_ALIASES[args.workload]]
         t0 = time.perf_counter()
@@ -814,7 +1014,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
-                    + sorted(BWD_ALIASES))
+                    + sorted(BWD_ALIASES) + sorted(TREE_ALIASES))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
