@@ -268,6 +268,46 @@ int sattn_tree_cross_fwd(const sattn_params* p, int32_t n_chunks, int32_t chunk_
                          int32_t alpha_leaf, const void* Q, const void* K, const void* V, void* O, float* lse,
                          int32_t* kept_index, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- SepLLM streaming KV cache ("SepLLM", section 6.2) ----
+ * Per sequence: an Initial cache (a slots, the first a tokens), a Separator
+ * cache (s slots), a Local window (w slots, the newest tokens) and a Past
+ * window that takes what leaves the Local window.  After each append, if the
+ * running size reaches c, Past's separators move (in order) behind the
+ * cached separators, the oldest separators go if more than s would stay,
+ * and the rest of Past is dropped.  Slots are ordered Initial | Separator |
+ * Past | Local (newest last); a decoding step attends over every slot with
+ * rolled positions: key x at rotary position x, the query at the last slot
+ * (the talk page, section "Streaming ARMS").  The state lives in caller-owned
+ * device memory; every decision is taken on the device (no host round trip,
+ * so the calls can be captured in a CUDA graph). */
+typedef struct sattn_stream_config {
+  int32_t B, Hkv, d; /* sequences, kv heads, head dim (64 or 128) */
+  int32_t a, s, w;   /* Initial, Separator, Local window slots (w >= 1) */
+  int32_t c;         /* capacity; a + s + w < c (SATTN_ERR_INVALID_ARG otherwise) */
+} sattn_stream_config;
+
+/* Bytes of device state for cfg (256-byte aligned buffer). */
+int sattn_stream_state_size(const sattn_stream_config* cfg, size_t* bytes);
+/* Empties every sequence's cache. */
+int sattn_stream_reset(const sattn_stream_config* cfg, void* state, size_t state_bytes, void* stream);
+/* Appends one token per sequence: K_new, V_new [B, Hkv, d] bf16 contiguous
+ * device (keys unrotated), is_sep [B] uint8 device or NULL (no separator),
+ * position = the token's index in the stream (recorded per slot). */
+int sattn_stream_append(const sattn_stream_config* cfg, void* state, size_t state_bytes, const void* K_new,
+                        const void* V_new, const uint8_t* is_sep, int64_t position, void* stream);
+/* Synchronises `stream`, then copies the region sizes [B, 4] (Initial,
+ * Separator, Past, Local) and, if positions != NULL, the stream index of
+ * every slot [B, c] to host memory. */
+int sattn_stream_read(const sattn_stream_config* cfg, const void* state, size_t state_bytes, int32_t* sizes,
+                      int32_t* positions, void* stream);
+/* Workspace for sattn_stream_decode: p gives Hq (Hq / Hkv in 1, 2, 4, 8),
+ * rope_theta, rope_pos_scale and the q / o strides; B, Hkv, d equal cfg's. */
+int sattn_stream_decode_workspace_size(const sattn_stream_config* cfg, const sattn_params* p, size_t* bytes);
+/* One decoding step per sequence over its cache (after the token's append):
+ * Q [B, Hq, 1, d] bf16 device, O [B, Hq, 1, d] bf16 out, lse [B, Hq] fp32 out. */
+int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, const void* state, size_t state_bytes,
+                        const void* Q, void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and reads the device status word of `ws` into
  * *device_status (SATTN_OK or SATTN_ERR_TIMEOUT).  Returns SATTN_ERR_CUDA if
  * the synchronisation itself failed (the CUDA error is then sticky). */

@@ -304,6 +304,82 @@ def tree_cross_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_chunk
     return out, lse
 
 
+class StreamKV:
+    """SepLLM's streaming KV cache (Initial | Separator | Past | Local) for B
+    sequences, its state in device memory.  ``append`` adds one token per
+    sequence (compacting on the device when the capacity is reached);
+    ``decode`` is one step of the newest tokens' queries over the cache with
+    rolled positions."""
+
+    def __init__(self, B: int, Hkv: int, d: int, a: int, s: int, w: int, c: int, device="cuda"):
+        self.cfg = _lib.StreamConfig(B, Hkv, d, a, s, w, c)
+        self.device = torch.device(device)
+        n = ctypes.c_size_t(0)
+        L = _lib.load()
+        _lib.check(L.sattn_stream_state_size(ctypes.byref(self.cfg), ctypes.byref(n)), "sattn_stream_state_size")
+        self.nbytes = int(n.value)
+        self.state = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=self.device)
+        off = (-self.state.data_ptr()) % 256
+        self.state = self.state[off:off + self.nbytes]
+        self.position = 0
+        self.reset()
+
+    def reset(self):
+        _lib.check(_lib.load().sattn_stream_reset(ctypes.byref(self.cfg), _ptr(self.state), self.nbytes,
+                                                  _stream_ptr(self.device)), "sattn_stream_reset")
+        self.position = 0
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, is_sep: Optional[torch.Tensor] = None):
+        """k_new, v_new [B, Hkv, d] bf16 (keys unrotated); is_sep [B] (0/1)."""
+        k_new, v_new = k_new.contiguous(), v_new.contiguous()
+        if is_sep is not None:
+            is_sep = is_sep.to(torch.uint8).contiguous()
+        rc = _lib.load().sattn_stream_append(ctypes.byref(self.cfg), _ptr(self.state), self.nbytes, _ptr(k_new),
+                                             _ptr(v_new), _ptr(is_sep), self.position, _stream_ptr(self.device))
+        _lib.check(rc, "sattn_stream_append")
+        self.position += 1
+
+    def read(self):
+        """(sizes [B, 4] Initial/Separator/Past/Local, stream position per slot [B, c]) as numpy."""
+        import numpy as np
+        sizes = np.zeros((self.cfg.B, 4), dtype=np.int32)
+        pos = np.zeros((self.cfg.B, self.cfg.c), dtype=np.int32)
+        rc = _lib.load().sattn_stream_read(ctypes.byref(self.cfg), _ptr(self.state), self.nbytes,
+                                           sizes.ctypes.data_as(ctypes.c_void_p), pos.ctypes.data_as(ctypes.c_void_p),
+                                           _stream_ptr(self.device))
+        _lib.check(rc, "sattn_stream_read")
+        return sizes, pos
+
+    def decode(self, q: torch.Tensor, rope_theta: float = 0.0, rope_pos_scale: float = 1.0,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None):
+        """q [B, Hq, 1, d] bf16 -> (O [B, Hq, 1, d], lse [B, Hq])."""
+        B, Hq, one, d = q.shape
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        p = _lib.SattnParams()
+        p.B, p.Hq, p.Hkv, p.T, p.d = B, Hq, self.cfg.Hkv, self.cfg.c, d
+        p.dtype = _dtype_code(q)
+        for name, t in (("q_stride", q), ("o_stride", out)):
+            st = _strides(t)
+            arr = getattr(p, name)
+            arr[0], arr[1], arr[2] = st
+        p.rope_theta = float(rope_theta)
+        p.rope_pos_scale = float(rope_pos_scale)
+        n = ctypes.c_size_t(0)
+        L = _lib.load()
+        _lib.check(L.sattn_stream_decode_workspace_size(ctypes.byref(self.cfg), ctypes.byref(p), ctypes.byref(n)),
+                   "sattn_stream_decode_workspace_size")
+        nbytes = int(n.value)
+        ws = _workspace(nbytes, q.device, workspace)
+        rc = L.sattn_stream_decode(ctypes.byref(self.cfg), ctypes.byref(p), _ptr(self.state), self.nbytes, _ptr(q),
+                                   _ptr(out), _ptr(lse), _ptr(ws), nbytes, _stream_ptr(q.device))
+        _lib.check(rc, "sattn_stream_decode")
+        return out, lse
+
+
 def stream_status(workspace: Optional[torch.Tensor] = None, device="cuda") -> int:
     """Synchronise the current stream and read the device status word of the
     workspace (the cached one when None)."""

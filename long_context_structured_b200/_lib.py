@@ -25,10 +25,15 @@ EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
     "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_bwd_workspace_size", "sattn_bwd",
-    "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd",
+    "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd", "sattn_stream_state_size", "sattn_stream_reset",
+    "sattn_stream_append", "sattn_stream_read", "sattn_stream_decode_workspace_size", "sattn_stream_decode",
     "sattn_stream_status",
     "sattn_build_blockmap_noalloc", "sattn_selftest_wait_timeout", "sattn_profile_enable", "sattn_profile_collect",
 )
+
+
+class StreamConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hkv", "d", "a", "s", "w", "c")]
 
 
 class SattnParams(ctypes.Structure):
@@ -93,6 +98,19 @@ def load():
         L.sattn_tree_cross_workspace_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
         L.sattn_tree_cross_fwd.restype = ctypes.c_int
         L.sattn_tree_cross_fwd.argtypes = [P, i32, i32, i32, i32] + [vp] * 7 + [sz, vp]
+        SC = ctypes.POINTER(StreamConfig)
+        L.sattn_stream_state_size.restype = ctypes.c_int
+        L.sattn_stream_state_size.argtypes = [SC, ctypes.POINTER(sz)]
+        L.sattn_stream_reset.restype = ctypes.c_int
+        L.sattn_stream_reset.argtypes = [SC, vp, sz, vp]
+        L.sattn_stream_append.restype = ctypes.c_int
+        L.sattn_stream_append.argtypes = [SC, vp, sz, vp, vp, vp, ctypes.c_int64, vp]
+        L.sattn_stream_read.restype = ctypes.c_int
+        L.sattn_stream_read.argtypes = [SC, vp, sz, vp, vp, vp]
+        L.sattn_stream_decode_workspace_size.restype = ctypes.c_int
+        L.sattn_stream_decode_workspace_size.argtypes = [SC, P, ctypes.POINTER(sz)]
+        L.sattn_stream_decode.restype = ctypes.c_int
+        L.sattn_stream_decode.argtypes = [SC, P, vp, sz, vp, vp, vp, vp, sz, vp]
         L.sattn_stream_status.restype = ctypes.c_int
         L.sattn_stream_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.sattn_build_blockmap_noalloc.restype = ctypes.c_int

@@ -1304,6 +1304,208 @@ int sattn_tree_cross_fwd(const sattn_params* p, int32_t n_chunks, int32_t chunk_
   return cuda_rc(launch_attn_tc2(a, m, st));
 }
 
+// ---------------------------------------------------------------------------
+// streaming KV cache
+// ---------------------------------------------------------------------------
+
+struct StreamLayout {
+  Region sizes, len, ctrl, pos, flag, dst, k, v, ks, vs, pos_s, flag_s;
+  size_t total = 0;
+};
+
+static int stream_layout(const sattn_stream_config* cfg, StreamLayout* out) {
+  if (!cfg) return SATTN_ERR_INVALID_ARG;
+  if (cfg->B < 1 || cfg->Hkv < 1 || cfg->a < 0 || cfg->s < 0 || cfg->w < 1) return SATTN_ERR_INVALID_ARG;
+  if ((int64_t)cfg->a + cfg->s + cfg->w >= cfg->c) return SATTN_ERR_INVALID_ARG;  // a full cache could not shrink
+  if (cfg->d != 64 && cfg->d != 128) return SATTN_ERR_UNSUPPORTED;
+  if (cfg->c > (1 << 24)) return SATTN_ERR_UNSUPPORTED;
+  const size_t B = cfg->B, H = cfg->Hkv, c = cfg->c, d = cfg->d;
+  StreamLayout L;
+  Alloc A;
+  L.sizes = A.take(B * 4 * 4);
+  L.len = A.take(B * 4);
+  L.ctrl = A.take(B * 2 * 4);
+  L.pos = A.take(B * c * 4);
+  L.flag = A.take(B * c);
+  L.dst = A.take(B * c * 4);
+  L.k = A.take(B * H * c * d * 2);
+  L.v = A.take(B * H * c * d * 2);
+  L.ks = A.take(B * H * c * d * 2);
+  L.vs = A.take(B * H * c * d * 2);
+  L.pos_s = A.take(B * c * 4);
+  L.flag_s = A.take(B * c);
+  L.total = A.cur;
+  *out = L;
+  return SATTN_OK;
+}
+
+static StreamArgs stream_args(const sattn_stream_config* cfg, const StreamLayout& L, void* state) {
+  StreamArgs a{};
+  a.B = cfg->B;
+  a.Hkv = cfg->Hkv;
+  a.d = cfg->d;
+  a.a = cfg->a;
+  a.s = cfg->s;
+  a.w = cfg->w;
+  a.c = cfg->c;
+  a.sizes = at<int32_t>(state, L.sizes);
+  a.len = at<int32_t>(state, L.len);
+  a.ctrl = at<int32_t>(state, L.ctrl);
+  a.pos = at<int32_t>(state, L.pos);
+  a.flag = at<uint8_t>(state, L.flag);
+  a.dst = at<int32_t>(state, L.dst);
+  a.K = at<__nv_bfloat16>(state, L.k);
+  a.V = at<__nv_bfloat16>(state, L.v);
+  a.Ks = at<__nv_bfloat16>(state, L.ks);
+  a.Vs = at<__nv_bfloat16>(state, L.vs);
+  a.pos_s = at<int32_t>(state, L.pos_s);
+  a.flag_s = at<uint8_t>(state, L.flag_s);
+  return a;
+}
+
+int sattn_stream_state_size(const sattn_stream_config* cfg, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  StreamLayout L;
+  int rc = stream_layout(cfg, &L);
+  if (rc) return rc;
+  *bytes = L.total;
+  return SATTN_OK;
+}
+
+static int stream_check_state(const sattn_stream_config* cfg, const void* state, size_t state_bytes,
+                              StreamLayout* L) {
+  int rc = stream_layout(cfg, L);
+  if (rc) return rc;
+  if (!state || state_bytes < L->total || (reinterpret_cast<uintptr_t>(state) & 255u)) return SATTN_ERR_INVALID_ARG;
+  return SATTN_OK;
+}
+
+int sattn_stream_reset(const sattn_stream_config* cfg, void* state, size_t state_bytes, void* stream) {
+  StreamLayout L;
+  int rc = stream_check_state(cfg, state, state_bytes, &L);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // sizes, lengths and plan flags start at zero (the three regions are contiguous)
+  SATTN_TRY(cudaMemsetAsync(state, 0, L.pos.off, st));
+  return SATTN_OK;
+}
+
+int sattn_stream_append(const sattn_stream_config* cfg, void* state, size_t state_bytes, const void* K_new,
+                        const void* V_new, const uint8_t* is_sep, int64_t position, void* stream) {
+  StreamLayout L;
+  int rc = stream_check_state(cfg, state, state_bytes, &L);
+  if (rc) return rc;
+  if (!K_new || !V_new || !aligned16(K_new) || !aligned16(V_new)) return SATTN_ERR_INVALID_ARG;
+  if (position < 0 || position > INT32_MAX) return SATTN_ERR_INVALID_ARG;
+  StreamArgs a = stream_args(cfg, L, state);
+  a.position = position;
+  a.K_new = static_cast<const __nv_bfloat16*>(K_new);
+  a.V_new = static_cast<const __nv_bfloat16*>(V_new);
+  a.sep_new = is_sep;
+  ProfScope ps("stream_append", 4, static_cast<cudaStream_t>(stream));
+  return cuda_rc(launch_stream_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sattn_stream_read(const sattn_stream_config* cfg, const void* state, size_t state_bytes, int32_t* sizes,
+                      int32_t* positions, void* stream) {
+  StreamLayout L;
+  int rc = stream_check_state(cfg, state, state_bytes, &L);
+  if (rc) return rc;
+  if (!sizes) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SATTN_ERR_CUDA;
+  const uint8_t* base = static_cast<const uint8_t*>(state);
+  if (cudaMemcpy(sizes, base + L.sizes.off, (size_t)cfg->B * 4 * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  if (positions && cudaMemcpy(positions, base + L.pos.off, (size_t)cfg->B * cfg->c * 4, cudaMemcpyDeviceToHost) !=
+                       cudaSuccess)
+    return SATTN_ERR_CUDA;
+  return SATTN_OK;
+}
+
+static int plan_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, DecPlan* out) {
+  StreamLayout L;
+  int rc = stream_layout(cfg, &L);
+  if (rc) return rc;
+  if (!p || p->B != cfg->B || p->Hkv != cfg->Hkv || p->d != cfg->d || p->dtype != SATTN_DTYPE_BF16)
+    return SATTN_ERR_INVALID_ARG;
+  if (p->Hq < 1 || p->Hq % p->Hkv) return SATTN_ERR_INVALID_ARG;
+  const int rep = p->Hq / p->Hkv;
+  if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return SATTN_ERR_UNSUPPORTED;
+  if (!(p->rope_theta >= 0.0) || !(p->rope_pos_scale >= 0.0) || p->rope_pos_scale > 1.0) return SATTN_ERR_INVALID_ARG;
+  DecPlan P{};
+  P.nQT = (cfg->c + kTile - 1) / kTile;
+  P.npos = cfg->c;
+  P.n_chunks = decode_chunks(cfg->c);
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (p->d / 2) * sizeof(float2));
+  P.part = A.take((size_t)p->B * p->Hq * (size_t)P.n_chunks * (p->d + 2) * 4);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_stream_decode_workspace_size(const sattn_stream_config* cfg, const sattn_params* p, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  DecPlan P;
+  int rc = plan_stream_decode(cfg, p, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, const void* state, size_t state_bytes,
+                        const void* Q, void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  DecPlan P;
+  int rc = plan_stream_decode(cfg, p, &P);
+  if (rc) return rc;
+  StreamLayout L;
+  rc = stream_check_state(cfg, state, state_bytes, &L);
+  if (rc) return rc;
+  if (!Q || !O || !lse || !aligned16(Q) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+  }
+  void* sp = const_cast<void*>(state);
+  const int64_t H = cfg->Hkv, c = cfg->c, d = cfg->d;
+  DecodeArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = cfg->c;
+  a.d = p->d;
+  a.n_start = 0;
+  a.window = cfg->c;  // every cached entry is kept
+  a.L = 0;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.K = at<__nv_bfloat16>(sp, L.k);
+  a.k_sb = H * c * d;
+  a.k_sh = c * d;
+  a.k_st = d;
+  a.V = at<__nv_bfloat16>(sp, L.v);
+  a.v_sb = H * c * d;
+  a.v_sh = c * d;
+  a.v_st = d;
+  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  a.seq_len = at<int32_t>(sp, L.len);
+  a.part = at<float>(ws, P.part);
+  a.n_chunks = P.n_chunks;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.lse = lse;
+  ProfScope ps("stream_decode", 2, st);
+  return cuda_rc(launch_decode(a, st));
+}
+
 int sattn_stream_status(void* stream, const void* ws, int32_t* device_status) {
   if (!ws || !device_status) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

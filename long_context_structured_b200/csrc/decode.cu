@@ -36,10 +36,15 @@ struct KeySet {
   __device__ __forceinline__ int n() const { return n_sink + n_win + n_sep; }
 };
 
+// cache length of sequence b: the per-sequence length when given (a
+// streaming cache), else T
+__device__ __forceinline__ int cache_len(const DecodeArgs& a, int b) { return a.seq_len ? a.seq_len[b] : a.T; }
+
 __device__ __forceinline__ KeySet key_set(const DecodeArgs& a, int b) {
   KeySet s;
-  const int i = a.T - 1;
-  s.n_sink = min(a.n_start, a.T);
+  const int Tb = cache_len(a, b);
+  const int i = Tb - 1;
+  s.n_sink = min(a.n_start, Tb);
   s.win_lo = max(s.n_sink, i - a.window);
   s.n_win = max(0, i - s.win_lo + 1);
   const int thr = i - a.window;  // separators kept: n_start <= j < i - w
@@ -69,7 +74,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
   const int e_begin = blockIdx.x * kChunk;
   if (e_begin >= ks.n()) return;  // this batch has fewer chunks
   const int e_end = min(ks.n(), e_begin + kChunk);
-  const int i = a.T - 1;
+  const int i = cache_len(a, b) - 1;
   const int c0 = PPL * lane;
 
   // the query of each head of the group, rotated to i (qi) and to the cap (qc), fp32

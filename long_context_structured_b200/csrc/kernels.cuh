@@ -163,6 +163,30 @@ cudaError_t launch_tree_prep(const TreeArgs& a, cudaStream_t st);
 int tree_kept_count(int chunk_len, int depth, int alpha_leaf);  // host; < 0 on bad arguments
 
 // ---------------------------------------------------------------------------
+// streaming KV cache (SepLLM's Initial | Separator | Past | Local)
+// ---------------------------------------------------------------------------
+struct StreamArgs {
+  int B, Hkv, d, a, s, w, c;
+  int64_t position;                 // stream index of the appended token
+  const __nv_bfloat16* K_new;       // [B, Hkv, d]
+  const __nv_bfloat16* V_new;
+  const uint8_t* sep_new;           // [B] or null
+  int32_t* sizes;                   // [B, 4]: Initial, Separator, Past, Local
+  int32_t* len;                     // [B] cache length (sum of the sizes)
+  int32_t* ctrl;                    // [B, 2]: compacting, slots before the compaction
+  int32_t* pos;                     // [B, c] stream index per slot
+  uint8_t* flag;                    // [B, c] separator flag per slot
+  int32_t* dst;                     // [B, c] compaction destination (-1: dropped)
+  __nv_bfloat16* K;                 // [B, Hkv, c, d]
+  __nv_bfloat16* V;
+  __nv_bfloat16* Ks;                // scratch copies for compaction
+  __nv_bfloat16* Vs;
+  int32_t* pos_s;
+  uint8_t* flag_s;
+};
+cudaError_t launch_stream_append(const StreamArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
 // backward pass, fp32 on CUDA cores
 // ---------------------------------------------------------------------------
 struct BwdF32Args {
@@ -326,6 +350,7 @@ struct DecodeArgs {
   const float2* tab;            // rotary table or null
   const int32_t* sep_prefix;    // [B, T+1] or null (no separators)
   const int32_t* sep_pos;       // [B, T]
+  const int32_t* seq_len;       // [B] cache length per sequence (<= T), or null: T for all
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
   int alibi;                    // ALiBi bias clipped at L (no rotation)
   int n_chunks;
