@@ -43,6 +43,12 @@ from long_context_structured_b200 import synth  # noqa: E402
 # decoding steps (one new token per sequence) over the caches of these workloads
 DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
 BWD_ALIASES = {"c2b": "c2_lminf_16k", "c3b": "c3_sepllm_gqa_8k"}
+STREAM_ALIASES = {"c3s": "stream_sepllm_gqa"}
+# SepLLM streaming generation: 16 sequences of the Llama-3-8B-shaped layer
+# (32 query / 8 kv heads, d = 128) with a 4096-slot cache (a = 4 initial,
+# s = 1024 separator, w = 2048 local slots), separators at rate 0.1
+STREAM_WORKLOADS = {"stream_sepllm_gqa": dict(B=16, Hq=32, Hkv=8, d=128, a=4, s=1024, w=2048, c=4096, rate=0.1,
+                                              rope_theta=5e5, warm_tokens=6144)}
 TREE_ALIASES = {"c6t": "tree_cross_128k"}
 # SharedLLM tree cross-attention: a 128K-token context in 64 chunks of 2048,
 # depth 3, leaf rate 2 (global compression 4), 4096 decoder queries
@@ -517,6 +523,49 @@ class TreeJob:
                 "tree_prep": ("hbm", 2 * rows_q + 4 * kept, "B")}
 
 
+class StreamJob:
+    """Streaming generation over SepLLM's four-part cache: each step appends
+    one token per sequence (compacting on the device when full) and decodes
+    its query over the cache.  The cache is warmed past several compactions
+    first; steps cycle through precomputed token rows."""
+
+    def __init__(self, cfg, seed, dev):
+        import torch
+
+        import long_context_structured_b200 as sa
+        self.sa, self.torch, self.cfg, self.dev = sa, torch, cfg, dev
+        c = cfg
+        g = torch.Generator().manual_seed(seed)
+        self.n_rows = 64
+        self.k = torch.randn(self.n_rows, c["B"], c["Hkv"], c["d"], generator=g).bfloat16().to(dev)
+        self.v = torch.randn(self.n_rows, c["B"], c["Hkv"], c["d"], generator=g).bfloat16().to(dev)
+        self.q = torch.randn(self.n_rows, c["B"], c["Hq"], 1, c["d"], generator=g).bfloat16().to(dev)
+        self.sep = (torch.rand(self.n_rows, c["B"], generator=g) < c["rate"]).to(torch.uint8).to(dev)
+        self.cache = sa.StreamKV(c["B"], c["Hkv"], c["d"], c["a"], c["s"], c["w"], c["c"], device=dev)
+        self.O = torch.empty(c["B"], c["Hq"], 1, c["d"], dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(c["B"], c["Hq"], dtype=torch.float32, device=dev)
+        self.t = 0
+        for _ in range(c["warm_tokens"]):
+            self.append_only()
+        torch.cuda.synchronize()
+        sizes, _ = self.cache.read()
+        self.len = sizes.sum(axis=1)
+
+    def append_only(self):
+        r = self.t % self.n_rows
+        self.cache.append(self.k[r], self.v[r], self.sep[r])
+        self.t += 1
+
+    def step(self):
+        r = self.t % self.n_rows
+        self.append_only()
+        self.cache.decode(self.q[r], rope_theta=self.cfg["rope_theta"], out=self.O, lse=self.lse)
+
+    def mean_len(self):
+        sizes, _ = self.cache.read()
+        return float(sizes.sum(axis=1).mean())
+
+
 def cpu_baseline_tree(cfg, n_rows=256):
     from oracle import oracle as O
     O.build()
@@ -617,6 +666,8 @@ def run_ours(args):
     tree = args.workload in TREE_ALIASES
     if tree:
         return run_tree(args, world, rank, dev)
+    if args.workload in STREAM_ALIASES:
+        return run_stream(args, world, rank, dev)
     aliases = DECODE_ALIASES if decode else (BWD_ALIASES if backward else WORKLOAD_ALIASES)
     wl = synth.WORKLOADS[aliases.get(args.workload, args.workload)]
     if args.heads:
@@ -848,6 +899,90 @@ def run_tree(args, world, rank, dev):
     print(json.dumps(line), flush=True)
 
 
+def run_stream(args, world, rank, dev):
+    """Streaming generation steps over the device-resident cache."""
+    import torch
+    import torch.distributed as dist
+
+    import long_context_structured_b200 as sa
+    from long_context_structured_b200 import _lib
+    cfg = dict(STREAM_WORKLOADS[STREAM_ALIASES[args.workload]])
+    job = StreamJob(cfg, seed=rank, dev=dev)
+    lib = _lib.load()
+    for _ in range(args.warmup):
+        job.step()
+    torch.cuda.synchronize()
+    len0 = job.mean_len()
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    profile_collect(lib)
+    lib.sattn_profile_enable(1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        job.step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    lib.sattn_profile_enable(0)
+    clk = clocks.stop()
+    prof = profile_collect(lib)
+    len1 = job.mean_len()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    c = cfg
+    mean_len = 0.5 * (len0 + len1)  # cached keys per sequence, averaged over the timed steps
+    flops = 4.0 * c["d"] * c["Hq"] * c["B"] * mean_len
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    kv_bytes = mean_len * c["B"] * c["Hkv"] * 2 * c["d"] * 2
+    work = {"stream_decode": ("hbm", kv_bytes + 4 * c["B"] * c["Hq"] * c["d"], "B"),
+            "stream_append": ("hbm", 2 * c["B"] * c["Hkv"] * c["d"] * 2 * 2, "B")}
+    kernels = {}
+    for g in sorted(prof):
+        n, ms = prof[g]
+        avg = ms / args.steps
+        kernels[g] = {"kernel": {"stream_decode": "decode_partial_kernel + decode_combine_kernel",
+                                 "stream_append": "stream_append/plan/move kernels"}.get(g, g),
+                      "launches": n, "ms_per_step": round(avg, 5),
+                      "share": round(ms / max(sum(v[1] for v in prof.values()), 1e-12), 4)}
+        if g in work and avg > 0:
+            r = roofline_of(g, work[g], avg, peaks, peak_src)
+            kernels[g].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+    roof = roofline_of("stream_decode", work["stream_decode"], prof["stream_decode"][1] / args.steps, peaks, peak_src)
+    roof["kernel"] = "decode_partial_kernel + decode_combine_kernel"
+    roof["traffic"] = None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) K/V/Q rows, Bernoulli separators)",
+        "config": {"workload": "SepLLM streaming generation: %d sequences, cache a=%d s=%d w=%d c=%d, one token "
+                               "appended (with on-device compaction) and decoded per sequence per step"
+                               % (c["B"], c["a"], c["s"], c["w"], c["c"]),
+                   "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "d": c["d"], "rope_theta": c["rope_theta"],
+                   "mean_cached_keys": round(mean_len, 1), "tokens_appended_before_timing": job.t - args.steps,
+                   "l2": "no flush: the caches hold %d MB of K/V, > 126 MB L2"
+                         % (c["B"] * c["Hkv"] * c["c"] * c["d"] * 4 >> 20)},
+        "tokens_per_s": round(c["B"] * world / (ms_step * 1e-3), 1),
+        "roofline": roof, "kernels": kernels, "gpu_launches": sum(n for n, _ in prof.values()),
+        "e2e": None, "cpu_baseline": None, "clocks": clk, "device_status": sa.stream_status(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
@@ -1014,7 +1149,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
-                    + sorted(BWD_ALIASES) + sorted(TREE_ALIASES))
+                    + sorted(BWD_ALIASES) + sorted(TREE_ALIASES) + sorted(STREAM_ALIASES))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
