@@ -836,6 +836,7 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   const int rep = p->Hq / p->Hkv;
   if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return SATTN_ERR_UNSUPPORTED;
   if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
+  if (p->T > decode_max_len()) return SATTN_ERR_UNSUPPORTED;
   DecPlan P;
   P.nQT = (p->T + kTile - 1) / kTile;
   P.npos = std::max(p->T, p->L_pretrain + 1);
@@ -1433,6 +1434,7 @@ static int plan_stream_decode(const sattn_stream_config* cfg, const sattn_params
   const int rep = p->Hq / p->Hkv;
   if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return SATTN_ERR_UNSUPPORTED;
   if (!(p->rope_theta >= 0.0) || !(p->rope_pos_scale >= 0.0) || p->rope_pos_scale > 1.0) return SATTN_ERR_INVALID_ARG;
+  if (cfg->c > decode_max_len()) return SATTN_ERR_UNSUPPORTED;
   DecPlan P{};
   P.nQT = (cfg->c + kTile - 1) / kTile;
   P.npos = cfg->c;

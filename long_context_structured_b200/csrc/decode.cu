@@ -11,16 +11,20 @@
 //
 // Split-K over the kept keys (memory-bound: each kept K and V row is read
 // once): a CTA takes a chunk of kChunk kept keys of one (batch, kv head) for
-// all query heads of that kv head's group; each warp walks its keys with the
-// head dimension spread over the lanes (a lane owns rotary pairs
-// c = PPL*lane .. PPL*lane + PPL - 1 and their partners c + d/2), loads kU
-// keys' K, V and rotary entries before using any of them, and keeps an
-// online softmax per query head.  The chunk's (max, sum, unnormalised O)
-// per head go to the workspace; a second kernel merges the chunks.
+// all query heads of that kv head's group; each warp walks its 32 keys with
+// the head dimension spread over the lanes (a lane owns rotary pairs
+// c = PPL*lane .. PPL*lane + PPL - 1 and their partners c + d/2), first the
+// logits (several keys' K rows and rotary entries loaded before any is
+// used), then, with the chunk's per-head maximum known, the weighted V rows.
+// The chunk's (max, sum, unnormalised O) per head go to the workspace; a
+// second kernel merges the chunks.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "kernels.cuh"
+#include "simt.cuh"
 #include "sm100.cuh"
 
 namespace sattn {
@@ -29,7 +33,6 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kChunk = 128;  // kept keys per CTA
-constexpr int kU = 4;        // keys per warp whose loads are in flight together
 
 struct KeySet {
   int n_sink, win_lo, n_win, n_sep;
@@ -59,184 +62,303 @@ __device__ __forceinline__ int key_at(const DecodeArgs& a, const KeySet& s, int 
   return a.sep_pos[(size_t)b * a.T + (e - s.n_win)];
 }
 
-// grid (ceil(T / kChunk), B * Hkv)
+// grid (B * Hkv, chunks): the (batch, kv head) index varies fastest, so the
+// chunks that hold keys (the low ones) are dispatched before the empty ones.
+//
+// A key is spread over LPK lanes (8, or 16 for eight query heads per kv
+// head), each holding EPL rotary pairs (16 or 8 elements of the row), so a
+// warp works on 32 / LPK keys at once with 16-byte loads.  Two passes over
+// the CTA's chunk of kept keys: (1) logits -- the raw key rotated on the fly
+// to R(j) k_j, or for a capped key (i - j > L) to R(i - L) k_j, which gives
+// the capped logit <R(L) q, k_j> = <R(i) q, R(i - L) k_j> with the one query
+// R(i) q; the lanes' partial dot products of all heads summed by one
+// transposed butterfly over the key's lanes; logits to shared memory; (2)
+// with the chunk's per-head maximum and the weights p = 2^(z - m) taken once
+// per (key, head): O += p v.  No running rescale.
 template <int D, int REP>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
   constexpr int half = D / 2;
-  constexpr int PPL = half / 32;  // rotary pairs per lane: 2 (d = 128) or 1 (d = 64)
-  __shared__ float red_m[kThreads / 32][REP];
-  __shared__ float red_l[kThreads / 32][REP];
+  constexpr int LPK = (REP >= 8) ? 16 : 8;      // lanes per key
+  constexpr int KPS = 32 / LPK;                 // keys per warp step
+  constexpr int EPL = half / LPK;               // rotary pairs per lane
+  constexpr int KPW = kChunk / (kThreads / 32);  // keys per warp: 32
+  constexpr int UNR = (REP >= 4) ? 1 : 2;       // warp steps whose loads are in flight together
+  static_assert(REP <= LPK && KPW % (KPS * UNR) == 0 && (EPL == 8 || EPL == 4 || EPL == 2), "decode tiling");
+  __shared__ float s_p[REP][kChunk];            // logits, then weights
+  __shared__ float s_m[REP], s_l[REP];
   __shared__ float red_o[kThreads / 32][REP][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bg = blockIdx.y;
+  const int sub = lane % LPK, kg = lane / LPK;
+  const int bg = blockIdx.x;
   const int g = bg % a.Hkv, b = bg / a.Hkv;
   const KeySet ks = key_set(a, b);
-  const int e_begin = blockIdx.x * kChunk;
+  const int e_begin = blockIdx.y * kChunk;
   if (e_begin >= ks.n()) return;  // this batch has fewer chunks
-  const int e_end = min(ks.n(), e_begin + kChunk);
+  const int n_here = min(ks.n() - e_begin, kChunk);
   const int i = cache_len(a, b) - 1;
-  const int c0 = PPL * lane;
+  const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
 
-  // the query of each head of the group, rotated to i (qi) and to the cap (qc), fp32
-  float qi0[REP][PPL], qi1[REP][PPL], qc0[REP][PPL], qc1[REP][PPL];
+  // the query of each head rotated to i, fp32
+  float q0[REP][EPL], q1[REP][EPL];
 #pragma unroll
   for (int r = 0; r < REP; ++r) {
-    const int h = g * REP + r;
-    const __nv_bfloat16* qp = a.Q + (size_t)b * a.q_sb + (size_t)h * a.q_sh;
+    const __nv_bfloat16* qp = a.Q + (size_t)b * a.q_sb + (size_t)(g * REP + r) * a.q_sh;
 #pragma unroll
-    for (int e = 0; e < PPL; ++e) {
-      const int c = c0 + e;
-      const float x0 = __bfloat162float(qp[c]), x1 = __bfloat162float(qp[c + half]);
-      const float2 ti = a.tab ? a.tab[(size_t)i * half + c] : make_float2(1.f, 0.f);
-      const float2 tl = (a.tab && a.L > 0) ? a.tab[(size_t)a.L * half + c] : make_float2(1.f, 0.f);
-      qi0[r][e] = x0 * ti.x - x1 * ti.y;
-      qi1[r][e] = x1 * ti.x + x0 * ti.y;
-      qc0[r][e] = x0 * tl.x - x1 * tl.y;
-      qc1[r][e] = x1 * tl.x + x0 * tl.y;
+    for (int e = 0; e < EPL; ++e) {
+      const float x0 = __bfloat162float(qp[p0 + e]), x1 = __bfloat162float(qp[p0 + e + half]);
+      const float2 t = a.tab ? a.tab[(size_t)i * half + p0 + e] : make_float2(1.f, 0.f);
+      q0[r][e] = x0 * t.x - x1 * t.y;
+      q1[r][e] = x1 * t.x + x0 * t.y;
     }
-  }
-  float m[REP], l[REP], o0[REP][PPL], o1[REP][PPL];
-#pragma unroll
-  for (int r = 0; r < REP; ++r) {
-    m[r] = -CUDART_INF_F;
-    l[r] = 0.f;
-#pragma unroll
-    for (int e = 0; e < PPL; ++e) o0[r][e] = o1[r][e] = 0.f;
   }
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
   const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
   const float sl2 = a.scale_log2;
+  const int w_lo = warp * KPW;
 
-  // warp w takes keys e_begin + w, + 4, ... of the chunk
-  for (int e0 = e_begin + warp; e0 < e_end; e0 += (kThreads / 32) * kU) {
-    int jj[kU];
-    float k0[kU][PPL], k1[kU][PPL], v0[kU][PPL], v1[kU][PPL], cs[kU][PPL], sn[kU][PPL];
+  // EPL consecutive bf16 as floats (16, 8 or 4 bytes)
+  auto load_e = [&](const __nv_bfloat16* p, float* out) {
+    if constexpr (EPL == 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(p);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int e = e0 + u * (kThreads / 32);
-      jj[u] = (e < e_end) ? key_at(a, ks, b, e) : -1;
+      for (int y = 0; y < 4; ++y) {
+        const float2 f = __bfloat1622float2(h[y]);
+        out[2 * y] = f.x;
+        out[2 * y + 1] = f.y;
+      }
+    } else if constexpr (EPL == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        const float2 f = __bfloat1622float2(h[y]);
+        out[2 * y] = f.x;
+        out[2 * y + 1] = f.y;
+      }
+    } else {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+      out[0] = f.x;
+      out[1] = f.y;
     }
+  };
+
+  // ---- pass 1: logits ----
+  for (int u0 = 0; u0 < KPW; u0 += KPS * UNR) {
+    int jj[UNR];
+    float k0[UNR][EPL], k1[UNR][EPL];
+    float2 cs[UNR][EPL];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int j = jj[u] < 0 ? 0 : jj[u];
-      const __nv_bfloat16* kp = kb + (size_t)j * a.k_st;
-      const __nv_bfloat16* vp = vb + (size_t)j * a.v_st;
+    for (int x = 0; x < UNR; ++x) {
+      const int el = w_lo + u0 + x * KPS + kg;
+      jj[x] = (el < n_here) ? key_at(a, ks, b, e_begin + el) : -1;
+      const int j = jj[x] < 0 ? 0 : jj[x];
+      const int rpos = (a.L > 0 && i - j > a.L) ? i - a.L : j;  // capped keys: R(i - L) k_j
+      load_e(kb + (size_t)j * a.k_st + p0, k0[x]);
+      load_e(kb + (size_t)j * a.k_st + p0 + half, k1[x]);
+      if (a.tab) {
+        const float4* tp = reinterpret_cast<const float4*>(a.tab + (size_t)rpos * half + p0);
 #pragma unroll
-      for (int e = 0; e < PPL; ++e) {
-        k0[u][e] = __bfloat162float(kp[c0 + e]);
-        k1[u][e] = __bfloat162float(kp[c0 + e + half]);
-        v0[u][e] = __bfloat162float(vp[c0 + e]);
-        v1[u][e] = __bfloat162float(vp[c0 + e + half]);
-        const float2 t = a.tab ? a.tab[(size_t)j * half + c0 + e] : make_float2(1.f, 0.f);
-        cs[u][e] = t.x;
-        sn[u][e] = t.y;
+        for (int e = 0; e < EPL; e += 2) {
+          const float4 t = tp[e / 2];
+          cs[x][e] = make_float2(t.x, t.y);
+          cs[x][e + 1] = make_float2(t.z, t.w);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) cs[x][e] = make_float2(1.f, 0.f);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      if (jj[u] < 0) continue;  // uniform over the warp
-      const bool capped = a.L > 0 && (i - jj[u]) > a.L;
-      float z[REP];
+    for (int x = 0; x < UNR; ++x) {
+      float v[REP];
 #pragma unroll
-      for (int r = 0; r < REP; ++r) {
-        float acc = 0.f;
+      for (int r = 0; r < REP; ++r) v[r] = 0.f;
 #pragma unroll
-        for (int e = 0; e < PPL; ++e) {
-          if (capped) {
-            acc = fmaf(qc0[r][e], k0[u][e], fmaf(qc1[r][e], k1[u][e], acc));
-          } else {
-            const float kr0 = k0[u][e] * cs[u][e] - k1[u][e] * sn[u][e];
-            const float kr1 = k1[u][e] * cs[u][e] + k0[u][e] * sn[u][e];
-            acc = fmaf(qi0[r][e], kr0, fmaf(qi1[r][e], kr1, acc));
-          }
-        }
+      for (int e = 0; e < EPL; ++e) {
+        const float kr0 = k0[x][e] * cs[x][e].x - k1[x][e] * cs[x][e].y;
+        const float kr1 = k1[x][e] * cs[x][e].x + k0[x][e] * cs[x][e].y;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        z[r] = acc * sl2;
-        if (a.alibi) {  // -m_h * min(i - j, L), in log2 units of the scaled logit
-          const int dist = (a.L > 0) ? min(i - jj[u], a.L) : (i - jj[u]);
-          z[r] -= exp2f(-8.f * (float)(g * REP + r + 1) / (float)a.Hq) * 1.4426950408889634f * (float)dist;
-        }
+        for (int r = 0; r < REP; ++r) v[r] = fmaf(q0[r][e], kr0, fmaf(q1[r][e], kr1, v[r]));
       }
-#pragma unroll
-      for (int r = 0; r < REP; ++r) {
-        const float m_new = fmaxf(m[r], z[r]);
-        const float alpha = ex2_approx(m[r] - m_new);  // 0 on the first key (m = -inf)
-        const float p = ex2_approx(z[r] - m_new);
-        l[r] = l[r] * alpha + p;
-#pragma unroll
-        for (int e = 0; e < PPL; ++e) {
-          o0[r][e] = fmaf(o0[r][e], alpha, p * v0[u][e]);
-          o1[r][e] = fmaf(o1[r][e], alpha, p * v1[u][e]);
+      group_reduce_transposed<REP, LPK>(v, 0xffffffffu, lane);
+      // lane sub now holds head sub / (LPK / REP)
+      constexpr int DUP = LPK / REP;
+      if (sub % DUP == 0) {
+        const int r = sub / DUP;
+        const int j = jj[x];
+        float z = v[0] * sl2;
+        if (a.alibi && j >= 0) {  // -m_h * min(i - j, L), in log2 units of the scaled logit
+          const int dist = (a.L > 0) ? min(i - j, a.L) : (i - j);
+          z -= exp2f(-8.f * (float)(g * REP + r + 1) / (float)a.Hq) * 1.4426950408889634f * (float)dist;
         }
-        m[r] = m_new;
+        s_p[r][w_lo + u0 + x * KPS + kg] = (j >= 0) ? z : -CUDART_INF_F;
       }
     }
   }
-  // merge the four warps of the CTA
+  __syncthreads();
+  // ---- per-head maximum, weights and their sum (warp r takes heads r, r + 4, ...) ----
+  for (int r = warp; r < REP; r += kThreads / 32) {
+    float mx = -CUDART_INF_F;
+    for (int e = lane; e < kChunk; e += 32) mx = fmaxf(mx, s_p[r][e]);
 #pragma unroll
-  for (int r = 0; r < REP; ++r) {
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+    for (int e = lane; e < kChunk; e += 32) {
+      const float p = (mx == -CUDART_INF_F) ? 0.f : ex2_approx(s_p[r][e] - mx);
+      s_p[r][e] = p;
+      sum += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) {
-      red_m[warp][r] = m[r];
-      red_l[warp][r] = l[r];
+      s_m[r] = mx;
+      s_l[r] = sum;
+    }
+  }
+  __syncthreads();
+  // ---- pass 2: O += p v ----
+  float o0[REP][EPL], o1[REP][EPL];
+#pragma unroll
+  for (int r = 0; r < REP; ++r)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o0[r][e] = o1[r][e] = 0.f;
+  for (int u0 = 0; u0 < KPW; u0 += KPS * UNR) {
+    float v0[UNR][EPL], v1[UNR][EPL];
+    int els[UNR];
+#pragma unroll
+    for (int x = 0; x < UNR; ++x) {
+      els[x] = w_lo + u0 + x * KPS + kg;
+      const int j = (els[x] < n_here) ? key_at(a, ks, b, e_begin + els[x]) : 0;
+      load_e(vb + (size_t)j * a.v_st + p0, v0[x]);
+      load_e(vb + (size_t)j * a.v_st + p0 + half, v1[x]);
     }
 #pragma unroll
-    for (int e = 0; e < PPL; ++e) {
-      red_o[warp][r][c0 + e] = o0[r][e];
-      red_o[warp][r][c0 + e + half] = o1[r][e];
+    for (int x = 0; x < UNR; ++x) {
+#pragma unroll
+      for (int r = 0; r < REP; ++r) {
+        const float p = s_p[r][els[x]];  // 0 for keys past the chunk's end
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          o0[r][e] = fmaf(p, v0[x][e], o0[r][e]);
+          o1[r][e] = fmaf(p, v1[x][e], o1[r][e]);
+        }
+      }
     }
+  }
+  // merge the warp's key slots (lanes sub, sub + LPK, ...), then the warps (fixed order)
+#pragma unroll
+  for (int o = LPK; o < 32; o <<= 1)
+#pragma unroll
+    for (int r = 0; r < REP; ++r)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        o0[r][e] += __shfl_xor_sync(0xffffffffu, o0[r][e], o);
+        o1[r][e] += __shfl_xor_sync(0xffffffffu, o1[r][e], o);
+      }
+  if (kg == 0) {
+#pragma unroll
+    for (int r = 0; r < REP; ++r)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        red_o[warp][r][p0 + e] = o0[r][e];
+        red_o[warp][r][p0 + e + half] = o1[r][e];
+      }
   }
   __syncthreads();
   for (int x = threadIdx.x; x < REP * D; x += kThreads) {
     const int r = x / D, c = x % D;
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < kThreads / 32; ++w) M = fmaxf(M, red_m[w][r]);
-    float L = 0.f, O = 0.f;
-    for (int w = 0; w < kThreads / 32; ++w) {
-      const float f = (red_m[w][r] == -CUDART_INF_F) ? 0.f : ex2_approx(red_m[w][r] - M);
-      L += red_l[w][r] * f;
-      O += red_o[w][r][c] * f;
-    }
+    float O = 0.f;
+    for (int w = 0; w < kThreads / 32; ++w) O += red_o[w][r][c];
     const int h = g * REP + r;
-    float* part = a.part + (((size_t)b * a.Hq + h) * a.n_chunks + blockIdx.x) * (D + 2);
+    float* part = a.part + (((size_t)b * a.Hq + h) * a.n_chunks + blockIdx.y) * (D + 2);
     part[2 + c] = O;
     if (c == 0) {
-      part[0] = M;
-      part[1] = L;
+      part[0] = s_m[r];
+      part[1] = s_l[r];
     }
   }
 }
 
-// grid (B * Hq), D threads: merge the chunks of one (batch, head)
+// grid (B * Hq), 4 D threads: merge the chunks of one (batch, head).  The
+// chunk maxima and weights are read in parallel into shared memory; thread
+// group q of 4 sums chunks q, q + 4, ... of each output column (independent
+// loads), then the four groups are added in a fixed order.
+constexpr int kCombineGroups = 4;
+constexpr int kCombineMaxChunks = 4096;
 template <int D>
-__global__ void decode_combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kCombineGroups * D) decode_combine_kernel(DecodeArgs a) {
+  __shared__ float s_f[kCombineMaxChunks];
+  __shared__ float s_red[kCombineGroups * D];
+  __shared__ float s_ml[2];
   const int bh = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const KeySet ks = key_set(a, b);
-  const int nc = (ks.n() + kChunk - 1) / kChunk;
+  const int nc = min((ks.n() + kChunk - 1) / kChunk, kCombineMaxChunks);
   const float* part = a.part + (size_t)bh * a.n_chunks * (D + 2);
-  const int c = threadIdx.x;
-  float M = -CUDART_INF_F;
-  for (int x = 0; x < nc; ++x) M = fmaxf(M, part[x * (D + 2)]);
-  float L = 0.f, O = 0.f;
-  for (int x = 0; x < nc; ++x) {
-    const float mx = part[x * (D + 2)];
-    const float f = (mx == -CUDART_INF_F) ? 0.f : ex2_approx(mx - M);
-    L += part[x * (D + 2) + 1] * f;
-    O += part[x * (D + 2) + 2 + c] * f;
+  const int tid = threadIdx.x;
+  float mx = -CUDART_INF_F;
+  for (int x = tid; x < nc; x += blockDim.x) {
+    s_f[x] = part[(size_t)x * (D + 2)];
+    mx = fmaxf(mx, s_f[x]);
   }
-  __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
-  op[c] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-  if (c == 0) a.lse[bh] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) s_red[tid >> 5] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) M = fmaxf(M, s_red[w]);
+    s_ml[0] = M;
+  }
+  __syncthreads();
+  const float M = s_ml[0];
+  float lsum = 0.f;
+  for (int x = tid; x < nc; x += blockDim.x) {
+    const float f = (s_f[x] == -CUDART_INF_F) ? 0.f : ex2_approx(s_f[x] - M);
+    s_f[x] = f;
+    lsum += part[(size_t)x * (D + 2) + 1] * f;
+  }
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  __syncthreads();  // s_red is reused
+  if ((tid & 31) == 0) s_red[tid >> 5] = lsum;
+  __syncthreads();
+  if (tid == 0) {
+    float L = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) L += s_red[w];
+    s_ml[1] = L;
+  }
+  const int q = tid / D, c = tid % D;
+  float O = 0.f;
+#pragma unroll 4
+  for (int x = q; x < nc; x += kCombineGroups) O = fmaf(part[(size_t)x * (D + 2) + 2 + c], s_f[x], O);
+  __syncthreads();
+  s_red[q * D + c] = O;
+  __syncthreads();
+  if (q == 0) {
+    float Ot = 0.f;
+    for (int y = 0; y < kCombineGroups; ++y) Ot += s_red[y * D + c];
+    const float L = s_ml[1];
+    __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
+    op[c] = __float2bfloat16_rn(L > 0.f ? Ot / L : 0.f);
+    if (c == 0) a.lse[bh] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
+  }
 }
 
 template <int D, int REP>
 cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
-  dim3 grid(a.n_chunks, a.B * a.Hkv);
+  // without separators or per-sequence lengths the kept-key count is a
+  // closed form: launch exactly its chunks
+  int chunks = a.n_chunks;
+  if (!a.sep_prefix && !a.seq_len) {
+    const int i = a.T - 1, ns = std::min(a.n_start, a.T);
+    const int win_lo = std::max(ns, i - a.window);
+    chunks = std::min(chunks, std::max(1, (ns + std::max(0, i - win_lo + 1) + kChunk - 1) / kChunk));
+  }
+  dim3 grid(a.B * a.Hkv, chunks);
   decode_partial_kernel<D, REP><<<grid, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<D><<<a.B * a.Hq, D, 0, st>>>(a);
+  decode_combine_kernel<D><<<a.B * a.Hq, kCombineGroups * D, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -254,6 +376,7 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 int decode_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+int decode_max_len() { return kCombineMaxChunks * kChunk; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;

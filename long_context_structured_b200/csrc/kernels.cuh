@@ -360,6 +360,7 @@ struct DecodeArgs {
 };
 // chunks of kept keys a decoding step of cache length T may need
 int decode_chunks(int T);
+int decode_max_len();  // longest key set one decoding step merges
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 }  // namespace sattn
