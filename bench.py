@@ -43,6 +43,10 @@ from long_context_structured_b200 import synth  # noqa: E402
 # decoding steps (one new token per sequence) over the caches of these workloads
 DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
 BWD_ALIASES = {"c2b": "c2_lminf_16k", "c3b": "c3_sepllm_gqa_8k"}
+# stress sizes for the HBM-bound helpers: the block map on B*T = 2^26 flags
+# (a2s) and the separator gather on the SepLLM layer at 16x its batch (c3x16)
+STRESS_ALIASES = {"a2s": "blockmap_stress_2e26"}
+EXTRA_WORKLOADS = {"c3x16": ("c3_sepllm_gqa_8k", dict(name="c3_sepllm_gqa_8k_x16", B=64))}
 STREAM_ALIASES = {"c3s": "stream_sepllm_gqa"}
 # SepLLM streaming generation: 16 sequences of the Llama-3-8B-shaped layer
 # (32 query / 8 kv heads, d = 128) with a 4096-slot cache (a = 4 initial,
@@ -668,8 +672,14 @@ def run_ours(args):
         return run_tree(args, world, rank, dev)
     if args.workload in STREAM_ALIASES:
         return run_stream(args, world, rank, dev)
+    if args.workload in STRESS_ALIASES:
+        return run_blockmap_stress(args, world, rank, dev)
     aliases = DECODE_ALIASES if decode else (BWD_ALIASES if backward else WORKLOAD_ALIASES)
-    wl = synth.WORKLOADS[aliases.get(args.workload, args.workload)]
+    if args.workload in EXTRA_WORKLOADS:
+        base, kw = EXTRA_WORKLOADS[args.workload]
+        wl = synth.WORKLOADS[base].scaled(**kw)
+    else:
+        wl = synth.WORKLOADS[aliases.get(args.workload, args.workload)]
     if args.heads:
         wl = wl.scaled(Hq=args.heads, Hkv=max(1, args.heads * wl.Hkv // wl.Hq),
                        long_heads=tuple(h for h in wl.long_heads if h < args.heads))
@@ -983,6 +993,58 @@ def run_stream(args, world, rank, dev):
     print(json.dumps(line), flush=True)
 
 
+def run_blockmap_stress(args, world, rank, dev):
+    """The block map at stress size: 2048 sequences of 32768 flags (rate
+    0.1), tile classes included; reported in GB/s of algorithmic bytes (flags
+    read; tile classes, separator positions, counts and ranges written)."""
+    import torch
+
+    import long_context_structured_b200 as sa
+    from long_context_structured_b200 import _lib
+    B, T, ns, w = 2048, 32768, 4, 256
+    g = torch.Generator().manual_seed(rank)
+    flags = (torch.rand(B, T, generator=g) < 0.1).to(torch.uint8).to(dev)
+    lib = _lib.load()
+    for _ in range(args.warmup):
+        sa.build_blockmap(flags, B=B, T=T, n_start=ns, window=w, device=dev)
+    torch.cuda.synchronize()
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    profile_collect(lib)
+    lib.sattn_profile_enable(1)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        sa.build_blockmap(flags, B=B, T=T, n_start=ns, window=w, device=dev)
+    e1.record()
+    torch.cuda.synchronize()
+    lib.sattn_profile_enable(0)
+    clk = clocks.stop()
+    prof = profile_collect(lib)
+    ms = e0.elapsed_time(e1) / args.steps
+    nqt = T // 128
+    nbytes = B * T + B * nqt * nqt + B * T * 4 + B * 4 + B * nqt * 8
+    kms = prof["blockmap"][1] / args.steps
+    peaks, peak_src = load_peaks()
+    roof = roofline_of("blockmap", ("hbm", nbytes, "B"), kms, peaks, peak_src)
+    roof["kernel"] = "sep_scan_kernel + tile_class_kernel"
+    roof["traffic"] = None
+    if rank == 0:
+        print(json.dumps({
+            "metric": "block map GB/s at stress size (algorithmic bytes)", "value": roof["achieved"], "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+            "data": "synthetic (seeded Bernoulli(0.1) separator flags)",
+            "config": {"workload": "block map of %d sequences x %d flags (2^26), n_start %d, window %d, tile classes "
+                                   "%dx%d per sequence" % (B, T, ns, w, nqt, nqt),
+                       "algorithmic_bytes": nbytes,
+                       "l2": "no flush: %d MB read and written per step, > 126 MB L2" % (nbytes >> 20)},
+            "roofline": roof, "kernels": {"blockmap": {"launches": prof["blockmap"][0], "ms_per_step": round(kms, 5)}},
+            "gpu_launches": prof["blockmap"][0], "clocks": clk, "e2e": None, "cpu_baseline": None}), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
@@ -1149,7 +1211,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
-                    + sorted(BWD_ALIASES) + sorted(TREE_ALIASES) + sorted(STREAM_ALIASES))
+                    + sorted(BWD_ALIASES) + sorted(TREE_ALIASES) + sorted(STREAM_ALIASES) + sorted(STRESS_ALIASES)
+                    + sorted(EXTRA_WORKLOADS))
     ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")

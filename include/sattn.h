@@ -318,10 +318,15 @@ int sattn_stream_status(void* stream, const void* ws, int32_t* device_status);
  * an extension running inside a host framework that owns all device memory,
  * or a latency-critical loop where an allocation -- which can synchronise
  * the device -- is not allowed).  Same arguments and outputs as
- * sattn_build_blockmap minus ws/ws_bytes; the scratch (separator prefix
- * counts) lives in a fixed 4 MiB device array that every GPU loading the
- * library keeps until exit.
- *  - B * (T + 1) <= 1048576, else SATTN_ERR_UNSUPPORTED (nothing launched).
+ * sattn_build_blockmap minus ws/ws_bytes; the scratch (a prefix count of
+ * the separator flags and tile-class tables) lives in a fixed 4 MiB device
+ * array that every GPU loading the library keeps until exit.
+ *  - The scratch takes 8 * B * (floor(T / 32) + 1) bytes rounded up to 16,
+ *    plus B * S_f + B * S_m with S_f = nQT rounded up to 16 and
+ *    S_m = 16 * nQT * min(ceil(nQT / 16), floor(bt / 16) + 2), where
+ *    nQT = ceil(T / 128) and bt = min(nQT, ceil(window / 128)).  Above
+ *    4194304 bytes the call returns SATTN_ERR_UNSUPPORTED (nothing
+ *    launched).
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.

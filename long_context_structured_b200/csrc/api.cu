@@ -117,7 +117,7 @@ int plan_fwd(const sattn_params* p, FwdPlan* pl) {
   Alloc A;
   P.status = A.take(kStatusBytes);
   if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
-  P.prefix = A.take(B * (T + 1) * 4);
+  P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
   if (P.bf16) {
     P.qr = A.take(B * Hq * T * d * 2);
     P.kr = A.take(B * Hkv * T * d * 2);
@@ -302,7 +302,7 @@ int run_blockmap(const sattn_params* p, const FwdPlan& P, const uint8_t* is_sep,
   a.n_start = p->n_start;
   a.window = p->window;
   a.is_sep = is_sep;
-  a.prefix = at<int32_t>(ws, P.prefix);
+  a.scratch = at<uint8_t>(ws, P.prefix);
   a.sep_pos = sep_pos;
   a.sep_count = sep_count;
   a.ranges = ranges;
@@ -593,7 +593,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.gather_mode = is_sep ? 1 : 0;
   a.q2 = q2;
   a.sep_pos = sep_pos;
-  a.sep_prefix = at<int32_t>(ws, P.prefix);
+  a.sep_words = at<uint2>(ws, P.prefix);
   a.ranges = ranges;
   a.window = p->window;
   for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
@@ -846,7 +846,7 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   P.status = A.take(kStatusBytes);
   if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
   if (p->with_separators) {
-    P.prefix = A.take(B * (T + 1) * 4);
+    P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
     P.sep_pos = A.take(B * T * 4);
     P.sep_count = A.take(B * 4);
     P.ranges = A.take(B * P.nQT * 2 * 4);
@@ -911,7 +911,7 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   a.v_sh = p->v_stride[1];
   a.v_st = p->v_stride[2];
   a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
-  a.sep_prefix = is_sep ? at<int32_t>(ws, P.prefix) : nullptr;
+  a.sep_words = is_sep ? at<uint2>(ws, P.prefix) : nullptr;
   a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
   a.part = at<float>(ws, P.part);
   a.n_chunks = P.n_chunks;
@@ -952,7 +952,7 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
   F.status = A.take(kStatusBytes);
   if (p->rope_theta != 0.0) F.tab = A.take((size_t)F.npos * (d / 2) * sizeof(float2));
   if (p->with_separators) {
-    F.prefix = A.take(B * (T + 1) * 4);
+    F.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
     F.sep_pos = A.take(B * T * 4);
     F.sep_count = A.take(B * 4);
     F.ranges = A.take(B * F.nQT * 2 * 4);
@@ -1082,7 +1082,7 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   a.capped_sep = (is_sep && F.capped_sep) ? 1 : 0;
   a.sep_pos = is_sep ? sep_pos : nullptr;
   a.sep_count = is_sep ? sep_count : nullptr;
-  a.sep_prefix = is_sep ? at<int32_t>(ws, F.prefix) : nullptr;
+  a.sep_words = is_sep ? at<uint2>(ws, F.prefix) : nullptr;
   a.ranges = is_sep ? ranges : nullptr;
   a.Dsum = at<float>(ws, P.dsum);
   a.nlse2 = at<float>(ws, P.nlse2);

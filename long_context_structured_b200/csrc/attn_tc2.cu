@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a.gather_mode == 1) {
             // separators kept by row i: pos < i - w; their count is a prefix count
             const int thr = i - a.window;
-            const int cnt = thr > 0 ? __ldg(a.sep_prefix + (size_t)b * (a.T + 1) + min(thr, a.T)) : 0;
+            const int cnt = thr > 0 ? sep_before(a.sep_words, a.T, b, thr) : 0;
             lim = max(0, min(lim, cnt - r0));
           }
           c_hi = lim - 1;

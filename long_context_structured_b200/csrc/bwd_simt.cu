@@ -314,9 +314,9 @@ __global__ void bwd_combine_kernel(BwdArgs a) {
     v[e] = vb[e];
   }
   if (a.gather && j >= a.n_start) {
-    const int32_t* pre = a.sep_prefix + (size_t)b * (a.T + 1);
-    const int r = pre[j];
-    if (pre[j + 1] > r) {  // j is a separator: its compacted slot r
+    const uint2 wd = a.sep_words[(size_t)b * (a.T / 32 + 1) + (j >> 5)];
+    if ((wd.y >> (j & 31)) & 1u) {  // j is a separator: its compacted slot r
+      const int r = (int)wd.x + __popc(wd.y & ((1u << (j & 31)) - 1u));
       const float* ks = a.dk_sep + (bg * a.Tpad + r) * a.d + c0;
       const float* vs = a.dv_sep + (bg * a.Tpad + r) * a.d + c0;
 #pragma unroll

@@ -51,7 +51,7 @@ __device__ __forceinline__ KeySet key_set(const DecodeArgs& a, int b) {
   s.win_lo = max(s.n_sink, i - a.window);
   s.n_win = max(0, i - s.win_lo + 1);
   const int thr = i - a.window;  // separators kept: n_start <= j < i - w
-  s.n_sep = (a.sep_prefix && thr > 0) ? a.sep_prefix[(size_t)b * (a.T + 1) + min(thr, a.T)] : 0;
+  s.n_sep = (a.sep_words && thr > 0) ? sep_before(a.sep_words, a.T, b, thr) : 0;
   return s;
 }
 
@@ -349,7 +349,7 @@ cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
   // without separators or per-sequence lengths the kept-key count is a
   // closed form: launch exactly its chunks
   int chunks = a.n_chunks;
-  if (!a.sep_prefix && !a.seq_len) {
+  if (!a.sep_words && !a.seq_len) {
     const int i = a.T - 1, ns = std::min(a.n_start, a.T);
     const int win_lo = std::max(ns, i - a.window);
     chunks = std::min(chunks, std::max(1, (ns + std::max(0, i - win_lo + 1) + kChunk - 1) / kChunk));

@@ -42,13 +42,27 @@ cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
 struct BlockmapArgs {
   int B, T, n_start, window;
   const uint8_t* is_sep;  // may be null
-  int32_t* prefix;        // [B, T+1] workspace: separators (j >= n_start) before x
+  void* scratch;          // blockmap_scratch_bytes(B, T, window) of workspace
   int32_t* sep_pos;       // [B, T]
   int32_t* sep_count;     // [B]
   int32_t* ranges;        // [B, nQT, 2]
   uint8_t* cls;           // [B, nQT, nKT] or null
 };
 cudaError_t launch_blockmap(const BlockmapArgs& a, cudaStream_t st);
+// scratch of launch_blockmap: word prefix of the separator flags, far and
+// near tile classes (0 for invalid sizes)
+size_t blockmap_scratch_bytes(int B, int T, int window);
+
+// The separator word prefix, the first part of the block map's scratch: per
+// sequence T/32 + 1 entries; entry x holds in .x the number of separators
+// (j >= n_start) before position 32 x and in .y a bit for each of the 32
+// positions from 32 x that is one.
+// Separators (j >= n_start) before position x, x clamped to [0, T].
+__device__ __forceinline__ int sep_before(const uint2* words, int T, int b, int x) {
+  x = max(0, min(T, x));
+  const uint2 e = __ldg(words + (size_t)b * (T / 32 + 1) + (x >> 5));
+  return (int)e.x + __popc(e.y & ((1u << (x & 31)) - 1u));
+}
 
 // ---------------------------------------------------------------------------
 // K3: separator K/V gather into dense per-(b, kv-head) arrays
@@ -89,7 +103,7 @@ struct AttnArgs {
   int cross_len;
   bool q2;                     // gathered tiles use the second query tile (Qc)
   const int32_t* sep_pos;      // [B, T]
-  const int32_t* sep_prefix;   // [B, T+1]: separators n_start <= j < x
+  const uint2* sep_words;      // separator word prefix (sep_before)
   const int32_t* ranges;       // [B, nQT, 2]
   int window;                  // w for the separator rule (sep kept iff pos < i - w)
   // segmented execution
@@ -241,7 +255,7 @@ struct BwdArgs {
   int capped_sep;               // gathered tiles take Qc and raw keys
   const int32_t* sep_pos;       // [B, T]
   const int32_t* sep_count;     // [B]
-  const int32_t* sep_prefix;    // [B, T+1]
+  const uint2* sep_words;       // separator word prefix (sep_before)
   const int32_t* ranges;        // [B, nQT, 2]
   // row statistics, padded to Tpad rows (pad: D = 0, -lse2 = -inf)
   float* Dsum;                  // [B, Hq, Tpad] dO_i . O_i
@@ -348,7 +362,7 @@ struct DecodeArgs {
   const __nv_bfloat16* V;
   int64_t v_sb, v_sh, v_st;
   const float2* tab;            // rotary table or null
-  const int32_t* sep_prefix;    // [B, T+1] or null (no separators)
+  const uint2* sep_words;       // separator word prefix (sep_before) or null (no separators)
   const int32_t* sep_pos;       // [B, T]
   const int32_t* seq_len;       // [B] cache length per sequence (<= T), or null: T for all
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials

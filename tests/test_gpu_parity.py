@@ -56,8 +56,15 @@ def _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=None):
 # block map (integer, bit-exact)
 # ---------------------------------------------------------------------------
 
+# Shapes reach both class paths (16-byte pieces when the tile count is a
+# multiple of 16, bytes otherwise), band tables as wide as the whole row
+# (window >= T), sinks over several tiles, a last flag word that is cut short
+# and rows whose flags are not 16-byte aligned (T % 16 != 0).
 @pytest.mark.parametrize("B,T,ns,w,rate", [(1, 1024, 4, 128, 0.08), (3, 1000, 4, 37, 0.2), (2, 300, 0, 0, 0.5),
-                                           (1, 129, 7, 300, 1.0), (4, 8192, 4, 256, 0.10), (2, 777, 2, 5, 0.0)])
+                                           (1, 129, 7, 300, 1.0), (4, 8192, 4, 256, 0.10), (2, 777, 2, 5, 0.0),
+                                           (2, 4096, 250, 700, 0.3), (1, 6149, 3, 5000, 0.05),
+                                           (2, 16384, 0, 20000, 0.1), (2, 4096, 4, 0, 1.0), (2, 4112, 4, 128, 0.2),
+                                           (1, 2048, 200, 100, 0.0)])
 def test_blockmap_bitexact(oracle_mod, B, T, ns, w, rate):
     rng = np.random.default_rng(B * 1000 + T)
     flags = (rng.random((B, T)) < rate).astype(np.uint8)
@@ -68,6 +75,24 @@ def test_blockmap_bitexact(oracle_mod, B, T, ns, w, rate):
     assert np.array_equal(out["sep_pos"].cpu().numpy(), pos)
     assert np.array_equal(out["qtile_sep_range"].cpu().numpy(), rng_)
     assert np.array_equal(out["cls"].cpu().numpy(), cls)
+
+
+def test_blockmap_stress_launch_sampled(oracle_mod):
+    """The block map at 2048 sequences x 32768 flags (2^26, the stress size
+    the benchmark times), checked on sampled sequences: each sequence is
+    computed independently, so the oracle runs on those alone."""
+    B, T, ns, w = 2048, 32768, 4, 256
+    g = torch.Generator().manual_seed(0)
+    flags = (torch.rand(B, T, generator=g) < 0.1).to(torch.uint8)
+    out = sa.build_blockmap(flags.cuda(), B=B, T=T, n_start=ns, window=w)
+    torch.cuda.synchronize()
+    for b in (0, 1337, B - 1):
+        f = flags[b:b + 1].numpy()
+        cls, pos, cnt, rng_ = oracle_mod.blockmap(1, T, ns, w, 128, 128, f)
+        assert int(out["sep_count"][b]) == int(cnt[0])
+        assert np.array_equal(out["sep_pos"][b].cpu().numpy(), pos[0])
+        assert np.array_equal(out["qtile_sep_range"][b].cpu().numpy(), rng_[0])
+        assert np.array_equal(out["cls"][b].cpu().numpy(), cls[0])
 
 
 def test_blockmap_c3_token_flags(oracle_mod):

@@ -19,7 +19,16 @@ from long_context_structured_b200 import _lib
 
 pytestmark = pytest.mark.gpu
 
-MAX_INTS = 1 << 20
+MAX_BYTES = 1 << 22
+
+
+def _scratch_bytes(B, T, window):
+    """The scratch size the header states for the no-alloc block map."""
+    up16 = lambda x: (x + 15) // 16 * 16
+    nqt = (T + 127) // 128
+    bt = min(nqt, (window + 127) // 128)
+    kc = min((nqt + 15) // 16, bt // 16 + 2)
+    return up16(B * 8 * (T // 32 + 1)) + B * up16(nqt) + B * 16 * nqt * kc
 
 
 def _params(B, T, n_start, window):
@@ -79,9 +88,12 @@ def test_noalloc_rejects_oversize_before_launch():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     lib = _lib.load()
-    T = 40000
-    B = MAX_INTS // (T + 1) + 1
-    p = _params(B, T, 4, 128)
+    T, w = 40000, 128
+    B = 1
+    while _scratch_bytes(B, T, w) <= MAX_BYTES:
+        B += 1
+    assert _scratch_bytes(B - 1, T, w) <= MAX_BYTES < _scratch_bytes(B, T, w)
+    p = _params(B, T, 4, w)
     fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check fails first
     assert lib.sattn_build_blockmap_noalloc(ctypes.byref(p), None, None, fake, fake, fake, None) == \
         _lib.SATTN_ERR_UNSUPPORTED
