@@ -755,7 +755,10 @@ def run_ours(args):
 
     # end to end through the public call with host buffers (H2D + D2H inside)
     n_e2e = max(3, min(10, args.steps))
-    outs = job.host_step()  # warm the host path
+    # warm the host path: pinned output buffers come from the caching host
+    # allocator once two calls' results have been alive at the same time
+    for _ in range(3):
+        outs = job.host_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -869,7 +872,8 @@ def run_tree(args, world, rank, dev):
         roof["kernel"] = kernel_name(None, dom)
         roof["traffic"] = None
     n_e2e = max(3, min(10, args.steps))
-    outs = job.host_step()
+    for _ in range(3):  # warm the host path (pinned buffers cached)
+        outs = job.host_step()
     torch.cuda.synchronize()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s0.record()

@@ -419,25 +419,25 @@ def selftest_wait_timeout(limit_ms: float = 20.0, device="cuda") -> tuple:
     return status, site
 
 
-def _host_chunks(B: int, Hq: int, Hkv: int, n: int):
-    """Independent pieces of a problem: ("b", b0, b1) batch ranges when B > 1,
-    else ("h", kv0, kv1) ranges of kv heads (whole GQA groups)."""
-    if B > 1:
-        n = min(n, B)
-        return [("b", B * c // n, B * (c + 1) // n) for c in range(n)]
-    n = min(n, Hkv)
-    return [("h", Hkv * c // n, Hkv * (c + 1) // n) for c in range(n)]
+def _host_chunks(B: int, Hkv: int, n: int):
+    """About n independent pieces of a problem, as (b0, b1, kv0, kv1): batch
+    ranges, each cut into groups of kv heads (whole GQA groups) when there
+    are fewer sequences than pieces."""
+    nb = min(n, B)
+    nh = min(max(1, n // nb), Hkv)
+    return [(B * i // nb, B * (i + 1) // nb, Hkv * j // nh, Hkv * (j + 1) // nh)
+            for i in range(nb) for j in range(nh)]
 
 
-def _host_call(fn, tensors, kw, n_chunks: int = 4):
+def _host_call(fn, tensors, kw, n_chunks: int = 8):
     """Host tensors in, host tensors out: the end-to-end path.
 
-    Batches (or, for one sequence, groups of kv heads) are independent, so the
-    problem is cut into a few pieces: one copy stream moves piece c+1 to the
-    device while the compute stream runs piece c, and a second copy stream
-    brings each piece's results back as soon as they are ready (the two
-    directions overlap).  Outputs land in pinned host memory; the result
-    equals the one-piece call bit for bit."""
+    Sequences and groups of kv heads are independent, so the problem is cut
+    into about n_chunks pieces: one copy stream moves piece c+1 to the device
+    while the compute stream runs piece c, and a second copy stream brings
+    each piece's results back as soon as they are ready (the two directions
+    overlap).  Outputs land in pinned host memory; the result equals the
+    one-piece call bit for bit."""
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = tensors
     B, Hq, T, d = q.shape
@@ -452,19 +452,16 @@ def _host_call(fn, tensors, kw, n_chunks: int = 4):
     dside = {name: torch.empty(t.shape, dtype=t.dtype, device=dev) for name, t in side.items()}
     outs_host = None
     res_keep = []
-    for kind, x0, x1 in _host_chunks(B, Hq, Hkv, n_chunks):
-        if kind == "b":
-            sl_q = sl_kv = sl_side = (slice(x0, x1),)
-        else:
-            sl_q = (slice(None), slice(x0 * rep, x1 * rep))
-            sl_kv = (slice(None), slice(x0, x1))
-            sl_side = (slice(None),)
+    for b0, b1, x0, x1 in _host_chunks(B, Hkv, n_chunks):
+        sl_q = (slice(b0, b1), slice(x0 * rep, x1 * rep))
+        sl_kv = (slice(b0, b1), slice(x0, x1))
+        sl_side = (slice(b0, b1),)
         with torch.cuda.stream(copy):
             for src, dst, sl in ((q, dq, sl_q), (k, dk, sl_kv), (v, dv, sl_kv)):
                 dst[sl].copy_(src[sl], non_blocking=True)
             for name, t in side.items():
                 if name == "is_sep":
-                    if kind == "b" or x0 == 0:  # flags are per sequence, shared by head pieces
+                    if x0 == 0:  # flags are per sequence, shared by the head pieces
                         dside[name][sl_side].copy_(t[sl_side], non_blocking=True)
                 else:
                     dside[name][sl_q].copy_(t[sl_q], non_blocking=True)
@@ -474,13 +471,13 @@ def _host_call(fn, tensors, kw, n_chunks: int = 4):
         ckw = dict(kw)
         for name, t in dside.items():
             ckw[name] = t[sl_side] if name == "is_sep" else t[sl_q]
-        if "is_long" in ckw and kind == "h":
+        if "is_long" in ckw:
             ckw["is_long"] = list(ckw["is_long"])[x0 * rep:x1 * rep]
         res = fn(dq[sl_q], dk[sl_kv], dv[sl_kv], **ckw)
         done = torch.cuda.Event()
         done.record(compute)
         if outs_host is None:
-            shapes = [((B,) + tuple(r.shape[1:])) if kind == "b" else ((B, Hq) + tuple(r.shape[2:])) for r in res]
+            shapes = [(B, Hq) + tuple(r.shape[2:]) for r in res]
             outs_host = tuple(torch.empty(sh, dtype=r.dtype, pin_memory=True) for sh, r in zip(shapes, res))
         back.wait_event(done)
         with torch.cuda.stream(back):
