@@ -355,6 +355,8 @@ __global__ void __launch_bounds__(kClassThreads) tile_class_kernel(BlockmapArgs 
   }
 }
 
+}  // namespace
+
 int sm_count() {
   static int cached[64] = {};
   int dev = 0;
@@ -365,8 +367,6 @@ int sm_count() {
   }
   return cached[dev];
 }
-
-}  // namespace
 
 size_t blockmap_scratch_bytes(int B, int T, int window) {
   if (B < 1 || T < 1 || window < 0) return 0;

@@ -49,6 +49,9 @@ struct BlockmapArgs {
   uint8_t* cls;           // [B, nQT, nKT] or null
 };
 cudaError_t launch_blockmap(const BlockmapArgs& a, cudaStream_t st);
+// streaming multiprocessors of the current device (cached per device)
+int sm_count();
+
 // scratch of launch_blockmap: word prefix of the separator flags, far and
 // near tile classes (0 for invalid sizes)
 size_t blockmap_scratch_bytes(int B, int T, int window);

@@ -57,6 +57,8 @@ CASES = [
                                    sep_rate=0.1, alibi=True)),
     ("alibi_unclipped_sep_d64", dict(B=1, Hq=4, Hkv=4, T=500, d=64, n_start=2, window=40, sep_rate=0.2,
                                      alibi=True)),
+    ("sep_capped_gqa2_d64", dict(B=2, Hq=4, Hkv=2, T=1500, d=64, n_start=4, window=80, L_pretrain=80,
+                                 rope_theta=1e4, sep_rate=0.15)),
 ]
 
 
