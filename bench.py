@@ -365,6 +365,32 @@ class DecodeJob:
         self.n_step += 1
         self.sa.decode_fwd(self.qd, k, v, is_sep=self.sep, out=self.O, lse=self.lse, **self.kw)
 
+    def capture(self):
+        """One CUDA graph per cache copy holding a whole step (rotary table,
+        block map, decode and merge kernels), as a generation loop replays
+        it: a step of tens of microseconds is otherwise timed at the speed
+        of the host's Python call path."""
+        torch = self.torch
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):
+            for _ in range(self.n_copies):
+                self.step()
+        torch.cuda.current_stream(self.dev).wait_stream(side)
+        torch.cuda.synchronize(self.dev)
+        self.graphs = []
+        for c in range(self.n_copies):
+            g = torch.cuda.CUDAGraph()
+            self.n_step = c
+            with torch.cuda.graph(g):
+                self.step()
+            self.graphs.append(g)
+        self.n_step = 0
+
+    def graph_step(self):
+        self.graphs[self.n_step % self.n_copies].replay()
+        self.n_step += 1
+
     def host_step(self):
         """The query from pinned host memory, the step on the device-resident
         cache, O and LSE back to pinned host memory."""
@@ -698,24 +724,12 @@ def run_ours(args):
     clocks = ClockSampler(gpu_uuid, phys)
     clocks.start()
     time.sleep(0.3)
-    profile_collect(lib)  # drop anything recorded before
-    lib.sattn_profile_enable(1)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        job.step()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    lib.sattn_profile_enable(0)
+    plain = None
+    if decode:
+        job.capture()
+        plain = job.graph_step
+    elapsed_ms, prof = timed_passes(job.step, args.steps, lib, world, plain_step=plain)
     clk = clocks.stop()
-    elapsed_ms = e0.elapsed_time(e1)
-    prof = profile_collect(lib)
     status = sa.stream_status()
 
     t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
@@ -802,7 +816,9 @@ def run_ours(args):
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_bf16_peak": round(value / world / peak, 4),
         "roofline": roof,
-        "kernels": kernels,
+        "kernels": kernels, "kernel_times": KERNEL_TIMES_NOTE,
+        "step_timing": ("CUDA-graph replays of the whole step (one graph per cache copy), as a generation loop "
+                        "runs it" if decode else "eager calls of the public API"),
         "gpu_launches": gpu_launches,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -834,23 +850,9 @@ def run_tree(args, world, rank, dev):
     clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
     clocks.start()
     time.sleep(0.3)
-    profile_collect(lib)
-    lib.sattn_profile_enable(1)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        job.step()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    lib.sattn_profile_enable(0)
+    el_ms, prof = timed_passes(job.step, args.steps, lib, world)
     clk = clocks.stop()
-    prof = profile_collect(lib)
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    t = torch.tensor([el_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
@@ -903,7 +905,8 @@ def run_tree(args, world, rank, dev):
                          % (job.h2d_bytes() >> 20)},
         "tokens_per_s": round(c["B"] * c["Tq"] * world / (ms_step * 1e-3), 1),
         "frac_of_bf16_peak": round(value / world / float(peaks["bf16_tflops"]), 4),
-        "roofline": roof, "kernels": kernels, "gpu_launches": sum(n for n, _ in prof.values()),
+        "roofline": roof, "kernels": kernels, "kernel_times": KERNEL_TIMES_NOTE,
+        "gpu_launches": sum(n for n, _ in prof.values()),
         "e2e": {"value": round(job.flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(ms_e2e, 3), "steps": n_e2e, "h2d_bytes_per_step": job.h2d_bytes(),
                 "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
@@ -931,24 +934,11 @@ def run_stream(args, world, rank, dev):
     clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
     clocks.start()
     time.sleep(0.3)
-    profile_collect(lib)
-    lib.sattn_profile_enable(1)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        job.step()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    lib.sattn_profile_enable(0)
+    el_ms, _ = timed_pass(job.step, args.steps, lib, world, False)
+    len1 = job.mean_len()  # the work of the step-time pass
+    _, prof = timed_pass(job.step, args.steps, lib, world, True)
     clk = clocks.stop()
-    prof = profile_collect(lib)
-    len1 = job.mean_len()
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    t = torch.tensor([el_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
@@ -991,10 +981,48 @@ def run_stream(args, world, rank, dev):
                    "l2": "no flush: the caches hold %d MB of K/V, > 126 MB L2"
                          % (c["B"] * c["Hkv"] * c["c"] * c["d"] * 4 >> 20)},
         "tokens_per_s": round(c["B"] * world / (ms_step * 1e-3), 1),
-        "roofline": roof, "kernels": kernels, "gpu_launches": sum(n for n, _ in prof.values()),
+        "roofline": roof, "kernels": kernels, "kernel_times": KERNEL_TIMES_NOTE,
+        "gpu_launches": sum(n for n, _ in prof.values()),
         "e2e": None, "cpu_baseline": None, "clocks": clk, "device_status": sa.stream_status(),
     }
     print(json.dumps(line), flush=True)
+
+
+def timed_pass(step, steps, lib, world, profiled):
+    """`steps` calls of `step` bracketed by a barrier and a synchronize on
+    both sides, with or without the library's per-launch-group CUDA events.
+    Returns (elapsed ms, {group: (launches, ms)})."""
+    import torch
+    import torch.distributed as dist
+
+    profile_collect(lib)  # drop anything recorded before
+    lib.sattn_profile_enable(1 if profiled else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    lib.sattn_profile_enable(0)
+    return e0.elapsed_time(e1), profile_collect(lib)
+
+
+def timed_passes(step, steps, lib, world, plain_step=None):
+    """The step time from a pass without per-launch events (of plain_step
+    when given, e.g. a CUDA-graph replay of the same step), the per-kernel
+    times from a second pass of `step` with them."""
+    ms, _ = timed_pass(plain_step or step, steps, lib, world, False)
+    _, prof = timed_pass(step, steps, lib, world, True)
+    return ms, prof
+
+
+KERNEL_TIMES_NOTE = ("per-kernel times from a second timed pass of the same steps with CUDA events around each "
+                     "launch group; the step time from the first pass, without them")
 
 
 def run_blockmap_stress(args, world, rank, dev):
@@ -1016,18 +1044,10 @@ def run_blockmap_stress(args, world, rank, dev):
     clocks = ClockSampler(gpu_uuid, int(os.environ.get("LOCAL_RANK", "0")))
     clocks.start()
     time.sleep(0.3)
-    profile_collect(lib)
-    lib.sattn_profile_enable(1)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        sa.build_blockmap(flags, B=B, T=T, n_start=ns, window=w, device=dev)
-    e1.record()
-    torch.cuda.synchronize()
-    lib.sattn_profile_enable(0)
+    el_ms, prof = timed_passes(lambda: sa.build_blockmap(flags, B=B, T=T, n_start=ns, window=w, device=dev),
+                               args.steps, lib, world)
     clk = clocks.stop()
-    prof = profile_collect(lib)
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = el_ms / args.steps
     nqt = T // 128
     nbytes = B * T + B * nqt * nqt + B * T * 4 + B * 4 + B * nqt * 8
     kms = prof["blockmap"][1] / args.steps
@@ -1046,6 +1066,7 @@ def run_blockmap_stress(args, world, rank, dev):
                        "algorithmic_bytes": nbytes,
                        "l2": "no flush: %d MB read and written per step, > 126 MB L2" % (nbytes >> 20)},
             "roofline": roof, "kernels": {"blockmap": {"launches": prof["blockmap"][0], "ms_per_step": round(kms, 5)}},
+            "kernel_times": KERNEL_TIMES_NOTE,
             "gpu_launches": prof["blockmap"][0], "clocks": clk, "e2e": None, "cpu_baseline": None}), flush=True)
 
 

@@ -879,7 +879,18 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
   if (P.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
-    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+    if (is_sep) {
+      // separators can sit at any earlier position
+      SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
+    } else {
+      // the step reads the rows of the sinks (j, or i - L when capped), of
+      // the window keys and of the query (i - w <= j <= i, uncapped since
+      // w <= L), and row i - L: [0, n_start) and [i - max(w, L), T)
+      const int i = p->T - 1;
+      const int row_lo = std::max(0, i - std::max(p->window, p->L_pretrain));
+      SATTN_TRY(launch_rope_table_rows(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p),
+                                       std::min(p->n_start, p->T), row_lo, st));
+    }
   }
   if (is_sep) {
     FwdPlan F;

@@ -17,6 +17,9 @@ constexpr int kMaxHeads = 256;
 // tab[p][c] = (cos, sin)(p * scale * theta^(-2c/d)), computed in fp64, stored
 // fp32; scale < 1 is position interpolation.
 cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, double scale, cudaStream_t st);
+// rows [0, n_low) and [row_lo, npos) only (the others are not written)
+cudaError_t launch_rope_table_rows(float2* tab, int npos, int d, double theta, double scale, int n_low, int row_lo,
+                                   cudaStream_t st);
 
 struct PrepArgs {
   int B, Hq, Hkv, T, d;

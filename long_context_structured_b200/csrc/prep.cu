@@ -21,6 +21,8 @@
 // positions of one head; the sink keys of that head's kv head are staged once
 // per block in shared memory (rotated to their own position, and in the
 // capped form R(-L) k used with the unrotated query).
+#include <cmath>
+
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -37,23 +39,31 @@ constexpr int kU = 2;  // rows per thread whose loads are in flight together
 constexpr int kMaxSmemSinks = 16;
 constexpr int kPairsPerThread = 8;
 
-__global__ void rope_table_kernel(float2* tab, int npos, int half, int d, double theta, double scale) {
-  __shared__ double inv_freq[128];
-  for (int c = threadIdx.x; c < half; c += blockDim.x) inv_freq[c] = pow(theta, -2.0 * (double)c / (double)d);
-  __syncthreads();
-  const int64_t n = (int64_t)npos * half;
-  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
-    const int p = (int)(x / half);
-    const int c = (int)(x % half);
+// theta^(-2c/d) for the d/2 rotary pairs, computed once on the host in
+// double and passed by value
+struct InvFreq {
+  double v[64];
+};
+
+// rows [0, n_low) and [row_lo, npos) of the table (the rows between are
+// left as they are); I is the index type (32 bits whenever the entries fit)
+template <typename I>
+__global__ void rope_table_kernel(float2* tab, int npos, int half, const InvFreq inv_freq, double scale, int n_low,
+                                  int row_lo) {
+  const I n = (I)(n_low + (npos - row_lo)) * (I)half;
+  for (I x = (I)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (I)gridDim.x * blockDim.x) {
+    const int q = (int)(x / (I)half);
+    const int c = (int)(x - (I)q * (I)half);
+    const int p = q < n_low ? q : row_lo + (q - n_low);
     // the angle in double, reduced by whole turns in double (exact to
     // ~1e-12 for the positions used), then the fp32 sine and cosine of the
     // reduced angle: within a few fp32 ulps of the double-precision values
-    const double ang = (double)p * scale * inv_freq[c];
+    const double ang = (double)p * scale * inv_freq.v[c];
     const double turns = rint(ang * (1.0 / 6.283185307179586));
     const float r = (float)fma(-turns, 6.283185307179586, ang);
     float s, co;
     sincosf(r, &s, &co);
-    tab[x] = make_float2(co, s);
+    tab[(size_t)p * half + c] = make_float2(co, s);
   }
 }
 
@@ -321,15 +331,27 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
 
 }  // namespace
 
-cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, double scale, cudaStream_t st) {
+cudaError_t launch_rope_table_rows(float2* tab, int npos, int d, double theta, double scale, int n_low, int row_lo,
+                                   cudaStream_t st) {
   const int half = d / 2;
-  const int64_t n = (int64_t)npos * half;
+  row_lo = std::max(0, std::min(row_lo, npos));
+  n_low = std::max(0, std::min(n_low, row_lo));
+  const int64_t n = ((int64_t)n_low + (npos - row_lo)) * half;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
-  // few blocks, each over many entries: the per-block inverse-frequency setup is amortised
   const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 4);
-  rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(tab, npos, half, d, theta, scale);
+  if (half > 64) return cudaErrorInvalidValue;
+  InvFreq inv{};
+  for (int c = 0; c < half; ++c) inv.v[c] = std::pow(theta, -2.0 * (double)c / (double)d);
+  if (n + blocks * threads < ((int64_t)1 << 32))
+    rope_table_kernel<uint32_t><<<(unsigned)blocks, threads, 0, st>>>(tab, npos, half, inv, scale, n_low, row_lo);
+  else
+    rope_table_kernel<uint64_t><<<(unsigned)blocks, threads, 0, st>>>(tab, npos, half, inv, scale, n_low, row_lo);
   return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(float2* tab, int npos, int d, double theta, double scale, cudaStream_t st) {
+  return launch_rope_table_rows(tab, npos, d, theta, scale, 0, 0, st);
 }
 
 template <int D>
