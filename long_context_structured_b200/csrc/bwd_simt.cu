@@ -195,6 +195,20 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
 // raw-frame dk part (R(j)^T of the uncapped sum plus the capped sum,
 // unscaled) and the dv part of each sink.
 constexpr int kSinkGroup = 4;
+constexpr int kRowsInFlight = 4;  // rows per warp whose loads are issued together
+
+// PL consecutive bf16 (one or two) as floats
+template <int PL>
+__device__ __forceinline__ void load_pl(const __nv_bfloat16* p, float* out) {
+  if constexpr (PL == 2) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    out[0] = f.x;
+    out[1] = f.y;
+  } else {
+    out[0] = __bfloat162float(*p);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_sink_keys_kernel(BwdArgs a) {
   constexpr int PL = D / 64;  // pairs per lane
@@ -220,41 +234,64 @@ __global__ void __launch_bounds__(256) bwd_sink_keys_kernel(BwdArgs a) {
   float2 cl[PL];
 #pragma unroll
   for (int e = 0; e < PL; ++e) cl[e] = a.L > 0 ? tab_at(a.tab, a.L, H, PL * lane + e) : make_float2(1.f, 0.f);
+  // a warp takes rows i0, i0 + 8, ..., i0 + 8 (kRowsInFlight - 1) together:
+  // their loads are issued before any is used
   for (int h = g * rep; h < (g + 1) * rep; ++h) {
     const int64_t bh = (int64_t)b * a.Hq + h;
-    for (int i = i_lo + warp; i < i_hi; i += 8) {
-      const int64_t wid = bh * a.T + i;
-      const __nv_bfloat16* qp = a.Q + b * a.q_sb + h * a.q_sh + (int64_t)i * a.q_st + PL * lane;
-      const __nv_bfloat16* gp = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)i * a.o_st + PL * lane;
-      float q0[PL], q1[PL], d0[PL], d1[PL], qi0[PL], qi1[PL], ql0[PL], ql1[PL];
+    for (int i0 = i_lo + warp; i0 < i_hi; i0 += 8 * kRowsInFlight) {
+      float q0[kRowsInFlight][PL], q1[kRowsInFlight][PL], d0[kRowsInFlight][PL], d1[kRowsInFlight][PL];
+      float2 ti[kRowsInFlight][PL];
+      float dsv[kRowsInFlight][kSinkGroup], pjv[kRowsInFlight][kSinkGroup];
 #pragma unroll
-      for (int e = 0; e < PL; ++e) {
-        q0[e] = bf(qp, e);
-        q1[e] = bf(qp, e + H);
-        d0[e] = bf(gp, e);
-        d1[e] = bf(gp, e + H);
-        rot(q0[e], q1[e], tab_at(a.tab, i, H, PL * lane + e), qi0[e], qi1[e]);
-        rot(q0[e], q1[e], cl[e], ql0[e], ql1[e]);
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const int i = i0 + 8 * u;
+        const int ic = i < i_hi ? i : i0;  // rows past the block: loads of row i0, results unused
+        const int64_t wid = bh * a.T + ic;
+        const __nv_bfloat16* qp = a.Q + b * a.q_sb + h * a.q_sh + (int64_t)ic * a.q_st + PL * lane;
+        const __nv_bfloat16* gp = a.dO + b * a.o_sb + h * a.o_sh + (int64_t)ic * a.o_st + PL * lane;
+        load_pl<PL>(qp, q0[u]);
+        load_pl<PL>(qp + H, q1[u]);
+        load_pl<PL>(gp, d0[u]);
+        load_pl<PL>(gp + H, d1[u]);
+#pragma unroll
+        for (int e = 0; e < PL; ++e) ti[u][e] = tab_at(a.tab, ic, H, PL * lane + e);
+#pragma unroll
+        for (int q = 0; q < kSinkGroup; ++q) {
+          const bool use = q < nj;
+          dsv[u][q] = use ? a.sink_ds[wid * a.n_sink + j0 + q] : 0.f;
+          pjv[u][q] = use ? a.sink_p[wid * a.n_sink + j0 + q] : 0.f;
+        }
       }
 #pragma unroll
-      for (int q = 0; q < kSinkGroup; ++q) {
-        if (q >= nj) break;
-        const int j = j0 + q;
-        if (i < j) continue;
-        const float ds = a.sink_ds[wid * a.n_sink + j];
-        const float pj = a.sink_p[wid * a.n_sink + j];
-        const bool capped = a.L > 0 && (i - j) > a.L;
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const int i = i0 + 8 * u;
+        if (i >= i_hi) break;
+        float qi0[PL], qi1[PL], ql0[PL], ql1[PL];
 #pragma unroll
         for (int e = 0; e < PL; ++e) {
-          if (capped) {
-            ac[q][e] = fmaf(ds, ql0[e], ac[q][e]);
-            ac[q][PL + e] = fmaf(ds, ql1[e], ac[q][PL + e]);
-          } else {
-            ar[q][e] = fmaf(ds, qi0[e], ar[q][e]);
-            ar[q][PL + e] = fmaf(ds, qi1[e], ar[q][PL + e]);
+          rot(q0[u][e], q1[u][e], ti[u][e], qi0[e], qi1[e]);
+          rot(q0[u][e], q1[u][e], cl[e], ql0[e], ql1[e]);
+        }
+#pragma unroll
+        for (int q = 0; q < kSinkGroup; ++q) {
+          if (q >= nj) break;
+          const int j = j0 + q;
+          if (i < j) continue;
+          const float ds = dsv[u][q];
+          const float pj = pjv[u][q];
+          const bool capped = a.L > 0 && (i - j) > a.L;
+#pragma unroll
+          for (int e = 0; e < PL; ++e) {
+            if (capped) {
+              ac[q][e] = fmaf(ds, ql0[e], ac[q][e]);
+              ac[q][PL + e] = fmaf(ds, ql1[e], ac[q][PL + e]);
+            } else {
+              ar[q][e] = fmaf(ds, qi0[e], ar[q][e]);
+              ar[q][PL + e] = fmaf(ds, qi1[e], ar[q][PL + e]);
+            }
+            av[q][e] = fmaf(pj, d0[u][e], av[q][e]);
+            av[q][PL + e] = fmaf(pj, d1[u][e], av[q][PL + e]);
           }
-          av[q][e] = fmaf(pj, d0[e], av[q][e]);
-          av[q][PL + e] = fmaf(pj, d1[e], av[q][PL + e]);
         }
       }
     }
