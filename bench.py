@@ -1238,7 +1238,7 @@ def main():
                     choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
                     + sorted(BWD_ALIASES) + sorted(TREE_ALIASES) + sorted(STREAM_ALIASES) + sorted(STRESS_ALIASES)
                     + sorted(EXTRA_WORKLOADS))
-    ap.add_argument("--cpu-rows", type=int, default=8192, help="rows in the CPU-oracle baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=32768, help="rows in the CPU-oracle baseline sample (~10 s)")
     ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling captures only)")
