@@ -989,7 +989,7 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
       P.nRB = (int)((T + bwd_sink_row_block() - 1) / bwd_sink_row_block());
       P.sink_part = A.take(B * Hkv * F.n_sink * (size_t)P.nRB * 2 * d * 4);
     }
-    if (F.n_sink > 0 || F.capped_sep) P.dq_side = A.take(B * Hq * T * d * 4);
+    if (F.capped_sep) P.dq_side = A.take(B * Hq * T * d * 4);  // the capped separators' dq (first dq pass)
     P.dk_band = A.take(B * Hkv * T * d * 4);
     P.dv_band = A.take(B * Hkv * T * d * 4);
   }
@@ -1114,7 +1114,10 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
     ProfScope ps("bwd_rows", 1, st);
     SATTN_TRY(launch_bwd_rows(a, st));
   }
-  a.side_valid = F.n_sink > 0;
+  // capped separators: a first dq pass writes their part to dq_side, the
+  // second adds it; the sink pairs' dq is formed in the second pass's epilogue
+  a.side_valid = false;
+  a.fold_sinks = 0;
   if (a.capped_sep) {
     a.dq_mode = 1;
     ProfScope ps("bwd_dq", 1, st);
@@ -1122,6 +1125,7 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
     a.side_valid = true;
   }
   a.dq_mode = 0;
+  a.fold_sinks = F.n_sink > 0 ? 1 : 0;
   {
     ProfScope ps("bwd_dq", 1, st);
     SATTN_TRY(launch_bwd_dq(a, m, st));

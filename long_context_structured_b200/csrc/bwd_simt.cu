@@ -6,9 +6,8 @@
 //                          (padded to whole 128-row tiles) and, since the
 //                          starting-span keys j < n_start ("LM-Infinite",
 //                          section 方法) are fp32 side keys in the forward and
-//                          here too, P and dS of the row's sink pairs and their
-//                          dq (capped pairs through R(L)^T, others through
-//                          R(i)^T of R(j) k_j);
+//                          here too, P and dS of the row's sink pairs (their
+//                          dq is added by the dq kernel's epilogue);
 //   bwd_sink_keys_kernel   dk and dv of the sink keys: fixed-order sums over
 //                          row blocks (no atomics);
 //   bwd_combine_kernel     dk_j, dv_j = band-tile part + separator part (its
@@ -45,11 +44,10 @@ __device__ __forceinline__ void rot_t(float y0, float y1, float2 cs, float& x0, 
 __device__ __forceinline__ float bf(const __nv_bfloat16* p, int64_t idx) { return __bfloat162float(p[idx]); }
 
 // Per-row pass: D_i = dO_i . O_i, -LSE_i log2(e) (padded rows: 0, -inf) and,
-// for the sink keys, P_ij, dS_ij and their dq (fp32, raw frame, scaled).
-// 8 lanes per row, lane l owning the rotary pairs [8l/2 .. ) -- E = D/16
-// pairs per lane: elements c0 + e and c0 + e + D/2 for c0 = l * E, e < E.
-// A block is 32 rows of one (b, h); the group's sink K (rotated and raw)
-// and V rows are staged in shared memory as fp32.
+// for the sink keys, P_ij and dS_ij.  8 lanes per row, lane l owning the
+// elements c0 + e and c0 + e + D/2 for c0 = l * E, e < E = D/16.  A block is
+// 32 rows of one (b, h); the group's sink V rows are staged in shared memory
+// as fp32.
 constexpr int kSinkStage = 16;  // sink rows staged in shared memory at a time
 
 // 8 consecutive bf16 (16 bytes, E = 8) or 4 (8 bytes, E = 4) as floats
@@ -80,7 +78,7 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
   constexpr int E = D / 16;  // pairs per lane
   constexpr int H = D / 2;
-  __shared__ float s_sink[kSinkStage][3][D];  // R(j) k_j, k_j, v_j of a stage of sinks
+  __shared__ float s_sink[kSinkStage][D];  // v_j of a stage of sinks
   const int blocks_per_head = a.Tpad / 32;
   const int64_t bh = blockIdx.x / blocks_per_head;
   const int i = (int)(blockIdx.x % blocks_per_head) * 32 + (threadIdx.x >> 3);
@@ -116,26 +114,13 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
   }
   if (ns_all == 0) return;  // uniform over the block
   const int ns = row_ok ? min(ns_all, i + 1) : 0;
-  float ar0[E], ar1[E], ac0[E], ac1[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) ar0[e] = ar1[e] = ac0[e] = ac1[e] = 0.f;
   const int64_t wid = bh * a.T + i;
   for (int js = 0; js < ns_all; js += kSinkStage) {
     const int nst = min(kSinkStage, ns_all - js);
     __syncthreads();  // the previous stage is consumed
-    for (int x = threadIdx.x; x < nst * H; x += blockDim.x) {
-      const int jj = x / H, p = x % H, j = js + jj;
-      const __nv_bfloat16* kp = a.K + b * a.k_sb + g * a.k_sh + (int64_t)j * a.k_st;
-      const __nv_bfloat16* vp = a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st;
-      const float k0 = bf(kp, p), k1 = bf(kp, p + H);
-      float r0, r1;
-      rot(k0, k1, tab_at(a.tab, j, H, p), r0, r1);
-      s_sink[jj][0][p] = r0;
-      s_sink[jj][0][p + H] = r1;
-      s_sink[jj][1][p] = k0;
-      s_sink[jj][1][p + H] = k1;
-      s_sink[jj][2][p] = bf(vp, p);
-      s_sink[jj][2][p + H] = bf(vp, p + H);
+    for (int x = threadIdx.x; x < nst * D; x += blockDim.x) {
+      const int jj = x / D, c = x % D, j = js + jj;
+      s_sink[jj][c] = bf(a.V + b * a.v_sb + g * a.v_sh + (int64_t)j * a.v_st, c);
     }
     __syncthreads();
     // every lane of a row takes the same branches (same i, same j)
@@ -143,7 +128,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
       const int j = js + jj;
       float dp = 0.f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) dp = fmaf(g0[e], s_sink[jj][2][c0 + e], fmaf(g1[e], s_sink[jj][2][c0 + e + H], dp));
+      for (int e = 0; e < E; ++e) dp = fmaf(g0[e], s_sink[jj][c0 + e], fmaf(g1[e], s_sink[jj][c0 + e + H], dp));
       dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 1);
       dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 2);
       dp += __shfl_xor_sync(0xffu << (threadIdx.x & 24), dp, 4);
@@ -153,36 +138,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
         a.sink_ds[wid * ns_all + j] = ds;
         a.sink_p[wid * ns_all + j] = p;
       }
-      const bool capped = a.L > 0 && (i - j) > a.L;
-      const float* kr = s_sink[jj][capped ? 1 : 0];
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        if (capped) {
-          ac0[e] = fmaf(ds, kr[c0 + e], ac0[e]);
-          ac1[e] = fmaf(ds, kr[c0 + e + H], ac1[e]);
-        } else {
-          ar0[e] = fmaf(ds, kr[c0 + e], ar0[e]);
-          ar1[e] = fmaf(ds, kr[c0 + e + H], ar1[e]);
-        }
-      }
     }
-  }
-  if (!row_ok) return;
-  const float scale = rsqrtf((float)D);
-  float* out = a.dq_side + wid * D;
-  float y0[E], y1[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float x0, x1, z0, z1;
-    rot_t(ar0[e], ar1[e], tab_at(a.tab, i, H, c0 + e), x0, x1);
-    rot_t(ac0[e], ac1[e], a.L > 0 ? tab_at(a.tab, a.L, H, c0 + e) : make_float2(1.f, 0.f), z0, z1);
-    y0[e] = (x0 + z0) * scale;
-    y1[e] = (x1 + z1) * scale;
-  }
-#pragma unroll
-  for (int e = 0; e < E; e += 4) {
-    *reinterpret_cast<float4*>(out + c0 + e) = make_float4(y0[e], y0[e + 1], y0[e + 2], y0[e + 3]);
-    *reinterpret_cast<float4*>(out + c0 + e + H) = make_float4(y1[e], y1[e + 1], y1[e + 2], y1[e + 3]);
   }
 }
 

@@ -90,6 +90,8 @@ __device__ __forceinline__ QPlan make_qplan(const BwdArgs& a, int b, int t) {
   return p;
 }
 
+constexpr int kFoldStage = 16;  // sink key rows staged at a time in the dq epilogue
+
 template <int D>
 struct QCfg {
   static constexpr uint32_t kTileBytes = D * kTile * 2;
@@ -357,7 +359,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int y = 0; y < 32; ++y) v[y] = 0.f;
       }
-      rotate_back(v, a.tab, pos, half, cc, hc);
+      if (a.fold_sinks) {
+        // the sink pairs (fp32 side keys; P and dS from the row pass): the
+        // uncapped sum of dS R(j) k_j joins v before the rotation back by
+        // R(i)^T, the capped sum of dS k_j is rotated back by R(L)^T.  The
+        // sink keys (rotated and raw, fp32) are staged in the K ring, free
+        // once the last MMA has completed; a lane reads the component (hc)
+        // of the pairs it holds.
+        float* s_kr = reinterpret_cast<float*>(sK);  // [kFoldStage][D] R(j) k_j
+        float* s_kw = s_kr + kFoldStage * D;          // [kFoldStage][D] k_j
+        float vc[32];
+#pragma unroll
+        for (int y = 0; y < 32; ++y) vc[y] = 0.f;
+        const int ns = row_ok ? min(a.n_sink, i + 1) : 0;
+        const float* dsr = a.sink_ds + grow * a.n_sink;
+        const bool restage = a.n_sink > kFoldStage || cc == 0;  // one stage serves both chunks
+        for (int js = 0; js < a.n_sink; js += kFoldStage) {
+          const int nst = min(kFoldStage, a.n_sink - js);
+          if (restage) {
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // the epilogue warps: the stage is free
+            for (int x = threadIdx.x; x < nst * half; x += 256) {
+              const int jj = x / half, p = x - jj * half, j = js + jj;
+              const __nv_bfloat16* kp = a.K + (int64_t)b * a.k_sb + (int64_t)g * a.k_sh + (int64_t)j * a.k_st;
+              const float k0 = __bfloat162float(kp[p]), k1 = __bfloat162float(kp[p + half]);
+              const float2 cs = tab_at(a.tab, j, half, p);
+              s_kr[jj * D + p] = k0 * cs.x - k1 * cs.y;
+              s_kr[jj * D + p + half] = k1 * cs.x + k0 * cs.y;
+              s_kw[jj * D + p] = k0;
+              s_kw[jj * D + p + half] = k1;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+          }
+          for (int jj = 0; jj < nst && js + jj < ns; ++jj) {
+            const int j = js + jj;
+            const float ds = dsr[j];
+            const bool capped = a.L > 0 && i - j > a.L;
+            const float* src = (capped ? s_kw : s_kr) + jj * D + hc * half + cc;
+#pragma unroll
+            for (int y = 0; y < 32; ++y) {
+              if (capped) vc[y] = fmaf(ds, src[y], vc[y]);
+              else v[y] = fmaf(ds, src[y], v[y]);
+            }
+          }
+        }
+        rotate_back(v, a.tab, pos, half, cc, hc);
+        if (a.L > 0) {
+          rotate_back(vc, a.tab, a.L, half, cc, hc);
+#pragma unroll
+          for (int y = 0; y < 32; ++y) v[y] += vc[y];
+        }
+      } else {
+        rotate_back(v, a.tab, pos, half, cc, hc);
+      }
       const int col = hc * half + cc;
       float* side = a.dq_side + grow * D + col;
       if (a.side_valid && row_ok) {

@@ -272,7 +272,7 @@ struct BwdArgs {
   float* sink_part;             // [B, Hkv, n_sink, nRB, 2, d] partial key-side sums per row block
   int nRB;                      // row blocks of the sink reduction
   // fp32 scratch
-  float* dq_side;               // [B, Hq, T, d] dq from sinks and capped separators (raw frame)
+  float* dq_side;               // [B, Hq, T, d] dq of the capped separators (raw frame, scaled)
   float* dk_band;               // [B, Hkv, T, d] band-tile dk (raw frame)
   float* dv_band;
   float* dk_sep;                // [B, Hkv, Tpad, d] separator dk, compacted order (raw frame)
@@ -284,6 +284,7 @@ struct BwdArgs {
   int32_t* status;
   int dq_mode;                  // dq kernel: 0 band (+ uncapped separators), 1 capped separators only
   bool side_valid;              // dq_side holds data (else it is not read)
+  int fold_sinks;               // dq kernel (mode 0): add the sink pairs' dq from sink_ds and the sink key rows
 };
 struct BwdMaps {
   CUtensorMap q, qc, dO, k, v, kg, vg;
