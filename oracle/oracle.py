@@ -83,6 +83,9 @@ def lib():
                 ctypes.c_int]
             L.oracle_bwd.restype = ctypes.c_int
             L.oracle_bwd.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
+            L.oracle_bwd_dq_rows.restype = ctypes.c_int
+            L.oracle_bwd_dq_rows.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 6 + [
+                ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
             L.oracle_blockmap.restype = ctypes.c_int
             L.oracle_blockmap.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 5
             L.oracle_segment_rows.restype = ctypes.c_int
@@ -193,6 +196,24 @@ def bwd(p: OracleParams, q, k, v, is_sep, dO, forced_topk=None, nthreads=None):
     if rc != 0:
         raise RuntimeError("oracle_bwd failed: %d" % rc)
     return dQ, dK, dV
+
+
+def bwd_dq_rows(p: OracleParams, q, k, v, is_sep, dO, rows, forced_topk=None, nthreads=None):
+    """dQ of the rows ``[(b, h, i)]`` alone -> [n, d] float64: the same row
+    arithmetic as ``bwd`` (a row's dq depends on that row only), for sizes
+    where the full backward is too slow."""
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    q, k, v = _inputs(p, q, k, v)
+    g = _c(dO, np.uint16 if p.dtype == 0 else np.float32)
+    assert g.size == q.size
+    s = _c(is_sep, np.uint8)
+    f = _c(forced_topk, np.int32)
+    dq = np.zeros((rows.shape[0], p.d), dtype=np.float64)
+    rc = lib().oracle_bwd_dq_rows(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(s), _ptr(f), _ptr(g),
+                                  rows.shape[0], _ptr(rows), _ptr(dq), nthreads or nthreads_default())
+    if rc != 0:
+        raise RuntimeError("oracle_bwd_dq_rows failed: %d" % rc)
+    return dq
 
 
 def tree_index(chunk_len, depth, alpha_leaf) -> np.ndarray:

@@ -512,10 +512,87 @@ typedef struct {
   double *dQ, *dK, *dV;
 } bwd_job;
 
+/* Row i of query head h (kv head of hc): its dq_i (raw frame) into dq and,
+ * when gKrot / gKraw / gV are given, the row's terms of the key-side sums
+ * (gKrot: d L / d (R(j) k_j) of uncapped pairs, gKraw: d L / d k_j of capped
+ * pairs, gV: d L / d v_j).  work holds 7 d doubles; m, P, dP, cands are
+ * per-thread row buffers of T (+1) entries. */
+static void bwd_row(head_ctx* hc, const void* Q, const void* dO, const int32_t* forced, int b, int h, int i,
+                    double* work, uint8_t* m, double* P, double* dP, cand_t* cands, double* gKrot,
+                    double* gKraw, double* gV, double* dq) {
+  const oracle_params* p = hc->p;
+  int T = p->T, d = p->d, L = p->L_pretrain, k = p->topk;
+  const double* Kraw = hc->Kraw;
+  const double* Krot = hc->Krot;
+  const double* Vd = hc->Vd;
+  double *qraw = work, *q_i = work + d, *q_L = work + 2 * d, *doi = work + 3 * d;
+  double *gqr = work + 4 * d, *gqc = work + 5 * d, *tmp = work + 6 * d;
+  double slope = p->alibi ? alibi_slope(p, h) : 0.0;
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  int64_t qb = (((int64_t)b * p->Hq + h) * T + i) * d;
+  for (int c = 0; c < d; ++c) {
+    qraw[c] = load_elem(Q, p->dtype, qb + c);
+    doi[c] = load_elem(dO, p->dtype, qb + c);
+  }
+  oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
+  oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
+  const int32_t* fr = forced ? forced + ((((int64_t)b * p->Hq + h) * T) + i) * k : NULL;
+  int64_t cnt = row_key_set(hc, q_i, q_L, h, i, fr, NULL, NULL, m, cands);
+  for (int c = 0; c < d; ++c) gqr[c] = gqc[c] = 0.0;
+  if (cnt > 0) {
+    /* forward quantities of the row: P_ij = exp(s_ij - LSE_i) */
+    double mx = -INFINITY;
+    for (int j = 0; j < T; ++j)
+      if (m[j]) {
+        P[j] = row_logit(hc, q_i, q_L, slope, i, j);
+        if (P[j] > mx) mx = P[j];
+      }
+    double sum = 0.0;
+    for (int j = 0; j < T; ++j)
+      if (m[j]) sum += exp(P[j] - mx);
+    double lse = mx + log(sum);
+    /* dP_ij = dO_i . v_j and D_i = sum_j P_ij dP_ij (= dO_i . O_i) */
+    double D = 0.0;
+    for (int j = 0; j < T; ++j)
+      if (m[j]) {
+        P[j] = exp(P[j] - lse);
+        dP[j] = dot(doi, Vd + (size_t)j * d, d);
+        D += P[j] * dP[j];
+      }
+    for (int j = 0; j < T; ++j) {
+      if (!m[j]) continue;
+      /* dL/dz_ij: softmax Jacobian, then the 1/sqrt(d) scale */
+      double dz = P[j] * (dP[j] - D) * inv_sqrt_d;
+      if (gV) {
+        double* gv = gV + (size_t)j * d;
+        for (int c = 0; c < d; ++c) gv[c] += P[j] * doi[c];
+      }
+      if (L > 0 && i - j > L) {
+        /* z = <R(L) q_i, k_j> */
+        for (int c = 0; c < d; ++c) {
+          gqc[c] += dz * Kraw[(size_t)j * d + c];
+          if (gKraw) gKraw[(size_t)j * d + c] += dz * q_L[c];
+        }
+      } else {
+        /* z = <R(i) q_i, R(j) k_j> */
+        for (int c = 0; c < d; ++c) {
+          gqr[c] += dz * Krot[(size_t)j * d + c];
+          if (gKrot) gKrot[(size_t)j * d + c] += dz * q_i[c];
+        }
+      }
+    }
+  }
+  /* back through the rotations: R(p)^T = R(-p) */
+  oracle_rope(gqr, d, -rot_pos(p, (double)i), p->rope_theta, tmp);
+  for (int c = 0; c < d; ++c) dq[c] = tmp[c];
+  oracle_rope(gqc, d, -rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, tmp);
+  for (int c = 0; c < d; ++c) dq[c] += tmp[c];
+}
+
 static void bwd_one(void* arg, int64_t t) {
   bwd_job* J = (bwd_job*)arg;
   const oracle_params* p = J->p;
-  int T = p->T, d = p->d, L = p->L_pretrain, k = p->topk;
+  int T = p->T, d = p->d;
   int b = (int)(t / p->Hkv), g = (int)(t % p->Hkv);
   double* Kraw = (double*)malloc(sizeof(double) * (size_t)T * d);
   double* Krot = (double*)malloc(sizeof(double) * (size_t)T * d);
@@ -528,8 +605,7 @@ static void bwd_one(void* arg, int64_t t) {
   double* dP = (double*)malloc(sizeof(double) * (size_t)T);
   cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T + 1));
   double* work = (double*)malloc(sizeof(double) * 8 * (size_t)d);
-  double *qraw = work, *q_i = work + d, *q_L = work + 2 * d, *doi = work + 3 * d;
-  double *gqr = work + 4 * d, *gqc = work + 5 * d, *tmp = work + 6 * d;
+  double* tmp = work + 7 * d;
   head_ctx hc;
   hc.p = p;
   hc.Kraw = Kraw;
@@ -538,69 +614,10 @@ static void bwd_one(void* arg, int64_t t) {
   hc.sep = J->is_sep ? J->is_sep + (size_t)b * T : NULL;
   load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
   int rep = p->Hq / p->Hkv;
-  double inv_sqrt_d = 1.0 / sqrt((double)d);
-  for (int h = g * rep; h < (g + 1) * rep; ++h) {
-    double slope = p->alibi ? alibi_slope(p, h) : 0.0;
-    for (int i = 0; i < T; ++i) {
-      int64_t qb = (((int64_t)b * p->Hq + h) * T + i) * d;
-      for (int c = 0; c < d; ++c) {
-        qraw[c] = load_elem(J->Q, p->dtype, qb + c);
-        doi[c] = load_elem(J->dO, p->dtype, qb + c);
-      }
-      oracle_rope(qraw, d, rot_pos(p, (double)i), p->rope_theta, q_i);
-      oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
-      const int32_t* fr = J->forced ? J->forced + ((((int64_t)b * p->Hq + h) * T) + i) * k : NULL;
-      int64_t cnt = row_key_set(&hc, q_i, q_L, h, i, fr, NULL, NULL, m, cands);
-      for (int c = 0; c < d; ++c) gqr[c] = gqc[c] = 0.0;
-      if (cnt > 0) {
-        /* forward quantities of the row: P_ij = exp(s_ij - LSE_i) */
-        double mx = -INFINITY;
-        for (int j = 0; j < T; ++j)
-          if (m[j]) {
-            P[j] = row_logit(&hc, q_i, q_L, slope, i, j);
-            if (P[j] > mx) mx = P[j];
-          }
-        double sum = 0.0;
-        for (int j = 0; j < T; ++j)
-          if (m[j]) sum += exp(P[j] - mx);
-        double lse = mx + log(sum);
-        /* dP_ij = dO_i . v_j and D_i = sum_j P_ij dP_ij (= dO_i . O_i) */
-        double D = 0.0;
-        for (int j = 0; j < T; ++j)
-          if (m[j]) {
-            P[j] = exp(P[j] - lse);
-            dP[j] = dot(doi, Vd + (size_t)j * d, d);
-            D += P[j] * dP[j];
-          }
-        for (int j = 0; j < T; ++j) {
-          if (!m[j]) continue;
-          /* dL/dz_ij: softmax Jacobian, then the 1/sqrt(d) scale */
-          double dz = P[j] * (dP[j] - D) * inv_sqrt_d;
-          double* gv = gV + (size_t)j * d;
-          for (int c = 0; c < d; ++c) gv[c] += P[j] * doi[c];
-          if (L > 0 && i - j > L) {
-            /* z = <R(L) q_i, k_j> */
-            for (int c = 0; c < d; ++c) {
-              gqc[c] += dz * Kraw[(size_t)j * d + c];
-              gKraw[(size_t)j * d + c] += dz * q_L[c];
-            }
-          } else {
-            /* z = <R(i) q_i, R(j) k_j> */
-            for (int c = 0; c < d; ++c) {
-              gqr[c] += dz * Krot[(size_t)j * d + c];
-              gKrot[(size_t)j * d + c] += dz * q_i[c];
-            }
-          }
-        }
-      }
-      /* back through the rotations: R(p)^T = R(-p) */
-      double* dq = J->dQ + qb;
-      oracle_rope(gqr, d, -rot_pos(p, (double)i), p->rope_theta, tmp);
-      for (int c = 0; c < d; ++c) dq[c] = tmp[c];
-      oracle_rope(gqc, d, -rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, tmp);
-      for (int c = 0; c < d; ++c) dq[c] += tmp[c];
-    }
-  }
+  for (int h = g * rep; h < (g + 1) * rep; ++h)
+    for (int i = 0; i < T; ++i)
+      bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, gKrot, gKraw, gV,
+              J->dQ + (((int64_t)b * p->Hq + h) * T + i) * d);
   int64_t kb = ((int64_t)b * p->Hkv + g) * (int64_t)T * d;
   for (int j = 0; j < T; ++j) {
     oracle_rope(gKrot + (size_t)j * d, d, -rot_pos(p, (double)j), p->rope_theta, tmp);
@@ -641,6 +658,74 @@ int oracle_bwd(const oracle_params* p, const void* Q, const void* K, const void*
   J.dK = dK;
   J.dV = dV;
   run_parallel(bwd_one, &J, (int64_t)p->B * p->Hkv, nthreads);
+  return OR_OK;
+}
+
+/* dq of the sampled rows [(b, h, i)] alone (row i's dq depends on row i
+ * only): the same row arithmetic as oracle_bwd, for sizes where the full
+ * backward is too slow.  dq [n, d] in double. */
+typedef struct {
+  const oracle_params* p;
+  const void *Q, *K, *V, *dO;
+  const uint8_t* is_sep;
+  const int32_t* forced;
+  const int64_t* rows;
+  double* dq;
+} bwd_rows_job;
+
+static void bwd_rows_one(void* arg, int64_t r) {
+  bwd_rows_job* J = (bwd_rows_job*)arg;
+  const oracle_params* p = J->p;
+  int T = p->T, d = p->d;
+  int b = (int)J->rows[3 * r], h = (int)J->rows[3 * r + 1], i = (int)J->rows[3 * r + 2];
+  int g = h / (p->Hq / p->Hkv);
+  double* Kraw = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Krot = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Vd = (double*)malloc(sizeof(double) * (size_t)T * d);
+  uint8_t* m = (uint8_t*)malloc((size_t)T);
+  double* P = (double*)malloc(sizeof(double) * (size_t)T);
+  double* dP = (double*)malloc(sizeof(double) * (size_t)T);
+  cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T + 1));
+  double* work = (double*)malloc(sizeof(double) * 8 * (size_t)d);
+  head_ctx hc;
+  hc.p = p;
+  hc.Kraw = Kraw;
+  hc.Krot = Krot;
+  hc.Vd = Vd;
+  hc.sep = J->is_sep ? J->is_sep + (size_t)b * T : NULL;
+  load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
+  bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, NULL, NULL, NULL, J->dq + r * d);
+  free(Kraw);
+  free(Krot);
+  free(Vd);
+  free(m);
+  free(P);
+  free(dP);
+  free(cands);
+  free(work);
+}
+
+int oracle_bwd_dq_rows(const oracle_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                       const int32_t* forced, const void* dO, int64_t n, const int64_t* rows, double* dq,
+                       int nthreads) {
+  if (!p || p->d <= 0 || (p->d & 1) || p->T <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv || n < 0 ||
+      (n > 0 && !rows))
+    return OR_ERR_ARG;
+  for (int64_t r = 0; r < n; ++r)
+    if (rows[3 * r] < 0 || rows[3 * r] >= p->B || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= p->Hq ||
+        rows[3 * r + 2] < 0 || rows[3 * r + 2] >= p->T)
+      return OR_ERR_ARG;
+  bwd_rows_job J;
+  J.p = p;
+  J.Q = Q;
+  J.K = K;
+  J.V = V;
+  J.dO = dO;
+  J.is_sep = is_sep;
+  J.forced = forced;
+  J.rows = rows;
+  J.dq = dq;
+  run_parallel(bwd_rows_one, &J, n, nthreads);
   return OR_OK;
 }
 

@@ -136,3 +136,40 @@ def test_bwd_rejects_missing_topk_selection():
     lse = torch.zeros((1, 1, 64), dtype=torch.float32, device="cuda")
     with pytest.raises(_lib.SattnError):
         sa.bwd(q, q, q, q, lse, q, window=4, L_pretrain=4, topk=2)
+
+
+@pytest.mark.parametrize("name", ["c2_lminf_16k", "c3_sepllm_gqa_8k"])
+def test_bwd_full_size_sampled(oracle_mod, name):
+    """The backward at the benchmark's full sizes (the launch the backward
+    workloads time): dQ on sampled rows against the oracle's rows entry, and
+    for every kv head the sum of dV over keys against its group's sum of dO
+    over rows (every row's weights sum to one), within 2^-7 of sum |dV|: the
+    rounding of each dV element to bf16 (2^-9) and the error of P recomputed
+    from bf16 operands."""
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_inputs(wl, seed=0)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    g = np.random.default_rng(7)
+    dO_h = (g.standard_normal(inp["q"].shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    dO = to_dev(dO_h)
+    O, lse = sa.fwd(q, k, v, is_sep=sep, **_kw(wl))
+    dq, dk, dv = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, **_kw(wl))
+    torch.cuda.synchronize()
+    assert sa.stream_status() == 0
+    rng = np.random.default_rng(1)
+    n = 48
+    rows = np.stack([rng.integers(0, wl.B, n), rng.integers(0, wl.Hq, n), rng.integers(0, wl.T, n)], axis=1)
+    rows[:4, 2] = [0, 1, wl.T // 2, wl.T - 1]
+    ref = oracle_mod.bwd_dq_rows(oracle_mod.params_of(wl), inp["q"], inp["k"], inp["v"], inp["is_sep"], dO_h, rows)
+    ri = torch.as_tensor(rows, device=dq.device)
+    got = dq[ri[:, 0], ri[:, 1], ri[:, 2]].float().cpu().numpy().astype(np.float64)
+    compare_grad("dQ rows", got, ref, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
+    rep = wl.Hq // wl.Hkv
+    dv64 = dv.double()
+    lhs = dv64.sum(dim=2)
+    rhs = dO.double().reshape(wl.B, wl.Hkv, rep, wl.T, wl.d).sum(dim=(2, 3))
+    bound = dv64.abs().sum(dim=2) * 2.0 ** -7 + 1e-6
+    excess = ((lhs - rhs).abs() - bound).max().item()
+    print("dV sum: max |lhs - rhs| %.3g, bound %.3g" % ((lhs - rhs).abs().max().item(), bound.min().item()))
+    assert excess <= 0.0

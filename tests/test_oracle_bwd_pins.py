@@ -151,3 +151,26 @@ def test_invariants(oracle_mod):
     p2 = O.params(B, Hq, Hkv, T, d, "f32", 2, 4, 6, 3, 1e2)
     _, dK2, _ = O.bwd(p2, q, k, v, sep, dO, nthreads=2)
     assert np.abs(dK2.sum(axis=2)).max() > 1e-3
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(dtype="f32", n_start=2, window=4, L_pretrain=6, topk=3, rope_theta=1e2),   # capped, separators, top-k
+    dict(dtype="f32", n_start=1, window=5, L_pretrain=5, topk=0, alibi=True),       # clipped ALiBi
+    dict(dtype="f32", n_start=0, window=100, L_pretrain=0, topk=0, rope_theta=0.0),  # full causal
+])
+def test_dq_rows_entry_equals_full_backward(oracle_mod, cfg):
+    """oracle_bwd_dq_rows (the rows-only entry used at full sizes) runs the
+    same row arithmetic as the pinned full backward: equal bits."""
+    O = oracle_mod
+    B, Hq, Hkv, T, d = 2, 4, 2, 40, 8
+    q, k, v, dO = _grid_inputs(B, Hq, Hkv, T, d, 11)
+    rng = np.random.default_rng(12)
+    sep = (rng.random((B, T)) < 0.3).astype(np.uint8)
+    p = O.params(B, Hq, Hkv, T, d, **cfg)
+    forced = _forced_of(O, p, q, k, v, sep) if p.topk else None
+    dQ, _, _ = O.bwd(p, q, k, v, sep, dO, forced_topk=forced, nthreads=2)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(Hq) for i in (0, 1, 7, 20, T - 1)])
+    dq = O.bwd_dq_rows(p, q, k, v, sep, dO, rows, forced_topk=forced, nthreads=2)
+    assert np.array_equal(dq, dQ[rows[:, 0], rows[:, 1], rows[:, 2]])
+    with pytest.raises(RuntimeError):
+        O.bwd_dq_rows(p, q, k, v, sep, dO, np.array([(0, 0, T)]))
