@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdArgs a) {
 // raw-frame dk part (R(j)^T of the uncapped sum plus the capped sum,
 // unscaled) and the dv part of each sink.
 constexpr int kSinkGroup = 4;
-constexpr int kRowsInFlight = 4;  // rows per warp whose loads are issued together
+constexpr int kRowsInFlight = 8;  // rows per warp whose loads are issued together
 
 // PL consecutive bf16 (one or two) as floats
 template <int PL>
