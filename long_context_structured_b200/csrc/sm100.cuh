@@ -114,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), 4-D tiled loads without multicast
+// TMA (cp.async.bulk.tensor), 4-D tiled loads into this CTA's shared memory
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

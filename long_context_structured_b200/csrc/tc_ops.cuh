@@ -50,7 +50,7 @@ __device__ __forceinline__ bool wait_raw(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// 1-D bulk copy global -> shared (no multicast), completing on `bar`.
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(
