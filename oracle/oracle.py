@@ -91,6 +91,9 @@ def lib():
             L.oracle_segment_rows.restype = ctypes.c_int
             L.oracle_segment_rows.argtypes = [P(OracleParams)] + [ctypes.c_int] * 4 + [
                 ctypes.c_void_p] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 4 + [ctypes.c_int]
+            L.oracle_segment_bwd.restype = ctypes.c_int
+            L.oracle_segment_bwd.argtypes = [P(OracleParams)] + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 8 + [
+                ctypes.c_int]
             L.oracle_segment_blocks.restype = ctypes.c_int
             L.oracle_segment_blocks.argtypes = [P(OracleParams)] + [ctypes.c_int] * 3 + [
                 ctypes.c_void_p] * 5
@@ -270,6 +273,23 @@ def segment_rows(p: OracleParams, S, M, R, blk, is_long, q, k, v, rows, nthreads
     if rc != 0:
         raise RuntimeError("oracle_segment_rows failed: %d" % rc)
     return O, lse, cnt
+
+
+def segment_bwd(p: OracleParams, S, M, R, blk, is_long, q, k, v, dO, nthreads=None):
+    """Gradients of sum(dO * O) for segmented execution, the retrieval held
+    fixed: (dQ [B,Hq,T,d], dK [B,Hkv,T,d], dV [B,Hkv,T,d]) in float64."""
+    il = np.ascontiguousarray(np.asarray(is_long, dtype=np.uint8))
+    q, k, v = _inputs(p, q, k, v)
+    g = _c(dO, np.uint16 if p.dtype == 0 else np.float32)
+    assert g.size == q.size
+    dQ = np.zeros((p.B, p.Hq, p.T, p.d), dtype=np.float64)
+    dK = np.zeros((p.B, p.Hkv, p.T, p.d), dtype=np.float64)
+    dV = np.zeros((p.B, p.Hkv, p.T, p.d), dtype=np.float64)
+    rc = lib().oracle_segment_bwd(ctypes.byref(p), S, M, R, blk, _ptr(il), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), nthreads or nthreads_default())
+    if rc != 0:
+        raise RuntimeError("oracle_segment_bwd failed: %d" % rc)
+    return dQ, dK, dV
 
 
 def segment_blocks(p: OracleParams, S, R, blk, is_long, q, k):

@@ -81,6 +81,11 @@
  *       top-k selection and the mask are constants (no gradient flows
  *       through a choice); a capped pair contributes to k_j directly and to
  *       q_i through R(L)^T, an uncapped one through R(j)^T and R(i)^T.
+ *   R14 segmented backward ([SEG] 整体框架 with R12): the same gradients
+ *       over each row's segmented key list; the retrieved blocks, like the
+ *       top-k sets, are constants, so a retrieved key's gradient goes back
+ *       to its source position through its re-based rotary position, and a
+ *       key used by several rows (or segments) sums their contributions.
  *
  * Parity pins: every function here is checked by the CPU tests against
  * closed forms, hand-written golden masks, library routines on degenerate
@@ -1120,6 +1125,134 @@ int oracle_segment_rows(const oracle_params* p, int S, int M, int R, int blk, co
   free(Krot);
   free(Vd);
   free(sel);
+  return OR_OK;
+}
+
+/* Backward of segmented execution: gradients of L = sum dO . O with each
+ * row's key list (tail or retrieved prefix, then the segment causally) and
+ * its rotary positions as in oracle_segment_rows; the retrieval selection,
+ * like the top-k sets, is a constant of the backward pass.  Per kept key x
+ * of row i (source position kj_x, rotary position kp_x, query position
+ * P + t): z_x = <R(P + t) q_i, R(kp_x) k_{kj_x}> / sqrt(d), p = softmax(z),
+ * dz_x = p_x (dO_i . v_{kj_x} - D_i), D_i = sum_x p_x dO_i . v_{kj_x};
+ * dq_i = R(P+t)^T sum_x dz_x R(kp_x) k, dk_{kj_x} += R(kp_x)^T dz_x R(P+t) q_i,
+ * dv_{kj_x} += p_x dO_i.  One job per (batch, kv head), rows in order. */
+typedef struct {
+  const oracle_params* p;
+  int S, M, R, blk;
+  const uint8_t* is_long;
+  const void *Q, *K, *V, *dO;
+  double *dQ, *dK, *dV;
+} segbwd_job;
+
+static void segbwd_one(void* a, int64_t t) {
+  segbwd_job* J = (segbwd_job*)a;
+  const oracle_params* p = J->p;
+  int T = p->T, d = p->d;
+  int b = (int)(t / p->Hkv), g = (int)(t % p->Hkv);
+  int nb = J->R / J->blk;
+  int cap = J->M + J->R + J->S + 1;
+  double* Kraw = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Krot = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Vd = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* gK = (double*)calloc((size_t)T * d, sizeof(double));
+  double* gV = (double*)calloc((size_t)T * d, sizeof(double));
+  int32_t* kj = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  int32_t* kp = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  int32_t* blocks = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nb + 1));
+  double* kr = (double*)malloc(sizeof(double) * (size_t)cap * d); /* R(kp_x) k_{kj_x} */
+  double* sbuf = (double*)malloc(sizeof(double) * (size_t)cap);
+  double* dpb = (double*)malloc(sizeof(double) * (size_t)cap);
+  double* w = (double*)malloc(sizeof(double) * 8 * (size_t)d);
+  double *q = w, *qrot = w + d, *doi = w + 2 * d, *gq = w + 3 * d, *tmp = w + 4 * d, *qlast = w + 6 * d;
+  load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
+  int rep = p->Hq / p->Hkv;
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  for (int h = g * rep; h < (g + 1) * rep; ++h) {
+    for (int i = 0; i < T; ++i) {
+      int s = i / J->S, tt = i - s * J->S;
+      int64_t qb = (((int64_t)b * p->Hq + h) * T + i) * d;
+      for (int c = 0; c < d; ++c) {
+        q[c] = load_elem(J->Q, p->dtype, qb + c);
+        doi[c] = load_elem(J->dO, p->dtype, qb + c);
+      }
+      int P = 0;
+      int n = segment_key_list(J->Q, p, Kraw, J->S, J->M, J->R, J->blk, J->is_long, b, h, i, kj, kp, &P, blocks,
+                               qlast);
+      oracle_rope(q, d, rot_pos(p, (double)(P + tt)), p->rope_theta, qrot);
+      double mx = -INFINITY;
+      for (int x = 0; x < n; ++x) {
+        oracle_rope(Kraw + (size_t)kj[x] * d, d, rot_pos(p, (double)kp[x]), p->rope_theta, kr + (size_t)x * d);
+        sbuf[x] = dot(qrot, kr + (size_t)x * d, d) * inv_sqrt_d;
+        if (sbuf[x] > mx) mx = sbuf[x];
+      }
+      double sum = 0.0;
+      for (int x = 0; x < n; ++x) sum += exp(sbuf[x] - mx);
+      double lse = mx + log(sum);
+      double D = 0.0;
+      for (int x = 0; x < n; ++x) {
+        sbuf[x] = exp(sbuf[x] - lse); /* now P_x */
+        dpb[x] = dot(doi, Vd + (size_t)kj[x] * d, d);
+        D += sbuf[x] * dpb[x];
+      }
+      for (int c = 0; c < d; ++c) gq[c] = 0.0;
+      for (int x = 0; x < n; ++x) {
+        double dz = sbuf[x] * (dpb[x] - D) * inv_sqrt_d;
+        double* gv = gV + (size_t)kj[x] * d;
+        for (int c = 0; c < d; ++c) {
+          gv[c] += sbuf[x] * doi[c];
+          gq[c] += dz * kr[(size_t)x * d + c];
+        }
+        /* d L / d k_{kj_x} = R(kp_x)^T dz R(P + t) q_i */
+        for (int c = 0; c < d; ++c) tmp[c] = dz * qrot[c];
+        oracle_rope(tmp, d, -rot_pos(p, (double)kp[x]), p->rope_theta, tmp + d);
+        double* gk = gK + (size_t)kj[x] * d;
+        for (int c = 0; c < d; ++c) gk[c] += tmp[d + c];
+      }
+      oracle_rope(gq, d, -rot_pos(p, (double)(P + tt)), p->rope_theta, tmp);
+      for (int c = 0; c < d; ++c) J->dQ[qb + c] = tmp[c];
+    }
+  }
+  int64_t kb = ((int64_t)b * p->Hkv + g) * (int64_t)T * d;
+  for (int64_t x = 0; x < (int64_t)T * d; ++x) {
+    J->dK[kb + x] = gK[x];
+    J->dV[kb + x] = gV[x];
+  }
+  free(Kraw);
+  free(Krot);
+  free(Vd);
+  free(gK);
+  free(gV);
+  free(kj);
+  free(kp);
+  free(blocks);
+  free(kr);
+  free(sbuf);
+  free(dpb);
+  free(w);
+}
+
+int oracle_segment_bwd(const oracle_params* p, int S, int M, int R, int blk, const uint8_t* is_long, const void* Q,
+                       const void* K, const void* V, const void* dO, double* dQ, double* dK, double* dV,
+                       int nthreads) {
+  if (!p || !is_long || S <= 0 || M < 0 || R < 0 || blk <= 0 || R % blk || p->T % S || p->Hq % p->Hkv ||
+      p->d <= 0 || (p->d & 1))
+    return OR_ERR_ARG;
+  segbwd_job J;
+  J.p = p;
+  J.S = S;
+  J.M = M;
+  J.R = R;
+  J.blk = blk;
+  J.is_long = is_long;
+  J.Q = Q;
+  J.K = K;
+  J.V = V;
+  J.dO = dO;
+  J.dQ = dQ;
+  J.dK = dK;
+  J.dV = dV;
+  run_parallel(segbwd_one, &J, (int64_t)p->B * p->Hkv, nthreads);
   return OR_OK;
 }
 
