@@ -65,3 +65,18 @@ def test_decode_step_equals_sdpa_with_rolled_positions(oracle_mod, theta):
         torch.from_numpy(qr), torch.from_numpy(kr).repeat_interleave(Hq // Hkv, 1),
         torch.from_numpy(v[None]).repeat_interleave(Hq // Hkv, 1)).numpy()[0, :, 0]
     assert np.abs(O - ref).max() < 1e-12
+
+
+def test_hand_worked_trace():
+    """The cache's contents after every token of a hand-worked stream
+    (tests/golden/stream_cache_a1_s2_w2_c6.txt)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "stream_cache_a1_s2_w2_c6.txt")
+    lines = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    a, s, w, c = (int(x) for x in lines[0])
+    seps = {int(x) for x in lines[1]}
+    cache = StreamCache(a, s, w, c)
+    for t_str, want in lines[2:]:
+        t = int(t_str)
+        cache.append(t, t in seps)
+        assert [e[0] for e in cache.slots()] == [int(x) for x in want.split(",")], "after token %d" % t
