@@ -797,3 +797,16 @@ def test_tree_cross_equals_sdpa_on_kept_rows(oracle_mod, theta, depth, alpha):
         assert np.abs(got - full).max() < 1e-12
     lref = _lse_ref(qq, kk, np.ones((T, len(rows)), dtype=bool))
     assert np.abs(lse - lref).max() < 1e-12
+
+
+def test_tree_index_hand_worked_ragged(oracle_mod):
+    """Uneven splits (chunk lengths not a power of two), worked out by hand
+    (tests/golden/tree_kept_ragged.txt)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tree_kept_ragged.txt")
+    for ln in open(path):
+        if not ln.strip() or ln.startswith("#"):
+            continue
+        l, depth, alpha, want = ln.split()
+        got = list(oracle_mod.tree_index(int(l), int(depth), int(alpha)))
+        assert got == [int(x) for x in want.split(",")], ln
