@@ -93,7 +93,7 @@ def _sdpa_grads(q, k, v, dO, mask):
     return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
 
 
-@pytest.mark.parametrize("ns,w", [(0, 100), (0, 5), (3, 4)])
+@pytest.mark.parametrize("ns,w", [(0, 100), (0, 5), (3, 4), (20, 3)])
 def test_autograd_sdpa_masks(oracle_mod, ns, w):
     """No rotation and no cap: the oracle's gradients equal torch autograd
     through fp64 SDPA with the Lambda mask (full causal, sliding window,

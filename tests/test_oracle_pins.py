@@ -256,14 +256,14 @@ def test_sliding_window_equals_sdpa(oracle_mod):
     assert np.abs(O.reshape(ref.shape) - ref).max() < 1e-12
 
 
-def test_sink_window_separator_equals_sdpa(oracle_mod):
+@pytest.mark.parametrize("ns,w", [(3, 4), (40, 5)])
+def test_sink_window_separator_equals_sdpa(oracle_mod, ns, w):
     """Sinks + window + separators with no rotation: SDPA with the mask read
-    from the hand-checked oracle mask rows."""
-    B, H, T, d = 2, 2, 45, 8
+    from the hand-checked oracle mask rows (a narrow and a wide sink span)."""
+    B, H, T, d = 2, 2, 80, 8
     q, k, v = _rand_inputs(B, H, H, T, d, 8)
     rng = np.random.default_rng(9)
     sep = (rng.random((B, T)) < 0.2).astype(np.uint8)
-    ns, w = 3, 4
     p = oracle_mod.params(B, H, H, T, d, "bf16", ns, w, 0, 0, 0.0)
     O, *_ = oracle_mod.fwd_rows(p, q, k, v, sep, oracle_mod.all_rows(B, H, T))
     O = O.reshape(B, H, T, d)
