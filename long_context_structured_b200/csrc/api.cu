@@ -307,7 +307,7 @@ int run_blockmap(const sattn_params* p, const FwdPlan& P, const uint8_t* is_sep,
   a.sep_count = sep_count;
   a.ranges = ranges;
   a.cls = cls;
-  ProfScope ps("blockmap", 2, st);
+  ProfScope ps("blockmap", cls ? 2 : 1, st);  // the class kernel runs only when classes are asked for
   return cuda_rc(launch_blockmap(a, st));
 }
 
