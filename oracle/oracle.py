@@ -16,6 +16,10 @@ Parity status of each function (pins live in ``tests/test_oracle_pins.py``):
   blockmap        pinned: numpy nonzero / searchsorted, interval geometry
   segment_rows    pinned: S = T gives causal; R = whole previous segment
                   gives causal over two segments; effective-context count
+  bwd, bwd_dq_rows, bwd_dkv_keys
+                  pinned: central finite differences of the pinned forward,
+                  autograd through fp64 SDPA, sum dV = sum dO; the rows and
+                  keys entries equal the full backward bit for bit
 """
 from __future__ import annotations
 
@@ -86,6 +90,9 @@ def lib():
             L.oracle_bwd_dq_rows.restype = ctypes.c_int
             L.oracle_bwd_dq_rows.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 6 + [
                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+            L.oracle_bwd_dkv_keys.restype = ctypes.c_int
+            L.oracle_bwd_dkv_keys.argtypes = [P(OracleParams)] + [ctypes.c_void_p] * 6 + [
+                ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
             L.oracle_blockmap.restype = ctypes.c_int
             L.oracle_blockmap.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 5
             L.oracle_segment_rows.restype = ctypes.c_int
@@ -217,6 +224,26 @@ def bwd_dq_rows(p: OracleParams, q, k, v, is_sep, dO, rows, forced_topk=None, nt
     if rc != 0:
         raise RuntimeError("oracle_bwd_dq_rows failed: %d" % rc)
     return dq
+
+
+def bwd_dkv_keys(p: OracleParams, q, k, v, is_sep, dO, keys, forced_topk=None, nthreads=None):
+    """dK and dV of the keys ``[(b, g, j)]`` (kv head g) alone -> ([n, d], [n, d])
+    float64: key j's terms of ``bwd``'s key-side sums over every row of the
+    query-head group, summed in the same order, for sizes where the full
+    backward is too slow."""
+    keys = np.ascontiguousarray(keys, dtype=np.int64).reshape(-1, 3)
+    q, k, v = _inputs(p, q, k, v)
+    g = _c(dO, np.uint16 if p.dtype == 0 else np.float32)
+    assert g.size == q.size
+    s = _c(is_sep, np.uint8)
+    f = _c(forced_topk, np.int32)
+    dk = np.zeros((keys.shape[0], p.d), dtype=np.float64)
+    dv = np.zeros((keys.shape[0], p.d), dtype=np.float64)
+    rc = lib().oracle_bwd_dkv_keys(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(s), _ptr(f), _ptr(g),
+                                   keys.shape[0], _ptr(keys), _ptr(dk), _ptr(dv), nthreads or nthreads_default())
+    if rc != 0:
+        raise RuntimeError("oracle_bwd_dkv_keys failed: %d" % rc)
+    return dk, dv
 
 
 def tree_index(chunk_len, depth, alpha_leaf) -> np.ndarray:

@@ -517,14 +517,16 @@ typedef struct {
   double *dQ, *dK, *dV;
 } bwd_job;
 
-/* Row i of query head h (kv head of hc): its dq_i (raw frame) into dq and,
- * when gKrot / gKraw / gV are given, the row's terms of the key-side sums
- * (gKrot: d L / d (R(j) k_j) of uncapped pairs, gKraw: d L / d k_j of capped
- * pairs, gV: d L / d v_j).  work holds 7 d doubles; m, P, dP, cands are
- * per-thread row buffers of T (+1) entries. */
+/* Row i of query head h (kv head of hc): its dq_i (raw frame) into dq (when
+ * dq != NULL) and, when gKrot / gKraw / gV are given, the row's terms of the
+ * key-side sums (gKrot: d L / d (R(j) k_j) of uncapped pairs, gKraw:
+ * d L / d k_j of capped pairs, gV: d L / d v_j).  With only_j >= 0 the
+ * key-side sums are those of key only_j alone, held in d-entry accumulators,
+ * and a row that does not keep only_j adds nothing.  work holds 7 d doubles;
+ * m, P, dP, cands are per-thread row buffers of T (+1) entries. */
 static void bwd_row(head_ctx* hc, const void* Q, const void* dO, const int32_t* forced, int b, int h, int i,
                     double* work, uint8_t* m, double* P, double* dP, cand_t* cands, double* gKrot,
-                    double* gKraw, double* gV, double* dq) {
+                    double* gKraw, double* gV, double* dq, int only_j) {
   const oracle_params* p = hc->p;
   int T = p->T, d = p->d, L = p->L_pretrain, k = p->topk;
   const double* Kraw = hc->Kraw;
@@ -543,6 +545,7 @@ static void bwd_row(head_ctx* hc, const void* Q, const void* dO, const int32_t* 
   oracle_rope(qraw, d, rot_pos(p, (double)(L > 0 ? L : 0)), p->rope_theta, q_L);
   const int32_t* fr = forced ? forced + ((((int64_t)b * p->Hq + h) * T) + i) * k : NULL;
   int64_t cnt = row_key_set(hc, q_i, q_L, h, i, fr, NULL, NULL, m, cands);
+  if (only_j >= 0 && (only_j > i || !m[only_j])) return;
   for (int c = 0; c < d; ++c) gqr[c] = gqc[c] = 0.0;
   if (cnt > 0) {
     /* forward quantities of the row: P_ij = exp(s_ij - LSE_i) */
@@ -568,25 +571,28 @@ static void bwd_row(head_ctx* hc, const void* Q, const void* dO, const int32_t* 
       if (!m[j]) continue;
       /* dL/dz_ij: softmax Jacobian, then the 1/sqrt(d) scale */
       double dz = P[j] * (dP[j] - D) * inv_sqrt_d;
-      if (gV) {
-        double* gv = gV + (size_t)j * d;
+      /* slot of key j in the key-side accumulators (-1: not accumulated) */
+      int64_t ks = only_j < 0 ? j : (j == only_j ? 0 : -1);
+      if (gV && ks >= 0) {
+        double* gv = gV + (size_t)ks * d;
         for (int c = 0; c < d; ++c) gv[c] += P[j] * doi[c];
       }
       if (L > 0 && i - j > L) {
         /* z = <R(L) q_i, k_j> */
         for (int c = 0; c < d; ++c) {
           gqc[c] += dz * Kraw[(size_t)j * d + c];
-          if (gKraw) gKraw[(size_t)j * d + c] += dz * q_L[c];
+          if (gKraw && ks >= 0) gKraw[(size_t)ks * d + c] += dz * q_L[c];
         }
       } else {
         /* z = <R(i) q_i, R(j) k_j> */
         for (int c = 0; c < d; ++c) {
           gqr[c] += dz * Krot[(size_t)j * d + c];
-          if (gKrot) gKrot[(size_t)j * d + c] += dz * q_i[c];
+          if (gKrot && ks >= 0) gKrot[(size_t)ks * d + c] += dz * q_i[c];
         }
       }
     }
   }
+  if (!dq) return;
   /* back through the rotations: R(p)^T = R(-p) */
   oracle_rope(gqr, d, -rot_pos(p, (double)i), p->rope_theta, tmp);
   for (int c = 0; c < d; ++c) dq[c] = tmp[c];
@@ -622,7 +628,7 @@ static void bwd_one(void* arg, int64_t t) {
   for (int h = g * rep; h < (g + 1) * rep; ++h)
     for (int i = 0; i < T; ++i)
       bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, gKrot, gKraw, gV,
-              J->dQ + (((int64_t)b * p->Hq + h) * T + i) * d);
+              J->dQ + (((int64_t)b * p->Hq + h) * T + i) * d, -1);
   int64_t kb = ((int64_t)b * p->Hkv + g) * (int64_t)T * d;
   for (int j = 0; j < T; ++j) {
     oracle_rope(gKrot + (size_t)j * d, d, -rot_pos(p, (double)j), p->rope_theta, tmp);
@@ -699,7 +705,7 @@ static void bwd_rows_one(void* arg, int64_t r) {
   hc.Vd = Vd;
   hc.sep = J->is_sep ? J->is_sep + (size_t)b * T : NULL;
   load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
-  bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, NULL, NULL, NULL, J->dq + r * d);
+  bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, NULL, NULL, NULL, J->dq + r * d, -1);
   free(Kraw);
   free(Krot);
   free(Vd);
@@ -731,6 +737,88 @@ int oracle_bwd_dq_rows(const oracle_params* p, const void* Q, const void* K, con
   J.rows = rows;
   J.dq = dq;
   run_parallel(bwd_rows_one, &J, n, nthreads);
+  return OR_OK;
+}
+
+/* dK and dV of sampled keys [(b, g, j)] (kv head g) alone: key j's terms of
+ * oracle_bwd's key-side sums, taken over every row of every query head of
+ * the group in the same order (head ascending, then row ascending), so each
+ * result equals oracle_bwd's dK / dV at that key bit for bit.  For sizes
+ * where the full backward is too slow.  dk, dv [n, d] in double. */
+typedef struct {
+  const oracle_params* p;
+  const void *Q, *K, *V, *dO;
+  const uint8_t* is_sep;
+  const int32_t* forced;
+  const int64_t* keys;
+  double *dk, *dv;
+} bwd_keys_job;
+
+static void bwd_keys_one(void* arg, int64_t r) {
+  bwd_keys_job* J = (bwd_keys_job*)arg;
+  const oracle_params* p = J->p;
+  int T = p->T, d = p->d;
+  int b = (int)J->keys[3 * r], g = (int)J->keys[3 * r + 1], j = (int)J->keys[3 * r + 2];
+  double* Kraw = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Krot = (double*)malloc(sizeof(double) * (size_t)T * d);
+  double* Vd = (double*)malloc(sizeof(double) * (size_t)T * d);
+  uint8_t* m = (uint8_t*)malloc((size_t)T);
+  double* P = (double*)malloc(sizeof(double) * (size_t)T);
+  double* dP = (double*)malloc(sizeof(double) * (size_t)T);
+  cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T + 1));
+  double* work = (double*)malloc(sizeof(double) * 8 * (size_t)d);
+  double* acc = (double*)calloc(3 * (size_t)d, sizeof(double));
+  double *gkr = acc, *gkc = acc + d, *gv = acc + 2 * d;
+  double* tmp = work + 7 * d;
+  head_ctx hc;
+  hc.p = p;
+  hc.Kraw = Kraw;
+  hc.Krot = Krot;
+  hc.Vd = Vd;
+  hc.sep = J->is_sep ? J->is_sep + (size_t)b * T : NULL;
+  load_head(p, J->K, J->V, b, g, Kraw, Krot, Vd);
+  int rep = p->Hq / p->Hkv;
+  for (int h = g * rep; h < (g + 1) * rep; ++h)
+    for (int i = j; i < T; ++i) /* a row i < j never keeps key j (causal) */
+      bwd_row(&hc, J->Q, J->dO, J->forced, b, h, i, work, m, P, dP, cands, gkr, gkc, gv, NULL, j);
+  oracle_rope(gkr, d, -rot_pos(p, (double)j), p->rope_theta, tmp);
+  for (int c = 0; c < d; ++c) {
+    J->dk[r * d + c] = tmp[c] + gkc[c];
+    J->dv[r * d + c] = gv[c];
+  }
+  free(Kraw);
+  free(Krot);
+  free(Vd);
+  free(m);
+  free(P);
+  free(dP);
+  free(cands);
+  free(work);
+  free(acc);
+}
+
+int oracle_bwd_dkv_keys(const oracle_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                        const int32_t* forced, const void* dO, int64_t n, const int64_t* keys, double* dk, double* dv,
+                        int nthreads) {
+  if (!p || p->d <= 0 || (p->d & 1) || p->T <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv || n < 0 ||
+      (n > 0 && !keys))
+    return OR_ERR_ARG;
+  for (int64_t r = 0; r < n; ++r)
+    if (keys[3 * r] < 0 || keys[3 * r] >= p->B || keys[3 * r + 1] < 0 || keys[3 * r + 1] >= p->Hkv ||
+        keys[3 * r + 2] < 0 || keys[3 * r + 2] >= p->T)
+      return OR_ERR_ARG;
+  bwd_keys_job J;
+  J.p = p;
+  J.Q = Q;
+  J.K = K;
+  J.V = V;
+  J.dO = dO;
+  J.is_sep = is_sep;
+  J.forced = forced;
+  J.keys = keys;
+  J.dk = dk;
+  J.dv = dv;
+  run_parallel(bwd_keys_one, &J, n, nthreads);
   return OR_OK;
 }
 

@@ -174,3 +174,29 @@ def test_dq_rows_entry_equals_full_backward(oracle_mod, cfg):
     assert np.array_equal(dq, dQ[rows[:, 0], rows[:, 1], rows[:, 2]])
     with pytest.raises(RuntimeError):
         O.bwd_dq_rows(p, q, k, v, sep, dO, np.array([(0, 0, T)]))
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(dtype="f32", n_start=2, window=4, L_pretrain=6, topk=3, rope_theta=1e2),   # capped, separators, top-k
+    dict(dtype="f32", n_start=1, window=5, L_pretrain=5, topk=0, alibi=True),       # clipped ALiBi
+    dict(dtype="f32", n_start=3, window=3, L_pretrain=3, topk=0, rope_theta=1e2, rope_pos_scale=0.5),
+])
+def test_dkv_keys_entry_equals_full_backward(oracle_mod, cfg):
+    """oracle_bwd_dkv_keys (the keys-only entry used at full sizes) takes the
+    same key-side sums as the pinned full backward, in the same order: equal
+    bits for sinks, separators, window and top-k keys, every kv head."""
+    O = oracle_mod
+    B, Hq, Hkv, T, d = 2, 4, 2, 40, 8
+    q, k, v, dO = _grid_inputs(B, Hq, Hkv, T, d, 13)
+    rng = np.random.default_rng(14)
+    sep = (rng.random((B, T)) < 0.3).astype(np.uint8)
+    p = O.params(B, Hq, Hkv, T, d, **cfg)
+    forced = _forced_of(O, p, q, k, v, sep) if p.topk else None
+    _, dK, dV = O.bwd(p, q, k, v, sep, dO, forced_topk=forced, nthreads=2)
+    keys = np.array([(b, g, j) for b in range(B) for g in range(Hkv) for j in (0, 1, 2, 5, 9, 17, 30, T - 1)])
+    dk, dv = O.bwd_dkv_keys(p, q, k, v, sep, dO, keys, forced_topk=forced, nthreads=2)
+    assert np.array_equal(dk, dK[keys[:, 0], keys[:, 1], keys[:, 2]])
+    assert np.array_equal(dv, dV[keys[:, 0], keys[:, 1], keys[:, 2]])
+    assert np.abs(dk).max() > 1e-3 and np.abs(dv).max() > 1e-3
+    with pytest.raises(RuntimeError):
+        O.bwd_dkv_keys(p, q, k, v, sep, dO, np.array([(0, Hkv, 0)]))

@@ -335,6 +335,58 @@ def test_cap_beyond_sequence_is_uncapped(oracle_mod):
     assert np.array_equal(a[0], b[0])
 
 
+@pytest.mark.parametrize("ns,w,L,kk", [(4, 6, 6, 0), (4, 6, 6, 2), (3, 4, 10, 2), (2, 5, 9, 0), (40, 3, 3, 1)])
+def test_capped_rope_forward_against_distance_capped_logits(oracle_mod, ns, w, L, kk):
+    """The capped-RoPE forward as a whole ("LM-Infinite", section 方法: the
+    distance d_ij = i - j is capped to d'_ij = min(d_ij, L) and the rotary
+    logit is taken at that distance).  The reference builds every kept
+    logit in the test as <R(j + d'_ij) q_i, R(j) k_j> -- the query rotated
+    to the key's position plus the capped distance, not the oracle's
+    <R(L) q_i, k_j> form -- and takes a plain fp64 softmax over the mask
+    rows plus forced top-k keys.  Sinks scaled x8, separators, windows equal
+    to and below the cap (so separators and top-k keys fall both inside and
+    past the cap), a sink span wider than the window."""
+    O = oracle_mod
+    B, Hq, Hkv, T, d, theta = 1, 2, 1, 48, 16, 1e4
+    q, k, v = _rand_inputs(B, Hq, Hkv, T, d, 31, "f32")
+    k = k.copy()
+    k[:, :, :4] *= 8.0
+    rng = np.random.default_rng(32)
+    sep = (rng.random((B, T)) < 0.2).astype(np.uint8)
+    forced = np.full((B, Hq, T, max(kk, 1)), -1, dtype=np.int32)
+    for h in range(Hq):
+        for i in range(T):
+            cand = [j for j in range(ns, i - w) if not sep[0, j]]
+            if kk and cand:
+                pick = rng.choice(cand, size=min(kk, len(cand)), replace=False)
+                forced[0, h, i, :len(pick)] = pick
+    p = O.params(B, Hq, Hkv, T, d, "f32", ns, w, L, kk, theta)
+    rows = O.all_rows(B, Hq, T)
+    got, lse, *_ = O.fwd_rows(p, q, k, v, sep, rows, forced_topk=forced[..., :kk] if kk else None)
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    n_capped = 0
+    for r, (b, h, i) in enumerate(rows):
+        g = h * Hkv // Hq
+        m, _ = O.mask_row(T, i, ns, w, sep[b])
+        for j in forced[b, h, i, :kk]:
+            if j >= 0:
+                m[j] = 1
+        js = np.flatnonzero(m)
+        z = np.empty(len(js))
+        for x, j in enumerate(js):
+            dd = min(i - j, L)
+            n_capped += (i - j) > L
+            z[x] = np.dot(O.rope(q64[b, h, i], j + dd, theta), O.rope(k64[b, g, j], j, theta))
+        s = z / math.sqrt(d)
+        mx = s.max()
+        wts = np.exp(s - mx)
+        ref_lse = mx + math.log(wts.sum())
+        ref_o = (np.exp(s - ref_lse)[:, None] * v64[b, g, js]).sum(0)
+        assert abs(lse[r] - ref_lse) < 1e-12
+        assert np.abs(got[r] - ref_o).max() < 1e-12
+    assert n_capped > 100  # the cap is exercised
+
+
 # ----------------------------------------------------------------------------
 # top-k middle tokens
 # ----------------------------------------------------------------------------
