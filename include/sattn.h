@@ -333,7 +333,10 @@ int sattn_stream_status(void* stream, const void* ws, int32_t* device_status);
  *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
  *  - All calls share the array, which keeps the last call's contents (no part
  *    of it needs to start at zero).  Calls that overlap on the GPU -- other
- *    streams, other host threads -- race on it: serialise them. */
+ *    streams, other host threads -- race on it: serialise them.
+ *  - The looked-up address is kept for the life of the process; a
+ *    cudaDeviceReset destroys the array with its context, so do not call
+ *    this entry point again after resetting the device. */
 int sattn_build_blockmap_noalloc(const sattn_params* p, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
                                  int32_t* sep_count, int32_t* qtile_sep_range, void* stream);
 

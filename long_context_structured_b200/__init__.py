@@ -9,6 +9,7 @@ Public calls (names follow the C ABI):
     fwd(q, k, v, ...)            -> (O, lse)
     topk_select(q, k, ...)       -> (idx, logit)
     build_blockmap(is_sep, ...)  -> dict(cls, sep_pos, sep_count, qtile_sep_range)
+    build_blockmap_noalloc(...)  -> the same, scratch inside the library (no workspace)
     segment_fwd(q, k, v, ...)    -> (O, lse, prefix_blocks)
     stream_status(workspace)     -> device status code
 
@@ -26,7 +27,7 @@ import torch
 from . import _lib
 from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
 
-__all__ = ["fwd", "topk_select", "build_blockmap", "segment_fwd", "stream_status", "workspace_size",
+__all__ = ["fwd", "topk_select", "build_blockmap", "build_blockmap_noalloc", "segment_fwd", "stream_status", "workspace_size",
            "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout",
            "decode_fwd"]
 
@@ -183,6 +184,26 @@ def build_blockmap(is_sep: Optional[torch.Tensor], *, B: int, T: int, n_start: i
     rc = _lib.load().sattn_build_blockmap(ctypes.byref(p), _ptr(is_sep), _ptr(cls), _ptr(sep_pos), _ptr(sep_count),
                                           _ptr(ranges), _ptr(ws), nbytes, _stream_ptr(sep_pos.device))
     _lib.check(rc, "sattn_build_blockmap")
+    return {"cls": cls, "sep_pos": sep_pos, "sep_count": sep_count, "qtile_sep_range": ranges}
+
+
+def build_blockmap_noalloc(is_sep: Optional[torch.Tensor], *, B: int, T: int, n_start: int, window: int,
+                           device="cuda", with_classes: bool = True):
+    """``build_blockmap`` through ``sattn_build_blockmap_noalloc``: the library
+    keeps the scratch in its own fixed device array, so no workspace is
+    passed (the outputs are still allocated here, by the caller)."""
+    nqt = (T + TILE - 1) // TILE
+    dummy = torch.empty((B, 1, T, 64), dtype=torch.bfloat16, device=device)
+    p = params(dummy, dummy, dummy, dummy, n_start=n_start, window=window, with_separators=True)
+    if is_sep is not None:
+        is_sep = is_sep.to(torch.uint8).contiguous()
+    cls = torch.empty((B, nqt, nqt), dtype=torch.uint8, device=device) if with_classes else None
+    sep_pos = torch.empty((B, T), dtype=torch.int32, device=device)
+    sep_count = torch.empty((B,), dtype=torch.int32, device=device)
+    ranges = torch.empty((B, nqt, 2), dtype=torch.int32, device=device)
+    rc = _lib.load().sattn_build_blockmap_noalloc(ctypes.byref(p), _ptr(is_sep), _ptr(cls), _ptr(sep_pos),
+                                                  _ptr(sep_count), _ptr(ranges), _stream_ptr(sep_pos.device))
+    _lib.check(rc, "sattn_build_blockmap_noalloc")
     return {"cls": cls, "sep_pos": sep_pos, "sep_count": sep_count, "qtile_sep_range": ranges}
 
 

@@ -18,6 +18,7 @@
 
 #include "../../include/sattn.h"
 #include "kernels.cuh"
+#include "prof.cuh"
 #include "status.cuh"
 
 using namespace sattn;
@@ -214,40 +215,39 @@ std::vector<ProfRec> g_prof_recs;
 std::vector<cudaEvent_t> g_prof_pool;
 
 cudaEvent_t prof_event() {
-  if (!g_prof_pool.empty()) {
-    cudaEvent_t e = g_prof_pool.back();
-    g_prof_pool.pop_back();
-    return e;
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    if (!g_prof_pool.empty()) {
+      cudaEvent_t e = g_prof_pool.back();
+      g_prof_pool.pop_back();
+      return e;
+    }
   }
   cudaEvent_t e = nullptr;
   cudaEventCreate(&e);
   return e;
 }
 
-// Records an event pair around one launch group when instrumentation is on.
-class ProfScope {
- public:
-  ProfScope(const char* name, int kernels, cudaStream_t st) : st_(st) {
-    if (!g_prof_on) return;
-    rec_.name = name;
-    rec_.kernels = kernels;
-    rec_.a = prof_event();
-    rec_.b = prof_event();
-    active_ = rec_.a && rec_.b && cudaEventRecord(rec_.a, st_) == cudaSuccess;
-  }
-  ~ProfScope() {
-    if (!active_) return;
-    if (cudaEventRecord(rec_.b, st_) == cudaSuccess) {
-      std::lock_guard<std::mutex> g(g_prof_mu);
-      g_prof_recs.push_back(rec_);
-    }
-  }
+}  // namespace
 
- private:
-  cudaStream_t st_;
-  ProfRec rec_{};
-  bool active_ = false;
-};
+sattn::ProfScope::ProfScope(const char* name, int kernels, cudaStream_t st) : st_(st) {
+  if (!g_prof_on) return;
+  name_ = name;
+  kernels_ = kernels;
+  a_ = prof_event();
+  b_ = prof_event();
+  active_ = a_ && b_ && cudaEventRecord(a_, st_) == cudaSuccess;
+}
+
+sattn::ProfScope::~ProfScope() {
+  if (!active_) return;
+  if (cudaEventRecord(b_, st_) == cudaSuccess) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_recs.push_back(ProfRec{name_, kernels_, a_, b_});
+  }
+}
+
+namespace {
 
 #define SATTN_TRY(expr)                   \
   do {                                    \

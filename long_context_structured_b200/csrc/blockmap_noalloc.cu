@@ -22,13 +22,17 @@
 //     undefined results; serialise them;
 //   - the array keeps the previous call's contents; nothing in it has to
 //     start at zero, because the scan kernel rewrites every entry the class
-//     kernel reads before it reads it.
+//     kernel reads before it reads it;
+//   - the array's device address is looked up once per device and kept; a
+//     cudaDeviceReset destroys the array with the context, so after a reset
+//     this entry point must not be called again in the same process.
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "../../include/sattn.h"
 #include "kernels.cuh"
+#include "prof.cuh"
 
 namespace {
 
@@ -78,5 +82,7 @@ extern "C" int sattn_build_blockmap_noalloc(const sattn_params* p, const uint8_t
   a.sep_count = sep_count;
   a.ranges = qtile_sep_range;
   a.cls = cls;
-  return sattn::launch_blockmap(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  sattn::ProfScope ps("blockmap_noalloc", cls ? 2 : 1, st);  // the class kernel runs only when classes are asked for
+  return sattn::launch_blockmap(a, st) == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }

@@ -41,27 +41,69 @@ def compare(name, got, ref, max_abs, mean_abs=None):
     return mx, mn
 
 
-def topk_agreement(gpu_idx, ref_idx, ref_z_ext, k):
-    """Rows whose GPU selection differs from the oracle only where the oracle
-    has a near tie are exempt.  ref_z_ext holds k+1 oracle logits per row.
-    Returns (n_exact, n_exempt, bad_rows)."""
+# oracle picks listed beyond the k-th, so that a near-tied run at the k-th
+# position can be followed past it
+TOPK_EXT = 4
+
+
+def _near(a, b):
+    return bool(np.isfinite(a) and np.isfinite(b) and abs(a - b) <= TIE_REL * max(abs(a), abs(b), 1e-30))
+
+
+def topk_row_verdict(g, o, z, k):
+    """One row: 'exact', 'exempt' or a reason string for a mismatch.
+
+    g: the GPU's k picks; o, z: the oracle's first k + e picks (e >= 1) and
+    their fp64 logits.  A row whose set differs from the oracle's passes only
+    under the near-tie rule ("LM-Infinite", section 方法, optional top-k: the
+    k largest logits; a fp32 selector may swap keys whose logits the fp32
+    rounding cannot separate): the oracle's k-th and (k+1)-th logits are
+    within TIE_REL relative, every oracle pick clearly above the k-th logit
+    is in the GPU set, and every GPU pick is an oracle candidate whose logit
+    is within TIE_REL of the k-th.  The GPU's list must also be ordered by
+    the oracle's logits, up to swaps of near-equal pairs, and pad with -1
+    exactly where the oracle does."""
+    g = [int(x) for x in g]
+    o = [int(x) for x in o]
+    if g == o[:k]:
+        return "exact"
+    n_pad = sum(1 for x in o[:k] if x < 0)
+    real = [x for x in g if x >= 0]
+    if len(real) != k - n_pad or any(x >= 0 for x in g[k - n_pad:]):
+        return "padding differs"
+    if len(set(real)) != len(real):
+        return "repeated key"
+    zof = {o[x]: float(z[x]) for x in range(len(o)) if o[x] >= 0}
+    if any(x not in zof for x in real):
+        return "a GPU pick is not among the oracle's first %d" % len(o)
+    ref = set(x for x in o[:k] if x >= 0)
+    if set(real) != ref:
+        zk = float(z[k - 1])
+        if not (k < len(o) and _near(zk, float(z[k]))):
+            return "set differs without a near tie at the k-th logit"
+        strict = set(o[x] for x in range(k) if o[x] >= 0 and not _near(float(z[x]), zk))
+        if not strict <= set(real):
+            return "an oracle pick above the tied run is missing"
+        if any(zof[x] < zk and not _near(zof[x], zk) for x in real):
+            return "a GPU pick is below the tied run"
+    for a, b in zip(real, real[1:]):
+        if zof[a] < zof[b] and not _near(zof[a], zof[b]):
+            return "order differs beyond a near tie"
+    return "exempt"
+
+
+def topk_agreement(gpu_idx, ref_idx_ext, ref_z_ext, k):
+    """Rows of GPU selections [n, k] against the oracle's first k + e picks
+    and logits [n, k + e]; see topk_row_verdict.  Returns (n_exact, n_exempt,
+    bad) with bad a list of (row, reason)."""
     n_exact = n_exempt = 0
     bad = []
     for r in range(gpu_idx.shape[0]):
-        g = list(gpu_idx[r])
-        o = list(ref_idx[r])
-        if g == o:
+        v = topk_row_verdict(gpu_idx[r], ref_idx_ext[r], ref_z_ext[r], k)
+        if v == "exact":
             n_exact += 1
-            continue
-        z = ref_z_ext[r]
-        # a near tie anywhere among the first k+1 oracle logits can reorder or swap
-        tie = False
-        for x in range(k):
-            a, b = z[x], z[x + 1]
-            if np.isfinite(a) and np.isfinite(b) and abs(a - b) <= TIE_REL * max(abs(a), abs(b), 1e-30):
-                tie = True
-        if tie and sorted(set(g) - {-1}) is not None:
+        elif v == "exempt":
             n_exempt += 1
         else:
-            bad.append(r)
+            bad.append((r, v))
     return n_exact, n_exempt, bad

@@ -85,6 +85,12 @@ def test_bwd_f32(oracle_mod, name, cfg):
     _run(oracle_mod, wl, 21, F32_GRAD_REL)
 
 
+def test_bwd_f32_sinks40(oracle_mod):
+    wl = synth.Workload(name="f32_sinks40", B=1, Hq=2, Hkv=1, T=300, d=64, dtype="f32", n_start=40, window=20,
+                        L_pretrain=20, rope_theta=1e4, sep_rate=0.1, sink_scale=8.0)
+    _run(oracle_mod, wl, 22, F32_GRAD_REL)
+
+
 def test_bwd_f32_sepllm_config(oracle_mod):
     """The fp32 SepLLM-mask layer (T=1024, d=64, separators at rate 0.08)."""
     _run(oracle_mod, synth.WORKLOADS["c1_f32_sep"], 0, F32_GRAD_REL)
@@ -113,6 +119,13 @@ BF16_CASES = [
                             rope_pos_scale=0.5)),
     ("window0_all_seps", dict(B=1, Hq=2, Hkv=2, T=257, d=128, n_start=1, window=0, sep_rate=1.0)),
     ("tiny", dict(B=1, Hq=1, Hkv=1, T=5, d=128, n_start=4, window=2, rope_theta=1e4)),
+    # sink spans wider than 16: the sink keys staged in several passes
+    ("sinks12_capped_gqa", dict(B=1, Hq=4, Hkv=2, T=600, d=128, n_start=12, window=64, L_pretrain=64,
+                                rope_theta=1e4, sink_scale=8.0)),
+    ("sinks40_sep_capped", dict(B=1, Hq=2, Hkv=2, T=700, d=128, n_start=40, window=64, L_pretrain=64,
+                                rope_theta=1e4, sep_rate=0.1, sink_scale=8.0)),
+    ("sinks40_d64_uncapped", dict(B=1, Hq=2, Hkv=1, T=500, d=64, n_start=40, window=30, rope_theta=5e5,
+                                  sep_rate=0.1)),
 ]
 
 
@@ -138,14 +151,35 @@ def test_bwd_rejects_missing_topk_selection():
         sa.bwd(q, q, q, q, lse, q, window=4, L_pretrain=4, topk=2)
 
 
+def _sample_keys(wl, flags, rng):
+    """Keys (b, kv head, j) of every kind the layer has: a sink, the first
+    non-sink key, tile and window edges, the last key, separators early and
+    late, and random keys."""
+    keys = []
+    js = [0, wl.n_start, 127, 128, wl.window, wl.window + 1, wl.T // 2, wl.T - 129, wl.T - 1]
+    js += [int(x) for x in rng.integers(wl.n_start, wl.T, 6)]
+    for x, j in enumerate(js):
+        keys.append((x % wl.B, x % wl.Hkv, j))
+    if flags is not None:
+        for b in sorted({0, wl.B - 1}):
+            sp = np.flatnonzero(flags[b][wl.n_start:]) + wl.n_start
+            for x, j in enumerate((sp[0], sp[len(sp) // 2], sp[-1])):
+                keys.append((b, (x + b) % wl.Hkv, int(j)))
+    keys.append((wl.B - 1, wl.Hkv - 1, int(rng.integers(wl.n_start, wl.T))))
+    return np.array(keys, dtype=np.int64)
+
+
 @pytest.mark.parametrize("name", ["c2_lminf_16k", "c3_sepllm_gqa_8k"])
 def test_bwd_full_size_sampled(oracle_mod, name):
     """The backward at the benchmark's full sizes (the launch the backward
-    workloads time): dQ on sampled rows against the oracle's rows entry, and
-    for every kv head the sum of dV over keys against its group's sum of dO
-    over rows (every row's weights sum to one), within 2^-7 of sum |dV|: the
-    rounding of each dV element to bf16 (2^-9) and the error of P recomputed
-    from bf16 operands."""
+    workloads time), element by element on samples: dQ of sampled rows
+    against the oracle's rows entry, dK and dV of sampled keys (sinks,
+    separators, window and tile edges) against its keys entry -- each the
+    same arithmetic as the full oracle backward, pinned equal to it bit for
+    bit.  Bars relative to each group's largest gradient (sink keys, whose
+    sums run over every row, separately).  Plus, for every kv head, the sum
+    of dV over keys against its group's sum of dO over rows (every row's
+    weights sum to one), within 2^-7 of sum |dV|."""
     wl = synth.WORKLOADS[name]
     inp = synth.make_inputs(wl, seed=0)
     q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
@@ -157,14 +191,25 @@ def test_bwd_full_size_sampled(oracle_mod, name):
     dq, dk, dv = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, **_kw(wl))
     torch.cuda.synchronize()
     assert sa.stream_status() == 0
+    p = oracle_mod.params_of(wl)
     rng = np.random.default_rng(1)
     n = 48
     rows = np.stack([rng.integers(0, wl.B, n), rng.integers(0, wl.Hq, n), rng.integers(0, wl.T, n)], axis=1)
     rows[:4, 2] = [0, 1, wl.T // 2, wl.T - 1]
-    ref = oracle_mod.bwd_dq_rows(oracle_mod.params_of(wl), inp["q"], inp["k"], inp["v"], inp["is_sep"], dO_h, rows)
+    ref = oracle_mod.bwd_dq_rows(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], dO_h, rows)
     ri = torch.as_tensor(rows, device=dq.device)
     got = dq[ri[:, 0], ri[:, 1], ri[:, 2]].float().cpu().numpy().astype(np.float64)
     compare_grad("dQ rows", got, ref, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
+    keys = _sample_keys(wl, inp["is_sep"], np.random.default_rng(2))
+    rdk, rdv = oracle_mod.bwd_dkv_keys(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], dO_h, keys)
+    ki = torch.as_tensor(keys, device=dk.device)
+    gdk = dk[ki[:, 0], ki[:, 1], ki[:, 2]].float().cpu().numpy().astype(np.float64)
+    gdv = dv[ki[:, 0], ki[:, 1], ki[:, 2]].float().cpu().numpy().astype(np.float64)
+    sink = keys[:, 2] < wl.n_start
+    for part, sel in (("sink keys", sink), ("other keys", ~sink)):
+        if sel.any():
+            compare_grad("dK " + part, gdk[sel], rdk[sel], BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
+            compare_grad("dV " + part, gdv[sel], rdv[sel], BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
     rep = wl.Hq // wl.Hkv
     dv64 = dv.double()
     lhs = dv64.sum(dim=2)

@@ -59,6 +59,13 @@ CASES = [
                                      alibi=True)),
     ("sep_capped_gqa2_d64", dict(B=2, Hq=4, Hkv=2, T=1500, d=64, n_start=4, window=80, L_pretrain=80,
                                  rope_theta=1e4, sep_rate=0.15)),
+    # sink spans wider than 8
+    ("sinks12_capped", dict(B=1, Hq=4, Hkv=2, T=1000, d=128, n_start=12, window=100, L_pretrain=100,
+                            rope_theta=1e4, sink_scale=8.0)),
+    ("sinks40_sep_capped_gqa8", dict(B=2, Hq=8, Hkv=1, T=900, d=128, n_start=40, window=64, L_pretrain=64,
+                                     rope_theta=1e4, sep_rate=0.1)),
+    ("sinks256_d64", dict(B=1, Hq=2, Hkv=2, T=700, d=64, n_start=256, window=30, rope_theta=5e5,
+                          sep_rate=0.05)),
 ]
 
 

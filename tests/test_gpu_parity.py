@@ -3,8 +3,9 @@ the same seeded inputs.
 
 Bars: block maps, separator lists, top-k selections and retrieved prefix
 blocks bit-exact (top-k / retrieval rows exempt only where the oracle's k-th
-and (k+1)-th logits are within 1e-4 relative); O and LSE within max-abs 2e-2
-and mean-abs 2e-3 for bf16 inputs, 1e-4 for the fp32 path.
+and (k+1)-th logits are within 1e-4 relative, and then only inside that tied
+run: ``_util.topk_row_verdict``); O and LSE within max-abs 2e-2 and mean-abs
+2e-3 for bf16 inputs, 1e-4 for the fp32 path.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,8 @@ import torch
 
 import long_context_structured_b200 as sa
 from long_context_structured_b200 import _lib, synth
-from _util import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, compare, gather_rows, to_dev, topk_agreement)
+from _util import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, TOPK_EXT, compare, gather_rows, to_dev,
+                   topk_agreement)
 
 pytestmark = pytest.mark.gpu
 
@@ -106,6 +108,68 @@ def test_blockmap_c3_token_flags(oracle_mod):
     assert np.array_equal(out["cls"].cpu().numpy(), cls)
 
 
+def _tile_class_bruteforce(oracle_mod, T, ns, w, flags, t, u):
+    """Class of tile (t, u) from the oracle's materialised mask rows."""
+    i0, i1 = t * 128, min(T, t * 128 + 128)
+    j0, j1 = u * 128, min(T, u * 128 + 128)
+    kept = np.stack([oracle_mod.mask_row(T, i, ns, w, flags)[0][j0:j1] for i in range(i0, i1)])
+    return 2 if kept.all() else (1 if kept.any() else 0)
+
+
+@pytest.mark.parametrize("noalloc", [False, True], ids=["workspace", "noalloc"])
+def test_blockmap_long_row_properties(oracle_mod, noalloc):
+    """One sequence of 400,003 flags: the separator word prefix (8 bytes per
+    32 positions, 100 KB) no longer fits the scan kernel's shared-memory
+    stage, so it is read from global memory.  The brute-force block map is
+    quadratic in T, so the check is by properties: separator positions
+    against numpy's nonzero, counts, per-tile ranges against prefix counts,
+    and sampled tiles (sink, diagonal, band edge, far) against the oracle's
+    mask rows."""
+    B, T, ns, w = 1, 400003, 4, 128
+    rng = np.random.default_rng(400003)
+    flags = (rng.random((B, T)) < 0.08).astype(np.uint8)
+    if noalloc:
+        out = sa.build_blockmap_noalloc(to_dev(flags), B=B, T=T, n_start=ns, window=w)
+    else:
+        out = sa.build_blockmap(to_dev(flags), B=B, T=T, n_start=ns, window=w)
+    torch.cuda.synchronize()
+    f = flags[0]
+    ref_pos = np.flatnonzero(f[ns:]) + ns
+    cnt = int(out["sep_count"][0])
+    assert cnt == len(ref_pos)
+    pos = out["sep_pos"][0].cpu().numpy()
+    assert np.array_equal(pos[:cnt], ref_pos) and np.all(pos[cnt:] == -1)
+    nQT = -(-T // 128)
+    t = np.arange(nQT)
+    last = np.minimum(T - 1, t * 128 + 127)
+    full_end = np.searchsorted(ref_pos, t * 128 - w, side="left")
+    end = np.searchsorted(ref_pos, last - w, side="left")
+    rng_ = out["qtile_sep_range"][0].cpu().numpy()
+    assert np.array_equal(rng_[:, 0], full_end) and np.array_equal(rng_[:, 1], end)
+    cls = out["cls"][0].cpu().numpy()
+    assert cls.shape == (nQT, nQT)
+    assert np.all(np.triu(cls, 1) == 0)  # above the diagonal nothing is kept
+    srng = np.random.default_rng(5)
+    tiles = []
+    for tq in [0, 1, 2, 1000, nQT // 2, nQT - 2, nQT - 1] + list(srng.integers(3, nQT, 4)):
+        for u in {0, tq, tq - 1, tq - 2, int(srng.integers(0, max(1, tq - 2)))}:
+            if 0 <= u <= tq:
+                tiles.append((int(tq), int(u)))
+    for tq, u in tiles:
+        assert cls[tq, u] == _tile_class_bruteforce(oracle_mod, T, ns, w, f, tq, u), (tq, u)
+
+
+def test_fwd_long_row_separators_sampled(oracle_mod):
+    """The forward on a 400,003-token SepLLM-mask sequence (about 32K
+    separators, word prefix in global memory), sampled rows."""
+    wl = synth.Workload(name="long_row", B=1, Hq=1, Hkv=1, T=400003, d=128, dtype="bf16", n_start=4,
+                        window=128, rope_theta=5e5, sep_rate=0.08)
+    inp = synth.make_inputs(wl, seed=2)
+    O, lse = _run_fwd(wl, inp)
+    rows = synth.sample_rows(wl, 24, seed=6)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows)
+
+
 # ---------------------------------------------------------------------------
 # fp32 path
 # ---------------------------------------------------------------------------
@@ -165,6 +229,18 @@ SMALL = [
                                     sink_scale=8.0, alibi=True)),
     ("alibi_sep_capped_even", dict(B=1, Hq=2, Hkv=1, T=1024, d=128, n_start=4, window=128, L_pretrain=128,
                                    sep_rate=0.1, alibi=True)),
+    # sink spans wider than 8: the 16-slot sink logits (9..16) and the
+    # global-memory ones (> 16) in prep and in the attention epilogue
+    ("sinks12_capped", dict(B=1, Hq=2, Hkv=1, T=1000, d=128, n_start=12, window=100, L_pretrain=100,
+                            rope_theta=1e4, sink_scale=8.0)),
+    ("sinks16_sep_d64", dict(B=2, Hq=4, Hkv=2, T=700, d=64, n_start=16, window=40, rope_theta=5e5,
+                             sep_rate=0.1)),
+    ("sinks40_sep_capped", dict(B=1, Hq=2, Hkv=2, T=900, d=128, n_start=40, window=64, L_pretrain=64,
+                                rope_theta=1e4, sep_rate=0.1, sink_scale=8.0)),
+    ("sinks200_capped_d64", dict(B=1, Hq=2, Hkv=1, T=700, d=64, n_start=200, window=64, L_pretrain=64,
+                                 rope_theta=1e4)),
+    ("sinks256_uncapped", dict(B=1, Hq=1, Hkv=1, T=600, d=128, n_start=256, window=30, rope_theta=1e4,
+                               sep_rate=0.05)),
 ]
 
 
@@ -186,11 +262,11 @@ def test_bf16_topk_small(oracle_mod):
     torch.cuda.synchronize()
     _status_ok()
     rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
-    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + 1))
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + TOPK_EXT))
     _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], None, rows)
     gi = idx.cpu().numpy().reshape(-1, wl.topk)
-    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
-    assert not bad, "rows %s differ without a near tie" % bad[:10]
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx, ref_z, wl.topk)
+    assert not bad, "rows differ beyond the near-tie rule: %s" % bad[:10]
     # logits of agreeing rows match the oracle's in fp32
     gz = z.cpu().numpy().reshape(-1, wl.topk).astype(np.float64)
     same = np.all(gi == ref_idx[:, : wl.topk], axis=1)
@@ -213,11 +289,61 @@ def test_bf16_topk_alibi(oracle_mod):
     torch.cuda.synchronize()
     _status_ok()
     rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
-    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(oracle_mod.params_of(wl.scaled(topk=wl.topk + 1)), inp["q"],
-                                                  inp["k"], inp["v"], None, rows)
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(oracle_mod.params_of(wl.scaled(topk=wl.topk + TOPK_EXT)),
+                                                  inp["q"], inp["k"], inp["v"], None, rows)
     gi = idx.cpu().numpy().reshape(-1, wl.topk)
-    _, _, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
-    assert not bad, "rows %s differ without a near tie" % bad[:10]
+    _, _, bad = topk_agreement(gi, ref_idx, ref_z, wl.topk)
+    assert not bad, "rows differ beyond the near-tie rule: %s" % bad[:10]
+    O, lse = _run_fwd(wl, inp)
+    _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi)
+
+
+TOPK_CASES = [
+    # LM-Infinite top-k together with SepLLM separators (candidates exclude
+    # the separators the mask already keeps), the capped rule with w = L
+    ("topk_separators", dict(B=1, Hq=4, Hkv=2, T=4096, d=128, n_start=4, window=512, L_pretrain=512,
+                             rope_theta=1e4, topk=5, plant=4, sep_rate=0.1)),
+    ("topk_d64", dict(B=2, Hq=2, Hkv=1, T=2048, d=64, n_start=4, window=256, L_pretrain=256, rope_theta=1e4,
+                      topk=5, plant=3)),
+    ("topk_d64_separators_k8", dict(B=1, Hq=2, Hkv=2, T=1500, d=64, n_start=2, window=128, L_pretrain=128,
+                                    rope_theta=5e5, topk=8, plant=2, sep_rate=0.2)),
+    ("topk_sinks40", dict(B=1, Hq=2, Hkv=1, T=2048, d=128, n_start=40, window=256, L_pretrain=256,
+                          rope_theta=1e4, topk=4, plant=2, sink_scale=8.0)),
+    ("topk_uncapped_k16_separators", dict(B=1, Hq=2, Hkv=2, T=1200, d=128, n_start=4, window=100,
+                                          rope_theta=1e4, topk=16, sep_rate=0.05)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", TOPK_CASES, ids=[c[0] for c in TOPK_CASES])
+def test_bf16_topk_selection_unforced(oracle_mod, name, cfg):
+    """The GPU selection against the oracle's own selection on every row
+    (bit-exact up to the near-tie rule), then the forward with the selection
+    made inside the call against the oracle forced to the GPU's picks."""
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    inp = synth.make_inputs(wl, seed=17)
+    q, k = to_dev(inp["q"]), to_dev(inp["k"])
+    sep = to_dev(inp["is_sep"])
+    idx, z = sa.topk_select(q, k, topk=wl.topk, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                            rope_theta=wl.rope_theta, is_sep=sep)
+    torch.cuda.synchronize()
+    _status_ok()
+    rows = oracle_mod.all_rows(wl.B, wl.Hq, wl.T)
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + TOPK_EXT))
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows)
+    gi = idx.cpu().numpy().reshape(-1, wl.topk)
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx, ref_z, wl.topk)
+    print("%s: %d rows exact, %d exempt" % (name, n_exact, n_exempt))
+    assert not bad, "rows differ beyond the near-tie rule: %s" % bad[:10]
+    assert n_exempt <= max(2, len(rows) // 100)
+    if inp["is_sep"] is not None:  # no separator is ever picked
+        flags = inp["is_sep"]
+        b_of = rows[:, 0]
+        picked = gi >= 0
+        assert not np.any(flags[b_of[:, None].repeat(wl.topk, 1)[picked], gi[picked]])
+    gz = z.cpu().numpy().reshape(-1, wl.topk).astype(np.float64)
+    same = np.all(gi == ref_idx[:, : wl.topk], axis=1)
+    fin = np.isfinite(ref_z[same, : wl.topk])
+    assert np.allclose(gz[same][fin], ref_z[same, : wl.topk][fin], rtol=1e-5, atol=1e-4)
     O, lse = _run_fwd(wl, inp)
     _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi)
 
@@ -336,11 +462,11 @@ def test_c4_topk_full_size_sampled(oracle_mod):
     _status_ok()
     planted_rows = [(b, h, s + x) for (b, h, j, s) in inp["meta"]["planted"][::16] for x in (0, 31)]
     rows = synth.sample_rows(wl, 6, seed=3, extra=planted_rows)
-    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + 1))
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + TOPK_EXT))
     _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], None, rows)
     gi = gather_rows(idx, rows).astype(np.int64)
-    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx[:, : wl.topk], ref_z, wl.topk)
-    assert not bad, "rows %s differ without a near tie" % [tuple(rows[r]) for r in bad[:10]]
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx, ref_z, wl.topk)
+    assert not bad, "rows differ beyond the near-tie rule: %s" % [(tuple(rows[r]), v) for r, v in bad[:10]]
     O, lse = _run_fwd(wl, inp)
     _check_fwd_rows(oracle_mod, wl, inp, O, lse, rows, forced=gi.astype(np.int32))
 

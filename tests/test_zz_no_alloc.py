@@ -84,6 +84,27 @@ def test_noalloc_matches_workspace_version_twice():
     _run_both(lib, 3, 1000, 2, 37, flags2, dev)
 
 
+@pytest.mark.parametrize("T,window", [(40000, 128), (4096, 5000)])
+def test_noalloc_largest_accepted_batch(T, window):
+    """The largest batch whose scratch fits the 4 MiB array runs and matches
+    the workspace version; one sequence more is refused on the host."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lib = _lib.load()
+    B = 1
+    while _scratch_bytes(B + 1, T, window) <= MAX_BYTES:
+        B += 1
+    rng = np.random.default_rng(T + window)
+    flags = (rng.random((B, T)) < 0.1).astype(np.uint8)
+    _run_both(lib, B, T, 4, window, flags, dev)
+    p = _params(B + 1, T, 4, window)
+    fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check fails first
+    assert lib.sattn_build_blockmap_noalloc(ctypes.byref(p), None, None, fake, fake, fake, None) == \
+        _lib.SATTN_ERR_UNSUPPORTED
+
+
 def test_noalloc_rejects_oversize_before_launch():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
