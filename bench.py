@@ -312,7 +312,7 @@ class Job:
         if self.n_sep:
             out["sep_gather"] = ("hbm", self.n_sep * wl.Hkv * 4 * wl.d * e, "B")
         if wl.topk > 0:
-            out["topk_score_rerank"] = ("tensor", 2.0 * wl.d * scored_candidates(wl), "FLOP")
+            out["topk_score"] = ("tensor", 2.0 * wl.d * scored_candidates(wl), "FLOP")
         return out
 
 
@@ -667,7 +667,7 @@ def kernel_name(wl, group):
     if group == "attn_tc_cross":
         return "attn_tc2_kernel<%d>" % TREE_WORKLOADS["tree_cross_128k"]["d"]
     d = wl.d if wl is not None else 128
-    return {"prep_rope": "prep_kernel", "topk_score_rerank": "topk_score_kernel + topk_rerank_kernel", "tree_prep": "tree_prep_kernel",
+    return {"prep_rope": "prep_kernel", "topk_score": "topk_score_kernel<%d>" % d, "topk_rerank": "topk_rerank_kernel<%d>" % d, "tree_prep": "tree_prep_kernel",
             "decode": "decode_partial_kernel + decode_combine_kernel",
             "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % d,
             "bwd_dkv": "bwd_dkv_kernel<%d>" % d, "bwd_f32": "bwd_f32_dq_kernel + bwd_f32_dkv_kernel",

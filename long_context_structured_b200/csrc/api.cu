@@ -35,10 +35,10 @@ struct Region {
 
 struct FwdPlan {
   bool bf16 = true;
-  int nQT = 0, Tpad = 0, npos = 0, n_sink = 0, short_len = 0;
+  int nQT = 0, Tpad = 0, npos = 0, n_sink = 0;
   bool need_qc = false, capped_sep = false;
   Region status, tab, qr, kr, qc, sink, kmax, prefix, sep_pos, sep_count, ranges, ks, vs, tk_idx, tk_z, fb,
-      short_idx, short_thr, n_cand;
+      cand_idx, cand_thr, cand_cnt;
   size_t total = 0;
 };
 
@@ -108,10 +108,6 @@ int plan_fwd(const sattn_params* p, FwdPlan* pl) {
   P.Tpad = P.nQT * kTile;
   P.npos = std::max(p->T, p->L_pretrain + 1);
   P.n_sink = std::min(p->n_start, p->T);
-  // shortlist of the scoring pass: wide enough that the gap between the k-th
-  // logit and the last shortlisted score almost always exceeds the bf16
-  // error bound, so that rows rarely need the exact fp32 rescan
-  P.short_len = p->topk <= 8 ? 16 : 32;
   P.capped_sep = p->L_pretrain > 0;
   P.need_qc = P.bf16 && p->L_pretrain > 0 && (p->with_separators || p->topk > 0);
   const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
@@ -140,9 +136,9 @@ int plan_fwd(const sattn_params* p, FwdPlan* pl) {
     if (P.bf16) {
       P.kmax = A.take(B * Hkv * 4);
       P.fb = A.take(B * Hq * T * 4);
-      P.short_idx = A.take(B * Hq * T * P.short_len * 4);
-      P.short_thr = A.take(B * Hq * T * 4);
-      P.n_cand = A.take(B * Hq * T * 4);
+      P.cand_idx = A.take(B * Hq * T * kCandCap * 8);
+      P.cand_thr = A.take(B * Hq * T * 4);
+      P.cand_cnt = A.take(B * Hq * T * 4);
     }
   }
   P.total = A.cur;
@@ -340,10 +336,9 @@ TopkArgs topk_args(const sattn_params* p, const FwdPlan& P, const void* Q, const
   a.z = z;
   a.fallback_rows = at<int32_t>(ws, P.fb);
   a.status = at<int32_t>(ws, P.status);
-  a.short_len = P.short_len;
-  a.short_idx = at<int32_t>(ws, P.short_idx);
-  a.short_thr = at<float>(ws, P.short_thr);
-  a.n_cand = at<int32_t>(ws, P.n_cand);
+  a.cand_idx = at<int2>(ws, P.cand_idx);
+  a.cand_thr = at<float>(ws, P.cand_thr);
+  a.cand_cnt = at<int32_t>(ws, P.cand_cnt);
   return a;
 }
 
@@ -367,8 +362,12 @@ int run_topk(const sattn_params* p, const FwdPlan& P, const void* Q, const void*
     if (!make_map(&m.ksel, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
   }
   {
-    ProfScope ps("topk_score_rerank", 2, st);
-    SATTN_TRY(launch_topk_tc(a, m, st));
+    ProfScope ps("topk_score", 1, st);
+    SATTN_TRY(launch_topk_score(a, m, st));
+  }
+  {
+    ProfScope ps("topk_rerank", 1, st);
+    SATTN_TRY(launch_topk_rerank(a, st));
   }
   ProfScope ps("topk_exact", 1, st);
   return cuda_rc(launch_topk_exact(a, false, st));

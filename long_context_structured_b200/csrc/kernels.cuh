@@ -314,18 +314,21 @@ struct TopkArgs {
   float* z;
   int32_t* fallback_rows;      // [B*Hq*T] rows whose bf16 shortlist was not certified
   int32_t* status;             // status[2] counts fallback rows
-  // shortlist from the tensor-core scoring pass
-  int short_len;               // shortlist length: 8, 16 or 32 (>= topk + 2)
-  int32_t* short_idx;          // [B*Hq*T, short_len]
-  float* short_thr;            // [B*Hq*T] coarse score of the last shortlisted key
-  int32_t* n_cand;             // [B*Hq*T] number of candidates of the row
+  // candidates from the tensor-core scoring pass: every key whose coarse
+  // score exceeds the row's threshold
+  int2* cand_idx;              // [B*Hq*T, kCandCap] (key position, coarse score bits), in key order
+  float* cand_thr;             // [B*Hq*T] the row's threshold (-inf: every candidate is listed)
+  int32_t* cand_cnt;           // [B*Hq*T] keys above the threshold (> kCandCap: the list overflowed)
 };
-constexpr int kShortlistMax = 32;
+constexpr int kCandCap = 128;
 struct TopkMaps {
   CUtensorMap qsel, ksel;      // bf16 scoring operands: (Qc, K) capped, (Qr, Kr) otherwise
 };
-// scoring + shortlist (tensor cores), then exact re-rank and certification
-cudaError_t launch_topk_tc(const TopkArgs& a, const TopkMaps& m, cudaStream_t st);
+// scoring on the tensor cores into per-row candidate lists
+cudaError_t launch_topk_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st);
+// exact re-rank of the lists and certification (uncertified rows are queued
+// for launch_topk_exact)
+cudaError_t launch_topk_rerank(const TopkArgs& a, cudaStream_t st);
 // exact fp32 scan for the rows listed in fallback_rows (count in status[2]),
 // or for every row when all_rows is set
 cudaError_t launch_topk_exact(const TopkArgs& a, bool all_rows, cudaStream_t st);

@@ -9,18 +9,21 @@
 //  1. scoring on the tensor cores: S = Qsel Ksel^T in bf16 x bf16 -> fp32
 //     (Qsel/Ksel = R(L)q / raw k when capped, R(i)q / R(j)k otherwise).  A
 //     CTA takes two 128-row query tiles; each K tile is loaded once and
-//     multiplied into both tiles' TMEM score buffers; one scan warpgroup per
-//     tile keeps, per row, a shortlist of the `short_len` best coarse scores;
-//  2. exact re-rank: a group of short_len lanes per row recomputes the
-//     shortlisted logits in fp32 from the exact inputs and certifies the
-//     result: every key left out has a coarse score <= the last shortlisted
-//     one, and the coarse score differs from the fp32 one by at most eps
-//     (operand rounding bound ||q - bf16(q)|| * max||k|| plus the
-//     accumulation bound), so if the k-th re-ranked logit exceeds that
-//     score + eps the top-k is exact;
-//  3. rows that fail the certificate (rare) are rescanned exactly in fp32
-//     over all their candidates.
+//     multiplied into both tiles' TMEM score buffers.  A sample of the key
+//     tiles is scored first and sets each row's threshold tau; then every
+//     candidate tile is scored and each key whose coarse score exceeds tau
+//     is appended to the row's candidate list (kCandCap entries);
+//  2. exact re-rank: a warp per row recomputes the listed keys' logits in
+//     fp32 from the exact inputs, takes the top k and certifies them: every
+//     key left out has a coarse score <= tau, and a coarse score differs from
+//     the fp32 logit by at most eps (operand rounding bound ||q - bf16(q)|| *
+//     max||k|| plus the accumulation bound), so the top k are exact when the
+//     k-th fp32 logit exceeds tau + eps;
+//  3. rows that fail the certificate or overflow their list (rare) are
+//     rescanned exactly in fp32 over all their candidates.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 #include <math_constants.h>
 
 #include "kernels.cuh"
@@ -32,9 +35,7 @@ namespace sattn {
 namespace {
 
 constexpr int kThreads = 320;  // 8 scan warps (two query tiles), TMA warp, MMA warp
-constexpr int kStages = 3;     // K tiles in flight
 constexpr int kSBuf = 2;       // TMEM score buffers per query tile
-constexpr int kScratchStride = 33;  // floats per scan thread's scratch row (odd: no bank conflicts)
 
 template <typename Tin>
 __device__ __forceinline__ float ld_in(const Tin* p);
@@ -75,30 +76,76 @@ __device__ __forceinline__ void list_insert(float v, int j, float (&vals)[KC], i
 }
 
 // ---------------------------------------------------------------------------
-// pass 1: tensor-core scoring with a per-row shortlist
+// pass 1: tensor-core scoring with a per-row candidate list
 // ---------------------------------------------------------------------------
-template <int D, int KC>
+// Key tiles are scored in two phases.  The sample phase scores every
+// stride-th key tile of the row's candidate range and keeps, per row, the 16
+// largest group maxima; the r-th of them becomes the row's threshold tau.
+// With a sample of 1/stride of the row, about r * stride candidates score
+// above the r-th largest 32-column chunk maximum (a Gamma(r)-distributed
+// count, scaled by the stride); the (stride, r) pairs below keep both "fewer
+// than about seven above tau" (the certificate would fail) and "more than
+// kCandCap above tau" (the list would overflow) near or below 0.03% of rows,
+// each of which then takes the exact rescan.  CTAs with few key tiles sample
+// every tile and take groups of 4 columns (the y = g mod 8 columns of a
+// 32-column chunk): the 16th largest group maximum leaves at least 15 and at
+// most 15 * 4 keys above it, so the list never overflows.  The main phase
+// scores every candidate tile in key order and appends each key above tau to
+// the row's list: per 32-column chunk a thread first takes the chunk
+// maximum, and only when some row of the warp has a chunk maximum above its
+// threshold does the warp build bit masks and append.
+constexpr int kSampleKeep = 16;  // group maxima kept per row in the sample phase
+constexpr int kStagesK = 3;      // K tiles in flight
+// floats per scan thread's scratch row: a multiple of 4 (16-byte stores) that
+// puts the eight rows of a quarter-warp on distinct bank groups
+constexpr int kScratchStride = 36;
+
+// Sample stride and rank for a CTA whose longer query tile scans `ntiles`
+// key tiles; `fine`: 4-column groups instead of 32-column chunks.
+__device__ __forceinline__ void sample_plan(int ntiles, int& stride, int& r, bool& fine) {
+  fine = false;
+  if (ntiles >= 48) { stride = 6; r = 8; }
+  else if (ntiles >= 16) { stride = 3; r = 12; }
+  else { stride = 1; r = 16; fine = true; }
+}
+
+// insert v into the descending list s (values only)
+template <int R>
+__device__ __forceinline__ void insert_val(float v, float (&s)[R]) {
+#pragma unroll
+  for (int x = 0; x < R; ++x) {
+    if (v > s[x]) {
+      const float t = s[x];
+      s[x] = v;
+      v = t;
+    }
+  }
+}
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const TopkArgs a, int nQB) {
+  constexpr int kSt = kStagesK;
+  constexpr int kR = kSampleKeep;
   constexpr uint32_t kTileBytes = D * kTile * 2;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kChunkBytes = kTile * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = base;  // Q0 | Q1
-  uint8_t* sk = base + 2 * kTileBytes;  // kStages K tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sk + kStages * kTileBytes);
+  uint8_t* sk = base + 2 * kTileBytes;  // kSt K tiles
+  float* scratch = reinterpret_cast<float*>(sk + kSt * kTileBytes);  // [256 scan threads][kScratchStride]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + 256 * kScratchStride);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + kStages;
-  uint64_t* s_full = k_empty + kStages;  // [2 tiles][kSBuf]
+  uint64_t* k_empty = k_full + kSt;
+  uint64_t* s_full = k_empty + kSt;  // [2 tiles][kSBuf]
   uint64_t* s_free = s_full + 2 * kSBuf;  // [2 tiles][kSBuf]
   uint64_t* drain = s_free + 2 * kSBuf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_i = reinterpret_cast<int*>(tmem_slot + 1);
   int* early = abort_i + 1;
-  float* scratch = reinterpret_cast<float*>(sk + kStages * kTileBytes + 1024);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = blockIdx.x % nQB;
@@ -117,12 +164,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   const int ntiles = max(nt[0], nt[1]);
+  // step sequence: the sample tiles 0, S, 2S, ... then every tile in order
+  int stride, r_tau;
+  bool fine;
+  sample_plan(ntiles, stride, r_tau, fine);
+  const int n_s = (ntiles + stride - 1) / stride;
+  const int n_steps = ntiles > 0 ? n_s + ntiles : 0;
+  auto tile_of = [&](int it) { return it < n_s ? it * stride : it - n_s; };
 
   if (threadIdx.x == 0) {
     *early = status_failed(a.status) ? 1 : 0;
     *abort_i = 0;
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
     }
@@ -147,42 +201,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ===== TMA producer: both query tiles once, then the K ring =====
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0 && n_steps > 0) {
       mbar_expect_tx(q_full, 2 * kTileBytes);
       for (int x = 0; x < 2; ++x)
         for (int c = 0; c < kChunks; ++c)
           tma_load_4d(sq + x * kTileBytes + c * kChunkBytes, &tmQ, q_full, c * 64, (2 * qb + x) * kTile, h, b);
       int issued = 0;
       bool ok = true;
-      for (int it = 0; it < ntiles; ++it) {
-        const int st = it % kStages;
-        if (it >= kStages) ok = mbar_wait(k_empty + st, ((it / kStages) - 1) & 1, abort_flag, a.status, 21);
+      for (int it = 0; it < n_steps; ++it) {
+        const int st = it % kSt;
+        if (it >= kSt) ok = mbar_wait(k_empty + st, ((it / kSt) - 1) & 1, abort_flag, a.status, 21);
         if (!ok) break;
         mbar_expect_tx(k_full + st, kTileBytes);
         for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sk + st * kTileBytes + c * kChunkBytes, &tmK, k_full + st, c * 64, (u_lo + it) * kTile, g, b);
+          tma_load_4d(sk + st * kTileBytes + c * kChunkBytes, &tmK, k_full + st, c * 64,
+                      (u_lo + tile_of(it)) * kTile, g, b);
         ++issued;
       }
       if (!ok) {
         mbar_wait_raw(q_full, 0);
-        for (int it = max(0, issued - kStages); it < issued; ++it) mbar_wait_raw(k_full + it % kStages, (it / kStages) & 1);
+        for (int it = max(0, issued - kSt); it < issued; ++it) mbar_wait_raw(k_full + it % kSt, (it / kSt) & 1);
       }
     }
   } else if (warp == 9) {
-    // ===== MMA issuer: per K tile, S_x = Q_x K^T for each query tile still scanning =====
-    if (lane == 0 && ntiles > 0) {
+    // ===== MMA issuer: per K tile, S_x = Q_x K^T for each query tile that needs it =====
+    if (lane == 0 && n_steps > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
       const uint32_t q_addr = smem_u32(sq);
       bool ok = mbar_wait(q_full, 0, abort_flag, a.status, 22);
-      for (int it = 0; it < ntiles && ok; ++it) {
-        const int st = it % kStages;
-        const int sb = it % kSBuf;
-        ok = mbar_wait(k_full + st, (it / kStages) & 1, abort_flag, a.status, 23);
+      int cnt[2] = {0, 0};  // score tiles produced per query tile
+      for (int it = 0; it < n_steps && ok; ++it) {
+        const int st = it % kSt;
+        ok = mbar_wait(k_full + st, (it / kSt) & 1, abort_flag, a.status, 23);
         if (!ok) break;
+        const int t = tile_of(it);
         const uint32_t k_addr = smem_u32(sk + st * kTileBytes);
         for (int x = 0; x < 2 && ok; ++x) {
-          if (it >= nt[x]) continue;
-          if (it >= kSBuf) ok = mbar_wait(s_free + x * kSBuf + sb, ((it / kSBuf) - 1) & 1, abort_flag, a.status, 24);
+          if (t >= nt[x]) continue;
+          const int c = cnt[x]++;
+          const int sb = c % kSBuf;
+          if (c >= kSBuf) ok = mbar_wait(s_free + x * kSBuf + sb, ((c / kSBuf) - 1) & 1, abort_flag, a.status, 24);
           if (!ok) break;
           tc_fence_after();
           const uint32_t qx = q_addr + x * kTileBytes;
@@ -211,24 +269,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     // candidates of this row: n_start <= j <= i - w - 1; of the warp's rows,
     // the smallest upper bound decides which tiles need no per-column mask
-    const int j_hi = i - a.window - 1;
-    float* my_scratch = scratch + threadIdx.x * kScratchStride;
-    const int warp_j_hi = i0 + (warp & 3) * 32 - a.window - 1;
-    float vals[KC];
-    int idxs[KC];
+    // (rows past the sequence end keep nothing)
+    const int j_hi = i < a.T ? i - a.window - 1 : -1;
+    const int warp_j_hi = (i0 + (warp & 3) * 32 + 31 < a.T) ? i0 + (warp & 3) * 32 - a.window - 1 : -1;
+    const size_t row = ((size_t)b * a.Hq + h) * a.T + (i < a.T ? i : a.T - 1);
+    int2* list = a.cand_idx + row * kCandCap;
+    float* my_scratch = scratch + (threadIdx.x & 255) * kScratchStride;
+    float samp[kR];
 #pragma unroll
-    for (int x = 0; x < KC; ++x) {
-      vals[x] = -CUDART_INF_F;
-      idxs[x] = -1;
-    }
-    int ncand = 0;
+    for (int x = 0; x < kR; ++x) samp[x] = -CUDART_INF_F;
+    float tau = -CUDART_INF_F;
+    int n = 0;  // keys above tau (list entries written: min(n, kCandCap))
+    int cx = 0; // score tiles consumed
     bool ok = true;
     const uint8_t* flags = a.is_sep ? a.is_sep + (size_t)b * a.T : nullptr;
-    for (int it = 0; it < ntx; ++it) {
-      const int sb = it % kSBuf;
-      ok = ok && mbar_wait(s_full + qt * kSBuf + sb, (it / kSBuf) & 1, abort_flag, a.status, 25);
+    for (int it = 0; it < n_steps; ++it) {
+      if (it == n_s) {  // end of the sample phase: tau = the r-th largest sampled chunk maximum
+#pragma unroll
+        for (int x = 0; x < kR; ++x)
+          if (x == r_tau - 1) tau = samp[x];
+      }
+      const int t = tile_of(it);
+      if (t >= ntx) continue;
+      const bool sample = it < n_s;
+      const int sb = cx % kSBuf;
+      ok = ok && mbar_wait(s_full + qt * kSBuf + sb, (cx / kSBuf) & 1, abort_flag, a.status, 25);
+      ++cx;
       tc_fence_after();
-      const int j0 = (u_lo + it) * kTile;
+      const int j0 = (u_lo + t) * kTile;
       const bool interior = (j0 >= a.n_start) && (j0 + kTile - 1 <= warp_j_hi);
       const int c_lo = max(0, a.n_start - j0);
       const int c_hi = min(kTile - 1, j_hi - j0);
@@ -259,18 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t vm = 0;
             if (lo <= hi) vm = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
             vm &= ~sepm;
-            ncand += __popc(vm);
 #pragma unroll
             for (int y = 0; y < 32; ++y) v[c2 * 32 + y] = ((vm >> y) & 1u) ? v[c2 * 32 + y] : -CUDART_INF_F;
           }
-        } else {
-          ncand += 64;
         }
-        // per 32-column chunk maxima (independent chains), then the insertion
-        // path only for chunks that beat the row's current threshold; such a
-        // chunk goes through this thread's shared scratch row, so one copy of
-        // the insertion code serves every column (an unrolled insertion per
-        // column would not fit the instruction cache)
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
           float pm[8];
@@ -280,29 +340,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int y = 8; y < 32; ++y) pm[y & 7] = fmaxf(pm[y & 7], v[c2 * 32 + y]);
           const float cm =
               fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-          if (cm > vals[KC - 1]) {
-            uint32_t msk = 0;
+          if (sample) {
+            if (fine) {
 #pragma unroll
-            for (int y = 0; y < 32; ++y) {
-              my_scratch[y] = v[c2 * 32 + y];
-              msk |= (v[c2 * 32 + y] > vals[KC - 1]) ? (1u << y) : 0u;
+              for (int y = 0; y < 8; ++y)
+                if (pm[y] > samp[kR - 1]) insert_val<kR>(pm[y], samp);
+            } else if (cm > samp[kR - 1]) {
+              insert_val<kR>(cm, samp);
             }
-            while (msk) {
-              const int y = __ffs(msk) - 1;
-              msk &= msk - 1;
-              const float z = my_scratch[y];
-              if (z > vals[KC - 1]) list_insert<KC>(z, j0 + hf * 64 + c2 * 32 + y, vals, idxs);
+            continue;
+          }
+          if (__any_sync(0xffffffffu, cm > tau) && cm > tau) {
+            // append this row's keys above tau with their coarse scores, in
+            // key order (the chunk goes through the thread's scratch row so
+            // that a score can be picked by a run-time column)
+            uint32_t m = 0;
+#pragma unroll
+            for (int y = 0; y < 32; ++y) m |= (v[c2 * 32 + y] > tau) ? (1u << y) : 0u;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              reinterpret_cast<float4*>(my_scratch)[q4] = make_float4(
+                  v[c2 * 32 + 4 * q4], v[c2 * 32 + 4 * q4 + 1], v[c2 * 32 + 4 * q4 + 2], v[c2 * 32 + 4 * q4 + 3]);
+            const int jbase = j0 + hf * 64 + c2 * 32;
+            while (m) {
+              const int y = __ffs(m) - 1;
+              m &= m - 1;
+              if (n < kCandCap) list[n] = make_int2(jbase + y, __float_as_int(my_scratch[y]));
+              ++n;
             }
           }
         }
       }
     }
     if (i < a.T) {
-      const size_t row = ((size_t)b * a.Hq + h) * a.T + i;
-#pragma unroll
-      for (int x = 0; x < KC; ++x) a.short_idx[row * KC + x] = idxs[x];
-      a.short_thr[row] = (ncand > KC) ? vals[KC - 1] : -CUDART_INF_F;
-      a.n_cand[row] = ncand;
+      a.cand_thr[row] = tau;
+      a.cand_cnt[row] = n;
     }
   }
 
@@ -314,141 +386,236 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// fp32 logit of key row kp (bf16, unrotated) against the staged fp32 query qv
+// (R(L) q when `capped`, else R(i) q, whose partner is the key rotated by
+// R(j) from the table); 16-byte key loads, two accumulators
+template <int HALF>
+__device__ __forceinline__ float exact_logit_bf16(const __nv_bfloat16* kp, const float* qv, bool capped,
+                                                  const float2* tab, int64_t j) {
+  float A0 = 0.f, A1 = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < HALF; c0 += 8) {
+    float k0[8], k1[8];
+    const uint4 lo = *reinterpret_cast<const uint4*>(kp + c0);
+    const uint4 hi = *reinterpret_cast<const uint4*>(kp + c0 + HALF);
+    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 p = __bfloat1622float2(l2[e]), r = __bfloat1622float2(h2[e]);
+      k0[2 * e] = p.x;
+      k0[2 * e + 1] = p.y;
+      k1[2 * e] = r.x;
+      k1[2 * e + 1] = r.y;
+    }
+    if (!capped && tab) {
+      const float4* t = reinterpret_cast<const float4*>(tab + j * HALF + c0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 cs = t[e];
+        const float a0 = k0[2 * e], a1 = k0[2 * e + 1], r0 = k1[2 * e], r1 = k1[2 * e + 1];
+        k0[2 * e] = a0 * cs.x - r0 * cs.y;
+        k1[2 * e] = r0 * cs.x + a0 * cs.y;
+        k0[2 * e + 1] = a1 * cs.z - r1 * cs.w;
+        k1[2 * e + 1] = r1 * cs.z + a1 * cs.w;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      fma2(A0, A1, qv[c0 + e], qv[c0 + e + 1], k0[e], k0[e + 1], A0, A1);
+      fma2(A0, A1, qv[HALF + c0 + e], qv[HALF + c0 + e + 1], k1[e], k1[e + 1], A0, A1);
+    }
+  }
+  return A0 + A1;
+}
+
 // ---------------------------------------------------------------------------
-// pass 2: exact re-rank of the shortlist + certificate
+// pass 2: exact re-rank of the candidate list + certificate
 // ---------------------------------------------------------------------------
-// A group of KC lanes per row (KC = shortlist length, 16 or 32): the group
-// stages the row's fp32 scoring query (R(L) q when capped, R(i) q otherwise)
-// in shared memory, lane x recomputes the fp32 logit of shortlist entry x
-// from the exact inputs (16-byte key loads), and a bitonic network over the
-// group's lanes orders the entries by (logit desc, j asc).  The certificate:
-// every key left out of the shortlist has a coarse score <= the row's
-// threshold (the last shortlisted coarse score), and a coarse score differs
-// from the fp32 logit by at most eps (query rounding ||q - bf16(q)|| * max||k||,
-// accumulation, and for rotated keys their rounding), so the top k are exact
-// when the k-th re-ranked logit exceeds threshold + eps.
-template <int D, int KC>
-__global__ void __launch_bounds__(256) topk_rerank_kernel(const TopkArgs a) {
+// A warp per row.  A coarse score c differs from the key's fp32 logit z by at
+// most eps (query rounding ||q - bf16(q)|| * max||k||, accumulation, and for
+// rotated keys their rounding).  If c' <= the k-th largest coarse score of the
+// list, at least k listed keys have z >= c' - eps, so the k-th fp32 logit
+// z_(k) >= c' - eps and only listed keys with c >= c' - 2 eps can be among the
+// top k.  c' is the k-th largest of the lanes' maxima (k distinct entries are
+// >= it).  The warp compacts the entries above the cut into shared memory,
+// recomputes their logits in fp32 from the exact inputs (four lanes per key,
+// each a quarter of the rotary pairs, 16-byte key loads; the row's fp32
+// scoring query, R(L) q when capped and R(i) q otherwise, staged in shared
+// memory), and ranks them by (logit desc, j asc) by counting.  Certificate:
+// every key left out of the list has a coarse score <= tau, hence
+// z <= tau + eps; the top k are exact when z_(k) > tau + eps (or tau = -inf:
+// the list holds every candidate).  Rows that fail, or whose list overflowed,
+// go to the exact rescan.
+constexpr int kRerankWarps = 8;
+constexpr int kPerLane = kCandCap / 32;
+
+template <int D>
+__global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const TopkArgs a) {
   constexpr int half = D / 2;
-  constexpr int RPB = 256 / KC;          // rows per block
-  constexpr int PPL = half / KC;         // rotary pairs staged per lane (2 or 4 for d=128)
-  __shared__ __align__(16) float sq[RPB][D];
-  const int grp = threadIdx.x / KC, x = threadIdx.x % KC;
-  const int lane = threadIdx.x & 31;
-  const unsigned gmask = (KC == 32) ? 0xffffffffu : (0xffffu << (lane & 16));
+  constexpr int PPL = half / 32;   // rotary pairs staged per lane
+  constexpr int QP = half / 4;     // rotary pairs per lane of a 4-lane group
+  __shared__ __align__(16) float sq[kRerankWarps][D];
+  __shared__ int sj[kRerankWarps][kCandCap];
+  __shared__ float2 se[kRerankWarps][kCandCap];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)a.B * a.Hq * a.T;
-  const int64_t row_raw = (int64_t)blockIdx.x * RPB + grp;
-  const bool live = row_raw < nrows;
-  const int64_t row = live ? row_raw : nrows - 1;  // dead groups compute a copy and write nothing
+  const int64_t row = (int64_t)blockIdx.x * kRerankWarps + wid;
+  if (row >= nrows) return;  // whole warps only: no block-wide barrier follows
   const int i = (int)(row % a.T);
   const int64_t bh = row / a.T;
   const int h = (int)(bh % a.Hq), b = (int)(bh / a.Hq);
   const int g = h / (a.Hq / a.Hkv);
   const bool capped_all = a.L > 0;  // capped scoring requires L == window: every candidate is capped
+  const int cnt = a.cand_cnt[row];
+  const float tau = a.cand_thr[row];
+  const int k = a.topk;
+  const int n = min(cnt, kCandCap);
+  const int2* list = a.cand_idx + row * kCandCap;
+  float c[kPerLane];
+  int jl[kPerLane];
+  float lm = -CUDART_INF_F;
+#pragma unroll
+  for (int x = 0; x < kPerLane; ++x) {
+    const int e = lane + 32 * x;
+    jl[x] = -1;
+    c[x] = -CUDART_INF_F;
+    if (e < n) {
+      const int2 v = list[e];
+      jl[x] = v.x;
+      c[x] = __int_as_float(v.y);
+      lm = fmaxf(lm, c[x]);
+    }
+  }
   const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(a.Q) + b * a.q_sb + h * a.q_sh +
                             (int64_t)i * a.q_st;
   // stage the scoring query and measure its bf16 rounding
   float dq2 = 0.f, qn2 = 0.f;
 #pragma unroll
   for (int e = 0; e < PPL; ++e) {
-    const int c = x * PPL + e;
-    const float x0 = __bfloat162float(qp[c]), x1 = __bfloat162float(qp[c + half]);
+    const int cc = lane * PPL + e;
+    const float x0 = __bfloat162float(qp[cc]), x1 = __bfloat162float(qp[cc + half]);
     const int64_t pos = capped_all ? a.L : i;
-    const float2 cs = a.tab ? a.tab[pos * half + c] : make_float2(1.f, 0.f);
+    const float2 cs = a.tab ? a.tab[pos * half + cc] : make_float2(1.f, 0.f);
     const float u0 = x0 * cs.x - x1 * cs.y, u1 = x1 * cs.x + x0 * cs.y;
-    sq[grp][c] = u0;
-    sq[grp][c + half] = u1;
+    sq[wid][cc] = u0;
+    sq[wid][cc + half] = u1;
     const float b0 = __bfloat162float(__float2bfloat16_rn(u0)), b1 = __bfloat162float(__float2bfloat16_rn(u1));
     dq2 += (u0 - b0) * (u0 - b0) + (u1 - b1) * (u1 - b1);
     qn2 += b0 * b0 + b1 * b1;
   }
 #pragma unroll
-  for (int o = KC / 2; o > 0; o >>= 1) {
-    dq2 += __shfl_xor_sync(gmask, dq2, o);
-    qn2 += __shfl_xor_sync(gmask, qn2, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    dq2 += __shfl_xor_sync(0xffffffffu, dq2, o);
+    qn2 += __shfl_xor_sync(0xffffffffu, qn2, o);
   }
-  __syncwarp();
   const float kmax = __uint_as_float(a.kmax[(size_t)b * a.Hkv + g]) * (1.f + 1.f / 128.f);
   const float qn = sqrtf(qn2);
   float eps = sqrtf(dq2) * kmax + qn * kmax * (1.f / 32768.f);
   if (!capped_all) eps += qn * kmax * (1.f / 256.f);  // rotated keys were rounded too
   eps *= 1.0625f;
 
-  // lane x: fp32 logit of shortlist entry x
-  const int j = a.short_idx[row * KC + x];
-  float z = -CUDART_INF_F;
-  if (j >= 0) {
-    const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(a.K) + b * a.k_sb + g * a.k_sh +
-                              (int64_t)j * a.k_st;
-    const float* qv = sq[grp];
-    float A0 = 0.f, A1 = 0.f;
+  // c' = the k-th largest lane maximum (-inf when fewer than k lanes hold entries)
+  float cp = -CUDART_INF_F;
+  {
+    float mv = lm;
+    for (int rr = 0; rr < k; ++rr) {
+      float wz = mv;
 #pragma unroll
-    for (int c0 = 0; c0 < half; c0 += 8) {
-      float k0[8], k1[8];
-      const uint4 lo = *reinterpret_cast<const uint4*>(kp + c0);
-      const uint4 hi = *reinterpret_cast<const uint4*>(kp + c0 + half);
-      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+      for (int o = 16; o > 0; o >>= 1) wz = fmaxf(wz, __shfl_xor_sync(0xffffffffu, wz, o));
+      const uint32_t holders = __ballot_sync(0xffffffffu, mv == wz);
+      if (lane == __ffs(holders) - 1) mv = -CUDART_INF_F;
+      cp = wz;
+    }
+  }
+  // compact the entries that can reach the top k
+  const float cut = cp - 2.f * eps;
+  int m = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 p = __bfloat1622float2(l2[e]), r = __bfloat1622float2(h2[e]);
-        k0[2 * e] = p.x;
-        k0[2 * e + 1] = p.y;
-        k1[2 * e] = r.x;
-        k1[2 * e + 1] = r.y;
-      }
-      if (!capped_all && a.tab) {
-        const float4* t = reinterpret_cast<const float4*>(a.tab + (int64_t)j * half + c0);
+  for (int x = 0; x < kPerLane; ++x) {
+    const bool p = jl[x] >= 0 && c[x] >= cut;
+    const uint32_t bal = __ballot_sync(0xffffffffu, p);
+    if (p) sj[wid][m + __popc(bal & ((1u << lane) - 1u))] = jl[x];
+    m += __popc(bal);
+  }
+  __syncwarp();
+  // fp32 logits: four lanes per entry, a quarter of the rotary pairs each
+  const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.K) + b * a.k_sb + g * a.k_sh;
+  const float* qv = sq[wid];
+  const int quarter = lane & 3;
+  for (int e0 = 0; e0 < m; e0 += 8) {
+    const int e = e0 + (lane >> 2);
+    float acc = 0.f;
+    int j = -1;
+    if (e < m) {
+      j = sj[wid][e];
+      const __nv_bfloat16* kp = kbase + (int64_t)j * a.k_st;
+      float A0 = 0.f, A1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 cs = t[e];
-          const float a0 = k0[2 * e], a1 = k0[2 * e + 1], r0 = k1[2 * e], r1 = k1[2 * e + 1];
-          k0[2 * e] = a0 * cs.x - r0 * cs.y;
-          k1[2 * e] = r0 * cs.x + a0 * cs.y;
-          k0[2 * e + 1] = a1 * cs.z - r1 * cs.w;
-          k1[2 * e + 1] = r1 * cs.z + a1 * cs.w;
+      for (int c0 = quarter * QP; c0 < quarter * QP + QP; c0 += 8) {
+        float k0[8], k1[8];
+        const uint4 lo = *reinterpret_cast<const uint4*>(kp + c0);
+        const uint4 hi = *reinterpret_cast<const uint4*>(kp + c0 + half);
+        const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const float2 p = __bfloat1622float2(l2[y]), r = __bfloat1622float2(h2[y]);
+          k0[2 * y] = p.x;
+          k0[2 * y + 1] = p.y;
+          k1[2 * y] = r.x;
+          k1[2 * y + 1] = r.y;
+        }
+        if (!capped_all && a.tab) {
+          const float4* t = reinterpret_cast<const float4*>(a.tab + (int64_t)j * half + c0);
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const float4 cs = t[y];
+            const float a0 = k0[2 * y], a1 = k0[2 * y + 1], r0 = k1[2 * y], r1 = k1[2 * y + 1];
+            k0[2 * y] = a0 * cs.x - r0 * cs.y;
+            k1[2 * y] = r0 * cs.x + a0 * cs.y;
+            k0[2 * y + 1] = a1 * cs.z - r1 * cs.w;
+            k1[2 * y + 1] = r1 * cs.z + a1 * cs.w;
+          }
+        }
+#pragma unroll
+        for (int y = 0; y < 8; y += 2) {
+          fma2(A0, A1, qv[c0 + y], qv[c0 + y + 1], k0[y], k0[y + 1], A0, A1);
+          fma2(A0, A1, qv[half + c0 + y], qv[half + c0 + y + 1], k1[y], k1[y + 1], A0, A1);
         }
       }
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        fma2(A0, A1, qv[c0 + e], qv[c0 + e + 1], k0[e], k0[e + 1], A0, A1);
-        fma2(A0, A1, qv[half + c0 + e], qv[half + c0 + e + 1], k1[e], k1[e + 1], A0, A1);
-      }
+      acc = A0 + A1;
     }
-    z = A0 + A1;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (e < m && quarter == 0) se[wid][e] = make_float2(acc, __int_as_float(j));
   }
-  // bitonic sort over the group's lanes: (z desc, j asc), invalid (j < 0) last
-  int jj = j;
-#pragma unroll
-  for (int k = 2; k <= KC; k <<= 1) {
-#pragma unroll
-    for (int o = k >> 1; o > 0; o >>= 1) {
-      const float oz = __shfl_xor_sync(gmask, z, o);
-      const int oj = __shfl_xor_sync(gmask, jj, o);
-      // does the partner's entry come before ours in the order?
-      const bool other_first = (oj >= 0) && (jj < 0 || oz > z || (oz == z && oj < jj));
-      const bool mine_first = (jj >= 0) && (oj < 0 || z > oz || (z == oz && jj < oj));
-      // in a run of ascending rank the lower lane of a pair keeps the earlier entry
-      const bool want_earlier = ((x & o) == 0) == ((x & k) == 0);
-      const bool take = want_earlier ? other_first : mine_first;
-      if (take) {
-        z = oz;
-        jj = oj;
-      }
+  __syncwarp();
+  // rank by counting: entry e precedes entry f when z_e > z_f, or equal with j_e < j_f
+  float zk = -CUDART_INF_F;
+  for (int e = lane; e < m; e += 32) {
+    const float2 me = se[wid][e];
+    const int mj = __float_as_int(me.y);
+    int rank = 0;
+    for (int f = 0; f < m; ++f) {
+      const float2 o = se[wid][f];
+      const int oj = __float_as_int(o.y);
+      rank += (o.x > me.x || (o.x == me.x && oj < mj)) ? 1 : 0;
     }
+    if (rank < k) {
+      a.idx[row * k + rank] = mj;
+      a.z[row * k + rank] = me.x;
+    }
+    if (rank == k - 1) zk = me.x;
   }
-  const int n = a.n_cand[row];
-  const float thr = a.short_thr[row];
-  const int k = a.topk;
-  const float zk = __shfl_sync(gmask, z, (lane & ~(KC - 1)) + k - 1);
-  const bool certified = (n <= KC) || (zk > thr + eps);
-  if (!live) return;
-  if (certified) {
-    if (x < k) {
-      a.idx[row * k + x] = (x < n) ? jj : -1;
-      a.z[row * k + x] = (x < n) ? z : -CUDART_INF_F;
-    }
-  } else if (x == 0) {
+  for (int r = m + lane; r < k; r += 32) {  // fewer than k entries: pad
+    a.idx[row * k + r] = -1;
+    a.z[row * k + r] = -CUDART_INF_F;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zk = fmaxf(zk, __shfl_xor_sync(0xffffffffu, zk, o));
+  const bool certified = cnt <= kCandCap && (tau == -CUDART_INF_F || zk > tau + eps);
+  if (!certified && lane == 0) {
     const int pos = atomicAdd(a.status + 2, 1);
     a.fallback_rows[pos] = (int32_t)row;
   }
@@ -499,22 +666,39 @@ __global__ void __launch_bounds__(kExactThreads) topk_exact_kernel(const TopkArg
     const Tin* kb = K + b * a.k_sb + g * a.k_sh;
     const uint8_t* flags = a.is_sep ? a.is_sep + (size_t)b * a.T : nullptr;
     const int jend = i - a.window;  // candidates j < i - w
-    for (int j = a.n_start + threadIdx.x; j < jend; j += blockDim.x) {
-      if (flags && flags[j]) continue;
-      const Tin* kp = kb + (int64_t)j * a.k_st;
-      const bool capped = a.L > 0 && (i - j) > a.L;
-      float acc = 0.f;
-      for (int c = 0; c < half; ++c) {
-        const float k0 = ld_in(kp + c), k1 = ld_in(kp + c + half);
-        if (capped) {
-          acc = fmaf(s_q[1][c], k0, fmaf(s_q[1][c + half], k1, acc));
-        } else {
-          const float2 cs = a.tab ? a.tab[(int64_t)j * half + c] : make_float2(1.f, 0.f);
-          acc = fmaf(s_q[0][c], k0 * cs.x - k1 * cs.y, fmaf(s_q[0][c + half], k1 * cs.x + k0 * cs.y, acc));
-        }
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+      // two keys per thread in flight, 16-byte loads
+      for (int j = a.n_start + threadIdx.x; j < jend; j += 2 * blockDim.x) {
+        const int j2 = j + blockDim.x;
+        const bool ok1 = !(flags && flags[j]);
+        const bool ok2 = j2 < jend && !(flags && flags[j2]);
+        const bool cap1 = a.L > 0 && (i - j) > a.L, cap2 = a.L > 0 && (i - j2) > a.L;
+        float z1 = -CUDART_INF_F, z2 = -CUDART_INF_F;
+        if (ok1) z1 = exact_logit_bf16<32 * PP>(kb + (int64_t)j * a.k_st, s_q[cap1 ? 1 : 0], cap1, a.tab, j);
+        if (ok2) z2 = exact_logit_bf16<32 * PP>(kb + (int64_t)j2 * a.k_st, s_q[cap2 ? 1 : 0], cap2, a.tab, j2);
+        if (ok1 && (z1 > vals[kMaxK - 1] || (z1 == vals[kMaxK - 1] && j < idxs[kMaxK - 1])))
+          list_insert<kMaxK>(z1, j, vals, idxs);
+        if (ok2 && (z2 > vals[kMaxK - 1] || (z2 == vals[kMaxK - 1] && j2 < idxs[kMaxK - 1])))
+          list_insert<kMaxK>(z2, j2, vals, idxs);
       }
-      if (acc > vals[kMaxK - 1] || (acc == vals[kMaxK - 1] && j < idxs[kMaxK - 1]))
-        list_insert<kMaxK>(acc, j, vals, idxs);
+    } else {
+      for (int j = a.n_start + threadIdx.x; j < jend; j += blockDim.x) {
+        if (flags && flags[j]) continue;
+        const Tin* kp = kb + (int64_t)j * a.k_st;
+        const bool capped = a.L > 0 && (i - j) > a.L;
+        float acc = 0.f;
+        for (int c = 0; c < half; ++c) {
+          const float k0 = ld_in(kp + c), k1 = ld_in(kp + c + half);
+          if (capped) {
+            acc = fmaf(s_q[1][c], k0, fmaf(s_q[1][c + half], k1, acc));
+          } else {
+            const float2 cs = a.tab ? a.tab[(int64_t)j * half + c] : make_float2(1.f, 0.f);
+            acc = fmaf(s_q[0][c], k0 * cs.x - k1 * cs.y, fmaf(s_q[0][c + half], k1 * cs.x + k0 * cs.y, acc));
+          }
+        }
+        if (acc > vals[kMaxK - 1] || (acc == vals[kMaxK - 1] && j < idxs[kMaxK - 1]))
+          list_insert<kMaxK>(acc, j, vals, idxs);
+      }
     }
     // k rounds of block-wide argmax over (z desc, j asc)
     int head = 0;  // next unused entry of this thread's sorted list
@@ -567,35 +751,36 @@ __global__ void __launch_bounds__(kExactThreads) topk_exact_kernel(const TopkArg
   }
 }
 
-template <int D, int KC>
+template <int D>
 cudaError_t launch_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
   const size_t tile = (size_t)D * kTile * 2;
-  // at least 116 KB: one CTA per SM, so the 512-column TMEM allocation never waits
-  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (2 + kStages) + 1024 + 256 * kScratchStride * 4);
-  cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  // Q tiles, K ring, scan scratch, barriers; at least 116 KB: one CTA per SM, so the
+  // 512-column TMEM allocation never waits
+  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (2 + kStagesK) + 256 * kScratchStride * 4 + 256);
+  cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   const int nQB = (a.nQT + 1) / 2;
-  topk_score_kernel<D, KC><<<(unsigned)(a.B * a.Hq * nQB), kThreads, bytes, st>>>(m.qsel, m.ksel, a, nQB);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int64_t rows = (int64_t)a.B * a.Hq * a.T;
-  const unsigned blocks = (unsigned)((rows * KC + 255) / 256);
-  topk_rerank_kernel<D, KC><<<blocks, 256, 0, st>>>(a);
+  topk_score_kernel<D><<<(unsigned)(a.B * a.Hq * nQB), kThreads, bytes, st>>>(m.qsel, m.ksel, a, nQB);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_topk_tc(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
+cudaError_t launch_topk_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
   if ((int64_t)a.B * a.Hq * a.T == 0) return cudaSuccess;
-  if (a.d == 128) {
-    if (a.short_len == 16) return launch_score<128, 16>(a, m, st);
-    if (a.short_len == 32) return launch_score<128, 32>(a, m, st);
-  } else if (a.d == 64) {
-    if (a.short_len == 16) return launch_score<64, 16>(a, m, st);
-    if (a.short_len == 32) return launch_score<64, 32>(a, m, st);
-  }
+  if (a.d == 128) return launch_score<128>(a, m, st);
+  if (a.d == 64) return launch_score<64>(a, m, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_topk_rerank(const TopkArgs& a, cudaStream_t st) {
+  const int64_t rows = (int64_t)a.B * a.Hq * a.T;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + kRerankWarps - 1) / kRerankWarps);
+  if (a.d == 128) topk_rerank_kernel<128><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+  else if (a.d == 64) topk_rerank_kernel<64><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_topk_exact(const TopkArgs& a, bool all_rows, cudaStream_t st) {
