@@ -3,10 +3,12 @@
 One step = one call of the whole hot path over one batch of synthetic input
 (rotary prep, block map / separator gather / top-k selection where the
 workload has them, and the tcgen05 attention kernel).  The default workload is
-the Llama-2-7B-shaped LM-Infinite layer: B=1, 32 heads, T=16384, d=128, bf16,
-n_start=4, L_pretrain=w=4096, capped RoPE theta=1e4, sink keys scaled x8.
-``--workload`` selects one of the other workloads (SepLLM GQA layer, top-k
-middle tokens, segmented execution) to measure their kernels the same way.
+the largest single-GPU configuration: the LM-Infinite layer with per-head
+top-k middle tokens, B=1, 32 heads, T=32768, d=128, bf16, n_start=4,
+L_pretrain=w=4096, capped RoPE theta=1e4, k=5 with 64 planted key/query
+clusters per head.  ``--workload`` selects one of the other workloads (the
+16K LM-Infinite layer, the SepLLM GQA layer, segmented execution, decoding,
+backward, ...) to measure their kernels the same way.
 Metric: effective TFLOP/s counted over unmasked (q, k) pairs at 4*d FLOPs
 each (whole job, all ranks), with tokens/s alongside.
 
@@ -61,16 +63,18 @@ TREE_WORKLOADS = {"tree_cross_128k": dict(B=1, Hq=32, Hkv=32, Tq=4096, d=128, n_
 BWD_FLOPS_PER_PAIR_D = 10  # backward: S recomputed, dP, dV, dK, dQ -- five products of 2d FLOPs per pair
 WORKLOAD_ALIASES = {"c2": "c2_lminf_16k", "c3": "c3_sepllm_gqa_8k", "c4": "c4_lminf_topk_32k",
                     "c5": "c5_segmented_32k"}
-DEFAULT_WORKLOAD = "c2"
+DEFAULT_WORKLOAD = "c4"
 METRIC = "effective TFLOP/s over unmasked pairs (fraction of bf16 TC peak), tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per launch of the attention kernel on the default
-# workload: dram__bytes_read.sum + dram__bytes_write.sum of an ncu capture of
-# the 8-head cut, times 4 for 32 heads (bytes scale with heads); None when
-# the kernel changed since the counters were taken.  The last capture
-# (117.6 MB x 4 = 470.3 MB) predates the kernel's separator lookup through
-# the block map's word prefix, so it is not reported.
-ATTN_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) per launch of the dominant kernel of the default
+# workload (topk_score_kernel): dram__bytes_read.sum + dram__bytes_write.sum of
+# an ncu capture of the 4-head cut, times 8 for 32 heads (the launch is a grid
+# over heads and every head reads and writes the same amount); None when the
+# kernel changed since the counters were taken.
+TOPK_SCORE_TRAFFIC_BYTES = (61026560 + 12509952) * 8
+# CPU-oracle rows per sample (about 10-30 s of host work on the GPU machine); the
+# top-k workload's oracle also scans every middle key per row
+CPU_ROWS = {"c4": 6144}
 
 
 def log(*a):
@@ -765,8 +769,8 @@ def run_ours(args):
     if dom is not None:
         roof = roofline_of(dom, work[dom], avg_ms[dom], peaks, peak_src)
         roof["kernel"] = kernel_name(wl, dom)
-        roof["traffic"] = ATTN_TRAFFIC_BYTES if (dom == "attn_tc" and args.workload == DEFAULT_WORKLOAD
-                                                 and not args.heads) else None
+        roof["traffic"] = TOPK_SCORE_TRAFFIC_BYTES if (dom == "topk_score" and args.workload == DEFAULT_WORKLOAD
+                                                       and not args.heads) else None
     gpu_launches = sum(n for n, _ in prof.values())
 
     # end to end through the public call with host buffers (H2D + D2H inside)
@@ -801,7 +805,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_bwd(wl) if backward else cpu_baseline(wl, job.inp, args.cpu_rows, decode=decode)
+        cpu = cpu_baseline_bwd(wl) if backward else cpu_baseline(wl, job.inp, cpu_rows_of(args), decode=decode)
 
     if world > 1:
         dist.barrier()
@@ -1113,6 +1117,17 @@ def _oracle_rows(O, wl, inp, rows, nthreads):
         O.fwd_rows(p, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows, nthreads=nthreads)
 
 
+def cpu_rows_of(args) -> int:
+    return args.cpu_rows if args.cpu_rows else CPU_ROWS.get(args.workload, 32768)
+
+
+def cpu_sample_rows(wl, n_rows):
+    """The CPU-oracle sample of a forward workload: seeded rows over all
+    batches, heads and positions, grouped by (batch, head)."""
+    rows = _oracle_sample(wl, n_rows, 1234)
+    return rows[np.lexsort((rows[:, 2], rows[:, 1], rows[:, 0]))]
+
+
 def cpu_baseline(wl, inp, n_rows, decode=False):
     from oracle import oracle as O
     O.build()
@@ -1120,7 +1135,7 @@ def cpu_baseline(wl, inp, n_rows, decode=False):
         base = np.array([(b, h, wl.T - 1) for b in range(wl.B) for h in range(wl.Hq)], dtype=np.int64)
         rows = np.tile(base, (max(1, n_rows // (16 * len(base))), 1))
     else:
-        rows = _oracle_sample(wl, n_rows, 1234)
+        rows = cpu_sample_rows(wl, n_rows)
     nthreads = O.nthreads_default()
     t0 = time.perf_counter()
     _oracle_rows(O, wl, inp, rows, nthreads)
@@ -1196,14 +1211,18 @@ def run_reference(args):
     wl = synth.WORKLOADS[(DECODE_ALIASES if decode else WORKLOAD_ALIASES).get(args.workload, args.workload)]
     inp = synth.make_inputs(wl, seed=0)
     nthreads = O.nthreads_default()
-    rows_per_step = args.ref_rows
+    # the CPU-baseline sample, one (batch, head) group per step, groups in
+    # turn: each step pays one head's set-up for that head's rows, as the
+    # baseline does, so the two figures measure the same thing
+    sample = cpu_sample_rows(wl, cpu_rows_of(args))
+    keys = sample[:, 0] * wl.Hq + sample[:, 1]
+    groups = [sample[keys == kk] for kk in np.unique(keys)]
 
     def step(s):
         if decode:  # the decoded row of every sequence, one head per step
             rows = np.array([(b, s % wl.Hq, wl.T - 1) for b in range(wl.B)], dtype=np.int64)
-        else:  # one head per step, rows spread over positions
-            rows = _oracle_sample(wl, rows_per_step, 100 + s)
-            rows[:, 1] = s % wl.Hq
+        else:
+            rows = groups[s % len(groups)]
         _oracle_rows(O, wl, inp, rows, nthreads)
         return _pairs_of_rows(wl, rows, inp["is_sep"])
 
@@ -1223,8 +1242,9 @@ def run_reference(args):
         "config": config_dict(wl, int(decode_keys(wl, inp["is_sep"]).sum()) * wl.Hq if decode
                               else unmasked_pairs(wl, inp["is_sep"]), decode=decode),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
-                         "sample": "each step: %d seeded rows of one head (heads cycle), fp64 C oracle"
-                                   % rows_per_step},
+                         "sample": ("each step: the decoded rows of one head (heads cycle)" if decode else
+                                    "each step: the rows of one (batch, head) of the %d-row CPU-baseline sample "
+                                    "(groups in turn)" % len(sample)) + ", fp64 C oracle"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -1240,8 +1260,8 @@ def main():
                     choices=sorted(WORKLOAD_ALIASES) + sorted(WORKLOAD_ALIASES.values()) + sorted(DECODE_ALIASES)
                     + sorted(BWD_ALIASES) + sorted(TREE_ALIASES) + sorted(STREAM_ALIASES) + sorted(STRESS_ALIASES)
                     + sorted(EXTRA_WORKLOADS))
-    ap.add_argument("--cpu-rows", type=int, default=32768, help="rows in the CPU-oracle baseline sample (~10 s)")
-    ap.add_argument("--ref-rows", type=int, default=32, help="rows per step of the reference arm")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="rows in the CPU-oracle baseline sample (default: 6144 on the top-k workload, else 32768)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling captures only)")
     args = ap.parse_args()

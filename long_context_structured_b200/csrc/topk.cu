@@ -34,7 +34,8 @@ namespace sattn {
 
 namespace {
 
-constexpr int kThreads = 320;  // 8 scan warps (two query tiles), TMA warp, MMA warp
+constexpr int kThreads = 576;  // 16 scan warps (two query tiles x two column halves), TMA warp, MMA warp
+constexpr int kTmaWarp = 16, kMmaWarp = 17;
 constexpr int kSBuf = 2;       // TMEM score buffers per query tile
 
 template <typename Tin>
@@ -95,7 +96,7 @@ __device__ __forceinline__ void list_insert(float v, int j, float (&vals)[KC], i
 // maximum, and only when some row of the warp has a chunk maximum above its
 // threshold does the warp build bit masks and append.
 constexpr int kSampleKeep = 16;  // group maxima kept per row in the sample phase
-constexpr int kStagesK = 3;      // K tiles in flight
+constexpr int kStagesK = 2;      // K tiles in flight
 // floats per scan thread's scratch row: a multiple of 4 (16-byte stores) that
 // puts the eight rows of a quarter-warp on distinct bank groups
 constexpr int kScratchStride = 36;
@@ -107,6 +108,29 @@ __device__ __forceinline__ void sample_plan(int ntiles, int& stride, int& r, boo
   if (ntiles >= 48) { stride = 6; r = 8; }
   else if (ntiles >= 16) { stride = 3; r = 12; }
   else { stride = 1; r = 16; fine = true; }
+}
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// (m << 2) | [v_hi > t] << 1 | [v_lo > t]: t - v has its sign bit set exactly
+// when v > t (t - v is +0 for v == t and a positive NaN for -inf - -inf); one
+// packed subtraction for the pair, one funnel shift per bit
+__device__ __forceinline__ uint32_t push_above2(uint32_t m, float v_lo, float v_hi, unsigned long long tt) {
+  uint32_t r;
+  asm("{\n\t.reg .b64 t, d;\n\t.reg .b32 lo, hi;\n\t"
+      "mov.b64 t, {%2, %3};\n\t"
+      "sub.rn.f32x2 d, %4, t;\n\t"
+      "mov.b64 {lo, hi}, d;\n\t"
+      "shf.l.clamp.b32 %0, hi, %1, 1;\n\t"
+      "shf.l.clamp.b32 %0, lo, %0, 1;\n\t}"
+      : "=r"(r)
+      : "r"(m), "f"(v_lo), "f"(v_hi), "l"(tt));
+  return r;
 }
 
 // insert v into the descending list s (values only)
@@ -135,8 +159,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = base;  // Q0 | Q1
   uint8_t* sk = base + 2 * kTileBytes;  // kSt K tiles
-  float* scratch = reinterpret_cast<float*>(sk + kSt * kTileBytes);  // [256 scan threads][kScratchStride]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + 256 * kScratchStride);
+  float* scratch = reinterpret_cast<float*>(sk + kSt * kTileBytes);  // [512 scan threads][kScratchStride]
+  int* rcnt = reinterpret_cast<int*>(scratch + 512 * kScratchStride);  // [256 rows] keys above tau
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rcnt + 256);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* k_empty = k_full + kSt;
@@ -182,14 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2 * kSBuf; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 128);
+      mbar_init(s_free + s, 256);  // both column halves of the tile's 128 rows
     }
     mbar_init(drain, 1);
     fence_mbar_init();
   }
+  for (int x = threadIdx.x; x < 256; x += blockDim.x) rcnt[x] = 0;
   __syncthreads();
   if (*early) return;
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -199,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_flag = abort_i;
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ===== TMA producer: both query tiles once, then the K ring =====
     if (lane == 0 && n_steps > 0) {
       mbar_expect_tx(q_full, 2 * kTileBytes);
@@ -223,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = max(0, issued - kSt); it < issued; ++it) mbar_wait_raw(k_full + it % kSt, (it / kSt) & 1);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ===== MMA issuer: per K tile, S_x = Q_x K^T for each query tile that needs it =====
     if (lane == 0 && n_steps > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
@@ -258,13 +284,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_raw(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 8) {
-    // scan warps: warpgroup qt = warp / 4 scans query tile qt; thread r of the
-    // warpgroup owns query row i0 + r (TMEM lane r)
-    const int qt = warp >> 2;
-    const int r = threadIdx.x & 127;
+  } else if (warp < 16) {
+    // scan warps: warp w scans query tile qt = (w / 4) % 2, rows 32 (w % 4)
+    // .. + 31 of it (TMEM lanes of the warp's quarter), columns 64 ch .. + 63
+    // of every key tile, ch = w / 8; the two threads of a row (warps w and
+    // w ^ 8) share the row's threshold and its candidate list
+    const int qt = (warp >> 2) & 1;
+    const int ch = warp >> 3;
+    const int rl = (warp & 3) * 32 + lane;  // row within the query tile
     const int i0 = (2 * qb + qt) * kTile;
-    const int i = i0 + r;
+    const int i = i0 + rl;
     const int ntx = nt[qt];
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     // candidates of this row: n_start <= j <= i - w - 1; of the warp's rows,
@@ -274,20 +303,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp_j_hi = (i0 + (warp & 3) * 32 + 31 < a.T) ? i0 + (warp & 3) * 32 - a.window - 1 : -1;
     const size_t row = ((size_t)b * a.Hq + h) * a.T + (i < a.T ? i : a.T - 1);
     int2* list = a.cand_idx + row * kCandCap;
-    float* my_scratch = scratch + (threadIdx.x & 255) * kScratchStride;
+    int* my_cnt = rcnt + qt * 128 + rl;
+    float* my_scratch = scratch + (threadIdx.x & 511) * kScratchStride;
+    const float* partner_scratch = scratch + ((threadIdx.x ^ 256) & 511) * kScratchStride;
+    const int bar_id = 1 + qt;  // named barrier of the query tile's 256 scan threads
     float samp[kR];
 #pragma unroll
     for (int x = 0; x < kR; ++x) samp[x] = -CUDART_INF_F;
     float tau = -CUDART_INF_F;
-    int n = 0;  // keys above tau (list entries written: min(n, kCandCap))
     int cx = 0; // score tiles consumed
     bool ok = true;
     const uint8_t* flags = a.is_sep ? a.is_sep + (size_t)b * a.T : nullptr;
     for (int it = 0; it < n_steps; ++it) {
-      if (it == n_s) {  // end of the sample phase: tau = the r-th largest sampled chunk maximum
+      if (it == n_s) {
+        // end of the sample phase: tau = the r-th largest of the maxima both
+        // halves of the row sampled (a merge of the two sorted lists)
 #pragma unroll
-        for (int x = 0; x < kR; ++x)
-          if (x == r_tau - 1) tau = samp[x];
+        for (int x = 0; x < kR; ++x) my_scratch[x] = samp[x];
+        asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
+        int pa = 0, pb = 0;
+        float other = partner_scratch[0];
+        for (int x = 0; x < r_tau; ++x) {
+          float mine = -CUDART_INF_F;
+#pragma unroll
+          for (int y = 0; y < kR; ++y)
+            if (y == pa) mine = samp[y];
+          if (mine >= other) {
+            tau = mine;
+            ++pa;
+          } else {
+            tau = other;
+            ++pb;
+            other = pb < kR ? partner_scratch[pb] : -CUDART_INF_F;
+          }
+        }
+        asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");  // scratch rows are reused below
       }
       const int t = tile_of(it);
       if (t >= ntx) continue;
@@ -300,87 +350,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool interior = (j0 >= a.n_start) && (j0 + kTile - 1 <= warp_j_hi);
       const int c_lo = max(0, a.n_start - j0);
       const int c_hi = min(kTile - 1, j_hi - j0);
-      // the row's 128 scores in two halves of 64 (keeps the scan within its
-      // register budget); the TMEM buffer goes back to the MMA warp as soon
-      // as the second half is in registers
+      // this thread's 64 columns as two chunks of 32; the TMEM buffer goes
+      // back to the MMA warp once the second chunk is in registers
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[64];
-        tmem_ld32(tmem + (qt * kSBuf + sb) * 128 + lane_off + hf * 64, v);
-        tmem_ld32(tmem + (qt * kSBuf + sb) * 128 + lane_off + hf * 64 + 32, v + 32);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int cb = ch * 64 + c2 * 32;  // first column of this 32-column chunk
+        float v[32];
+        tmem_ld32(tmem + (qt * kSBuf + sb) * 128 + lane_off + cb, v);
         tc_wait_ld();
-        if (hf == 1) {
+        if (c2 == 1) {
           tc_fence_before();
           if (ok) mbar_arrive(s_free + qt * kSBuf + sb);
         }
         if (!interior || flags) {
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const int cb = hf * 64 + c2 * 32;  // first column of this 32-column chunk
-            uint32_t sepm = 0;
-            if (flags) {
-              const int jj = j0 + cb + lane;
-              sepm = __ballot_sync(0xffffffffu, jj < a.T && flags[jj] != 0);
-            }
-            const int lo = max(c_lo - cb, 0);
-            const int hi = min(c_hi - cb, 31);
-            uint32_t vm = 0;
-            if (lo <= hi) vm = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
-            vm &= ~sepm;
-#pragma unroll
-            for (int y = 0; y < 32; ++y) v[c2 * 32 + y] = ((vm >> y) & 1u) ? v[c2 * 32 + y] : -CUDART_INF_F;
+          uint32_t sepm = 0;
+          if (flags) {
+            const int jj = j0 + cb + lane;
+            sepm = __ballot_sync(0xffffffffu, jj < a.T && flags[jj] != 0);
           }
+          const int lo = max(c_lo - cb, 0);
+          const int hi = min(c_hi - cb, 31);
+          uint32_t vm = 0;
+          if (lo <= hi) vm = (hi == 31 ? 0xffffffffu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u);
+          vm &= ~sepm;
+#pragma unroll
+          for (int y = 0; y < 32; ++y) v[y] = ((vm >> y) & 1u) ? v[y] : -CUDART_INF_F;
         }
+        // group maxima pm[g] over columns g, g + 8, g + 16, g + 24, then the chunk maximum
+        float pm[8];
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          float pm[8];
+        for (int y = 0; y < 8; ++y) pm[y] = fmaxf(fmax3(v[y], v[y + 8], v[y + 16]), v[y + 24]);
+        const float cm = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        if (sample) {
+          if (fine) {
 #pragma unroll
-          for (int y = 0; y < 8; ++y) pm[y] = v[c2 * 32 + y];
-#pragma unroll
-          for (int y = 8; y < 32; ++y) pm[y & 7] = fmaxf(pm[y & 7], v[c2 * 32 + y]);
-          const float cm =
-              fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-          if (sample) {
-            if (fine) {
-#pragma unroll
-              for (int y = 0; y < 8; ++y)
-                if (pm[y] > samp[kR - 1]) insert_val<kR>(pm[y], samp);
-            } else if (cm > samp[kR - 1]) {
-              insert_val<kR>(cm, samp);
-            }
-            continue;
+            for (int y = 0; y < 8; ++y)
+              if (pm[y] > samp[kR - 1]) insert_val<kR>(pm[y], samp);
+          } else if (cm > samp[kR - 1]) {
+            insert_val<kR>(cm, samp);
           }
-          if (__any_sync(0xffffffffu, cm > tau) && cm > tau) {
-            // append this row's keys above tau with their coarse scores, in
-            // key order (the chunk goes through the thread's scratch row so
-            // that a score can be picked by a run-time column)
-            uint32_t m = 0;
+          continue;
+        }
+        if (__any_sync(0xffffffffu, cm > tau) && cm > tau) {
+          // append this row's keys above tau with their coarse scores (the
+          // chunk goes through the thread's scratch row so that a score can
+          // be picked by a run-time column)
+          const unsigned long long tt = (unsigned long long)__float_as_uint(tau) << 32 | __float_as_uint(tau);
+          // bit y: column y above tau (four independent 8-bit chains)
+          uint32_t mq[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int y = 0; y < 32; ++y) m |= (v[c2 * 32 + y] > tau) ? (1u << y) : 0u;
+          for (int y = 7; y > 0; y -= 2)
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              reinterpret_cast<float4*>(my_scratch)[q4] = make_float4(
-                  v[c2 * 32 + 4 * q4], v[c2 * 32 + 4 * q4 + 1], v[c2 * 32 + 4 * q4 + 2], v[c2 * 32 + 4 * q4 + 3]);
-            const int jbase = j0 + hf * 64 + c2 * 32;
-            while (m) {
-              const int y = __ffs(m) - 1;
-              m &= m - 1;
-              if (n < kCandCap) list[n] = make_int2(jbase + y, __float_as_int(my_scratch[y]));
-              ++n;
-            }
+            for (int q4 = 0; q4 < 4; ++q4) mq[q4] = push_above2(mq[q4], v[8 * q4 + y - 1], v[8 * q4 + y], tt);
+          uint32_t m = mq[0] | mq[1] << 8 | mq[2] << 16 | mq[3] << 24;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            reinterpret_cast<float4*>(my_scratch)[q4] =
+                make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          const int jbase = j0 + cb;
+          while (m) {
+            const int y = __ffs(m) - 1;
+            m &= m - 1;
+            const int pos = atomicAdd(my_cnt, 1);
+            if (pos < kCandCap) list[pos] = make_int2(jbase + y, __float_as_int(my_scratch[y]));
           }
         }
       }
     }
-    if (i < a.T) {
+    asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");  // both halves have appended
+    if (ch == 0 && i < a.T) {
       a.cand_thr[row] = tau;
-      a.cand_cnt[row] = n;
+      a.cand_cnt[row] = *my_cnt;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -624,7 +670,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
 // ---------------------------------------------------------------------------
 // pass 3: exact fp32 scan of all candidates of a row (block per row)
 // ---------------------------------------------------------------------------
-constexpr int kExactThreads = 256;
+constexpr int kExactThreads = 512;
 constexpr int kMaxK = 16;
 
 template <typename Tin, int PP>
@@ -756,7 +802,8 @@ cudaError_t launch_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) 
   const size_t tile = (size_t)D * kTile * 2;
   // Q tiles, K ring, scan scratch, barriers; at least 116 KB: one CTA per SM, so the
   // 512-column TMEM allocation never waits
-  const size_t bytes = std::max<size_t>(116 * 1024, 1024 + tile * (2 + kStagesK) + 256 * kScratchStride * 4 + 256);
+  const size_t bytes =
+      std::max<size_t>(116 * 1024, 1024 + tile * (2 + kStagesK) + 512 * kScratchStride * 4 + 256 * 4 + 256);
   cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   const int nQB = (a.nQT + 1) / 2;
