@@ -41,12 +41,19 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "attn_common.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 
 namespace sattn {
 
 namespace {
+
+using attn::exp2_neg_int;
+using attn::kSumAccept;
+using attn::kSumRebase;
+using attn::make_plan;
+using attn::Plan;
 
 constexpr int kThreads = 384;  // 2 softmax warpgroups + 1 warpgroup holding the producer and MMA warps
 // register split (per thread): the producer/MMA warpgroup gives registers to
@@ -57,59 +64,8 @@ static_assert(2 * 128 * kRegSoftmax + 128 * kRegCtrl <= kThreads * 168, "registe
 constexpr int kKS = 2;         // K stages (K is consumed early: both S products of a position)
 constexpr int kVS = 3;         // V stages (V is consumed one position later, by the PV products)
 constexpr uint32_t kTmemCols = 512;
-// A tile's P is computed against the row's running reference m (log2
-// units) without first taking the tile's row maximum.  That is exact
-// arithmetic for softmax as long as nothing overflows: P = 2^(s - m) is
-// stored in bf16 and summed in fp32, both of which keep their relative
-// precision at any magnitude.  A row whose tile sum exceeds 2^kSumAccept
-// (this includes +inf) redoes the tile against its true maximum; a row whose
-// accepted sum exceeds 2^kSumRebase moves m up by a power of two before its
-// next tile, so the rescale of O and l is exact.
-constexpr float kSumAccept = 0x1p32f;
 constexpr int kMaxSideTopk = 16;  // top-k side keys per row (the library's limit on k)
 constexpr int kSinkSmem = 16;     // sink V rows staged in shared memory up to this many
-constexpr float kSumRebase = 0x1p8f;
-__device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
-  uint32_t a = smem_u32(bar);
-  uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer_ns() - t0 > 100000000ull) return false;
-  }
-  return true;
-}
-
-// MMA and commit issued by one elected lane of a warp that runs the issue
-// loop in lockstep: the loop's values stay warp-uniform (so they live in
-// uniform registers), and a single lane issues each instruction.
-// D[tmem] (+)= A[smem] * B[smem]^T
-__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]^T
-__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void commit_elect(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
 
 // 32 consecutive 32-bit columns of this thread's lane
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
@@ -123,24 +79,6 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-
-// paired fp32 arithmetic (one instruction for two lanes of work)
-__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
-                                     float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
-  asm("{\n\t.reg .b64 ra, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
-      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1));
-}
-
 
 // P = 2^(s*sl2 + neg_m) for this thread's row of a 128-key tile, packed to
 // bf16 and stored to TMEM over the first 64 S columns (keys 64h..64h+63 go
@@ -179,57 +117,6 @@ __device__ __forceinline__ void scale_o(uint32_t taddr, float f) {
     for (int y = 0; y < 32; ++y) ov[y] *= f;
     tmem_st32(taddr + c * 32, ov);
   }
-}
-
-// 2^-e for an integer e in [0, 126]
-__device__ __forceinline__ float exp2_neg_int(int e) { return __int_as_float((127 - e) << 23); }
-
-
-// Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
-// then band key tiles [u_lo, u_lo + n_band).
-struct Plan {
-  int g_count, g_full, n_gather, band_lo, u_lo, n_band, rows;  // rows: valid rows of the tile (0 = none)
-};
-
-__device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t) {
-  Plan p;
-  p.g_count = 0;
-  p.g_full = 0;
-  p.band_lo = 0;
-  const int i0 = t * kTile;
-  p.rows = (i0 < a.T) ? min(kTile, a.T - i0) : 0;
-  if (p.rows == 0) {
-    p.n_gather = p.n_band = p.u_lo = 0;
-    return p;
-  }
-  if (a.gather_mode == 1) {
-    p.g_full = a.ranges[(b * a.nQT + t) * 2 + 0];
-    p.g_count = a.ranges[(b * a.nQT + t) * 2 + 1];
-  } else if (a.gather_mode == 3) {
-    // cross-attention over a compressed context: every row keeps all of it
-    p.g_count = p.g_full = a.cross_len;
-  } else if (a.gather_mode == 2) {
-    const int s = i0 / a.seg_S;
-    const int seg0 = s * a.seg_S;
-    const int slot = a.long_slot[h];
-    if (slot >= 0) {
-      p.band_lo = seg0;
-      if (s > 0) p.g_count = p.g_full = a.prefix_cnt[(b * a.n_long + slot) * a.seg_N + s];
-    } else {
-      p.band_lo = s > 0 ? max(0, seg0 - a.seg_M) : 0;
-    }
-  }
-  p.n_gather = (p.g_count + kTile - 1) / kTile;
-  const int i_last = i0 + p.rows - 1;
-  const int j_lo = max(max(p.band_lo, 0), max(i0 - a.w_eff, a.ns_band));
-  if (j_lo > i_last || a.gather_mode == 3) {
-    p.u_lo = 0;
-    p.n_band = 0;
-  } else {
-    p.u_lo = j_lo / kTile;
-    p.n_band = i_last / kTile - p.u_lo + 1;
-  }
-  return p;
 }
 
 // Union order: gathered positions [0, NG), then band tiles u in [U0, U1].
@@ -365,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++issued;
       }
       if (!ok) {
-        if (kstream) mbar_wait_raw(q_full, 0);
-        for (int p = max(0, issued - NS); p < issued; ++p) mbar_wait_raw(full + p % NS, (p / NS) & 1);
+        if (kstream) tc::wait_raw(q_full, 0);
+        for (int p = max(0, issued - NS); p < issued; ++p) tc::wait_raw(full + p % NS, (p / NS) & 1);
       }
     }
     } else if (warp == 9) {
@@ -402,11 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bv = dv + (uint64_t)((vs * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts_elect(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
+          tc::mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
                        (n_pv[x] > 0 || kk > 0) ? 1u : 0u);
-        commit_elect(o_done + x);
+        tc::commit(o_done + x);
         // the V stage is free once every tile that uses this position ran its PV
-        if (--v_users[vs] == 0) commit_elect(v_empty + vs);
+        if (--v_users[vs] == 0) tc::commit(v_empty + vs);
         ++n_pv[x];
         prev[x] = -1;
         return true;
@@ -431,26 +318,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-            mma_ss_elect(tmem + x * 128, ba + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
+            tc::mma_ss(tmem + x * 128, ba + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          commit_elect(s_full + x);
+          tc::commit(s_full + x);
           prev[x] = p;
-          if (!((x == 0) && need[1])) commit_elect(k_empty + ks);
+          if (!((x == 0) && need[1])) tc::commit(k_empty + ks);
         }
         if (ok && users == 0) {
           // no tile reads this position (cannot happen for contiguous plans); release it
           ok = wait_all(k_full + ks, (p / kKS) & 1, 40);
           if (!ok) break;
-          commit_elect(k_empty + ks);
+          tc::commit(k_empty + ks);
           ok = wait_all(v_full + p % kVS, (p / kVS) & 1, 36);
-          if (ok) commit_elect(v_empty + p % kVS);
+          if (ok) tc::commit(v_empty + p % kVS);
         }
       }
       // pending PVs of the last positions
       for (int x = 0; x < 2 && ok; ++x)
         if (prev[x] >= 0) ok = issue_pv(x);
-      commit_elect(drain);
-      mbar_wait_raw(drain, 0);
+      tc::commit(drain);
+      tc::wait_raw(drain, 0);
     }
     __syncwarp();
     }

@@ -45,6 +45,7 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "attn_common.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -52,105 +53,15 @@ namespace sattn {
 
 namespace {
 
+using attn::exp2_neg_int;
+using attn::kSumAccept;
+using attn::kSumRebase;
+using attn::make_plan;
+using attn::Plan;
+
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 384;  // O columns (S buffers at 0, 128, 256)
-constexpr float kSumAccept = 0x1p32f;
-constexpr float kSumRebase = 0x1p8f;
-
-__device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
-  uint32_t a = smem_u32(bar);
-  uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer_ns() - t0 > 100000000ull) return false;
-  }
-  return true;
-}
-
-// MMA and commit issued by one elected lane of a warp that runs the issue
-// loop in lockstep: the loop's values stay warp-uniform (so they live in
-// uniform registers), and a single lane issues each instruction.
-// D[tmem] (+)= A[smem] * B[smem]^T
-__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]^T
-__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void commit_elect(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-// TMEM accesses of shape 16x32bx2: a warp reaches 16 lanes (the address's
-// lane field, inside the warp's quadrant); lanes 0-15 of the warp take 32
-// consecutive columns from the address, lanes 16-31 the same lanes' 32
-// columns from the address + SPLIT.
-#define SATTN_R32(p)                                                                                            \
-  "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]), "r"(p[8]), "r"(p[9]), \
-      "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15]), "r"(p[16]), "r"(p[17]), "r"(p[18]),  \
-      "r"(p[19]), "r"(p[20]), "r"(p[21]), "r"(p[22]), "r"(p[23]), "r"(p[24]), "r"(p[25]), "r"(p[26]), "r"(p[27]),  \
-      "r"(p[28]), "r"(p[29]), "r"(p[30]), "r"(p[31])
-#define SATTN_W32(p)                                                                                             \
-  "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]), "=r"(p[7]), "=r"(p[8]),    \
-      "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]), "=r"(p[13]), "=r"(p[14]), "=r"(p[15]), "=r"(p[16]),      \
-      "=r"(p[17]), "=r"(p[18]), "=r"(p[19]), "=r"(p[20]), "=r"(p[21]), "=r"(p[22]), "=r"(p[23]), "=r"(p[24]),     \
-      "=r"(p[25]), "=r"(p[26]), "=r"(p[27]), "=r"(p[28]), "=r"(p[29]), "=r"(p[30]), "=r"(p[31])
-template <int SPLIT>
-__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float* v) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], %33;"
-      : SATTN_W32(r)
-      : "r"(taddr), "n"(SPLIT)
-      : "memory");
-}
-template <int SPLIT>
-__device__ __forceinline__ void tmem_st16x2(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
-      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, "
-      "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};" ::"r"(taddr),
-      "n"(SPLIT), SATTN_R32(r)
-      : "memory");
-}
-
-// paired fp32 arithmetic (one instruction for two lanes of work)
-__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
-                                     float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
-  asm("{\n\t.reg .b64 ra, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
-      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1));
-}
 
 // P = 2^(s*sl2 + neg_m) for this thread's half row (64 keys), packed to
 // bf16 and stored to TMEM: the pair owning the row writes P columns 0-31
@@ -170,7 +81,7 @@ __device__ __forceinline__ float emit_p(const float (&sv)[64], float sl2, float 
     add2(ps[(c >> 1) & 3], ps[4 + ((c >> 1) & 3)], p0, p1);
     pk[c >> 1] = pack_bf16x2(p0, p1);
   }
-  tmem_st16x2<32>(taddr, pk);
+  tc::st16x2<32>(taddr, pk);
   return ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
 }
 
@@ -197,58 +108,12 @@ __device__ __forceinline__ void scale_o(uint32_t taddr, float f) {
 #pragma unroll 1
   for (int c = 0; c < D / 2; c += 32) {
     float ov[32];
-    tmem_ld16x2<D / 2>(taddr + c, ov);
+    tc::ld16x2<D / 2>(taddr + c, ov);
     tc_wait_ld();
 #pragma unroll
     for (int y = 0; y < 32; ++y) ov[y] *= f;
-    tmem_st16x2<D / 2>(taddr + c, reinterpret_cast<const uint32_t*>(ov));
+    tc::st16x2<D / 2>(taddr + c, reinterpret_cast<const uint32_t*>(ov));
   }
-}
-
-// 2^-e for an integer e in [0, 126]
-__device__ __forceinline__ float exp2_neg_int(int e) { return __int_as_float((127 - e) << 23); }
-
-// Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
-// then band key tiles [u_lo, u_lo + n_band).
-struct Plan {
-  int g_count, g_full, n_gather, band_lo, u_lo, n_band, rows;  // rows: valid rows of the tile
-};
-
-__device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t) {
-  Plan p;
-  p.g_count = 0;
-  p.g_full = 0;
-  p.band_lo = 0;
-  const int i0 = t * kTile;
-  p.rows = min(kTile, a.T - i0);
-  if (a.gather_mode == 1) {
-    p.g_full = a.ranges[(b * a.nQT + t) * 2 + 0];
-    p.g_count = a.ranges[(b * a.nQT + t) * 2 + 1];
-  } else if (a.gather_mode == 3) {
-    // cross-attention over a compressed context: every row keeps all of it
-    p.g_count = p.g_full = a.cross_len;
-  } else if (a.gather_mode == 2) {
-    const int s = i0 / a.seg_S;
-    const int seg0 = s * a.seg_S;
-    const int slot = a.long_slot[h];
-    if (slot >= 0) {
-      p.band_lo = seg0;
-      if (s > 0) p.g_count = p.g_full = a.prefix_cnt[(b * a.n_long + slot) * a.seg_N + s];
-    } else {
-      p.band_lo = s > 0 ? max(0, seg0 - a.seg_M) : 0;
-    }
-  }
-  p.n_gather = (p.g_count + kTile - 1) / kTile;
-  const int i_last = i0 + p.rows - 1;
-  const int j_lo = max(max(p.band_lo, 0), max(i0 - a.w_eff, a.ns_band));
-  if (j_lo > i_last || a.gather_mode == 3) {
-    p.u_lo = 0;
-    p.n_band = 0;
-  } else {
-    p.u_lo = j_lo / kTile;
-    p.n_band = i_last / kTile - p.u_lo + 1;
-  }
-  return p;
 }
 
 template <int D, bool Q2>
@@ -373,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // let the loads in flight land before the CTA's shared memory goes away
-        if (kstream) mbar_wait_raw(q_full, 0);
-        for (int j = max(0, issued - NS); j < issued; ++j) mbar_wait_raw(full + j % NS, (j / NS) & 1);
+        if (kstream) tc::wait_raw(q_full, 0);
+        for (int j = max(0, issued - NS); j < issued; ++j) tc::wait_raw(full + j % NS, (j / NS) & 1);
       }
     }
   } else if (warp == 9) {
@@ -406,10 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-            mma_ss_elect(tmem + (j % 3) * 128, ba + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
+            tc::mma_ss(tmem + (j % 3) * 128, ba + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          commit_elect(s_full + (j % 3));
-          commit_elect(k_empty + ks);
+          tc::commit(s_full + (j % 3));
+          tc::commit(k_empty + ks);
         }
         if (j >= 2) {
           const int jj = j - 2;
@@ -421,15 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bv = dv + (uint64_t)((vs * kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts_elect(tmem + kTmemO, tmem + (jj % 3) * 128 + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4),
+            tc::mma_ts(tmem + kTmemO, tmem + (jj % 3) * 128 + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4),
                          idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
-          commit_elect(o_done + (jj & 1));
-          commit_elect(v_empty + vs);
-          if (jj == n - 1) commit_elect(o_final);
+          tc::commit(o_done + (jj & 1));
+          tc::commit(v_empty + vs);
+          if (jj == n - 1) tc::commit(o_final);
         }
       }
-      commit_elect(drain);
-      mbar_wait_raw(drain, 0);
+      tc::commit(drain);
+      tc::wait_raw(drain, 0);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -486,8 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       c_hi -= 64 * hc;
       const bool partial = (c_lo > 0 || c_hi < 63);
       float sv[64];
-      tmem_ld16x2<64>(tS, sv);
-      tmem_ld16x2<64>(tS + 32, sv + 32);
+      tc::ld16x2<64>(tS, sv);
+      tc::ld16x2<64>(tS + 32, sv + 32);
       tc_wait_ld();
       if (partial) {
 #pragma unroll
@@ -588,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < D / 2; c += 32) {
       float ov[32];
       if (n > 0) {
-        tmem_ld16x2<D / 2>(tO + c, ov);
+        tc::ld16x2<D / 2>(tO + c, ov);
         tc_wait_ld();
 #pragma unroll
         for (int y = 0; y < 32; ++y) ov[y] *= alpha * o_rebase;

@@ -1,6 +1,6 @@
-// simt.cuh -- small CUDA-core helpers shared by the elementwise kernels:
-// paired fp32 fused multiply-add and a transposed reduction of several
-// values over a group of lanes.
+// simt.cuh -- small CUDA-core helpers shared by the kernels: paired fp32
+// fused multiply-add and add, and a transposed reduction of several values
+// over a group of lanes.
 #pragma once
 
 namespace sattn {
@@ -13,6 +13,15 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// d0 += a0, d1 += a1 as one paired fp32 instruction
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
 }
 
 // Sum NV per-lane values over each group of W consecutive lanes (W a power

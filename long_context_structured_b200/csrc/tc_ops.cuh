@@ -1,6 +1,5 @@
 // tc_ops.cuh -- warp-level tcgen05 issue helpers and TMEM accesses shared by
-// the backward-pass kernels (the forward kernels keep their own copies so
-// that their code generation stays as measured).
+// the tensor-core kernels (forward attention and backward pass).
 #pragma once
 
 #include "sm100.cuh"
