@@ -231,9 +231,11 @@ int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes);
  * fp32: CUDA cores, one kernel writes dq per query row, another dk and dv
  * per key.  bf16: tensor cores (a dq kernel per 128-row query tile, a dk/dv
  * kernel per 128-key tile of positions or of compacted separators, both
- * recomputing P from lse), the sink keys on CUDA cores, fp32 partial sums
- * combined in a fixed order; bf16 with topk > 0: SATTN_ERR_UNSUPPORTED.
- * Deterministic (no atomics).  Asynchronous on `stream`. */
+ * recomputing P from lse), the sink and top-k keys on CUDA cores (the top-k
+ * key side through each key's list of selecting rows, summed in ascending
+ * (head, row) order), fp32 partial sums combined in a fixed order.  bf16
+ * with topk > 0 needs B * Hq * T * topk < 2^31 (else SATTN_ERR_UNSUPPORTED).
+ * Deterministic (no floating-point atomics).  Asynchronous on `stream`. */
 int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
               const int32_t* topk_idx, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
               void* dV, void* ws, size_t ws_bytes, void* stream);

@@ -940,7 +940,8 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
 struct BwdPlan {
   FwdPlan F;  // regions shared with the forward's steps (status, table, prep products, block map, gather)
   int nRB = 0;
-  Region dsum, nlse2, sink_ds, sink_p, sink_part, dq_side, dk_band, dv_band, dk_sep, dv_sep;
+  Region dsum, nlse2, sink_ds, sink_p, sink_part, dq_side, dk_band, dv_band, dk_sep, dv_sep, tk_ds, tk_p, tk_cnt,
+      tk_off, tk_cur, tk_code, tk_sorted;
   size_t total = 0;
 };
 
@@ -950,7 +951,9 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
   BwdPlan P;
   FwdPlan& F = P.F;
   F.bf16 = p->dtype == SATTN_DTYPE_BF16;
-  if (F.bf16 && p->topk > 0) return SATTN_ERR_UNSUPPORTED;  // top-k backward: fp32 path only
+  // top-k key lists are indexed in 32 bits
+  if (F.bf16 && p->topk > 0 && (int64_t)p->B * p->Hq * p->T * p->topk >= ((int64_t)1 << 31))
+    return SATTN_ERR_UNSUPPORTED;
   F.nQT = (p->T + kTile - 1) / kTile;
   F.Tpad = F.nQT * kTile;
   F.npos = std::max(p->T, p->L_pretrain + 1);
@@ -988,9 +991,20 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
       P.nRB = (int)((T + bwd_sink_row_block() - 1) / bwd_sink_row_block());
       P.sink_part = A.take(B * Hkv * F.n_sink * (size_t)P.nRB * 2 * d * 4);
     }
-    if (F.capped_sep) P.dq_side = A.take(B * Hq * T * d * 4);  // the capped separators' dq (first dq pass)
+    // the capped separators' dq (first dq pass) and the top-k pairs' dq
+    if (F.capped_sep || p->topk > 0) P.dq_side = A.take(B * Hq * T * d * 4);
     P.dk_band = A.take(B * Hkv * T * d * 4);
     P.dv_band = A.take(B * Hkv * T * d * 4);
+    if (p->topk > 0) {
+      const size_t sel = B * Hq * T * (size_t)p->topk;
+      P.tk_ds = A.take(sel * 4);
+      P.tk_p = A.take(sel * 4);
+      P.tk_cnt = A.take(B * Hkv * T * 4);
+      P.tk_off = A.take(B * Hkv * T * 4);
+      P.tk_cur = A.take(B * Hkv * T * 4);
+      P.tk_code = A.take(sel * 4);
+      P.tk_sorted = A.take(sel * 4);
+    }
   }
   P.total = A.cur;
   *out = P;
@@ -998,8 +1012,8 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
 }
 
 static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, const void* K, const void* V,
-                        const uint8_t* is_sep, const void* O, const float* lse, const void* dO, void* dQ, void* dK,
-                        void* dV, void* ws, cudaStream_t st) {
+                        const uint8_t* is_sep, const int32_t* topk_idx, const void* O, const float* lse,
+                        const void* dO, void* dQ, void* dK, void* dV, void* ws, cudaStream_t st) {
   const FwdPlan& F = P.F;
   const int64_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
   int rc = run_prep_bf16(p, F, Q, K, ws, F.n_sink > 0, false, st);
@@ -1109,18 +1123,33 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   a.dK = static_cast<__nv_bfloat16*>(dK);
   a.dV = static_cast<__nv_bfloat16*>(dV);
   a.status = at<int32_t>(ws, F.status);
+  a.topk = p->topk;
+  a.tk_idx = p->topk > 0 ? topk_idx : nullptr;
+  a.tk_ds = at<float>(ws, P.tk_ds);
+  a.tk_p = at<float>(ws, P.tk_p);
+  a.tk_cnt = at<int>(ws, P.tk_cnt);
+  a.tk_off = at<int>(ws, P.tk_off);
+  a.tk_cur = at<int>(ws, P.tk_cur);
+  a.tk_code = at<int>(ws, P.tk_code);
+  a.tk_sorted = at<int>(ws, P.tk_sorted);
   {
     ProfScope ps("bwd_rows", 1, st);
     SATTN_TRY(launch_bwd_rows(a, st));
   }
   // capped separators: a first dq pass writes their part to dq_side, the
-  // second adds it; the sink pairs' dq is formed in the second pass's epilogue
+  // second adds it; the top-k pairs' dq joins dq_side in between; the sink
+  // pairs' dq is formed in the second pass's epilogue
   a.side_valid = false;
   a.fold_sinks = 0;
   if (a.capped_sep) {
     a.dq_mode = 1;
     ProfScope ps("bwd_dq", 1, st);
     SATTN_TRY(launch_bwd_dq(a, m, st));
+    a.side_valid = true;
+  }
+  if (p->topk > 0) {
+    ProfScope ps("bwd_topk_rows", 1, st);
+    SATTN_TRY(launch_bwd_topk_rows(a, a.side_valid, st));
     a.side_valid = true;
   }
   a.dq_mode = 0;
@@ -1132,6 +1161,10 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   {
     ProfScope ps("bwd_dkv", 1, st);
     SATTN_TRY(launch_bwd_dkv(a, m, st));
+  }
+  if (p->topk > 0) {
+    ProfScope ps("bwd_topk_keys", 5, st);
+    SATTN_TRY(launch_bwd_topk_keys(a, st));
   }
   if (F.n_sink > 0) {
     ProfScope ps("bwd_sink_keys", 1, st);
@@ -1165,7 +1198,7 @@ int sattn_bwd(const sattn_params* p, const void* Q, const void* K, const void* V
     return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
-  if (F.bf16) return run_bwd_bf16(p, P, Q, K, V, is_sep, O, lse, dO, dQ, dK, dV, ws, st);
+  if (F.bf16) return run_bwd_bf16(p, P, Q, K, V, is_sep, topk_idx, O, lse, dO, dQ, dK, dV, ws, st);
   if (F.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
     SATTN_TRY(launch_rope_table(at<float2>(ws, F.tab), F.npos, p->d, p->rope_theta, pos_scale(p), st));

@@ -24,12 +24,6 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSinkRowBlock = 256;  // rows per partial sum of the sink-key reduction
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ float2 tab_at(const float2* tab, int64_t pos, int half, int c) {
   return tab ? tab[pos * half + c] : make_float2(1.f, 0.f);
 }

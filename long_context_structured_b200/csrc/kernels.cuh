@@ -285,6 +285,16 @@ struct BwdArgs {
   int dq_mode;                  // dq kernel: 0 band (+ uncapped separators), 1 capped separators only
   bool side_valid;              // dq_side holds data (else it is not read)
   int fold_sinks;               // dq kernel (mode 0): add the sink pairs' dq from sink_ds and the sink key rows
+  // top-k keys (fp32 side keys; the forward's selection is an input)
+  int topk;
+  const int32_t* tk_idx;        // [B, Hq, T, topk] selected keys (-1: none)
+  float* tk_ds;                 // [B, Hq, T, topk] dS of the selected pairs (unscaled)
+  float* tk_p;                  // [B, Hq, T, topk] P of the selected pairs
+  int* tk_cnt;                  // [B, Hkv, T] selections per key
+  int* tk_off;                  // [B, Hkv, T] offset of each key's codes within its (b, kv head) segment
+  int* tk_cur;                  // [B, Hkv, T] fill cursors
+  int* tk_code;                 // [B, Hkv, rep * T * topk] codes ((local head * T + row) * topk + slot) by key
+  int* tk_sorted;               // same layout, each key's codes in ascending order
 };
 struct BwdMaps {
   CUtensorMap q, qc, dO, k, v, kg, vg;
@@ -294,6 +304,12 @@ cudaError_t launch_bwd_sink_keys(const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_dq(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
 cudaError_t launch_bwd_dkv(const BwdArgs& a, const BwdMaps& m, cudaStream_t st);
 cudaError_t launch_bwd_combine(const BwdArgs& a, cudaStream_t st);
+// top-k pairs: the rows' P, dS and dq part (added to dq_side when add_side,
+// else written there)
+cudaError_t launch_bwd_topk_rows(const BwdArgs& a, bool add_side, cudaStream_t st);
+// top-k pairs, key side: dk and dv of every selected key, added to dk_band /
+// dv_band in a fixed order (after the dk/dv kernel has written them)
+cudaError_t launch_bwd_topk_keys(const BwdArgs& a, cudaStream_t st);
 int bwd_sink_row_block();  // rows per partial sum of the sink-key reduction
 
 // ---------------------------------------------------------------------------

@@ -126,6 +126,17 @@ BF16_CASES = [
                                 rope_theta=1e4, sep_rate=0.1, sink_scale=8.0)),
     ("sinks40_d64_uncapped", dict(B=1, Hq=2, Hkv=1, T=500, d=64, n_start=40, window=30, rope_theta=5e5,
                                   sep_rate=0.1)),
+    # top-k middle keys (fp32 side keys, the selection a constant): capped
+    # (L = w), with separators, uncapped (L = 0), and with the clipped ALiBi bias
+    ("topk_capped_sinks_gqa", dict(B=1, Hq=4, Hkv=2, T=700, d=128, n_start=4, window=64, L_pretrain=64,
+                                   rope_theta=1e4, topk=4, sink_scale=8.0)),
+    ("topk_sep_d64", dict(B=2, Hq=2, Hkv=1, T=600, d=64, n_start=2, window=50, L_pretrain=50, rope_theta=1e4,
+                          topk=3, sep_rate=0.1)),
+    ("topk_uncapped_k8", dict(B=1, Hq=2, Hkv=2, T=500, d=128, n_start=4, window=40, rope_theta=1e4, topk=8)),
+    ("topk_alibi", dict(B=1, Hq=4, Hkv=1, T=400, d=128, n_start=4, window=64, L_pretrain=64, topk=3,
+                        alibi=True)),
+    ("topk16_sinks20_sep", dict(B=1, Hq=2, Hkv=2, T=640, d=128, n_start=20, window=48, L_pretrain=48,
+                                rope_theta=1e4, topk=16, sep_rate=0.05)),
 ]
 
 
@@ -135,13 +146,15 @@ def test_bwd_bf16(oracle_mod, name, cfg):
     _run(oracle_mod, wl, 31, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
 
 
-def test_bwd_bf16_deterministic(oracle_mod):
+@pytest.mark.parametrize("topk", [0, 5])
+def test_bwd_bf16_deterministic(oracle_mod, topk):
     wl = synth.Workload(name="det16", B=1, Hq=4, Hkv=2, T=600, d=128, dtype="bf16", n_start=4, window=64,
-                        L_pretrain=64, rope_theta=1e4, sep_rate=0.1)
+                        L_pretrain=64, rope_theta=1e4, sep_rate=0.1, topk=topk)
     grads, (q, k, v, O, lse, dO, sep, idx) = _run(oracle_mod, wl, 8, BF16_GRAD_REL, BF16_GRAD_MEAN_REL)
-    again = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, **_kw(wl))
-    torch.cuda.synchronize()
-    assert all(torch.equal(a, b) for a, b in zip(grads, again))
+    for _ in range(2):
+        again = sa.bwd(q, k, v, O, lse, dO, is_sep=sep, topk=wl.topk, topk_idx=idx, **_kw(wl))
+        torch.cuda.synchronize()
+        assert all(torch.equal(a, b) for a, b in zip(grads, again))
 
 
 def test_bwd_rejects_missing_topk_selection():
