@@ -183,6 +183,30 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
                       const uint8_t* is_long, const void* Q, const void* K, const void* V, void* O, float* lse,
                       int32_t* prefix_blocks, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace needed by sattn_segment_bwd. */
+int sattn_segment_bwd_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                                     size_t* bytes);
+
+/* Backward pass of sattn_segment_fwd ("Training-Inference Consistent
+ * Segmented Execution", sections 整体框架 and 损失函数 / 训练策略: training
+ * runs segment by segment): the gradients of sum(dO * O) with respect to Q,
+ * K and V for the same parameters and key lists as the forward.  The
+ * retrieved blocks are constants (the forward's prefix_blocks are an
+ * input): a retrieved key's gradient returns to its source position through
+ * the rotary position it had in the prefix, and a key used by several rows,
+ * heads or segments sums their contributions.
+ *   is_long        [Hq] uint8 HOST array, as for the forward.
+ *   Q, K, V, O, lse, prefix_blocks   the forward's inputs and outputs.
+ *   dO             gradient of the loss w.r.t. O, strides o_stride.
+ *   dQ, dK, dV     out, shaped and strided like Q, K, V (bf16).
+ * Runs on the CUDA cores in fp32 (a warp per query row for dQ, a warp per
+ * key for dK and dV, each key's rows in a fixed order); deterministic.
+ * Validation as sattn_segment_fwd.  Asynchronous on `stream`. */
+int sattn_segment_bwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                      const uint8_t* is_long, const void* Q, const void* K, const void* V, const void* O,
+                      const float* lse, const int32_t* prefix_blocks, const void* dO, void* dQ, void* dK, void* dV,
+                      void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of workspace needed by sattn_decode_fwd for *p (p->T = cache length). */
 int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
 

@@ -11,6 +11,7 @@ Public calls (names follow the C ABI):
     build_blockmap(is_sep, ...)  -> dict(cls, sep_pos, sep_count, qtile_sep_range)
     build_blockmap_noalloc(...)  -> the same, scratch inside the library (no workspace)
     segment_fwd(q, k, v, ...)    -> (O, lse, prefix_blocks)
+    segment_bwd(q, k, v, o, lse, prefix_blocks, do, ...) -> (dq, dk, dv)
     stream_status(workspace)     -> device status code
 
 ``fwd`` and ``segment_fwd`` also accept host (CPU) tensors: the inputs are
@@ -27,7 +28,7 @@ import torch
 from . import _lib
 from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
 
-__all__ = ["fwd", "topk_select", "build_blockmap", "build_blockmap_noalloc", "segment_fwd", "stream_status", "workspace_size",
+__all__ = ["fwd", "topk_select", "build_blockmap", "build_blockmap_noalloc", "segment_fwd", "segment_bwd", "stream_status", "workspace_size",
            "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout",
            "decode_fwd"]
 
@@ -231,6 +232,36 @@ def segment_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, S: int, M:
                                        _ptr(lse), _ptr(prefix), _ptr(ws), nbytes, _stream_ptr(q.device))
     _lib.check(rc, "sattn_segment_fwd")
     return out, lse, prefix[..., :nb]
+
+
+def segment_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                prefix_blocks: torch.Tensor, do: torch.Tensor, *, S: int, M: int, R: int, retr_block: int, is_long,
+                rope_theta: float = 0.0, rope_pos_scale: float = 1.0, workspace: Optional[torch.Tensor] = None,
+                grads: Optional[tuple] = None):
+    """Backward pass of ``segment_fwd``: gradients of sum(do * o), the
+    forward's retrieval (``prefix_blocks``) held fixed.  Returns (dq, dk, dv)
+    shaped and strided like q, k, v."""
+    if do.stride() != o.stride() or do.dtype != o.dtype or do.shape != o.shape:
+        raise ValueError("do must match o in shape, dtype and strides")
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    for g, x in ((dq, q), (dk, k), (dv, v)):
+        if g.stride() != x.stride():
+            raise ValueError("gradient buffers must share the strides of their inputs")
+    il_list = [int(x) for x in (is_long.tolist() if hasattr(is_long, "tolist") else is_long)]
+    il = (ctypes.c_uint8 * len(il_list))(*il_list)
+    p = params(q, k, v, o, rope_theta=rope_theta, rope_pos_scale=rope_pos_scale)
+    n = ctypes.c_size_t(0)
+    L = _lib.load()
+    _lib.check(L.sattn_segment_bwd_workspace_size(ctypes.byref(p), S, M, R, retr_block, ctypes.byref(n)),
+               "sattn_segment_bwd_workspace_size")
+    nbytes = int(n.value)
+    ws = _workspace(nbytes, q.device, workspace)
+    pb = prefix_blocks.to(torch.int32).contiguous()
+    rc = L.sattn_segment_bwd(ctypes.byref(p), S, M, R, retr_block, il, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                             _ptr(lse), _ptr(pb), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), nbytes,
+                             _stream_ptr(q.device))
+    _lib.check(rc, "sattn_segment_bwd")
+    return dq, dk, dv
 
 
 def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, window: int = 0,

@@ -24,6 +24,7 @@ DTYPE_F32 = 1
 EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
+    "sattn_segment_bwd_workspace_size", "sattn_segment_bwd",
     "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_bwd_workspace_size", "sattn_bwd",
     "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd", "sattn_stream_state_size", "sattn_stream_reset",
     "sattn_stream_append", "sattn_stream_read", "sattn_stream_decode_workspace_size", "sattn_stream_decode",
@@ -86,6 +87,10 @@ def load():
         L.sattn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sattn_segment_fwd.restype = ctypes.c_int
         L.sattn_segment_fwd.argtypes = [P, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sattn_segment_bwd_workspace_size.restype = ctypes.c_int
+        L.sattn_segment_bwd_workspace_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
+        L.sattn_segment_bwd.restype = ctypes.c_int
+        L.sattn_segment_bwd.argtypes = [P, i32, i32, i32, i32] + [vp] * 11 + [vp, sz, vp]
         L.sattn_decode_workspace_size.restype = ctypes.c_int
         L.sattn_decode_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_decode_fwd.restype = ctypes.c_int

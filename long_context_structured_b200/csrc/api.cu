@@ -780,6 +780,111 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
 }
 
 // ---------------------------------------------------------------------------
+// segmented execution: backward
+// ---------------------------------------------------------------------------
+
+struct SegBwdPlan {
+  Region status, tab, dsum;
+  size_t total = 0;
+};
+
+static int plan_seg_bwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t blk, SegBwdPlan* out) {
+  SegPlan F;
+  int rc = plan_seg(p, S, M, R, blk, nullptr, &F);  // the forward's rules
+  if (rc) return rc;
+  SegBwdPlan P;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  if (p->rope_theta != 0.0) P.tab = A.take((size_t)p->T * (p->d / 2) * sizeof(float2));
+  P.dsum = A.take((size_t)p->B * p->Hq * p->T * 4);
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_segment_bwd_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                                     size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  SegBwdPlan P;
+  int rc = plan_seg_bwd(p, S, M, R, retr_block, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_segment_bwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                      const uint8_t* is_long, const void* Q, const void* K, const void* V, const void* O,
+                      const float* lse, const int32_t* prefix_blocks, const void* dO, void* dQ, void* dK, void* dV,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (!is_long) return SATTN_ERR_INVALID_ARG;
+  SegBwdPlan P;
+  int rc = plan_seg_bwd(p, S, M, R, retr_block, &P);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV) return SATTN_ERR_INVALID_ARG;
+  if (R > 0 && !prefix_blocks) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  if (P.tab.bytes) {
+    ProfScope ps("rope_table", 1, st);
+    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), p->T, p->d, p->rope_theta, pos_scale(p), st));
+  }
+  SegBwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.d = p->d;
+  a.S = S;
+  a.N = p->T / S;
+  a.M = M;
+  a.R = R;
+  a.blk = retr_block;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.O = static_cast<const __nv_bfloat16*>(O);
+  a.dO = static_cast<const __nv_bfloat16*>(dO);
+  a.q_sb = p->q_stride[0];
+  a.q_sh = p->q_stride[1];
+  a.q_st = p->q_stride[2];
+  a.k_sb = p->k_stride[0];
+  a.k_sh = p->k_stride[1];
+  a.k_st = p->k_stride[2];
+  a.v_sb = p->v_stride[0];
+  a.v_sh = p->v_stride[1];
+  a.v_st = p->v_stride[2];
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.prefix_blocks = prefix_blocks;
+  for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
+  {
+    int slot = 0;
+    for (int h = 0; h < p->Hq; ++h)
+      if (is_long[h]) a.long_slot[h] = (int16_t)slot++;
+  }
+  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  a.Dsum = at<float>(ws, P.dsum);
+  a.dQ = static_cast<__nv_bfloat16*>(dQ);
+  a.dK = static_cast<__nv_bfloat16*>(dK);
+  a.dV = static_cast<__nv_bfloat16*>(dV);
+  a.dq_sb = p->q_stride[0];
+  a.dq_sh = p->q_stride[1];
+  a.dq_st = p->q_stride[2];
+  a.dk_sb = p->k_stride[0];
+  a.dk_sh = p->k_stride[1];
+  a.dk_st = p->k_stride[2];
+  a.dv_sb = p->v_stride[0];
+  a.dv_sh = p->v_stride[1];
+  a.dv_st = p->v_stride[2];
+  ProfScope ps("segment_bwd", 2, st);
+  return cuda_rc(launch_segment_bwd(a, st));
+}
+
+// ---------------------------------------------------------------------------
 // SharedLLM tree cross-attention
 // ---------------------------------------------------------------------------
 

@@ -374,6 +374,28 @@ size_t segment_score_bytes(int B, int n_long, int N, int T, int blk);
 bool segment_retrieval_supported(int T, int S, int blk);
 cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st);
 
+// backward of segmented execution (CUDA cores)
+struct SegBwdArgs {
+  int B, Hq, Hkv, T, d, S, N, M, R, blk;
+  float scale_log2;            // log2(e) / sqrt(d)
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const __nv_bfloat16* O;
+  const __nv_bfloat16* dO;     // strides of O
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st, o_sb, o_sh, o_st;
+  const float* lse;            // [B, Hq, T]
+  const int32_t* prefix_blocks;  // [B, Hq, N, R/blk], the forward's retrieval (-1: none)
+  int16_t long_slot[kMaxHeads];  // head -> index among long heads, -1 for local
+  const float2* tab;           // rotary table over positions [0, T) (null: no rotation)
+  float* Dsum;                 // [B, Hq, T] dO_i . O_i
+  __nv_bfloat16* dQ;           // strides of Q
+  __nv_bfloat16* dK;           // strides of K
+  __nv_bfloat16* dV;           // strides of V
+  int64_t dq_sb, dq_sh, dq_st, dk_sb, dk_sh, dk_st, dv_sb, dv_sh, dv_st;
+};
+cudaError_t launch_segment_bwd(const SegBwdArgs& a, cudaStream_t st);
+
 // ---------------------------------------------------------------------------
 // decoding step: one query per (batch, head) at position T - 1
 // ---------------------------------------------------------------------------
