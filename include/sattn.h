@@ -155,8 +155,11 @@ int sattn_topk_select(const sattn_params* p, const void* Q, const void* K, const
  *   lse         [B, Hq, T] float, out: natural-log logsumexp of the scaled
  *               logits of each row.
  * bf16 runs on the tensor cores; fp32 runs on the CUDA cores in fp32.
- * With bf16 and L_pretrain > 0: window <= L_pretrain, and when separators
- * or top-k are used, window == L_pretrain. */
+ * With bf16 and L_pretrain > 0: window <= L_pretrain, and with top-k
+ * window == L_pretrain.  Separators may sit on either side of the cap when
+ * window < L_pretrain: those with window < i - j <= L_pretrain take the
+ * uncapped logit, the farther ones the capped one.
+ * SATTN_ERR_UNSUPPORTED otherwise. */
 int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
               const int32_t* topk_idx, const float* topk_logit, void* O, float* lse, void* ws, size_t ws_bytes,
               void* stream);

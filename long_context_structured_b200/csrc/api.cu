@@ -55,6 +55,15 @@ struct Alloc {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// bf16 with separators, a cap and a window below it: separators with
+// w < i - j <= L are uncapped and go through the band tiles (which then
+// reach back to i - L), those with i - j > L through the compacted capped
+// tiles, so the block map's separator ranges are taken at distance L
+bool sep_band_extended(const sattn_params* p) {
+  return p->dtype == SATTN_DTYPE_BF16 && p->with_separators && p->L_pretrain > 0 && p->window < p->L_pretrain;
+}
+int sep_split_of(const sattn_params* p) { return sep_band_extended(p) ? p->L_pretrain : p->window; }
+
 int check_common(const sattn_params* p) {
   if (!p) return SATTN_ERR_INVALID_ARG;
   if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->T < 1) return SATTN_ERR_INVALID_ARG;
@@ -92,8 +101,9 @@ int check_fwd_rules(const sattn_params* p) {
   if (p->dtype == SATTN_DTYPE_BF16) {
     if (p->n_start > 256) return SATTN_ERR_UNSUPPORTED;
     if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
-    if (p->L_pretrain > 0 && (p->with_separators || p->topk > 0) && p->window != p->L_pretrain)
-      return SATTN_ERR_UNSUPPORTED;
+    // top-k candidates are scored with one operand pair: every candidate
+    // must be past the cap (w = L) or none capped (L = 0)
+    if (p->L_pretrain > 0 && p->topk > 0 && p->window != p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
     if (p->Hq > 65535) return SATTN_ERR_UNSUPPORTED;
   }
   return SATTN_OK;
@@ -114,7 +124,7 @@ int plan_fwd(const sattn_params* p, FwdPlan* pl) {
   Alloc A;
   P.status = A.take(kStatusBytes);
   if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
-  P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
+  P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, std::max(p->window, sep_split_of(p))));
   if (P.bf16) {
     P.qr = A.take(B * Hq * T * d * 2);
     P.kr = A.take(B * Hkv * T * d * 2);
@@ -291,12 +301,12 @@ int run_prep_bf16(const sattn_params* p, const FwdPlan& P, const void* Q, const 
 }
 
 int run_blockmap(const sattn_params* p, const FwdPlan& P, const uint8_t* is_sep, uint8_t* cls, int32_t* sep_pos,
-                 int32_t* sep_count, int32_t* ranges, void* ws, cudaStream_t st) {
+                 int32_t* sep_count, int32_t* ranges, void* ws, cudaStream_t st, int window = -1) {
   BlockmapArgs a{};
   a.B = p->B;
   a.T = p->T;
   a.n_start = p->n_start;
-  a.window = p->window;
+  a.window = window >= 0 ? window : p->window;
   a.is_sep = is_sep;
   a.scratch = at<uint8_t>(ws, P.prefix);
   a.sep_pos = sep_pos;
@@ -526,7 +536,7 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   m.vg = m.v;
   bool q2 = false;
   if (is_sep) {
-    rc = run_blockmap(p, P, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
+    rc = run_blockmap(p, P, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st, sep_split_of(p));
     if (rc) return rc;
     GatherArgs ga{};
     ga.B = p->B;
@@ -594,7 +604,8 @@ int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V
   a.sep_pos = sep_pos;
   a.sep_words = at<uint2>(ws, P.prefix);
   a.ranges = ranges;
-  a.window = p->window;
+  a.window = sep_split_of(p);
+  a.w_sepband = (is_sep && sep_band_extended(p)) ? p->L_pretrain : 0;
   for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.o_sb = p->o_stride[0];
@@ -1070,7 +1081,7 @@ static int plan_bwd(const sattn_params* p, BwdPlan* out) {
   F.status = A.take(kStatusBytes);
   if (p->rope_theta != 0.0) F.tab = A.take((size_t)F.npos * (d / 2) * sizeof(float2));
   if (p->with_separators) {
-    F.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
+    F.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, std::max(p->window, sep_split_of(p))));
     F.sep_pos = A.take(B * T * 4);
     F.sep_count = A.take(B * 4);
     F.ranges = A.take(B * F.nQT * 2 * 4);
@@ -1135,7 +1146,7 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   int32_t* sep_count = at<int32_t>(ws, F.sep_count);
   int32_t* ranges = at<int32_t>(ws, F.ranges);
   if (is_sep) {
-    rc = run_blockmap(p, F, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st);
+    rc = run_blockmap(p, F, is_sep, nullptr, sep_pos, sep_count, ranges, ws, st, sep_split_of(p));
     if (rc) return rc;
     GatherArgs ga{};
     ga.B = p->B;
@@ -1182,6 +1193,8 @@ static int run_bwd_bf16(const sattn_params* p, const BwdPlan& P, const void* Q, 
   a.n_start = p->n_start;
   a.window = p->window;
   a.L = p->L_pretrain;
+  a.sep_split = sep_split_of(p);
+  a.w_sepband = (is_sep && sep_band_extended(p)) ? p->L_pretrain : 0;
   a.alibi = p->alibi ? 1 : 0;
   a.alibi_cap = p->L_pretrain;
   a.tab = F.tab.bytes ? at<float2>(ws, F.tab) : nullptr;

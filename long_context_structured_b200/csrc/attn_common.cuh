@@ -63,7 +63,7 @@ __device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t
   }
   p.n_gather = (p.g_count + kTile - 1) / kTile;
   const int i_last = i0 + p.rows - 1;
-  const int j_lo = max(max(p.band_lo, 0), max(i0 - a.w_eff, a.ns_band));
+  const int j_lo = max(max(p.band_lo, 0), max(i0 - max(a.w_eff, a.w_sepband), a.ns_band));
   if (j_lo > i_last || a.gather_mode == 3) {
     p.u_lo = 0;
     p.n_band = 0;

@@ -329,14 +329,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r0 + kTile > pl.g_full) {
           int lim = min(kTile, pl.g_count - r0);
           if (a.gather_mode == 1) {
-            // separators kept by row i: pos < i - w; their count is a prefix count
+            // gathered separators kept by row i: pos < i - window (window = L
+            // when the band keeps the nearer ones); a prefix count
             const int thr = i - a.window;
             const int cnt = thr > 0 ? sep_before(a.sep_words, a.T, b, thr) : 0;
             lim = max(0, min(lim, cnt - r0));
           }
           c_hi = lim - 1;
         }
-      } else {
+      }
+      uint64_t xm = 0;  // separators kept beyond the window (this lane's 64 columns)
+      if (j >= pl.n_gather) {
         const int j0 = (pl.u_lo + j - pl.n_gather) * kTile;
         const int lo_fix = max(pl.band_lo, a.ns_band);
         const bool full = (j0 + kTile - 1 <= i0) && (j0 >= max(lo_fix, i0 + kTile - 1 - a.w_eff)) &&
@@ -345,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           c_lo = max(lo_fix, i - a.w_eff) - j0;
           c_hi = i - j0;
         }
+        if (a.w_sepband > a.w_eff)  // window below the cap: uncapped separators i - L <= j < i - w
+          xm = sep_bits64(a.sep_words, a.T, b, j0 + 64 * hc, max(lo_fix, i - a.w_sepband), i - a.w_eff - 1);
       }
       // this lane's columns are 64*hc + [0, 64)
       c_lo -= 64 * hc;
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (partial) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (c < c_lo || c > c_hi) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
+          if ((c < c_lo || c > c_hi) && !((xm >> c) & 1ull)) sv[c] = -CUDART_INF_F;  // exp2(-inf) = 0 below
       }
       if constexpr (kAlibi) {
         // ALiBi bias in units of q.k: band keys -m (i - j) (inside the window,

@@ -81,7 +81,7 @@ __device__ __forceinline__ QPlan make_qplan(const BwdArgs& a, int b, int t) {
   }
   if (a.dq_mode == 0) {
     const int i_last = i0 + rows - 1;
-    const int j_lo = max(i0 - a.window, a.n_start);
+    const int j_lo = max(i0 - max(a.window, a.w_sepband), a.n_start);
     if (j_lo <= i_last) {
       p.u_lo = j_lo / kTile;
       p.n_band = i_last / kTile - p.u_lo + 1;
@@ -295,15 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r0 = j * kTile;
         if (r0 + kTile > pl.g_full) {
           int lim = min(kTile, pl.g_count - r0);
-          const int thr = i - a.window;  // separators kept by row i: pos < i - w
+          const int thr = i - a.sep_split;  // compacted separators kept by row i: pos < i - split
           const int cnt = thr > 0 ? sep_before(a.sep_words, a.T, b, thr) : 0;
           lim = max(0, min(lim, cnt - r0));
           c_hi = lim - 1;
         }
-      } else {
+      }
+      uint64_t xm = 0;  // uncapped separators beyond the window (this lane's 64 columns)
+      if (j >= pl.n_gather) {
         const int j0 = (pl.u_lo + j - pl.n_gather) * kTile;
         c_lo = max(a.n_start, i - a.window) - j0;
         c_hi = i - j0;
+        if (a.w_sepband > a.window)
+          xm = sep_bits64(a.sep_words, a.T, b, j0 + 64 * hc, max(a.n_start, i - a.w_sepband), i - a.window - 1);
       }
       c_lo -= 64 * hc;
       c_hi -= 64 * hc;
@@ -324,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 #pragma unroll
-      for (int c = 0; c < 64; ++c) sv[c] = (c < c_lo || c > c_hi) ? 0.f : ex2_approx(fmaf(sv[c], sl2, nl2));
+      for (int c = 0; c < 64; ++c)
+        sv[c] = ((c < c_lo || c > c_hi) && !((xm >> c) & 1ull)) ? 0.f : ex2_approx(fmaf(sv[c], sl2, nl2));
       ok = ok && mbar_wait(dp_full, j & 1, abort_flag, a.status, 67);
       tc_fence_after();
       float dp[64];
@@ -484,13 +489,13 @@ __device__ __forceinline__ KVPlan make_kvplan(const BwdArgs& a, int b, int tile_
     const int j_hi = min(p.tile * kTile + kTile, a.T) - 1;
     if (j_lo > j_hi) return p;
     p.t_lo = j_lo / kTile;
-    const int t_hi = min(a.nQT - 1, (j_hi + a.window) / kTile);
+    const int t_hi = min(a.nQT - 1, (j_hi + max(a.window, a.w_sepband)) / kTile);
     p.n_t = t_hi - p.t_lo + 1;
   } else {
     const int cnt = a.sep_count[b];
     if (p.tile * kTile >= cnt) return p;
     const int j_first = a.sep_pos[(size_t)b * a.T + p.tile * kTile];
-    const int i_first = j_first + a.window + 1;
+    const int i_first = j_first + a.sep_split + 1;
     if (i_first >= a.T) return p;
     p.t_lo = i_first / kTile;
     p.n_t = a.nQT - p.t_lo;
@@ -683,6 +688,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       j = a.sep_pos[(size_t)b * a.T + pl.tile * kTile + rr];
     }
     const bool live = j >= 0 && (pl.sep || j >= a.n_start);  // band rows of sink keys take no part
+    // a band key that is a separator kept by the band beyond the window
+    bool key_sep = false;
+    if (!pl.sep && live && a.w_sepband > a.window) {
+      const uint2 wd = a.sep_words[(size_t)b * (a.T / 32 + 1) + (j >> 5)];
+      key_sep = ((wd.y >> (j & 31)) & 1u) != 0;
+    }
     bool ok = true;
     for (int s = 0; s < n; ++s) {
       const int h = g * rep + s / pl.n_t;
@@ -692,16 +703,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* dss = nls + kTile;
       ok = ok && mbar_wait(s_full, s & 1, abort_flag, a.status, 75);
       tc_fence_after();
-      // kept columns [c_lo, c_hi]: band rows j <= i <= j + w; separators i > j + w
+      // kept columns [c_lo, c_hi]: band rows j <= i <= j + w (j + w_sepband
+      // for a separator when the band also carries the uncapped ones);
+      // compacted separators i > j + split
       int c_lo, c_hi;
       if (!live) {
         c_lo = 1;
         c_hi = 0;
       } else if (!pl.sep) {
         c_lo = j - ic;
-        c_hi = j + a.window - ic;
+        c_hi = j + (key_sep ? a.w_sepband : a.window) - ic;
       } else {
-        c_lo = j + a.window + 1 - ic;
+        c_lo = j + a.sep_split + 1 - ic;
         c_hi = 63;
       }
       c_hi = min(c_hi, a.T - 1 - ic);

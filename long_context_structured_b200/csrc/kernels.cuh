@@ -70,6 +70,20 @@ __device__ __forceinline__ int sep_before(const uint2* words, int T, int b, int 
   return (int)e.x + __popc(e.y & ((1u << (x & 31)) - 1u));
 }
 
+// Bit c (c < 64): position j64 + c (j64 a multiple of 32) is a separator
+// j >= n_start with lo <= j64 + c <= hi.
+__device__ __forceinline__ uint64_t sep_bits64(const uint2* words, int T, int b, int j64, int lo, int hi) {
+  if (hi < lo || hi < j64 || lo > j64 + 63) return 0ull;
+  const uint2* wb = words + (size_t)b * (T / 32 + 1);
+  const int w0 = j64 >> 5;
+  const uint64_t m0 = w0 <= T / 32 ? __ldg(wb + w0).y : 0u;
+  const uint64_t m1 = w0 + 1 <= T / 32 ? __ldg(wb + w0 + 1).y : 0u;
+  uint64_t m = m0 | m1 << 32;
+  const int a = max(0, lo - j64), e = min(63, hi - j64);  // keep bits [a, e]
+  m &= (e == 63 ? ~0ull : ((1ull << (e + 1)) - 1ull)) & ~((1ull << a) - 1ull);
+  return m;
+}
+
 // ---------------------------------------------------------------------------
 // K3: separator K/V gather into dense per-(b, kv-head) arrays
 // ---------------------------------------------------------------------------
@@ -95,6 +109,9 @@ struct AttnArgs {
   // band tiles over the main K/V
   int ns_band;       // keys j < ns_band never go through the band (sinks use the side path)
   int w_eff;         // band keeps j >= i - w_eff
+  int w_sepband;     // > w_eff: band tiles reach back to i - w_sepband and also keep the separators
+                     // with i - w_sepband <= j < i - w_eff (the uncapped ones when the window is
+                     // below the cap); 0 otherwise
   // side keys (fp32 logits)
   const float* sink_z;  // [B, Hq, T, n_sink]
   int n_sink;
@@ -241,6 +258,9 @@ struct BwdArgs {
   int B, Hq, Hkv, T, d, nQT, Tpad;
   float scale_log2;             // log2(e) / sqrt(d)
   int n_start, window, L;       // L: distance cap (0 = none)
+  int sep_split;                // separators with i - j > sep_split go through the compacted tiles
+  int w_sepband;                // > window: band tiles reach back to i - w_sepband for the separators
+                                // with window < i - j <= w_sepband; 0 otherwise
   int alibi, alibi_cap;
   const float2* tab;            // rotary table (null: no rotation)
   // the forward's inputs and outputs (raw layouts, explicit strides)

@@ -126,6 +126,14 @@ BF16_CASES = [
                                 rope_theta=1e4, sep_rate=0.1, sink_scale=8.0)),
     ("sinks40_d64_uncapped", dict(B=1, Hq=2, Hkv=1, T=500, d=64, n_start=40, window=30, rope_theta=5e5,
                                   sep_rate=0.1)),
+    # separators with the window below the cap: the uncapped ones (w < i - j
+    # <= L) in the band tiles, the capped ones in the compacted tiles
+    ("sep_window_below_cap", dict(B=1, Hq=2, Hkv=2, T=700, d=128, n_start=4, window=50, L_pretrain=130,
+                                  rope_theta=1e4, sep_rate=0.15)),
+    ("sep_window_below_cap_d64_gqa", dict(B=2, Hq=4, Hkv=2, T=600, d=64, n_start=2, window=30, L_pretrain=200,
+                                          rope_theta=5e5, sep_rate=0.2)),
+    ("alibi_sep_window_below_cap", dict(B=1, Hq=4, Hkv=1, T=500, d=128, n_start=4, window=40, L_pretrain=150,
+                                        sep_rate=0.2, alibi=True)),
     # top-k middle keys (fp32 side keys, the selection a constant): capped
     # (L = w), with separators, uncapped (L = 0), and with the clipped ALiBi bias
     ("topk_capped_sinks_gqa", dict(B=1, Hq=4, Hkv=2, T=700, d=128, n_start=4, window=64, L_pretrain=64,

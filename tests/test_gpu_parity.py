@@ -229,6 +229,16 @@ SMALL = [
                                     sink_scale=8.0, alibi=True)),
     ("alibi_sep_capped_even", dict(B=1, Hq=2, Hkv=1, T=1024, d=128, n_start=4, window=128, L_pretrain=128,
                                    sep_rate=0.1, alibi=True)),
+    # separators with the window below the cap: those with w < i - j <= L
+    # are uncapped and ride in the band tiles, the farther ones capped
+    ("sep_window_below_cap", dict(B=1, Hq=2, Hkv=2, T=900, d=128, n_start=4, window=64, L_pretrain=128,
+                                  rope_theta=1e4, sep_rate=0.1)),
+    ("sep_window_below_cap_d64_gqa", dict(B=2, Hq=4, Hkv=2, T=700, d=64, n_start=2, window=30, L_pretrain=200,
+                                          rope_theta=5e5, sep_rate=0.2)),
+    ("alibi_sep_window_below_cap", dict(B=1, Hq=4, Hkv=1, T=800, d=128, n_start=4, window=40, L_pretrain=150,
+                                        sep_rate=0.15, alibi=True)),
+    ("sep_window0_capped", dict(B=1, Hq=2, Hkv=2, T=600, d=128, n_start=4, window=0, L_pretrain=100,
+                                rope_theta=1e4, sep_rate=0.5)),
     # sink spans wider than 8: the 16-slot sink logits (9..16) and the
     # global-memory ones (> 16) in prep and in the attention epilogue
     ("sinks12_capped", dict(B=1, Hq=2, Hkv=1, T=1000, d=128, n_start=12, window=100, L_pretrain=100,
