@@ -15,10 +15,14 @@ each (whole job, all ranks), with tokens/s alongside.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload c2|c3|c4|c5]
 
-Multi-GPU: one process per GPU (torchrun); every rank runs its own
-independent problem (heads/batches are independent), so per-GPU work is
+Multi-GPU: one process per GPU (torchrun).  By default every rank runs its
+own independent problem (heads/batches are independent), so per-GPU work is
 fixed as N grows ("scaling": "weak") and no data-path collective exists;
 the only collectives are the barrier and the max-over-ranks of the timings.
+``--split heads`` instead splits ONE layer over the ranks by kv-head groups
+("scaling": "strong"): each rank computes its heads' block, and the blocks
+are all-gathered once after the timed steps (NCCL; its time reported apart
+as ``head_gather``).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores (rank 0
 only) on bounded row samples of the same workload.
@@ -157,7 +161,7 @@ def describe(wl) -> str:
     return s
 
 
-def config_dict(wl, pairs_per_rank, decode=False, n_copies=0, backward=False):
+def config_dict(wl, pairs_per_rank, decode=False, n_copies=0, backward=False, parallelism="dp1"):
     prefix = ("decoding step (one new token per sequence at position T-1) over the cache of " if decode else
               "backward pass (dQ, dK, dV of sum(dO*O); %d FLOPs per kept pair per d) of " % BWD_FLOPS_PER_PAIR_D
               if backward else "")
@@ -169,6 +173,7 @@ def config_dict(wl, pairs_per_rank, decode=False, n_copies=0, backward=False):
         c.update({"n_start": wl.n_start, "window": wl.window, "L_pretrain": wl.L_pretrain,
                   "rope_theta": wl.rope_theta, "topk": wl.topk})
     c["unmasked_pairs_per_rank"] = pairs_per_rank
+    c["parallelism"] = parallelism
     in_bytes = (wl.B * wl.Hq + 2 * wl.B * wl.Hkv) * wl.T * wl.d * 2
     if decode:
         c["l2"] = ("no flush: steps cycle through %d copies of the K/V cache, so successive steps read "
@@ -253,12 +258,20 @@ class Job:
     """Inputs of one workload on one rank (pinned host copies and device
     copies) and the hot-path call over them."""
 
-    def __init__(self, wl, seed, dev):
+    def __init__(self, wl, seed, dev, heads=None):
         import torch
 
         import long_context_structured_b200 as sa
-        self.sa, self.torch, self.wl, self.dev = sa, torch, wl, dev
         inp = synth.make_inputs(wl, seed=seed)
+        self.full_wl, self.full_inp = wl, inp
+        if heads is not None:
+            # this rank's block of one layer: query heads [q0, q1) and the kv
+            # heads [kv0, kv1) they read, cut from the full layer's inputs
+            q0, q1, kv0, kv1 = heads
+            cut = lambda a, lo, hi: np.ascontiguousarray(a[:, lo:hi])
+            inp = dict(inp, q=cut(inp["q"], q0, q1), k=cut(inp["k"], kv0, kv1), v=cut(inp["v"], kv0, kv1))
+            wl = wl.scaled(Hq=q1 - q0, Hkv=kv1 - kv0)
+        self.sa, self.torch, self.wl, self.dev = sa, torch, wl, dev
         self.inp = inp
         to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
         self.host = {x: to_t(inp[x]).pin_memory() for x in ("q", "k", "v")}
@@ -276,6 +289,7 @@ class Job:
                            rope_theta=wl.rope_theta, topk=wl.topk)
         self.pairs = unmasked_pairs(wl, inp["is_sep"])
         self.flops = 4.0 * wl.d * self.pairs
+        self.full_flops = 4.0 * wl.d * unmasked_pairs(self.full_wl, inp["is_sep"]) if heads is not None else None
         self.n_sep = 0 if inp["is_sep"] is None else int(inp["is_sep"][:, wl.n_start:].sum())
 
     def step(self):
@@ -715,7 +729,17 @@ def run_ours(args):
     if args.heads:
         wl = wl.scaled(Hq=args.heads, Hkv=max(1, args.heads * wl.Hkv // wl.Hq),
                        long_heads=tuple(h for h in wl.long_heads if h < args.heads))
-    job = (DecodeJob if decode else (BwdJob if backward else Job))(wl, seed=rank, dev=dev)
+    split = args.split == "heads"
+    if split:
+        # one layer split over the ranks by kv-head groups (strong scaling)
+        if decode or backward or wl.segmented:
+            raise SystemExit("--split heads runs the prefill workloads c2, c3 and c4")
+        if world > wl.Hkv:
+            raise SystemExit("--split heads needs at most Hkv = %d ranks" % wl.Hkv)
+        from long_context_structured_b200.shard import head_shard
+        job = Job(wl, seed=0, dev=dev, heads=head_shard(wl.Hq, wl.Hkv, world, rank))
+    else:
+        job = (DecodeJob if decode else (BwdJob if backward else Job))(wl, seed=rank, dev=dev)
     lib = _lib.load()
 
     for _ in range(args.warmup):
@@ -742,8 +766,10 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step = float(t.item()) / args.steps
-    value = job.flops * world / (ms_step * 1e-3) / 1e12
-    tokens_s = wl.B * (1 if decode else wl.T) * world / (ms_step * 1e-3)
+    # whole-job work: every rank's own problem (weak), or the one split layer (strong)
+    job_flops = job.full_flops if split else job.flops * world
+    value = job_flops / (ms_step * 1e-3) / 1e12
+    tokens_s = wl.B * (1 if decode else wl.T) * (1 if split else world) / (ms_step * 1e-3)
 
     # per-group device time per step (every group runs once per step; a group
     # may hold more than one kernel), max over ranks (same group order on
@@ -793,7 +819,7 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     ms_e2e = float(te.item())
-    e2e = {"value": round(job.flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    e2e = {"value": round(job_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
            "ms_per_step": round(ms_e2e, 3), "steps": n_e2e, "h2d_bytes_per_step": job.h2d_bytes(),
            "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)),
            "path": ("long_context_structured_b200.decode_fwd: query from pinned host memory, device-resident cache, "
@@ -802,6 +828,26 @@ def run_ours(args):
                     "into pinned host memory") if backward else
                    ("long_context_structured_b200.%s on pinned host tensors (outputs into pinned host memory)"
                     % ("segment_fwd" if wl.segmented else "fwd"))}
+
+    gather = None
+    if split and world > 1:
+        # the head blocks back into one layer on every rank (NCCL all-gather),
+        # once, outside the timed steps
+        from long_context_structured_b200.shard import gather_heads
+        full = job.full_wl
+        gather_heads(job.O, job.lse, full.Hq, full.Hkv, world)  # warm the communicator
+        torch.cuda.synchronize()
+        dist.barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        O_full, _ = gather_heads(job.O, job.lse, full.Hq, full.Hkv, world)
+        g1.record()
+        torch.cuda.synchronize()
+        tg = torch.tensor([g0.elapsed_time(g1)], dtype=torch.float64, device=dev)
+        dist.all_reduce(tg, op=dist.ReduceOp.MAX)
+        gather = {"ms": round(float(tg.item()), 4), "bytes_per_rank_out": int(job.O.nbytes + job.lse.nbytes),
+                  "full_shape": list(O_full.shape), "note": "all_gather of O and LSE, not in the step time"}
+        del O_full
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -815,10 +861,14 @@ def run_ours(args):
     peak = float(peaks["bf16_tflops"])
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "f32" if wl.dtype == "f32" else "bf16",
         "data": "synthetic (seeded N(0,1)%s)" % ("; keys 0-3 x8" if wl.sink_scale != 1.0 else ""),
-        "config": config_dict(wl, job.pairs, decode=decode, n_copies=getattr(job, "n_copies", 0), backward=backward),
+        "config": config_dict(job.full_wl if split else wl, job.pairs, decode=decode,
+                              n_copies=getattr(job, "n_copies", 0), backward=backward,
+                              parallelism=("heads%d (kv-head groups of one layer per rank)" % world) if split else
+                              ("dp%d (an independent layer per rank)" % world)),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_bf16_peak": round(value / world / peak, 4),
         "roofline": roof,
@@ -831,6 +881,8 @@ def run_ours(args):
         "clocks": clk,
         "device_status": status,
     }
+    if gather is not None:
+        line["head_gather"] = gather
     print(json.dumps(line), flush=True)
 
 
@@ -1264,6 +1316,9 @@ def main():
                     help="rows in the CPU-oracle baseline sample (default: 6144 on the top-k workload, else 32768)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling captures only)")
+    ap.add_argument("--split", choices=["none", "heads"], default="none",
+                    help="none: an independent layer per rank (weak scaling); heads: one layer split over the "
+                         "ranks by kv-head groups (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -44,6 +44,10 @@ def sharded_fwd(q, k, v, *, world: int, rank: int, compute: Optional[Callable] =
 
     if compute is None:
         from . import fwd as compute
+    if kw.get("alibi"):
+        # the ALiBi slope of a head depends on its index among all Hq heads,
+        # which a head block run on its own does not know
+        raise NotImplementedError("head sharding with ALiBi is not supported")
     Hq, Hkv = q.shape[1], k.shape[1]
     q0, q1, kv0, kv1 = head_shard(Hq, Hkv, world, rank)
     if q1 > q0:
@@ -53,9 +57,17 @@ def sharded_fwd(q, k, v, *, world: int, rank: int, compute: Optional[Callable] =
         lse = torch.empty((q.shape[0], 0, q.shape[2]), dtype=torch.float32, device=q.device)
     if not gather:
         return O, lse, (q0, q1)
+    O_full, l_full = gather_heads(O, lse, Hq, Hkv, world, group=group)
+    return O_full, l_full, (0, Hq)
+
+
+def gather_heads(O, lse, Hq: int, Hkv: int, world: int, group=None):
+    """All-gather every rank's head block (O [B, h_r, T, d], lse [B, h_r, T])
+    into the full layer in head order.  Blocks are padded to the largest so
+    that one all_gather of equal shapes moves them."""
+    import torch
     import torch.distributed as dist
 
-    # pad every block to the largest so all_gather sees equal shapes
     sizes = [head_shard(Hq, Hkv, world, r)[1] - head_shard(Hq, Hkv, world, r)[0] for r in range(world)]
     hmax = max(sizes)
     Op = O.new_zeros((O.shape[0], hmax, O.shape[2], O.shape[3]))
@@ -68,7 +80,7 @@ def sharded_fwd(q, k, v, *, world: int, rank: int, compute: Optional[Callable] =
     dist.all_gather(ls, lp.contiguous(), group=group)
     O_full = torch.cat([Os[r][:, : sizes[r]] for r in range(world)], dim=1)
     l_full = torch.cat([ls[r][:, : sizes[r]] for r in range(world)], dim=1)
-    return O_full, l_full, (0, Hq)
+    return O_full, l_full
 
 
 def max_over_ranks(value: float, group=None, device=None) -> float:
