@@ -139,7 +139,9 @@ int sattn_build_blockmap(const sattn_params* p, const uint8_t* is_sep, uint8_t* 
  *   idx        [B, Hq, T, topk] int32, out: selected j sorted by (z desc, j asc);
  *              -1 when fewer than topk candidates exist.
  *   logit      [B, Hq, T, topk] float, out: z_ij in fp32; -inf for padding.
- * bf16 only.  Requires L_pretrain == 0 or L_pretrain == window. */
+ * bf16 only.  With 0 < window < L_pretrain a candidate with i - j <= L_pretrain
+ * is scored with the uncapped logit <R(i) q, R(j) k>, a farther one with the
+ * capped <R(L) q, k>. */
 int sattn_topk_select(const sattn_params* p, const void* Q, const void* K, const uint8_t* is_sep,
                       int32_t* idx, float* logit, void* ws, size_t ws_bytes, void* stream);
 
@@ -155,11 +157,10 @@ int sattn_topk_select(const sattn_params* p, const void* Q, const void* K, const
  *   lse         [B, Hq, T] float, out: natural-log logsumexp of the scaled
  *               logits of each row.
  * bf16 runs on the tensor cores; fp32 runs on the CUDA cores in fp32.
- * With bf16 and L_pretrain > 0: window <= L_pretrain, and with top-k
- * window == L_pretrain.  Separators may sit on either side of the cap when
- * window < L_pretrain: those with window < i - j <= L_pretrain take the
- * uncapped logit, the farther ones the capped one.
- * SATTN_ERR_UNSUPPORTED otherwise. */
+ * With bf16 and L_pretrain > 0: window <= L_pretrain (SATTN_ERR_UNSUPPORTED
+ * otherwise).  Separators and top-k keys may sit on either side of the cap
+ * when window < L_pretrain: those with window < i - j <= L_pretrain take the
+ * uncapped logit, the farther ones the capped one. */
 int sattn_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
               const int32_t* topk_idx, const float* topk_logit, void* O, float* lse, void* ws, size_t ws_bytes,
               void* stream);

@@ -101,9 +101,6 @@ int check_fwd_rules(const sattn_params* p) {
   if (p->dtype == SATTN_DTYPE_BF16) {
     if (p->n_start > 256) return SATTN_ERR_UNSUPPORTED;
     if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
-    // top-k candidates are scored with one operand pair: every candidate
-    // must be past the cap (w = L) or none capped (L = 0)
-    if (p->L_pretrain > 0 && p->topk > 0 && p->window != p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
     if (p->Hq > 65535) return SATTN_ERR_UNSUPPORTED;
   }
   return SATTN_OK;
@@ -363,13 +360,17 @@ int run_topk(const sattn_params* p, const FwdPlan& P, const void* Q, const void*
   }
   TopkMaps m;
   const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  // uncapped operands (R(i) q, R(j) k): the only pair when L = 0, the pair of
+  // the candidates within the cap when 0 < w < L
+  if (!make_map(&m.qsel2, at<void>(ws, P.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.ksel2, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
   if (p->L_pretrain > 0) {
     if (!make_map(&m.qsel, at<void>(ws, P.qc), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
     if (!make_map(&m.ksel, K, p->d, p->T, Hkv, B, p->k_stride[2], p->k_stride[1], p->k_stride[0]))
       return SATTN_ERR_CUDA;
   } else {
-    if (!make_map(&m.qsel, at<void>(ws, P.qr), p->d, p->T, Hq, B, d, T * d, Hq * T * d)) return SATTN_ERR_CUDA;
-    if (!make_map(&m.ksel, at<void>(ws, P.kr), p->d, p->T, Hkv, B, d, T * d, Hkv * T * d)) return SATTN_ERR_CUDA;
+    m.qsel = m.qsel2;
+    m.ksel = m.ksel2;
   }
   {
     ProfScope ps("topk_score", 1, st);

@@ -359,6 +359,7 @@ struct TopkArgs {
 constexpr int kCandCap = 128;
 struct TopkMaps {
   CUtensorMap qsel, ksel;      // bf16 scoring operands: (Qc, K) capped, (Qr, Kr) otherwise
+  CUtensorMap qsel2, ksel2;    // with 0 < window < L: (Qr, Kr) for the pairs within the cap
 };
 // scoring on the tensor cores into per-row candidate lists
 cudaError_t launch_topk_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st);

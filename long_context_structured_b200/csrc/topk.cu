@@ -146,9 +146,19 @@ __device__ __forceinline__ void insert_val(float v, float (&s)[R]) {
   }
 }
 
-template <int D>
+// kDual (a cap with the window below it, 0 < w < L): candidates with
+// i - j <= L take the uncapped logit <R(i) q, R(j) k>, the farther ones the
+// capped <R(L) q, k>.  A CTA then takes ONE query tile and stages both of
+// its scoring queries (Qc in the first query slot, Qr in the second); a key
+// tile whose pairs are all capped is scored as Qc K^T, one whose pairs are
+// all within the cap as Qr Kr^T, and a tile that straddles the cap both ways
+// (two K ring entries, the products in the first and the idle second query
+// tile's TMEM buffers), the scan warps taking each column from the product
+// that holds its row's logit.
+template <int D, bool kDual>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmQ2, const __grid_constant__ CUtensorMap tmK2,
                       const TopkArgs a, int nQB) {
   constexpr int kSt = kStagesK;
   constexpr int kR = kSampleKeep;
@@ -177,13 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.x / nQB;
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
+  // query tiles of this CTA: 2 qb and 2 qb + 1, or the one tile qb (kDual)
+  auto qtile = [&](int x) { return kDual ? qb : 2 * qb + x; };
   // key tiles each query tile scans: [u_lo, u_lo + nt[x]); the union is the longer
   const int u_lo = a.n_start / kTile;
   int nt[2];
   for (int x = 0; x < 2; ++x) {
-    const int i0x = (2 * qb + x) * kTile;
+    const int i0x = qtile(x) * kTile;
     nt[x] = 0;
-    if (i0x < a.T) {
+    if ((!kDual || x == 0) && i0x < a.T) {
       const int hi_key = min(a.T - 1, i0x + kTile - 1) - a.window - 1;
       if (hi_key >= a.n_start) nt[x] = hi_key / kTile - u_lo + 1;
     }
@@ -196,6 +208,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_s = (ntiles + stride - 1) / stride;
   const int n_steps = ntiles > 0 ? n_s + ntiles : 0;
   auto tile_of = [&](int it) { return it < n_s ? it * stride : it - n_s; };
+  // kDual: 0 = every pair of the key tile capped, 1 = every pair within the
+  // cap, 2 = both (rows past the sequence end count as rows; they keep nothing)
+  auto ttype = [&](int t) -> int {
+    if (!kDual) return 0;
+    const int i0d = qb * kTile;
+    const int j0 = (u_lo + t) * kTile;
+    if (i0d - (j0 + kTile - 1) > a.L) return 0;
+    if (i0d + kTile - 1 - j0 <= a.L) return 1;
+    return 2;
+  };
 
   if (threadIdx.x == 0) {
     *early = status_failed(a.status) ? 1 : 0;
@@ -231,18 +253,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(q_full, 2 * kTileBytes);
       for (int x = 0; x < 2; ++x)
         for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sq + x * kTileBytes + c * kChunkBytes, &tmQ, q_full, c * 64, (2 * qb + x) * kTile, h, b);
+          tma_load_4d(sq + x * kTileBytes + c * kChunkBytes, (kDual && x == 1) ? &tmQ2 : &tmQ, q_full, c * 64,
+                      qtile(x) * kTile, h, b);
+      // ring entries: one K tile per step (raw K, or Kr for a tile within
+      // the cap), two for a straddling tile (raw K, then Kr)
       int issued = 0;
       bool ok = true;
-      for (int it = 0; it < n_steps; ++it) {
-        const int st = it % kSt;
-        if (it >= kSt) ok = mbar_wait(k_empty + st, ((it / kSt) - 1) & 1, abort_flag, a.status, 21);
-        if (!ok) break;
-        mbar_expect_tx(k_full + st, kTileBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_4d(sk + st * kTileBytes + c * kChunkBytes, &tmK, k_full + st, c * 64,
-                      (u_lo + tile_of(it)) * kTile, g, b);
-        ++issued;
+      for (int it = 0; it < n_steps && ok; ++it) {
+        const int ty = ttype(tile_of(it));
+        for (int e = 0; e < (ty == 2 ? 2 : 1); ++e) {
+          const int st = issued % kSt;
+          if (issued >= kSt) ok = mbar_wait(k_empty + st, ((issued / kSt) - 1) & 1, abort_flag, a.status, 21);
+          if (!ok) break;
+          mbar_expect_tx(k_full + st, kTileBytes);
+          const CUtensorMap* km = (ty == 1 || e == 1) ? &tmK2 : &tmK;
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_4d(sk + st * kTileBytes + c * kChunkBytes, km, k_full + st, c * 64,
+                        (u_lo + tile_of(it)) * kTile, g, b);
+          ++issued;
+        }
       }
       if (!ok) {
         mbar_wait_raw(q_full, 0);
@@ -256,43 +285,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = smem_u32(sq);
       bool ok = mbar_wait(q_full, 0, abort_flag, a.status, 22);
       int cnt[2] = {0, 0};  // score tiles produced per query tile
+      int used = 0;         // K ring entries consumed
+      auto mma_tile = [&](uint32_t d_tmem, uint32_t qa, uint32_t ka) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          tc_mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idesc,
+                    kk > 0 ? 1u : 0u);
+        }
+      };
       for (int it = 0; it < n_steps && ok; ++it) {
-        const int st = it % kSt;
-        ok = mbar_wait(k_full + st, (it / kSt) & 1, abort_flag, a.status, 23);
-        if (!ok) break;
         const int t = tile_of(it);
+        const int ty = ttype(t);
+        const int st = used % kSt, st2 = (used + 1) % kSt;
+        ok = mbar_wait(k_full + st, (used / kSt) & 1, abort_flag, a.status, 23);
+        if (ok && ty == 2) ok = mbar_wait(k_full + st2, ((used + 1) / kSt) & 1, abort_flag, a.status, 23);
+        if (!ok) break;
         const uint32_t k_addr = smem_u32(sk + st * kTileBytes);
-        for (int x = 0; x < 2 && ok; ++x) {
+        for (int x = 0; x < (kDual ? 1 : 2) && ok; ++x) {
           if (t >= nt[x]) continue;
           const int c = cnt[x]++;
           const int sb = c % kSBuf;
           if (c >= kSBuf) ok = mbar_wait(s_free + x * kSBuf + sb, ((c / kSBuf) - 1) & 1, abort_flag, a.status, 24);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t qx = q_addr + x * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            tc_mma_ss(tmem + (x * kSBuf + sb) * 128, smem_desc_sw128(qx + off, 16, 1024),
-                      smem_desc_sw128(k_addr + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-          }
+          // the query slot: the tile's own, or in kDual Qc (slot 0) / Qr (slot 1)
+          const int slot = kDual ? (ty == 1 ? 1 : 0) : x;
+          mma_tile(tmem + (x * kSBuf + sb) * 128, q_addr + slot * kTileBytes, k_addr);
+          if (kDual && ty == 2)  // the within-cap product into the idle second tile's buffer
+            mma_tile(tmem + (kSBuf + sb) * 128, q_addr + kTileBytes, smem_u32(sk + st2 * kTileBytes));
           tc_commit(s_full + x * kSBuf + sb);
         }
         tc_commit(k_empty + st);
+        if (ty == 2) tc_commit(k_empty + st2);
+        used += ty == 2 ? 2 : 1;
       }
       tc_commit(drain);
       mbar_wait_raw(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 16) {
+  } else if (warp < 16 && !(kDual && ((warp >> 2) & 1))) {
     // scan warps: warp w scans query tile qt = (w / 4) % 2, rows 32 (w % 4)
     // .. + 31 of it (TMEM lanes of the warp's quarter), columns 64 ch .. + 63
     // of every key tile, ch = w / 8; the two threads of a row (warps w and
-    // w ^ 8) share the row's threshold and its candidate list
+    // w ^ 8) share the row's threshold and its candidate list (kDual: the
+    // second tile's warps idle)
     const int qt = (warp >> 2) & 1;
     const int ch = warp >> 3;
     const int rl = (warp & 3) * 32 + lane;  // row within the query tile
-    const int i0 = (2 * qb + qt) * kTile;
+    const int i0 = qtile(qt) * kTile;
     const int i = i0 + rl;
     const int ntx = nt[qt];
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -341,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int t = tile_of(it);
       if (t >= ntx) continue;
+      const int ty = ttype(t);
       const bool sample = it < n_s;
       const int sb = cx % kSBuf;
       ok = ok && mbar_wait(s_full + qt * kSBuf + sb, (cx / kSBuf) & 1, abort_flag, a.status, 25);
@@ -356,8 +398,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c2 = 0; c2 < 2; ++c2) {
         const int cb = ch * 64 + c2 * 32;  // first column of this 32-column chunk
         float v[32];
-        tmem_ld32(tmem + (qt * kSBuf + sb) * 128 + lane_off + cb, v);
-        tc_wait_ld();
+        const uint32_t tb = tmem + (qt * kSBuf + sb) * 128 + lane_off + cb;
+        if (kDual && ty == 2) {
+          // columns j >= i - L hold their logit in the second product
+          const int yc = i - a.L - (j0 + cb);
+          if (__all_sync(0xffffffffu, yc <= 0)) {
+            tmem_ld32(tb + kSBuf * 128, v);
+            tc_wait_ld();
+          } else {
+            tmem_ld32(tb, v);
+            if (__any_sync(0xffffffffu, yc < 32)) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                float w16[16];
+                tmem_ld16(tb + kSBuf * 128 + 16 * hh, w16);
+                tc_wait_ld();
+#pragma unroll
+                for (int y = 0; y < 16; ++y)
+                  if (16 * hh + y >= yc) v[16 * hh + y] = w16[y];
+              }
+            } else {
+              tc_wait_ld();
+            }
+          }
+        } else {
+          tmem_ld32(tb, v);
+          tc_wait_ld();
+        }
         if (c2 == 1) {
           tc_fence_before();
           if (ok) mbar_arrive(s_free + qt * kSBuf + sb);
@@ -496,12 +563,13 @@ __device__ __forceinline__ float exact_logit_bf16(const __nv_bfloat16* kp, const
 constexpr int kRerankWarps = 8;
 constexpr int kPerLane = kCandCap / 32;
 
-template <int D>
+template <int D, bool kDual>
 __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const TopkArgs a) {
   constexpr int half = D / 2;
   constexpr int PPL = half / 32;   // rotary pairs staged per lane
   constexpr int QP = half / 4;     // rotary pairs per lane of a 4-lane group
   __shared__ __align__(16) float sq[kRerankWarps][D];
+  __shared__ __align__(16) float sqc[kDual ? kRerankWarps : 1][kDual ? D : 4];  // R(L) q when 0 < w < L
   __shared__ int sj[kRerankWarps][kCandCap];
   __shared__ float2 se[kRerankWarps][kCandCap];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -512,7 +580,9 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   const int64_t bh = row / a.T;
   const int h = (int)(bh % a.Hq), b = (int)(bh / a.Hq);
   const int g = h / (a.Hq / a.Hkv);
-  const bool capped_all = a.L > 0;  // capped scoring requires L == window: every candidate is capped
+  // w >= L: every candidate is capped; 0 < w < L: those with i - j <= L are not
+  constexpr bool dual = kDual;  // the launch picks it: a.L > 0 && a.window < a.L
+  const bool capped_all = a.L > 0 && !dual;
   const int cnt = a.cand_cnt[row];
   const float tau = a.cand_thr[row];
   const int k = a.topk;
@@ -535,8 +605,9 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   }
   const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(a.Q) + b * a.q_sb + h * a.q_sh +
                             (int64_t)i * a.q_st;
-  // stage the scoring query and measure its bf16 rounding
-  float dq2 = 0.f, qn2 = 0.f;
+  // stage the scoring query (and with 0 < w < L the capped one as well) and
+  // measure their bf16 rounding
+  float dq2 = 0.f, qn2 = 0.f, dq2c = 0.f, qn2c = 0.f;
 #pragma unroll
   for (int e = 0; e < PPL; ++e) {
     const int cc = lane * PPL + e;
@@ -549,16 +620,32 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     const float b0 = __bfloat162float(__float2bfloat16_rn(u0)), b1 = __bfloat162float(__float2bfloat16_rn(u1));
     dq2 += (u0 - b0) * (u0 - b0) + (u1 - b1) * (u1 - b1);
     qn2 += b0 * b0 + b1 * b1;
+    if constexpr (kDual) {
+      const float2 cl = a.tab ? a.tab[(int64_t)a.L * half + cc] : make_float2(1.f, 0.f);
+      const float w0 = x0 * cl.x - x1 * cl.y, w1 = x1 * cl.x + x0 * cl.y;
+      sqc[wid][cc] = w0;
+      sqc[wid][cc + half] = w1;
+      const float c0 = __bfloat162float(__float2bfloat16_rn(w0)), c1 = __bfloat162float(__float2bfloat16_rn(w1));
+      dq2c += (w0 - c0) * (w0 - c0) + (w1 - c1) * (w1 - c1);
+      qn2c += c0 * c0 + c1 * c1;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     dq2 += __shfl_xor_sync(0xffffffffu, dq2, o);
     qn2 += __shfl_xor_sync(0xffffffffu, qn2, o);
+    dq2c += __shfl_xor_sync(0xffffffffu, dq2c, o);
+    qn2c += __shfl_xor_sync(0xffffffffu, qn2c, o);
   }
   const float kmax = __uint_as_float(a.kmax[(size_t)b * a.Hkv + g]) * (1.f + 1.f / 128.f);
   const float qn = sqrtf(qn2);
   float eps = sqrtf(dq2) * kmax + qn * kmax * (1.f / 32768.f);
   if (!capped_all) eps += qn * kmax * (1.f / 256.f);  // rotated keys were rounded too
+  if constexpr (kDual) {
+    // the capped scores' bound (unrotated keys are exact)
+    const float qnc = sqrtf(qn2c);
+    eps = fmaxf(eps, sqrtf(dq2c) * kmax + qnc * kmax * (1.f / 32768.f));
+  }
   eps *= 1.0625f;
 
   // c' = the k-th largest lane maximum (-inf when fewer than k lanes hold entries)
@@ -587,7 +674,6 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   __syncwarp();
   // fp32 logits: four lanes per entry, a quarter of the rotary pairs each
   const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.K) + b * a.k_sb + g * a.k_sh;
-  const float* qv = sq[wid];
   const int quarter = lane & 3;
   for (int e0 = 0; e0 < m; e0 += 8) {
     const int e = e0 + (lane >> 2);
@@ -595,6 +681,13 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     int j = -1;
     if (e < m) {
       j = sj[wid][e];
+      // the pair's operands: capped (R(L) q, raw key) or rotated (R(i) q, R(j) k)
+      bool cap = capped_all;
+      const float* qv = sq[wid];
+      if constexpr (kDual) {
+        cap = i - j > a.L;
+        if (cap) qv = sqc[wid];
+      }
       const __nv_bfloat16* kp = kbase + (int64_t)j * a.k_st;
       float A0 = 0.f, A1 = 0.f;
 #pragma unroll
@@ -612,7 +705,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
           k1[2 * y] = r.x;
           k1[2 * y + 1] = r.y;
         }
-        if (!capped_all && a.tab) {
+        if (!cap && a.tab) {
           const float4* t = reinterpret_cast<const float4*>(a.tab + (int64_t)j * half + c0);
 #pragma unroll
           for (int y = 0; y < 4; ++y) {
@@ -797,17 +890,19 @@ __global__ void __launch_bounds__(kExactThreads) topk_exact_kernel(const TopkArg
   }
 }
 
-template <int D>
+template <int D, bool kDual>
 cudaError_t launch_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
   const size_t tile = (size_t)D * kTile * 2;
   // Q tiles, K ring, scan scratch, barriers; at least 116 KB: one CTA per SM, so the
   // 512-column TMEM allocation never waits
   const size_t bytes =
       std::max<size_t>(116 * 1024, 1024 + tile * (2 + kStagesK) + 512 * kScratchStride * 4 + 256 * 4 + 256);
-  cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  cudaError_t e =
+      cudaFuncSetAttribute(topk_score_kernel<D, kDual>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  const int nQB = (a.nQT + 1) / 2;
-  topk_score_kernel<D><<<(unsigned)(a.B * a.Hq * nQB), kThreads, bytes, st>>>(m.qsel, m.ksel, a, nQB);
+  const int nQB = kDual ? a.nQT : (a.nQT + 1) / 2;
+  topk_score_kernel<D, kDual>
+      <<<(unsigned)(a.B * a.Hq * nQB), kThreads, bytes, st>>>(m.qsel, m.ksel, m.qsel2, m.ksel2, a, nQB);
   return cudaGetLastError();
 }
 
@@ -815,8 +910,9 @@ cudaError_t launch_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) 
 
 cudaError_t launch_topk_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t st) {
   if ((int64_t)a.B * a.Hq * a.T == 0) return cudaSuccess;
-  if (a.d == 128) return launch_score<128>(a, m, st);
-  if (a.d == 64) return launch_score<64>(a, m, st);
+  const bool dual = a.L > 0 && a.window < a.L;
+  if (a.d == 128) return dual ? launch_score<128, true>(a, m, st) : launch_score<128, false>(a, m, st);
+  if (a.d == 64) return dual ? launch_score<64, true>(a, m, st) : launch_score<64, false>(a, m, st);
   return cudaErrorInvalidValue;
 }
 
@@ -824,9 +920,16 @@ cudaError_t launch_topk_rerank(const TopkArgs& a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.B * a.Hq * a.T;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((rows + kRerankWarps - 1) / kRerankWarps);
-  if (a.d == 128) topk_rerank_kernel<128><<<blocks, kRerankWarps * 32, 0, st>>>(a);
-  else if (a.d == 64) topk_rerank_kernel<64><<<blocks, kRerankWarps * 32, 0, st>>>(a);
-  else return cudaErrorInvalidValue;
+  const bool dual = a.L > 0 && a.window < a.L;
+  if (a.d == 128) {
+    if (dual) topk_rerank_kernel<128, true><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+    else topk_rerank_kernel<128, false><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+  } else if (a.d == 64) {
+    if (dual) topk_rerank_kernel<64, true><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+    else topk_rerank_kernel<64, false><<<blocks, kRerankWarps * 32, 0, st>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

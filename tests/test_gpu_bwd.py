@@ -143,6 +143,8 @@ BF16_CASES = [
     ("topk_uncapped_k8", dict(B=1, Hq=2, Hkv=2, T=500, d=128, n_start=4, window=40, rope_theta=1e4, topk=8)),
     ("topk_alibi", dict(B=1, Hq=4, Hkv=1, T=400, d=128, n_start=4, window=64, L_pretrain=64, topk=3,
                         alibi=True)),
+    ("topk_window_below_cap_sep", dict(B=1, Hq=2, Hkv=2, T=700, d=128, n_start=4, window=50, L_pretrain=130,
+                                       rope_theta=1e4, topk=4, sep_rate=0.1)),
     ("topk16_sinks20_sep", dict(B=1, Hq=2, Hkv=2, T=640, d=128, n_start=20, window=48, L_pretrain=48,
                                 rope_theta=1e4, topk=16, sep_rate=0.05)),
 ]

@@ -321,6 +321,15 @@ TOPK_CASES = [
                           rope_theta=1e4, topk=4, plant=2, sink_scale=8.0)),
     ("topk_uncapped_k16_separators", dict(B=1, Hq=2, Hkv=2, T=1200, d=128, n_start=4, window=100,
                                           rope_theta=1e4, topk=16, sep_rate=0.05)),
+    # the window below the cap: candidates with w < i - j <= L scored with the
+    # uncapped pair, the farther ones capped, key tiles straddling i - L both
+    # ways; long rows (sampled threshold), short rows (every tile sampled)
+    ("topk_window_below_cap_sep", dict(B=1, Hq=4, Hkv=2, T=4096, d=128, n_start=4, window=256, L_pretrain=512,
+                                       rope_theta=1e4, topk=5, plant=4, sep_rate=0.1)),
+    ("topk_window_below_cap_d64_k8", dict(B=2, Hq=2, Hkv=1, T=2048, d=64, n_start=4, window=100, L_pretrain=300,
+                                          rope_theta=5e5, topk=8, plant=2)),
+    ("topk_window_below_cap_short", dict(B=1, Hq=2, Hkv=2, T=1000, d=128, n_start=2, window=50, L_pretrain=200,
+                                         rope_theta=1e4, topk=4, sep_rate=0.05)),
 ]
 
 
