@@ -47,7 +47,7 @@ sys.path.insert(0, ROOT)
 from long_context_structured_b200 import synth  # noqa: E402
 
 # decoding steps (one new token per sequence) over the caches of these workloads
-DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k"}
+DECODE_ALIASES = {"c2d": "c2_lminf_16k", "c3d": "c3_sepllm_gqa_8k", "c4d": "c4_lminf_topk_32k"}
 BWD_ALIASES = {"c2b": "c2_lminf_16k", "c3b": "c3_sepllm_gqa_8k"}
 # stress sizes for the HBM-bound helpers: the block map on B*T = 2^26 flags
 # (a2s) and the separator gather on the SepLLM layer at 16x its batch (c3x16)
@@ -375,8 +375,15 @@ class DecodeJob:
         self.qd = self.host["q"].to(dev)
         self.O = torch.empty_like(self.qd)
         self.lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
-        self.kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta)
+        self.kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta,
+                       topk=wl.topk)
         self.pairs = int(keys.sum()) * wl.Hq
+        if wl.topk > 0:
+            # top-k: every middle candidate's K row is scored (read once per
+            # kv group), and k more kept keys per head
+            ncand = max(0, wl.T - 1 - wl.window - wl.n_start)
+            self.kv_bytes += wl.B * wl.Hkv * ncand * wl.d * 2
+            self.pairs += wl.B * wl.Hq * min(wl.topk, ncand)
         self.flops = 4.0 * wl.d * self.pairs
         self.n_step = 0
 
@@ -685,6 +692,8 @@ def kernel_name(wl, group):
     if group == "attn_tc_cross":
         return "attn_tc2_kernel<%d>" % TREE_WORKLOADS["tree_cross_128k"]["d"]
     d = wl.d if wl is not None else 128
+    if group == "decode" and wl is not None and wl.topk > 0:
+        return "decode_topk_logits_kernel + decode_topk_select_kernel + decode_partial_kernel + decode_combine_kernel"
     return {"prep_rope": "prep_kernel", "topk_score": "topk_score_kernel<%d>" % d, "topk_rerank": "topk_rerank_kernel<%d>" % d, "tree_prep": "tree_prep_kernel",
             "decode": "decode_partial_kernel + decode_combine_kernel",
             "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % d,

@@ -221,8 +221,9 @@ int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
  * window i-w <= j <= i ("LM-Infinite", section 方法), earlier separators
  * n_start <= j < i-w ("SepLLM", section 五.2), the capped logit
  * <R(L) q, k_j> for i-j > L_pretrain and <R(i) q, R(j) k_j> otherwise.
- *   p        shape and mask parameters; T is the cache length, topk must be
- *            0, Hq/Hkv one of 1, 2, 4, 8, bf16 only.
+ *   p        shape and mask parameters; T is the cache length, Hq/Hkv one
+ *            of 1, 2, 4, 8, bf16 only.  topk > 0 adds the query's top-k
+ *            middle tokens as in sattn_fwd (see sattn_decode_topk_fwd).
  *   Q        [B, Hq, 1, d] bf16 device, strides q_stride[0..1].
  *   K, V     [B, Hkv, T, d] bf16 device cache (keys unrotated), strides as
  *            in sattn_fwd.
@@ -234,6 +235,24 @@ int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
  * Asynchronous on `stream`; validation as sattn_fwd. */
 int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
                      void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* sattn_decode_fwd that also returns the top-k selection of the decoding
+ * query ("LM-Infinite", section 方法, optional top-k, applied at generation):
+ * per query head the p->topk candidates n_start <= j < i-w (i = T-1) that are
+ * not separators with the largest unscaled logit z_ij (the capped one past
+ * L_pretrain), ties to the smaller j, computed in fp32 from the raw inputs;
+ * they join the step's key set with those logits.
+ *   topk_idx    [B, Hq, topk] int32 device, out, or NULL: positions sorted by
+ *               (z desc, j asc); -1 when fewer than topk candidates exist.
+ *   topk_logit  [B, Hq, topk] float device, out, or NULL: z; -inf padding.
+ * Every candidate key row is read once per kv-head group (a logit pass over
+ * the middle of the cache), then a block per (batch, head) selects and adds
+ * the selected keys' partial to the chunk merge.  SATTN_ERR_UNSUPPORTED with
+ * ALiBi unless L_pretrain > 0 and window >= L_pretrain.  Other arguments as
+ * sattn_decode_fwd. */
+int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                          void* O, float* lse, int32_t* topk_idx, float* topk_logit, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* Bytes of workspace needed by sattn_bwd for *p. */
 int sattn_bwd_workspace_size(const sattn_params* p, size_t* bytes);

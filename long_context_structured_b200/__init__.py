@@ -267,9 +267,12 @@ def segment_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tens
 def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: int = 0, window: int = 0,
                L_pretrain: int = 0, rope_theta: float = 0.0, is_sep: Optional[torch.Tensor] = None,
                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-               workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False):
+               workspace: Optional[torch.Tensor] = None, rope_pos_scale: float = 1.0, alibi: bool = False,
+               topk: int = 0, return_topk: bool = False):
     """One decoding step: q [B, Hq, 1, d] is the query of the cache's last
-    position (k, v [B, Hkv, T, d]).  Returns (O [B, Hq, 1, d], lse [B, Hq])."""
+    position (k, v [B, Hkv, T, d]).  Returns (O [B, Hq, 1, d], lse [B, Hq]);
+    with topk > 0 the query's top-k middle tokens join its key set, and
+    return_topk adds their (idx [B, Hq, topk] int32, logit [B, Hq, topk])."""
     B, Hq, one, d = q.shape
     if one != 1:
         raise ValueError("decode_fwd takes one query per (batch, head): q is [B, Hq, 1, d]")
@@ -281,17 +284,23 @@ def decode_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_start: in
     if is_sep is not None:
         is_sep = is_sep.to(torch.uint8).contiguous()
     p = params(q, k, v, out, n_start=n_start, window=window, L_pretrain=L_pretrain, rope_theta=rope_theta,
-               with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale, alibi=alibi)
+               topk=topk, with_separators=is_sep is not None, rope_pos_scale=rope_pos_scale, alibi=alibi)
     p.T = T
     n = ctypes.c_size_t(0)
     L = _lib.load()
     _lib.check(L.sattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)), "sattn_decode_workspace_size")
     nbytes = int(n.value)
     ws = _workspace(nbytes, q.device, workspace)
-    rc = L.sattn_decode_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(out), _ptr(lse),
-                            _ptr(ws), nbytes, _stream_ptr(q.device))
-    _lib.check(rc, "sattn_decode_fwd")
-    return out, lse
+    idx = z = None
+    if return_topk:
+        if topk < 1:
+            raise ValueError("return_topk needs topk > 0")
+        idx = torch.empty((B, Hq, topk), dtype=torch.int32, device=q.device)
+        z = torch.empty((B, Hq, topk), dtype=torch.float32, device=q.device)
+    rc = L.sattn_decode_topk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(is_sep), _ptr(out), _ptr(lse),
+                                 _ptr(idx), _ptr(z), _ptr(ws), nbytes, _stream_ptr(q.device))
+    _lib.check(rc, "sattn_decode_topk_fwd")
+    return (out, lse, idx, z) if return_topk else (out, lse)
 
 
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,

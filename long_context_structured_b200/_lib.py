@@ -25,7 +25,8 @@ EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
     "sattn_segment_bwd_workspace_size", "sattn_segment_bwd",
-    "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_bwd_workspace_size", "sattn_bwd",
+    "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_decode_topk_fwd", "sattn_bwd_workspace_size",
+    "sattn_bwd",
     "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd", "sattn_stream_state_size", "sattn_stream_reset",
     "sattn_stream_append", "sattn_stream_read", "sattn_stream_decode_workspace_size", "sattn_stream_decode",
     "sattn_stream_status",
@@ -95,6 +96,8 @@ def load():
         L.sattn_decode_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_decode_fwd.restype = ctypes.c_int
         L.sattn_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sattn_decode_topk_fwd.restype = ctypes.c_int
+        L.sattn_decode_topk_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sattn_bwd_workspace_size.restype = ctypes.c_int
         L.sattn_bwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_bwd.restype = ctypes.c_int

@@ -940,7 +940,7 @@ static int plan_tree(const sattn_params* p, int32_t n_chunks, int32_t chunk_len,
 
 struct DecPlan {
   int nQT, npos, n_chunks;
-  Region status, tab, prefix, sep_pos, sep_count, ranges, part;
+  Region status, tab, prefix, sep_pos, sep_count, ranges, part, tk_zall, tk_idx, tk_z, tk_part;
   size_t total;
 };
 
@@ -948,7 +948,8 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   int rc = check_common(p);
   if (rc) return rc;
   if (p->dtype != SATTN_DTYPE_BF16) return SATTN_ERR_UNSUPPORTED;
-  if (p->topk != 0) return SATTN_ERR_UNSUPPORTED;
+  // top-k with ALiBi ranks by q.k only when every candidate is past the cap
+  if (p->alibi && p->topk > 0 && (p->L_pretrain == 0 || p->window < p->L_pretrain)) return SATTN_ERR_UNSUPPORTED;
   const int rep = p->Hq / p->Hkv;
   if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return SATTN_ERR_UNSUPPORTED;
   if (p->L_pretrain > 0 && p->window > p->L_pretrain) return SATTN_ERR_UNSUPPORTED;
@@ -968,6 +969,12 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
     P.ranges = A.take(B * P.nQT * 2 * 4);
   }
   P.part = A.take(B * Hq * (size_t)P.n_chunks * (d + 2) * 4);
+  if (p->topk > 0) {
+    P.tk_zall = A.take(B * Hq * T * 4);
+    P.tk_idx = A.take(B * Hq * (size_t)p->topk * 4);
+    P.tk_z = A.take(B * Hq * (size_t)p->topk * 4);
+    P.tk_part = A.take(B * Hq * (d + 2) * 4);
+  }
   P.total = A.cur;
   *out = P;
   return SATTN_OK;
@@ -984,6 +991,12 @@ int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes) {
 
 int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
                      void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return sattn_decode_topk_fwd(p, Q, K, V, is_sep, O, lse, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, const void* V, const uint8_t* is_sep,
+                          void* O, float* lse, int32_t* topk_idx, float* topk_logit, void* ws, size_t ws_bytes,
+                          void* stream) {
   DecPlan P;
   int rc = plan_decode(p, &P);
   if (rc) return rc;
@@ -995,10 +1008,12 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
   if (P.tab.bytes) {
     ProfScope ps("rope_table", 1, st);
-    if (is_sep) {
-      // separators can sit at any earlier position
+    if (is_sep || (p->topk > 0 && p->L_pretrain == 0)) {
+      // separators (or uncapped top-k candidates) can sit at any earlier position
       SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
     } else {
+      // (top-k candidates past the cap use row i - L, the nearer ones rows
+      // in [i - L, i - w): both inside the rows below)
       // the step reads the rows of the sinks (j, or i - L when capped), of
       // the window keys and of the query (i - w <= j <= i, uncapped since
       // w <= L), and row i - L: [0, n_start) and [i - max(w, L), T)
@@ -1042,11 +1057,19 @@ int sattn_decode_fwd(const sattn_params* p, const void* Q, const void* K, const 
   a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
   a.part = at<float>(ws, P.part);
   a.n_chunks = P.n_chunks;
+  if (p->topk > 0) {
+    a.topk = p->topk;
+    a.tk_zall = at<float>(ws, P.tk_zall);
+    a.tk_idx = topk_idx ? topk_idx : at<int32_t>(ws, P.tk_idx);
+    a.tk_z = topk_logit ? topk_logit : at<float>(ws, P.tk_z);
+    a.tk_part = at<float>(ws, P.tk_part);
+  }
   a.O = static_cast<__nv_bfloat16*>(O);
   a.o_sb = p->o_stride[0];
   a.o_sh = p->o_stride[1];
   a.lse = lse;
-  ProfScope ps("decode", 2, st);
+  const int n_topk_kernels = p->topk > 0 ? (p->T - 1 - p->window - p->n_start > 0 ? 2 : 1) : 0;
+  ProfScope ps("decode", 2 + n_topk_kernels, st);
   return cuda_rc(launch_decode(a, st));
 }
 

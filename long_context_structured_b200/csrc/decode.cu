@@ -24,6 +24,7 @@
 #include <math_constants.h>
 
 #include "kernels.cuh"
+#include "select.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
 
@@ -75,31 +76,56 @@ __device__ __forceinline__ int key_at(const DecodeArgs& a, const KeySet& s, int 
 // transposed butterfly over the key's lanes; logits to shared memory; (2)
 // with the chunk's per-head maximum and the weights p = 2^(z - m) taken once
 // per (key, head): O += p v.  No running rescale.
+// Lane layout of the logit pass.  A key is spread over LPK lanes (8, or 16
+// for eight query heads per kv head), each holding EPL rotary pairs (16 or 8
+// elements of the row), so a warp works on 32 / LPK keys at once with
+// 16-byte loads; KPW key slots per warp, UNR warp steps in flight.
 template <int D, int REP>
-__global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
-  constexpr int half = D / 2;
-  constexpr int LPK = (REP >= 8) ? 16 : 8;      // lanes per key
-  constexpr int KPS = 32 / LPK;                 // keys per warp step
-  constexpr int EPL = half / LPK;               // rotary pairs per lane
-  constexpr int KPW = kChunk / (kThreads / 32);  // keys per warp: 32
-  constexpr int UNR = (REP >= 4) ? 1 : 2;       // warp steps whose loads are in flight together
+struct Tiling {
+  static constexpr int half = D / 2;
+  static constexpr int LPK = (REP >= 8) ? 16 : 8;       // lanes per key
+  static constexpr int KPS = 32 / LPK;                  // keys per warp step
+  static constexpr int EPL = half / LPK;                // rotary pairs per lane
+  static constexpr int KPW = kChunk / (kThreads / 32);  // keys per warp: 32
+  static constexpr int UNR = (REP >= 4) ? 1 : 2;        // warp steps whose loads are in flight together
   static_assert(REP <= LPK && KPW % (KPS * UNR) == 0 && (EPL == 8 || EPL == 4 || EPL == 2), "decode tiling");
-  __shared__ float s_p[REP][kChunk];            // logits, then weights
-  __shared__ float s_m[REP], s_l[REP];
-  __shared__ float red_o[kThreads / 32][REP][D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane % LPK, kg = lane / LPK;
-  const int bg = blockIdx.x;
-  const int g = bg % a.Hkv, b = bg / a.Hkv;
-  const KeySet ks = key_set(a, b);
-  const int e_begin = blockIdx.y * kChunk;
-  if (e_begin >= ks.n()) return;  // this batch has fewer chunks
-  const int n_here = min(ks.n() - e_begin, kChunk);
-  const int i = cache_len(a, b) - 1;
-  const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
+};
 
-  // the query of each head rotated to i, fp32
-  float q0[REP][EPL], q1[REP][EPL];
+// EPL consecutive bf16 as floats (16, 8 or 4 bytes)
+template <int EPL>
+__device__ __forceinline__ void load_e(const __nv_bfloat16* p, float* out) {
+  if constexpr (EPL == 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const float2 f = __bfloat1622float2(h[y]);
+      out[2 * y] = f.x;
+      out[2 * y + 1] = f.y;
+    }
+  } else if constexpr (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int y = 0; y < 2; ++y) {
+      const float2 f = __bfloat1622float2(h[y]);
+      out[2 * y] = f.x;
+      out[2 * y + 1] = f.y;
+    }
+  } else {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    out[0] = f.x;
+    out[1] = f.y;
+  }
+}
+
+// This lane's pairs [p0, p0 + EPL) of the query of each head of kv group g,
+// rotated to i, in fp32.
+template <int D, int REP>
+__device__ __forceinline__ void rotated_query(const DecodeArgs& a, int b, int g, int i, int p0,
+                                              float (&q0)[REP][Tiling<D, REP>::EPL],
+                                              float (&q1)[REP][Tiling<D, REP>::EPL]) {
+  constexpr int half = D / 2, EPL = Tiling<D, REP>::EPL;
 #pragma unroll
   for (int r = 0; r < REP; ++r) {
     const __nv_bfloat16* qp = a.Q + (size_t)b * a.q_sb + (size_t)(g * REP + r) * a.q_sh;
@@ -111,51 +137,35 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       q1[r][e] = x1 * t.x + x0 * t.y;
     }
   }
-  const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
-  const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
-  const float sl2 = a.scale_log2;
-  const int w_lo = warp * KPW;
+}
 
-  // EPL consecutive bf16 as floats (16, 8 or 4 bytes)
-  auto load_e = [&](const __nv_bfloat16* p, float* out) {
-    if constexpr (EPL == 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const float2 f = __bfloat1622float2(h[y]);
-        out[2 * y] = f.x;
-        out[2 * y + 1] = f.y;
-      }
-    } else if constexpr (EPL == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(p);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int y = 0; y < 2; ++y) {
-        const float2 f = __bfloat1622float2(h[y]);
-        out[2 * y] = f.x;
-        out[2 * y + 1] = f.y;
-      }
-    } else {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-      out[0] = f.x;
-      out[1] = f.y;
-    }
-  };
-
-  // ---- pass 1: logits ----
+// The logit pass over one warp's KPW key slots [w_lo, w_lo + KPW): the raw
+// key rotated on the fly to R(j) k_j, or for a capped key (i - j > L) to
+// R(i - L) k_j, which gives the capped logit <R(L) q, k_j> = <R(i) q,
+// R(i - L) k_j> with the one query R(i) q; the lanes' partial dot products
+// of all heads summed by one transposed butterfly over the key's lanes.
+// key_of(slot) gives the slot's key position (-1: none); emit(r, slot, j,
+// dot) receives head r's unscaled logit on one lane per (key, head).
+template <int D, int REP, class KeyOf, class Emit>
+__device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __nv_bfloat16* kb, int w_lo,
+                                            int lane, const float (&q0)[REP][Tiling<D, REP>::EPL],
+                                            const float (&q1)[REP][Tiling<D, REP>::EPL], KeyOf key_of,
+                                            Emit emit) {
+  using TL = Tiling<D, REP>;
+  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, KPW = TL::KPW, UNR = TL::UNR;
+  const int sub = lane % LPK, kg = lane / LPK;
+  const int p0 = sub * EPL;
   for (int u0 = 0; u0 < KPW; u0 += KPS * UNR) {
     int jj[UNR];
     float k0[UNR][EPL], k1[UNR][EPL];
     float2 cs[UNR][EPL];
 #pragma unroll
     for (int x = 0; x < UNR; ++x) {
-      const int el = w_lo + u0 + x * KPS + kg;
-      jj[x] = (el < n_here) ? key_at(a, ks, b, e_begin + el) : -1;
+      jj[x] = key_of(w_lo + u0 + x * KPS + kg);
       const int j = jj[x] < 0 ? 0 : jj[x];
       const int rpos = (a.L > 0 && i - j > a.L) ? i - a.L : j;  // capped keys: R(i - L) k_j
-      load_e(kb + (size_t)j * a.k_st + p0, k0[x]);
-      load_e(kb + (size_t)j * a.k_st + p0 + half, k1[x]);
+      load_e<EPL>(kb + (size_t)j * a.k_st + p0, k0[x]);
+      load_e<EPL>(kb + (size_t)j * a.k_st + p0 + half, k1[x]);
       if (a.tab) {
         const float4* tp = reinterpret_cast<const float4*>(a.tab + (size_t)rpos * half + p0);
 #pragma unroll
@@ -184,18 +194,52 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       group_reduce_transposed<REP, LPK>(v, 0xffffffffu, lane);
       // lane sub now holds head sub / (LPK / REP)
       constexpr int DUP = LPK / REP;
-      if (sub % DUP == 0) {
-        const int r = sub / DUP;
-        const int j = jj[x];
-        float z = v[0] * sl2;
+      if (sub % DUP == 0) emit(sub / DUP, w_lo + u0 + x * KPS + kg, jj[x], v[0]);
+    }
+  }
+}
+
+// grid (B * Hkv, chunks): the (batch, kv head) index varies fastest, so the
+// chunks that hold keys (the low ones) are dispatched before the empty ones.
+// Two passes over the CTA's chunk of kept keys: (1) logits (logits_pass) to
+// shared memory; (2) with the chunk's per-head maximum and the weights
+// p = 2^(z - m) taken once per (key, head): O += p v.  No running rescale.
+template <int D, int REP>
+__global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
+  using TL = Tiling<D, REP>;
+  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, KPW = TL::KPW, UNR = TL::UNR;
+  __shared__ float s_p[REP][kChunk];            // logits, then weights
+  __shared__ float s_m[REP], s_l[REP];
+  __shared__ float red_o[kThreads / 32][REP][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPK, kg = lane / LPK;
+  const int bg = blockIdx.x;
+  const int g = bg % a.Hkv, b = bg / a.Hkv;
+  const KeySet ks = key_set(a, b);
+  const int e_begin = blockIdx.y * kChunk;
+  if (e_begin >= ks.n()) return;  // this batch has fewer chunks
+  const int n_here = min(ks.n() - e_begin, kChunk);
+  const int i = cache_len(a, b) - 1;
+  const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
+  float q0[REP][EPL], q1[REP][EPL];
+  rotated_query<D, REP>(a, b, g, i, p0, q0, q1);
+  const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
+  const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
+  const float sl2 = a.scale_log2;
+  const int w_lo = warp * KPW;
+
+  // ---- pass 1: logits ----
+  logits_pass<D, REP>(
+      a, i, kb, w_lo, lane, q0, q1,
+      [&](int el) { return el < n_here ? key_at(a, ks, b, e_begin + el) : -1; },
+      [&](int r, int el, int j, float dot) {
+        float z = dot * sl2;
         if (a.alibi && j >= 0) {  // -m_h * min(i - j, L), in log2 units of the scaled logit
           const int dist = (a.L > 0) ? min(i - j, a.L) : (i - j);
           z -= exp2f(-8.f * (float)(g * REP + r + 1) / (float)a.Hq) * 1.4426950408889634f * (float)dist;
         }
-        s_p[r][w_lo + u0 + x * KPS + kg] = (j >= 0) ? z : -CUDART_INF_F;
-      }
-    }
-  }
+        s_p[r][el] = (j >= 0) ? z : -CUDART_INF_F;
+      });
   __syncthreads();
   // ---- per-head maximum, weights and their sum (warp r takes heads r, r + 4, ...) ----
   for (int r = warp; r < REP; r += kThreads / 32) {
@@ -230,8 +274,8 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
     for (int x = 0; x < UNR; ++x) {
       els[x] = w_lo + u0 + x * KPS + kg;
       const int j = (els[x] < n_here) ? key_at(a, ks, b, e_begin + els[x]) : 0;
-      load_e(vb + (size_t)j * a.v_st + p0, v0[x]);
-      load_e(vb + (size_t)j * a.v_st + p0 + half, v1[x]);
+      load_e<EPL>(vb + (size_t)j * a.v_st + p0, v0[x]);
+      load_e<EPL>(vb + (size_t)j * a.v_st + p0 + half, v1[x]);
     }
 #pragma unroll
     for (int x = 0; x < UNR; ++x) {
@@ -280,6 +324,108 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
   }
 }
 
+// ---------------------------------------------------------------------------
+// top-k middle tokens of the decoding query ("LM-Infinite", section 方法,
+// optional top-k): candidates n_start <= j < i - w that are not separators,
+// ranked per query head by the unscaled logit (the capped one past L), ties
+// to the smaller position.  Reading every candidate key is what the method
+// asks for here; the K rows are read once per kv group.
+// ---------------------------------------------------------------------------
+
+// grid (B * Hkv, candidate chunks of kChunk positions): every candidate's
+// logit for every query head of the group (the logit pass over consecutive
+// positions) into tk_zall.  Separators are scored too and skipped by the
+// selection.
+template <int D, int REP>
+__global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs a) {
+  using TL = Tiling<D, REP>;
+  constexpr int EPL = TL::EPL, LPK = TL::LPK, KPW = TL::KPW;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x % a.Hkv, b = blockIdx.x / a.Hkv;
+  const int i = a.T - 1;
+  const int jend = i - a.window;  // candidates j < i - w
+  const int j0 = a.n_start + blockIdx.y * kChunk;
+  if (j0 >= jend) return;
+  const int p0 = (lane % LPK) * EPL;
+  float q0[REP][EPL], q1[REP][EPL];
+  rotated_query<D, REP>(a, b, g, i, p0, q0, q1);
+  const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
+  float* zb = a.tk_zall + ((size_t)b * a.Hq + (size_t)g * REP) * a.T;
+  logits_pass<D, REP>(
+      a, i, kb, warp * KPW, lane, q0, q1, [&](int el) { return j0 + el < jend ? j0 + el : -1; },
+      [&](int r, int, int j, float dot) {
+        if (j >= 0) zb[(size_t)r * a.T + j] = dot;
+      });
+}
+
+constexpr int kSelThreads = 512;
+constexpr int kSelMaxK = 16;
+
+// grid (B * Hq): the k best candidates of one (batch, head) -- a strided
+// pass keeping a sorted list per thread, then k rounds of a block argmax --
+// written out, and the selected keys' softmax partial (their maximum, sum of
+// weights and weighted V rows) for the chunk merge.
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeArgs a) {
+  __shared__ float red_z[kSelThreads / 32];
+  __shared__ int red_j[kSelThreads / 32];
+  __shared__ float s_z[kSelMaxK];
+  __shared__ int s_j[kSelMaxK];
+  const int bh = blockIdx.x;
+  const int b = bh / a.Hq, h = bh % a.Hq, g = h / (a.Hq / a.Hkv);
+  const int i = a.T - 1;
+  const int jend = i - a.window;
+  const float* zr = a.tk_zall + (size_t)bh * a.T;
+  const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
+  float vals[kSelMaxK];
+  int idxs[kSelMaxK];
+#pragma unroll
+  for (int y = 0; y < kSelMaxK; ++y) {
+    vals[y] = -CUDART_INF_F;
+    idxs[y] = -1;
+  }
+  // each thread visits its positions in increasing order, so a strict >
+  // leaves the smaller position first among equal logits
+  for (int j = a.n_start + (int)threadIdx.x; j < jend; j += kSelThreads) {
+    if (words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u)) continue;
+    const float z = zr[j];
+    if (z > vals[kSelMaxK - 1]) list_insert<kSelMaxK>(z, j, vals, idxs);
+  }
+  block_topk_rounds<kSelMaxK>(a.topk, vals, idxs, red_z, red_j, [&](int r, float wz, int wj) {
+    s_j[r] = wj;
+    s_z[r] = wj >= 0 ? wz : -CUDART_INF_F;
+  });
+  __syncthreads();
+  const int k = a.topk;
+  if ((int)threadIdx.x < k) {
+    a.tk_idx[(size_t)bh * k + threadIdx.x] = s_j[threadIdx.x];
+    a.tk_z[(size_t)bh * k + threadIdx.x] = s_z[threadIdx.x];
+  }
+  // scaled log2-unit logits of the picks; with ALiBi every candidate is
+  // past the cap (w >= L) and takes -m_h L
+  const float sl2 = a.scale_log2;
+  const float bias = a.alibi ? exp2f(-8.f * (float)(h + 1) / (float)a.Hq) * 1.4426950408889634f * (float)a.L : 0.f;
+  float m = -CUDART_INF_F;
+  for (int r = 0; r < k; ++r)
+    if (s_j[r] >= 0) m = fmaxf(m, s_z[r] * sl2 - bias);
+  float* part = a.tk_part + (size_t)bh * (D + 2);
+  const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
+  for (int c = threadIdx.x; c < D; c += kSelThreads) {
+    float l = 0.f, o = 0.f;
+    for (int r = 0; r < k; ++r) {
+      if (s_j[r] < 0) continue;
+      const float p = ex2_approx(s_z[r] * sl2 - bias - m);
+      l += p;
+      o = fmaf(p, __bfloat162float(vb[(size_t)s_j[r] * a.v_st + c]), o);
+    }
+    part[2 + c] = o;
+    if (c == 0) {
+      part[0] = m;
+      part[1] = l;
+    }
+  }
+}
+
 // grid (B * Hq), 4 D threads: merge the chunks of one (batch, head).  The
 // chunk maxima and weights are read in parallel into shared memory; thread
 // group q of 4 sums chunks q, q + 4, ... of each output column (independent
@@ -288,18 +434,21 @@ constexpr int kCombineGroups = 4;
 constexpr int kCombineMaxChunks = 4096;
 template <int D>
 __global__ void __launch_bounds__(kCombineGroups * D) decode_combine_kernel(DecodeArgs a) {
-  __shared__ float s_f[kCombineMaxChunks];
+  __shared__ float s_f[kCombineMaxChunks + 1];
   __shared__ float s_red[kCombineGroups * D];
   __shared__ float s_ml[2];
   const int bh = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq;
   const KeySet ks = key_set(a, b);
-  const int nc = min((ks.n() + kChunk - 1) / kChunk, kCombineMaxChunks);
-  const float* part = a.part + (size_t)bh * a.n_chunks * (D + 2);
+  const int nc0 = min((ks.n() + kChunk - 1) / kChunk, kCombineMaxChunks);
+  // the chunks' partials, then the top-k keys' one
+  const int nc = nc0 + (a.tk_part ? 1 : 0);
+  const float* part0 = a.part + (size_t)bh * a.n_chunks * (D + 2);
+  auto slot = [&](int x) { return x < nc0 ? part0 + (size_t)x * (D + 2) : a.tk_part + (size_t)bh * (D + 2); };
   const int tid = threadIdx.x;
   float mx = -CUDART_INF_F;
   for (int x = tid; x < nc; x += blockDim.x) {
-    s_f[x] = part[(size_t)x * (D + 2)];
+    s_f[x] = slot(x)[0];
     mx = fmaxf(mx, s_f[x]);
   }
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -316,7 +465,7 @@ __global__ void __launch_bounds__(kCombineGroups * D) decode_combine_kernel(Deco
   for (int x = tid; x < nc; x += blockDim.x) {
     const float f = (s_f[x] == -CUDART_INF_F) ? 0.f : ex2_approx(s_f[x] - M);
     s_f[x] = f;
-    lsum += part[(size_t)x * (D + 2) + 1] * f;
+    lsum += slot(x)[1] * f;
   }
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
   __syncthreads();  // s_red is reused
@@ -330,7 +479,7 @@ __global__ void __launch_bounds__(kCombineGroups * D) decode_combine_kernel(Deco
   const int q = tid / D, c = tid % D;
   float O = 0.f;
 #pragma unroll 4
-  for (int x = q; x < nc; x += kCombineGroups) O = fmaf(part[(size_t)x * (D + 2) + 2 + c], s_f[x], O);
+  for (int x = q; x < nc; x += kCombineGroups) O = fmaf(slot(x)[2 + c], s_f[x], O);
   __syncthreads();
   s_red[q * D + c] = O;
   __syncthreads();
@@ -354,9 +503,22 @@ cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
     const int win_lo = std::max(ns, i - a.window);
     chunks = std::min(chunks, std::max(1, (ns + std::max(0, i - win_lo + 1) + kChunk - 1) / kChunk));
   }
+  cudaError_t e;
+  if (a.topk > 0) {
+    const int ncand = a.T - 1 - a.window - a.n_start;
+    if (ncand > 0) {
+      dim3 gt(a.B * a.Hkv, (ncand + kChunk - 1) / kChunk);
+      decode_topk_logits_kernel<D, REP><<<gt, kThreads, 0, st>>>(a);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    decode_topk_select_kernel<D><<<a.B * a.Hq, kSelThreads, 0, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid(a.B * a.Hkv, chunks);
   decode_partial_kernel<D, REP><<<grid, kThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<D><<<a.B * a.Hq, kCombineGroups * D, 0, st>>>(a);
   return cudaGetLastError();

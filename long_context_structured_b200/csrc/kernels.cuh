@@ -437,6 +437,12 @@ struct DecodeArgs {
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
   int alibi;                    // ALiBi bias clipped at L (no rotation)
   int n_chunks;
+  // top-k middle tokens of the query (topk > 0; seq_len must be null)
+  int topk;
+  float* tk_zall;               // [B, Hq, T] candidate logits (unscaled)
+  int32_t* tk_idx;              // [B, Hq, topk] the selection (-1 padding)
+  float* tk_z;                  // [B, Hq, topk] its logits (-inf padding)
+  float* tk_part;               // [B, Hq, d + 2] the selected keys' partial (max, sum, O)
   __nv_bfloat16* O;             // [B, Hq, 1, d]
   int64_t o_sb, o_sh;
   float* lse;                   // [B, Hq]

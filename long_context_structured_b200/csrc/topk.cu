@@ -27,6 +27,7 @@
 #include <math_constants.h>
 
 #include "kernels.cuh"
+#include "select.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
 
@@ -57,23 +58,6 @@ __device__ __forceinline__ bool mbar_wait_raw(uint64_t* bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > 100000000ull) return false;
   }
   return true;
-}
-
-// insert (v, j) into the descending list (vals, idxs); strict > keeps the
-// earlier (smaller j) entry first among equal scores
-template <int KC>
-__device__ __forceinline__ void list_insert(float v, int j, float (&vals)[KC], int (&idxs)[KC]) {
-#pragma unroll
-  for (int x = 0; x < KC; ++x) {
-    if (v > vals[x]) {
-      const float tv = vals[x];
-      const int tj = idxs[x];
-      vals[x] = v;
-      idxs[x] = j;
-      v = tv;
-      j = tj;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -776,7 +760,6 @@ __global__ void __launch_bounds__(kExactThreads) topk_exact_kernel(const TopkArg
   const Tin* Q = reinterpret_cast<const Tin*>(a.Q);
   const Tin* K = reinterpret_cast<const Tin*>(a.K);
   const int half = a.d / 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t x = blockIdx.x; x < count; x += gridDim.x) {
     const int64_t row = all_rows ? x : a.fallback_rows[x];
     const int i = (int)(row % a.T);
@@ -840,53 +823,10 @@ __global__ void __launch_bounds__(kExactThreads) topk_exact_kernel(const TopkArg
       }
     }
     // k rounds of block-wide argmax over (z desc, j asc)
-    int head = 0;  // next unused entry of this thread's sorted list
-    for (int r = 0; r < a.topk; ++r) {
-      float bz = -CUDART_INF_F;
-      int bj = -1;
-#pragma unroll
-      for (int y = 0; y < kMaxK; ++y)
-        if (y == head) {
-          bz = vals[y];
-          bj = idxs[y];
-        }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (oj >= 0 && (bj < 0 || oz > bz || (oz == bz && oj < bj))) {
-          bz = oz;
-          bj = oj;
-        }
-      }
-      if (lane == 0) {
-        red_z[warp] = bz;
-        red_j[warp] = bj;
-      }
-      __syncthreads();
-      float wz = red_z[0];
-      int wj = red_j[0];
-      for (int w = 1; w < kExactThreads / 32; ++w) {
-        const float oz = red_z[w];
-        const int oj = red_j[w];
-        if (oj >= 0 && (wj < 0 || oz > wz || (oz == wz && oj < wj))) {
-          wz = oz;
-          wj = oj;
-        }
-      }
-      __syncthreads();
-      if (wj >= 0 && head < kMaxK) {
-        int hj = -2;
-#pragma unroll
-        for (int y = 0; y < kMaxK; ++y)
-          if (y == head) hj = idxs[y];
-        if (hj == wj) ++head;
-      }
-      if (threadIdx.x == 0) {
-        a.idx[row * a.topk + r] = wj;
-        a.z[row * a.topk + r] = (wj >= 0) ? wz : -CUDART_INF_F;
-      }
-    }
+    block_topk_rounds<kMaxK>(a.topk, vals, idxs, red_z, red_j, [&](int r, float wz, int wj) {
+      a.idx[row * a.topk + r] = wj;
+      a.z[row * a.topk + r] = (wj >= 0) ? wz : -CUDART_INF_F;
+    });
   }
 }
 

@@ -116,3 +116,92 @@ def test_decode_rejects_unsupported():
     k = torch.zeros((1, 1, 10, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(_lib.SattnError):
         sa.decode_fwd(q, k, k)  # Hq / Hkv = 3
+
+
+# ---------------------------------------------------------------------------
+# top-k middle tokens during decoding
+# ---------------------------------------------------------------------------
+
+TOPK_CASES = [
+    # capped (w = L) with planted clusters, GQA
+    ("topk_capped_planted_gqa2", dict(B=2, Hq=4, Hkv=2, T=2048, d=128, n_start=4, window=256, L_pretrain=256,
+                                      rope_theta=1e4, topk=5, plant=3)),
+    # window below the cap: candidates on both sides of it; separators excluded
+    ("topk_window_below_cap_sep_gqa8_d64", dict(B=1, Hq=8, Hkv=1, T=1500, d=64, n_start=2, window=60,
+                                                L_pretrain=300, rope_theta=5e5, topk=8, sep_rate=0.15)),
+    # uncapped, k = 16, separators
+    ("topk16_uncapped_sep", dict(B=2, Hq=2, Hkv=2, T=900, d=128, n_start=4, window=100, rope_theta=1e4,
+                                 topk=16, sep_rate=0.1)),
+    # clipped ALiBi past the cap
+    ("topk_alibi_capped_gqa4", dict(B=1, Hq=8, Hkv=2, T=1200, d=128, n_start=4, window=64, L_pretrain=64,
+                                    topk=3, alibi=True)),
+    # fewer candidates than k: all of them, then -1 / -inf padding
+    ("topk_few_candidates", dict(B=1, Hq=2, Hkv=1, T=40, d=128, n_start=4, window=30, L_pretrain=30,
+                                 rope_theta=1e4, topk=8)),
+    # no candidate at all
+    ("topk_no_candidates", dict(B=1, Hq=2, Hkv=2, T=20, d=64, n_start=4, window=30, L_pretrain=30,
+                                rope_theta=1e4, topk=4)),
+]
+
+
+def _decode_topk_and_check(oracle_mod, wl, seed):
+    from _util import TOPK_EXT, topk_agreement
+    inp = synth.make_inputs(wl, seed=seed)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    qd = q[:, :, wl.T - 1:wl.T, :].contiguous()
+    O, lse, idx, z = sa.decode_fwd(qd, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                                   rope_theta=wl.rope_theta, is_sep=sep, alibi=wl.alibi, topk=wl.topk,
+                                   return_topk=True)
+    torch.cuda.synchronize()
+    assert sa.stream_status() == 0
+    rows = np.array([(b, h, wl.T - 1) for b in range(wl.B) for h in range(wl.Hq)], dtype=np.int64)
+    # the selection: the oracle's own, bit-exact up to the near-tie rule
+    p_ext = oracle_mod.params_of(wl.scaled(topk=wl.topk + TOPK_EXT))
+    _, _, ref_idx, ref_z, _ = oracle_mod.fwd_rows(p_ext, inp["q"], inp["k"], inp["v"], inp["is_sep"], rows)
+    gi = idx.reshape(-1, wl.topk).cpu().numpy()
+    n_exact, n_exempt, bad = topk_agreement(gi, ref_idx, ref_z, wl.topk)
+    assert not bad, "rows differ beyond the near-tie rule: %s" % bad[:10]
+    gz = z.reshape(-1, wl.topk).cpu().numpy().astype(np.float64)
+    same = np.all(gi == ref_idx[:, : wl.topk], axis=1)
+    fin = np.isfinite(ref_z[same, : wl.topk])
+    assert np.allclose(gz[same][fin], ref_z[same, : wl.topk][fin], rtol=1e-5, atol=1e-4)
+    assert np.all(np.isneginf(gz[gi < 0]))
+    # the step against the oracle's row with the GPU's selection
+    Oref, lref, *_ = oracle_mod.fwd_rows(oracle_mod.params_of(wl), inp["q"], inp["k"], inp["v"], inp["is_sep"],
+                                         rows, forced_topk=gi)
+    got = O[:, :, 0, :].reshape(-1, wl.d).float().cpu().numpy().astype(np.float64)
+    gl = lse.reshape(-1).float().cpu().numpy().astype(np.float64)
+    compare("O", got, Oref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare("LSE", gl, lref, BF16_MAX_ABS, BF16_MEAN_ABS)
+    # the step without return_topk is the same call
+    O2, lse2 = sa.decode_fwd(qd, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain,
+                             rope_theta=wl.rope_theta, is_sep=sep, alibi=wl.alibi, topk=wl.topk)
+    assert torch.equal(O2, O) and torch.equal(lse2, lse)
+    return gi
+
+
+@pytest.mark.parametrize("name,cfg", TOPK_CASES, ids=[c[0] for c in TOPK_CASES])
+def test_decode_topk_matches_oracle(oracle_mod, name, cfg):
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    gi = _decode_topk_and_check(oracle_mod, wl, seed=23)
+    if name == "topk_no_candidates":
+        assert np.all(gi == -1)
+    if name == "topk_few_candidates":
+        n_cand = wl.T - 1 - wl.window - wl.n_start
+        assert np.all(gi[:, :n_cand] >= 0) and np.all(gi[:, n_cand:] == -1)
+
+
+def test_decode_topk_full_size():
+    """The 32K-token top-k layer's last position (32 heads, k = 5, planted
+    clusters), against the oracle."""
+    from oracle import oracle as O
+    O.build()
+    _decode_topk_and_check(O, synth.WORKLOADS["c4_lminf_topk_32k"], seed=0)
+
+
+def test_decode_topk_alibi_below_cap_rejected():
+    q = torch.zeros((1, 2, 1, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 2, 300, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.SattnError):
+        sa.decode_fwd(q, kv, kv, n_start=4, window=30, L_pretrain=100, topk=2, alibi=True)
