@@ -211,6 +211,57 @@ int sattn_segment_bwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
                       const float* lse, const int32_t* prefix_blocks, const void* dO, void* dQ, void* dK, void* dV,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* ---- segmented execution one segment at a time (explicit carried state) ----
+ *
+ * "Training-Inference Consistent Segmented Execution for Long-Context LLMs"
+ * (section 整体框架) applies the layer per segment,
+ * (C_i, o^(i)) = F(x^(i), C_{i-1}, R_{i-1}): the local heads carry the tail
+ * of the earlier tokens, the long heads retrieve from the pool of earlier
+ * keys with the previous segment's last query.  These calls run that
+ * operator on one segment at a time with the carried part in a caller-owned
+ * device buffer (the state): every earlier token's raw K and V, its key
+ * rotated at its position, the previous segment's last query of every head
+ * and a header counting the segments taken.  Steps 0, 1, ..., N-1 give the
+ * O, LSE and retrieved blocks of sattn_segment_fwd on the concatenated
+ * segments (the same kernels on the same operands).
+ *
+ * Common arguments: p gives B, Hq, Hkv, d, the rotary base and scale, bf16,
+ * and p->T = the capacity (the longest total length, a multiple of S); S, M,
+ * R, retr_block as in sattn_segment_fwd, with the same rules
+ * (SATTN_ERR_UNSUPPORTED / SATTN_ERR_INVALID_ARG). */
+
+/* Bytes of the state for a capacity of p->T positions. */
+int sattn_segment_state_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                             size_t* bytes);
+
+/* Starts a sequence: no segment taken; builds the rotary table of every
+ * position.  state: device, 256-byte aligned, at least the size above.
+ * Asynchronous on `stream`. */
+int sattn_segment_state_reset(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                              void* state, size_t state_bytes, void* stream);
+
+/* Bytes of workspace needed by sattn_segment_step. */
+int sattn_segment_step_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                                      const uint8_t* is_long, size_t* bytes);
+
+/* Segment `seg` (0, 1, ... in order; (seg + 1) S <= p->T):
+ *   is_long        [Hq] host flags, as in sattn_segment_fwd.
+ *   Q, K, V        the segment's [B, Hq, S, d] / [B, Hkv, S, d] bf16 device
+ *                  inputs (positions seg S ..), strides q/k/v_stride.
+ *   state          the carried state; the segment is appended and its last
+ *                  query kept for the next step.
+ *   O, lse         [B, Hq, S, d] bf16 (o_stride) and [B, Hq, S] fp32, out.
+ *   prefix_blocks  [B, Hq, R / retr_block] int32, out: the long heads'
+ *                  retrieved blocks for this segment (-1 for local heads,
+ *                  segment 0 and unused slots); may be NULL when R = 0.
+ * A step that is not the next segment of the state (or a state that was
+ * never reset) writes nothing and leaves SATTN_ERR_INVALID_ARG in the
+ * workspace's status word (sattn_stream_status).  Asynchronous on `stream`. */
+int sattn_segment_step(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                       const uint8_t* is_long, int32_t seg, const void* Q, const void* K, const void* V, void* state,
+                       size_t state_bytes, void* O, float* lse, int32_t* prefix_blocks, void* ws, size_t ws_bytes,
+                       void* stream);
+
 /* Bytes of workspace needed by sattn_decode_fwd for *p (p->T = cache length). */
 int sattn_decode_workspace_size(const sattn_params* p, size_t* bytes);
 

@@ -28,7 +28,8 @@ import torch
 from . import _lib
 from ._lib import DTYPE_BF16, DTYPE_F32, SattnError, SattnParams
 
-__all__ = ["fwd", "topk_select", "build_blockmap", "build_blockmap_noalloc", "segment_fwd", "segment_bwd", "stream_status", "workspace_size",
+__all__ = ["fwd", "topk_select", "build_blockmap", "build_blockmap_noalloc", "segment_fwd", "segment_bwd",
+           "SegmentStream", "stream_status", "workspace_size",
            "segment_workspace_size", "params", "SattnError", "version", "TILE", "selftest_wait_timeout",
            "decode_fwd"]
 
@@ -232,6 +233,87 @@ def segment_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, S: int, M:
                                        _ptr(lse), _ptr(prefix), _ptr(ws), nbytes, _stream_ptr(q.device))
     _lib.check(rc, "sattn_segment_fwd")
     return out, lse, prefix[..., :nb]
+
+
+class SegmentStream:
+    """Segmented execution of one layer one segment at a time, the carried
+    part (every earlier token's K and V, their rotated keys, the previous
+    segment's last query) in a device state buffer.  ``step(q, k, v)`` takes
+    the next segment's [B, H, S, d] inputs and returns its (O, lse,
+    prefix_blocks [B, Hq, R / retr_block]); steps 0 .. N-1 give what
+    ``segment_fwd`` gives on the concatenated segments."""
+
+    def __init__(self, *, B: int, Hq: int, Hkv: int, d: int, capacity: int, S: int, M: int, R: int,
+                 retr_block: int, is_long, rope_theta: float = 0.0, rope_pos_scale: float = 1.0, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.d, self.capacity = B, Hq, Hkv, d, capacity
+        self.S, self.M, self.R, self.retr_block = S, M, R, retr_block
+        self.rope_theta, self.rope_pos_scale = float(rope_theta), float(rope_pos_scale)
+        self.device = torch.device(device)
+        il = [int(x) for x in (is_long.tolist() if hasattr(is_long, "tolist") else is_long)]
+        if len(il) != Hq:
+            raise ValueError("is_long needs one flag per query head")
+        self.is_long = (ctypes.c_uint8 * Hq)(*il)
+        p = self._params()
+        n = ctypes.c_size_t(0)
+        L = _lib.load()
+        _lib.check(L.sattn_segment_state_size(ctypes.byref(p), S, M, R, retr_block, ctypes.byref(n)),
+                   "sattn_segment_state_size")
+        self.state = torch.empty(int(n.value), dtype=torch.uint8, device=self.device)
+        _lib.check(L.sattn_segment_step_workspace_size(ctypes.byref(p), S, M, R, retr_block, self.is_long,
+                                                       ctypes.byref(n)), "sattn_segment_step_workspace_size")
+        self.workspace = torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=self.device)
+        self.reset()
+
+    def _params(self, q=None, k=None, v=None, o=None) -> SattnParams:
+        if q is None:
+            p = SattnParams()
+            p.B, p.Hq, p.Hkv, p.d = self.B, self.Hq, self.Hkv, self.d
+            p.dtype = _lib.DTYPE_BF16
+            for name, H in (("q_stride", self.Hq), ("k_stride", self.Hkv), ("v_stride", self.Hkv),
+                            ("o_stride", self.Hq)):
+                arr = getattr(p, name)
+                arr[0], arr[1], arr[2] = H * self.S * self.d, self.S * self.d, self.d
+            p.rope_theta, p.rope_pos_scale = self.rope_theta, self.rope_pos_scale
+        else:
+            p = params(q, k, v, o, rope_theta=self.rope_theta, rope_pos_scale=self.rope_pos_scale)
+        p.T = self.capacity
+        return p
+
+    def reset(self):
+        """Start a new sequence (no segment taken)."""
+        p = self._params()
+        _lib.check(_lib.load().sattn_segment_state_reset(ctypes.byref(p), self.S, self.M, self.R, self.retr_block,
+                                                         _ptr(self.state), self.state.numel(),
+                                                         _stream_ptr(self.device)), "sattn_segment_state_reset")
+        self.seg = 0
+
+    def step(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None, seg: Optional[int] = None):
+        """The next segment (or segment ``seg``; a step that is not the next
+        one writes nothing and leaves an error in the status word)."""
+        B, Hq, S, d = q.shape
+        if S != self.S:
+            raise ValueError("a step takes one segment of S = %d positions" % self.S)
+        if out is None:
+            out = torch.empty((B, Hq, S, d), dtype=q.dtype, device=q.device)
+        if lse is None:
+            lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+        nb = self.R // self.retr_block
+        prefix = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=q.device)
+        p = self._params(q, k, v, out)
+        s = self.seg if seg is None else int(seg)
+        rc = _lib.load().sattn_segment_step(ctypes.byref(p), self.S, self.M, self.R, self.retr_block, self.is_long, s,
+                                            _ptr(q), _ptr(k), _ptr(v), _ptr(self.state), self.state.numel(),
+                                            _ptr(out), _ptr(lse), _ptr(prefix), _ptr(self.workspace),
+                                            self.workspace.numel(), _stream_ptr(q.device))
+        _lib.check(rc, "sattn_segment_step")
+        if seg is None:
+            self.seg += 1
+        return out, lse, prefix[..., :nb]
+
+    def status(self) -> int:
+        """Synchronise and read the status word of the last step."""
+        return stream_status(self.workspace)
 
 
 def segment_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,

@@ -24,7 +24,8 @@ DTYPE_F32 = 1
 EXPORTS = (
     "sattn_strerror", "sattn_version", "sattn_workspace_size", "sattn_segment_workspace_size",
     "sattn_build_blockmap", "sattn_topk_select", "sattn_fwd", "sattn_segment_fwd",
-    "sattn_segment_bwd_workspace_size", "sattn_segment_bwd",
+    "sattn_segment_bwd_workspace_size", "sattn_segment_bwd", "sattn_segment_state_size", "sattn_segment_state_reset",
+    "sattn_segment_step_workspace_size", "sattn_segment_step",
     "sattn_decode_workspace_size", "sattn_decode_fwd", "sattn_decode_topk_fwd", "sattn_bwd_workspace_size",
     "sattn_bwd",
     "sattn_tree_cross_workspace_size", "sattn_tree_cross_fwd", "sattn_stream_state_size", "sattn_stream_reset",
@@ -92,6 +93,14 @@ def load():
         L.sattn_segment_bwd_workspace_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
         L.sattn_segment_bwd.restype = ctypes.c_int
         L.sattn_segment_bwd.argtypes = [P, i32, i32, i32, i32] + [vp] * 11 + [vp, sz, vp]
+        L.sattn_segment_state_size.restype = ctypes.c_int
+        L.sattn_segment_state_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
+        L.sattn_segment_state_reset.restype = ctypes.c_int
+        L.sattn_segment_state_reset.argtypes = [P, i32, i32, i32, i32, vp, sz, vp]
+        L.sattn_segment_step_workspace_size.restype = ctypes.c_int
+        L.sattn_segment_step_workspace_size.argtypes = [P, i32, i32, i32, i32, vp, ctypes.POINTER(sz)]
+        L.sattn_segment_step.restype = ctypes.c_int
+        L.sattn_segment_step.argtypes = [P, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp, vp, vp, vp, sz, vp]
         L.sattn_decode_workspace_size.restype = ctypes.c_int
         L.sattn_decode_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.sattn_decode_fwd.restype = ctypes.c_int

@@ -732,6 +732,8 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
     ra.R = R;
     ra.blk = retr_block;
     ra.n_long = P.n_long;
+    ra.s_lo = 1;  // every segment after the first, all of them held
+    ra.s_base = 0;
     ra.Q = static_cast<const __nv_bfloat16*>(Q);
     ra.K = static_cast<const __nv_bfloat16*>(K);
     ra.V = static_cast<const __nv_bfloat16*>(V);
@@ -789,6 +791,288 @@ int sattn_segment_fwd(const sattn_params* p, int32_t S, int32_t M, int32_t R, in
   a.status = at<int32_t>(ws, P.status);
   ProfScope ps("attn_tc_segment", 1, st);
   return cuda_rc((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc3(a, m, st));
+}
+
+// ---------------------------------------------------------------------------
+// segmented execution one segment at a time (explicit carried state)
+// ---------------------------------------------------------------------------
+
+// The state of a layer of capacity p->T (a multiple of S): header, rotary
+// table of every position, raw K and V and the keys rotated at their
+// positions for every position taken, the last segment's last query.
+struct SegStateLayout {
+  Region header, tab, khist, vhist, krot, qend;
+  size_t total = 0;
+};
+
+static int seg_stream_rules(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t blk) {
+  int rc = check_common(p);
+  if (rc) return rc;
+  if (p->dtype != SATTN_DTYPE_BF16 || p->alibi) return SATTN_ERR_UNSUPPORTED;
+  if (S < kTile || S % kTile || p->T % S || M < 0 || R < 0 || blk < 1 || R % blk) return SATTN_ERR_INVALID_ARG;
+  if (R / blk > 1024 || p->Hq > kMaxHeads) return SATTN_ERR_UNSUPPORTED;
+  if (!segment_retrieval_supported(p->T, S, blk)) return SATTN_ERR_UNSUPPORTED;
+  return SATTN_OK;
+}
+
+static int seg_state_layout(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t blk,
+                            SegStateLayout* out) {
+  int rc = seg_stream_rules(p, S, M, R, blk);
+  if (rc) return rc;
+  SegStateLayout L;
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, T = p->T, d = p->d;
+  Alloc A;
+  L.header = A.take(256);
+  if (p->rope_theta != 0.0) L.tab = A.take(T * (d / 2) * sizeof(float2));
+  L.khist = A.take(B * Hkv * T * d * 2);
+  L.vhist = A.take(B * Hkv * T * d * 2);
+  L.krot = A.take(B * Hkv * T * d * 2);
+  L.qend = A.take(B * Hq * d * 2);
+  L.total = A.cur;
+  *out = L;
+  return SATTN_OK;
+}
+
+struct SegStepPlan {
+  int n_long = 0, Rpad = 0;
+  Region status, qr, pcnt, score, kpre, vpre;
+  size_t total = 0;
+};
+
+static int plan_seg_step(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t blk, const uint8_t* is_long,
+                         SegStepPlan* out) {
+  int rc = seg_stream_rules(p, S, M, R, blk);
+  if (rc) return rc;
+  SegStepPlan P;
+  for (int h = 0; h < p->Hq; ++h) P.n_long += (is_long == nullptr || is_long[h]) ? 1 : 0;
+  P.Rpad = (R + kTile - 1) / kTile * kTile;
+  const size_t B = p->B, Hq = p->Hq, d = p->d;
+  Alloc A;
+  P.status = A.take(kStatusBytes);
+  P.qr = A.take(B * Hq * (size_t)S * d * 2);
+  P.pcnt = A.take(B * std::max(P.n_long, 1) * 4);
+  if (P.n_long > 0 && R > 0) {
+    P.score = A.take(segment_score_bytes(p->B, P.n_long, 1, p->T, blk));
+    P.kpre = A.take(B * P.n_long * (size_t)P.Rpad * d * 2);
+    P.vpre = A.take(B * P.n_long * (size_t)P.Rpad * d * 2);
+  }
+  P.total = A.cur;
+  *out = P;
+  return SATTN_OK;
+}
+
+int sattn_segment_state_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                             size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  SegStateLayout L;
+  int rc = seg_state_layout(p, S, M, R, retr_block, &L);
+  if (rc) return rc;
+  *bytes = L.total;
+  return SATTN_OK;
+}
+
+int sattn_segment_state_reset(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                              void* state, size_t state_bytes, void* stream) {
+  SegStateLayout L;
+  int rc = seg_state_layout(p, S, M, R, retr_block, &L);
+  if (rc) return rc;
+  if (!state || state_bytes < L.total || (reinterpret_cast<uintptr_t>(state) & 255u)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SATTN_TRY(cudaMemsetAsync(state, 0, L.header.bytes, st));
+  SATTN_TRY(launch_segstate_reset(at<int32_t>(state, L.header), S, p->T, st));
+  if (L.tab.bytes)
+    SATTN_TRY(launch_rope_table(at<float2>(state, L.tab), p->T, p->d, p->rope_theta, pos_scale(p), st));
+  return SATTN_OK;
+}
+
+int sattn_segment_step_workspace_size(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                                      const uint8_t* is_long, size_t* bytes) {
+  if (!bytes) return SATTN_ERR_INVALID_ARG;
+  SegStepPlan P;
+  int rc = plan_seg_step(p, S, M, R, retr_block, is_long, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return SATTN_OK;
+}
+
+int sattn_segment_step(const sattn_params* p, int32_t S, int32_t M, int32_t R, int32_t retr_block,
+                       const uint8_t* is_long, int32_t seg, const void* Q, const void* K, const void* V, void* state,
+                       size_t state_bytes, void* O, float* lse, int32_t* prefix_blocks, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (!is_long) return SATTN_ERR_INVALID_ARG;
+  SegStateLayout L;
+  int rc = seg_state_layout(p, S, M, R, retr_block, &L);
+  if (rc) return rc;
+  SegStepPlan P;
+  rc = plan_seg_step(p, S, M, R, retr_block, is_long, &P);
+  if (rc) return rc;
+  if (seg < 0 || (int64_t)(seg + 1) * S > p->T) return SATTN_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !lse || (R > 0 && !prefix_blocks)) return SATTN_ERR_INVALID_ARG;
+  if (!state || state_bytes < L.total || (reinterpret_cast<uintptr_t>(state) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
+  if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t B = p->B, Hq = p->Hq, Hkv = p->Hkv, Tcap = p->T, d = p->d;
+  const int Tnow = (seg + 1) * S;  // positions taken once this segment is in
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+  int32_t* status = at<int32_t>(ws, P.status);
+
+  // 1. the segment joins the history (after checking it is the next one)
+  SegStateArgs sa{};
+  sa.B = p->B;
+  sa.Hq = p->Hq;
+  sa.Hkv = p->Hkv;
+  sa.d = p->d;
+  sa.S = S;
+  sa.T_cap = p->T;
+  sa.seg = seg;
+  sa.header = at<int32_t>(state, L.header);
+  sa.Q = static_cast<const __nv_bfloat16*>(Q);
+  sa.K = static_cast<const __nv_bfloat16*>(K);
+  sa.V = static_cast<const __nv_bfloat16*>(V);
+  sa.q_sb = p->q_stride[0];
+  sa.q_sh = p->q_stride[1];
+  sa.q_st = p->q_stride[2];
+  sa.k_sb = p->k_stride[0];
+  sa.k_sh = p->k_stride[1];
+  sa.k_st = p->k_stride[2];
+  sa.v_sb = p->v_stride[0];
+  sa.v_sh = p->v_stride[1];
+  sa.v_st = p->v_stride[2];
+  sa.Khist = at<__nv_bfloat16>(state, L.khist);
+  sa.Vhist = at<__nv_bfloat16>(state, L.vhist);
+  sa.q_end = at<__nv_bfloat16>(state, L.qend);
+  sa.status = status;
+  {
+    ProfScope ps("segment_state_append", 1, st);
+    SATTN_TRY(launch_segstate_append(sa, st));
+  }
+  // 2. rotation at the global positions: the segment's queries into the
+  //    workspace, its keys into the state's rotated history
+  {
+    PrepArgs pa{};
+    pa.B = p->B;
+    pa.Hq = p->Hq;
+    pa.Hkv = p->Hkv;
+    pa.T = S;
+    pa.d = p->d;
+    pa.Q = Q;
+    pa.K = K;
+    pa.q_sb = p->q_stride[0];
+    pa.q_sh = p->q_stride[1];
+    pa.q_st = p->q_stride[2];
+    pa.k_sb = p->k_stride[0];
+    pa.k_sh = p->k_stride[1];
+    pa.k_st = p->k_stride[2];
+    pa.tab = L.tab.bytes ? at<float2>(state, L.tab) : nullptr;
+    pa.Qr = at<__nv_bfloat16>(ws, P.qr);
+    pa.Kr = at<__nv_bfloat16>(state, L.krot);
+    pa.pos0 = seg * S;
+    pa.kr_rows = p->T;
+    pa.kr_row0 = seg * S;
+    pa.status = status;
+    ProfScope ps("prep_rope", 1, st);
+    SATTN_TRY(launch_prep(pa, st));
+  }
+  // 3. retrieval for the long heads from the pool [0, seg S) with the carried query
+  const int nb = R / retr_block;
+  if (nb > 0) SATTN_TRY(cudaMemsetAsync(prefix_blocks, 0xFF, B * Hq * nb * 4, st));
+  SATTN_TRY(cudaMemsetAsync(at<uint8_t>(ws, P.pcnt), 0, P.pcnt.bytes, st));
+  AttnArgs a{};
+  for (int h = 0; h < kMaxHeads; ++h) a.long_slot[h] = -1;
+  SegRetrArgs ra{};
+  {
+    int slot = 0;
+    for (int h = 0; h < p->Hq; ++h)
+      if (is_long[h]) {
+        a.long_slot[h] = (int16_t)slot;
+        ra.long_heads[slot] = (int16_t)h;
+        ++slot;
+      }
+  }
+  AttnMaps m;
+  if (!make_map(&m.q, at<void>(ws, P.qr), p->d, S, Hq, B, d, (int64_t)S * d, Hq * S * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.k, at<void>(state, L.krot), p->d, p->T, Hkv, B, d, Tcap * d, Hkv * Tcap * d)) return SATTN_ERR_CUDA;
+  if (!make_map(&m.v, at<void>(state, L.vhist), p->d, p->T, Hkv, B, d, Tcap * d, Hkv * Tcap * d)) return SATTN_ERR_CUDA;
+  m.q2 = m.q;
+  m.kg = m.k;
+  m.vg = m.v;
+  if (P.n_long > 0 && R > 0 && seg > 0) {
+    ra.B = p->B;
+    ra.Hq = p->Hq;
+    ra.Hkv = p->Hkv;
+    ra.T = Tnow;
+    ra.d = p->d;
+    ra.S = S;
+    ra.N = seg + 1;
+    ra.R = R;
+    ra.blk = retr_block;
+    ra.n_long = P.n_long;
+    ra.s_lo = seg;  // this segment alone, its arrays the only ones held
+    ra.s_base = seg;
+    ra.Q = nullptr;
+    ra.q_end = at<__nv_bfloat16>(state, L.qend);
+    ra.qe_sb = (int64_t)Hq * d;
+    ra.qe_sh = d;
+    ra.K = at<__nv_bfloat16>(state, L.khist);
+    ra.V = at<__nv_bfloat16>(state, L.vhist);
+    ra.k_sb = ra.v_sb = (int64_t)Hkv * Tcap * d;
+    ra.k_sh = ra.v_sh = (int64_t)Tcap * d;
+    ra.k_st = ra.v_st = d;
+    ra.tab = L.tab.bytes ? at<float2>(state, L.tab) : nullptr;
+    ra.prefix_blocks = prefix_blocks;
+    ra.prefix_cnt = at<int32_t>(ws, P.pcnt);
+    ra.Kpre = at<__nv_bfloat16>(ws, P.kpre);
+    ra.Vpre = at<__nv_bfloat16>(ws, P.vpre);
+    ra.score = at<float>(ws, P.score);
+    {
+      ProfScope ps("segment_retrieval", 3, st);
+      SATTN_TRY(launch_segment_retrieval(ra, st));
+    }
+    const int64_t planes = P.n_long;
+    if (!make_map(&m.kg, ra.Kpre, p->d, P.Rpad, planes, B, d, (int64_t)P.Rpad * d, planes * P.Rpad * d))
+      return SATTN_ERR_CUDA;
+    if (!make_map(&m.vg, ra.Vpre, p->d, P.Rpad, planes, B, d, (int64_t)P.Rpad * d, planes * P.Rpad * d))
+      return SATTN_ERR_CUDA;
+  }
+  // 4. attention of the segment's rows over the state
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.T = Tnow;
+  a.d = p->d;
+  a.nQT = S / kTile;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->d));
+  a.ns_band = 0;
+  a.w_eff = 0x3fffffff;
+  a.V = at<__nv_bfloat16>(state, L.vhist);
+  a.v_sb = (int64_t)Hkv * Tcap * d;
+  a.v_sh = (int64_t)Tcap * d;
+  a.v_st = d;
+  a.gather_mode = 2;
+  a.q2 = false;
+  a.seg_S = S;
+  a.seg_M = M;
+  a.seg_N = seg + 1;
+  a.seg_R = R;
+  a.seg_s0 = seg;
+  a.q_pos0 = seg * S;
+  a.T_q = S;
+  a.prefix_cnt = at<int32_t>(ws, P.pcnt);
+  a.n_long = std::max(P.n_long, 1);
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.o_sb = p->o_stride[0];
+  a.o_sh = p->o_stride[1];
+  a.o_st = p->o_stride[2];
+  a.lse = lse;
+  a.status = status;
+  {
+    ProfScope ps("attn_tc_segment", 1, st);
+    SATTN_TRY((S % (2 * kTile) == 0) ? launch_attn_tc2(a, m, st) : launch_attn_tc3(a, m, st));
+  }
+  // 5. the segment's last query is carried to the next step
+  ProfScope ps("segment_state_finish", 1, st);
+  return cuda_rc(launch_segstate_finish(sa, st));
 }
 
 // ---------------------------------------------------------------------------

@@ -27,8 +27,17 @@ constexpr float kSumRebase = 0x1p8f;
 // 2^-e for an integer e in [0, 126]
 __device__ __forceinline__ float exp2_neg_int(int e) { return __int_as_float((127 - e) << 23); }
 
+// Rows of the Q / O / LSE tensors, and the prefix plane of a long head's
+// query tile (tile: position / kTile).
+__device__ __forceinline__ int q_rows(const AttnArgs& a) { return a.T_q > 0 ? a.T_q : a.T; }
+__device__ __forceinline__ int prefix_plane(const AttnArgs& a, int h, int g, int tile) {
+  return (a.gather_mode == 2 && a.long_slot[h] >= 0)
+             ? a.long_slot[h] * (a.seg_N - a.seg_s0) + (tile * kTile) / a.seg_S - a.seg_s0
+             : g;
+}
+
 // Key tiles one 128-row query tile visits: gathered tiles [0, n_gather),
-// then band key tiles [u_lo, u_lo + n_band).
+// then band key tiles [u_lo, u_lo + n_band).  t: the tile's position / kTile.
 struct Plan {
   int g_count, g_full, n_gather, band_lo, u_lo, n_band, rows;  // rows: valid rows of the tile (0 = none)
 };
@@ -56,7 +65,7 @@ __device__ __forceinline__ Plan make_plan(const AttnArgs& a, int b, int h, int t
     const int slot = a.long_slot[h];
     if (slot >= 0) {
       p.band_lo = seg0;
-      if (s > 0) p.g_count = p.g_full = a.prefix_cnt[(b * a.n_long + slot) * a.seg_N + s];
+      if (s > 0) p.g_count = p.g_full = a.prefix_cnt[(b * a.n_long + slot) * (a.seg_N - a.seg_s0) + (s - a.seg_s0)];
     } else {
       p.band_lo = s > 0 ? max(0, seg0 - a.seg_M) : 0;
     }

@@ -161,13 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qb = blockIdx.x % nQB;
+  const int qb = blockIdx.x % nQB;          // query tiles 2 qb, 2 qb + 1 of the Q / O tensors
+  const int tg0 = 2 * qb + a.q_pos0 / kTile;  // the first one's position / kTile
   const int bh = blockIdx.x / nQB;
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const Plan pl0 = make_plan(a, b, h, 2 * qb);
-  const Plan pl1 = make_plan(a, b, h, 2 * qb + 1);
+  const Plan pl0 = make_plan(a, b, h, tg0);
+  const Plan pl1 = make_plan(a, b, h, tg0 + 1);
   Union un;
   un.NG = max(pl0.n_gather, pl1.n_gather);
   {
@@ -183,9 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     un.U0 = (u1 >= 0) ? u0 : 0;
     un.n = un.NG + ((u1 >= 0) ? (u1 - u0 + 1) : 0);
   }
-  const int g_plane = (a.gather_mode == 2 && a.long_slot[h] >= 0)
-                          ? a.long_slot[h] * a.seg_N + (2 * qb * kTile) / a.seg_S
-                          : g;
+  const int g_plane = attn::prefix_plane(a, h, g, tg0);
 
   if (threadIdx.x == 0) {
     *early = status_failed(a.status) ? 1 : 0;
@@ -347,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = warp >> 2;  // query tile of this warpgroup
     const Plan& pl = x == 0 ? pl0 : pl1;
     const int r = threadIdx.x & 127;
-    const int i0 = (2 * qb + x) * kTile;
+    const int i0 = (tg0 + x) * kTile;
     const int i = i0 + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + x * 128;
@@ -470,7 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const bool row_ok = (i < a.T);
     const int ir = row_ok ? i : a.T - 1;
-    const size_t row_id = ((size_t)b * a.Hq + h) * a.T + ir;
+    const int il = ir - a.q_pos0;  // row of the O / LSE tensors
+    const size_t row_id = ((size_t)b * a.Hq + h) * attn::q_rows(a) + il;
     const int n_sink = min(a.n_sink, ir + 1);
     const float* sz = a.sink_z ? a.sink_z + row_id * a.n_sink : nullptr;
     const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;
     const __nv_bfloat16* vbase = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
-    __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)ir * a.o_st;
+    __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)il * a.o_st;
     // The sinks' V rows are the same for every row of the tile: stage them in
     // this warpgroup's Q tile (free once its last MMA completed).
     const bool sinks_smem = a.n_sink > 0 && a.n_sink <= kSinkSmem;

@@ -159,16 +159,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x % a.nQT;
+  const int t = blockIdx.x % a.nQT;         // query tile of the Q / O tensors
+  const int tg = t + a.q_pos0 / kTile;      // its position / kTile
   const int bh = blockIdx.x / a.nQT;
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const Plan pl = make_plan(a, b, h, t);
+  const Plan pl = make_plan(a, b, h, tg);
   const int n = pl.n_gather + pl.n_band;  // key tiles of this query tile
-  const int g_plane = (a.gather_mode == 2 && a.long_slot[h] >= 0)
-                          ? a.long_slot[h] * a.seg_N + (t * kTile) / a.seg_S
-                          : g;
+  const int g_plane = attn::prefix_plane(a, h, g, tg);
 
   if (threadIdx.x == 0) {
     *early = status_failed(a.status) ? 1 : 0;
@@ -301,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================== softmax + epilogue (warps 0-7) =====================
     const int rr = 32 * (warp & 3) + 16 * (warp >> 2) + (lane & 15);  // row of the query tile
     const int hc = lane >> 4;                                           // which half of the row's columns
-    const int i0 = t * kTile;
+    const int i0 = tg * kTile;
     const int i = i0 + rr;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3) + 16 * (warp >> 2)) << 16;
     const uint32_t tO = tmem + kTmemO + lane_off;
@@ -433,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const bool row_ok = (i < a.T);
     const int ir = row_ok ? i : a.T - 1;
-    const size_t row_id = ((size_t)b * a.Hq + h) * a.T + ir;
+    const int il = ir - a.q_pos0;  // row of the O / LSE tensors
+    const size_t row_id = ((size_t)b * a.Hq + h) * attn::q_rows(a) + il;
     const int n_sink = min(a.n_sink, ir + 1);
     const float* sz = a.sink_z ? a.sink_z + row_id * a.n_sink : nullptr;
     const int32_t* tki = a.tk_idx ? a.tk_idx + row_id * a.topk : nullptr;
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv_l = (l_fin > 0.f) ? 1.f / l_fin : 0.f;
     const int col0 = hc * (D / 2);
     const __nv_bfloat16* vbase = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh + col0;
-    __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)ir * a.o_st + col0;
+    __nv_bfloat16* orow = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh + (size_t)il * a.o_st + col0;
 #pragma unroll 1
     for (int c = 0; c < D / 2; c += 32) {
       float ov[32];

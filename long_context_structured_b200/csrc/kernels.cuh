@@ -36,6 +36,10 @@ struct PrepArgs {
   int n_sink;
   int alibi;          // nonzero: sink logits carry the clipped ALiBi bias (in q.k units)
   uint32_t* kmax;     // [B*Hkv] max_j ||k_j|| as float bits (may be null)
+  // input row r is position pos0 + r (no sink logits then); Kr holds
+  // kr_rows rows per (b, kv head) (0: T) and row r goes to row kr_row0 + r
+  int pos0, kr_rows, kr_row0;
+  const int32_t* status;  // when not null: nothing is written once it reports a failure
 };
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
 
@@ -132,8 +136,13 @@ struct AttnArgs {
   // segmented execution
   int seg_S, seg_M, seg_N, seg_R;
   int16_t long_slot[kMaxHeads]; // head -> index among long heads, -1 for local
-  const int32_t* prefix_cnt;   // [B, Hl, N] number of prefix keys
+  const int32_t* prefix_cnt;   // [B, Hl, N - seg_s0] number of prefix keys
   int n_long;
+  int seg_s0;                  // prefix planes and counts held for segments seg_s0 .. N-1
+  // query rows: row r of the Q / O / LSE tensors is position q_pos0 + r
+  // (a multiple of the tile), those tensors hold T_q rows (0: T); keys and
+  // masks use positions (T: the sequence so far)
+  int q_pos0, T_q;
   // ALiBi: s_ij gets -m_h * min(i - j, L) (L = 0: no clip), m_h = 2^(-8 (h+1) / Hq)
   int alibi, alibi_cap;
   // outputs
@@ -381,11 +390,18 @@ struct SegRetrArgs {
   int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st;
   int16_t long_heads[kMaxHeads]; // head id of each long slot
   const float2* tab;
-  int32_t* prefix_blocks;      // [B, Hq, N, R/blk] (all heads; -1 filled)
-  int32_t* prefix_cnt;         // [B, n_long, N]
-  __nv_bfloat16* Kpre;         // [B, n_long, N, R, d] rotated at virtual positions
+  // segments retrieved: s_lo .. N-1 (s_lo >= 1); the per-segment arrays
+  // below hold segments s_base .. N-1 (Ns = N - s_base of them)
+  int s_lo, s_base;
+  // segment-end query of segment s_lo (q_{s_lo S - 1}) when not null, in
+  // place of Q's row (a step that holds only its own segment's queries)
+  const __nv_bfloat16* q_end;  // [B, Hq, d]
+  int64_t qe_sb, qe_sh;
+  int32_t* prefix_blocks;      // [B, Hq, Ns, R/blk] (all heads; -1 filled)
+  int32_t* prefix_cnt;         // [B, n_long, Ns]
+  __nv_bfloat16* Kpre;         // [B, n_long, Ns, R, d] rotated at virtual positions
   __nv_bfloat16* Vpre;
-  float* score;                // [B, n_long, N, T / blk] block scores (workspace)
+  float* score;                // [B, n_long, Ns, T / blk] block scores (workspace)
 };
 // largest shared-memory sort buffer of the block selection (bytes)
 constexpr size_t kSegSelectSmemMax = 128 * 1024;
@@ -416,6 +432,25 @@ struct SegBwdArgs {
   int64_t dq_sb, dq_sh, dq_st, dk_sb, dk_sh, dk_st, dv_sb, dv_sh, dv_st;
 };
 cudaError_t launch_segment_bwd(const SegBwdArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// segmented execution one segment at a time: the carried state
+// ---------------------------------------------------------------------------
+struct SegStateArgs {
+  int B, Hq, Hkv, d, S, T_cap, seg;
+  int32_t* header;              // state header: magic, segments taken, S, T_cap
+  const __nv_bfloat16* Q;       // the segment's [B, Hq, S, d]
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  int64_t q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st;
+  __nv_bfloat16* Khist;         // [B, Hkv, T_cap, d] raw keys of every position taken
+  __nv_bfloat16* Vhist;
+  __nv_bfloat16* q_end;         // [B, Hq, d] the last segment's last query
+  int32_t* status;
+};
+cudaError_t launch_segstate_reset(int32_t* header, int S, int T_cap, cudaStream_t st);
+cudaError_t launch_segstate_append(const SegStateArgs& a, cudaStream_t st);
+cudaError_t launch_segstate_finish(const SegStateArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
 // decoding step: one query per (batch, head) at position T - 1

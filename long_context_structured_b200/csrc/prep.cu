@@ -28,6 +28,7 @@
 
 #include "kernels.cuh"
 #include "simt.cuh"
+#include "status.cuh"
 
 namespace sattn {
 
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
   __shared__ __align__(16) float s_sink_rot[NS_SMEM][D];  // R(j) k_j: dotted with R(i) q_i
   __shared__ __align__(16) float s_lc[half];
   __shared__ __align__(16) float s_ls[half];  // cos/sin of the rotation to the cap L
+  if (a.status && status_failed(a.status)) return;
   const int sub = threadIdx.x % tpr;       // which 8-pair chunk of the row
   const int c0 = sub * kPairsPerThread;
   const int b = blockIdx.z;
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
         const __nv_bfloat16* qp = Q + (int64_t)ii[u] * a.q_st;
         qa[u] = *reinterpret_cast<const uint4*>(qp + c0);
         qb[u] = *reinterpret_cast<const uint4*>(qp + c0 + half);
-        load_tab8_raw(a.tab, ii[u], half, c0, t[u]);
+        load_tab8_raw(a.tab, (int64_t)ii[u] + a.pos0, half, c0, t[u]);
         if (do_k) {
           const __nv_bfloat16* kp = Kh + (int64_t)ii[u] * a.k_st;
           ka[u] = *reinterpret_cast<const uint4*>(kp + c0);
@@ -233,7 +235,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrepArgs a) {
         if (a.Kr) {
           float r0[8], r1[8];
           rotate8(k0, k1, t[u], r0, r1);
-          __nv_bfloat16* kr = a.Kr + (((int64_t)b * a.Hkv + h) * a.T + i) * D;
+          __nv_bfloat16* kr =
+              a.Kr + (((int64_t)b * a.Hkv + h) * (a.kr_rows > 0 ? a.kr_rows : a.T) + a.kr_row0 + i) * D;
           *reinterpret_cast<uint4*>(kr + c0) = pack8(r0);
           *reinterpret_cast<uint4*>(kr + c0 + half) = pack8(r1);
         }
@@ -368,6 +371,7 @@ cudaError_t launch_prep_d(const PrepArgs& a, cudaStream_t st) {
 
 cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st) {
   if (a.f32) return cudaErrorInvalidValue;  // the fp32 path rotates inside its own kernel
+  if (a.pos0 != 0 && a.sink_z) return cudaErrorInvalidValue;  // sink logits assume row = position
   if (a.B == 0 || a.T == 0) return cudaSuccess;
   if (a.d == 128) return launch_prep_d<128>(a, st);
   if (a.d == 64) return launch_prep_d<64>(a, st);

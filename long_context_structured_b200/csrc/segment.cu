@@ -43,6 +43,10 @@ constexpr int kThreads = 256;
 constexpr int kChunkKeys = 128;  // keys scored per pass of a CTA
 constexpr int kQG = 16;          // segment-end queries per pass
 
+// index of segment s in the per-segment arrays, and their count
+__device__ __forceinline__ size_t seg_at(const SegRetrArgs& a, int s) { return (size_t)(s - a.s_base); }
+__device__ __forceinline__ size_t seg_n(const SegRetrArgs& a) { return (size_t)(a.N - a.s_base); }
+
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -54,7 +58,7 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
 }
 
 // grid (ceil(nblk_pool / nblk_cta), n_long, B).  CTA x scores blocks
-// [x * nblk_cta, ...) of the pool of its long head for every segment s >= 1:
+// [x * nblk_cta, ...) of the pool of its long head for every segment s >= s_lo:
 // score[b, slot, s, u] = max over the block's keys of <q_{sS-1}, k_j>.
 // Entries whose block lies beyond segment s's pool are written too and
 // never read.
@@ -73,15 +77,17 @@ __global__ void __launch_bounds__(kThreads) block_score_kernel(SegRetrArgs a, in
   const int u1 = min(u0 + nblk_cta, nblk_pool);
   const int k_begin = u0 * a.blk, k_end = u1 * a.blk;
   const __nv_bfloat16* kb = a.K + b * a.k_sb + g * a.k_sh;
-  const __nv_bfloat16* qb = a.Q + b * a.q_sb + h * a.q_sh;
-  for (int s0 = 1; s0 < a.N; s0 += kQG) {
+  const __nv_bfloat16* qb = a.q_end ? nullptr : a.Q + b * a.q_sb + h * a.q_sh;
+  for (int s0 = a.s_lo; s0 < a.N; s0 += kQG) {
     // this lane's 8 elements of the (up to) 16 segment-end queries
     float qr[kQG][8];
 #pragma unroll
     for (int q = 0; q < kQG; ++q) {
       const int s = s0 + q;
       if (s < a.N) {
-        unpack8(*reinterpret_cast<const uint4*>(qb + (int64_t)(s * a.S - 1) * a.q_st + sub * 8), qr[q]);
+        const __nv_bfloat16* qe = a.q_end ? a.q_end + b * a.qe_sb + h * a.qe_sh
+                                          : qb + (int64_t)(s * a.S - 1) * a.q_st;
+        unpack8(*reinterpret_cast<const uint4*>(qe + sub * 8), qr[q]);
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) qr[q][e] = 0.f;
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) block_score_kernel(SegRetrArgs a, in
     for (int x = threadIdx.x; x < (u1 - u0) * kQG; x += kThreads) {
       const int bl = x / kQG, q = x % kQG;
       const int s = s0 + q;
-      if (s < a.N) a.score[(((size_t)b * a.n_long + slot) * a.N + s) * nblk_all + u0 + bl] = smax[bl][q];
+      if (s < a.N) a.score[(((size_t)b * a.n_long + slot) * seg_n(a) + seg_at(a, s)) * nblk_all + u0 + bl] = smax[bl][q];
     }
     __syncthreads();
   }
@@ -154,12 +160,12 @@ __device__ __forceinline__ unsigned long long order_key(float z, int u) {
   return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)u);
 }
 
-// grid (N - 1, n_long, B): segment s = blockIdx.x + 1.  Dynamic shared
-// memory: next_pow2(blocks of the largest pool) 64-bit keys.
+// grid (N - s_lo, n_long, B): segment s = blockIdx.x + s_lo.  Dynamic
+// shared memory: next_pow2(blocks of the largest pool) 64-bit keys.
 __global__ void __launch_bounds__(kThreads) block_select_kernel(SegRetrArgs a) {
   extern __shared__ unsigned long long keys[];
   __shared__ int chosen[1024];
-  const int s = blockIdx.x + 1;
+  const int s = blockIdx.x + a.s_lo;
   const int slot = blockIdx.y;
   const int b = blockIdx.z;
   const int h = a.long_heads[slot];
@@ -169,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) block_select_kernel(SegRetrArgs a) {
   int P2 = 1;
   while (P2 < nblocks) P2 <<= 1;
   const int nblk_all = a.T / a.blk;
-  const float* score = a.score + (((size_t)b * a.n_long + slot) * a.N + s) * nblk_all;
+  const float* score = a.score + (((size_t)b * a.n_long + slot) * seg_n(a) + seg_at(a, s)) * nblk_all;
   for (int u = threadIdx.x; u < P2; u += kThreads) keys[u] = (u < nblocks) ? order_key(score[u], u) : 0ull;
   __syncthreads();
   // bitonic sort, descending
@@ -200,12 +206,12 @@ __global__ void __launch_bounds__(kThreads) block_select_kernel(SegRetrArgs a) {
     chosen[rank] = u;
   }
   __syncthreads();
-  if (threadIdx.x == 0) a.prefix_cnt[((size_t)b * a.n_long + slot) * a.N + s] = nsel * a.blk;
-  int32_t* out = a.prefix_blocks + (((size_t)b * a.Hq + h) * a.N + s) * nb;
+  if (threadIdx.x == 0) a.prefix_cnt[((size_t)b * a.n_long + slot) * seg_n(a) + seg_at(a, s)] = nsel * a.blk;
+  int32_t* out = a.prefix_blocks + (((size_t)b * a.Hq + h) * seg_n(a) + seg_at(a, s)) * nb;
   for (int x = threadIdx.x; x < nb; x += kThreads) out[x] = x < nsel ? chosen[x] : -1;
 }
 
-// grid (Rpad / 8, (N - 1) * n_long, B); one warp per prefix row.  Lanes
+// grid (Rpad / 8, (N - s_lo) * n_long, B); one warp per prefix row.  Lanes
 // [0, d/8) rotate 4 pairs of K each (8-byte loads from both halves, the
 // virtual position's cos/sin as two float4), lanes [16, 16 + d/8) copy 16
 // bytes of V each.
@@ -215,14 +221,14 @@ __global__ void prefix_assemble_kernel(SegRetrArgs a, int Rpad) {
   constexpr int kLanes = D / 8;  // K lanes (4 pairs each) = V lanes (16 bytes each)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x * 8 + warp;
-  const int s = blockIdx.y % (a.N - 1) + 1;
-  const int slot = blockIdx.y / (a.N - 1);
+  const int s = blockIdx.y % (a.N - a.s_lo) + a.s_lo;
+  const int slot = blockIdx.y / (a.N - a.s_lo);
   const int b = blockIdx.z;
   if (p >= Rpad) return;
   const int h = a.long_heads[slot];
   const int g = h / (a.Hq / a.Hkv);
-  const int cnt = a.prefix_cnt[((size_t)b * a.n_long + slot) * a.N + s];
-  const size_t orow = ((((size_t)b * a.n_long + slot) * a.N + s) * Rpad + p) * D;
+  const int cnt = a.prefix_cnt[((size_t)b * a.n_long + slot) * seg_n(a) + seg_at(a, s)];
+  const size_t orow = ((((size_t)b * a.n_long + slot) * seg_n(a) + seg_at(a, s)) * Rpad + p) * D;
   if (p >= cnt) {
     if (lane < kLanes) {
       reinterpret_cast<uint4*>(a.Kpre + orow)[lane] = make_uint4(0, 0, 0, 0);
@@ -231,7 +237,7 @@ __global__ void prefix_assemble_kernel(SegRetrArgs a, int Rpad) {
     return;
   }
   const int nb = a.R / a.blk;
-  const int blk_id = a.prefix_blocks[(((size_t)b * a.Hq + h) * a.N + s) * nb + p / a.blk];
+  const int blk_id = a.prefix_blocks[(((size_t)b * a.Hq + h) * seg_n(a) + seg_at(a, s)) * nb + p / a.blk];
   const int j = blk_id * a.blk + p % a.blk;
   const int vpos = s * a.S - cnt + p;
   if (lane < kLanes) {
@@ -295,12 +301,12 @@ cudaError_t launch_d(const SegRetrArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)P2 * sizeof(unsigned long long);
   cudaError_t e = cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 g2(a.N - 1, a.n_long, a.B);
+  dim3 g2(a.N - a.s_lo, a.n_long, a.B);
   block_select_kernel<<<g2, kThreads, smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int Rpad = (a.R + kTile - 1) / kTile * kTile;
-  dim3 g3(Rpad / 8, (a.N - 1) * a.n_long, a.B);
+  dim3 g3(Rpad / 8, (a.N - a.s_lo) * a.n_long, a.B);
   prefix_assemble_kernel<D><<<g3, 256, 0, st>>>(a, Rpad);
   return cudaGetLastError();
 }
@@ -319,7 +325,8 @@ bool segment_retrieval_supported(int T, int S, int blk) {
 }
 
 cudaError_t launch_segment_retrieval(const SegRetrArgs& a, cudaStream_t st) {
-  if (a.N <= 1 || a.n_long == 0 || a.R == 0 || a.B == 0) return cudaSuccess;
+  if (a.s_lo < 1 || a.s_base < 0 || a.s_base > a.s_lo) return cudaErrorInvalidValue;
+  if (a.N <= a.s_lo || a.n_long == 0 || a.R == 0 || a.B == 0) return cudaSuccess;
   if (a.d == 128) return launch_d<128>(a, st);
   if (a.d == 64) return launch_d<64>(a, st);
   return cudaErrorInvalidValue;

@@ -103,6 +103,33 @@ def test_segment_workspace(lib):
     assert lib.sattn_segment_workspace_size(ctypes.byref(p), 256, 64, 100, 64, il, ctypes.byref(n)) == -1
 
 
+def test_segment_stream_sizes_and_validation(lib):
+    """The carried state holds K, V and rotated K of every position of the
+    capacity plus the table; the step's workspace holds one segment's
+    queries and prefix.  Bad shapes and out-of-range steps are refused on the
+    host before any launch."""
+    n = ctypes.c_size_t(0)
+    il = (ctypes.c_uint8 * 4)(0, 0, 1, 1)
+    p = _p(Hq=4, Hkv=2, T=1024, rope_theta=1e4)
+    assert lib.sattn_segment_state_size(ctypes.byref(p), 256, 64, 128, 64, ctypes.byref(n)) == 0
+    kv = 2 * 1024 * 128 * 2  # one of K, V, rotated K: B * Hkv * T * d bf16
+    assert n.value >= 3 * kv + 1024 * 64 * 8
+    assert lib.sattn_segment_step_workspace_size(ctypes.byref(p), 256, 64, 128, 64, il, ctypes.byref(n)) == 0
+    assert n.value >= 4 * 256 * 128 * 2  # the segment's rotated queries
+    assert lib.sattn_segment_state_size(ctypes.byref(p), 100, 64, 128, 64, ctypes.byref(n)) == -1  # S % 128
+    assert lib.sattn_segment_state_size(ctypes.byref(p), 384, 64, 128, 64, ctypes.byref(n)) == -1  # T % S
+    assert lib.sattn_segment_state_size(ctypes.byref(p), 256, 64, 100, 64, ctypes.byref(n)) == -1  # R % blk
+    fake = ctypes.c_void_p(0x100000)  # never dereferenced: validation fails first
+    big = ctypes.c_size_t(1 << 40).value
+    for seg in (-1, 4):  # capacity 1024 = 4 segments
+        assert lib.sattn_segment_step(ctypes.byref(p), 256, 64, 128, 64, il, seg, fake, fake, fake, fake, big,
+                                      fake, fake, fake, fake, big, None) == -1
+    assert lib.sattn_segment_step(ctypes.byref(p), 256, 64, 128, 64, None, 0, fake, fake, fake, fake, big,
+                                  fake, fake, fake, fake, big, None) == -1  # is_long required
+    pa = _p(Hq=4, Hkv=2, T=1024, alibi=1)
+    assert lib.sattn_segment_state_size(ctypes.byref(pa), 256, 64, 128, 64, ctypes.byref(n)) == -2
+
+
 def test_entry_points_reject_bad_arguments_before_launch(lib):
     p = _p()
     rc, n = _ws(lib, p)
