@@ -365,7 +365,7 @@ struct TopkArgs {
   float* cand_thr;             // [B*Hq*T] the row's threshold (-inf: every candidate is listed)
   int32_t* cand_cnt;           // [B*Hq*T] keys above the threshold (> kCandCap: the list overflowed)
 };
-constexpr int kCandCap = 128;
+constexpr int kCandCap = 192;  // list entries per row (a multiple of 32)
 struct TopkMaps {
   CUtensorMap qsel, ksel;      // bf16 scoring operands: (Qc, K) capped, (Qr, Kr) otherwise
   CUtensorMap qsel2, ksel2;    // with 0 < window < L: (Qr, Kr) for the pairs within the cap
