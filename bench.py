@@ -75,7 +75,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # an ncu capture of the 4-head cut, times 8 for 32 heads (the launch is a grid
 # over heads and every head reads and writes the same amount); None when the
 # kernel changed since the counters were taken.
-TOPK_SCORE_TRAFFIC_BYTES = (61026560 + 12509952) * 8
+TOPK_SCORE_TRAFFIC_BYTES = (61482752 + 13227264) * 8
 # CPU-oracle rows per sample (about 10-30 s of host work on the GPU machine); the
 # top-k workload's oracle also scans every middle key per row
 CPU_ROWS = {"c4": 6144}
