@@ -529,13 +529,13 @@ __device__ __forceinline__ float exact_logit_bf16(const __nv_bfloat16* kp, const
 // ---------------------------------------------------------------------------
 // pass 2: exact re-rank of the candidate list + certificate
 // ---------------------------------------------------------------------------
-// A warp per row.  A coarse score c differs from the key's fp32 logit z by at
+// Per row: a coarse score c differs from the key's fp32 logit z by at
 // most eps (query rounding ||q - bf16(q)|| * max||k||, accumulation, and for
 // rotated keys their rounding).  If c' <= the k-th largest coarse score of the
 // list, at least k listed keys have z >= c' - eps, so the k-th fp32 logit
 // z_(k) >= c' - eps and only listed keys with c >= c' - 2 eps can be among the
 // top k.  c' is the k-th largest of the lanes' maxima (k distinct entries are
-// >= it).  The warp compacts the entries above the cut into shared memory,
+// >= it).  The row's lanes compact the entries above the cut into shared memory,
 // recomputes their logits in fp32 from the exact inputs (four lanes per key,
 // each a quarter of the rotary pairs, 16-byte key loads; the row's fp32
 // scoring query, R(L) q when capped and R(i) q otherwise, staged in shared
@@ -544,22 +544,32 @@ __device__ __forceinline__ float exact_logit_bf16(const __nv_bfloat16* kp, const
 // z <= tau + eps; the top k are exact when z_(k) > tau + eps (or tau = -inf:
 // the list holds every candidate).  Rows that fail, or whose list overflowed,
 // go to the exact rescan.
-constexpr int kRerankWarps = 8;
-constexpr int kPerLane = kCandCap / 32;
+// Two rows per warp, 16 lanes each: the per-row work that does not grow with
+// the list (the k rounds that find c', the query staging and its rounding
+// measure, the ranking, the certificate) is shared by two rows per warp
+// instruction; every shuffle stays inside its 16-lane group.
+constexpr int kRerankWarps = 6;  // (12 rows: the static shared memory of the dual case stays under 48 KB)
+constexpr int kRerankRows = 2 * kRerankWarps;  // rows per block
+constexpr int kPerLane = kCandCap / 16;
 
 template <int D, bool kDual>
 __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const TopkArgs a) {
   constexpr int half = D / 2;
-  constexpr int PPL = half / 32;   // rotary pairs staged per lane
+  constexpr int PPL = half / 16;   // rotary pairs staged per lane
   constexpr int QP = half / 4;     // rotary pairs per lane of a 4-lane group
-  __shared__ __align__(16) float sq[kRerankWarps][D];
-  __shared__ __align__(16) float sqc[kDual ? kRerankWarps : 1][kDual ? D : 4];  // R(L) q when 0 < w < L
-  __shared__ int sj[kRerankWarps][kCandCap];
-  __shared__ float2 se[kRerankWarps][kCandCap];
+  __shared__ __align__(16) float sq[kRerankRows][D];
+  __shared__ __align__(16) float sqc[kDual ? kRerankRows : 1][kDual ? D : 4];  // R(L) q when 0 < w < L
+  __shared__ int sj[kRerankRows][kCandCap];
+  __shared__ float2 se[kRerankRows][kCandCap];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 4, gl = lane & 15;  // the row group of the lane and its lane in it
+  const int slot = 2 * wid + grp;
+  const uint32_t lt = (1u << gl) - 1u;        // this lane's predecessors in its group
+  auto group_bits = [&](uint32_t ballot) { return (ballot >> (16 * grp)) & 0xFFFFu; };
   const int64_t nrows = (int64_t)a.B * a.Hq * a.T;
-  const int64_t row = (int64_t)blockIdx.x * kRerankWarps + wid;
-  if (row >= nrows) return;  // whole warps only: no block-wide barrier follows
+  const int64_t row0 = (int64_t)blockIdx.x * kRerankRows + slot;
+  const bool live = row0 < nrows;  // both groups of a warp take part in every shuffle
+  const int64_t row = live ? row0 : nrows - 1;
   const int i = (int)(row % a.T);
   const int64_t bh = row / a.T;
   const int h = (int)(bh % a.Hq), b = (int)(bh / a.Hq);
@@ -567,7 +577,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   // w >= L: every candidate is capped; 0 < w < L: those with i - j <= L are not
   constexpr bool dual = kDual;  // the launch picks it: a.L > 0 && a.window < a.L
   const bool capped_all = a.L > 0 && !dual;
-  const int cnt = a.cand_cnt[row];
+  const int cnt = live ? a.cand_cnt[row] : 0;
   const float tau = a.cand_thr[row];
   const int k = a.topk;
   const int n = min(cnt, kCandCap);
@@ -577,7 +587,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   float lm = -CUDART_INF_F;
 #pragma unroll
   for (int x = 0; x < kPerLane; ++x) {
-    const int e = lane + 32 * x;
+    const int e = gl + 16 * x;
     jl[x] = -1;
     c[x] = -CUDART_INF_F;
     if (e < n) {
@@ -594,32 +604,34 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   float dq2 = 0.f, qn2 = 0.f, dq2c = 0.f, qn2c = 0.f;
 #pragma unroll
   for (int e = 0; e < PPL; ++e) {
-    const int cc = lane * PPL + e;
+    const int cc = gl * PPL + e;
     const float x0 = __bfloat162float(qp[cc]), x1 = __bfloat162float(qp[cc + half]);
     const int64_t pos = capped_all ? a.L : i;
     const float2 cs = a.tab ? a.tab[pos * half + cc] : make_float2(1.f, 0.f);
     const float u0 = x0 * cs.x - x1 * cs.y, u1 = x1 * cs.x + x0 * cs.y;
-    sq[wid][cc] = u0;
-    sq[wid][cc + half] = u1;
+    sq[slot][cc] = u0;
+    sq[slot][cc + half] = u1;
     const float b0 = __bfloat162float(__float2bfloat16_rn(u0)), b1 = __bfloat162float(__float2bfloat16_rn(u1));
     dq2 += (u0 - b0) * (u0 - b0) + (u1 - b1) * (u1 - b1);
     qn2 += b0 * b0 + b1 * b1;
     if constexpr (kDual) {
       const float2 cl = a.tab ? a.tab[(int64_t)a.L * half + cc] : make_float2(1.f, 0.f);
       const float w0 = x0 * cl.x - x1 * cl.y, w1 = x1 * cl.x + x0 * cl.y;
-      sqc[wid][cc] = w0;
-      sqc[wid][cc + half] = w1;
+      sqc[slot][cc] = w0;
+      sqc[slot][cc + half] = w1;
       const float c0 = __bfloat162float(__float2bfloat16_rn(w0)), c1 = __bfloat162float(__float2bfloat16_rn(w1));
       dq2c += (w0 - c0) * (w0 - c0) + (w1 - c1) * (w1 - c1);
       qn2c += c0 * c0 + c1 * c1;
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = 8; o > 0; o >>= 1) {
     dq2 += __shfl_xor_sync(0xffffffffu, dq2, o);
     qn2 += __shfl_xor_sync(0xffffffffu, qn2, o);
-    dq2c += __shfl_xor_sync(0xffffffffu, dq2c, o);
-    qn2c += __shfl_xor_sync(0xffffffffu, qn2c, o);
+    if constexpr (kDual) {
+      dq2c += __shfl_xor_sync(0xffffffffu, dq2c, o);
+      qn2c += __shfl_xor_sync(0xffffffffu, qn2c, o);
+    }
   }
   const float kmax = __uint_as_float(a.kmax[(size_t)b * a.Hkv + g]) * (1.f + 1.f / 128.f);
   const float qn = sqrtf(qn2);
@@ -632,16 +644,17 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   }
   eps *= 1.0625f;
 
-  // c' = the k-th largest lane maximum (-inf when fewer than k lanes hold entries)
+  // c' = the k-th largest lane maximum of the group (-inf when fewer than k
+  // lanes hold entries)
   float cp = -CUDART_INF_F;
   {
     float mv = lm;
-    for (int rr = 0; rr < k; ++rr) {
+    for (int r = 0; r < k; ++r) {
       float wz = mv;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wz = fmaxf(wz, __shfl_xor_sync(0xffffffffu, wz, o));
-      const uint32_t holders = __ballot_sync(0xffffffffu, mv == wz);
-      if (lane == __ffs(holders) - 1) mv = -CUDART_INF_F;
+      for (int o = 8; o > 0; o >>= 1) wz = fmaxf(wz, __shfl_xor_sync(0xffffffffu, wz, o));
+      const uint32_t holders = group_bits(__ballot_sync(0xffffffffu, mv == wz));
+      if (gl == __ffs(holders) - 1) mv = -CUDART_INF_F;
       cp = wz;
     }
   }
@@ -651,26 +664,28 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
 #pragma unroll
   for (int x = 0; x < kPerLane; ++x) {
     const bool p = jl[x] >= 0 && c[x] >= cut;
-    const uint32_t bal = __ballot_sync(0xffffffffu, p);
-    if (p) sj[wid][m + __popc(bal & ((1u << lane) - 1u))] = jl[x];
+    const uint32_t bal = group_bits(__ballot_sync(0xffffffffu, p));
+    if (p) sj[slot][m + __popc(bal & lt)] = jl[x];
     m += __popc(bal);
   }
   __syncwarp();
-  // fp32 logits: four lanes per entry, a quarter of the rotary pairs each
+  // fp32 logits: four lanes per entry, a quarter of the rotary pairs each;
+  // both groups run the loop as often as the longer of the two needs
+  const int m_warp = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
   const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.K) + b * a.k_sb + g * a.k_sh;
-  const int quarter = lane & 3;
-  for (int e0 = 0; e0 < m; e0 += 8) {
-    const int e = e0 + (lane >> 2);
+  const int quarter = gl & 3;
+  for (int e0 = 0; e0 < m_warp; e0 += 4) {
+    const int e = e0 + (gl >> 2);
     float acc = 0.f;
     int j = -1;
     if (e < m) {
-      j = sj[wid][e];
+      j = sj[slot][e];
       // the pair's operands: capped (R(L) q, raw key) or rotated (R(i) q, R(j) k)
       bool cap = capped_all;
-      const float* qv = sq[wid];
+      const float* qv = sq[slot];
       if constexpr (kDual) {
         cap = i - j > a.L;
-        if (cap) qv = sqc[wid];
+        if (cap) qv = sqc[slot];
       }
       const __nv_bfloat16* kp = kbase + (int64_t)j * a.k_st;
       float A0 = 0.f, A1 = 0.f;
@@ -711,34 +726,35 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (e < m && quarter == 0) se[wid][e] = make_float2(acc, __int_as_float(j));
+    if (e < m && quarter == 0) se[slot][e] = make_float2(acc, __int_as_float(j));
   }
   __syncwarp();
   // rank by counting: entry e precedes entry f when z_e > z_f, or equal with j_e < j_f
   float zk = -CUDART_INF_F;
-  for (int e = lane; e < m; e += 32) {
-    const float2 me = se[wid][e];
+  for (int e = gl; e < m; e += 16) {
+    const float2 me = se[slot][e];
     const int mj = __float_as_int(me.y);
     int rank = 0;
     for (int f = 0; f < m; ++f) {
-      const float2 o = se[wid][f];
+      const float2 o = se[slot][f];
       const int oj = __float_as_int(o.y);
       rank += (o.x > me.x || (o.x == me.x && oj < mj)) ? 1 : 0;
     }
-    if (rank < k) {
+    if (rank < k && live) {
       a.idx[row * k + rank] = mj;
       a.z[row * k + rank] = me.x;
     }
     if (rank == k - 1) zk = me.x;
   }
-  for (int r = m + lane; r < k; r += 32) {  // fewer than k entries: pad
-    a.idx[row * k + r] = -1;
-    a.z[row * k + r] = -CUDART_INF_F;
-  }
+  if (live)
+    for (int r = m + gl; r < k; r += 16) {  // fewer than k entries: pad
+      a.idx[row * k + r] = -1;
+      a.z[row * k + r] = -CUDART_INF_F;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) zk = fmaxf(zk, __shfl_xor_sync(0xffffffffu, zk, o));
+  for (int o = 8; o > 0; o >>= 1) zk = fmaxf(zk, __shfl_xor_sync(0xffffffffu, zk, o));
   const bool certified = cnt <= kCandCap && (tau == -CUDART_INF_F || zk > tau + eps);
-  if (!certified && lane == 0) {
+  if (live && !certified && gl == 0) {
     const int pos = atomicAdd(a.status + 2, 1);
     a.fallback_rows[pos] = (int32_t)row;
   }
@@ -859,7 +875,7 @@ cudaError_t launch_topk_score(const TopkArgs& a, const TopkMaps& m, cudaStream_t
 cudaError_t launch_topk_rerank(const TopkArgs& a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.B * a.Hq * a.T;
   if (rows == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)((rows + kRerankWarps - 1) / kRerankWarps);
+  const unsigned blocks = (unsigned)((rows + kRerankRows - 1) / kRerankRows);
   const bool dual = a.L > 0 && a.window < a.L;
   if (a.d == 128) {
     if (dual) topk_rerank_kernel<128, true><<<blocks, kRerankWarps * 32, 0, st>>>(a);
