@@ -1224,7 +1224,8 @@ static int plan_tree(const sattn_params* p, int32_t n_chunks, int32_t chunk_len,
 
 struct DecPlan {
   int nQT, npos, n_chunks;
-  Region status, tab, prefix, sep_pos, sep_count, ranges, part, tk_zall, tk_idx, tk_z, tk_part;
+  Region status, tab, prefix, sep_pos, sep_count, ranges, part, tk_cz, tk_cj, tk_idx, tk_z, tk_part;
+  int tk_nchunks = 0;
   size_t total;
 };
 
@@ -1254,7 +1255,10 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   }
   P.part = A.take(B * Hq * (size_t)P.n_chunks * (d + 2) * 4);
   if (p->topk > 0) {
-    P.tk_zall = A.take(B * Hq * T * 4);
+    P.tk_nchunks = decode_topk_chunks(p->T - 1 - p->window - p->n_start);
+    const size_t nc = (size_t)std::max(P.tk_nchunks, 1) * p->topk;
+    P.tk_cz = A.take(B * Hq * nc * 4);
+    P.tk_cj = A.take(B * Hq * nc * 4);
     P.tk_idx = A.take(B * Hq * (size_t)p->topk * 4);
     P.tk_z = A.take(B * Hq * (size_t)p->topk * 4);
     P.tk_part = A.take(B * Hq * (d + 2) * 4);
@@ -1343,7 +1347,9 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   a.n_chunks = P.n_chunks;
   if (p->topk > 0) {
     a.topk = p->topk;
-    a.tk_zall = at<float>(ws, P.tk_zall);
+    a.tk_nchunks = P.tk_nchunks;
+    a.tk_cz = at<float>(ws, P.tk_cz);
+    a.tk_cj = at<int32_t>(ws, P.tk_cj);
     a.tk_idx = topk_idx ? topk_idx : at<int32_t>(ws, P.tk_idx);
     a.tk_z = topk_logit ? topk_logit : at<float>(ws, P.tk_z);
     a.tk_part = at<float>(ws, P.tk_part);

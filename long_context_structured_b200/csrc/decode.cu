@@ -334,12 +334,15 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 
 // grid (B * Hkv, candidate chunks of kChunk positions): every candidate's
 // logit for every query head of the group (the logit pass over consecutive
-// positions) into tk_zall.  Separators are scored too and skipped by the
-// selection.
+// positions), then per head the chunk's k best (separators excluded by
+// their flag bit) into tk_cz / tk_cj: the top k of the whole row is the top
+// k of the chunks' top k, so the selection merges k entries per chunk
+// rather than every candidate.
 template <int D, int REP>
 __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs a) {
   using TL = Tiling<D, REP>;
   constexpr int EPL = TL::EPL, LPK = TL::LPK, KPW = TL::KPW;
+  __shared__ float s_z[REP][kChunk];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % a.Hkv, b = blockIdx.x / a.Hkv;
   const int i = a.T - 1;
@@ -350,21 +353,67 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   float q0[REP][EPL], q1[REP][EPL];
   rotated_query<D, REP>(a, b, g, i, p0, q0, q1);
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
-  float* zb = a.tk_zall + ((size_t)b * a.Hq + (size_t)g * REP) * a.T;
+  const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
   logits_pass<D, REP>(
       a, i, kb, warp * KPW, lane, q0, q1, [&](int el) { return j0 + el < jend ? j0 + el : -1; },
-      [&](int r, int, int j, float dot) {
-        if (j >= 0) zb[(size_t)r * a.T + j] = dot;
+      [&](int r, int el, int j, float dot) {
+        const bool sep = j >= 0 && words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u);
+        s_z[r][el] = (j >= 0 && !sep) ? dot : -CUDART_INF_F;
       });
+  __syncthreads();
+  // per head: k rounds of a warp argmax by (z desc, j asc) over the chunk
+  // (lane l holds keys l, l + 32, l + 64, l + 96)
+  const int k = a.topk;
+  const int chunk = blockIdx.y;
+  for (int r = warp; r < REP; r += kThreads / 32) {
+    float zv[kChunk / 32];
+    int jv[kChunk / 32];
+#pragma unroll
+    for (int u = 0; u < kChunk / 32; ++u) {
+      const int el = lane + 32 * u;
+      zv[u] = s_z[r][el];
+      jv[u] = (zv[u] == -CUDART_INF_F) ? -1 : j0 + el;
+    }
+    const size_t base = (((size_t)b * a.Hq + (size_t)g * REP + r) * a.tk_nchunks + chunk) * k;
+    for (int y = 0; y < k; ++y) {
+      float bz = -CUDART_INF_F;
+      int bj = -1;
+#pragma unroll
+      for (int u = 0; u < kChunk / 32; ++u)
+        if (sel_before(zv[u], jv[u], bz, bj)) {
+          bz = zv[u];
+          bj = jv[u];
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (sel_before(oz, oj, bz, bj)) {
+          bz = oz;
+          bj = oj;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kChunk / 32; ++u)
+        if (jv[u] == bj && bj >= 0) {  // the winner leaves its list (positions are distinct)
+          jv[u] = -1;
+          zv[u] = -CUDART_INF_F;
+        }
+      if (lane == 0) {
+        a.tk_cz[base + y] = bj >= 0 ? bz : -CUDART_INF_F;
+        a.tk_cj[base + y] = bj;
+      }
+    }
+  }
 }
 
 constexpr int kSelThreads = 512;
 constexpr int kSelMaxK = 16;
 
-// grid (B * Hq): the k best candidates of one (batch, head) -- a strided
-// pass keeping a sorted list per thread, then k rounds of a block argmax --
-// written out, and the selected keys' softmax partial (their maximum, sum of
-// weights and weighted V rows) for the chunk merge.
+// grid (B * Hq): the k best candidates of one (batch, head) from the chunks'
+// top k -- a strided pass keeping a sorted list per thread, then k rounds of
+// a block argmax -- written out, and the selected keys' softmax partial
+// (their maximum, sum of weights and weighted V rows) for the chunk merge.
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeArgs a) {
   __shared__ float red_z[kSelThreads / 32];
@@ -373,10 +422,9 @@ __global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeA
   __shared__ int s_j[kSelMaxK];
   const int bh = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq, g = h / (a.Hq / a.Hkv);
-  const int i = a.T - 1;
-  const int jend = i - a.window;
-  const float* zr = a.tk_zall + (size_t)bh * a.T;
-  const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
+  const int n_c = a.tk_nchunks * a.topk;  // the chunks' picks (-1 padding)
+  const float* czr = a.tk_cz + (size_t)bh * n_c;
+  const int32_t* cjr = a.tk_cj + (size_t)bh * n_c;
   float vals[kSelMaxK];
   int idxs[kSelMaxK];
 #pragma unroll
@@ -384,12 +432,28 @@ __global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeA
     vals[y] = -CUDART_INF_F;
     idxs[y] = -1;
   }
-  // each thread visits its positions in increasing order, so a strict >
-  // leaves the smaller position first among equal logits
-  for (int j = a.n_start + (int)threadIdx.x; j < jend; j += kSelThreads) {
-    if (words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u)) continue;
-    const float z = zr[j];
-    if (z > vals[kSelMaxK - 1]) list_insert<kSelMaxK>(z, j, vals, idxs);
+  // each thread visits its entries in increasing position order (chunks in
+  // order, each chunk's picks by (z desc, j asc) but a thread sees one
+  // chunk's entries a stride apart), so ties are settled by position
+  for (int e = (int)threadIdx.x; e < n_c; e += kSelThreads) {
+    const int j = cjr[e];
+    if (j < 0) continue;
+    const float z = czr[e];
+    if (sel_before(z, j, vals[kSelMaxK - 1], idxs[kSelMaxK - 1])) {
+      float v = z;
+      int jj = j;
+#pragma unroll
+      for (int y = 0; y < kSelMaxK; ++y) {
+        if (sel_before(v, jj, vals[y], idxs[y])) {
+          const float tv = vals[y];
+          const int tj = idxs[y];
+          vals[y] = v;
+          idxs[y] = jj;
+          v = tv;
+          jj = tj;
+        }
+      }
+    }
   }
   block_topk_rounds<kSelMaxK>(a.topk, vals, idxs, red_z, red_j, [&](int r, float wz, int wj) {
     s_j[r] = wj;
@@ -507,7 +571,7 @@ cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
   if (a.topk > 0) {
     const int ncand = a.T - 1 - a.window - a.n_start;
     if (ncand > 0) {
-      dim3 gt(a.B * a.Hkv, (ncand + kChunk - 1) / kChunk);
+      dim3 gt(a.B * a.Hkv, a.tk_nchunks);
       decode_topk_logits_kernel<D, REP><<<gt, kThreads, 0, st>>>(a);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
@@ -538,6 +602,7 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 int decode_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+int decode_topk_chunks(int n_candidates) { return n_candidates > 0 ? (n_candidates + kChunk - 1) / kChunk : 0; }
 int decode_max_len() { return kCombineMaxChunks * kChunk; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {

@@ -474,7 +474,9 @@ struct DecodeArgs {
   int n_chunks;
   // top-k middle tokens of the query (topk > 0; seq_len must be null)
   int topk;
-  float* tk_zall;               // [B, Hq, T] candidate logits (unscaled)
+  int tk_nchunks;                // candidate chunks of 128 positions (decode_topk_chunks)
+  float* tk_cz;                 // [B, Hq, tk_nchunks, topk] each chunk's best logits (unscaled)
+  int32_t* tk_cj;               // [B, Hq, tk_nchunks, topk] their positions (-1 padding)
   int32_t* tk_idx;              // [B, Hq, topk] the selection (-1 padding)
   float* tk_z;                  // [B, Hq, topk] its logits (-inf padding)
   float* tk_part;               // [B, Hq, d + 2] the selected keys' partial (max, sum, O)
@@ -484,6 +486,7 @@ struct DecodeArgs {
 };
 // chunks of kept keys a decoding step of cache length T may need
 int decode_chunks(int T);
+int decode_topk_chunks(int n_candidates);  // candidate chunks of the top-k logit pass
 int decode_max_len();  // longest key set one decoding step merges
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
