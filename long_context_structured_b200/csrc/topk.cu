@@ -544,28 +544,31 @@ __device__ __forceinline__ float exact_logit_bf16(const __nv_bfloat16* kp, const
 // z <= tau + eps; the top k are exact when z_(k) > tau + eps (or tau = -inf:
 // the list holds every candidate).  Rows that fail, or whose list overflowed,
 // go to the exact rescan.
-// Two rows per warp, 16 lanes each: the per-row work that does not grow with
-// the list (the k rounds that find c', the query staging and its rounding
-// measure, the ranking, the certificate) is shared by two rows per warp
-// instruction; every shuffle stays inside its 16-lane group.
-constexpr int kRerankWarps = 6;  // (12 rows: the static shared memory of the dual case stays under 48 KB)
-constexpr int kRerankRows = 2 * kRerankWarps;  // rows per block
-constexpr int kPerLane = kCandCap / 16;
+// kRerankG lanes per row, 32 / kRerankG rows per warp: the per-row work that
+// does not grow with the list (the k rounds that find c', the query staging
+// and its rounding measure, the ranking, the certificate) is shared by the
+// warp's rows per instruction; every shuffle stays inside its lane group.
+constexpr int kRerankG = 16;                   // lanes per row (8 measured slower: 0.94 vs 0.74 ms)
+constexpr int kRerankRows = 12;                // rows per block (the dual case's static shared memory < 48 KB)
+constexpr int kRerankWarps = kRerankRows * kRerankG / 32;
+constexpr int kPerLane = kCandCap / kRerankG;
+static_assert(kRerankRows * kRerankG % 32 == 0 && kCandCap % kRerankG == 0, "re-rank tiling");
 
 template <int D, bool kDual>
 __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const TopkArgs a) {
   constexpr int half = D / 2;
-  constexpr int PPL = half / 16;   // rotary pairs staged per lane
+  constexpr int G = kRerankG;
+  constexpr int PPL = half / G;    // rotary pairs staged per lane
   constexpr int QP = half / 4;     // rotary pairs per lane of a 4-lane group
   __shared__ __align__(16) float sq[kRerankRows][D];
   __shared__ __align__(16) float sqc[kDual ? kRerankRows : 1][kDual ? D : 4];  // R(L) q when 0 < w < L
   __shared__ int sj[kRerankRows][kCandCap];
   __shared__ float2 se[kRerankRows][kCandCap];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane >> 4, gl = lane & 15;  // the row group of the lane and its lane in it
-  const int slot = 2 * wid + grp;
+  const int grp = lane / G, gl = lane % G;  // the row group of the lane and its lane in it
+  const int slot = (32 / G) * wid + grp;
   const uint32_t lt = (1u << gl) - 1u;        // this lane's predecessors in its group
-  auto group_bits = [&](uint32_t ballot) { return (ballot >> (16 * grp)) & 0xFFFFu; };
+  auto group_bits = [&](uint32_t ballot) { return (ballot >> (G * grp)) & ((1u << G) - 1u); };
   const int64_t nrows = (int64_t)a.B * a.Hq * a.T;
   const int64_t row0 = (int64_t)blockIdx.x * kRerankRows + slot;
   const bool live = row0 < nrows;  // both groups of a warp take part in every shuffle
@@ -587,7 +590,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   float lm = -CUDART_INF_F;
 #pragma unroll
   for (int x = 0; x < kPerLane; ++x) {
-    const int e = gl + 16 * x;
+    const int e = gl + G * x;
     jl[x] = -1;
     c[x] = -CUDART_INF_F;
     if (e < n) {
@@ -625,7 +628,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     }
   }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) {
+  for (int o = G / 2; o > 0; o >>= 1) {
     dq2 += __shfl_xor_sync(0xffffffffu, dq2, o);
     qn2 += __shfl_xor_sync(0xffffffffu, qn2, o);
     if constexpr (kDual) {
@@ -652,7 +655,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     for (int r = 0; r < k; ++r) {
       float wz = mv;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) wz = fmaxf(wz, __shfl_xor_sync(0xffffffffu, wz, o));
+      for (int o = G / 2; o > 0; o >>= 1) wz = fmaxf(wz, __shfl_xor_sync(0xffffffffu, wz, o));
       const uint32_t holders = group_bits(__ballot_sync(0xffffffffu, mv == wz));
       if (gl == __ffs(holders) - 1) mv = -CUDART_INF_F;
       cp = wz;
@@ -671,10 +674,12 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   __syncwarp();
   // fp32 logits: four lanes per entry, a quarter of the rotary pairs each;
   // both groups run the loop as often as the longer of the two needs
-  const int m_warp = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+  int m_warp = m;
+#pragma unroll
+  for (int o = G; o < 32; o <<= 1) m_warp = max(m_warp, __shfl_xor_sync(0xffffffffu, m_warp, o));
   const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.K) + b * a.k_sb + g * a.k_sh;
   const int quarter = gl & 3;
-  for (int e0 = 0; e0 < m_warp; e0 += 4) {
+  for (int e0 = 0; e0 < m_warp; e0 += G / 4) {
     const int e = e0 + (gl >> 2);
     float acc = 0.f;
     int j = -1;
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
   __syncwarp();
   // rank by counting: entry e precedes entry f when z_e > z_f, or equal with j_e < j_f
   float zk = -CUDART_INF_F;
-  for (int e = gl; e < m; e += 16) {
+  for (int e = gl; e < m; e += G) {
     const float2 me = se[slot][e];
     const int mj = __float_as_int(me.y);
     int rank = 0;
@@ -747,12 +752,12 @@ __global__ void __launch_bounds__(kRerankWarps * 32) topk_rerank_kernel(const To
     if (rank == k - 1) zk = me.x;
   }
   if (live)
-    for (int r = m + gl; r < k; r += 16) {  // fewer than k entries: pad
+    for (int r = m + gl; r < k; r += G) {  // fewer than k entries: pad
       a.idx[row * k + r] = -1;
       a.z[row * k + r] = -CUDART_INF_F;
     }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) zk = fmaxf(zk, __shfl_xor_sync(0xffffffffu, zk, o));
+  for (int o = G / 2; o > 0; o >>= 1) zk = fmaxf(zk, __shfl_xor_sync(0xffffffffu, zk, o));
   const bool certified = cnt <= kCandCap && (tau == -CUDART_INF_F || zk > tau + eps);
   if (live && !certified && gl == 0) {
     const int pos = atomicAdd(a.status + 2, 1);
