@@ -301,3 +301,95 @@ def test_stream_cache():
     for gg, name in ((go, "O"), (gl, "lse"), (ws, "workspace"), (st, "stream state")):
         gg.check(name)
     gaps_untouched(go, shape, 128, spo, q.dtype, "O")
+
+
+def test_decode_topk_fwd():
+    L = _lib.load()
+    cfg = dict(B=2, Hq=8, Hkv=2, T=1200, d=128, n_start=4, window=64, L_pretrain=200, rope_theta=1e4, topk=5,
+               sep_rate=0.1)
+    wl, inp, q, k, v, sep = _inputs(cfg)
+    qd = q[:, :, -1:, :].contiguous()
+    shape = (wl.B, wl.Hq, 1, wl.d)
+    go, O, sp = padded(shape, wl.d, qd.dtype)
+    gl = Guarded(wl.B * wl.Hq * 4)
+    gi = Guarded(wl.B * wl.Hq * wl.topk * 4)
+    gz = Guarded(wl.B * wl.Hq * wl.topk * 4)
+    p = sa.params(qd, k, v, O, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, topk=wl.topk,
+                  rope_theta=wl.rope_theta, with_separators=True)
+    p.T = wl.T
+    ws, nb = _ws(L.sattn_decode_workspace_size, ctypes.byref(p))
+    rc = L.sattn_decode_topk_fwd(ctypes.byref(p), ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                 ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(sep.data_ptr()), go.ptr, gl.ptr,
+                                 gi.ptr, gz.ptr, ws.ptr, nb, _stream())
+    assert rc == 0
+    for g, name in ((go, "O"), (gl, "lse"), (gi, "topk_idx"), (gz, "topk_logit"), (ws, "workspace")):
+        g.check(name)
+    gaps_untouched(go, shape, wl.d, sp, qd.dtype, "O")
+    O_ref, _, idx_ref, z_ref = sa.decode_fwd(qd, k, v, n_start=wl.n_start, window=wl.window,
+                                             L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta, is_sep=sep,
+                                             topk=wl.topk, return_topk=True)
+    assert torch.equal(O, O_ref)
+    assert torch.equal(gi.view(torch.int32, idx_ref.shape), idx_ref)
+    assert torch.equal(gz.view(torch.float32, z_ref.shape), z_ref)
+
+
+def test_fwd_topk_window_below_cap():
+    """The two-operand selector instantiation (window below the cap) and the
+    separators' extended band."""
+    L = _lib.load()
+    cfg = dict(B=1, Hq=4, Hkv=2, T=900, d=128, n_start=4, window=64, L_pretrain=256, rope_theta=1e4, topk=4,
+               sep_rate=0.1)
+    wl, inp, q, k, v, sep = _inputs(cfg)
+    shape = (wl.B, wl.Hq, wl.T, wl.d)
+    go, O, sp = padded(shape, wl.d, q.dtype)
+    gl = Guarded(wl.B * wl.Hq * wl.T * 4)
+    p = sa.params(q, k, v, O, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, topk=wl.topk,
+                  rope_theta=wl.rope_theta, with_separators=True)
+    ws, nb = _ws(L.sattn_workspace_size, ctypes.byref(p))
+    rc = L.sattn_fwd(ctypes.byref(p), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                     ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(sep.data_ptr()), None, None, go.ptr, gl.ptr,
+                     ws.ptr, nb, _stream())
+    assert rc == 0
+    for g, name in ((go, "O"), (gl, "lse"), (ws, "workspace")):
+        g.check(name)
+    gaps_untouched(go, shape, wl.d, sp, q.dtype, "O")
+    O_ref, l_ref = sa.fwd(q, k, v, n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, topk=wl.topk,
+                          rope_theta=wl.rope_theta, is_sep=sep)
+    assert torch.equal(O, O_ref) and torch.equal(gl.view(torch.float32, (wl.B, wl.Hq, wl.T)), l_ref)
+
+
+def test_segment_step():
+    """The carried state and every step's outputs and workspace."""
+    L = _lib.load()
+    cfg = dict(B=1, Hq=4, Hkv=2, T=768, d=128, rope_theta=1e4, seg_S=256, seg_M=64, seg_R=128, retr_block=64,
+               long_heads=(1, 2))
+    wl, inp, q, k, v, _ = _inputs(cfg)
+    S, N, nb_blk = wl.seg_S, wl.T // wl.seg_S, wl.seg_R // wl.retr_block
+    il = (ctypes.c_uint8 * wl.Hq)(*[int(x) for x in inp["is_long"]])
+    seg = lambda t, s: t[:, :, s * S:(s + 1) * S].contiguous()
+    shape = (wl.B, wl.Hq, S, wl.d)
+    go, O, sp = padded(shape, wl.d, q.dtype)
+    p = sa.params(seg(q, 0), seg(k, 0), seg(v, 0), O, rope_theta=wl.rope_theta)
+    p.T = wl.T  # the capacity
+    n = ctypes.c_size_t(0)
+    assert L.sattn_segment_state_size(ctypes.byref(p), S, wl.seg_M, wl.seg_R, wl.retr_block, ctypes.byref(n)) == 0
+    st = Guarded(int(n.value))
+    assert L.sattn_segment_state_reset(ctypes.byref(p), S, wl.seg_M, wl.seg_R, wl.retr_block, st.ptr, int(n.value),
+                                       _stream()) == 0
+    ws, nb = _ws(L.sattn_segment_step_workspace_size, ctypes.byref(p), S, wl.seg_M, wl.seg_R, wl.retr_block, il)
+    O_ref, _, pb_ref = sa.segment_fwd(q, k, v, S=S, M=wl.seg_M, R=wl.seg_R, retr_block=wl.retr_block,
+                                      is_long=inp["is_long"], rope_theta=wl.rope_theta)
+    for s in range(N):
+        gl = Guarded(wl.B * wl.Hq * S * 4)
+        gp = Guarded(wl.B * wl.Hq * nb_blk * 4)
+        qs, ks, vs = seg(q, s), seg(k, s), seg(v, s)
+        rc = L.sattn_segment_step(ctypes.byref(p), S, wl.seg_M, wl.seg_R, wl.retr_block, il, s,
+                                  ctypes.c_void_p(qs.data_ptr()), ctypes.c_void_p(ks.data_ptr()),
+                                  ctypes.c_void_p(vs.data_ptr()), st.ptr, int(n.value), go.ptr, gl.ptr, gp.ptr,
+                                  ws.ptr, nb, _stream())
+        assert rc == 0
+        for g, name in ((go, "O"), (gl, "lse"), (gp, "prefix_blocks"), (ws, "workspace"), (st, "state")):
+            g.check("%s (segment %d)" % (name, s))
+        gaps_untouched(go, shape, wl.d, sp, q.dtype, "O")
+        assert torch.equal(O, O_ref[:, :, s * S:(s + 1) * S])
+        assert torch.equal(gp.view(torch.int32, (wl.B, wl.Hq, nb_blk)), pb_ref[:, :, s])
