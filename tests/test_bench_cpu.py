@@ -81,3 +81,31 @@ def test_decode_key_counts_match_oracle(oracle_mod):
         *_, cnt = O.fwd_rows(O.params_of(wl.scaled(topk=0)), inp["q"], inp["k"], inp["v"], inp["is_sep"], rows,
                              nthreads=2)
         assert list(bench.decode_keys(wl, inp["is_sep"])) == list(cnt)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_head_split_work_adds_up(world):
+    """The strong-scaling mode reports the whole layer's FLOPs: the ranks'
+    head blocks (whole kv groups) count exactly the layer's kept pairs."""
+    from long_context_structured_b200.shard import head_shard
+    wl = synth.Workload(name="sep", B=2, Hq=16, Hkv=8, T=300, d=16, dtype="bf16", n_start=3, window=20,
+                        rope_theta=5e5, sep_rate=0.2)
+    inp = synth.make_inputs(wl, seed=4)
+    total = bench.unmasked_pairs(wl, inp["is_sep"])
+    parts = 0
+    for r in range(world):
+        q0, q1, kv0, kv1 = head_shard(wl.Hq, wl.Hkv, world, r)
+        if q1 > q0:
+            parts += bench.unmasked_pairs(wl.scaled(Hq=q1 - q0, Hkv=kv1 - kv0), inp["is_sep"])
+    assert parts == total
+
+
+def test_decode_topk_pairs():
+    """A decoding step with top-k keeps the structured keys plus k middle
+    keys per head (fewer when fewer candidates exist)."""
+    wl = synth.Workload(name="d", B=1, Hq=4, Hkv=4, T=100, d=16, dtype="bf16", n_start=4, window=30,
+                        L_pretrain=30, rope_theta=1e4, topk=5)
+    keys = bench.decode_keys(wl, None)
+    assert int(keys[0]) == 4 + 31  # sinks + window (i - w .. i)
+    ncand = wl.T - 1 - wl.window - wl.n_start
+    assert ncand == 65 and min(wl.topk, ncand) == 5
