@@ -94,6 +94,10 @@ typedef struct sattn_params {
                          SATTN_ERR_UNSUPPORTED: with top-k unless L_pretrain > 0 and
                          window >= L_pretrain; with separators on the bf16 path unless
                          L_pretrain > 0; in sattn_segment_fwd */
+  int32_t tile_m;     /* query tile (rows per tile of the block map and the kernels): 0 or 128 */
+  int32_t tile_n;     /* key tile: 0 or 128.  The kernels are built for 128 x 128 tiles (the
+                         tensor-core tile and the TMEM layout); other sizes return
+                         SATTN_ERR_UNSUPPORTED */
 } sattn_params;
 
 /* Text of a status code (static storage). */

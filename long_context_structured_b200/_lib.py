@@ -47,7 +47,8 @@ class SattnParams(ctypes.Structure):
         ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
         ("n_start", ctypes.c_int32), ("window", ctypes.c_int32), ("L_pretrain", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("with_separators", ctypes.c_int32), ("rope_theta", ctypes.c_double),
-        ("rope_pos_scale", ctypes.c_double), ("alibi", ctypes.c_int32),
+        ("rope_pos_scale", ctypes.c_double), ("alibi", ctypes.c_int32), ("tile_m", ctypes.c_int32),
+        ("tile_n", ctypes.c_int32),
     ]
 
 

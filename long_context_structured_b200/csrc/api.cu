@@ -69,6 +69,7 @@ int check_common(const sattn_params* p) {
   if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->T < 1) return SATTN_ERR_INVALID_ARG;
   if (p->Hq % p->Hkv) return SATTN_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SATTN_ERR_UNSUPPORTED;
+  if ((p->tile_m != 0 && p->tile_m != kTile) || (p->tile_n != 0 && p->tile_n != kTile)) return SATTN_ERR_UNSUPPORTED;
   if (p->dtype != SATTN_DTYPE_BF16 && p->dtype != SATTN_DTYPE_F32) return SATTN_ERR_INVALID_ARG;
   if (p->n_start < 0 || p->window < 0 || p->L_pretrain < 0 || p->topk < 0) return SATTN_ERR_INVALID_ARG;
   if (p->topk > 16) return SATTN_ERR_UNSUPPORTED;

@@ -75,6 +75,10 @@ def test_workspace_size_and_validation(lib):
     # top-k with the window below the cap is taken, except with the ALiBi bias
     assert _ws(lib, _p(window=30, L_pretrain=50, topk=2))[0] == 0
     assert _ws(lib, _p(window=30, L_pretrain=50, topk=2, alibi=1, rope_theta=0.0))[0] == _lib.SATTN_ERR_UNSUPPORTED
+    # tiles: 128 x 128 (or 0, the default) only
+    assert _ws(lib, _p(tile_m=128, tile_n=128))[0] == 0
+    assert _ws(lib, _p(tile_m=64))[0] == _lib.SATTN_ERR_UNSUPPORTED
+    assert _ws(lib, _p(tile_n=256))[0] == _lib.SATTN_ERR_UNSUPPORTED
     # separators with the window below the cap are taken
     assert _ws(lib, _p(window=30, L_pretrain=50, with_separators=1))[0] == 0
     assert _ws(lib, _p(dtype=7))[0] == _lib.SATTN_ERR_INVALID_ARG
