@@ -1225,10 +1225,18 @@ static int plan_tree(const sattn_params* p, int32_t n_chunks, int32_t chunk_len,
 
 struct DecPlan {
   int nQT, npos, n_chunks;
-  Region status, tab, prefix, sep_pos, sep_count, ranges, part, tk_cz, tk_cj, tk_idx, tk_z, tk_part;
+  Region status, ticket, prefix, sep_pos, sep_count, ranges, part, tk_cz, tk_cj, tk_idx, tk_z, tk_part;
   int tk_nchunks = 0;
   size_t total;
 };
+
+// the decoding step's rotation: theta^(-2c/d) per pair in double (the
+// prefill table's values) and the position scale
+static void set_decode_rope(DecodeArgs& a, const sattn_params* p) {
+  a.rope = p->rope_theta != 0.0 ? 1 : 0;
+  a.rope_scale = pos_scale(p);
+  for (int c = 0; c < p->d / 2 && c < 64; ++c) a.inv_freq[c] = std::pow(p->rope_theta, -2.0 * (double)c / (double)p->d);
+}
 
 static int plan_decode(const sattn_params* p, DecPlan* out) {
   int rc = check_common(p);
@@ -1247,7 +1255,7 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   const size_t B = p->B, Hq = p->Hq, T = p->T, d = p->d;
   Alloc A;
   P.status = A.take(kStatusBytes);
-  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (d / 2) * sizeof(float2));
+  P.ticket = A.take(B * (size_t)p->Hkv * 4);
   if (p->with_separators) {
     P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
     P.sep_pos = A.take(B * T * 4);
@@ -1294,24 +1302,8 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
   if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
-  if (P.tab.bytes) {
-    ProfScope ps("rope_table", 1, st);
-    if (is_sep || (p->topk > 0 && p->L_pretrain == 0)) {
-      // separators (or uncapped top-k candidates) can sit at any earlier position
-      SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
-    } else {
-      // (top-k candidates past the cap use row i - L, the nearer ones rows
-      // in [i - L, i - w): both inside the rows below)
-      // the step reads the rows of the sinks (j, or i - L when capped), of
-      // the window keys and of the query (i - w <= j <= i, uncapped since
-      // w <= L), and row i - L: [0, n_start) and [i - max(w, L), T)
-      const int i = p->T - 1;
-      const int row_lo = std::max(0, i - std::max(p->window, p->L_pretrain));
-      SATTN_TRY(launch_rope_table_rows(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p),
-                                       std::min(p->n_start, p->T), row_lo, st));
-    }
-  }
+  // the status word and the chunk tickets start at zero
+  SATTN_TRY(cudaMemsetAsync(ws, 0, P.ticket.off + P.ticket.bytes, st));
   if (is_sep) {
     FwdPlan F;
     F.prefix = P.prefix;
@@ -1341,10 +1333,11 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   a.v_sb = p->v_stride[0];
   a.v_sh = p->v_stride[1];
   a.v_st = p->v_stride[2];
-  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  set_decode_rope(a, p);
   a.sep_words = is_sep ? at<uint2>(ws, P.prefix) : nullptr;
   a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
   a.part = at<float>(ws, P.part);
+  a.ticket = at<int32_t>(ws, P.ticket);
   a.n_chunks = P.n_chunks;
   if (p->topk > 0) {
     a.topk = p->topk;
@@ -1360,7 +1353,7 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   a.o_sh = p->o_stride[1];
   a.lse = lse;
   const int n_topk_kernels = p->topk > 0 ? (p->T - 1 - p->window - p->n_start > 0 ? 2 : 1) : 0;
-  ProfScope ps("decode", 2 + n_topk_kernels, st);
+  ProfScope ps("decode", 1 + n_topk_kernels, st);
   return cuda_rc(launch_decode(a, st));
 }
 
@@ -1921,7 +1914,7 @@ static int plan_stream_decode(const sattn_stream_config* cfg, const sattn_params
   P.n_chunks = decode_chunks(cfg->c);
   Alloc A;
   P.status = A.take(kStatusBytes);
-  if (p->rope_theta != 0.0) P.tab = A.take((size_t)P.npos * (p->d / 2) * sizeof(float2));
+  P.ticket = A.take((size_t)p->B * p->Hkv * 4);
   P.part = A.take((size_t)p->B * p->Hq * (size_t)P.n_chunks * (p->d + 2) * 4);
   P.total = A.cur;
   *out = P;
@@ -1948,11 +1941,8 @@ int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, c
   if (!Q || !O || !lse || !aligned16(Q) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
   if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
-  if (P.tab.bytes) {
-    ProfScope ps("rope_table", 1, st);
-    SATTN_TRY(launch_rope_table(at<float2>(ws, P.tab), P.npos, p->d, p->rope_theta, pos_scale(p), st));
-  }
+  // the status word and the chunk tickets start at zero
+  SATTN_TRY(cudaMemsetAsync(ws, 0, P.ticket.off + P.ticket.bytes, st));
   void* sp = const_cast<void*>(state);
   const int64_t H = cfg->Hkv, c = cfg->c, d = cfg->d;
   DecodeArgs a{};
@@ -1976,15 +1966,16 @@ int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, c
   a.v_sb = H * c * d;
   a.v_sh = c * d;
   a.v_st = d;
-  a.tab = P.tab.bytes ? at<float2>(ws, P.tab) : nullptr;
+  set_decode_rope(a, p);
   a.seq_len = at<int32_t>(sp, L.len);
   a.part = at<float>(ws, P.part);
+  a.ticket = at<int32_t>(ws, P.ticket);
   a.n_chunks = P.n_chunks;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.o_sb = p->o_stride[0];
   a.o_sh = p->o_stride[1];
   a.lse = lse;
-  ProfScope ps("stream_decode", 2, st);
+  ProfScope ps("stream_decode", 1, st);
   return cuda_rc(launch_decode(a, st));
 }
 

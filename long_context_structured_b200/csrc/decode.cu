@@ -11,14 +11,23 @@
 //
 // Split-K over the kept keys (memory-bound: each kept K and V row is read
 // once): a CTA takes a chunk of kChunk kept keys of one (batch, kv head) for
-// all query heads of that kv head's group; each warp walks its 32 keys with
-// the head dimension spread over the lanes (a lane owns rotary pairs
-// c = PPL*lane .. PPL*lane + PPL - 1 and their partners c + d/2), first the
-// logits (several keys' K rows and rotary entries loaded before any is
-// used), then, with the chunk's per-head maximum known, the weighted V rows.
-// The chunk's (max, sum, unnormalised O) per head go to the workspace; a
-// second kernel merges the chunks.
+// all query heads of that kv head's group.  It first issues asynchronous
+// copies of all the chunk's K and V rows into shared memory (64 KB at d =
+// 128, so that every byte the CTA needs is in flight at once), then computes
+// the logits from the staged K rows (each warp walks 32 keys with the head
+// dimension spread over the lanes: a lane owns rotary pairs c = PPL*lane ..
+// PPL*lane + PPL - 1 and their partners c + d/2), then, with the chunk's
+// per-head maximum known, the weighted V rows.  The chunk's (max, sum,
+// unnormalised O) per head go to the workspace, and the last CTA of a
+// (batch, kv head) to finish merges them into O and LSE.
+//
+// The rotations are computed in the kernel, not read from a table: the
+// angle of a position in double, reduced by whole turns, then the fp32 sine
+// and cosine (the prefill's table arithmetic); along a run of consecutive
+// positions a lane steps its keys' (cos, sin) by one fixed rotation
+// (angle addition in fp32) instead.
 #include <algorithm>
+#include <cmath>
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -34,6 +43,26 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kChunk = 128;  // kept keys per CTA
+static_assert(kThreads == kChunk, "a thread looks up one slot's key position");
+constexpr int kMaxChunks = 4096;  // chunks one step may merge (keys up to 4096 * kChunk)
+
+// programmatic dependent launch: let the next kernel of the step start its
+// independent work early / wait for the previous kernel's results
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// 16-byte asynchronous copy global -> shared; `valid` false fills zeros
+// without reading the source
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 struct KeySet {
   int n_sink, win_lo, n_win, n_sep;
@@ -63,175 +92,421 @@ __device__ __forceinline__ int key_at(const DecodeArgs& a, const KeySet& s, int 
   return a.sep_pos[(size_t)b * a.T + (e - s.n_win)];
 }
 
-// grid (B * Hkv, chunks): the (batch, kv head) index varies fastest, so the
-// chunks that hold keys (the low ones) are dispatched before the empty ones.
-//
-// A key is spread over LPK lanes (8, or 16 for eight query heads per kv
-// head), each holding EPL rotary pairs (16 or 8 elements of the row), so a
-// warp works on 32 / LPK keys at once with 16-byte loads.  Two passes over
-// the CTA's chunk of kept keys: (1) logits -- the raw key rotated on the fly
-// to R(j) k_j, or for a capped key (i - j > L) to R(i - L) k_j, which gives
-// the capped logit <R(L) q, k_j> = <R(i) q, R(i - L) k_j> with the one query
-// R(i) q; the lanes' partial dot products of all heads summed by one
-// transposed butterfly over the key's lanes; logits to shared memory; (2)
-// with the chunk's per-head maximum and the weights p = 2^(z - m) taken once
-// per (key, head): O += p v.  No running rescale.
+// ---- packed fp32 pairs (one f32x2 instruction per two lanes of work) ----
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// two bf16 (one 32-bit word, low half first) as a float pair
+__device__ __forceinline__ float2 bf2f(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// EPL consecutive bf16 (16, 8 or 4 bytes) as EPL / 2 float pairs
+template <int H>
+__device__ __forceinline__ void load_pairs(const __nv_bfloat16* p, float2 (&out)[H]) {
+  if constexpr (H == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    out[0] = bf2f(u.x);
+    out[1] = bf2f(u.y);
+    out[2] = bf2f(u.z);
+    out[3] = bf2f(u.w);
+  } else if constexpr (H == 2) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    out[0] = bf2f(u.x);
+    out[1] = bf2f(u.y);
+  } else {
+    out[0] = bf2f(*reinterpret_cast<const uint32_t*>(p));
+  }
+}
+
+// (cos, sin) of rotary pair c at position p: the angle p s theta^(-2c/d) in
+// double, reduced by whole turns in double (exact to ~1e-12 for the
+// positions used), then the hardware sine and cosine of the reduced angle
+// in [-pi, pi] (absolute error about 2^-21).
+__device__ __forceinline__ float2 rope_cs(const DecodeArgs& a, int p, int c) {
+  const double ang = (double)p * a.rope_scale * a.inv_freq[c];
+  const double turns = rint(ang * (1.0 / 6.283185307179586));
+  const float r = (float)fma(-turns, 6.283185307179586, ang);
+  float s, co;
+  __sincosf(r, &s, &co);
+  return make_float2(co, s);
+}
+
+// A lane's rotation for its EPL = 2H pairs [p0, p0 + EPL): cosines C[h] and
+// sines S[h] of pairs (p0 + 2h, p0 + 2h + 1).
+template <int H>
+struct Rot {
+  float2 C[H], S[H];
+};
+
+template <int H>
+__device__ __forceinline__ Rot<H> rope_rot(const DecodeArgs& a, int p, int p0) {
+  Rot<H> t;
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    float2 u = make_float2(1.f, 0.f), v = make_float2(1.f, 0.f);
+    if (a.rope) {
+      u = rope_cs(a, p, p0 + 2 * h);
+      v = rope_cs(a, p, p0 + 2 * h + 1);
+    }
+    t.C[h] = make_float2(u.x, v.x);
+    t.S[h] = make_float2(u.y, v.y);
+  }
+  return t;
+}
+
+// (x0, x1) <- R (x0, x1) per pair: x0 c - x1 s, x1 c + x0 s
+template <int H>
+__device__ __forceinline__ void rotate(float2 (&x0)[H], float2 (&x1)[H], const Rot<H>& t) {
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    const float2 y0 = fsub2(fmul2(x0[h], t.C[h]), fmul2(x1[h], t.S[h]));
+    const float2 y1 = ffma2(x0[h], t.S[h], fmul2(x1[h], t.C[h]));
+    x0[h] = y0;
+    x1[h] = y1;
+  }
+}
+
+// t <- t composed with the rotation (sc, ss) (angle addition), nss = -ss
+template <int H>
+__device__ __forceinline__ void rot_advance(Rot<H>& t, const Rot<H>& st, const float2 (&nss)[H]) {
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    const float2 c = ffma2(t.S[h], nss[h], fmul2(t.C[h], st.C[h]));
+    const float2 s = ffma2(t.C[h], st.S[h], fmul2(t.S[h], st.C[h]));
+    t.C[h] = c;
+    t.S[h] = s;
+  }
+}
+
 // Lane layout of the logit pass.  A key is spread over LPK lanes (8, or 16
 // for eight query heads per kv head), each holding EPL rotary pairs (16 or 8
-// elements of the row), so a warp works on 32 / LPK keys at once with
-// 16-byte loads; KPW key slots per warp, UNR warp steps in flight.
+// elements of the row) as H = EPL / 2 float pairs, so a warp works on KPS =
+// 32 / LPK keys at once with 16-byte shared-memory loads; KPW key slots per
+// warp, KPL keys per lane (a lane's keys are the warp's slots kg, kg + KPS,
+// ...).  A lane accumulates the partial dot products of NB keys for all REP
+// heads (NB * REP = LPK values) before one transposed reduction over the
+// key's lanes hands each lane one finished logit.
 template <int D, int REP>
 struct Tiling {
   static constexpr int half = D / 2;
   static constexpr int LPK = (REP >= 8) ? 16 : 8;       // lanes per key
   static constexpr int KPS = 32 / LPK;                  // keys per warp step
   static constexpr int EPL = half / LPK;                // rotary pairs per lane
+  static constexpr int H = EPL / 2;                     // float pairs per half row
   static constexpr int KPW = kChunk / (kThreads / 32);  // keys per warp: 32
-  static constexpr int UNR = (REP >= 4) ? 1 : 2;        // warp steps whose loads are in flight together
-  static_assert(REP <= LPK && KPW % (KPS * UNR) == 0 && (EPL == 8 || EPL == 4 || EPL == 2), "decode tiling");
+  static constexpr int KPL = KPW / KPS;                 // keys per lane
+  static constexpr int NB = LPK / REP;                  // keys per reduction
+  static constexpr int UNR = (REP >= 4) ? 1 : 2;        // pass 2: key steps loaded together
+  static_assert(REP <= LPK && KPL % NB == 0 && KPW % (KPS * UNR) == 0 && (EPL == 8 || EPL == 4 || EPL == 2),
+                "decode tiling");
 };
 
-// EPL consecutive bf16 as floats (16, 8 or 4 bytes)
-template <int EPL>
-__device__ __forceinline__ void load_e(const __nv_bfloat16* p, float* out) {
-  if constexpr (EPL == 8) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      const float2 f = __bfloat1622float2(h[y]);
-      out[2 * y] = f.x;
-      out[2 * y + 1] = f.y;
-    }
-  } else if constexpr (EPL == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int y = 0; y < 2; ++y) {
-      const float2 f = __bfloat1622float2(h[y]);
-      out[2 * y] = f.x;
-      out[2 * y + 1] = f.y;
-    }
-  } else {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-    out[0] = f.x;
-    out[1] = f.y;
-  }
-}
-
-// This lane's pairs [p0, p0 + EPL) of the query of each head of kv group g,
-// rotated to i, in fp32.
+// This lane's raw query pairs of each head of kv group g: first-half
+// elements p0 .. p0 + EPL - 1 in q0, their partners in q1.
 template <int D, int REP>
-__device__ __forceinline__ void rotated_query(const DecodeArgs& a, int b, int g, int i, int p0,
-                                              float (&q0)[REP][Tiling<D, REP>::EPL],
-                                              float (&q1)[REP][Tiling<D, REP>::EPL]) {
-  constexpr int half = D / 2, EPL = Tiling<D, REP>::EPL;
+__device__ __forceinline__ void load_query(const DecodeArgs& a, int b, int g, int p0,
+                                           float2 (&q0)[REP][Tiling<D, REP>::H],
+                                           float2 (&q1)[REP][Tiling<D, REP>::H]) {
+  constexpr int half = D / 2, H = Tiling<D, REP>::H;
 #pragma unroll
   for (int r = 0; r < REP; ++r) {
     const __nv_bfloat16* qp = a.Q + (size_t)b * a.q_sb + (size_t)(g * REP + r) * a.q_sh;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const float x0 = __bfloat162float(qp[p0 + e]), x1 = __bfloat162float(qp[p0 + e + half]);
-      const float2 t = a.tab ? a.tab[(size_t)i * half + p0 + e] : make_float2(1.f, 0.f);
-      q0[r][e] = x0 * t.x - x1 * t.y;
-      q1[r][e] = x1 * t.x + x0 * t.y;
-    }
+    load_pairs<H>(qp + p0, q0[r]);
+    load_pairs<H>(qp + p0 + half, q1[r]);
   }
 }
 
-// The logit pass over one warp's KPW key slots [w_lo, w_lo + KPW): the raw
-// key rotated on the fly to R(j) k_j, or for a capped key (i - j > L) to
-// R(i - L) k_j, which gives the capped logit <R(L) q, k_j> = <R(i) q,
-// R(i - L) k_j> with the one query R(i) q; the lanes' partial dot products
-// of all heads summed by one transposed butterfly over the key's lanes.
-// key_of(slot) gives the slot's key position (-1: none); emit(r, slot, j,
-// dot) receives head r's unscaled logit on one lane per (key, head).
+// Stage the CTA's kChunk rows of one kv head's cache into dst[slot * D ..]:
+// row `slot` is position key(slot), or zeros when key(slot) < 0.  16-byte
+// pieces; a thread keeps one piece column, consecutive threads take
+// consecutive pieces of a row.
+template <int D, class Key>
+__device__ __forceinline__ void stage_rows(__nv_bfloat16* dst, const __nv_bfloat16* base, int64_t st, Key key) {
+  constexpr int PR = D / 8;            // pieces per row
+  constexpr int RPP = kThreads / PR;   // rows per pass
+  const int c = (int)threadIdx.x % PR;
+#pragma unroll
+  for (int slot = (int)threadIdx.x / PR; slot < kChunk; slot += RPP) {
+    const int j = key(slot);
+    cp_async16(dst + slot * D + c * 8, base + (int64_t)(j < 0 ? 0 : j) * st + c * 8, j >= 0);
+  }
+}
+
+// How the logit pass pairs a staged raw key k_j with the query q (position i):
+//   kRotNone: as they are (no rotation; or every key of the warp lies past
+//             the cap and the query is rotated to L: <R(L) q, k_j>);
+//   kRotRun:  the warp's slots hold consecutive positions run_j0, run_j0 + 1,
+//             ...: <R(i) q, R(j) k_j> = <R(i - j) q, k_j>.  With one or two
+//             query heads per kv head the lane's rotated queries are
+//             stepped by R(-KPS) from key to key; with more, the key's
+//             rotation R(j) is stepped by R(KPS) and applied to the key;
+//   kRotEach: each key's rotation R(j) computed from its position.
+// A key past the cap (i - j > L) takes <R(L) q, k_j> in every mode.
+enum { kRotNone = 0, kRotRun = 1, kRotEach = 2 };
+
+// The logit pass over one warp's KPW staged key slots [w_lo, w_lo + KPW)
+// (sK: the chunk's K rows, raw) against the lane's raw query pairs q0 / q1:
+// per lane NB keys' partial dot products for every head, then one
+// transposed butterfly over the key's lanes, after which lane sub holds the
+// logit of key sub / REP of the batch for head sub % REP.  key_of(slot)
+// gives the slot's key position (-1: none); emit(r, slot, j, dot) receives
+// head r's unscaled logit, once per (key, head).  mode kRotNone with
+// none_pos >= 0 rotates the query to none_pos first.
 template <int D, int REP, class KeyOf, class Emit>
-__device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __nv_bfloat16* kb, int w_lo,
-                                            int lane, const float (&q0)[REP][Tiling<D, REP>::EPL],
-                                            const float (&q1)[REP][Tiling<D, REP>::EPL], KeyOf key_of,
+__device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __nv_bfloat16* sK, int w_lo, int mode,
+                                            int run_j0, int none_pos, int lane,
+                                            const float2 (&qr0)[REP][Tiling<D, REP>::H],
+                                            const float2 (&qr1)[REP][Tiling<D, REP>::H], KeyOf key_of,
                                             Emit emit) {
   using TL = Tiling<D, REP>;
-  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, KPW = TL::KPW, UNR = TL::UNR;
+  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, H = TL::H, KPL = TL::KPL, NB = TL::NB;
+  constexpr bool kStepQuery = REP <= 2;  // run mode: step the query rotation, not the key's
   const int sub = lane % LPK, kg = lane / LPK;
   const int p0 = sub * EPL;
-  for (int u0 = 0; u0 < KPW; u0 += KPS * UNR) {
-    int jj[UNR];
-    float k0[UNR][EPL], k1[UNR][EPL];
-    float2 cs[UNR][EPL];
+  const bool need_cap = mode != kRotNone && a.L > 0 && i > a.L && (mode == kRotEach || run_j0 < i - a.L);
+  // q: the query the keys are dotted with (rotated per mode); qc: rotated to L
+  float2 q0[REP][H], q1[REP][H], qc0[REP][H], qc1[REP][H];
+  auto rotated = [&](int pos, float2 (&y0)[REP][H], float2 (&y1)[REP][H]) {
+    const Rot<H> t = rope_rot<H>(a, pos, p0);
 #pragma unroll
-    for (int x = 0; x < UNR; ++x) {
-      jj[x] = key_of(w_lo + u0 + x * KPS + kg);
-      const int j = jj[x] < 0 ? 0 : jj[x];
-      const int rpos = (a.L > 0 && i - j > a.L) ? i - a.L : j;  // capped keys: R(i - L) k_j
-      load_e<EPL>(kb + (size_t)j * a.k_st + p0, k0[x]);
-      load_e<EPL>(kb + (size_t)j * a.k_st + p0 + half, k1[x]);
-      if (a.tab) {
-        const float4* tp = reinterpret_cast<const float4*>(a.tab + (size_t)rpos * half + p0);
+    for (int r = 0; r < REP; ++r) {
 #pragma unroll
-        for (int e = 0; e < EPL; e += 2) {
-          const float4 t = tp[e / 2];
-          cs[x][e] = make_float2(t.x, t.y);
-          cs[x][e + 1] = make_float2(t.z, t.w);
+      for (int h = 0; h < H; ++h) {
+        y0[r][h] = qr0[r][h];
+        y1[r][h] = qr1[r][h];
+      }
+      rotate<H>(y0[r], y1[r], t);
+    }
+  };
+  const bool step_q = mode == kRotRun && kStepQuery;
+  if (mode == kRotNone) {
+    if (none_pos >= 0) rotated(none_pos, q0, q1);
+    else {
+#pragma unroll
+      for (int r = 0; r < REP; ++r)
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          q0[r][h] = qr0[r][h];
+          q1[r][h] = qr1[r][h];
         }
+    }
+  } else if (step_q) {
+    rotated(i - (run_j0 + kg), q0, q1);  // R(i - j) q for the lane's first key
+    if (need_cap) rotated(a.L, qc0, qc1);
+  } else {
+    rotated(i, q0, q1);
+  }
+  // run stepping: (sc, ss) the rotation by KPS positions, nss = -ss
+  Rot<H> st, cur, cap;
+  float2 nss[H];
+  if (mode == kRotRun) {
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const float2 u = a.step_cs[p0 + 2 * h], v = a.step_cs[p0 + 2 * h + 1];
+      st.C[h] = make_float2(u.x, v.x);
+      st.S[h] = make_float2(u.y, v.y);
+      nss[h] = make_float2(-u.y, -v.y);
+    }
+    if (!kStepQuery) cur = rope_rot<H>(a, run_j0 + kg, p0);
+  }
+  if (need_cap && !step_q) cap = rope_rot<H>(a, i - a.L, p0);
+#pragma unroll 1
+  for (int m0 = 0; m0 < KPL; m0 += NB) {
+    float2 acc[LPK];  // [NB keys][REP heads], pairwise partial sums
+#pragma unroll
+    for (int x = 0; x < LPK; ++x) acc[x] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int kb = 0; kb < NB; ++kb) {
+      const int el = w_lo + kg + KPS * (m0 + kb);
+      float2 k0[H], k1[H];
+      load_pairs<H>(sK + el * D + p0, k0);
+      load_pairs<H>(sK + el * D + p0 + half, k1);
+      const int j = (mode == kRotRun) ? run_j0 + (el - w_lo) : key_of(el);
+      const bool capped = need_cap && i - j > a.L;
+      if (step_q) {
+        // keys past the cap pair with R(L) q, the others with R(i - j) q
+#pragma unroll
+        for (int r = 0; r < REP; ++r)
+#pragma unroll
+          for (int h = 0; h < H; ++h) {
+            const float2 x0 = capped ? qc0[r][h] : q0[r][h], x1 = capped ? qc1[r][h] : q1[r][h];
+            acc[kb * REP + r] = ffma2(x0, k0[h], ffma2(x1, k1[h], acc[kb * REP + r]));
+          }
+        // R(i - j - KPS) q = R(-KPS) R(i - j) q: rotate by (sc, -ss)
+#pragma unroll
+        for (int r = 0; r < REP; ++r)
+#pragma unroll
+          for (int h = 0; h < H; ++h) {
+            const float2 y0 = ffma2(q1[r][h], st.S[h], fmul2(q0[r][h], st.C[h]));
+            const float2 y1 = ffma2(q0[r][h], nss[h], fmul2(q1[r][h], st.C[h]));
+            q0[r][h] = y0;
+            q1[r][h] = y1;
+          }
       } else {
+        if (mode != kRotNone) {
+          if (capped) {
+            rotate<H>(k0, k1, cap);
+          } else if (mode == kRotRun) {
+            rotate<H>(k0, k1, cur);
+          } else {
+            rotate<H>(k0, k1, rope_rot<H>(a, j < 0 ? 0 : j, p0));
+          }
+          if (mode == kRotRun) rot_advance<H>(cur, st, nss);
+        }
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) cs[x][e] = make_float2(1.f, 0.f);
+        for (int r = 0; r < REP; ++r)
+#pragma unroll
+          for (int h = 0; h < H; ++h) acc[kb * REP + r] = ffma2(q0[r][h], k0[h], ffma2(q1[r][h], k1[h], acc[kb * REP + r]));
       }
     }
+    float v[LPK];
 #pragma unroll
-    for (int x = 0; x < UNR; ++x) {
-      float v[REP];
+    for (int x = 0; x < LPK; ++x) v[x] = acc[x].x + acc[x].y;
+    group_reduce_transposed<LPK, LPK>(v, 0xffffffffu, lane);
+    const int el = w_lo + kg + KPS * (m0 + sub / REP);
+    emit(sub % REP, el, key_of(el), v[0]);
+  }
+}
+
+// The last CTA of a (batch, kv head) to finish merges the nc0 chunk
+// partials of each head of the group, and the top-k keys' partial when there
+// is one, into O and LSE: a running maximum with rescaling over the chunks
+// in chunk order (eight chunks' loads in flight at a time).  The partials
+// were written by other CTAs, so they are read from L2.
+template <int D, int REP>
+__device__ __forceinline__ void merge_chunks(const DecodeArgs& a, int b, int g, int nc0) {
+  constexpr int U = 8;
+  const int nc = nc0 + (a.tk_part ? 1 : 0);
+  for (int x = threadIdx.x; x < REP * D; x += kThreads) {
+    const int r = x / D, c = x % D;
+    const int h = g * REP + r;
+    const size_t bh = (size_t)b * a.Hq + h;
+    const float* part0 = a.part + bh * a.n_chunks * (D + 2);
+    const float* tkp = a.tk_part ? a.tk_part + bh * (D + 2) : nullptr;
+    float m = -CUDART_INF_F, l = 0.f, o = 0.f;
+    for (int y0 = 0; y0 < nc; y0 += U) {
+      float pm[U], pl[U], po[U];
 #pragma unroll
-      for (int r = 0; r < REP; ++r) v[r] = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        const float kr0 = k0[x][e] * cs[x][e].x - k1[x][e] * cs[x][e].y;
-        const float kr1 = k1[x][e] * cs[x][e].x + k0[x][e] * cs[x][e].y;
-#pragma unroll
-        for (int r = 0; r < REP; ++r) v[r] = fmaf(q0[r][e], kr0, fmaf(q1[r][e], kr1, v[r]));
+      for (int u = 0; u < U; ++u) {
+        const int y = y0 + u;
+        pm[u] = -CUDART_INF_F;
+        pl[u] = po[u] = 0.f;
+        if (y < nc) {
+          const float* src = y < nc0 ? part0 + (size_t)y * (D + 2) : tkp;
+          pm[u] = __ldcg(src);
+          pl[u] = __ldcg(src + 1);
+          po[u] = __ldcg(src + 2 + c);
+        }
       }
-      group_reduce_transposed<REP, LPK>(v, 0xffffffffu, lane);
-      // lane sub now holds head sub / (LPK / REP)
-      constexpr int DUP = LPK / REP;
-      if (sub % DUP == 0) emit(sub / DUP, w_lo + u0 + x * KPS + kg, jj[x], v[0]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (pm[u] == -CUDART_INF_F) continue;  // no key in this partial
+        if (pm[u] > m) {
+          const float s = (m == -CUDART_INF_F) ? 0.f : ex2_approx(m - pm[u]);
+          l *= s;
+          o *= s;
+          m = pm[u];
+        }
+        const float f = ex2_approx(pm[u] - m);
+        l = fmaf(pl[u], f, l);
+        o = fmaf(po[u], f, o);
+      }
     }
+    __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
+    op[c] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+    if (c == 0) a.lse[bh] = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
   }
 }
 
 // grid (B * Hkv, chunks): the (batch, kv head) index varies fastest, so the
 // chunks that hold keys (the low ones) are dispatched before the empty ones.
-// Two passes over the CTA's chunk of kept keys: (1) logits (logits_pass) to
-// shared memory; (2) with the chunk's per-head maximum and the weights
-// p = 2^(z - m) taken once per (key, head): O += p v.  No running rescale.
+// The chunk's K and V rows are copied to shared memory first (K and V as two
+// copy groups); then (1) logits (logits_pass) to shared memory, (2) with the
+// chunk's per-head maximum and the weights p = 2^(z - m) taken once per
+// (key, head): O += p v.  No running rescale.  The chunk's partials go to
+// the workspace; a per-(batch, kv head) ticket elects the last CTA, which
+// merges them (merge_chunks).
 template <int D, int REP>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
   using TL = Tiling<D, REP>;
-  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, KPW = TL::KPW, UNR = TL::UNR;
-  __shared__ float s_p[REP][kChunk];            // logits, then weights
+  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, H = TL::H, KPW = TL::KPW, UNR = TL::UNR;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dsm);  // [kChunk][D]
+  __nv_bfloat16* sV = sK + kChunk * D;                         // [kChunk][D]
+  float* red_o = reinterpret_cast<float*>(dsm);                // [warps][REP][D], over sK after pass 1
+  static_assert((kThreads / 32) * REP * D * 4 <= kChunk * D * 2, "the O reduction fits over the K rows");
+  __shared__ float s_p[REP][kChunk];  // logits, then weights
+  __shared__ int s_j[kChunk];         // slot -> key position (-1: none)
   __shared__ float s_m[REP], s_l[REP];
-  __shared__ float red_o[kThreads / 32][REP][D];
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPK, kg = lane / LPK;
   const int bg = blockIdx.x;
   const int g = bg % a.Hkv, b = bg / a.Hkv;
+  // the key set of a cache with separators comes from the block map, the
+  // previous kernel's output; without them it is a closed form, and the K
+  // and V copies start before that kernel has finished
+  if (a.sep_words) grid_dep_wait();
   const KeySet ks = key_set(a, b);
+  const int n = ks.n();
   const int e_begin = blockIdx.y * kChunk;
-  if (e_begin >= ks.n()) return;  // this batch has fewer chunks
-  const int n_here = min(ks.n() - e_begin, kChunk);
+  if (e_begin >= n) {  // this batch has fewer chunks
+    grid_dep_wait();
+    return;
+  }
+  const int n_here = min(n - e_begin, kChunk);
   const int i = cache_len(a, b) - 1;
-  const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
-  float q0[REP][EPL], q1[REP][EPL];
-  rotated_query<D, REP>(a, b, g, i, p0, q0, q1);
+  s_j[threadIdx.x] = (int)threadIdx.x < n_here ? key_at(a, ks, b, e_begin + threadIdx.x) : -1;
+  __syncthreads();
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
   const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
+  stage_rows<D>(sK, kb, a.k_st, [&](int s) { return s_j[s]; });
+  cp_async_commit();
+  stage_rows<D>(sV, vb, a.v_st, [&](int s) { return s_j[s]; });
+  cp_async_commit();
+  grid_dep_wait();
+  const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
+  float2 q0[REP][H], q1[REP][H];
+  load_query<D, REP>(a, b, g, p0, q0, q1);
   const float sl2 = a.scale_log2;
   const int w_lo = warp * KPW;
+  // a warp whose keys all lie in the window holds consecutive positions
+  const int e_w = e_begin + w_lo, e_w_end = min(e_w + KPW, n);
+  const bool run = e_w >= ks.n_sink && e_w_end <= ks.n_sink + ks.n_win;
+  cp_async_wait<1>();
+  __syncthreads();
 
   // ---- pass 1: logits ----
+  const int mode = !a.rope ? kRotNone : (run ? kRotRun : kRotEach);
   logits_pass<D, REP>(
-      a, i, kb, w_lo, lane, q0, q1,
-      [&](int el) { return el < n_here ? key_at(a, ks, b, e_begin + el) : -1; },
+      a, i, sK, w_lo, mode, run ? ks.win_lo + (e_w - ks.n_sink) : -1, -1, lane, q0, q1,
+      [&](int el) { return s_j[el]; },
       [&](int r, int el, int j, float dot) {
         float z = dot * sl2;
         if (a.alibi && j >= 0) {  // -m_h * min(i - j, L), in log2 units of the scaled logit
@@ -260,32 +535,33 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       s_l[r] = sum;
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
-  // ---- pass 2: O += p v ----
-  float o0[REP][EPL], o1[REP][EPL];
+  // ---- pass 2: O += p v (rows past the chunk's end are zeros with p = 0) ----
+  float2 o0[REP][H], o1[REP][H];
 #pragma unroll
   for (int r = 0; r < REP; ++r)
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) o0[r][e] = o1[r][e] = 0.f;
+    for (int h = 0; h < H; ++h) o0[r][h] = o1[r][h] = make_float2(0.f, 0.f);
   for (int u0 = 0; u0 < KPW; u0 += KPS * UNR) {
-    float v0[UNR][EPL], v1[UNR][EPL];
+    float2 v0[UNR][H], v1[UNR][H];
     int els[UNR];
 #pragma unroll
     for (int x = 0; x < UNR; ++x) {
       els[x] = w_lo + u0 + x * KPS + kg;
-      const int j = (els[x] < n_here) ? key_at(a, ks, b, e_begin + els[x]) : 0;
-      load_e<EPL>(vb + (size_t)j * a.v_st + p0, v0[x]);
-      load_e<EPL>(vb + (size_t)j * a.v_st + p0 + half, v1[x]);
+      load_pairs<H>(sV + els[x] * D + p0, v0[x]);
+      load_pairs<H>(sV + els[x] * D + p0 + half, v1[x]);
     }
 #pragma unroll
     for (int x = 0; x < UNR; ++x) {
 #pragma unroll
       for (int r = 0; r < REP; ++r) {
-        const float p = s_p[r][els[x]];  // 0 for keys past the chunk's end
+        const float p = s_p[r][els[x]];
+        const float2 pp = make_float2(p, p);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          o0[r][e] = fmaf(p, v0[x][e], o0[r][e]);
-          o1[r][e] = fmaf(p, v1[x][e], o1[r][e]);
+        for (int h = 0; h < H; ++h) {
+          o0[r][h] = ffma2(pp, v0[x][h], o0[r][h]);
+          o1[r][h] = ffma2(pp, v1[x][h], o1[r][h]);
         }
       }
     }
@@ -296,24 +572,26 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 #pragma unroll
     for (int r = 0; r < REP; ++r)
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        o0[r][e] += __shfl_xor_sync(0xffffffffu, o0[r][e], o);
-        o1[r][e] += __shfl_xor_sync(0xffffffffu, o1[r][e], o);
+      for (int h = 0; h < H; ++h) {
+        o0[r][h].x += __shfl_xor_sync(0xffffffffu, o0[r][h].x, o);
+        o0[r][h].y += __shfl_xor_sync(0xffffffffu, o0[r][h].y, o);
+        o1[r][h].x += __shfl_xor_sync(0xffffffffu, o1[r][h].x, o);
+        o1[r][h].y += __shfl_xor_sync(0xffffffffu, o1[r][h].y, o);
       }
   if (kg == 0) {
 #pragma unroll
     for (int r = 0; r < REP; ++r)
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        red_o[warp][r][p0 + e] = o0[r][e];
-        red_o[warp][r][p0 + e + half] = o1[r][e];
+      for (int h = 0; h < H; ++h) {
+        *reinterpret_cast<float2*>(&red_o[(warp * REP + r) * D + p0 + 2 * h]) = o0[r][h];
+        *reinterpret_cast<float2*>(&red_o[(warp * REP + r) * D + p0 + 2 * h + half]) = o1[r][h];
       }
   }
   __syncthreads();
   for (int x = threadIdx.x; x < REP * D; x += kThreads) {
     const int r = x / D, c = x % D;
     float O = 0.f;
-    for (int w = 0; w < kThreads / 32; ++w) O += red_o[w][r][c];
+    for (int w = 0; w < kThreads / 32; ++w) O += red_o[(w * REP + r) * D + c];
     const int h = g * REP + r;
     float* part = a.part + (((size_t)b * a.Hq + h) * a.n_chunks + blockIdx.y) * (D + 2);
     part[2 + c] = O;
@@ -322,6 +600,15 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       part[1] = s_l[r];
     }
   }
+  // count this chunk in; the group's last chunk merges
+  const int nc0 = (n + kChunk - 1) / kChunk;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(a.ticket + bg, 1) == nc0 - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  merge_chunks<D, REP>(a, b, g, nc0);
 }
 
 // ---------------------------------------------------------------------------
@@ -332,30 +619,43 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 // asks for here; the K rows are read once per kv group.
 // ---------------------------------------------------------------------------
 
-// grid (B * Hkv, candidate chunks of kChunk positions): every candidate's
-// logit for every query head of the group (the logit pass over consecutive
-// positions), then per head the chunk's k best (separators excluded by
-// their flag bit) into tk_cz / tk_cj: the top k of the whole row is the top
-// k of the chunks' top k, so the selection merges k entries per chunk
-// rather than every candidate.
+// grid (B * Hkv, candidate chunks of kChunk positions): the chunk's K rows
+// staged in shared memory, every candidate's logit for every query head of
+// the group (the logit pass over consecutive positions), then per head the
+// chunk's k best (separators excluded by their flag bit) into tk_cz / tk_cj:
+// the top k of the whole row is the top k of the chunks' top k, so the
+// selection merges k entries per chunk rather than every candidate.
 template <int D, int REP>
 __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs a) {
   using TL = Tiling<D, REP>;
-  constexpr int EPL = TL::EPL, LPK = TL::LPK, KPW = TL::KPW;
+  constexpr int EPL = TL::EPL, H = TL::H, LPK = TL::LPK, KPW = TL::KPW;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dsm);  // [kChunk][D]
   __shared__ float s_z[REP][kChunk];
+  grid_dep_launch();  // the selection kernel may be scheduled now; it waits for this grid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % a.Hkv, b = blockIdx.x / a.Hkv;
   const int i = a.T - 1;
   const int jend = i - a.window;  // candidates j < i - w
   const int j0 = a.n_start + blockIdx.y * kChunk;
   if (j0 >= jend) return;
-  const int p0 = (lane % LPK) * EPL;
-  float q0[REP][EPL], q1[REP][EPL];
-  rotated_query<D, REP>(a, b, g, i, p0, q0, q1);
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
+  stage_rows<D>(sK, kb, a.k_st, [&](int s) { return j0 + s < jend ? j0 + s : -1; });
+  cp_async_commit();
+  // a warp whose candidates all lie past the cap scores the raw keys with
+  // the query rotated to L; the others rotate their keys
+  const int jw = j0 + warp * KPW;
+  const bool all_capped = a.rope && a.L > 0 && i - (jw + KPW - 1) > a.L;
+  const int mode = !a.rope || all_capped ? kRotNone : kRotRun;
+  const int p0 = (lane % LPK) * EPL;
+  float2 q0[REP][H], q1[REP][H];
+  load_query<D, REP>(a, b, g, p0, q0, q1);
   const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
+  cp_async_wait<0>();
+  __syncthreads();
   logits_pass<D, REP>(
-      a, i, kb, warp * KPW, lane, q0, q1, [&](int el) { return j0 + el < jend ? j0 + el : -1; },
+      a, i, sK, warp * KPW, mode, jw, all_capped ? a.L : -1, lane, q0, q1,
+      [&](int el) { return j0 + el < jend ? j0 + el : -1; },
       [&](int r, int el, int j, float dot) {
         const bool sep = j >= 0 && words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u);
         s_z[r][el] = (j >= 0 && !sep) ? dot : -CUDART_INF_F;
@@ -407,6 +707,7 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   }
 }
 
+
 constexpr int kSelThreads = 512;
 constexpr int kSelMaxK = 16;
 
@@ -420,8 +721,10 @@ __global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeA
   __shared__ int red_j[kSelThreads / 32];
   __shared__ float s_z[kSelMaxK];
   __shared__ int s_j[kSelMaxK];
+  grid_dep_launch();  // the split-K kernel may start its K / V copies now
   const int bh = blockIdx.x;
   const int b = bh / a.Hq, h = bh % a.Hq, g = h / (a.Hq / a.Hkv);
+  grid_dep_wait();  // the chunks' picks
   const int n_c = a.tk_nchunks * a.topk;  // the chunks' picks (-1 padding)
   const float* czr = a.tk_cz + (size_t)bh * n_c;
   const int32_t* cjr = a.tk_cj + (size_t)bh * n_c;
@@ -490,75 +793,38 @@ __global__ void __launch_bounds__(kSelThreads) decode_topk_select_kernel(DecodeA
   }
 }
 
-// grid (B * Hq), 4 D threads: merge the chunks of one (batch, head).  The
-// chunk maxima and weights are read in parallel into shared memory; thread
-// group q of 4 sums chunks q, q + 4, ... of each output column (independent
-// loads), then the four groups are added in a fixed order.
-constexpr int kCombineGroups = 4;
-constexpr int kCombineMaxChunks = 4096;
-template <int D>
-__global__ void __launch_bounds__(kCombineGroups * D) decode_combine_kernel(DecodeArgs a) {
-  __shared__ float s_f[kCombineMaxChunks + 1];
-  __shared__ float s_red[kCombineGroups * D];
-  __shared__ float s_ml[2];
-  const int bh = blockIdx.x;
-  const int b = bh / a.Hq, h = bh % a.Hq;
-  const KeySet ks = key_set(a, b);
-  const int nc0 = min((ks.n() + kChunk - 1) / kChunk, kCombineMaxChunks);
-  // the chunks' partials, then the top-k keys' one
-  const int nc = nc0 + (a.tk_part ? 1 : 0);
-  const float* part0 = a.part + (size_t)bh * a.n_chunks * (D + 2);
-  auto slot = [&](int x) { return x < nc0 ? part0 + (size_t)x * (D + 2) : a.tk_part + (size_t)bh * (D + 2); };
-  const int tid = threadIdx.x;
-  float mx = -CUDART_INF_F;
-  for (int x = tid; x < nc; x += blockDim.x) {
-    s_f[x] = slot(x)[0];
-    mx = fmaxf(mx, s_f[x]);
-  }
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((tid & 31) == 0) s_red[tid >> 5] = mx;
-  __syncthreads();
-  if (tid == 0) {
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) M = fmaxf(M, s_red[w]);
-    s_ml[0] = M;
-  }
-  __syncthreads();
-  const float M = s_ml[0];
-  float lsum = 0.f;
-  for (int x = tid; x < nc; x += blockDim.x) {
-    const float f = (s_f[x] == -CUDART_INF_F) ? 0.f : ex2_approx(s_f[x] - M);
-    s_f[x] = f;
-    lsum += slot(x)[1] * f;
-  }
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  __syncthreads();  // s_red is reused
-  if ((tid & 31) == 0) s_red[tid >> 5] = lsum;
-  __syncthreads();
-  if (tid == 0) {
-    float L = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) L += s_red[w];
-    s_ml[1] = L;
-  }
-  const int q = tid / D, c = tid % D;
-  float O = 0.f;
-#pragma unroll 4
-  for (int x = q; x < nc; x += kCombineGroups) O = fmaf(slot(x)[2 + c], s_f[x], O);
-  __syncthreads();
-  s_red[q * D + c] = O;
-  __syncthreads();
-  if (q == 0) {
-    float Ot = 0.f;
-    for (int y = 0; y < kCombineGroups; ++y) Ot += s_red[y * D + c];
-    const float L = s_ml[1];
-    __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
-    op[c] = __float2bfloat16_rn(L > 0.f ? Ot / L : 0.f);
-    if (c == 0) a.lse[bh] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
-  }
+template <class Kern>
+cudaError_t launch_k(Kern kern, dim3 grid, int threads, size_t smem, bool pdl, const DecodeArgs& a,
+                     cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// dynamic shared memory above the default 48 KB
+template <class Kern>
+cudaError_t allow_smem(Kern kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 template <int D, int REP>
-cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_dr(const DecodeArgs& a0, cudaStream_t st) {
+  // the rotation by KPS positions that steps a lane from one of its keys to
+  // the next along a run, from the angle in double
+  DecodeArgs a = a0;
+  constexpr int KPS = Tiling<D, REP>::KPS;
+  for (int c = 0; c < D / 2; ++c) {
+    const double ang = KPS * a.rope_scale * a.inv_freq[c];
+    a.step_cs[c] = a.rope ? make_float2((float)std::cos(ang), (float)std::sin(ang)) : make_float2(1.f, 0.f);
+  }
   // without separators or per-sequence lengths the kept-key count is a
   // closed form: launch exactly its chunks
   int chunks = a.n_chunks;
@@ -567,25 +833,27 @@ cudaError_t launch_dr(const DecodeArgs& a, cudaStream_t st) {
     const int win_lo = std::max(ns, i - a.window);
     chunks = std::min(chunks, std::max(1, (ns + std::max(0, i - win_lo + 1) + kChunk - 1) / kChunk));
   }
+  const size_t rows_bytes = (size_t)kChunk * D * sizeof(__nv_bfloat16);
   cudaError_t e;
+  bool after_kernel = false;  // a kernel of this step precedes the next launch in the stream
   if (a.topk > 0) {
     const int ncand = a.T - 1 - a.window - a.n_start;
     if (ncand > 0) {
-      dim3 gt(a.B * a.Hkv, a.tk_nchunks);
-      decode_topk_logits_kernel<D, REP><<<gt, kThreads, 0, st>>>(a);
-      e = cudaGetLastError();
+      e = allow_smem(decode_topk_logits_kernel<D, REP>, rows_bytes);
       if (e != cudaSuccess) return e;
+      e = launch_k(decode_topk_logits_kernel<D, REP>, dim3(a.B * a.Hkv, a.tk_nchunks), kThreads, rows_bytes, false,
+                   a, st);
+      if (e != cudaSuccess) return e;
+      after_kernel = true;
     }
-    decode_topk_select_kernel<D><<<a.B * a.Hq, kSelThreads, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_k(decode_topk_select_kernel<D>, dim3(a.B * a.Hq), kSelThreads, 0, after_kernel, a, st);
     if (e != cudaSuccess) return e;
+    after_kernel = true;
   }
-  dim3 grid(a.B * a.Hkv, chunks);
-  decode_partial_kernel<D, REP><<<grid, kThreads, 0, st>>>(a);
-  e = cudaGetLastError();
+  e = allow_smem(decode_partial_kernel<D, REP>, 2 * rows_bytes);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<D><<<a.B * a.Hq, kCombineGroups * D, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_k(decode_partial_kernel<D, REP>, dim3(a.B * a.Hkv, chunks), kThreads, 2 * rows_bytes, after_kernel,
+                  a, st);
 }
 
 template <int D>
@@ -603,10 +871,11 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t st) {
 
 int decode_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 int decode_topk_chunks(int n_candidates) { return n_candidates > 0 ? (n_candidates + kChunk - 1) / kChunk : 0; }
-int decode_max_len() { return kCombineMaxChunks * kChunk; }
+int decode_max_len() { return kMaxChunks * kChunk; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
+  if (a.d / 2 > (int)(sizeof(a.inv_freq) / sizeof(a.inv_freq[0]))) return cudaErrorInvalidValue;
   if (a.d == 128) return launch_d<128>(a, st);
   if (a.d == 64) return launch_d<64>(a, st);
   return cudaErrorInvalidValue;

@@ -465,11 +465,16 @@ struct DecodeArgs {
   int64_t k_sb, k_sh, k_st;
   const __nv_bfloat16* V;
   int64_t v_sb, v_sh, v_st;
-  const float2* tab;            // rotary table or null
+  // rotation (rope != 0): pair c at position p turns by p * rope_scale * inv_freq[c]
+  int rope;
+  double rope_scale;
+  double inv_freq[64];          // theta^(-2c/d), c < d/2
+  float2 step_cs[64];           // (cos, sin) of the rotation by a fixed number of positions (kernel-set)
   const uint2* sep_words;       // separator word prefix (sep_before) or null (no separators)
   const int32_t* sep_pos;       // [B, T]
   const int32_t* seq_len;       // [B] cache length per sequence (<= T), or null: T for all
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
+  int32_t* ticket;              // [B, Hkv] finished chunks per group, zero before the launch
   int alibi;                    // ALiBi bias clipped at L (no rotation)
   int n_chunks;
   // top-k middle tokens of the query (topk > 0; seq_len must be null)
