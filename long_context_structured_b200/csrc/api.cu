@@ -1225,7 +1225,7 @@ static int plan_tree(const sattn_params* p, int32_t n_chunks, int32_t chunk_len,
 
 struct DecPlan {
   int nQT, npos, n_chunks;
-  Region status, ticket, prefix, sep_pos, sep_count, ranges, part, tk_cz, tk_cj, tk_idx, tk_z, tk_part;
+  Region status, prefix, sep_pos, sep_count, ranges, part, tk_cz, tk_cj, tk_idx, tk_z, tk_part;
   int tk_nchunks = 0;
   size_t total;
 };
@@ -1255,7 +1255,6 @@ static int plan_decode(const sattn_params* p, DecPlan* out) {
   const size_t B = p->B, Hq = p->Hq, T = p->T, d = p->d;
   Alloc A;
   P.status = A.take(kStatusBytes);
-  P.ticket = A.take(B * (size_t)p->Hkv * 4);
   if (p->with_separators) {
     P.prefix = A.take(blockmap_scratch_bytes(p->B, p->T, p->window));
     P.sep_pos = A.take(B * T * 4);
@@ -1302,8 +1301,7 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
   if (!pointers_ok_bf16(Q, K, V) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // the status word and the chunk tickets start at zero
-  SATTN_TRY(cudaMemsetAsync(ws, 0, P.ticket.off + P.ticket.bytes, st));
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
   if (is_sep) {
     FwdPlan F;
     F.prefix = P.prefix;
@@ -1337,7 +1335,7 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   a.sep_words = is_sep ? at<uint2>(ws, P.prefix) : nullptr;
   a.sep_pos = is_sep ? at<int32_t>(ws, P.sep_pos) : nullptr;
   a.part = at<float>(ws, P.part);
-  a.ticket = at<int32_t>(ws, P.ticket);
+  a.status = at<int32_t>(ws, P.status);
   a.n_chunks = P.n_chunks;
   if (p->topk > 0) {
     a.topk = p->topk;
@@ -1353,7 +1351,7 @@ int sattn_decode_topk_fwd(const sattn_params* p, const void* Q, const void* K, c
   a.o_sh = p->o_stride[1];
   a.lse = lse;
   const int n_topk_kernels = p->topk > 0 ? (p->T - 1 - p->window - p->n_start > 0 ? 2 : 1) : 0;
-  ProfScope ps("decode", 1 + n_topk_kernels, st);
+  ProfScope ps("decode", 2 + n_topk_kernels, st);
   return cuda_rc(launch_decode(a, st));
 }
 
@@ -1914,7 +1912,6 @@ static int plan_stream_decode(const sattn_stream_config* cfg, const sattn_params
   P.n_chunks = decode_chunks(cfg->c);
   Alloc A;
   P.status = A.take(kStatusBytes);
-  P.ticket = A.take((size_t)p->B * p->Hkv * 4);
   P.part = A.take((size_t)p->B * p->Hq * (size_t)P.n_chunks * (p->d + 2) * 4);
   P.total = A.cur;
   *out = P;
@@ -1941,8 +1938,7 @@ int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, c
   if (!Q || !O || !lse || !aligned16(Q) || !aligned16(O)) return SATTN_ERR_INVALID_ARG;
   if (!ws || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // the status word and the chunk tickets start at zero
-  SATTN_TRY(cudaMemsetAsync(ws, 0, P.ticket.off + P.ticket.bytes, st));
+  SATTN_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
   void* sp = const_cast<void*>(state);
   const int64_t H = cfg->Hkv, c = cfg->c, d = cfg->d;
   DecodeArgs a{};
@@ -1969,13 +1965,13 @@ int sattn_stream_decode(const sattn_stream_config* cfg, const sattn_params* p, c
   set_decode_rope(a, p);
   a.seq_len = at<int32_t>(sp, L.len);
   a.part = at<float>(ws, P.part);
-  a.ticket = at<int32_t>(ws, P.ticket);
+  a.status = at<int32_t>(ws, P.status);
   a.n_chunks = P.n_chunks;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.o_sb = p->o_stride[0];
   a.o_sh = p->o_stride[1];
   a.lse = lse;
-  ProfScope ps("stream_decode", 1, st);
+  ProfScope ps("stream_decode", 2, st);
   return cuda_rc(launch_decode(a, st));
 }
 

@@ -41,9 +41,17 @@ namespace sattn {
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kChunk = 128;  // kept keys per CTA
-static_assert(kThreads == kChunk, "a thread looks up one slot's key position");
+constexpr int kThreads = 128;  // top-k logit kernel: 4 warps
+constexpr int kChunk = 128;    // kept keys per CTA
+static_assert(kThreads >= kChunk, "a thread looks up one slot's key position");
+// split-K kernel: 8 warps (two CTAs per SM) with one or two query heads per
+// kv head, 4 warps (three CTAs per SM, by shared memory) with more, whose
+// per-lane query state needs the registers
+template <int REP>
+struct PartCfg {
+  static constexpr int NT = REP <= 2 ? 256 : 128;
+  static constexpr int MIN_BLOCKS = REP <= 2 ? 2 : 3;
+};
 constexpr int kMaxChunks = 4096;  // chunks one step may merge (keys up to 4096 * kChunk)
 
 // programmatic dependent launch: let the next kernel of the step start its
@@ -62,6 +70,59 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// one bulk copy (the copy engine) of `bytes` contiguous bytes global ->
+// shared, completing on the mbarrier's transaction count; no multicast
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// wait sites reported in the status word
+constexpr int kSiteDecodeK = 101, kSiteDecodeV = 102, kSiteTopkK = 103;
+
+// Staging of a chunk's rows: one bulk copy per tensor when the rows are
+// consecutive in memory (bars[t] completes when they land), else 16-byte
+// asynchronous copies per piece (tensor t is copy group t).
+struct StageWait {
+  bool bulk;
+  uint64_t* bars;
+  volatile int* abort_flag;
+  int32_t* status;
+  // wait for tensor t (0: first, 1: second) of a two-tensor staging, or the
+  // only tensor of a one-tensor staging (ntensors 1); true when it landed.
+  // Every thread of the block calls it; the result is uniform.
+  __device__ __forceinline__ bool wait(int t, int ntensors, int site) {
+    if (bulk) {
+      mbar_wait(bars + t, 0, abort_flag, status, site);
+    } else if (ntensors == 2 && t == 0) {
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    return *abort_flag == 0;
+  }
+  // after a failed wait: give the copies still in flight a bounded time to land
+  __device__ __forceinline__ void drain(int ntensors) {
+    if (!bulk) return;
+    for (int t = 0; t < ntensors; ++t) {
+      const uint32_t a = smem_u32(bars + t);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+};
+
+// zero 16-byte pieces [from, to) of a shared array (rows past a chunk's end
+// when the chunk was bulk-copied)
+__device__ __forceinline__ void zero_pieces(void* base, int from, int to, int nthreads) {
+  uint4* p = reinterpret_cast<uint4*>(base);
+  for (int x = from + (int)threadIdx.x; x < to; x += nthreads) p[x] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 struct KeySet {
@@ -144,16 +205,38 @@ __device__ __forceinline__ void load_pairs(const __nv_bfloat16* p, float2 (&out)
   }
 }
 
-// (cos, sin) of rotary pair c at position p: the angle p s theta^(-2c/d) in
-// double, reduced by whole turns in double (exact to ~1e-12 for the
-// positions used), then the hardware sine and cosine of the reduced angle
-// in [-pi, pi] (absolute error about 2^-21).
-__device__ __forceinline__ float2 rope_cs(const DecodeArgs& a, int p, int c) {
-  const double ang = (double)p * a.rope_scale * a.inv_freq[c];
-  const double turns = rint(ang * (1.0 / 6.283185307179586));
-  const float r = (float)fma(-turns, 6.283185307179586, ang);
+// (cos, sin) of rotary pair c at position p.  The angle in turns, p f_c
+// with f_c = s theta^(-2c/d) / (2 pi) split on the host into fp32 parts
+// hi + lo: p * hi is formed with its exact rounding residual (one fma), its
+// whole turns removed exactly, and p * lo added, which leaves the reduced
+// angle to about 1e-7 turns for positions below 2^24; then the hardware
+// sine and cosine of that angle in [-pi, pi] (absolute error about 2^-21).
+// The per-pair rotation constants, copied once per CTA from the kernel
+// parameters into shared memory (lanes index them by pair, which a
+// parameter-space load would serialise).
+struct RopeTab {
+  float hi[64], lo[64];  // turns per position, hi + lo
+  float2 st[64];         // (cos, sin) of the rotation by KPS positions
+};
+
+__device__ __forceinline__ void load_rope_tab(const DecodeArgs& a, RopeTab& t, int half, int nwarps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int x = warp; x < half; x += nwarps)  // warp-uniform index: one broadcast load per element
+    if (lane == 0) {
+      t.hi[x] = a.turn_hi[x];
+      t.lo[x] = a.turn_lo[x];
+      t.st[x] = a.step_cs[x];
+    }
+}
+
+__device__ __forceinline__ float2 rope_cs(const RopeTab& t, int p, int c) {
+  const float fp = (float)p;
+  const float hi = t.hi[c];
+  const float t1 = fp * hi;
+  const float e1 = fmaf(fp, hi, -t1);
+  const float r = (t1 - rintf(t1)) + fmaf(fp, t.lo[c], e1);
   float s, co;
-  __sincosf(r, &s, &co);
+  __sincosf(r * 6.283185307179586f, &s, &co);
   return make_float2(co, s);
 }
 
@@ -165,14 +248,14 @@ struct Rot {
 };
 
 template <int H>
-__device__ __forceinline__ Rot<H> rope_rot(const DecodeArgs& a, int p, int p0) {
+__device__ __forceinline__ Rot<H> rope_rot(const DecodeArgs& a, const RopeTab& rt, int p, int p0) {
   Rot<H> t;
 #pragma unroll
   for (int h = 0; h < H; ++h) {
     float2 u = make_float2(1.f, 0.f), v = make_float2(1.f, 0.f);
     if (a.rope) {
-      u = rope_cs(a, p, p0 + 2 * h);
-      v = rope_cs(a, p, p0 + 2 * h + 1);
+      u = rope_cs(rt, p, p0 + 2 * h);
+      v = rope_cs(rt, p, p0 + 2 * h + 1);
     }
     t.C[h] = make_float2(u.x, v.x);
     t.S[h] = make_float2(u.y, v.y);
@@ -212,16 +295,17 @@ __device__ __forceinline__ void rot_advance(Rot<H>& t, const Rot<H>& st, const f
 // ...).  A lane accumulates the partial dot products of NB keys for all REP
 // heads (NB * REP = LPK values) before one transposed reduction over the
 // key's lanes hands each lane one finished logit.
-template <int D, int REP>
+template <int D, int REP, int NW = kThreads / 32>
 struct Tiling {
   static constexpr int half = D / 2;
   static constexpr int LPK = (REP >= 8) ? 16 : 8;       // lanes per key
   static constexpr int KPS = 32 / LPK;                  // keys per warp step
   static constexpr int EPL = half / LPK;                // rotary pairs per lane
   static constexpr int H = EPL / 2;                     // float pairs per half row
-  static constexpr int KPW = kChunk / (kThreads / 32);  // keys per warp: 32
+  static constexpr int KPW = kChunk / NW;              // keys per warp
   static constexpr int KPL = KPW / KPS;                 // keys per lane
-  static constexpr int NB = LPK / REP;                  // keys per reduction
+  static constexpr int NB = (LPK / REP < KPL) ? LPK / REP : KPL;  // keys per reduction
+  static constexpr int NV = NB * REP;                   // values per reduction (<= LPK)
   static constexpr int UNR = (REP >= 4) ? 1 : 2;        // pass 2: key steps loaded together
   static_assert(REP <= LPK && KPL % NB == 0 && KPW % (KPS * UNR) == 0 && (EPL == 8 || EPL == 4 || EPL == 2),
                 "decode tiling");
@@ -246,10 +330,10 @@ __device__ __forceinline__ void load_query(const DecodeArgs& a, int b, int g, in
 // row `slot` is position key(slot), or zeros when key(slot) < 0.  16-byte
 // pieces; a thread keeps one piece column, consecutive threads take
 // consecutive pieces of a row.
-template <int D, class Key>
+template <int D, int NT, class Key>
 __device__ __forceinline__ void stage_rows(__nv_bfloat16* dst, const __nv_bfloat16* base, int64_t st, Key key) {
-  constexpr int PR = D / 8;            // pieces per row
-  constexpr int RPP = kThreads / PR;   // rows per pass
+  constexpr int PR = D / 8;       // pieces per row
+  constexpr int RPP = NT / PR;    // rows per pass
   const int c = (int)threadIdx.x % PR;
 #pragma unroll
   for (int slot = (int)threadIdx.x / PR; slot < kChunk; slot += RPP) {
@@ -278,14 +362,16 @@ enum { kRotNone = 0, kRotRun = 1, kRotEach = 2 };
 // gives the slot's key position (-1: none); emit(r, slot, j, dot) receives
 // head r's unscaled logit, once per (key, head).  mode kRotNone with
 // none_pos >= 0 rotates the query to none_pos first.
-template <int D, int REP, class KeyOf, class Emit>
-__device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __nv_bfloat16* sK, int w_lo, int mode,
+template <int D, int REP, int NW, class KeyOf, class Emit>
+__device__ __forceinline__ void logits_pass(const DecodeArgs& a, const RopeTab& rt, int i, const __nv_bfloat16* sK,
+                                            int w_lo, int mode,
                                             int run_j0, int none_pos, int lane,
                                             const float2 (&qr0)[REP][Tiling<D, REP>::H],
                                             const float2 (&qr1)[REP][Tiling<D, REP>::H], KeyOf key_of,
                                             Emit emit) {
-  using TL = Tiling<D, REP>;
-  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, H = TL::H, KPL = TL::KPL, NB = TL::NB;
+  using TL = Tiling<D, REP, NW>;
+  constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, H = TL::H, KPL = TL::KPL, NB = TL::NB,
+                NV = TL::NV;
   constexpr bool kStepQuery = REP <= 2;  // run mode: step the query rotation, not the key's
   const int sub = lane % LPK, kg = lane / LPK;
   const int p0 = sub * EPL;
@@ -293,7 +379,7 @@ __device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __
   // q: the query the keys are dotted with (rotated per mode); qc: rotated to L
   float2 q0[REP][H], q1[REP][H], qc0[REP][H], qc1[REP][H];
   auto rotated = [&](int pos, float2 (&y0)[REP][H], float2 (&y1)[REP][H]) {
-    const Rot<H> t = rope_rot<H>(a, pos, p0);
+    const Rot<H> t = rope_rot<H>(a, rt, pos, p0);
 #pragma unroll
     for (int r = 0; r < REP; ++r) {
 #pragma unroll
@@ -328,19 +414,19 @@ __device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __
   if (mode == kRotRun) {
 #pragma unroll
     for (int h = 0; h < H; ++h) {
-      const float2 u = a.step_cs[p0 + 2 * h], v = a.step_cs[p0 + 2 * h + 1];
+      const float2 u = rt.st[p0 + 2 * h], v = rt.st[p0 + 2 * h + 1];
       st.C[h] = make_float2(u.x, v.x);
       st.S[h] = make_float2(u.y, v.y);
       nss[h] = make_float2(-u.y, -v.y);
     }
-    if (!kStepQuery) cur = rope_rot<H>(a, run_j0 + kg, p0);
+    if (!kStepQuery) cur = rope_rot<H>(a, rt, run_j0 + kg, p0);
   }
-  if (need_cap && !step_q) cap = rope_rot<H>(a, i - a.L, p0);
+  if (need_cap && !step_q) cap = rope_rot<H>(a, rt, i - a.L, p0);
 #pragma unroll 1
   for (int m0 = 0; m0 < KPL; m0 += NB) {
-    float2 acc[LPK];  // [NB keys][REP heads], pairwise partial sums
+    float2 acc[NV];  // [NB keys][REP heads], pairwise partial sums
 #pragma unroll
-    for (int x = 0; x < LPK; ++x) acc[x] = make_float2(0.f, 0.f);
+    for (int x = 0; x < NV; ++x) acc[x] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int kb = 0; kb < NB; ++kb) {
       const int el = w_lo + kg + KPS * (m0 + kb);
@@ -375,7 +461,7 @@ __device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __
           } else if (mode == kRotRun) {
             rotate<H>(k0, k1, cur);
           } else {
-            rotate<H>(k0, k1, rope_rot<H>(a, j < 0 ? 0 : j, p0));
+            rotate<H>(k0, k1, rope_rot<H>(a, rt, j < 0 ? 0 : j, p0));
           }
           if (mode == kRotRun) rot_advance<H>(cur, st, nss);
         }
@@ -385,62 +471,15 @@ __device__ __forceinline__ void logits_pass(const DecodeArgs& a, int i, const __
           for (int h = 0; h < H; ++h) acc[kb * REP + r] = ffma2(q0[r][h], k0[h], ffma2(q1[r][h], k1[h], acc[kb * REP + r]));
       }
     }
-    float v[LPK];
+    float v[NV];
 #pragma unroll
-    for (int x = 0; x < LPK; ++x) v[x] = acc[x].x + acc[x].y;
-    group_reduce_transposed<LPK, LPK>(v, 0xffffffffu, lane);
-    const int el = w_lo + kg + KPS * (m0 + sub / REP);
-    emit(sub % REP, el, key_of(el), v[0]);
-  }
-}
-
-// The last CTA of a (batch, kv head) to finish merges the nc0 chunk
-// partials of each head of the group, and the top-k keys' partial when there
-// is one, into O and LSE: a running maximum with rescaling over the chunks
-// in chunk order (eight chunks' loads in flight at a time).  The partials
-// were written by other CTAs, so they are read from L2.
-template <int D, int REP>
-__device__ __forceinline__ void merge_chunks(const DecodeArgs& a, int b, int g, int nc0) {
-  constexpr int U = 8;
-  const int nc = nc0 + (a.tk_part ? 1 : 0);
-  for (int x = threadIdx.x; x < REP * D; x += kThreads) {
-    const int r = x / D, c = x % D;
-    const int h = g * REP + r;
-    const size_t bh = (size_t)b * a.Hq + h;
-    const float* part0 = a.part + bh * a.n_chunks * (D + 2);
-    const float* tkp = a.tk_part ? a.tk_part + bh * (D + 2) : nullptr;
-    float m = -CUDART_INF_F, l = 0.f, o = 0.f;
-    for (int y0 = 0; y0 < nc; y0 += U) {
-      float pm[U], pl[U], po[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int y = y0 + u;
-        pm[u] = -CUDART_INF_F;
-        pl[u] = po[u] = 0.f;
-        if (y < nc) {
-          const float* src = y < nc0 ? part0 + (size_t)y * (D + 2) : tkp;
-          pm[u] = __ldcg(src);
-          pl[u] = __ldcg(src + 1);
-          po[u] = __ldcg(src + 2 + c);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (pm[u] == -CUDART_INF_F) continue;  // no key in this partial
-        if (pm[u] > m) {
-          const float s = (m == -CUDART_INF_F) ? 0.f : ex2_approx(m - pm[u]);
-          l *= s;
-          o *= s;
-          m = pm[u];
-        }
-        const float f = ex2_approx(pm[u] - m);
-        l = fmaf(pl[u], f, l);
-        o = fmaf(po[u], f, o);
-      }
-    }
-    __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
-    op[c] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
-    if (c == 0) a.lse[bh] = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+    for (int x = 0; x < NV; ++x) v[x] = acc[x].x + acc[x].y;
+    group_reduce_transposed<NV, LPK>(v, 0xffffffffu, lane);
+    // value sub / DUP (DUP lanes hold each)
+    constexpr int DUP = LPK / NV;
+    const int vi = sub / DUP;
+    const int el = w_lo + kg + KPS * (m0 + vi / REP);
+    if (sub % DUP == 0) emit(vi % REP, el, key_of(el), v[0]);
   }
 }
 
@@ -450,25 +489,29 @@ __device__ __forceinline__ void merge_chunks(const DecodeArgs& a, int b, int g, 
 // copy groups); then (1) logits (logits_pass) to shared memory, (2) with the
 // chunk's per-head maximum and the weights p = 2^(z - m) taken once per
 // (key, head): O += p v.  No running rescale.  The chunk's partials go to
-// the workspace; a per-(batch, kv head) ticket elects the last CTA, which
-// merges them (merge_chunks).
+// the workspace for the merge kernel.
 template <int D, int REP>
-__global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
-  using TL = Tiling<D, REP>;
+__global__ void __launch_bounds__(PartCfg<REP>::NT, PartCfg<REP>::MIN_BLOCKS) decode_partial_kernel(DecodeArgs a) {
+  constexpr int kPartThreads = PartCfg<REP>::NT;
+  constexpr int NW = kPartThreads / 32;
+  using TL = Tiling<D, REP, NW>;
   constexpr int half = D / 2, LPK = TL::LPK, KPS = TL::KPS, EPL = TL::EPL, H = TL::H, KPW = TL::KPW, UNR = TL::UNR;
   extern __shared__ __align__(16) unsigned char dsm[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dsm);  // [kChunk][D]
   __nv_bfloat16* sV = sK + kChunk * D;                         // [kChunk][D]
   float* red_o = reinterpret_cast<float*>(dsm);                // [warps][REP][D], over sK after pass 1
-  static_assert((kThreads / 32) * REP * D * 4 <= kChunk * D * 2, "the O reduction fits over the K rows");
+  static_assert(NW * REP * D * 4 <= kChunk * D * 2, "the O reduction fits over the K rows");
   __shared__ float s_p[REP][kChunk];  // logits, then weights
   __shared__ int s_j[kChunk];         // slot -> key position (-1: none)
   __shared__ float s_m[REP], s_l[REP];
-  __shared__ int s_last;
+  __shared__ RopeTab s_rt;
+  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ int s_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPK, kg = lane / LPK;
   const int bg = blockIdx.x;
   const int g = bg % a.Hkv, b = bg / a.Hkv;
+  grid_dep_launch();  // the merge kernel may be scheduled now; it waits for this grid
   // the key set of a cache with separators comes from the block map, the
   // previous kernel's output; without them it is a closed form, and the K
   // and V copies start before that kernel has finished
@@ -482,14 +525,40 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
   }
   const int n_here = min(n - e_begin, kChunk);
   const int i = cache_len(a, b) - 1;
-  s_j[threadIdx.x] = (int)threadIdx.x < n_here ? key_at(a, ks, b, e_begin + threadIdx.x) : -1;
+  // a chunk inside the window holds consecutive positions: with contiguous
+  // rows its K and V are one bulk copy each
+  const bool bulk = e_begin >= ks.n_sink && e_begin + n_here <= ks.n_sink + ks.n_win && a.k_st == D && a.v_st == D;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    if (bulk) {
+      mbar_init(&s_bar[0], 1);
+      mbar_init(&s_bar[1], 1);
+      fence_mbar_init();
+    }
+  }
+  if (threadIdx.x < kChunk) s_j[threadIdx.x] = (int)threadIdx.x < n_here ? key_at(a, ks, b, e_begin + threadIdx.x) : -1;
+  if (a.rope) load_rope_tab(a, s_rt, half, NW);
   __syncthreads();
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
   const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
-  stage_rows<D>(sK, kb, a.k_st, [&](int s) { return s_j[s]; });
-  cp_async_commit();
-  stage_rows<D>(sV, vb, a.v_st, [&](int s) { return s_j[s]; });
-  cp_async_commit();
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      const size_t j0 = (size_t)(ks.win_lo + (e_begin - ks.n_sink));
+      const uint32_t bytes = (uint32_t)n_here * D * 2;
+      mbar_expect_tx(&s_bar[0], bytes);
+      bulk_copy(sK, kb + j0 * D, bytes, &s_bar[0]);
+      mbar_expect_tx(&s_bar[1], bytes);
+      bulk_copy(sV, vb + j0 * D, bytes, &s_bar[1]);
+    }
+    zero_pieces(sK, n_here * D / 8, kChunk * D / 8, kPartThreads);
+    zero_pieces(sV, n_here * D / 8, kChunk * D / 8, kPartThreads);
+  } else {
+    stage_rows<D, kPartThreads>(sK, kb, a.k_st, [&](int s) { return s_j[s]; });
+    cp_async_commit();
+    stage_rows<D, kPartThreads>(sV, vb, a.v_st, [&](int s) { return s_j[s]; });
+    cp_async_commit();
+  }
+  StageWait sw{bulk, s_bar, &s_abort, a.status};
   grid_dep_wait();
   const int p0 = sub * EPL;  // this lane's pairs [p0, p0 + EPL)
   float2 q0[REP][H], q1[REP][H];
@@ -499,13 +568,15 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
   // a warp whose keys all lie in the window holds consecutive positions
   const int e_w = e_begin + w_lo, e_w_end = min(e_w + KPW, n);
   const bool run = e_w >= ks.n_sink && e_w_end <= ks.n_sink + ks.n_win;
-  cp_async_wait<1>();
-  __syncthreads();
+  if (!sw.wait(0, 2, kSiteDecodeK)) {
+    sw.drain(2);
+    return;
+  }
 
   // ---- pass 1: logits ----
   const int mode = !a.rope ? kRotNone : (run ? kRotRun : kRotEach);
-  logits_pass<D, REP>(
-      a, i, sK, w_lo, mode, run ? ks.win_lo + (e_w - ks.n_sink) : -1, -1, lane, q0, q1,
+  logits_pass<D, REP, NW>(
+      a, s_rt, i, sK, w_lo, mode, run ? ks.win_lo + (e_w - ks.n_sink) : -1, -1, lane, q0, q1,
       [&](int el) { return s_j[el]; },
       [&](int r, int el, int j, float dot) {
         float z = dot * sl2;
@@ -517,7 +588,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       });
   __syncthreads();
   // ---- per-head maximum, weights and their sum (warp r takes heads r, r + 4, ...) ----
-  for (int r = warp; r < REP; r += kThreads / 32) {
+  for (int r = warp; r < REP; r += NW) {
     float mx = -CUDART_INF_F;
     for (int e = lane; e < kChunk; e += 32) mx = fmaxf(mx, s_p[r][e]);
 #pragma unroll
@@ -535,8 +606,10 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       s_l[r] = sum;
     }
   }
-  cp_async_wait<0>();
-  __syncthreads();
+  if (!sw.wait(1, 2, kSiteDecodeV)) {
+    sw.drain(2);
+    return;
+  }
   // ---- pass 2: O += p v (rows past the chunk's end are zeros with p = 0) ----
   float2 o0[REP][H], o1[REP][H];
 #pragma unroll
@@ -588,10 +661,10 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       }
   }
   __syncthreads();
-  for (int x = threadIdx.x; x < REP * D; x += kThreads) {
+  for (int x = threadIdx.x; x < REP * D; x += kPartThreads) {
     const int r = x / D, c = x % D;
     float O = 0.f;
-    for (int w = 0; w < kThreads / 32; ++w) O += red_o[(w * REP + r) * D + c];
+    for (int w = 0; w < NW; ++w) O += red_o[(w * REP + r) * D + c];
     const int h = g * REP + r;
     float* part = a.part + (((size_t)b * a.Hq + h) * a.n_chunks + blockIdx.y) * (D + 2);
     part[2 + c] = O;
@@ -600,15 +673,94 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
       part[1] = s_l[r];
     }
   }
-  // count this chunk in; the group's last chunk merges
-  const int nc0 = (n + kChunk - 1) / kChunk;
-  __threadfence();
+}
+
+// grid (B * Hq), kCombThreads threads: merge the chunk partials of one
+// (batch, head), and the top-k keys' partial when there is one, into O and
+// LSE.  Every load is issued before any arithmetic: the chunks' maxima and
+// sums into shared memory, up to kCombRegs output partials per thread into
+// registers (thread group q of G takes chunks q, q + G, ...); then the
+// maximum, the weights 2^(m_x - M) and their sum, the weighted outputs, and
+// the G groups added in a fixed order.
+constexpr int kCombThreads = 512;
+constexpr int kCombRegs = 8;
+template <int D>
+__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(DecodeArgs a) {
+  constexpr int G = kCombThreads / D;
+  constexpr int NWp = kCombThreads / 32;
+  __shared__ float s_f[kMaxChunks + 1];  // chunk maxima, then weights
+  __shared__ float s_s[kMaxChunks + 1];  // chunk sums
+  __shared__ float s_red[G * D];
+  __shared__ float s_ml[2];
+  const int bh = blockIdx.x;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const KeySet ks = key_set(a, b);  // reads the block map, which preceded the split-K kernel
+  const int nc0 = min((ks.n() + kChunk - 1) / kChunk, kMaxChunks);
+  const int nc = nc0 + (a.tk_part ? 1 : 0);
+  const float* part0 = a.part + (size_t)bh * a.n_chunks * (D + 2);
+  auto slot = [&](int x) { return x < nc0 ? part0 + (size_t)x * (D + 2) : a.tk_part + (size_t)bh * (D + 2); };
+  const int tid = threadIdx.x, q = tid / D, c = tid % D;
+  grid_dep_wait();  // the partials
+  float ov[kCombRegs];
+#pragma unroll
+  for (int u = 0; u < kCombRegs; ++u) {
+    const int x = q + G * u;
+    ov[u] = x < nc ? slot(x)[2 + c] : 0.f;
+  }
+  float mx = -CUDART_INF_F;
+  for (int x = tid; x < nc; x += kCombThreads) {
+    const float* sp = slot(x);
+    const float m = sp[0];
+    s_f[x] = m;
+    s_s[x] = sp[1];
+    mx = fmaxf(mx, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) s_red[tid >> 5] = mx;
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(a.ticket + bg, 1) == nc0 - 1) ? 1 : 0;
+  if (tid == 0) {
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < NWp; ++w) M = fmaxf(M, s_red[w]);
+    s_ml[0] = M;
+  }
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  merge_chunks<D, REP>(a, b, g, nc0);
+  const float M = s_ml[0];
+  float lsum = 0.f;
+  for (int x = tid; x < nc; x += kCombThreads) {
+    const float f = (s_f[x] == -CUDART_INF_F) ? 0.f : ex2_approx(s_f[x] - M);
+    s_f[x] = f;
+    lsum = fmaf(s_s[x], f, lsum);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  __syncthreads();  // s_red is reused
+  if ((tid & 31) == 0) s_red[tid >> 5] = lsum;
+  __syncthreads();
+  if (tid == 0) {
+    float L = 0.f;
+    for (int w = 0; w < NWp; ++w) L += s_red[w];
+    s_ml[1] = L;
+  }
+  float O = 0.f;
+#pragma unroll
+  for (int u = 0; u < kCombRegs; ++u) {
+    const int x = q + G * u;
+    if (x < nc) O = fmaf(s_f[x], ov[u], O);
+  }
+  for (int x = q + G * kCombRegs; x < nc; x += G) O = fmaf(s_f[x], slot(x)[2 + c], O);
+  __syncthreads();  // s_red is reused
+  s_red[q * D + c] = O;
+  __syncthreads();
+  if (q == 0) {
+    float Ot = 0.f;
+#pragma unroll
+    for (int y = 0; y < G; ++y) Ot += s_red[y * D + c];
+    const float L = s_ml[1];
+    __nv_bfloat16* op = a.O + (size_t)b * a.o_sb + (size_t)h * a.o_sh;
+    op[c] = __float2bfloat16_rn(L > 0.f ? Ot / L : 0.f);
+    if (c == 0) a.lse[bh] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -CUDART_INF_F;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -632,6 +784,9 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   extern __shared__ __align__(16) unsigned char dsm[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dsm);  // [kChunk][D]
   __shared__ float s_z[REP][kChunk];
+  __shared__ RopeTab s_rt;
+  __shared__ __align__(8) uint64_t s_bar[1];
+  __shared__ int s_abort;
   grid_dep_launch();  // the selection kernel may be scheduled now; it waits for this grid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % a.Hkv, b = blockIdx.x / a.Hkv;
@@ -640,8 +795,30 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   const int j0 = a.n_start + blockIdx.y * kChunk;
   if (j0 >= jend) return;
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
-  stage_rows<D>(sK, kb, a.k_st, [&](int s) { return j0 + s < jend ? j0 + s : -1; });
-  cp_async_commit();
+  const int n_here = min(jend - j0, kChunk);
+  // consecutive positions: one bulk copy when the rows are contiguous
+  const bool bulk = a.k_st == D;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    if (bulk) {
+      mbar_init(&s_bar[0], 1);
+      fence_mbar_init();
+    }
+  }
+  if (a.rope) load_rope_tab(a, s_rt, D / 2, kThreads / 32);
+  __syncthreads();
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      const uint32_t bytes = (uint32_t)n_here * D * 2;
+      mbar_expect_tx(&s_bar[0], bytes);
+      bulk_copy(sK, kb + (size_t)j0 * D, bytes, &s_bar[0]);
+    }
+    zero_pieces(sK, n_here * D / 8, kChunk * D / 8, kThreads);
+  } else {
+    stage_rows<D, kThreads>(sK, kb, a.k_st, [&](int s) { return j0 + s < jend ? j0 + s : -1; });
+    cp_async_commit();
+  }
+  StageWait sw{bulk, s_bar, &s_abort, a.status};
   // a warp whose candidates all lie past the cap scores the raw keys with
   // the query rotated to L; the others rotate their keys
   const int jw = j0 + warp * KPW;
@@ -651,10 +828,12 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   float2 q0[REP][H], q1[REP][H];
   load_query<D, REP>(a, b, g, p0, q0, q1);
   const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
-  cp_async_wait<0>();
-  __syncthreads();
-  logits_pass<D, REP>(
-      a, i, sK, warp * KPW, mode, jw, all_capped ? a.L : -1, lane, q0, q1,
+  if (!sw.wait(0, 1, kSiteTopkK)) {
+    sw.drain(1);
+    return;
+  }
+  logits_pass<D, REP, kThreads / 32>(
+      a, s_rt, i, sK, warp * KPW, mode, jw, all_capped ? a.L : -1, lane, q0, q1,
       [&](int el) { return j0 + el < jend ? j0 + el : -1; },
       [&](int r, int el, int j, float dot) {
         const bool sep = j >= 0 && words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u);
@@ -824,6 +1003,10 @@ cudaError_t launch_dr(const DecodeArgs& a0, cudaStream_t st) {
   for (int c = 0; c < D / 2; ++c) {
     const double ang = KPS * a.rope_scale * a.inv_freq[c];
     a.step_cs[c] = a.rope ? make_float2((float)std::cos(ang), (float)std::sin(ang)) : make_float2(1.f, 0.f);
+    // turns per position as a sum of two floats
+    const double f = a.rope_scale * a.inv_freq[c] / 6.283185307179586;
+    a.turn_hi[c] = (float)f;
+    a.turn_lo[c] = (float)(f - (double)a.turn_hi[c]);
   }
   // without separators or per-sequence lengths the kept-key count is a
   // closed form: launch exactly its chunks
@@ -852,8 +1035,10 @@ cudaError_t launch_dr(const DecodeArgs& a0, cudaStream_t st) {
   }
   e = allow_smem(decode_partial_kernel<D, REP>, 2 * rows_bytes);
   if (e != cudaSuccess) return e;
-  return launch_k(decode_partial_kernel<D, REP>, dim3(a.B * a.Hkv, chunks), kThreads, 2 * rows_bytes, after_kernel,
-                  a, st);
+  e = launch_k(decode_partial_kernel<D, REP>, dim3(a.B * a.Hkv, chunks), PartCfg<REP>::NT, 2 * rows_bytes,
+               after_kernel, a, st);
+  if (e != cudaSuccess) return e;
+  return launch_k(decode_combine_kernel<D>, dim3(a.B * a.Hq), kCombThreads, 0, true, a, st);
 }
 
 template <int D>

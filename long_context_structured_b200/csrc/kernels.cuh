@@ -470,11 +470,12 @@ struct DecodeArgs {
   double rope_scale;
   double inv_freq[64];          // theta^(-2c/d), c < d/2
   float2 step_cs[64];           // (cos, sin) of the rotation by a fixed number of positions (kernel-set)
+  float turn_hi[64], turn_lo[64];  // turns per position of pair c, as hi + lo (kernel-set)
   const uint2* sep_words;       // separator word prefix (sep_before) or null (no separators)
   const int32_t* sep_pos;       // [B, T]
   const int32_t* seq_len;       // [B] cache length per sequence (<= T), or null: T for all
   float* part;                  // [B, Hq, n_chunks, d + 2] chunk partials
-  int32_t* ticket;              // [B, Hkv] finished chunks per group, zero before the launch
+  int32_t* status;              // the workspace's status word (a wait that gave up)
   int alibi;                    // ALiBi bias clipped at L (no rotation)
   int n_chunks;
   // top-k middle tokens of the query (topk > 0; seq_len must be null)
