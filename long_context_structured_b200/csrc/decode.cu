@@ -97,7 +97,8 @@ struct StageWait {
   // Every thread of the block calls it; the result is uniform.
   __device__ __forceinline__ bool wait(int t, int ntensors, int site) {
     if (bulk) {
-      mbar_wait(bars + t, 0, abort_flag, status, site);
+      // one thread polls; the others wait at the barrier without issuing
+      if (threadIdx.x == 0) mbar_wait(bars + t, 0, abort_flag, status, site);
     } else if (ntensors == 2 && t == 0) {
       cp_async_wait<1>();
     } else {
@@ -108,7 +109,7 @@ struct StageWait {
   }
   // after a failed wait: give the copies still in flight a bounded time to land
   __device__ __forceinline__ void drain(int ntensors) {
-    if (!bulk) return;
+    if (!bulk || threadIdx.x != 0) return;
     for (int t = 0; t < ntensors; ++t) {
       const uint32_t a = smem_u32(bars + t);
       const uint64_t t0 = globaltimer_ns();
@@ -219,22 +220,26 @@ struct RopeTab {
   float2 st[64];         // (cos, sin) of the rotation by KPS positions
 };
 
-__device__ __forceinline__ void load_rope_tab(const DecodeArgs& a, RopeTab& t, int half, int nwarps) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int x = warp; x < half; x += nwarps)  // warp-uniform index: one broadcast load per element
-    if (lane == 0) {
-      t.hi[x] = a.turn_hi[x];
-      t.lo[x] = a.turn_lo[x];
-      t.st[x] = a.step_cs[x];
-    }
+__device__ __forceinline__ void load_rope_tab(const DecodeArgs& a, RopeTab& t, int half) {
+  const int x = threadIdx.x;
+  if (x < half) {
+    t.hi[x] = a.turn_hi[x];
+    t.lo[x] = a.turn_lo[x];
+    t.st[x] = a.step_cs[x];
+  }
 }
 
+// |p| < 2^22 and |t1| < 2^22: the int-to-float conversion and the rounding
+// to a whole number of turns are done by adding 1.5 * 2^23 (exact at that
+// magnitude), which keeps them off the conversion unit.
 __device__ __forceinline__ float2 rope_cs(const RopeTab& t, int p, int c) {
-  const float fp = (float)p;
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+  const float fp = __int_as_float(0x4B400000 + p) - kMagic;
   const float hi = t.hi[c];
   const float t1 = fp * hi;
   const float e1 = fmaf(fp, hi, -t1);
-  const float r = (t1 - rintf(t1)) + fmaf(fp, t.lo[c], e1);
+  const float whole = __fsub_rn(__fadd_rn(t1, kMagic), kMagic);
+  const float r = (t1 - whole) + fmaf(fp, t.lo[c], e1);
   float s, co;
   __sincosf(r * 6.283185307179586f, &s, &co);
   return make_float2(co, s);
@@ -537,7 +542,7 @@ __global__ void __launch_bounds__(PartCfg<REP>::NT, PartCfg<REP>::MIN_BLOCKS) de
     }
   }
   if (threadIdx.x < kChunk) s_j[threadIdx.x] = (int)threadIdx.x < n_here ? key_at(a, ks, b, e_begin + threadIdx.x) : -1;
-  if (a.rope) load_rope_tab(a, s_rt, half, NW);
+  if (a.rope) load_rope_tab(a, s_rt, half);
   __syncthreads();
   const __nv_bfloat16* kb = a.K + (size_t)b * a.k_sb + (size_t)g * a.k_sh;
   const __nv_bfloat16* vb = a.V + (size_t)b * a.v_sb + (size_t)g * a.v_sh;
@@ -784,6 +789,7 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   extern __shared__ __align__(16) unsigned char dsm[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(dsm);  // [kChunk][D]
   __shared__ float s_z[REP][kChunk];
+  __shared__ __align__(8) float s_qL[REP * D];  // R(L) q of the group's heads
   __shared__ RopeTab s_rt;
   __shared__ __align__(8) uint64_t s_bar[1];
   __shared__ int s_abort;
@@ -805,7 +811,7 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
       fence_mbar_init();
     }
   }
-  if (a.rope) load_rope_tab(a, s_rt, D / 2, kThreads / 32);
+  if (a.rope) load_rope_tab(a, s_rt, D / 2);
   __syncthreads();
   if (bulk) {
     if (threadIdx.x == 0) {
@@ -820,20 +826,42 @@ __global__ void __launch_bounds__(kThreads) decode_topk_logits_kernel(DecodeArgs
   }
   StageWait sw{bulk, s_bar, &s_abort, a.status};
   // a warp whose candidates all lie past the cap scores the raw keys with
-  // the query rotated to L; the others rotate their keys
+  // the query rotated to L; the others rotate their keys.  When the whole
+  // chunk is past the cap, R(L) q is formed once per CTA in shared memory.
+  constexpr int half = D / 2;
+  const bool cta_capped = a.rope && a.L > 0 && i - (j0 + kChunk - 1) > a.L;
+  if (cta_capped) {
+    for (int x = threadIdx.x; x < REP * half; x += kThreads) {
+      const int r = x / half, c = x % half;
+      const float2 cs = rope_cs(s_rt, a.L, c);
+      const __nv_bfloat16* qp = a.Q + (size_t)b * a.q_sb + (size_t)(g * REP + r) * a.q_sh;
+      const float x0 = __bfloat162float(qp[c]), x1 = __bfloat162float(qp[c + half]);
+      s_qL[r * D + c] = x0 * cs.x - x1 * cs.y;
+      s_qL[r * D + c + half] = x1 * cs.x + x0 * cs.y;
+    }
+  }
   const int jw = j0 + warp * KPW;
   const bool all_capped = a.rope && a.L > 0 && i - (jw + KPW - 1) > a.L;
   const int mode = !a.rope || all_capped ? kRotNone : kRotRun;
   const int p0 = (lane % LPK) * EPL;
   float2 q0[REP][H], q1[REP][H];
-  load_query<D, REP>(a, b, g, p0, q0, q1);
+  if (!cta_capped) load_query<D, REP>(a, b, g, p0, q0, q1);
   const uint2* words = a.sep_words ? a.sep_words + (size_t)b * (a.T / 32 + 1) : nullptr;
   if (!sw.wait(0, 1, kSiteTopkK)) {
     sw.drain(1);
     return;
   }
+  if (cta_capped) {
+#pragma unroll
+    for (int r = 0; r < REP; ++r)
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        q0[r][h] = *reinterpret_cast<const float2*>(&s_qL[r * D + p0 + 2 * h]);
+        q1[r][h] = *reinterpret_cast<const float2*>(&s_qL[r * D + p0 + 2 * h + half]);
+      }
+  }
   logits_pass<D, REP, kThreads / 32>(
-      a, s_rt, i, sK, warp * KPW, mode, jw, all_capped ? a.L : -1, lane, q0, q1,
+      a, s_rt, i, sK, warp * KPW, mode, jw, all_capped && !cta_capped ? a.L : -1, lane, q0, q1,
       [&](int el) { return j0 + el < jend ? j0 + el : -1; },
       [&](int r, int el, int j, float dot) {
         const bool sep = j >= 0 && words && ((__ldg(&words[j >> 5].y) >> (j & 31)) & 1u);
