@@ -693,9 +693,9 @@ def kernel_name(wl, group):
         return "attn_tc2_kernel<%d>" % TREE_WORKLOADS["tree_cross_128k"]["d"]
     d = wl.d if wl is not None else 128
     if group == "decode" and wl is not None and wl.topk > 0:
-        return "decode_topk_logits_kernel + decode_topk_select_kernel + decode_partial_kernel"
+        return "decode_topk_logits_kernel + decode_topk_select_kernel + decode_partial_kernel + decode_combine_kernel"
     return {"prep_rope": "prep_kernel", "topk_score": "topk_score_kernel<%d>" % d, "topk_rerank": "topk_rerank_kernel<%d>" % d, "tree_prep": "tree_prep_kernel",
-            "decode": "decode_partial_kernel",
+            "decode": "decode_partial_kernel + decode_combine_kernel",
             "sep_gather": "sep_gather_kernel", "bwd_dq": "bwd_dq_kernel<%d>" % d,
             "bwd_dkv": "bwd_dkv_kernel<%d>" % d, "bwd_f32": "bwd_f32_dq_kernel + bwd_f32_dkv_kernel",
             "bwd_rows": "bwd_rows_kernel", "bwd_combine": "bwd_combine_kernel",
@@ -1021,7 +1021,7 @@ def run_stream(args, world, rank, dev):
     for g in sorted(prof):
         n, ms = prof[g]
         avg = ms / args.steps
-        kernels[g] = {"kernel": {"stream_decode": "decode_partial_kernel",
+        kernels[g] = {"kernel": {"stream_decode": "decode_partial_kernel + decode_combine_kernel",
                                  "stream_append": "stream_append/plan/move kernels"}.get(g, g),
                       "launches": n, "ms_per_step": round(avg, 5),
                       "share": round(ms / max(sum(v[1] for v in prof.values()), 1e-12), 4)}
@@ -1029,7 +1029,7 @@ def run_stream(args, world, rank, dev):
             r = roofline_of(g, work[g], avg, peaks, peak_src)
             kernels[g].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
     roof = roofline_of("stream_decode", work["stream_decode"], prof["stream_decode"][1] / args.steps, peaks, peak_src)
-    roof["kernel"] = "decode_partial_kernel"
+    roof["kernel"] = "decode_partial_kernel + decode_combine_kernel"
     roof["traffic"] = None
     if world > 1:
         dist.barrier()
