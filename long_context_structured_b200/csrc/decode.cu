@@ -210,8 +210,9 @@ __device__ __forceinline__ void load_pairs(const __nv_bfloat16* p, float2 (&out)
 // with f_c = s theta^(-2c/d) / (2 pi) split on the host into fp32 parts
 // hi + lo: p * hi is formed with its exact rounding residual (one fma), its
 // whole turns removed exactly, and p * lo added, which leaves the reduced
-// angle to about 1e-7 turns for positions below 2^24; then the hardware
-// sine and cosine of that angle in [-pi, pi] (absolute error about 2^-21).
+// angle to about 3e-8 turns for the positions a step uses (below 2^19);
+// then the hardware sine and cosine of that angle, within 1.02 pi of zero
+// (absolute error about 2^-21).
 // The per-pair rotation constants, copied once per CTA from the kernel
 // parameters into shared memory (lanes index them by pair, which a
 // parameter-space load would serialise).
