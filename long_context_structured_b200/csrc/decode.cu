@@ -11,21 +11,22 @@
 //
 // Split-K over the kept keys (memory-bound: each kept K and V row is read
 // once): a CTA takes a chunk of kChunk kept keys of one (batch, kv head) for
-// all query heads of that kv head's group.  It first issues asynchronous
-// copies of all the chunk's K and V rows into shared memory (64 KB at d =
-// 128, so that every byte the CTA needs is in flight at once), then computes
-// the logits from the staged K rows (each warp walks 32 keys with the head
-// dimension spread over the lanes: a lane owns rotary pairs c = PPL*lane ..
-// PPL*lane + PPL - 1 and their partners c + d/2), then, with the chunk's
-// per-head maximum known, the weighted V rows.  The chunk's (max, sum,
-// unnormalised O) per head go to the workspace, and the last CTA of a
-// (batch, kv head) to finish merges them into O and LSE.
+// all query heads of that kv head's group.  It first stages all the chunk's
+// K and V rows in shared memory (64 KB at d = 128, so that every byte the
+// CTA needs is in flight at once: one bulk copy per tensor for a run of
+// consecutive rows, else 16-byte asynchronous copies), then computes the
+// logits from the staged K rows (a key's head dimension spread over a few
+// lanes, each holding some rotary pairs and their partners c + d/2), then,
+// with the chunk's per-head maximum known, the weighted V rows.  The chunk's
+// (max, sum, unnormalised O) per head go to the workspace; a merge kernel,
+// launched as the split-K kernel's programmatic dependent, combines them
+// into O and LSE.
 //
 // The rotations are computed in the kernel, not read from a table: the
-// angle of a position in double, reduced by whole turns, then the fp32 sine
-// and cosine (the prefill's table arithmetic); along a run of consecutive
-// positions a lane steps its keys' (cos, sin) by one fixed rotation
-// (angle addition in fp32) instead.
+// angle of a position in turns from a two-float turn rate, reduced by whole
+// turns in fp32 without rounding loss, then the hardware sine and cosine;
+// along a run of consecutive positions a lane steps its query's (or its
+// keys') rotation by one fixed rotation (angle addition in fp32) instead.
 #include <algorithm>
 #include <cmath>
 
