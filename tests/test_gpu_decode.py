@@ -205,3 +205,36 @@ def test_decode_topk_alibi_below_cap_rejected():
     kv = torch.zeros((1, 2, 300, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(_lib.SattnError):
         sa.decode_fwd(q, kv, kv, n_start=4, window=30, L_pretrain=100, topk=2, alibi=True)
+
+
+def _padded(t, pad=8):
+    """The same values in a [B, H, T, d] view whose rows are d + pad apart."""
+    B, H, T, d = t.shape
+    buf = torch.full((B, H, T, d + pad), 5.0, dtype=t.dtype, device=t.device)
+    buf[..., :d] = t
+    return buf[..., :d]
+
+
+@pytest.mark.parametrize("name,cfg", [TOPK_CASES[0], TOPK_CASES[1], CASES[0]], ids=lambda x: x if isinstance(x, str) else "")
+def test_decode_strided_cache_equals_contiguous(name, cfg):
+    """A cache whose rows are not adjacent is staged piece by piece instead
+    of by one bulk copy per chunk; the step is the same bit for bit."""
+    wl = synth.Workload(name=name, dtype="bf16", **cfg)
+    inp = synth.make_inputs(wl, seed=31)
+    q, k, v = (to_dev(inp[x]) for x in ("q", "k", "v"))
+    sep = to_dev(inp["is_sep"])
+    qd = q[:, :, wl.T - 1:wl.T, :].contiguous()
+    kw = dict(n_start=wl.n_start, window=wl.window, L_pretrain=wl.L_pretrain, rope_theta=wl.rope_theta, is_sep=sep,
+              alibi=wl.alibi, topk=wl.topk)
+    kp, vp = _padded(k), _padded(v)
+    assert kp.stride(2) == wl.d + 8 and not kp.is_contiguous()
+    if wl.topk > 0:
+        a = sa.decode_fwd(qd, k, v, return_topk=True, **kw)
+        b = sa.decode_fwd(qd, kp, vp, return_topk=True, **kw)
+    else:
+        a = sa.decode_fwd(qd, k, v, **kw)
+        b = sa.decode_fwd(qd, kp, vp, **kw)
+    torch.cuda.synchronize()
+    assert sa.stream_status() == 0
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
