@@ -465,12 +465,12 @@ struct DecodeArgs {
   int64_t k_sb, k_sh, k_st;
   const __nv_bfloat16* V;
   int64_t v_sb, v_sh, v_st;
-  // rotation (rope != 0): pair c at position p turns by p * rope_scale * inv_freq[c]
+  // rotation (rope != 0): pair c at position p rotates by the angle p * rope_scale * inv_freq[c]
   int rope;
   double rope_scale;
   double inv_freq[64];          // theta^(-2c/d), c < d/2
-  float2 step_cs[64];           // (cos, sin) of the rotation by a fixed number of positions (kernel-set)
-  float turn_hi[64], turn_lo[64];  // turns per position of pair c, as hi + lo (kernel-set)
+  float2 step_cs[64];           // (cos, sin) of the rotation by KPS positions (set by the launcher)
+  float turn_hi[64], turn_lo[64];  // turns per position of pair c, as hi + lo (set by the launcher)
   const uint2* sep_words;       // separator word prefix (sep_before) or null (no separators)
   const int32_t* sep_pos;       // [B, T]
   const int32_t* seq_len;       // [B] cache length per sequence (<= T), or null: T for all
