@@ -1,5 +1,6 @@
 // attn_tc3.cu -- K5, one 128-row query tile per CTA with the score tile
-// double-buffered in tensor memory: the production prefill attention kernel.
+// triple-buffered in tensor memory: the prefill attention kernel for capped
+// separator tiles and for segment lengths that are not a multiple of 256.
 //
 // Mathematics (same as attn_tc2.cu): the kept keys of a query row are the
 // band keys (the recent window of LM-Infinite's Lambda-shaped mask, section

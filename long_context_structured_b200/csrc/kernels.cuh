@@ -162,7 +162,7 @@ struct AttnMaps {
 // two query tiles per CTA; not for q2 (capped separator tiles) and, in
 // segmented mode, only when the segment length is a multiple of 256
 cudaError_t launch_attn_tc2(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
-// one query tile per CTA with the score tile double-buffered in TMEM; every case
+// one query tile per CTA with the score tile triple-buffered in TMEM; every case
 cudaError_t launch_attn_tc3(const AttnArgs& a, const AttnMaps& m, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
