@@ -9,7 +9,9 @@
 //  1. scoring on the tensor cores: S = Qsel Ksel^T in bf16 x bf16 -> fp32
 //     (Qsel/Ksel = R(L)q / raw k when capped, R(i)q / R(j)k otherwise).  A
 //     CTA takes two 128-row query tiles; each K tile is loaded once and
-//     multiplied into both tiles' TMEM score buffers.  A sample of the key
+//     multiplied into both tiles' TMEM score buffers (with the window below
+//     the cap, one query tile per CTA whose two slots hold R(L)q and R(i)q,
+//     a key tile straddling the cap scored against both).  A sample of the key
 //     tiles is scored first and sets each row's threshold tau; then every
 //     candidate tile is scored and each key whose coarse score exceeds tau
 //     is appended to the row's candidate list (kCandCap entries);
